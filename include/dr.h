@@ -1,0 +1,126 @@
+/*
+ * dr.h -- C ABI of the chunkwise gated delta-rule linear-attention library
+ * (libdr.so, CUDA, sm_100a).
+ *
+ * Operation (per batch b and head h; S is d_v x d_k):
+ *
+ *   S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *   o_t = S_t q_t                       (the state is read after the write)
+ *
+ * This is the real, phase-free form of the delta-rule update in the SFDA
+ * explainer ("Semidirect Fourier Delta Attention", gist.science, section
+ * "Kernarchitektur"; zero phase recovers KDA), transposed so that S maps keys
+ * to values.  alpha_t = exp(g_t) with g the log-gate: absent (DeltaNet), one
+ * scalar per head and token (GDN) or one per key channel (KDA), as named in
+ * the ReWY abstract (paperdot listing).  In Kaczmarz mode (KLA abstract,
+ * thelatestinai.com) beta_t = eta_t / (||k_t||^2 + eps) and the beta argument
+ * carries eta.
+ *
+ * dr_chunk_fwd evaluates the recurrence chunkwise (chunk = 64 tokens): an
+ * intra-chunk UT transform (I + A) [U' | W] = diag(beta) [V | K e^gamma] with
+ * A the beta- and gate-scaled strictly-lower key Gram, an inter-chunk state
+ * scan S <- S Diag(e^{gamma_C}) + U^T K~ ("exact affine chunk transfer", SFDA
+ * explainer, "Zentrale Beiträge"), and the output q S^T plus the causal
+ * intra-chunk term.  dr_chunk_bwd returns the exact gradients of the same
+ * function; the chunk correction is differentiated as one triangular residual
+ * system (ReWY abstract), so no adjoint of the inverse is formed.
+ *
+ * Conventions for every entry point:
+ *  - Tensor pointers are DEVICE pointers, 16-byte aligned, row-major and
+ *    contiguous, owned by the caller; the library never allocates device
+ *    memory and keeps no pointer after a call returns.
+ *  - Layouts: q, k [B, T, H, dk]; v, o, dO [B, T, H, dv] (storage dtype
+ *    dr_problem.dtype); beta [B, T, H] fp32; g [B, T, H] fp32 (scalar gate)
+ *    or [B, T, H, dk] fp32 (per-channel gate), NULL for gate NONE;
+ *    S0, ST, dST, dS0 [B, H, dv, dk] fp32.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Arguments are validated on the host before any launch; a
+ *    non-DR_OK status means nothing was launched, except DR_ERR_CUDA, which
+ *    reports a launch failure.  Device-side conditions (a bounded wait that
+ *    timed out) are recorded in a device flag and reported by
+ *    dr_last_device_error.
+ *  - Calls on different streams must not share a workspace or saved buffer.
+ */
+#ifndef DR_H
+#define DR_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DR_OK = 0,
+  DR_ERR_INVALID_ARG = 1,  /* null required pointer, bad size, misaligned pointer */
+  DR_ERR_UNSUPPORTED = 2,  /* valid but not implemented (chunk != 64, head dim) */
+  DR_ERR_WORKSPACE = 3,    /* workspace or saved buffer missing or too small */
+  DR_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
+  DR_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up */
+} dr_status;
+
+typedef enum { DR_F32 = 0, DR_BF16 = 1 } dr_dtype;
+typedef enum { DR_GATE_NONE = 0, DR_GATE_SCALAR = 1, DR_GATE_CHANNEL = 2 } dr_gate;
+typedef enum { DR_BETA_DIRECT = 0, DR_BETA_KACZMARZ = 1 } dr_beta_mode;
+
+/* Problem description.  Supported: B, H, T >= 1; chunk == 64;
+   dk, dv multiples of 16 in [16, 128]; dtype DR_F32 or DR_BF16.
+   eps is used only in Kaczmarz mode (must be >= 0). */
+typedef struct {
+  int B, H, T, dk, dv, chunk;
+  int dtype;      /* dr_dtype */
+  int gate;       /* dr_gate */
+  int beta_mode;  /* dr_beta_mode */
+  float eps;
+} dr_problem;
+
+/* Bytes of scratch ("workspace") that dr_chunk_fwd (pass 0) or dr_chunk_bwd
+   (pass 1) needs for problem *p.  Writes *bytes; host only, no CUDA call. */
+dr_status dr_workspace_size(const dr_problem* p, int pass, size_t* bytes);
+
+/* Bytes of the forward-to-backward "saved" buffer (per-chunk start states,
+   internal layout).  Host only. */
+dr_status dr_saved_size(const dr_problem* p, size_t* bytes);
+
+/* Chunkwise forward.
+   In:  q, k, v, beta (eta in Kaczmarz mode), g (NULL iff gate NONE),
+        S0 (NULL = zero initial state).
+   Out: o (storage dtype), ST (final state, fp32; NULL = not wanted),
+        saved (NULL = not wanted; else dr_saved_size bytes, which dr_chunk_bwd
+        may then read instead of recomputing the states).
+   ws:  at least dr_workspace_size(p, 0) bytes of device scratch, 256-byte
+        aligned; its contents are undefined after the call. */
+dr_status dr_chunk_fwd(const dr_problem* p, const void* q, const void* k, const void* v,
+                       const float* beta, const float* g, const float* S0, void* o,
+                       float* ST, void* saved, void* ws, size_t ws_bytes, void* stream);
+
+/* Chunkwise backward of the same call.
+   In:  the forward inputs, dO (storage dtype), dST (upstream gradient of the
+        final state, fp32; NULL = zero), saved (the buffer a previous
+        dr_chunk_fwd filled for the same inputs, or NULL to recompute).
+   Out: dq, dk, dv (storage dtype), dbeta (fp32; d/deta in Kaczmarz mode),
+        dg (fp32, shaped like g; ignored and may be NULL for gate NONE),
+        dS0 (fp32; NULL = not wanted).
+   ws:  at least dr_workspace_size(p, 1) bytes, 256-byte aligned. */
+dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const void* v,
+                       const float* beta, const float* g, const float* S0, const void* dO,
+                       const float* dST, const void* saved, void* dq, void* dk, void* dv,
+                       float* dbeta, float* dg, float* dS0, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* dr_status_string(dr_status s);
+
+/* Synchronises `stream`, then reports and clears the device error flag:
+   DR_ERR_TIMEOUT if a bounded device wait gave up since the last check,
+   DR_ERR_CUDA if the stream reported an error, else DR_OK. */
+dr_status dr_last_device_error(void* stream);
+
+/* Library ABI version (major * 100 + minor). */
+int dr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DR_H */
