@@ -1,0 +1,450 @@
+#!/usr/bin/env python
+"""Benchmark: forward + backward tokens/s of the chunkwise gated delta-rule
+operator (dr_chunk_fwd + dr_chunk_bwd through the C ABI) and its fraction of
+the B200 roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the fp64 CPU oracle, timed on host cores
+
+One step = one forward (saving chunk states) and one backward over one batch of
+the workload, inputs resident in HBM.  Default workload: KDA per-channel gate,
+bf16, B=4, H=16, T=8192, d_k=d_v=128, chunk 64.  Under torchrun each rank runs
+its own batch (weak scaling, no collective on the data path); timing is the
+max over ranks.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fwd+bwd tokens/s (GDN/KDA, bf16, d=128); % of B200 tensor-core/HBM roofline"
+UNIT = "tokens/s"
+# Used only when the measured-peaks file is absent (an earlier measurement on this GPU pool).
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2 ** 20
+FP32_LANES_PER_SM = 128
+NUM_SMS = 148
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["dr", "reference"], default="dr")
+    ap.add_argument("--workload", default=None, help="workload name (default: the headline KDA workload)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch size (smaller profiling captures)")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end run")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target wall time of the timed oracle sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic_step(w):
+    """Per-step algorithmic FLOPs and HBM bytes of forward + backward.
+
+    FLOPs per token-head: forward 10 C d + 6 d^2, backward with recompute
+    28 C d + 14 d^2 (d = d_k = d_v).  Bytes: every input read and output
+    written once per pass (q, k, v, g, beta, o forward; q, k, v, g, beta, dO
+    read and dq, dk, dv, dg, dbeta written backward), plus the state tensors
+    the step actually reads or writes (S0, S_T, dS_T, dS0) at d_v d_k fp32 per
+    head.  Chunk states and other scratch are policy, not algorithm."""
+    C, d = w.chunk, w.dk
+    es = 2 if w.dtype == "bf16" else 4
+    gb = {"none": 0, "scalar": 4, "channel": 4 * w.dk}[w.gate]
+    th = w.token_heads
+    flops = th * (10 * C * d + 6 * d * d + 28 * C * d + 14 * d * d)
+    io = (2 * w.dk + w.dv) * es + gb + 4
+    fwd = io + w.dv * es
+    bwd = io + w.dv * es + (2 * w.dk + w.dv) * es + gb + 4
+    nstate = 2 + (2 if w.s0_std > 0 else 0)  # S_T, dS0 (+ S0 read twice)
+    state = w.B * w.H * w.dv * w.dk * 4 * nstate
+    return flops, th * (fwd + bwd) + state
+
+
+def reduce_max(x: float, device) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tokens_per_s(world: int, tokens_per_step: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_step * steps / (max_ms / 1e3)
+
+
+def csrc_hash():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "delta_rule_linear_chunkwise_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("csrc_hash") != csrc_hash() or e.get("workload") != workload:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x10: "sync_boost"}
+
+    def __init__(self, index, period=0.01):
+        self.index, self.period = index, period
+        self.samples, self._stop = [], threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that, keep benchmarking
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = set()
+        for _, rs in self.samples:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(self.samples), "source": "nvml"}
+
+
+def cpu_baseline(w, inp, seconds):
+    """Time the fp64 oracle (forward + backward) on host cores on a bounded
+    sample: all heads, the first T_s tokens, T_s sized to about `seconds`."""
+    import oracle
+
+    mode = oracle.BETA_KACZMARZ if w.beta_mode == "kaczmarz" else oracle.BETA_DIRECT
+
+    def run(Ts):
+        sl = {n: (None if inp[n] is None else inp[n][:, :Ts].double().numpy())
+              for n in ("q", "k", "v", "beta", "g", "dO")}
+        S0 = None if inp["S0"] is None else inp["S0"].double().numpy()
+        t0 = time.perf_counter()
+        _, _, thr = oracle.recurrent_fwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0,
+                                         beta_mode=mode, eps=w.eps, return_threads=True)
+        oracle.recurrent_bwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0, sl["dO"],
+                             beta_mode=mode, eps=w.eps)
+        return time.perf_counter() - t0, thr
+
+    probe = min(w.T, 128)
+    dt, _ = run(probe)
+    Ts = int(max(probe, min(w.T, probe * seconds / max(dt, 1e-3))))
+    dt, thr = run(Ts)
+    tokens_equiv = w.B * Ts  # all heads of B x Ts tokens
+    return {"value": tokens_equiv / dt, "unit": UNIT, "cores": thr, "kind": "oracle",
+            "sample": f"fp64 oracle forward+backward on all {w.B * w.H} heads x the first "
+                      f"{Ts} of {w.T} tokens of the same inputs, wall clock {dt:.1f} s",
+            "seconds": dt}
+
+
+def run_reference(args):
+    """The fp64 CPU oracle as the reference arm: each step is one oracle
+    forward+backward on a bounded sample of the workload (rank 0 only)."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import torch  # noqa: F401  (the workload generator draws with torch)
+    import oracle
+    from delta_rule_linear_chunkwise_b200 import HEADLINE, WORKLOADS, make_inputs
+
+    w = WORKLOADS[args.workload or HEADLINE]
+    inp = make_inputs(w)
+    oracle.build()
+    mode = oracle.BETA_KACZMARZ if w.beta_mode == "kaczmarz" else oracle.BETA_DIRECT
+    total_steps = args.steps + args.warmup
+    budget = 150.0  # seconds for the whole run
+    per_step = budget / max(total_steps, 1)
+
+    def sample(Ts):
+        return ({n: (None if inp[n] is None else inp[n][:, :Ts].double().numpy())
+                 for n in ("q", "k", "v", "beta", "g", "dO")},
+                None if inp["S0"] is None else inp["S0"].double().numpy())
+
+    def step(sl, S0):
+        t0 = time.perf_counter()
+        _, _, thr = oracle.recurrent_fwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0,
+                                         beta_mode=mode, eps=w.eps, return_threads=True)
+        oracle.recurrent_bwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0, sl["dO"],
+                             beta_mode=mode, eps=w.eps)
+        return time.perf_counter() - t0, thr
+
+    probe = min(w.T, 64)
+    dt, _ = step(*sample(probe))
+    Ts = int(max(16, min(w.T, probe * per_step / max(dt, 1e-3))))
+    sl, S0 = sample(Ts)
+    for _ in range(args.warmup):
+        step(sl, S0)
+    times, thr = [], 1
+    for _ in range(args.steps):
+        dt, thr = step(sl, S0)
+        times.append(dt)
+    tot = sum(times)
+    value = w.B * Ts * args.steps / tot
+    desc = (f"fp64 oracle forward+backward per step on all {w.B * w.H} heads x the first {Ts} "
+            f"of {w.T} tokens of the workload's inputs")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
+                   "chunk": w.chunk, "gate": w.gate, "beta_mode": w.beta_mode,
+                   "sample_tokens_per_head": Ts},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    from delta_rule_linear_chunkwise_b200 import HEADLINE, WORKLOADS, binding, make_inputs
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    w = WORKLOADS[args.workload or HEADLINE]
+    if args.batch:
+        w = w.with_(B=args.batch)
+    inp = make_inputs(w, seed=w.seed + 1000 * rank)
+    d = {n: (None if x is None else x.to(dev)) for n, x in inp.items()}
+    plan = binding.Plan.for_workload(w, device=dev)
+    saved = plan.new_saved()
+    o, ST, _ = plan.fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], saved=saved)
+    grads = plan.bwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], d["dO"], None, saved)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        plan.fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], o=o, ST=ST, saved=saved)
+        plan.bwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], d["dO"], None, saved,
+                 out=grads)
+
+    in_bytes = sum(x.numel() * x.element_size() for x in d.values() if x is not None)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    binding.profile_enable(True)
+    with ClockSampler(local) as clk:
+        for e0, e1 in ev:
+            flush.fill_(float(len(ev)))       # evict L2 between timed steps (not timed)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+    kernels = binding.profile_read()
+    binding.profile_enable(False)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    assert binding.last_device_error() == binding.DR_OK
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    tot_ms = reduce_max(sum(step_ms), dev)
+    ms_per_step = tot_ms / args.steps
+    value = aggregate_tokens_per_s(world, w.tokens, args.steps, tot_ms)
+
+    # End to end through the public API with host buffers: pinned host inputs
+    # copied in and every output copied back, inside the timed region.
+    e2e = None
+    if not args.no_e2e:
+        hin = {n: (None if x is None else x.pin_memory()) for n, x in inp.items()}
+        hout = {"o": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
+                "ST": torch.empty(ST.shape, dtype=ST.dtype).pin_memory()}
+        for n, x in grads.items():
+            if x is not None:
+                hout[n] = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+        dev_in = {n: (None if x is None else torch.empty_like(x, device=dev)) for n, x in hin.items()}
+
+        def e2e_step():
+            for n, x in hin.items():
+                if x is not None:
+                    dev_in[n].copy_(x, non_blocking=True)
+            plan.fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"], dev_in["g"],
+                     dev_in["S0"], o=o, ST=ST, saved=saved)
+            plan.bwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"], dev_in["g"],
+                     dev_in["S0"], dev_in["dO"], None, saved, out=grads)
+            hout["o"].copy_(o, non_blocking=True)
+            hout["ST"].copy_(ST, non_blocking=True)
+            for n, x in grads.items():
+                if x is not None:
+                    hout[n].copy_(x, non_blocking=True)
+
+        k2 = max(3, min(args.steps, 10))
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(k2):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        t_e2e = reduce_max(a.elapsed_time(b), dev)
+        h2d = sum(x.numel() * x.element_size() for x in hin.values() if x is not None)
+        d2h = sum(x.numel() * x.element_size() for x in hout.values())
+        e2e = {"value": aggregate_tokens_per_s(world, w.tokens, k2, t_e2e), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k2}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    clocks = clk.summary()
+    # Dominant kernel: largest summed event time inside the timed region.
+    top = max(kernels, key=lambda k: k["ms_total"])
+    per_launch_s = top["ms_total"] / top["launches"] / 1e3
+    tensor = top["name"].startswith("tc_")
+    gbs = top["bytes_per_launch"] / per_launch_s / 1e9
+    tflops = top["flops_per_launch"] / per_launch_s / 1e12
+    hbm_frac = gbs / peaks["hbm_gbs"]
+    if tensor:
+        fpeak, fsrc = peaks["bf16_tflops_sustained"], f"{peak_src} bf16 dense, sustained"
+    else:
+        sm = clocks.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
+        fpeak = NUM_SMS * FP32_LANES_PER_SM * 2 * sm * 1e6 / 1e12
+        fsrc = f"fp32 FMA: {NUM_SMS} SMs x {FP32_LANES_PER_SM} lanes x 2 x {sm:.0f} MHz"
+    flop_frac = tflops / fpeak
+    if hbm_frac >= flop_frac:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": hbm_frac, "peak_source": f"{peak_src} HBM copy"}
+    else:
+        roof = {"bound": "tensor" if tensor else "alu", "achieved": tflops, "peak": fpeak,
+                "unit": "TFLOP/s", "frac": flop_frac, "peak_source": fsrc}
+    roof.update({"kernel": top["name"], "launches": top["launches"],
+                 "us_per_launch": per_launch_s * 1e6,
+                 "share_of_step": top["ms_total"] / max(sum(step_ms), 1e-9),
+                 "algorithmic_bytes_per_launch": top["bytes_per_launch"],
+                 "algorithmic_flops_per_launch": top["flops_per_launch"],
+                 "traffic": ncu_traffic(top["name"], w.name)})
+
+    flops, nbytes = algorithmic_step(w)
+    t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_roof = max(t_tc, t_hbm)
+    step_roof = {"flops": flops, "bytes": nbytes, "roofline_us": t_roof * 1e6,
+                 "tensor_us": t_tc * 1e6, "hbm_us": t_hbm * 1e6,
+                 "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                 "frac": t_roof / (ms_per_step / 1e3), "peak_source": peak_src}
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cpu = cpu_baseline(w, inp, args.cpu_seconds)
+
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
+                   "chunk": w.chunk, "gate": w.gate, "beta_mode": w.beta_mode,
+                   "global_batch": w.B * world, "seq_len": w.T,
+                   "parallelism": f"replicas x{world} (independent batches, no collective)",
+                   "l2": f"L2 flushed between timed steps ({2 * L2_BYTES >> 20} MiB write); "
+                         f"inputs {in_bytes >> 20} MiB per step",
+                   "policy": "forward saves chunk states; backward reads them"},
+        "roofline": roof,
+        "step_roofline": step_roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": sum(k["launches"] for k in kernels),
+        "kernels": {k["name"]: {"launches": k["launches"],
+                                "us_per_launch": k["ms_total"] / k["launches"] * 1e3}
+                    for k in kernels},
+        "clocks": clocks,
+    }
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -29,6 +29,12 @@ class DrProblem(ctypes.Structure):
                 ("eps", ctypes.c_float)]
 
 
+class KernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int),
+                ("ms_total", ctypes.c_double), ("bytes_per_launch", ctypes.c_double),
+                ("flops_per_launch", ctypes.c_double)]
+
+
 class DrError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
@@ -63,6 +69,10 @@ def load() -> ctypes.CDLL:
     lib.dr_last_device_error.restype = i
     lib.dr_version.argtypes = []
     lib.dr_version.restype = i
+    lib.dr_profile_enable.argtypes = [i]
+    lib.dr_profile_enable.restype = i
+    lib.dr_profile_read.argtypes = [ctypes.POINTER(KernelTime), i]
+    lib.dr_profile_read.restype = i
     _lib = lib
     return lib
 
@@ -243,3 +253,19 @@ def chunk_bwd(q, k, v, beta, g, S0, dO, dST=None, saved=None, *, beta_mode="dire
     plan = Plan(B, H, T, dk, dv, dtype=dtype, gate=gate, beta_mode=beta_mode, eps=eps,
                 chunk=chunk, device=q.device)
     return plan.bwd(q, k, v, beta, g, S0, dO, dST, saved, stream=stream)
+
+
+def profile_enable(on: bool = True) -> None:
+    """Bracket every library launch with CUDA events on its stream (or stop)."""
+    _check(load().dr_profile_enable(1 if on else 0), "dr_profile_enable")
+
+
+def profile_read() -> list[dict]:
+    """Per-kernel launches, summed event time and work model since the last read."""
+    buf = (KernelTime * 64)()
+    n = load().dr_profile_read(buf, 64)
+    if n < 0:
+        raise DrError(DR_ERR_CUDA, "dr_profile_read")
+    return [dict(name=buf[i].name.decode(), launches=buf[i].launches,
+                 ms_total=buf[i].ms_total, bytes_per_launch=buf[i].bytes_per_launch,
+                 flops_per_launch=buf[i].flops_per_launch) for i in range(n)]

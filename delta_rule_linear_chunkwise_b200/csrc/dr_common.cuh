@@ -63,6 +63,17 @@ __device__ __forceinline__ void store_f<__nv_bfloat16>(__nv_bfloat16* p, float x
   *p = __float2bfloat16_rn(x);
 }
 
+// Kernel ids for the opt-in per-kernel timing (profile.cu).
+enum {
+  kKIntraFwd = 0, kKScanFwd, kKScanBwd, kKStateGrads, kKIntraBwd,
+  kKTcIntraFwd, kKTcScanFwd, kKTcScanBwd, kKTcChunkBwd
+};
+const char* kernel_name(int id);
+// Bracket one launch with events on its stream when profiling is enabled.
+// bytes / flops: the launch's algorithmic HBM traffic and arithmetic.
+void prof_begin(int kernel, double bytes, double flops, cudaStream_t st);
+void prof_end(cudaStream_t st);
+
 // Reads the device-side error word (bounded waits that gave up record a
 // nonzero code there) into *flag and clears it.
 cudaError_t read_and_clear_device_error(int* flag);

@@ -660,6 +660,60 @@ size_t intra_bwd_smem(const Problem& p) {
 
 int pick_bv(const Problem& p) { return (p.dv % 32 == 0) ? 32 : 16; }
 
+// Work models per launch (whole grid): algorithmic HBM bytes = every tensor
+// the kernel must read or write once (inputs, outputs and the workspace
+// tensors it exchanges with the other kernels); FLOPs = 2 x multiply-adds of
+// its products, triangular products counted at their triangle.
+struct Work {
+  double bytes, flops;
+};
+Work work_of(int kernel, const Problem& p, int es, bool states_io) {
+  const double nb = (double)p.B * p.H * p.NC, C = kC, dk = p.dk, dv = p.dv, gk = p.gk;
+  const double ntok = nb * C;  // padded token-heads
+  const double grid_in = ntok * (gk * 4 + 4);          // g, beta
+  const double st = nb * dv * dk * 4;                  // one fp32 state per chunk
+  Work w{0, 0};
+  switch (kernel) {
+    case kKIntraFwd:
+      w.bytes = ntok * (2 * dk + dv) * es + grid_in +
+                ntok * (gk * 4 + 8) + nb * C * C * 8 + ntok * (dk + dv) * 4;
+      w.flops = nb * (2 * C * C * dk + C * C * C / 3 + C * C * (dk + dv));
+      break;
+    case kKScanFwd:
+      w.bytes = ntok * ((dk + dv) * 4 + gk * 4 + 2 * dk * es) + nb * C * C * 4 +
+                ntok * dv * es + (states_io ? st : 0);
+      w.flops = nb * (6 * C * dk * dv + C * C * dv);
+      break;
+    case kKScanBwd:
+      w.bytes = ntok * (dk * 4 + gk * 4 + 2 * dk * es + dv * es) + nb * C * C * 4 + st +
+                ntok * dv * 4;
+      w.flops = nb * (6 * C * dk * dv + C * C * dv);
+      break;
+    case kKStateGrads:
+      w.bytes = 2 * st + ntok * (dk * 4 + 2 * dv * 4 + dv * es) + ntok * (dv * 4 + 3 * dk * 4) +
+                nb * dk * 4;
+      w.flops = nb * 8 * C * dk * dv;
+      break;
+    case kKIntraBwd:
+      w.bytes = ntok * ((2 * dk + 2 * dv) * es + gk * 4 + 12) + nb * C * C * 4 +
+                ntok * (3 * dv + 4 * dk) * 4 + nb * dk * 4 + ntok * ((2 * dk + dv) * es + gk * 4 + 4);
+      w.flops = nb * (C * C * dv + 2 * C * C * dk + 2 * C * C * (dk + dv) + 2 * C * C * dk);
+      break;
+  }
+  return w;
+}
+
+template <typename F>
+cudaError_t timed_launch(int kernel, const Problem& p, int es, bool states_io, cudaStream_t st,
+                         F&& launch) {
+  const Work w = work_of(kernel, p, es, states_io);
+  prof_begin(kernel, w.bytes, w.flops, st);
+  launch();
+  cudaError_t e = cudaGetLastError();
+  prof_end(st);
+  return e;
+}
+
 template <typename K>
 cudaError_t set_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
@@ -672,15 +726,20 @@ cudaError_t launch_generic_fwd(const Problem& p, const TIn* q, const TIn* k, con
                                const float* beta, const float* g, const float* S0, TIn* o,
                                float* ST, float* hsave, const Ws& ws, cudaStream_t st) {
   cudaError_t e;
+  const int es = sizeof(TIn);
   const size_t s1 = intra_fwd_smem(p);
   if ((e = set_smem(k_intra_fwd<TIn>, s1)) != cudaSuccess) return e;
-  k_intra_fwd<TIn><<<dim3(p.NC, p.H, p.B), NT, s1, st>>>(p, q, k, v, beta, g, ws);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = timed_launch(kKIntraFwd, p, es, false, st, [&] {
+    k_intra_fwd<TIn><<<dim3(p.NC, p.H, p.B), NT, s1, st>>>(p, q, k, v, beta, g, ws);
+  });
+  if (e != cudaSuccess) return e;
   const int BV = pick_bv(p);
   const size_t s2 = scan_smem(p, BV);
   if ((e = set_smem(k_scan_fwd<TIn>, s2)) != cudaSuccess) return e;
-  k_scan_fwd<TIn><<<dim3(p.dv / BV, p.H, p.B), NT, s2, st>>>(p, BV, q, k, S0, o, ST, hsave, ws);
-  return cudaGetLastError();
+  return timed_launch(kKScanFwd, p, es, hsave != nullptr, st, [&] {
+    k_scan_fwd<TIn><<<dim3(p.dv / BV, p.H, p.B), NT, s2, st>>>(p, BV, q, k, S0, o, ST, hsave,
+                                                               ws);
+  });
 }
 
 template <typename TIn>
@@ -690,32 +749,42 @@ cudaError_t launch_generic_bwd(const Problem& p, const TIn* q, const TIn* k, con
                                TIn* dq, TIn* dk, TIn* dv, float* dbeta, float* dg,
                                float* dS0, const Ws& ws, cudaStream_t st) {
   cudaError_t e;
+  const int es = sizeof(TIn);
   const size_t s1 = intra_fwd_smem(p);
   if ((e = set_smem(k_intra_fwd<TIn>, s1)) != cudaSuccess) return e;
-  k_intra_fwd<TIn><<<dim3(p.NC, p.H, p.B), NT, s1, st>>>(p, q, k, v, beta, g, ws);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = timed_launch(kKIntraFwd, p, es, false, st, [&] {
+    k_intra_fwd<TIn><<<dim3(p.NC, p.H, p.B), NT, s1, st>>>(p, q, k, v, beta, g, ws);
+  });
+  if (e != cudaSuccess) return e;
   const int BV = pick_bv(p);
   const size_t s2 = scan_smem(p, BV);
   const float* hst = hsaved;
   if (!hst) {
     if ((e = set_smem(k_scan_fwd<TIn>, s2)) != cudaSuccess) return e;
-    k_scan_fwd<TIn><<<dim3(p.dv / BV, p.H, p.B), NT, s2, st>>>(p, BV, q, k, S0, nullptr,
-                                                               nullptr, ws.h, ws);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = timed_launch(kKScanFwd, p, es, true, st, [&] {
+      k_scan_fwd<TIn><<<dim3(p.dv / BV, p.H, p.B), NT, s2, st>>>(p, BV, q, k, S0, nullptr,
+                                                                 nullptr, ws.h, ws);
+    });
+    if (e != cudaSuccess) return e;
     hst = ws.h;
   }
   if ((e = set_smem(k_scan_bwd<TIn>, s2)) != cudaSuccess) return e;
-  k_scan_bwd<TIn><<<dim3(p.dv / BV, p.H, p.B), NT, s2, st>>>(p, BV, q, k, dO, dST, dS0, ws);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = timed_launch(kKScanBwd, p, es, true, st, [&] {
+    k_scan_bwd<TIn><<<dim3(p.dv / BV, p.H, p.B), NT, s2, st>>>(p, BV, q, k, dO, dST, dS0, ws);
+  });
+  if (e != cudaSuccess) return e;
   const size_t s3 = state_grads_smem(p);
   if ((e = set_smem(k_state_grads<TIn>, s3)) != cudaSuccess) return e;
-  k_state_grads<TIn><<<dim3(p.NC, p.H, p.B), NT, s3, st>>>(p, dO, hst, ws);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = timed_launch(kKStateGrads, p, es, true, st, [&] {
+    k_state_grads<TIn><<<dim3(p.NC, p.H, p.B), NT, s3, st>>>(p, dO, hst, ws);
+  });
+  if (e != cudaSuccess) return e;
   const size_t s4 = intra_bwd_smem(p);
   if ((e = set_smem(k_intra_bwd<TIn>, s4)) != cudaSuccess) return e;
-  k_intra_bwd<TIn><<<dim3(p.NC, p.H, p.B), NT, s4, st>>>(p, q, k, v, dO, beta, dq, dk, dv,
-                                                         dbeta, dg, ws);
-  return cudaGetLastError();
+  return timed_launch(kKIntraBwd, p, es, true, st, [&] {
+    k_intra_bwd<TIn><<<dim3(p.NC, p.H, p.B), NT, s4, st>>>(p, q, k, v, dO, beta, dq, dk, dv,
+                                                           dbeta, dg, ws);
+  });
 }
 
 template cudaError_t launch_generic_fwd<float>(const Problem&, const float*, const float*,

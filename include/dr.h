@@ -116,6 +116,27 @@ const char* dr_status_string(dr_status s);
    DR_ERR_CUDA if the stream reported an error, else DR_OK. */
 dr_status dr_last_device_error(void* stream);
 
+/* Opt-in per-kernel timing, for benchmarking.  While enabled (on != 0),
+   every kernel the library launches is bracketed by two CUDA events recorded
+   on the launch stream.  The first enable creates the events (no device
+   memory is allocated); enabling or disabling discards pending records. */
+dr_status dr_profile_enable(int on);
+
+/* Per-kernel summary of the launches recorded since the last read or enable:
+   name, launch count, summed event time, and the kernel's work model per
+   launch (algorithmic HBM bytes and FLOPs for the problem it ran on). */
+typedef struct {
+  char name[32];
+  int launches;
+  double ms_total;
+  double bytes_per_launch;
+  double flops_per_launch;
+} dr_kernel_time;
+
+/* Waits for the recorded events, writes up to max_out entries to out and
+   returns their number (-1 on a CUDA error); clears the records. */
+int dr_profile_read(dr_kernel_time* out, int max_out);
+
 /* Library ABI version (major * 100 + minor). */
 int dr_version(void);
 
