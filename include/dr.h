@@ -108,6 +108,35 @@ dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const 
                        float* dbeta, float* dg, float* dS0, void* ws, size_t ws_bytes,
                        void* stream);
 
+/* Size of the library's built-in forward scratch (64 MiB), held on every GPU
+   that loads the library, until the process exits. */
+#define DR_STATIC_SCRATCH_BYTES (64u << 20)
+
+/* Chunkwise forward that allocates nothing and takes no workspace, for
+   callers that cannot call cudaMalloc (for example a plugin inside a host
+   framework that owns all device memory through its own pool, or a
+   latency-critical path that cannot afford cudaMalloc's implicit device
+   synchronisation).  It has no counterpart in the paper.
+   Same arguments and results as dr_chunk_fwd without saved and workspace:
+   the scratch is a static device array of DR_STATIC_SCRATCH_BYTES shared by
+   every call in the process.
+   - Returns DR_ERR_WORKSPACE, launching nothing, when the problem's forward
+     scratch (dr_workspace_size(p, 0)) exceeds DR_STATIC_SCRATCH_BYTES; for
+     example a per-channel gate with dk = dv = 128 fits at most about 400
+     (batch x head x 64-token chunk) blocks.
+   - Uses the device current at the call, which must own `stream` and every
+     pointer.  The first call on a device looks up the scratch's device
+     address (cudaGetSymbolAddress) with that device current; make that first
+     call before any stream capture.
+   - Calls that overlap on the GPU (for example on concurrent streams, or from
+     several host threads using one device) race on the shared scratch:
+     serialise them.  The
+     scratch keeps the last call's contents; nothing in it needs clearing,
+     because each call writes every scratch region before reading it. */
+dr_status dr_chunk_fwd_static(const dr_problem* p, const void* q, const void* k,
+                              const void* v, const float* beta, const float* g,
+                              const float* S0, void* o, float* ST, void* stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* dr_status_string(dr_status s);
 
