@@ -5,6 +5,7 @@
 
 #include "../../include/dr.h"
 #include "dr_common.cuh"
+#include "fast.cuh"
 
 namespace {
 
@@ -81,7 +82,12 @@ Layout layout(const Problem& p, int pass) {
     L.off[i] = o;
     o += round_up(sz[i] * sizeof(float));
   }
-  L.total = o;
+  // The tensor-core path carves its own regions from the same workspace.
+  const size_t nb2 = (size_t)p.B * p.H * p.NC;
+  size_t fast = round_up(dr::fast::saved_bytes(p));
+  if (pass == 1)
+    fast += round_up(nb2 * dr::fast::kUBytes) + round_up(nb2 * dr::fast::kStateBytes);
+  L.total = o > fast ? o : fast;
   return L;
 }
 
@@ -110,7 +116,9 @@ Ws carve(const Layout& L, void* base, int pass) {
 }
 
 size_t saved_bytes(const Problem& p) {
-  return round_up((size_t)p.B * p.H * p.NC * p.dv * p.dk * sizeof(float));
+  const size_t generic = (size_t)p.B * p.H * p.NC * p.dv * p.dk * sizeof(float);
+  const size_t fast = dr::fast::saved_bytes(p);
+  return round_up(generic > fast ? generic : fast);
 }
 
 }  // namespace
@@ -152,6 +160,18 @@ dr_status dr_chunk_fwd(const dr_problem* p, const void* q, const void* k, const 
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
   if (P.gate == DR_GATE_NONE) g = nullptr;
+  if (dr::fast::eligible(P, p->dtype == DR_BF16)) {
+    // Tensor-core path: T and beta go to the saved buffer when given (the
+    // backward reuses them), else to the start of the workspace.
+    dr::fast::Saved sv = dr::fast::carve_saved(P, saved ? saved : ws);
+    using bf = __nv_bfloat16;
+    e = dr::fast::launch_prep(P, (const bf*)k, beta, g, sv.T, sv.beta, st);
+    if (e == cudaSuccess)
+      e = dr::fast::launch_fwd_scan(P, (const bf*)q, (const bf*)k, (const bf*)v, g, sv.T,
+                                    sv.beta, S0, (bf*)o, ST, saved ? sv.h : nullptr,
+                                    saved ? sv.U : nullptr, st);
+    return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+  }
   if (p->dtype == DR_F32)
     e = dr::launch_generic_fwd<float>(P, (const float*)q, (const float*)k, (const float*)v,
                                       beta, g, S0, (float*)o, ST, (float*)saved, w, st);
@@ -182,6 +202,34 @@ dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const 
   const Ws w = carve(L, ws, 1);
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
+  if (dr::fast::eligible(P, p->dtype == DR_BF16)) {
+    using bf = __nv_bfloat16;
+    // Saved tensors (T, beta, chunk start states h, pseudo-values U) come from
+    // the forward's saved buffer or are recomputed into the workspace.
+    char* wsb = (char*)ws;
+    dr::fast::Saved sv;
+    if (saved) {
+      sv = dr::fast::carve_saved(P, (void*)saved);
+    } else {
+      sv = dr::fast::carve_saved(P, wsb);
+      e = dr::fast::launch_prep(P, (const bf*)k, beta, g, sv.T, sv.beta, st);
+      if (e == cudaSuccess)
+        e = dr::fast::launch_fwd_scan(P, (const bf*)q, (const bf*)k, (const bf*)v, g, sv.T,
+                                      sv.beta, S0, nullptr, nullptr, sv.h, sv.U, st);
+      if (e != cudaSuccess) return DR_ERR_CUDA;
+      wsb += round_up(dr::fast::saved_bytes(P));
+    }
+    const size_t nb = (size_t)P.B * P.H * P.NC;
+    bf* dU = (bf*)wsb;
+    bf* dh = (bf*)(wsb + round_up(nb * dr::fast::kUBytes));
+    e = dr::fast::launch_bwd_scan(P, (const bf*)q, (const bf*)k, (const bf*)dO, g, sv.T,
+                                  sv.beta, dST, dS0, dU, dh, st);
+    if (e == cudaSuccess)
+      e = dr::fast::launch_bwd_chunk(P, (const bf*)q, (const bf*)k, (const bf*)v,
+                                     (const bf*)dO, g, sv.T, sv.beta, sv.h, dh, sv.U, dU,
+                                     (bf*)dq, (bf*)dk, (bf*)dv, dbeta, dg, st);
+    return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+  }
   if (p->dtype == DR_F32)
     e = dr::launch_generic_bwd<float>(P, (const float*)q, (const float*)k, (const float*)v,
                                       beta, g, S0, (const float*)dO, dST,

@@ -1,0 +1,727 @@
+// fast_bwd.cu -- tensor-core backward for bf16 storage, d_k = d_v = 128, C = 64.
+//
+// tc_bwd_scan (sequential in reverse over chunks, one CTA per (b, h, 64-wide
+// value tile)): with the fp32 gradient dS of the chunk's end state held in
+// registers,
+//   dU = M^T dO + Kt dS^T                      (M = tril(Q^c Kb^c^T), Kt = k e^{gamma_C - gamma})
+//   dS <- dS Diag(e^{gamma_C}) + dO^T (q e^gamma) - dU^T W
+// recomputing M and W = T diag(beta) (k e^gamma) per chunk from q, k, g, T.
+// Emits dU (bf16) and dh_n = dS at the end of chunk n (bf16) for the
+// chunk-parallel kernel, and dS0.
+// tc_bwd_chunk (chunk-parallel): everything else, through the triangular
+// residual system (I + A)[U' | W] = diag(beta)[V | K e^gamma]:
+//   W, U' = T diag(beta) [K e^gamma | V];  dQs = dO S;  dW = -dU S;  dKt = U dS';
+//   dM = tril(dO U^T);  Lambda = T^T [dU | dW];  dA = -strict_tril(Lambda [U' | W]^T);
+//   dQ^c = dM Kb^c;  x = dA Kb^c;  dKb^c = dM^T Q^c + dA^T diag(beta) K^c
+// and the gate chain rule (reverse cumulative sum of the per-row log-gate
+// gradient), dbeta and the Kaczmarz chain rule.
+
+#include "dr_common.cuh"
+#include "fast.cuh"
+#include "frag.cuh"
+
+namespace dr {
+namespace fast {
+
+using frag::bf16;
+
+namespace {
+
+constexpr int C = 64, D = 128;
+constexpr int LDD = D + 8;
+constexpr int LDC = C + 8;
+constexpr int BV = 64;
+constexpr int NTS = 256;
+
+__device__ __forceinline__ int centre_row(int nvalid) { return (nvalid - 1) / 2; }
+
+__device__ __forceinline__ void cumsum_col(float* G, int ld, int col) {
+  float v[C];
+#pragma unroll
+  for (int i = 0; i < C; ++i) v[i] = G[i * ld + col];
+#pragma unroll
+  for (int i = 1; i < C; ++i) v[i] += v[i - 1];
+#pragma unroll
+  for (int i = 0; i < C; ++i) G[i * ld + col] = v[i];
+}
+
+__device__ __forceinline__ void gate8(const float* G, int gk, int i, int c, float* out) {
+  if (gk == 1) {
+    const float x = G[i];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = x;
+  } else {
+    const float4 a = *reinterpret_cast<const float4*>(G + i * gk + c);
+    const float4 b = *reinterpret_cast<const float4*>(G + i * gk + c + 4);
+    out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+    out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// tc_bwd_scan
+struct BscanSmem {
+  bf16 q[C * LDD];
+  bf16 k[C * LDD];
+  bf16 dO[C * LDC];   // [i][a] slice of dO (raw, then operand)
+  bf16 T[C * LDC];
+  float beta[C];
+  bf16 Qc[C * LDD];   // then M [i][j] (stride LDC)
+  bf16 Kb[C * LDD];
+  bf16 BK[C * LDD];   // then W [i][c]
+  bf16 Qh[C * LDD];
+  bf16 Kt[C * LDD];
+  bf16 dOs[C * LDC];  // operand copy of the dO slice (the raw buffer is refilled early)
+  bf16 dU[C * LDC];
+  bf16 dS[BV * LDD];  // bf16 copy of the state gradient [a][c]
+  float dec[D];
+  float G[1];
+};
+
+__device__ void bscan_load_chunk(const Problem& p, BscanSmem& s, const bf16* q, const bf16* k,
+                                 const bf16* dO, const float* g, const bf16* T,
+                                 const float* beta, int b, int h, int n, int a0) {
+  const int tid = threadIdx.x, gk = p.gk, t0 = n * C, nvalid = min(C, p.T - t0);
+  const size_t cb = chunk_id(p, b, h, n);
+  for (int idx = tid; idx < C * (D / 8); idx += NTS) {
+    const int i = idx >> 4, j = idx & 15;
+    const bool ok = i < nvalid;
+    const size_t rr = row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 8;
+    frag::cp16(s.q + i * LDD + j * 8, q + rr, ok);
+    frag::cp16(s.k + i * LDD + j * 8, k + rr, ok);
+  }
+  for (int idx = tid; idx < C * (BV / 8); idx += NTS) {
+    const int i = idx >> 3, j = idx & 7;
+    const bool ok = i < nvalid;
+    frag::cp16(s.dO + i * LDC + j * 8, dO + row_id(p, b, t0 + (ok ? i : 0), h) * D + a0 + j * 8, ok);
+    frag::cp16(s.T + i * LDC + j * 8, T + cb * C * C + i * C + j * 8, true);
+  }
+  if (gk == D) {
+    for (int idx = tid; idx < C * (D / 4); idx += NTS) {
+      const int i = idx >> 5, j = idx & 31;
+      const bool ok = i < nvalid && p.gate != kGateNone;
+      frag::cp16(s.G + i * D + j * 4, g + row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 4, ok);
+    }
+  }
+  if (tid < C / 4) frag::cp16(s.beta + tid * 4, beta + cb * C + tid * 4, true);
+  frag::cp_commit();
+  if (gk == 1 && tid < C)
+    s.G[tid] = (tid < nvalid && p.gate != kGateNone) ? g[row_id(p, b, t0 + tid, h)] : 0.f;
+}
+
+__global__ void __launch_bounds__(NTS, 1)
+    k_bwd_scan(Problem p, const bf16* __restrict__ q, const bf16* __restrict__ k,
+               const bf16* __restrict__ dO, const float* __restrict__ g,
+               const bf16* __restrict__ Tg, const float* __restrict__ beta,
+               const float* __restrict__ dST, float* __restrict__ dS0,
+               bf16* __restrict__ dUout, bf16* __restrict__ dhout) {
+  extern __shared__ __align__(16) unsigned char smraw[];
+  BscanSmem& s = *reinterpret_cast<BscanSmem*>(smraw);
+  bf16* sW = s.BK;
+  bf16* sM = s.Qc;
+  const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31, gk = p.gk;
+  const int rb = warp & 3, hf = warp >> 2;
+  const int a0 = blockIdx.x * BV;
+  const int lr = lane >> 2, lc = 2 * (lane & 3);
+  const size_t sbase = ((size_t)b * p.H + h) * D * D;
+
+  float dS[8][4];  // rows a0 + 16rb.., key columns 64hf..
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int a = rb * 16 + lr + (e >> 1) * 8, c = hf * 64 + j * 8 + lc + (e & 1);
+      dS[j][e] = dST ? dST[sbase + (size_t)(a0 + a) * D + c] : 0.f;
+    }
+  frag::st_c(dS, s.dS, LDD, rb * 16, hf * 64);
+
+  bscan_load_chunk(p, s, q, k, dO, g, Tg, beta, b, h, p.NC - 1, a0);
+  for (int n = p.NC - 1; n >= 0; --n) {
+    const int t0 = n * C, nvalid = min(C, p.T - t0);
+    const size_t cb = chunk_id(p, b, h, n);
+    frag::cp_wait<0>();
+    __syncthreads();
+    if (tid < gk) cumsum_col(s.G, gk, tid);
+    __syncthreads();
+    const int r = centre_row(nvalid);
+    for (int idx = tid; idx < C * (D / 8); idx += NTS) {
+      const int i = idx >> 4, j = idx & 15;
+      const uint4 rq = *reinterpret_cast<const uint4*>(s.q + i * LDD + j * 8);
+      const uint4 rk = *reinterpret_cast<const uint4*>(s.k + i * LDD + j * 8);
+      const uint32_t* wq = reinterpret_cast<const uint32_t*>(&rq);
+      const uint32_t* wk = reinterpret_cast<const uint32_t*>(&rk);
+      const float bi = s.beta[i];
+      uint32_t oqc[4], okb[4], obk[4], oqh[4], okt[4];
+      float g8[8], r8[8], c8[8];
+      gate8(s.G, gk, i, j * 8, g8);
+      gate8(s.G, gk, r, j * 8, r8);
+      gate8(s.G, gk, C - 1, j * 8, c8);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fq = frag::unpack(wq[e]), fk = frag::unpack(wk[e]);
+        const float gi0 = g8[2 * e], gi1 = g8[2 * e + 1];
+        const float ep0 = __expf(gi0 - r8[2 * e]), ep1 = __expf(gi1 - r8[2 * e + 1]);
+        const float em0 = __expf(r8[2 * e] - gi0), em1 = __expf(r8[2 * e + 1] - gi1);
+        const float ea0 = __expf(gi0), ea1 = __expf(gi1);
+        const float et0 = __expf(c8[2 * e] - gi0), et1 = __expf(c8[2 * e + 1] - gi1);
+        oqc[e] = frag::pack(fq.x * ep0, fq.y * ep1);
+        okb[e] = frag::pack(fk.x * em0, fk.y * em1);
+        obk[e] = frag::pack(bi * fk.x * ea0, bi * fk.y * ea1);
+        oqh[e] = frag::pack(fq.x * ea0, fq.y * ea1);
+        okt[e] = frag::pack(fk.x * et0, fk.y * et1);
+      }
+      *reinterpret_cast<uint4*>(s.Qc + i * LDD + j * 8) = make_uint4(oqc[0], oqc[1], oqc[2], oqc[3]);
+      *reinterpret_cast<uint4*>(s.Kb + i * LDD + j * 8) = make_uint4(okb[0], okb[1], okb[2], okb[3]);
+      *reinterpret_cast<uint4*>(s.BK + i * LDD + j * 8) = make_uint4(obk[0], obk[1], obk[2], obk[3]);
+      *reinterpret_cast<uint4*>(s.Qh + i * LDD + j * 8) = make_uint4(oqh[0], oqh[1], oqh[2], oqh[3]);
+      *reinterpret_cast<uint4*>(s.Kt + i * LDD + j * 8) = make_uint4(okt[0], okt[1], okt[2], okt[3]);
+    }
+    for (int idx = tid; idx < C * (BV / 8); idx += NTS) {
+      const int i = idx >> 3, j = idx & 7;
+      *reinterpret_cast<uint4*>(s.dOs + i * LDC + j * 8) =
+          *reinterpret_cast<const uint4*>(s.dO + i * LDC + j * 8);
+    }
+    if (tid < D) s.dec[tid] = __expf((gk == D) ? s.G[(C - 1) * D + tid] : s.G[C - 1]);
+    __syncthreads();
+
+    float Wc[8][4], Mc[4][4];
+    frag::zero(Wc);
+    frag::mm_rows<8, 4, true>(Wc, s.T, LDC, rb * 16, s.BK, LDD, hf * 64);
+    frag::zero(Mc);
+    frag::mm_rows<4, 8, false>(Mc, s.Qc, LDD, rb * 16, s.Kb, LDD, hf * 32);
+#pragma unroll
+    for (int jt = 0; jt < 4; ++jt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = rb * 16 + lr + (e >> 1) * 8, jj = hf * 32 + jt * 8 + lc + (e & 1);
+        if (jj > i) Mc[jt][e] = 0.f;
+      }
+    __syncthreads();
+    frag::st_c(Wc, sW, LDD, rb * 16, hf * 64);
+    frag::st_c(Mc, sM, LDC, rb * 16, hf * 32);
+    if (n > 0) bscan_load_chunk(p, s, q, k, dO, g, Tg, beta, b, h, n - 1, a0);
+    // dh_n: gradient of this chunk's end state
+    for (int idx = tid; idx < BV * (D / 8); idx += NTS) {
+      const int a = idx >> 4, j = idx & 15;
+      *reinterpret_cast<uint4*>(dhout + cb * D * D + (size_t)(a0 + a) * D + j * 8) =
+          *reinterpret_cast<const uint4*>(s.dS + a * LDD + j * 8);
+    }
+    __syncthreads();
+
+    // dU = M^T dO + Kt dS^T, rows i = 16rb.., values 32hf..
+    {
+      float du[4][4];
+      frag::zero(du);
+      frag::mm_rows_at<4, 4, true>(du, sM, LDC, rb * 16, s.dOs, LDC, hf * 32);
+      frag::mm_rows<4, 8, false>(du, s.Kt, LDD, rb * 16, s.dS, LDD, hf * 32);
+      frag::st_c(du, s.dU, LDC, rb * 16, hf * 32);
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C * (BV / 8); idx += NTS) {
+      const int i = idx >> 3, j = idx & 7;
+      *reinterpret_cast<uint4*>(dUout + (cb * C + i) * D + a0 + j * 8) =
+          *reinterpret_cast<const uint4*>(s.dU + i * LDC + j * 8);
+    }
+    // dS <- dS Diag(e^{gamma_C}) + dO^T Qh - dU^T W, rows a = 16rb.., keys 64hf..
+    {
+      float pa[8][4], pb[8][4];
+      frag::zero(pa);
+      frag::mm_rows_at<8, 4, true>(pa, s.dOs, LDC, rb * 16, s.Qh, LDD, hf * 64);
+      frag::zero(pb);
+      frag::mm_rows_at<8, 4, true>(pb, s.dU, LDC, rb * 16, sW, LDD, hf * 64);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          dS[j][e] = dS[j][e] * s.dec[hf * 64 + j * 8 + lc + (e & 1)] + pa[j][e] - pb[j][e];
+    }
+    __syncthreads();
+    frag::st_c(dS, s.dS, LDD, rb * 16, hf * 64);
+  }
+  if (dS0) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int a = rb * 16 + lr + (e >> 1) * 8, c = hf * 64 + j * 8 + lc + (e & 1);
+        dS0[sbase + (size_t)(a0 + a) * D + c] = dS[j][e];
+      }
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// tc_bwd_chunk: 16 warps = 4 row blocks (16 chunk rows) x 4 column quarters.
+constexpr int NTB = 512;
+
+struct BchunkSmem {
+  bf16 Qc[C * LDD];     // q e^{gamma - gamma_r}
+  bf16 k[C * LDD];      // raw k
+  bf16 W[C * LDD];      // T diag(beta) k e^gamma      [j][c]
+  bf16 Up[C * LDD];     // T diag(beta) v              [j][a]
+  bf16 dO[C * LDD];
+  bf16 dU[C * LDD];
+  bf16 U[C * LDD];      // then dA [i][j] (stride LDC)
+  bf16 dW[C * LDD];
+  bf16 dM[C * LDC];     // tril(dO U^T)               [i][j]
+  bf16 T[C * LDC];
+  bf16 R[2 * C * LDD];  // beta k e^gamma | beta v  ->  S half | dS' half  ->  Lambda_U | Lambda_W
+                        // -> Kb^c | beta K^c  ->  dgamma (fp32 [C][D])
+  float beta[C];
+  float knorm[C];
+  float dbp[C * 4];     // dbeta partial sums per column quarter
+  float dgc[4 * D];     // colsum(dS' .* S) partials per row quarter
+  float ktk[4 * D];     // colsum(Kt .* dKt) partials per row block
+  float G[1];           // [C][gk] cumulative gate (dynamic tail)
+};
+
+__global__ void __launch_bounds__(NTB, 1)
+    k_bwd_chunk(Problem p, const bf16* __restrict__ q, const bf16* __restrict__ k,
+                const bf16* __restrict__ v, const bf16* __restrict__ dO,
+                const float* __restrict__ g, const bf16* __restrict__ Tg,
+                const float* __restrict__ beta, const bf16* __restrict__ hst,
+                const bf16* __restrict__ dhst, const bf16* __restrict__ Ug,
+                const bf16* __restrict__ dUg, bf16* __restrict__ dq, bf16* __restrict__ dk,
+                bf16* __restrict__ dv, float* __restrict__ dbeta, float* __restrict__ dg) {
+  extern __shared__ __align__(16) unsigned char smraw[];
+  BchunkSmem& s = *reinterpret_cast<BchunkSmem*>(smraw);
+  const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31, gk = p.gk;
+  const int rb = warp & 3, qt = warp >> 2;
+  const int lr = lane >> 2, lc = 2 * (lane & 3);
+  const int t0 = n * C, nvalid = min(C, p.T - t0);
+  const size_t cb = chunk_id(p, b, h, n);
+  bf16* R0 = s.R;            // first half of the shared region
+  bf16* R1 = s.R + C * LDD;  // second half
+  bf16* sdA = s.U;
+
+  // ---- loads: q (into Qc), k, v (into R1), dO, dU, U, T, gate, beta
+  for (int idx = tid; idx < C * (D / 8); idx += NTB) {
+    const int i = idx >> 4, j = idx & 15;
+    const bool ok = i < nvalid;
+    const size_t rr = row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 8;
+    frag::cp16(s.Qc + i * LDD + j * 8, q + rr, ok);
+    frag::cp16(s.k + i * LDD + j * 8, k + rr, ok);
+    frag::cp16(R1 + i * LDD + j * 8, v + rr, ok);
+    frag::cp16(s.dO + i * LDD + j * 8, dO + rr, ok);
+    frag::cp16(s.dU + i * LDD + j * 8, dUg + (cb * C + i) * D + j * 8, true);
+    frag::cp16(s.U + i * LDD + j * 8, Ug + (cb * C + i) * D + j * 8, true);
+  }
+  for (int idx = tid; idx < C * (C / 8); idx += NTB) {
+    const int i = idx >> 3, j = idx & 7;
+    frag::cp16(s.T + i * LDC + j * 8, Tg + cb * C * C + i * C + j * 8, true);
+  }
+  if (gk == D) {
+    for (int idx = tid; idx < C * (D / 4); idx += NTB) {
+      const int i = idx >> 5, j = idx & 31;
+      const bool ok = i < nvalid && p.gate != kGateNone;
+      frag::cp16(s.G + i * D + j * 4, g + row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 4, ok);
+    }
+  } else if (tid < C) {
+    s.G[tid] = (tid < nvalid && p.gate != kGateNone) ? g[row_id(p, b, t0 + tid, h)] : 0.f;
+  }
+  if (tid < C) s.beta[tid] = beta[cb * C + tid];
+  frag::cp_commit();
+  frag::cp_wait<0>();
+  __syncthreads();
+  if (tid < gk) cumsum_col(s.G, gk, tid);
+  __syncthreads();
+
+  const int r = centre_row(nvalid);
+  // per-element gate: gamma(i, c)
+  auto gam = [&](int i, int c) -> float { return gk == D ? s.G[i * D + c] : s.G[i]; };
+
+  // ---- build: Q^c in place, beta k e^gamma into R0, beta v in place in R1, key norms
+  for (int idx = tid; idx < C * (D / 8); idx += NTB) {
+    const int i = idx >> 4, j = idx & 15;
+    uint4 rq = *reinterpret_cast<const uint4*>(s.Qc + i * LDD + j * 8);
+    uint4 rk = *reinterpret_cast<const uint4*>(s.k + i * LDD + j * 8);
+    uint4 rv = *reinterpret_cast<const uint4*>(R1 + i * LDD + j * 8);
+    uint32_t* wq = reinterpret_cast<uint32_t*>(&rq);
+    const uint32_t* wk = reinterpret_cast<const uint32_t*>(&rk);
+    uint32_t* wv = reinterpret_cast<uint32_t*>(&rv);
+    const float bi = s.beta[i];
+    float g8[8], r8[8];
+    gate8(s.G, gk, i, j * 8, g8);
+    gate8(s.G, gk, r, j * 8, r8);
+    uint32_t obk[4];
+    float nn = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 fq = frag::unpack(wq[e]), fk = frag::unpack(wk[e]), fv = frag::unpack(wv[e]);
+      wq[e] = frag::pack(fq.x * __expf(g8[2 * e] - r8[2 * e]), fq.y * __expf(g8[2 * e + 1] - r8[2 * e + 1]));
+      obk[e] = frag::pack(bi * fk.x * __expf(g8[2 * e]), bi * fk.y * __expf(g8[2 * e + 1]));
+      wv[e] = frag::pack(bi * fv.x, bi * fv.y);
+      nn += fk.x * fk.x + fk.y * fk.y;
+    }
+    *reinterpret_cast<uint4*>(s.Qc + i * LDD + j * 8) = rq;
+    *reinterpret_cast<uint4*>(R0 + i * LDD + j * 8) = make_uint4(obk[0], obk[1], obk[2], obk[3]);
+    *reinterpret_cast<uint4*>(R1 + i * LDD + j * 8) = rv;
+    nn += __shfl_xor_sync(0xffffffffu, nn, 8);
+    nn += __shfl_xor_sync(0xffffffffu, nn, 4);
+    nn += __shfl_xor_sync(0xffffffffu, nn, 2);
+    nn += __shfl_xor_sync(0xffffffffu, nn, 1);
+    if (j == 0) s.knorm[i] = nn;
+  }
+  __syncthreads();
+
+  // ---- phase 1a: W = T (beta K e^gamma), U' = T (beta V); rows 16rb.., cols 32qt..
+  {
+    float w4[4][4], u4[4][4];
+    frag::zero(w4);
+    frag::mm_rows<4, 4, true>(w4, s.T, LDC, rb * 16, R0, LDD, qt * 32);
+    frag::zero(u4);
+    frag::mm_rows<4, 4, true>(u4, s.T, LDC, rb * 16, R1, LDD, qt * 32);
+    frag::st_c(w4, s.W, LDD, rb * 16, qt * 32);
+    frag::st_c(u4, s.Up, LDD, rb * 16, qt * 32);
+  }
+  __syncthreads();
+
+  // ---- phase 1b/1c over two halves of the value dimension a
+  float zq[4][4], adw[4][4], akt[4][4], adm[2][4];
+  frag::zero(zq);
+  frag::zero(adw);
+  frag::zero(akt);
+  frag::zero(adm);
+  for (int ah = 0; ah < 2; ++ah) {
+    for (int idx = tid; idx < C * (D / 8); idx += NTB) {
+      const int a = idx >> 4, j = idx & 15;
+      frag::cp16(R0 + a * LDD + j * 8, hst + cb * D * D + (size_t)(ah * 64 + a) * D + j * 8, true);
+      frag::cp16(R1 + a * LDD + j * 8, dhst + cb * D * D + (size_t)(ah * 64 + a) * D + j * 8, true);
+    }
+    frag::cp_commit();
+    frag::cp_wait<0>();
+    __syncthreads();
+    // dQs += dO S ; dW' += dU S ; dKt += U dS'   (contraction over this half of a)
+    // The half tiles hold local rows 0..63; mm_rows indexes B rows from k0 = 64ah.
+    const bf16* Sh = R0 - ah * 64 * LDD;
+    const bf16* dSh = R1 - ah * 64 * LDD;
+    frag::mm_rows<4, 4, true>(zq, s.dO, LDD, rb * 16, Sh, LDD, qt * 32, ah * 64);
+    frag::mm_rows<4, 4, true>(adw, s.dU, LDD, rb * 16, Sh, LDD, qt * 32, ah * 64);
+    frag::mm_rows<4, 4, true>(akt, s.U, LDD, rb * 16, dSh, LDD, qt * 32, ah * 64);
+    // dM += dO U^T  (U stored [j][a] = [n][k])
+    frag::mm_rows<2, 4, false>(adm, s.dO, LDD, rb * 16, s.U, LDD, qt * 16, ah * 64);
+    // colsum(dS' .* S) over this half: thread -> column c, row quarter rq
+    {
+      const int c = tid & 127, rq = tid >> 7;
+      float acc = 0.f;
+#pragma unroll 4
+      for (int a = rq * 16; a < rq * 16 + 16; ++a)
+        acc += __bfloat162float(R0[a * LDD + c]) * __bfloat162float(R1[a * LDD + c]);
+      s.dgc[rq * D + c] = (ah == 0 ? 0.f : s.dgc[rq * D + c]) + acc;
+    }
+    __syncthreads();
+  }
+  // dW = -dW', dM masked (inclusive lower), stored for the later phases
+  {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) adw[j][e] = -adw[j][e];
+    frag::st_c(adw, s.dW, LDD, rb * 16, qt * 32);
+#pragma unroll
+    for (int jt = 0; jt < 2; ++jt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = rb * 16 + lr + (e >> 1) * 8, jj = qt * 16 + jt * 8 + lc + (e & 1);
+        if (jj > i) adm[jt][e] = 0.f;
+      }
+    frag::st_c(adm, s.dM, LDC, rb * 16, qt * 16);
+  }
+
+  // Per-element bookkeeping: thread element (jt, e) -> row i, key column c.
+  float dkacc[4][4], dgacc[4][4];
+  float gr4[4][2], gc4[4][2];  // gamma_r and gamma_C of this thread's columns
+#pragma unroll
+  for (int jt = 0; jt < 4; ++jt)
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int c = qt * 32 + jt * 8 + lc + u;
+      gr4[jt][u] = gam(r, c);
+      gc4[jt][u] = gam(C - 1, c);
+    }
+  // consume dKt: dk += e^{gamma_C - gamma} dKt ; dgamma -= Kt dKt ; column sums of Kt dKt
+  {
+    float cs[4][2] = {};
+#pragma unroll
+    for (int jt = 0; jt < 4; ++jt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = rb * 16 + lr + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
+        const float et = __expf(gc4[jt][e & 1] - gam(i, c));
+        const float kt = __bfloat162float(s.k[i * LDD + c]) * et;
+        dkacc[jt][e] = et * akt[jt][e];
+        dgacc[jt][e] = -kt * akt[jt][e];
+        cs[jt][e & 1] += kt * akt[jt][e];
+        // Q-side: Z = e^{gamma_r} dQs (dq and the q terms are finished in phase 4)
+        zq[jt][e] *= __expf(gr4[jt][e & 1]);
+      }
+#pragma unroll
+    for (int jt = 0; jt < 4; ++jt)
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        float x = cs[jt][u];
+        x += __shfl_xor_sync(0xffffffffu, x, 4);
+        x += __shfl_xor_sync(0xffffffffu, x, 8);
+        x += __shfl_xor_sync(0xffffffffu, x, 16);
+        if (lr == 0) s.ktk[rb * D + qt * 32 + jt * 8 + lc + u] = x;
+      }
+  }
+  __syncthreads();
+
+  // ---- phase 2: Lambda = T^T [dU | dW]
+  float dbrow[2] = {0.f, 0.f};  // this thread's dbeta partials for rows lr, lr + 8
+  {
+    float lu[4][4];
+    frag::zero(lu);
+    frag::mm_rows_at<4, 4, true>(lu, s.T, LDC, rb * 16, s.dU, LDD, qt * 32);
+#pragma unroll
+    for (int jt = 0; jt < 4; ++jt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int i = rb * 16 + lr + hh * 8, a = qt * 32 + jt * 8 + lc;
+        const float bi = s.beta[i];
+        if (i < nvalid) {
+          const size_t rr = row_id(p, b, t0 + i, h) * D + a;
+          *reinterpret_cast<uint32_t*>(dv + rr) =
+              frag::pack(bi * lu[jt][2 * hh], bi * lu[jt][2 * hh + 1]);
+          const float2 vv = frag::unpack(*reinterpret_cast<const uint32_t*>(v + rr));
+          dbrow[hh] += lu[jt][2 * hh] * vv.x + lu[jt][2 * hh + 1] * vv.y;
+        }
+      }
+    frag::st_c(lu, R0, LDD, rb * 16, qt * 32);
+    float lw[4][4];
+    frag::zero(lw);
+    frag::mm_rows_at<4, 4, true>(lw, s.T, LDC, rb * 16, s.dW, LDD, qt * 32);
+#pragma unroll
+    for (int jt = 0; jt < 4; ++jt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = rb * 16 + lr + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
+        const float ea = __expf(gam(i, c));
+        const float kh = __bfloat162float(s.k[i * LDD + c]) * ea;  // K e^gamma
+        const float bi = s.beta[i];
+        dkacc[jt][e] += ea * bi * lw[jt][e];
+        dgacc[jt][e] += kh * bi * lw[jt][e];
+        dbrow[e >> 1] += lw[jt][e] * kh;
+      }
+    frag::st_c(lw, R1, LDD, rb * 16, qt * 32);
+  }
+  __syncthreads();
+
+  // ---- phase 3: dA = -strict_tril(Lambda_U U'^T + Lambda_W W^T), rows 16rb.., cols 16qt..
+  {
+    float da[2][4];
+    frag::zero(da);
+    frag::mm_rows<2, 8, false>(da, R0, LDD, rb * 16, s.Up, LDD, qt * 16);
+    frag::mm_rows<2, 8, false>(da, R1, LDD, rb * 16, s.W, LDD, qt * 16);
+#pragma unroll
+    for (int jt = 0; jt < 2; ++jt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = rb * 16 + lr + (e >> 1) * 8, jj = qt * 16 + jt * 8 + lc + (e & 1);
+        da[jt][e] = (jj < i) ? -da[jt][e] : 0.f;
+      }
+    frag::st_c(da, sdA, LDC, rb * 16, qt * 16);
+  }
+  __syncthreads();
+
+  // ---- phase 4: Kb^c into R0, beta K^c into R1
+  for (int idx = tid; idx < C * (D / 8); idx += NTB) {
+    const int i = idx >> 4, j = idx & 15;
+    const uint4 rk = *reinterpret_cast<const uint4*>(s.k + i * LDD + j * 8);
+    const uint32_t* wk = reinterpret_cast<const uint32_t*>(&rk);
+    const float bi = s.beta[i];
+    float g8[8], r8[8];
+    gate8(s.G, gk, i, j * 8, g8);
+    gate8(s.G, gk, r, j * 8, r8);
+    uint32_t okb[4], obc[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 fk = frag::unpack(wk[e]);
+      okb[e] = frag::pack(fk.x * __expf(r8[2 * e] - g8[2 * e]), fk.y * __expf(r8[2 * e + 1] - g8[2 * e + 1]));
+      obc[e] = frag::pack(bi * fk.x * __expf(g8[2 * e] - r8[2 * e]), bi * fk.y * __expf(g8[2 * e + 1] - r8[2 * e + 1]));
+    }
+    *reinterpret_cast<uint4*>(R0 + i * LDD + j * 8) = make_uint4(okb[0], okb[1], okb[2], okb[3]);
+    *reinterpret_cast<uint4*>(R1 + i * LDD + j * 8) = make_uint4(obc[0], obc[1], obc[2], obc[3]);
+  }
+  __syncthreads();
+  {
+    // dQ^c = dM Kb^c -> dq = e^{gamma - gamma_r} (Z + dQ^c); dgamma += Q^c (Z + dQ^c)
+    float dqc[4][4];
+    frag::zero(dqc);
+    frag::mm_rows<4, 4, true>(dqc, s.dM, LDC, rb * 16, R0, LDD, qt * 32);
+#pragma unroll
+    for (int jt = 0; jt < 4; ++jt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int i = rb * 16 + lr + hh * 8, c = qt * 32 + jt * 8 + lc;
+        float out[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int e = 2 * hh + u;
+          const float zz = zq[jt][e] + dqc[jt][e];
+          out[u] = __expf(gam(i, c + u) - gr4[jt][u]) * zz;
+          dgacc[jt][e] += __bfloat162float(s.Qc[i * LDD + c + u]) * zz;
+        }
+        if (i < nvalid)
+          *reinterpret_cast<uint32_t*>(dq + row_id(p, b, t0 + i, h) * D + c) = frag::pack(out[0], out[1]);
+      }
+    // x = dA Kb^c: dk += e^{gamma - gamma_r} beta x; dgamma += K^c beta x; dbeta += K^c . x
+    float x[4][4];
+    frag::zero(x);
+    frag::mm_rows<4, 4, true>(x, sdA, LDC, rb * 16, R0, LDD, qt * 32);
+#pragma unroll
+    for (int jt = 0; jt < 4; ++jt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = rb * 16 + lr + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
+        const float ep = __expf(gam(i, c) - gr4[jt][e & 1]);
+        const float kc = __bfloat162float(s.k[i * LDD + c]) * ep;
+        const float bi = s.beta[i];
+        dkacc[jt][e] += ep * bi * x[jt][e];
+        dgacc[jt][e] += kc * bi * x[jt][e];
+        dbrow[e >> 1] += kc * x[jt][e];
+      }
+    // y = dM^T Q^c + dA^T (beta K^c): dk += e^{gamma_r - gamma} y; dgamma -= Kb^c y
+    float y[4][4];
+    frag::zero(y);
+    frag::mm_rows_at<4, 4, true>(y, s.dM, LDC, rb * 16, s.Qc, LDD, qt * 32);
+    frag::mm_rows_at<4, 4, true>(y, sdA, LDC, rb * 16, R1, LDD, qt * 32);
+#pragma unroll
+    for (int jt = 0; jt < 4; ++jt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = rb * 16 + lr + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
+        const float em = __expf(gr4[jt][e & 1] - gam(i, c));
+        const float kb = __bfloat162float(s.k[i * LDD + c]) * em;
+        dkacc[jt][e] += em * y[jt][e];
+        dgacc[jt][e] -= kb * y[jt][e];
+      }
+  }
+  // dbeta partials: reduce the 4 lanes that share a row, then one slot per quarter
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    float xx = dbrow[hh];
+    xx += __shfl_xor_sync(0xffffffffu, xx, 1);
+    xx += __shfl_xor_sync(0xffffffffu, xx, 2);
+    if ((lane & 3) == 0) s.dbp[(rb * 16 + lr + hh * 8) * 4 + qt] = xx;
+  }
+  __syncthreads();  // R0/R1 free: reuse as the fp32 dgamma tile
+  float* sdg = reinterpret_cast<float*>(s.R);
+#pragma unroll
+  for (int jt = 0; jt < 4; ++jt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = rb * 16 + lr + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
+      sdg[i * D + c] = dgacc[jt][e];
+    }
+  if (tid < C) {
+    const float db = s.dbp[tid * 4] + s.dbp[tid * 4 + 1] + s.dbp[tid * 4 + 2] + s.dbp[tid * 4 + 3];
+    s.dbp[tid * 4] = db;  // total d(beta_eff) of row tid
+  }
+  __syncthreads();
+  // dk (with the Kaczmarz chain rule) and dbeta
+#pragma unroll
+  for (int jt = 0; jt < 4; ++jt)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int i = rb * 16 + lr + hh * 8, c = qt * 32 + jt * 8 + lc;
+      float out[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        float val = dkacc[jt][2 * hh + u];
+        if (p.beta_mode == kBetaKaczmarz)
+          val += -2.f * s.beta[i] * s.dbp[i * 4] * __bfloat162float(s.k[i * LDD + c + u]) /
+                 (s.knorm[i] + p.eps);
+        out[u] = val;
+      }
+      if (i < nvalid)
+        *reinterpret_cast<uint32_t*>(dk + row_id(p, b, t0 + i, h) * D + c) = frag::pack(out[0], out[1]);
+    }
+  if (tid < nvalid) {
+    float db = s.dbp[tid * 4];
+    if (p.beta_mode == kBetaKaczmarz) db /= (s.knorm[tid] + p.eps);
+    dbeta[row_id(p, b, t0 + tid, h)] = db;
+  }
+  // dgamma: last row gets the chunk-decay terms, then reverse cumulative sum per channel
+  if (tid < D) {
+    const int c = tid;
+    const float eC = __expf(gam(C - 1, c));
+    float extra = s.ktk[c] + s.ktk[D + c] + s.ktk[2 * D + c] + s.ktk[3 * D + c];
+    extra += eC * (s.dgc[c] + s.dgc[D + c] + s.dgc[2 * D + c] + s.dgc[3 * D + c]);
+    sdg[(C - 1) * D + c] += extra;
+    float run = 0.f;
+    for (int i = C - 1; i >= 0; --i) {
+      run += sdg[i * D + c];
+      sdg[i * D + c] = run;
+      if (gk == D && i < nvalid) dg[row_id(p, b, t0 + i, h) * D + c] = run;
+    }
+  }
+  if (gk == 1 && p.gate != kGateNone) {
+    __syncthreads();
+    if (tid < nvalid) {
+      float sum = 0.f;
+      for (int c = 0; c < D; ++c) sum += sdg[tid * D + c];
+      dg[row_id(p, b, t0 + tid, h)] = sum;
+    }
+  }
+}
+
+}  // namespace
+
+size_t bwd_scan_smem(const Problem& p) { return sizeof(BscanSmem) + sizeof(float) * (C * p.gk); }
+
+cudaError_t launch_bwd_scan(const Problem& p, const bf16* q, const bf16* k, const bf16* dO,
+                            const float* g, const bf16* T, const float* beta_eff,
+                            const float* dST, float* dS0, bf16* dU, bf16* dh, cudaStream_t st) {
+  const size_t sm = bwd_scan_smem(p);
+  cudaError_t e =
+      cudaFuncSetAttribute(k_bwd_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  const double nb = (double)p.B * p.H * p.NC, ntok = nb * C, heads = (double)p.B * p.H;
+  double bytes = ntok * (2 * D * 2 + D * 2 + p.gk * 4 + 4) + nb * C * C * 2 + ntok * D * 2 +
+                 nb * D * D * 2 + heads * D * D * 4 * ((dST ? 1 : 0) + (dS0 ? 1 : 0));
+  const double per_tile = 2.0 * C * C * D * 2 + 2.0 * C * C * BV + 2.0 * C * BV * D * 3;
+  const double flops = nb * (D / BV) * per_tile;
+  prof_begin(kKTcScanBwd, bytes, flops, st);
+  k_bwd_scan<<<dim3(D / BV, p.H, p.B), NTS, sm, st>>>(p, q, k, dO, g, T, beta_eff, dST, dS0,
+                                                      dU, dh);
+  e = cudaGetLastError();
+  prof_end(st);
+  return e;
+}
+
+size_t bwd_chunk_smem(const Problem& p) {
+  return sizeof(BchunkSmem) + sizeof(float) * (C * p.gk);
+}
+
+cudaError_t launch_bwd_chunk(const Problem& p, const bf16* q, const bf16* k, const bf16* v,
+                             const bf16* dO, const float* g, const bf16* T,
+                             const float* beta_eff, const bf16* h, const bf16* dh,
+                             const bf16* U, const bf16* dU, bf16* dq, bf16* dk, bf16* dv,
+                             float* dbeta, float* dg, cudaStream_t st) {
+  const size_t sm = bwd_chunk_smem(p);
+  cudaError_t e =
+      cudaFuncSetAttribute(k_bwd_chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  const double nb = (double)p.B * p.H * p.NC, ntok = nb * C;
+  const double bytes = ntok * (4 * D * 2 + p.gk * 4 + 4) + nb * C * C * 2 + nb * 2.0 * D * D * 2 +
+                       ntok * 2 * D * 2 + ntok * (3 * D * 2 + p.gk * 4 + 4);
+  const double mac = (double)C * D * C * 2      // W, U'
+                     + (double)C * D * D * 3    // dO S, dU S, U dS'
+                     + (double)C * C * D        // dO U^T
+                     + (double)C * D * C * 2    // Lambda
+                     + (double)C * C * D * 2    // dA
+                     + (double)C * D * C * 4;   // dM Kb, dA Kb, dM^T Q^c, dA^T K^c
+  prof_begin(kKTcChunkBwd, bytes, nb * 2.0 * mac, st);
+  k_bwd_chunk<<<dim3(p.NC, p.H, p.B), NTB, sm, st>>>(p, q, k, v, dO, g, T, beta_eff, h, dh, U,
+                                                     dU, dq, dk, dv, dbeta, dg);
+  e = cudaGetLastError();
+  prof_end(st);
+  return e;
+}
+
+}  // namespace fast
+}  // namespace dr
