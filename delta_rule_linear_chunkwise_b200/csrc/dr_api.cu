@@ -161,15 +161,13 @@ dr_status dr_chunk_fwd(const dr_problem* p, const void* q, const void* k, const 
   cudaError_t e;
   if (P.gate == DR_GATE_NONE) g = nullptr;
   if (dr::fast::eligible(P, p->dtype == DR_BF16)) {
-    // Tensor-core path: T and beta go to the saved buffer when given (the
-    // backward reuses them), else to the start of the workspace.
+    // Tensor-core path: the per-chunk tiles go to the saved buffer when given
+    // (the backward reuses them), else to the workspace.
     dr::fast::Saved sv = dr::fast::carve_saved(P, saved ? saved : ws);
     using bf = __nv_bfloat16;
-    e = dr::fast::launch_prep(P, (const bf*)k, beta, g, sv.T, sv.beta, st);
+    e = dr::fast::launch_prep(P, (const bf*)q, (const bf*)k, (const bf*)v, beta, g, sv, st);
     if (e == cudaSuccess)
-      e = dr::fast::launch_fwd_scan(P, (const bf*)q, (const bf*)k, (const bf*)v, g, sv.T,
-                                    sv.beta, S0, (bf*)o, ST, saved ? sv.h : nullptr,
-                                    saved ? sv.U : nullptr, st);
+      e = dr::fast::launch_fwd_scan(P, sv, S0, (bf*)o, ST, saved != nullptr, st);
     return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
   }
   if (p->dtype == DR_F32)
@@ -204,30 +202,27 @@ dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const 
   cudaError_t e;
   if (dr::fast::eligible(P, p->dtype == DR_BF16)) {
     using bf = __nv_bfloat16;
-    // Saved tensors (T, beta, chunk start states h, pseudo-values U) come from
-    // the forward's saved buffer or are recomputed into the workspace.
+    // The forward's per-chunk tensors come from its saved buffer or are
+    // recomputed into the workspace.
     char* wsb = (char*)ws;
     dr::fast::Saved sv;
     if (saved) {
       sv = dr::fast::carve_saved(P, (void*)saved);
     } else {
       sv = dr::fast::carve_saved(P, wsb);
-      e = dr::fast::launch_prep(P, (const bf*)k, beta, g, sv.T, sv.beta, st);
-      if (e == cudaSuccess)
-        e = dr::fast::launch_fwd_scan(P, (const bf*)q, (const bf*)k, (const bf*)v, g, sv.T,
-                                      sv.beta, S0, nullptr, nullptr, sv.h, sv.U, st);
+      e = dr::fast::launch_prep(P, (const bf*)q, (const bf*)k, (const bf*)v, beta, g, sv, st);
+      if (e == cudaSuccess) e = dr::fast::launch_fwd_scan(P, sv, S0, nullptr, nullptr, true, st);
       if (e != cudaSuccess) return DR_ERR_CUDA;
       wsb += round_up(dr::fast::saved_bytes(P));
     }
     const size_t nb = (size_t)P.B * P.H * P.NC;
     bf* dU = (bf*)wsb;
     bf* dh = (bf*)(wsb + round_up(nb * dr::fast::kUBytes));
-    e = dr::fast::launch_bwd_scan(P, (const bf*)q, (const bf*)k, (const bf*)dO, g, sv.T,
-                                  sv.beta, dST, dS0, dU, dh, st);
+    e = dr::fast::launch_bwd_scan(P, sv, (const bf*)dO, dST, dS0, dU, dh, st);
     if (e == cudaSuccess)
       e = dr::fast::launch_bwd_chunk(P, (const bf*)q, (const bf*)k, (const bf*)v,
-                                     (const bf*)dO, g, sv.T, sv.beta, sv.h, dh, sv.U, dU,
-                                     (bf*)dq, (bf*)dk, (bf*)dv, dbeta, dg, st);
+                                     (const bf*)dO, g, sv, dh, dU, (bf*)dq, (bf*)dk, (bf*)dv,
+                                     dbeta, dg, st);
     return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
   }
   if (p->dtype == DR_F32)

@@ -59,68 +59,49 @@ __device__ __forceinline__ void gate8(const float* G, int gk, int i, int c, floa
 }
 
 // ---------------------------------------------------------------------------
-// tc_bwd_scan
-struct BscanSmem {
-  bf16 q[C * LDD];
-  bf16 k[C * LDD];
-  bf16 dO[C * LDC];   // [i][a] slice of dO (raw, then operand)
-  bf16 T[C * LDC];
-  float beta[C];
-  bf16 Qc[C * LDD];   // then M [i][j] (stride LDC)
-  bf16 Kb[C * LDD];
-  bf16 BK[C * LDD];   // then W [i][c]
+// tc_bwd_scan (thin): streams W, Qh, Kt, M, dec and the dO slice of each chunk
+// through a two-stage cp.async pipeline; only the state-gradient chain runs here.
+struct BscanStage {
+  bf16 W[C * LDD];
   bf16 Qh[C * LDD];
   bf16 Kt[C * LDD];
-  bf16 dOs[C * LDC];  // operand copy of the dO slice (the raw buffer is refilled early)
-  bf16 dU[C * LDC];
-  bf16 dS[BV * LDD];  // bf16 copy of the state gradient [a][c]
+  bf16 M[C * LDC];
+  bf16 dO[C * LDC];   // dO[:, a0 .. a0+63]
   float dec[D];
-  float G[1];
+};
+struct BscanSmem {
+  BscanStage st[2];
+  bf16 dS[BV * LDD];  // bf16 copy of the state gradient [a][c]
+  bf16 dU[C * LDC];
 };
 
-__device__ void bscan_load_chunk(const Problem& p, BscanSmem& s, const bf16* q, const bf16* k,
-                                 const bf16* dO, const float* g, const bf16* T,
-                                 const float* beta, int b, int h, int n, int a0) {
-  const int tid = threadIdx.x, gk = p.gk, t0 = n * C, nvalid = min(C, p.T - t0);
+__device__ void bscan_issue(const Problem& p, BscanStage& s, const Saved& sv, const bf16* dO,
+                            int b, int h, int n, int a0) {
+  const int tid = threadIdx.x, t0 = n * C, nvalid = min(C, p.T - t0);
   const size_t cb = chunk_id(p, b, h, n);
   for (int idx = tid; idx < C * (D / 8); idx += NTS) {
     const int i = idx >> 4, j = idx & 15;
-    const bool ok = i < nvalid;
-    const size_t rr = row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 8;
-    frag::cp16(s.q + i * LDD + j * 8, q + rr, ok);
-    frag::cp16(s.k + i * LDD + j * 8, k + rr, ok);
+    const size_t o = (cb * C + i) * D + j * 8;
+    frag::cp16(s.W + i * LDD + j * 8, sv.W + o, true);
+    frag::cp16(s.Qh + i * LDD + j * 8, sv.Qh + o, true);
+    frag::cp16(s.Kt + i * LDD + j * 8, sv.Kt + o, true);
   }
-  for (int idx = tid; idx < C * (BV / 8); idx += NTS) {
+  for (int idx = tid; idx < C * (C / 8); idx += NTS) {
     const int i = idx >> 3, j = idx & 7;
     const bool ok = i < nvalid;
+    frag::cp16(s.M + i * LDC + j * 8, sv.M + cb * C * C + i * C + j * 8, true);
     frag::cp16(s.dO + i * LDC + j * 8, dO + row_id(p, b, t0 + (ok ? i : 0), h) * D + a0 + j * 8, ok);
-    frag::cp16(s.T + i * LDC + j * 8, T + cb * C * C + i * C + j * 8, true);
   }
-  if (gk == D) {
-    for (int idx = tid; idx < C * (D / 4); idx += NTS) {
-      const int i = idx >> 5, j = idx & 31;
-      const bool ok = i < nvalid && p.gate != kGateNone;
-      frag::cp16(s.G + i * D + j * 4, g + row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 4, ok);
-    }
-  }
-  if (tid < C / 4) frag::cp16(s.beta + tid * 4, beta + cb * C + tid * 4, true);
-  frag::cp_commit();
-  if (gk == 1 && tid < C)
-    s.G[tid] = (tid < nvalid && p.gate != kGateNone) ? g[row_id(p, b, t0 + tid, h)] : 0.f;
+  if (tid < D / 4) frag::cp16(s.dec + tid * 4, sv.dec + cb * D + tid * 4, true);
 }
 
 __global__ void __launch_bounds__(NTS, 1)
-    k_bwd_scan(Problem p, const bf16* __restrict__ q, const bf16* __restrict__ k,
-               const bf16* __restrict__ dO, const float* __restrict__ g,
-               const bf16* __restrict__ Tg, const float* __restrict__ beta,
-               const float* __restrict__ dST, float* __restrict__ dS0,
-               bf16* __restrict__ dUout, bf16* __restrict__ dhout) {
+    k_bwd_scan(Problem p, Saved sv, const bf16* __restrict__ dO, const float* __restrict__ dST,
+               float* __restrict__ dS0, bf16* __restrict__ dUout, bf16* __restrict__ dhout) {
   extern __shared__ __align__(16) unsigned char smraw[];
   BscanSmem& s = *reinterpret_cast<BscanSmem*>(smraw);
-  bf16* sW = s.BK;
-  bf16* sM = s.Qc;
   const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31, gk = p.gk;
+  const int warp = tid >> 5, lane = tid & 31;
   const int rb = warp & 3, hf = warp >> 2;
   const int a0 = blockIdx.x * BV;
   const int lr = lane >> 2, lc = 2 * (lane & 3);
@@ -136,85 +117,27 @@ __global__ void __launch_bounds__(NTS, 1)
     }
   frag::st_c(dS, s.dS, LDD, rb * 16, hf * 64);
 
-  bscan_load_chunk(p, s, q, k, dO, g, Tg, beta, b, h, p.NC - 1, a0);
-  for (int n = p.NC - 1; n >= 0; --n) {
-    const int t0 = n * C, nvalid = min(C, p.T - t0);
+  bscan_issue(p, s.st[0], sv, dO, b, h, p.NC - 1, a0);
+  frag::cp_commit();
+  if (p.NC > 1) bscan_issue(p, s.st[1], sv, dO, b, h, p.NC - 2, a0);
+  frag::cp_commit();
+  for (int n = p.NC - 1, it = 0; n >= 0; --n, ++it) {
     const size_t cb = chunk_id(p, b, h, n);
-    frag::cp_wait<0>();
+    BscanStage& st = s.st[it & 1];
+    frag::cp_wait<1>();
     __syncthreads();
-    if (tid < gk) cumsum_col(s.G, gk, tid);
-    __syncthreads();
-    const int r = centre_row(nvalid);
-    for (int idx = tid; idx < C * (D / 8); idx += NTS) {
-      const int i = idx >> 4, j = idx & 15;
-      const uint4 rq = *reinterpret_cast<const uint4*>(s.q + i * LDD + j * 8);
-      const uint4 rk = *reinterpret_cast<const uint4*>(s.k + i * LDD + j * 8);
-      const uint32_t* wq = reinterpret_cast<const uint32_t*>(&rq);
-      const uint32_t* wk = reinterpret_cast<const uint32_t*>(&rk);
-      const float bi = s.beta[i];
-      uint32_t oqc[4], okb[4], obk[4], oqh[4], okt[4];
-      float g8[8], r8[8], c8[8];
-      gate8(s.G, gk, i, j * 8, g8);
-      gate8(s.G, gk, r, j * 8, r8);
-      gate8(s.G, gk, C - 1, j * 8, c8);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 fq = frag::unpack(wq[e]), fk = frag::unpack(wk[e]);
-        const float gi0 = g8[2 * e], gi1 = g8[2 * e + 1];
-        const float ep0 = __expf(gi0 - r8[2 * e]), ep1 = __expf(gi1 - r8[2 * e + 1]);
-        const float em0 = __expf(r8[2 * e] - gi0), em1 = __expf(r8[2 * e + 1] - gi1);
-        const float ea0 = __expf(gi0), ea1 = __expf(gi1);
-        const float et0 = __expf(c8[2 * e] - gi0), et1 = __expf(c8[2 * e + 1] - gi1);
-        oqc[e] = frag::pack(fq.x * ep0, fq.y * ep1);
-        okb[e] = frag::pack(fk.x * em0, fk.y * em1);
-        obk[e] = frag::pack(bi * fk.x * ea0, bi * fk.y * ea1);
-        oqh[e] = frag::pack(fq.x * ea0, fq.y * ea1);
-        okt[e] = frag::pack(fk.x * et0, fk.y * et1);
-      }
-      *reinterpret_cast<uint4*>(s.Qc + i * LDD + j * 8) = make_uint4(oqc[0], oqc[1], oqc[2], oqc[3]);
-      *reinterpret_cast<uint4*>(s.Kb + i * LDD + j * 8) = make_uint4(okb[0], okb[1], okb[2], okb[3]);
-      *reinterpret_cast<uint4*>(s.BK + i * LDD + j * 8) = make_uint4(obk[0], obk[1], obk[2], obk[3]);
-      *reinterpret_cast<uint4*>(s.Qh + i * LDD + j * 8) = make_uint4(oqh[0], oqh[1], oqh[2], oqh[3]);
-      *reinterpret_cast<uint4*>(s.Kt + i * LDD + j * 8) = make_uint4(okt[0], okt[1], okt[2], okt[3]);
-    }
-    for (int idx = tid; idx < C * (BV / 8); idx += NTS) {
-      const int i = idx >> 3, j = idx & 7;
-      *reinterpret_cast<uint4*>(s.dOs + i * LDC + j * 8) =
-          *reinterpret_cast<const uint4*>(s.dO + i * LDC + j * 8);
-    }
-    if (tid < D) s.dec[tid] = __expf((gk == D) ? s.G[(C - 1) * D + tid] : s.G[C - 1]);
-    __syncthreads();
-
-    float Wc[8][4], Mc[4][4];
-    frag::zero(Wc);
-    frag::mm_rows<8, 4, true>(Wc, s.T, LDC, rb * 16, s.BK, LDD, hf * 64);
-    frag::zero(Mc);
-    frag::mm_rows<4, 8, false>(Mc, s.Qc, LDD, rb * 16, s.Kb, LDD, hf * 32);
-#pragma unroll
-    for (int jt = 0; jt < 4; ++jt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = rb * 16 + lr + (e >> 1) * 8, jj = hf * 32 + jt * 8 + lc + (e & 1);
-        if (jj > i) Mc[jt][e] = 0.f;
-      }
-    __syncthreads();
-    frag::st_c(Wc, sW, LDD, rb * 16, hf * 64);
-    frag::st_c(Mc, sM, LDC, rb * 16, hf * 32);
-    if (n > 0) bscan_load_chunk(p, s, q, k, dO, g, Tg, beta, b, h, n - 1, a0);
     // dh_n: gradient of this chunk's end state
     for (int idx = tid; idx < BV * (D / 8); idx += NTS) {
       const int a = idx >> 4, j = idx & 15;
       *reinterpret_cast<uint4*>(dhout + cb * D * D + (size_t)(a0 + a) * D + j * 8) =
           *reinterpret_cast<const uint4*>(s.dS + a * LDD + j * 8);
     }
-    __syncthreads();
-
     // dU = M^T dO + Kt dS^T, rows i = 16rb.., values 32hf..
     {
       float du[4][4];
       frag::zero(du);
-      frag::mm_rows_at<4, 4, true>(du, sM, LDC, rb * 16, s.dOs, LDC, hf * 32);
-      frag::mm_rows<4, 8, false>(du, s.Kt, LDD, rb * 16, s.dS, LDD, hf * 32);
+      frag::mm_rows_at<4, 4, true>(du, st.M, LDC, rb * 16, st.dO, LDC, hf * 32);
+      frag::mm_rows<4, 8, false>(du, st.Kt, LDD, rb * 16, s.dS, LDD, hf * 32);
       frag::st_c(du, s.dU, LDC, rb * 16, hf * 32);
     }
     __syncthreads();
@@ -223,20 +146,22 @@ __global__ void __launch_bounds__(NTS, 1)
       *reinterpret_cast<uint4*>(dUout + (cb * C + i) * D + a0 + j * 8) =
           *reinterpret_cast<const uint4*>(s.dU + i * LDC + j * 8);
     }
-    // dS <- dS Diag(e^{gamma_C}) + dO^T Qh - dU^T W, rows a = 16rb.., keys 64hf..
+    // dS <- dS Diag(dec) + dO^T Qh - dU^T W, rows a = 16rb.., keys 64hf..
     {
       float pa[8][4], pb[8][4];
       frag::zero(pa);
-      frag::mm_rows_at<8, 4, true>(pa, s.dOs, LDC, rb * 16, s.Qh, LDD, hf * 64);
+      frag::mm_rows_at<8, 4, true>(pa, st.dO, LDC, rb * 16, st.Qh, LDD, hf * 64);
       frag::zero(pb);
-      frag::mm_rows_at<8, 4, true>(pb, s.dU, LDC, rb * 16, sW, LDD, hf * 64);
+      frag::mm_rows_at<8, 4, true>(pb, s.dU, LDC, rb * 16, st.W, LDD, hf * 64);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          dS[j][e] = dS[j][e] * s.dec[hf * 64 + j * 8 + lc + (e & 1)] + pa[j][e] - pb[j][e];
+          dS[j][e] = dS[j][e] * st.dec[hf * 64 + j * 8 + lc + (e & 1)] + pa[j][e] - pb[j][e];
     }
     __syncthreads();
+    if (n >= 2) bscan_issue(p, st, sv, dO, b, h, n - 2, a0);
+    frag::cp_commit();
     frag::st_c(dS, s.dS, LDD, rb * 16, hf * 64);
   }
   if (dS0) {
@@ -249,7 +174,6 @@ __global__ void __launch_bounds__(NTS, 1)
       }
   }
 }
-
 
 // ---------------------------------------------------------------------------
 // tc_bwd_chunk: 16 warps = 4 row blocks (16 chunk rows) x 4 column quarters.
@@ -266,7 +190,7 @@ struct BchunkSmem {
   bf16 dW[C * LDD];
   bf16 dM[C * LDC];     // tril(dO U^T)               [i][j]
   bf16 T[C * LDC];
-  bf16 R[2 * C * LDD];  // beta k e^gamma | beta v  ->  S half | dS' half  ->  Lambda_U | Lambda_W
+  bf16 R[2 * C * LDD];  // S half | dS' half  ->  Lambda_U | Lambda_W
                         // -> Kb^c | beta K^c  ->  dgamma (fp32 [C][D])
   float beta[C];
   float knorm[C];
@@ -282,7 +206,8 @@ __global__ void __launch_bounds__(NTB, 1)
                 const float* __restrict__ g, const bf16* __restrict__ Tg,
                 const float* __restrict__ beta, const bf16* __restrict__ hst,
                 const bf16* __restrict__ dhst, const bf16* __restrict__ Ug,
-                const bf16* __restrict__ dUg, bf16* __restrict__ dq, bf16* __restrict__ dk,
+                const bf16* __restrict__ dUg, const bf16* __restrict__ Wg,
+                const bf16* __restrict__ Upg, bf16* __restrict__ dq, bf16* __restrict__ dk,
                 bf16* __restrict__ dv, float* __restrict__ dbeta, float* __restrict__ dg) {
   extern __shared__ __align__(16) unsigned char smraw[];
   BchunkSmem& s = *reinterpret_cast<BchunkSmem*>(smraw);
@@ -296,15 +221,16 @@ __global__ void __launch_bounds__(NTB, 1)
   bf16* R1 = s.R + C * LDD;  // second half
   bf16* sdA = s.U;
 
-  // ---- loads: q (into Qc), k, v (into R1), dO, dU, U, T, gate, beta
+  // ---- loads: q (into Qc), k, dO, W, U', dU, U, T, gate, beta
   for (int idx = tid; idx < C * (D / 8); idx += NTB) {
     const int i = idx >> 4, j = idx & 15;
     const bool ok = i < nvalid;
     const size_t rr = row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 8;
     frag::cp16(s.Qc + i * LDD + j * 8, q + rr, ok);
     frag::cp16(s.k + i * LDD + j * 8, k + rr, ok);
-    frag::cp16(R1 + i * LDD + j * 8, v + rr, ok);
     frag::cp16(s.dO + i * LDD + j * 8, dO + rr, ok);
+    frag::cp16(s.W + i * LDD + j * 8, Wg + (cb * C + i) * D + j * 8, true);
+    frag::cp16(s.Up + i * LDD + j * 8, Upg + (cb * C + i) * D + j * 8, true);
     frag::cp16(s.dU + i * LDD + j * 8, dUg + (cb * C + i) * D + j * 8, true);
     frag::cp16(s.U + i * LDD + j * 8, Ug + (cb * C + i) * D + j * 8, true);
   }
@@ -332,49 +258,29 @@ __global__ void __launch_bounds__(NTB, 1)
   // per-element gate: gamma(i, c)
   auto gam = [&](int i, int c) -> float { return gk == D ? s.G[i * D + c] : s.G[i]; };
 
-  // ---- build: Q^c in place, beta k e^gamma into R0, beta v in place in R1, key norms
+  // ---- build: Q^c in place, key norms
   for (int idx = tid; idx < C * (D / 8); idx += NTB) {
     const int i = idx >> 4, j = idx & 15;
     uint4 rq = *reinterpret_cast<const uint4*>(s.Qc + i * LDD + j * 8);
-    uint4 rk = *reinterpret_cast<const uint4*>(s.k + i * LDD + j * 8);
-    uint4 rv = *reinterpret_cast<const uint4*>(R1 + i * LDD + j * 8);
+    const uint4 rk = *reinterpret_cast<const uint4*>(s.k + i * LDD + j * 8);
     uint32_t* wq = reinterpret_cast<uint32_t*>(&rq);
     const uint32_t* wk = reinterpret_cast<const uint32_t*>(&rk);
-    uint32_t* wv = reinterpret_cast<uint32_t*>(&rv);
-    const float bi = s.beta[i];
     float g8[8], r8[8];
     gate8(s.G, gk, i, j * 8, g8);
     gate8(s.G, gk, r, j * 8, r8);
-    uint32_t obk[4];
     float nn = 0.f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float2 fq = frag::unpack(wq[e]), fk = frag::unpack(wk[e]), fv = frag::unpack(wv[e]);
+      const float2 fq = frag::unpack(wq[e]), fk = frag::unpack(wk[e]);
       wq[e] = frag::pack(fq.x * __expf(g8[2 * e] - r8[2 * e]), fq.y * __expf(g8[2 * e + 1] - r8[2 * e + 1]));
-      obk[e] = frag::pack(bi * fk.x * __expf(g8[2 * e]), bi * fk.y * __expf(g8[2 * e + 1]));
-      wv[e] = frag::pack(bi * fv.x, bi * fv.y);
       nn += fk.x * fk.x + fk.y * fk.y;
     }
     *reinterpret_cast<uint4*>(s.Qc + i * LDD + j * 8) = rq;
-    *reinterpret_cast<uint4*>(R0 + i * LDD + j * 8) = make_uint4(obk[0], obk[1], obk[2], obk[3]);
-    *reinterpret_cast<uint4*>(R1 + i * LDD + j * 8) = rv;
     nn += __shfl_xor_sync(0xffffffffu, nn, 8);
     nn += __shfl_xor_sync(0xffffffffu, nn, 4);
     nn += __shfl_xor_sync(0xffffffffu, nn, 2);
     nn += __shfl_xor_sync(0xffffffffu, nn, 1);
     if (j == 0) s.knorm[i] = nn;
-  }
-  __syncthreads();
-
-  // ---- phase 1a: W = T (beta K e^gamma), U' = T (beta V); rows 16rb.., cols 32qt..
-  {
-    float w4[4][4], u4[4][4];
-    frag::zero(w4);
-    frag::mm_rows<4, 4, true>(w4, s.T, LDC, rb * 16, R0, LDD, qt * 32);
-    frag::zero(u4);
-    frag::mm_rows<4, 4, true>(u4, s.T, LDC, rb * 16, R1, LDD, qt * 32);
-    frag::st_c(w4, s.W, LDD, rb * 16, qt * 32);
-    frag::st_c(u4, s.Up, LDD, rb * 16, qt * 32);
   }
   __syncthreads();
 
@@ -671,23 +577,20 @@ __global__ void __launch_bounds__(NTB, 1)
 
 }  // namespace
 
-size_t bwd_scan_smem(const Problem& p) { return sizeof(BscanSmem) + sizeof(float) * (C * p.gk); }
-
-cudaError_t launch_bwd_scan(const Problem& p, const bf16* q, const bf16* k, const bf16* dO,
-                            const float* g, const bf16* T, const float* beta_eff,
-                            const float* dST, float* dS0, bf16* dU, bf16* dh, cudaStream_t st) {
-  const size_t sm = bwd_scan_smem(p);
+cudaError_t launch_bwd_scan(const Problem& p, const Saved& sv, const bf16* dO, const float* dST,
+                            float* dS0, bf16* dU, bf16* dh, cudaStream_t st) {
+  const size_t sm = sizeof(BscanSmem);
   cudaError_t e =
       cudaFuncSetAttribute(k_bwd_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const double nb = (double)p.B * p.H * p.NC, ntok = nb * C, heads = (double)p.B * p.H;
-  double bytes = ntok * (2 * D * 2 + D * 2 + p.gk * 4 + 4) + nb * C * C * 2 + ntok * D * 2 +
-                 nb * D * D * 2 + heads * D * D * 4 * ((dST ? 1 : 0) + (dS0 ? 1 : 0));
-  const double per_tile = 2.0 * C * C * D * 2 + 2.0 * C * C * BV + 2.0 * C * BV * D * 3;
-  const double flops = nb * (D / BV) * per_tile;
+  // reads W, Qh, Kt, M, dec, dO; writes dU, dh
+  const double bytes = nb * (3.0 * kTileBytes + kMBytes + kDecBytes) + ntok * D * 2 +
+                       nb * ((double)kUBytes + kStateBytes) +
+                       heads * D * D * 4 * ((dST ? 1 : 0) + (dS0 ? 1 : 0));
+  const double flops = nb * (D / BV) * (2.0 * C * C * BV + 2.0 * C * BV * D * 3);
   prof_begin(kKTcScanBwd, bytes, flops, st);
-  k_bwd_scan<<<dim3(D / BV, p.H, p.B), NTS, sm, st>>>(p, q, k, dO, g, T, beta_eff, dST, dS0,
-                                                      dU, dh);
+  k_bwd_scan<<<dim3(D / BV, p.H, p.B), NTS, sm, st>>>(p, sv, dO, dST, dS0, dU, dh);
   e = cudaGetLastError();
   prof_end(st);
   return e;
@@ -698,26 +601,25 @@ size_t bwd_chunk_smem(const Problem& p) {
 }
 
 cudaError_t launch_bwd_chunk(const Problem& p, const bf16* q, const bf16* k, const bf16* v,
-                             const bf16* dO, const float* g, const bf16* T,
-                             const float* beta_eff, const bf16* h, const bf16* dh,
-                             const bf16* U, const bf16* dU, bf16* dq, bf16* dk, bf16* dv,
-                             float* dbeta, float* dg, cudaStream_t st) {
+                             const bf16* dO, const float* g, const Saved& sv, const bf16* dh,
+                             const bf16* dU, bf16* dq, bf16* dk, bf16* dv, float* dbeta,
+                             float* dg, cudaStream_t st) {
   const size_t sm = bwd_chunk_smem(p);
   cudaError_t e =
       cudaFuncSetAttribute(k_bwd_chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const double nb = (double)p.B * p.H * p.NC, ntok = nb * C;
+  // reads q, k, v, dO, g, beta, T, h, dh, U, dU, W, U'; writes dq, dk, dv, dbeta, dg
   const double bytes = ntok * (4 * D * 2 + p.gk * 4 + 4) + nb * C * C * 2 + nb * 2.0 * D * D * 2 +
-                       ntok * 2 * D * 2 + ntok * (3 * D * 2 + p.gk * 4 + 4);
-  const double mac = (double)C * D * C * 2      // W, U'
-                     + (double)C * D * D * 3    // dO S, dU S, U dS'
+                       ntok * 4 * D * 2 + ntok * (3 * D * 2 + p.gk * 4 + 4);
+  const double mac = (double)C * D * D * 3      // dO S, dU S, U dS'
                      + (double)C * C * D        // dO U^T
                      + (double)C * D * C * 2    // Lambda
                      + (double)C * C * D * 2    // dA
                      + (double)C * D * C * 4;   // dM Kb, dA Kb, dM^T Q^c, dA^T K^c
   prof_begin(kKTcChunkBwd, bytes, nb * 2.0 * mac, st);
-  k_bwd_chunk<<<dim3(p.NC, p.H, p.B), NTB, sm, st>>>(p, q, k, v, dO, g, T, beta_eff, h, dh, U,
-                                                     dU, dq, dk, dv, dbeta, dg);
+  k_bwd_chunk<<<dim3(p.NC, p.H, p.B), NTB, sm, st>>>(p, q, k, v, dO, g, sv.T, sv.beta, sv.h, dh,
+                                                     sv.U, dU, sv.W, sv.Up, dq, dk, dv, dbeta, dg);
   e = cudaGetLastError();
   prof_end(st);
   return e;

@@ -1,20 +1,19 @@
 // fast_fwd.cu -- tensor-core forward for bf16 storage, d_k = d_v = 128, C = 64.
 //
-// tc_prep (chunk-parallel, one CTA per (b, h, chunk)):
-//   gamma = inclusive cumulative log-gate, beta (Kaczmarz step applied),
-//   A = diag(beta) strict_tril(K^c Kb^c^T) on tensor cores (centred factors
-//   K^c = k e^{gamma - gamma_r}, Kb^c = k e^{gamma_r - gamma}),
-//   T = (I + A)^{-1} by blocked forward substitution in fp32 (16 x 16 diagonal
-//   blocks per warp, then three levels of off-diagonal block products).
-//   Writes T (bf16, row-major 64 x 64) and beta per chunk.
+// tc_prep (chunk-parallel, one CTA per (b, h, chunk); every state-independent
+// quantity of the chunk, computed once):
+//   gamma = inclusive cumulative log-gate; beta (Kaczmarz step applied);
+//   centred factors K^c = k e^{gamma - gamma_r}, Kb^c = k e^{gamma_r - gamma},
+//   Q^c = q e^{gamma - gamma_r} (gamma_r: gate of the chunk's centre row);
+//   [A ; M] = [K^c ; Q^c] Kb^c^T on tensor cores, A = diag(beta) strict_tril(.),
+//   M = tril(.);  T = (I + A)^{-1} by blocked forward substitution in fp32
+//   (16 x 16 diagonal blocks per warp, off-diagonal block products in tf32);
+//   W = T diag(beta) (k e^gamma),  U' = T diag(beta) V  on tensor cores;
+//   Qh = q e^gamma,  Kt = k e^{gamma_C - gamma},  dec = e^{gamma_C}.
 // tc_fwd_scan (sequential over chunks, one CTA per (b, h, 64-wide value tile)):
-//   per chunk, recomputes from q, k, v, g, T:
-//     M = tril(Q^c Kb^c^T), W = T diag(beta) (k e^gamma), U' = T diag(beta) V,
-//   then with the fp32 state S (registers) and its bf16 copy (shared memory):
-//     U = U' - W S^T,  O = (q e^gamma) S^T + M U,  S <- S Diag(e^{gamma_C}) + U^T Kt
-//   (Kt = k e^{gamma_C - gamma}).  Optionally saves each chunk's start state
-//   (bf16) and U (bf16) for the backward.  The raw inputs of chunk n+1 are
-//   fetched with cp.async while chunk n's state products run.
+// with the fp32 state S in registers and its bf16 copy in shared memory,
+//   U = U' - W S^T,  O = Qh S^T + M U,  S <- S Diag(dec) + U^T Kt,
+// streaming the precomputed chunk tiles through a two-stage cp.async pipeline.
 
 #include "dr_common.cuh"
 #include "fast.cuh"
@@ -31,12 +30,12 @@ constexpr int C = 64, D = 128;
 constexpr int LDD = D + 8;   // bf16 stride of 128-wide tiles
 constexpr int LDC = C + 8;   // bf16 stride of 64-wide tiles
 constexpr int LDA = C + 1;   // fp32 stride of the 64 x 64 solve tiles
-constexpr int NTH = 128;     // threads per CTA (4 warps x 16 rows)
+constexpr int NT = 256;      // threads per CTA (8 warps)
+constexpr int BV = 64;       // value columns per scan CTA
 
 __device__ __forceinline__ int centre_row(int nvalid) { return (nvalid - 1) / 2; }
 
-// In-place inclusive cumulative sum down the 64 rows of column `col` of a
-// [C][ld] fp32 tile: all loads first, then the scan in registers.
+// In-place inclusive cumulative sum down the 64 rows of column `col`.
 __device__ __forceinline__ void cumsum_col(float* G, int ld, int col) {
   float v[C];
 #pragma unroll
@@ -47,8 +46,7 @@ __device__ __forceinline__ void cumsum_col(float* G, int ld, int col) {
   for (int i = 0; i < C; ++i) G[i * ld + col] = v[i];
 }
 
-// Eight consecutive gate values of row i starting at channel c (scalar gate:
-// broadcast of the row's value).
+// Eight consecutive gate values of row i from channel c (scalar gate: broadcast).
 __device__ __forceinline__ void gate8(const float* G, int gk, int i, int c, float* out) {
   if (gk == 1) {
     const float x = G[i];
@@ -62,77 +60,110 @@ __device__ __forceinline__ void gate8(const float* G, int gk, int i, int c, floa
   }
 }
 
+__device__ __forceinline__ void unpack8(const uint4& r, float* f) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(&r);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 x = frag::unpack(w[e]);
+    f[2 * e] = x.x;
+    f[2 * e + 1] = x.y;
+  }
+}
+__device__ __forceinline__ uint4 pack8(const float* f) {
+  return make_uint4(frag::pack(f[0], f[1]), frag::pack(f[2], f[3]), frag::pack(f[4], f[5]),
+                    frag::pack(f[6], f[7]));
+}
+
+// Row-major bf16 global store of accumulators (rows r0.., cols n0..), 4-byte pairs.
+template <int NTL>
+__device__ __forceinline__ void st_c_global(const float (&c)[NTL][4], bf16* g, int ld, int r0,
+                                            int n0) {
+  const int l = threadIdx.x & 31;
+  const int r = r0 + (l >> 2), cc = n0 + 2 * (l & 3);
+#pragma unroll
+  for (int j = 0; j < NTL; ++j) {
+    *reinterpret_cast<uint32_t*>(g + (size_t)r * ld + cc + j * 8) = frag::pack(c[j][0], c[j][1]);
+    *reinterpret_cast<uint32_t*>(g + (size_t)(r + 8) * ld + cc + j * 8) =
+        frag::pack(c[j][2], c[j][3]);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // tc_prep
 struct PrepSmem {
-  bf16 Kc[C * LDD];
-  bf16 Kb[C * LDD];
-  float A[C * LDA];
-  float T[C * LDA];
+  bf16 R1[C * LDD];            // K^c, then beta k e^gamma
+  bf16 R2[C * LDD];            // Kb^c, then A (fp32 [C][LDA]), then T (bf16 [C][LDC])
+  bf16 R3[C * LDD];            // Q^c, then T (fp32 [C][LDA])
+  float RG[C * D + 512];       // cumulative gate [C][gk], then beta v (bf16 [C][LDD])
   float X[16 * 48];
   float beta[C];
-  float G[1];  // [C][gk], dynamic tail
 };
 
-__global__ void __launch_bounds__(NTH) k_prep(Problem p, const bf16* __restrict__ k,
-                                              const float* __restrict__ beta_in,
-                                              const float* __restrict__ g,
-                                              bf16* __restrict__ Tout,
-                                              float* __restrict__ beta_out) {
+__global__ void __launch_bounds__(NT, 2)
+    k_prep(Problem p, const bf16* __restrict__ q, const bf16* __restrict__ k,
+           const bf16* __restrict__ v, const float* __restrict__ beta_in,
+           const float* __restrict__ g, Saved sv) {
   extern __shared__ __align__(16) unsigned char smraw[];
   PrepSmem& s = *reinterpret_cast<PrepSmem*>(smraw);
   const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-  const int gk = p.gk, t0 = n * C, nvalid = min(C, p.T - t0);
+  const int warp = tid >> 5, lane = tid & 31, gk = p.gk;
+  const int lr = lane >> 2, lc = 2 * (lane & 3);
+  const int t0 = n * C, nvalid = min(C, p.T - t0);
   const size_t cb = chunk_id(p, b, h, n);
-  float* G = s.G;
+  float* G = s.RG;
+  float* sA = reinterpret_cast<float*>(s.R2);
+  float* sT = reinterpret_cast<float*>(s.R3);
+  bf16* sTb = s.R2;
+  bf16* sBV = reinterpret_cast<bf16*>(s.RG);
 
-  // gate -> shared, then inclusive cumulative sum per channel
   if (gk == D) {
-    for (int idx = tid; idx < C * D / 4; idx += NTH) {
-      const int i = idx / (D / 4), c4 = idx % (D / 4);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (i < nvalid && p.gate != kGateNone)
-        v = *reinterpret_cast<const float4*>(g + row_id(p, b, t0 + i, h) * D + c4 * 4);
-      *reinterpret_cast<float4*>(G + i * D + c4 * 4) = v;
+    for (int idx = tid; idx < C * (D / 4); idx += NT) {
+      const int i = idx >> 5, j = idx & 31;
+      const bool ok = i < nvalid && p.gate != kGateNone;
+      frag::cp16(G + i * D + j * 4, g + row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 4, ok);
     }
+    frag::cp_commit();
+    frag::cp_wait<0>();
   } else if (tid < C) {
     G[tid] = (tid < nvalid && p.gate != kGateNone) ? g[row_id(p, b, t0 + tid, h)] : 0.f;
   }
-  for (int idx = tid; idx < C * LDA; idx += NTH) s.T[idx] = 0.f;
   __syncthreads();
   if (tid < gk) cumsum_col(G, gk, tid);
   __syncthreads();
 
-  // centred key factors (bf16) and beta
+  // Factors: K^c, Kb^c, Q^c to shared memory; Qh, Kt, beta, dec to global.
   const int r = centre_row(nvalid);
-#pragma unroll 1
-  for (int pass = 0; pass < C * (D / 8) / NTH; ++pass) {
-    const int idx = tid + pass * NTH;
+  for (int idx = tid; idx < C * (D / 8); idx += NT) {
     const int i = idx >> 4, j = idx & 15;
     const bool valid = i < nvalid;
-    uint4 raw = make_uint4(0, 0, 0, 0);
-    if (valid) raw = *reinterpret_cast<const uint4*>(k + row_id(p, b, t0 + i, h) * D + j * 8);
-    const uint32_t* rw = reinterpret_cast<const uint32_t*>(&raw);
-    float kv[8];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float2 f = frag::unpack(rw[e]);
-      kv[2 * e] = f.x;
-      kv[2 * e + 1] = f.y;
+    uint4 rk = make_uint4(0, 0, 0, 0), rq = rk;
+    if (valid) {
+      const size_t rr = row_id(p, b, t0 + i, h) * D + j * 8;
+      rk = *reinterpret_cast<const uint4*>(k + rr);
+      rq = *reinterpret_cast<const uint4*>(q + rr);
     }
-    float nn = 0.f;
-    uint32_t oc[4], ob[4];
-    float gi[8], gr[8];
-    gate8(G, gk, i, j * 8, gi);
-    gate8(G, gk, r, j * 8, gr);
+    float kv[8], qv[8], g8[8], r8[8], c8[8];
+    unpack8(rk, kv);
+    unpack8(rq, qv);
+    gate8(G, gk, i, j * 8, g8);
+    gate8(G, gk, r, j * 8, r8);
+    gate8(G, gk, C - 1, j * 8, c8);
+    float kc[8], kb[8], qc[8], qh[8], kt[8], nn = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      oc[e / 2] = frag::pack(kv[e] * __expf(gi[e] - gr[e]), kv[e + 1] * __expf(gi[e + 1] - gr[e + 1]));
-      ob[e / 2] = frag::pack(kv[e] * __expf(gr[e] - gi[e]), kv[e + 1] * __expf(gr[e + 1] - gi[e + 1]));
-      nn += kv[e] * kv[e] + kv[e + 1] * kv[e + 1];
+    for (int e = 0; e < 8; ++e) {
+      const float ep = __expf(g8[e] - r8[e]), em = __expf(r8[e] - g8[e]);
+      kc[e] = kv[e] * ep;
+      kb[e] = kv[e] * em;
+      qc[e] = qv[e] * ep;
+      qh[e] = qv[e] * __expf(g8[e]);
+      kt[e] = kv[e] * __expf(c8[e] - g8[e]);
+      nn += kv[e] * kv[e];
     }
-    *reinterpret_cast<uint4*>(s.Kc + i * LDD + j * 8) = make_uint4(oc[0], oc[1], oc[2], oc[3]);
-    *reinterpret_cast<uint4*>(s.Kb + i * LDD + j * 8) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+    *reinterpret_cast<uint4*>(s.R1 + i * LDD + j * 8) = pack8(kc);
+    *reinterpret_cast<uint4*>(s.R2 + i * LDD + j * 8) = pack8(kb);
+    *reinterpret_cast<uint4*>(s.R3 + i * LDD + j * 8) = pack8(qc);
+    *reinterpret_cast<uint4*>(sv.Qh + (cb * C + i) * D + j * 8) = pack8(qh);
+    *reinterpret_cast<uint4*>(sv.Kt + (cb * C + i) * D + j * 8) = pack8(kt);
     nn += __shfl_xor_sync(0xffffffffu, nn, 8);
     nn += __shfl_xor_sync(0xffffffffu, nn, 4);
     nn += __shfl_xor_sync(0xffffffffu, nn, 2);
@@ -144,161 +175,175 @@ __global__ void __launch_bounds__(NTH) k_prep(Problem p, const bf16* __restrict_
         bb = (p.beta_mode == kBetaKaczmarz) ? in / (nn + p.eps) : in;
       }
       s.beta[i] = bb;
-      beta_out[cb * C + i] = bb;
+      sv.beta[cb * C + i] = bb;
     }
   }
+  if (tid < D) sv.dec[cb * D + tid] = __expf(gk == D ? G[(C - 1) * D + tid] : G[C - 1]);
   __syncthreads();
 
-  // Gram on tensor cores: warp w owns rows 16w..16w+15, all 64 columns.
-  const int warp = tid >> 5, lane = tid & 31;
-  {
-    float acc[8][4];
-    frag::zero(acc);
-    frag::mm_rows<8, 8, false>(acc, s.Kc, LDD, warp * 16, s.Kb, LDD);
-    const int r0 = warp * 16 + (lane >> 2), c0 = 2 * (lane & 3);
+  // [A ; M] = [K^c ; Q^c] Kb^c^T: warps 0-3 -> A rows 16w.., warps 4-7 -> M rows 16(w-4)..
+  const int rb = warp & 3;
+  float gram[8][4];
+  frag::zero(gram);
+  frag::mm_rows<8, 8, false>(gram, warp < 4 ? s.R1 : s.R3, LDD, rb * 16, s.R2, LDD);
+  if (warp >= 4) {
 #pragma unroll
-    for (int jt = 0; jt < 8; ++jt) {
+    for (int jt = 0; jt < 8; ++jt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int i = r0 + (e >> 1) * 8, jj = jt * 8 + c0 + (e & 1);
-        s.A[i * LDA + jj] = (jj < i) ? s.beta[i] * acc[jt][e] : 0.f;
+        const int i = rb * 16 + lr + (e >> 1) * 8, jj = jt * 8 + lc + (e & 1);
+        if (jj > i) gram[jt][e] = 0.f;
       }
-    }
+    st_c_global(gram, sv.M + cb * C * C, C, rb * 16, 0);
   }
-  __syncthreads();
+  __syncthreads();  // K^c, Kb^c, Q^c consumed
+  if (warp < 4) {
+#pragma unroll
+    for (int jt = 0; jt < 8; ++jt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = rb * 16 + lr + (e >> 1) * 8, jj = jt * 8 + lc + (e & 1);
+        sA[i * LDA + jj] = (jj < i) ? s.beta[i] * gram[jt][e] : 0.f;
+      }
+  }
+  for (int idx = tid; idx < C * LDA; idx += NT) sT[idx] = 0.f;
+  // beta k e^gamma into R1 (k reloaded; L2-resident)
+  for (int idx = tid; idx < C * (D / 8); idx += NT) {
+    const int i = idx >> 4, j = idx & 15;
+    uint4 rk = make_uint4(0, 0, 0, 0);
+    if (i < nvalid) rk = *reinterpret_cast<const uint4*>(k + row_id(p, b, t0 + i, h) * D + j * 8);
+    float kv[8], g8[8];
+    unpack8(rk, kv);
+    gate8(G, gk, i, j * 8, g8);
+    const float bi = s.beta[i];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) kv[e] *= bi * __expf(g8[e]);
+    *reinterpret_cast<uint4*>(s.R1 + i * LDD + j * 8) = pack8(kv);
+  }
+  __syncthreads();  // A ready; the gate is no longer needed
 
-  // Diagonal 16 x 16 blocks: warp w inverts block w; lane l < 16 owns column l.
-  if (lane < 16) {
-    const int base = warp * 16, l = lane;
-    float t[16];
+  // T = (I + A)^{-1}: diagonal 16 x 16 blocks (warps 0-3, lane l < 16 owns column l)
+  if (warp < 4) {
+    if (lane < 16) {
+      const int base = warp * 16, l = lane;
+      float t[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) t[i] = (i == l) ? 1.f : 0.f;
+      for (int i = 0; i < 16; ++i) t[i] = (i == l) ? 1.f : 0.f;
 #pragma unroll
-    for (int i = 1; i < 16; ++i) {
-      if (i > l) {
-        float acc = 0.f;
+      for (int i = 1; i < 16; ++i) {
+        if (i > l) {
+          float acc = 0.f;
 #pragma unroll
-        for (int m = 0; m < 15; ++m)
-          if (m >= l && m < i) acc += s.A[(base + i) * LDA + base + m] * t[m];
-        t[i] = -acc;
+          for (int m = 0; m < 15; ++m)
+            if (m >= l && m < i) acc += sA[(base + i) * LDA + base + m] * t[m];
+          t[i] = -acc;
+        }
       }
-    }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) s.T[(base + i) * LDA + base + l] = t[i];
+      for (int i = 0; i < 16; ++i) sT[(base + i) * LDA + base + l] = t[i];
+    }
+  } else {
+    // meanwhile: beta v into the freed gate region
+    for (int idx = tid - 128; idx < C * (D / 8); idx += NT - 128) {
+      const int i = idx >> 4, j = idx & 15;
+      uint4 rv = make_uint4(0, 0, 0, 0);
+      if (i < nvalid) rv = *reinterpret_cast<const uint4*>(v + row_id(p, b, t0 + i, h) * D + j * 8);
+      float vv[8];
+      unpack8(rv, vv);
+      const float bi = s.beta[i];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) vv[e] *= bi;
+      *reinterpret_cast<uint4*>(sBV + i * LDD + j * 8) = pack8(vv);
+    }
   }
   __syncthreads();
-  // Off-diagonal blocks, block row bi = 1..3, on tensor cores (tf32):
-  //   X_j = sum_{m = 16j}^{16bi - 1} A[16bi.., m] T[m, 16j..]   (warp j < bi)
+  // Off-diagonal blocks, block row bi = 1..3, tf32 tensor cores:
+  //   X_j = sum_{m = 16j}^{16bi - 1} A[16bi.., m] T[m, 16j..]  (warp j < bi),
   //   T[bi, j] = -T[bi, bi] X_j
   for (int bi = 1; bi < 4; ++bi) {
     if (warp < bi) {
       const int j = warp, w = 16 * bi;
       float x[2][4] = {};
-      frag::mm16x16_tf32(x, s.A, LDA, w, s.T, LDA, 16 * j, 16 * j, w - 16 * j);
-      const int g = lane >> 2, t = lane & 3;
+      frag::mm16x16_tf32(x, sA, LDA, w, sT, LDA, 16 * j, 16 * j, w - 16 * j);
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
-        s.X[g * 48 + 16 * j + nt * 8 + 2 * t] = x[nt][0];
-        s.X[g * 48 + 16 * j + nt * 8 + 2 * t + 1] = x[nt][1];
-        s.X[(g + 8) * 48 + 16 * j + nt * 8 + 2 * t] = x[nt][2];
-        s.X[(g + 8) * 48 + 16 * j + nt * 8 + 2 * t + 1] = x[nt][3];
+        s.X[lr * 48 + 16 * j + nt * 8 + lc] = x[nt][0];
+        s.X[lr * 48 + 16 * j + nt * 8 + lc + 1] = x[nt][1];
+        s.X[(lr + 8) * 48 + 16 * j + nt * 8 + lc] = x[nt][2];
+        s.X[(lr + 8) * 48 + 16 * j + nt * 8 + lc + 1] = x[nt][3];
       }
       __syncwarp();
       float y[2][4] = {};
-      frag::mm16x16_tf32(y, s.T + w, LDA, w, s.X + 16 * j, 48, 0, 0, 16);
+      frag::mm16x16_tf32(y, sT + w, LDA, w, s.X + 16 * j, 48, 0, 0, 16);
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
-        s.T[(w + g) * LDA + 16 * j + nt * 8 + 2 * t] = -y[nt][0];
-        s.T[(w + g) * LDA + 16 * j + nt * 8 + 2 * t + 1] = -y[nt][1];
-        s.T[(w + g + 8) * LDA + 16 * j + nt * 8 + 2 * t] = -y[nt][2];
-        s.T[(w + g + 8) * LDA + 16 * j + nt * 8 + 2 * t + 1] = -y[nt][3];
+        sT[(w + lr) * LDA + 16 * j + nt * 8 + lc] = -y[nt][0];
+        sT[(w + lr) * LDA + 16 * j + nt * 8 + lc + 1] = -y[nt][1];
+        sT[(w + lr + 8) * LDA + 16 * j + nt * 8 + lc] = -y[nt][2];
+        sT[(w + lr + 8) * LDA + 16 * j + nt * 8 + lc + 1] = -y[nt][3];
       }
     }
     __syncthreads();
   }
-  // T -> global (bf16, row-major)
-  for (int idx = tid; idx < C * C / 8; idx += NTH) {
+  // T -> bf16: global and the tensor-core A operand (over the dead A tile)
+  for (int idx = tid; idx < C * C / 8; idx += NT) {
     const int i = idx >> 3, j = idx & 7;
-    const float* src = s.T + i * LDA + j * 8;
-    uint4 v = make_uint4(frag::pack(src[0], src[1]), frag::pack(src[2], src[3]),
-                         frag::pack(src[4], src[5]), frag::pack(src[6], src[7]));
-    *reinterpret_cast<uint4*>(Tout + cb * C * C + i * C + j * 8) = v;
+    const uint4 val = pack8(sT + i * LDA + j * 8);
+    *reinterpret_cast<uint4*>(sv.T + cb * C * C + i * C + j * 8) = val;
+    *reinterpret_cast<uint4*>(sTb + i * LDC + j * 8) = val;
+  }
+  __syncthreads();
+  // W = T (beta k e^gamma) (warps 0-3), U' = T (beta v) (warps 4-7): rows 16rb.., 128 columns
+  {
+    float acc[16][4];
+    frag::zero(acc);
+    frag::mm_rows<16, 4, true>(acc, sTb, LDC, rb * 16, warp < 4 ? s.R1 : sBV, LDD);
+    st_c_global(acc, (warp < 4 ? sv.W : sv.Up) + cb * C * D, D, rb * 16, 0);
   }
 }
 
 // ---------------------------------------------------------------------------
 // tc_fwd_scan
-constexpr int BV = 64;  // value columns per CTA
-
+struct FwdStage {
+  bf16 W[C * LDD];
+  bf16 Qh[C * LDD];
+  bf16 Kt[C * LDD];
+  bf16 M[C * LDC];
+  bf16 Up[C * LDC];   // U'[:, a0 .. a0+63]
+  float dec[D];
+};
 struct FwdSmem {
-  // raw inputs of the current chunk (refilled by cp.async for the next chunk)
-  bf16 q[C * LDD];
-  bf16 k[C * LDD];
-  bf16 v[C * LDC];
-  bf16 T[C * LDC];
-  float beta[C];
-  // operand tiles
-  bf16 Qc[C * LDD];   // q e^{gamma - gamma_r}
-  bf16 Kb[C * LDD];   // k e^{gamma_r - gamma}
-  bf16 BK[C * LDD];   // beta k e^{gamma}          ([j][c], B operand, k-rows)
-  bf16 Qh[C * LDD];   // q e^{gamma}
-  bf16 Kt[C * LDD];   // k e^{gamma_C - gamma}     ([i][c], B operand, k-rows)
-  bf16 BV_[C * LDC];  // beta v                    ([j][a])
-  bf16 U[C * LDC];    // pseudo-values U           ([i][a])
-  bf16 S[BV * LDD];   // bf16 copy of the state    ([a][c])
-  float dec[D];       // e^{gamma_C}
-  float G[1];         // [C][gk] raw gate, then cumulative (dynamic tail)
+  FwdStage st[2];
+  bf16 S[BV * LDD];   // bf16 copy of the state rows a0.. [a][c]
+  bf16 U[C * LDC];    // pseudo-values [i][a]
 };
 
-// Issue the cp.async loads of chunk n's raw inputs (one commit group).
-__device__ void fwd_load_chunk(const Problem& p, FwdSmem& s, const bf16* q, const bf16* k,
-                               const bf16* v, const float* g, const bf16* T,
-                               const float* beta, int b, int h, int n, int a0) {
-  const int tid = threadIdx.x, gk = p.gk, t0 = n * C, nvalid = min(C, p.T - t0);
-  const int NTH = blockDim.x;
+__device__ void fwd_issue(const Problem& p, FwdStage& s, const Saved& sv, int b, int h, int n,
+                          int a0) {
+  const int tid = threadIdx.x;
   const size_t cb = chunk_id(p, b, h, n);
-  for (int idx = tid; idx < C * (D / 8); idx += NTH) {
+  for (int idx = tid; idx < C * (D / 8); idx += NT) {
     const int i = idx >> 4, j = idx & 15;
-    const bool ok = i < nvalid;
-    const size_t rr = row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 8;
-    frag::cp16(s.q + i * LDD + j * 8, q + rr, ok);
-    frag::cp16(s.k + i * LDD + j * 8, k + rr, ok);
+    const size_t o = (cb * C + i) * D + j * 8;
+    frag::cp16(s.W + i * LDD + j * 8, sv.W + o, true);
+    frag::cp16(s.Qh + i * LDD + j * 8, sv.Qh + o, true);
+    frag::cp16(s.Kt + i * LDD + j * 8, sv.Kt + o, true);
   }
-  for (int idx = tid; idx < C * (BV / 8); idx += NTH) {
+  for (int idx = tid; idx < C * (C / 8); idx += NT) {
     const int i = idx >> 3, j = idx & 7;
-    const bool ok = i < nvalid;
-    frag::cp16(s.v + i * LDC + j * 8, v + row_id(p, b, t0 + (ok ? i : 0), h) * D + a0 + j * 8, ok);
-    frag::cp16(s.T + i * LDC + j * 8, T + cb * C * C + i * C + j * 8, true);
+    frag::cp16(s.M + i * LDC + j * 8, sv.M + cb * C * C + i * C + j * 8, true);
+    frag::cp16(s.Up + i * LDC + j * 8, sv.Up + (cb * C + i) * D + a0 + j * 8, true);
   }
-  if (gk == D) {
-    for (int idx = tid; idx < C * (D / 4); idx += NTH) {
-      const int i = idx >> 5, j = idx & 31;
-      const bool ok = i < nvalid && p.gate != kGateNone;
-      frag::cp16(s.G + i * D + j * 4, g + row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 4, ok);
-    }
-  }
-  if (tid < C / 4) frag::cp16(s.beta + tid * 4, beta + cb * C + tid * 4, true);
-  frag::cp_commit();
-  if (gk == 1 && tid < C) {
-    // scalar gate: plain loads (4 bytes per row)
-    s.G[tid] = (tid < nvalid && p.gate != kGateNone) ? g[row_id(p, b, t0 + tid, h)] : 0.f;
-  }
+  if (tid < D / 4) frag::cp16(s.dec + tid * 4, sv.dec + cb * D + tid * 4, true);
 }
 
-constexpr int NTS = 256;  // threads of the scan CTA: 8 warps = 4 row blocks x 2 halves
-
-__global__ void __launch_bounds__(NTS, 1)
-    k_fwd_scan(Problem p, const bf16* __restrict__ q, const bf16* __restrict__ k,
-               const bf16* __restrict__ v, const float* __restrict__ g,
-               const bf16* __restrict__ Tg, const float* __restrict__ beta,
-               const float* __restrict__ S0, bf16* __restrict__ o, float* __restrict__ ST,
-               bf16* __restrict__ hsave, bf16* __restrict__ Usave) {
+__global__ void __launch_bounds__(NT, 1)
+    k_fwd_scan(Problem p, Saved sv, const float* __restrict__ S0, bf16* __restrict__ o,
+               float* __restrict__ ST, int save) {
   extern __shared__ __align__(16) unsigned char smraw[];
   FwdSmem& s = *reinterpret_cast<FwdSmem*>(smraw);
-  bf16* sW = s.BK;  // W  [i][c], written once beta K e^gamma is consumed
-  bf16* sM = s.Qc;  // M  [i][j] (stride LDC), written once Q^c is consumed
   const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31, gk = p.gk;
+  const int warp = tid >> 5, lane = tid & 31;
   const int rb = warp & 3, hf = warp >> 2;  // row block (16 rows), column half
   const int a0 = blockIdx.x * BV;
   const int lr = lane >> 2, lc = 2 * (lane & 3);
@@ -315,114 +360,49 @@ __global__ void __launch_bounds__(NTS, 1)
     }
   frag::st_c(S, s.S, LDD, rb * 16, hf * 64);
 
-  fwd_load_chunk(p, s, q, k, v, g, Tg, beta, b, h, 0, a0);
+  fwd_issue(p, s.st[0], sv, b, h, 0, a0);
+  frag::cp_commit();
+  if (p.NC > 1) fwd_issue(p, s.st[1], sv, b, h, 1, a0);
+  frag::cp_commit();
   for (int n = 0; n < p.NC; ++n) {
     const int t0 = n * C, nvalid = min(C, p.T - t0);
     const size_t cb = chunk_id(p, b, h, n);
-    frag::cp_wait<0>();
+    FwdStage& st = s.st[n & 1];
+    frag::cp_wait<1>();
     __syncthreads();
-    if (tid < gk) cumsum_col(s.G, gk, tid);
-    __syncthreads();
-    const int r = centre_row(nvalid);
-    for (int idx = tid; idx < C * (D / 8); idx += NTS) {
-      const int i = idx >> 4, j = idx & 15;
-      const uint4 rq = *reinterpret_cast<const uint4*>(s.q + i * LDD + j * 8);
-      const uint4 rk = *reinterpret_cast<const uint4*>(s.k + i * LDD + j * 8);
-      const uint32_t* wq = reinterpret_cast<const uint32_t*>(&rq);
-      const uint32_t* wk = reinterpret_cast<const uint32_t*>(&rk);
-      const float bi = s.beta[i];
-      uint32_t oqc[4], okb[4], obk[4], oqh[4], okt[4];
-      float g8[8], r8[8], c8[8];
-      gate8(s.G, gk, i, j * 8, g8);
-      gate8(s.G, gk, r, j * 8, r8);
-      gate8(s.G, gk, C - 1, j * 8, c8);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 fq = frag::unpack(wq[e]), fk = frag::unpack(wk[e]);
-        const float gi0 = g8[2 * e], gi1 = g8[2 * e + 1];
-        const float ep0 = __expf(gi0 - r8[2 * e]), ep1 = __expf(gi1 - r8[2 * e + 1]);
-        const float em0 = __expf(r8[2 * e] - gi0), em1 = __expf(r8[2 * e + 1] - gi1);
-        const float ea0 = __expf(gi0), ea1 = __expf(gi1);
-        const float et0 = __expf(c8[2 * e] - gi0), et1 = __expf(c8[2 * e + 1] - gi1);
-        oqc[e] = frag::pack(fq.x * ep0, fq.y * ep1);
-        okb[e] = frag::pack(fk.x * em0, fk.y * em1);
-        obk[e] = frag::pack(bi * fk.x * ea0, bi * fk.y * ea1);
-        oqh[e] = frag::pack(fq.x * ea0, fq.y * ea1);
-        okt[e] = frag::pack(fk.x * et0, fk.y * et1);
-      }
-      *reinterpret_cast<uint4*>(s.Qc + i * LDD + j * 8) = make_uint4(oqc[0], oqc[1], oqc[2], oqc[3]);
-      *reinterpret_cast<uint4*>(s.Kb + i * LDD + j * 8) = make_uint4(okb[0], okb[1], okb[2], okb[3]);
-      *reinterpret_cast<uint4*>(s.BK + i * LDD + j * 8) = make_uint4(obk[0], obk[1], obk[2], obk[3]);
-      *reinterpret_cast<uint4*>(s.Qh + i * LDD + j * 8) = make_uint4(oqh[0], oqh[1], oqh[2], oqh[3]);
-      *reinterpret_cast<uint4*>(s.Kt + i * LDD + j * 8) = make_uint4(okt[0], okt[1], okt[2], okt[3]);
-    }
-    for (int idx = tid; idx < C * (BV / 8); idx += NTS) {
-      const int i = idx >> 3, j = idx & 7;
-      const uint4 rv = *reinterpret_cast<const uint4*>(s.v + i * LDC + j * 8);
-      const uint32_t* wv = reinterpret_cast<const uint32_t*>(&rv);
-      const float bi = s.beta[i];
-      uint32_t ov[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = frag::unpack(wv[e]);
-        ov[e] = frag::pack(bi * f.x, bi * f.y);
-      }
-      *reinterpret_cast<uint4*>(s.BV_ + i * LDC + j * 8) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
-    }
-    if (tid < D) s.dec[tid] = __expf((gk == D) ? s.G[(C - 1) * D + tid] : s.G[C - 1]);
-    __syncthreads();
-
-    // State-independent products for rows 16rb..: W (key half hf), M (column
-    // half hf, inclusive causal mask), U' (value half hf).
-    float Wc[8][4], Mc[4][4], Up[4][4];
-    frag::zero(Wc);
-    frag::mm_rows<8, 4, true>(Wc, s.T, LDC, rb * 16, s.BK, LDD, hf * 64);
-    frag::zero(Mc);
-    frag::mm_rows<4, 8, false>(Mc, s.Qc, LDD, rb * 16, s.Kb, LDD, hf * 32);
-#pragma unroll
-    for (int jt = 0; jt < 4; ++jt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = rb * 16 + lr + (e >> 1) * 8, jj = hf * 32 + jt * 8 + lc + (e & 1);
-        if (jj > i) Mc[jt][e] = 0.f;
-      }
-    frag::zero(Up);
-    frag::mm_rows<4, 4, true>(Up, s.T, LDC, rb * 16, s.BV_, LDC, hf * 32);
-    __syncthreads();  // Q^c, Kb^c, beta K e^gamma, T, beta V and the raw tiles are consumed
-    frag::st_c(Wc, sW, LDD, rb * 16, hf * 64);
-    frag::st_c(Mc, sM, LDC, rb * 16, hf * 32);
-    if (n + 1 < p.NC) fwd_load_chunk(p, s, q, k, v, g, Tg, beta, b, h, n + 1, a0);
-    if (hsave)
-      for (int idx = tid; idx < BV * (D / 8); idx += NTS) {
+    if (save)
+      for (int idx = tid; idx < BV * (D / 8); idx += NT) {
         const int a = idx >> 4, j = idx & 15;
-        *reinterpret_cast<uint4*>(hsave + cb * D * D + (size_t)(a0 + a) * D + j * 8) =
+        *reinterpret_cast<uint4*>(sv.h + cb * D * D + (size_t)(a0 + a) * D + j * 8) =
             *reinterpret_cast<const uint4*>(s.S + a * LDD + j * 8);
       }
-    __syncthreads();
-
-    // U = U' - W S^T and the inter-chunk part of O, rows 16rb.., values 32hf..
-    float oc[4][4];
+    // U = U' - W S^T and the inter-chunk part of O; rows 16rb.., values 32hf..
+    float oc[4][4], u[4][4];
     {
-      float ws[4][4];
-      frag::zero(ws);
-      frag::mm_rows<4, 8, false>(ws, sW, LDD, rb * 16, s.S, LDD, hf * 32);
+      frag::zero(u);
+      frag::mm_rows<4, 8, false>(u, st.W, LDD, rb * 16, s.S, LDD, hf * 32);
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+      for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) Up[j][e] -= ws[j][e];
-      frag::st_c(Up, s.U, LDC, rb * 16, hf * 32);
+        for (int hh = 0; hh < 2; ++hh) {
+          const float2 up = frag::unpack(*reinterpret_cast<const uint32_t*>(
+              st.Up + (rb * 16 + lr + hh * 8) * LDC + hf * 32 + jt * 8 + lc));
+          u[jt][2 * hh] = up.x - u[jt][2 * hh];
+          u[jt][2 * hh + 1] = up.y - u[jt][2 * hh + 1];
+        }
+      frag::st_c(u, s.U, LDC, rb * 16, hf * 32);
       frag::zero(oc);
-      frag::mm_rows<4, 8, false>(oc, s.Qh, LDD, rb * 16, s.S, LDD, hf * 32);
+      frag::mm_rows<4, 8, false>(oc, st.Qh, LDD, rb * 16, s.S, LDD, hf * 32);
     }
     __syncthreads();
-    if (Usave)
-      for (int idx = tid; idx < C * (BV / 8); idx += NTS) {
+    if (save)
+      for (int idx = tid; idx < C * (BV / 8); idx += NT) {
         const int i = idx >> 3, j = idx & 7;
-        *reinterpret_cast<uint4*>(Usave + (cb * C + i) * D + a0 + j * 8) =
+        *reinterpret_cast<uint4*>(sv.U + (cb * C + i) * D + a0 + j * 8) =
             *reinterpret_cast<const uint4*>(s.U + i * LDC + j * 8);
       }
     // O += M U
-    frag::mm_rows<4, 4, true>(oc, sM, LDC, rb * 16, s.U, LDC, hf * 32);
+    frag::mm_rows<4, 4, true>(oc, st.M, LDC, rb * 16, s.U, LDC, hf * 32);
     if (o) {
 #pragma unroll
       for (int jt = 0; jt < 4; ++jt)
@@ -434,18 +414,20 @@ __global__ void __launch_bounds__(NTS, 1)
                 frag::pack(oc[jt][2 * hh], oc[jt][2 * hh + 1]);
         }
     }
-    // S <- S Diag(e^{gamma_C}) + U^T Kt for state rows 16rb.., key columns 64hf..
+    // S <- S Diag(dec) + U^T Kt for state rows 16rb.., key columns 64hf..
     {
       float ds[8][4];
       frag::zero(ds);
-      frag::mm_rows_at<8, 4, true>(ds, s.U, LDC, rb * 16, s.Kt, LDD, hf * 64);
+      frag::mm_rows_at<8, 4, true>(ds, s.U, LDC, rb * 16, st.Kt, LDD, hf * 64);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          S[j][e] = S[j][e] * s.dec[hf * 64 + j * 8 + lc + (e & 1)] + ds[j][e];
+          S[j][e] = S[j][e] * st.dec[hf * 64 + j * 8 + lc + (e & 1)] + ds[j][e];
     }
-    __syncthreads();  // every warp is done with the bf16 state and the tiles
+    __syncthreads();  // this stage, the bf16 state and U are consumed
+    if (n + 2 < p.NC) fwd_issue(p, st, sv, b, h, n + 2, a0);
+    frag::cp_commit();
     frag::st_c(S, s.S, LDD, rb * 16, hf * 64);
   }
   if (ST) {
@@ -461,43 +443,38 @@ __global__ void __launch_bounds__(NTS, 1)
 
 }  // namespace
 
-size_t prep_smem(const Problem& p) { return sizeof(PrepSmem) + sizeof(float) * (C * p.gk); }
-size_t fwd_scan_smem(const Problem& p) { return sizeof(FwdSmem) + sizeof(float) * (C * p.gk); }
-
-cudaError_t launch_prep(const Problem& p, const bf16* k, const float* beta, const float* g,
-                        bf16* T, float* beta_eff, cudaStream_t st) {
-  const size_t sm = prep_smem(p);
+cudaError_t launch_prep(const Problem& p, const bf16* q, const bf16* k, const bf16* v,
+                        const float* beta, const float* g, const Saved& sv, cudaStream_t st) {
+  const size_t sm = sizeof(PrepSmem);
   cudaError_t e = cudaFuncSetAttribute(k_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const double nb = (double)p.B * p.H * p.NC, ntok = nb * C;
-  const double bytes = ntok * (D * 2 + p.gk * 4 + 4) + nb * C * C * 2 + ntok * 4;
-  const double flops = nb * 2.0 * C * C * D;
+  // reads q, k, v, g, beta; writes T, beta, dec, W, U', M, Qh, Kt
+  const double bytes = ntok * (3 * D * 2 + p.gk * 4 + 4) +
+                       nb * ((double)kTBytes + kBetaBytes + kDecBytes + 4.0 * kTileBytes + kMBytes);
+  const double flops = nb * (2.0 * 2 * C * C * D + 2.0 * 2 * C * C * D);  // [A;M] Gram, W|U'
   prof_begin(kKTcIntraFwd, bytes, flops, st);
-  k_prep<<<dim3(p.NC, p.H, p.B), NTH, sm, st>>>(p, k, beta, g, T, beta_eff);
+  k_prep<<<dim3(p.NC, p.H, p.B), NT, sm, st>>>(p, q, k, v, beta, g, sv);
   e = cudaGetLastError();
   prof_end(st);
   return e;
 }
 
-cudaError_t launch_fwd_scan(const Problem& p, const bf16* q, const bf16* k, const bf16* v,
-                            const float* g, const bf16* T, const float* beta_eff,
-                            const float* S0, bf16* o, float* ST, bf16* hsave, bf16* Usave,
-                            cudaStream_t st) {
-  const size_t sm = fwd_scan_smem(p);
+cudaError_t launch_fwd_scan(const Problem& p, const Saved& sv, const float* S0, bf16* o,
+                            float* ST, bool save, cudaStream_t st) {
+  const size_t sm = sizeof(FwdSmem);
   cudaError_t e =
       cudaFuncSetAttribute(k_fwd_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const double nb = (double)p.B * p.H * p.NC, ntok = nb * C, heads = (double)p.B * p.H;
-  double bytes = ntok * (2 * D * 2 + D * 2 + p.gk * 4 + 4) + nb * C * C * 2;
+  // reads W, Qh, Kt, M, U', dec; writes o (+ chunk states and U when saving)
+  double bytes = nb * (3.0 * kTileBytes + kMBytes + kTileBytes + kDecBytes);
   if (o) bytes += ntok * D * 2;
-  if (hsave) bytes += nb * D * D * 2;
-  if (Usave) bytes += ntok * D * 2;
+  if (save) bytes += nb * ((double)kStateBytes + kUBytes);
   bytes += heads * D * D * 4 * ((S0 ? 1 : 0) + (ST ? 1 : 0));
-  const double per_tile = 2.0 * C * C * D * 2 + 2.0 * C * C * BV * 2 + 2.0 * C * BV * D * 3;
-  const double flops = nb * (D / BV) * per_tile;
+  const double flops = nb * (D / BV) * (2.0 * C * BV * D * 3 + 2.0 * C * C * BV);
   prof_begin(kKTcScanFwd, bytes, flops, st);
-  k_fwd_scan<<<dim3(D / BV, p.H, p.B), NTS, sm, st>>>(p, q, k, v, g, T, beta_eff, S0, o, ST,
-                                                      hsave, Usave);
+  k_fwd_scan<<<dim3(D / BV, p.H, p.B), NT, sm, st>>>(p, sv, S0, o, ST, save ? 1 : 0);
   e = cudaGetLastError();
   prof_end(st);
   return e;
