@@ -133,15 +133,24 @@ __global__ void __launch_bounds__(NT, 2)
 
   // Factors: K^c, Kb^c, Q^c to shared memory; Qh, Kt, beta, dec to global.
   const int r = centre_row(nvalid);
-  for (int idx = tid; idx < C * (D / 8); idx += NT) {
-    const int i = idx >> 4, j = idx & 15;
-    const bool valid = i < nvalid;
-    uint4 rk = make_uint4(0, 0, 0, 0), rq = rk;
-    if (valid) {
+  constexpr int ITEMS = C * (D / 8) / NT;  // 16-byte row segments per thread
+  uint4 kr[ITEMS], qr[ITEMS], vr[ITEMS];
+#pragma unroll
+  for (int it = 0; it < ITEMS; ++it) {
+    const int idx = tid + it * NT, i = idx >> 4, j = idx & 15;
+    kr[it] = qr[it] = vr[it] = make_uint4(0, 0, 0, 0);
+    if (i < nvalid) {
       const size_t rr = row_id(p, b, t0 + i, h) * D + j * 8;
-      rk = *reinterpret_cast<const uint4*>(k + rr);
-      rq = *reinterpret_cast<const uint4*>(q + rr);
+      kr[it] = *reinterpret_cast<const uint4*>(k + rr);
+      qr[it] = *reinterpret_cast<const uint4*>(q + rr);
+      vr[it] = *reinterpret_cast<const uint4*>(v + rr);
     }
+  }
+#pragma unroll
+  for (int it = 0; it < ITEMS; ++it) {
+    const int idx = tid + it * NT, i = idx >> 4, j = idx & 15;
+    const bool valid = i < nvalid;
+    const uint4 rk = kr[it], rq = qr[it];
     float kv[8], qv[8], g8[8], r8[8], c8[8];
     unpack8(rk, kv);
     unpack8(rq, qv);
@@ -207,13 +216,12 @@ __global__ void __launch_bounds__(NT, 2)
       }
   }
   for (int idx = tid; idx < C * LDA; idx += NT) sT[idx] = 0.f;
-  // beta k e^gamma into R1 (k reloaded; L2-resident)
-  for (int idx = tid; idx < C * (D / 8); idx += NT) {
-    const int i = idx >> 4, j = idx & 15;
-    uint4 rk = make_uint4(0, 0, 0, 0);
-    if (i < nvalid) rk = *reinterpret_cast<const uint4*>(k + row_id(p, b, t0 + i, h) * D + j * 8);
+  // beta k e^gamma into R1 (k kept in registers)
+#pragma unroll
+  for (int it = 0; it < ITEMS; ++it) {
+    const int idx = tid + it * NT, i = idx >> 4, j = idx & 15;
     float kv[8], g8[8];
-    unpack8(rk, kv);
+    unpack8(kr[it], kv);
     gate8(G, gk, i, j * 8, g8);
     const float bi = s.beta[i];
 #pragma unroll
@@ -242,21 +250,19 @@ __global__ void __launch_bounds__(NT, 2)
 #pragma unroll
       for (int i = 0; i < 16; ++i) sT[(base + i) * LDA + base + l] = t[i];
     }
-  } else {
-    // meanwhile: beta v into the freed gate region
-    for (int idx = tid - 128; idx < C * (D / 8); idx += NT - 128) {
-      const int i = idx >> 4, j = idx & 15;
-      uint4 rv = make_uint4(0, 0, 0, 0);
-      if (i < nvalid) rv = *reinterpret_cast<const uint4*>(v + row_id(p, b, t0 + i, h) * D + j * 8);
-      float vv[8];
-      unpack8(rv, vv);
-      const float bi = s.beta[i];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) vv[e] *= bi;
-      *reinterpret_cast<uint4*>(sBV + i * LDD + j * 8) = pack8(vv);
-    }
   }
   __syncthreads();
+  // beta v into the freed gate region (v kept in registers); read after the solve
+#pragma unroll
+  for (int it = 0; it < ITEMS; ++it) {
+    const int idx = tid + it * NT, i = idx >> 4, j = idx & 15;
+    float vv[8];
+    unpack8(vr[it], vv);
+    const float bi = s.beta[i];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) vv[e] *= bi;
+    *reinterpret_cast<uint4*>(sBV + i * LDD + j * 8) = pack8(vv);
+  }
   // Off-diagonal blocks, block row bi = 1..3, tf32 tensor cores:
   //   X_j = sum_{m = 16j}^{16bi - 1} A[16bi.., m] T[m, 16j..]  (warp j < bi),
   //   T[bi, j] = -T[bi, bi] X_j
@@ -380,7 +386,8 @@ __global__ void __launch_bounds__(NT, 1)
     float oc[4][4], u[4][4];
     {
       frag::zero(u);
-      frag::mm_rows<4, 8, false>(u, st.W, LDD, rb * 16, s.S, LDD, hf * 32);
+      frag::zero(oc);
+      frag::mm_rows2<4, 8, false>(u, oc, st.W, st.Qh, LDD, rb * 16, s.S, LDD, hf * 32);
 #pragma unroll
       for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
@@ -391,8 +398,6 @@ __global__ void __launch_bounds__(NT, 1)
           u[jt][2 * hh + 1] = up.y - u[jt][2 * hh + 1];
         }
       frag::st_c(u, s.U, LDC, rb * 16, hf * 32);
-      frag::zero(oc);
-      frag::mm_rows<4, 8, false>(oc, st.Qh, LDD, rb * 16, s.S, LDD, hf * 32);
     }
     __syncthreads();
     if (save)

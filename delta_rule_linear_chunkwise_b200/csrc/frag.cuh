@@ -32,12 +32,14 @@ __device__ __forceinline__ float2 unpack(uint32_t x) {
 __device__ __forceinline__ void ldsm_x4(uint32_t* r, const bf16* p) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(tc::smem_u32(p)));
+               : "r"(tc::smem_u32(p))
+               : "memory");
 }
 __device__ __forceinline__ void ldsm_x4_t(uint32_t* r, const bf16* p) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(tc::smem_u32(p)));
+               : "r"(tc::smem_u32(p))
+               : "memory");
 }
 
 // A fragment of rows r0..r0+15, cols k0..k0+15 of a row-major tile.
@@ -94,6 +96,30 @@ __device__ __forceinline__ void mm_rows(float (&acc)[NT][4], const bf16* A, int 
         ld_b_nk(b, B, ldb, n0 + j * 8, k0 + ks * 16);
       tc::mma16816(acc[j], a, b);
       tc::mma16816(acc[j + 1], a, b + 2);
+    }
+  }
+}
+// Two products sharing the B operand: acc1 += A1 B, acc2 += A2 B (rows r0..).
+template <int NT, int KS, bool B_KN>
+__device__ __forceinline__ void mm_rows2(float (&acc1)[NT][4], float (&acc2)[NT][4],
+                                         const bf16* A1, const bf16* A2, int lda, int r0,
+                                         const bf16* B, int ldb, int n0 = 0, int k0 = 0) {
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    uint32_t a1[4], a2[4];
+    ld_a(a1, A1, lda, r0, k0 + ks * 16);
+    ld_a(a2, A2, lda, r0, k0 + ks * 16);
+#pragma unroll
+    for (int j = 0; j < NT; j += 2) {
+      uint32_t b[4];
+      if (B_KN)
+        ld_b_kn(b, B, ldb, k0 + ks * 16, n0 + j * 8);
+      else
+        ld_b_nk(b, B, ldb, n0 + j * 8, k0 + ks * 16);
+      tc::mma16816(acc1[j], a1, b);
+      tc::mma16816(acc1[j + 1], a1, b + 2);
+      tc::mma16816(acc2[j], a2, b);
+      tc::mma16816(acc2[j + 1], a2, b + 2);
     }
   }
 }
@@ -155,7 +181,7 @@ __device__ __forceinline__ uint32_t to_tf32(float x) {
   return r;
 }
 __device__ __forceinline__ void mma1688_tf32(float* d, const uint32_t* a, const uint32_t* b) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])

@@ -126,8 +126,10 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
 }
 
 // --- legacy warp-level MMA (m16n8k16, bf16 in, fp32 accumulate) ----------
+// Not volatile: the instruction touches registers only, so the compiler may
+// interleave independent accumulation chains.
 __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, const uint32_t* b) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
