@@ -1,6 +1,7 @@
 // dr_api.cu -- the C ABI declared in include/dr.h: argument validation,
 // workspace carving and kernel dispatch.  No device memory is allocated here.
 
+#include <stdlib.h>
 #include <string.h>
 
 #include "../../include/dr.h"
@@ -115,6 +116,14 @@ Ws carve(const Layout& L, void* base, int pass) {
   return w;
 }
 
+// The chunk-parallel backward has two implementations with identical results:
+// warp-level mma.sync tiles (default, 16 warps per CTA) and tcgen05 with TMEM
+// accumulators (DR_TCGEN05_BWD=1).
+bool use_tcgen05_chunk_bwd() {
+  const char* e = getenv("DR_TCGEN05_BWD");
+  return e && e[0] == '1';
+}
+
 size_t saved_bytes(const Problem& p) {
   const size_t generic = (size_t)p.B * p.H * p.NC * p.dv * p.dk * sizeof(float);
   const size_t fast = dr::fast::saved_bytes(p);
@@ -220,9 +229,13 @@ dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const 
     bf* dh = (bf*)(wsb + round_up(nb * dr::fast::kUBytes));
     e = dr::fast::launch_bwd_scan(P, sv, (const bf*)dO, dST, dS0, dU, dh, st);
     if (e == cudaSuccess)
-      e = dr::fast::launch_bwd_chunk(P, (const bf*)q, (const bf*)k, (const bf*)v,
-                                     (const bf*)dO, g, sv, dh, dU, (bf*)dq, (bf*)dk, (bf*)dv,
-                                     dbeta, dg, st);
+      e = use_tcgen05_chunk_bwd()
+              ? dr::fast::launch_bwd_chunk_tc(P, (const bf*)q, (const bf*)k, (const bf*)v,
+                                              (const bf*)dO, g, sv, dh, dU, (bf*)dq, (bf*)dk,
+                                              (bf*)dv, dbeta, dg, st)
+              : dr::fast::launch_bwd_chunk(P, (const bf*)q, (const bf*)k, (const bf*)v,
+                                           (const bf*)dO, g, sv, dh, dU, (bf*)dq, (bf*)dk,
+                                           (bf*)dv, dbeta, dg, st);
     return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
   }
   if (p->dtype == DR_F32)

@@ -77,6 +77,8 @@ void prof_end(cudaStream_t st);
 // Reads the device-side error word (bounded waits that gave up record a
 // nonzero code there) into *flag and clears it.
 cudaError_t read_and_clear_device_error(int* flag);
+// Device address of that error word on the current device (nullptr on failure).
+int* device_error_word();
 
 // Launchers of the generic (fp32 SIMT) kernels; TIn is float or __nv_bfloat16.
 template <typename TIn>

@@ -34,10 +34,12 @@ struct Saved {
   __nv_bfloat16* Kt;   // [nb][64][128]   k e^{gamma_C - gamma}
   __nv_bfloat16* h;    // [nb][128][128]  chunk start state S (value-major)
   __nv_bfloat16* U;    // [nb][64][128]   U = U' - W S^T
+  float* knorm;        // [nb][64]        ||k||^2 of each row
 };
 inline size_t saved_bytes(const Problem& p) {
   const size_t nb = (size_t)p.B * p.H * p.NC;
-  return nb * (kTBytes + kBetaBytes + kDecBytes + 4 * kTileBytes + kMBytes + kStateBytes + kUBytes);
+  return nb * (kTBytes + 2 * kBetaBytes + kDecBytes + 4 * kTileBytes + kMBytes + kStateBytes +
+               kUBytes);
 }
 inline Saved carve_saved(const Problem& p, void* base) {
   const size_t nb = (size_t)p.B * p.H * p.NC;
@@ -52,7 +54,8 @@ inline Saved carve_saved(const Problem& p, void* base) {
   s.Qh = (__nv_bfloat16*)c;           c += nb * kTileBytes;
   s.Kt = (__nv_bfloat16*)c;           c += nb * kTileBytes;
   s.h = (__nv_bfloat16*)c;            c += nb * kStateBytes;
-  s.U = (__nv_bfloat16*)c;
+  s.U = (__nv_bfloat16*)c;             c += nb * kUBytes;
+  s.knorm = (float*)c;
   return s;
 }
 
@@ -72,6 +75,13 @@ cudaError_t launch_bwd_chunk(const Problem& p, const __nv_bfloat16* q, const __n
                              const Saved& sv, const __nv_bfloat16* dh,
                              const __nv_bfloat16* dU, __nv_bfloat16* dq, __nv_bfloat16* dk,
                              __nv_bfloat16* dv, float* dbeta, float* dg, cudaStream_t st);
+
+cudaError_t launch_bwd_chunk_tc(const Problem& p, const __nv_bfloat16* q,
+                                const __nv_bfloat16* k, const __nv_bfloat16* v,
+                                const __nv_bfloat16* dO, const float* g, const Saved& sv,
+                                const __nv_bfloat16* dh, const __nv_bfloat16* dU,
+                                __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv,
+                                float* dbeta, float* dg, cudaStream_t st);
 
 // Backward scratch beyond the saved tensors: per chunk dU (bf16) and dh (bf16).
 inline size_t bwd_extra_bytes(const Problem& p) {

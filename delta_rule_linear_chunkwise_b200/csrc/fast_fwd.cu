@@ -185,6 +185,7 @@ __global__ void __launch_bounds__(NT, 2)
       }
       s.beta[i] = bb;
       sv.beta[cb * C + i] = bb;
+      sv.knorm[cb * C + i] = nn;
     }
   }
   if (tid < D) sv.dec[cb * D + tid] = __expf(gk == D ? G[(C - 1) * D + tid] : G[C - 1]);

@@ -22,6 +22,12 @@ namespace dr {
 
 __device__ int g_device_error = 0;
 
+int* device_error_word() {
+  int* ptr = nullptr;
+  if (cudaGetSymbolAddress((void**)&ptr, g_device_error) != cudaSuccess) return nullptr;
+  return ptr;
+}
+
 cudaError_t read_and_clear_device_error(int* flag) {
   cudaError_t e = cudaMemcpyFromSymbol(flag, g_device_error, sizeof(int));
   if (e != cudaSuccess || *flag == 0) return e;
