@@ -35,28 +35,10 @@ constexpr int NTS = 256;
 
 __device__ __forceinline__ int centre_row(int nvalid) { return (nvalid - 1) / 2; }
 
-__device__ __forceinline__ void cumsum_col(float* G, int ld, int col) {
-  float v[C];
-#pragma unroll
-  for (int i = 0; i < C; ++i) v[i] = G[i * ld + col];
-#pragma unroll
-  for (int i = 1; i < C; ++i) v[i] += v[i - 1];
-#pragma unroll
-  for (int i = 0; i < C; ++i) G[i * ld + col] = v[i];
-}
-
-__device__ __forceinline__ void gate8(const float* G, int gk, int i, int c, float* out) {
-  if (gk == 1) {
-    const float x = G[i];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) out[e] = x;
-  } else {
-    const float4 a = *reinterpret_cast<const float4*>(G + i * gk + c);
-    const float4 b = *reinterpret_cast<const float4*>(G + i * gk + c + 4);
-    out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
-    out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
-  }
-}
+// Position of gate element (i, c) in a [C][D] fp32 tile whose 4-column groups
+// are XOR-swizzled by row, so that the 8 rows of an mma fragment hit distinct
+// banks without padding the row.
+__device__ __forceinline__ int gsw(int i, int c) { return i * D + (c ^ ((i & 7) << 2)); }
 
 // ---------------------------------------------------------------------------
 // tc_bwd_scan (thin): streams W, Qh, Kt, M, dec and the dO slice of each chunk
@@ -197,7 +179,9 @@ struct BchunkSmem {
   float dbp[C * 4];     // dbeta partial sums per column quarter
   float dgc[4 * D];     // colsum(dS' .* S) partials per row quarter
   float ktk[4 * D];     // colsum(Kt .* dKt) partials per row block
-  float G[1];           // [C][gk] cumulative gate (dynamic tail)
+  float er[D];          // e^{gamma_r}
+  float erc[D];         // e^{gamma_C - gamma_r}
+  float G[1];           // [C][D] swizzled (gsw) cumulative gate, then e^{gamma - gamma_r}
 };
 
 __global__ void __launch_bounds__(NTB, 1)
@@ -207,7 +191,8 @@ __global__ void __launch_bounds__(NTB, 1)
                 const float* __restrict__ beta, const bf16* __restrict__ hst,
                 const bf16* __restrict__ dhst, const bf16* __restrict__ Ug,
                 const bf16* __restrict__ dUg, const bf16* __restrict__ Wg,
-                const bf16* __restrict__ Upg, bf16* __restrict__ dq, bf16* __restrict__ dk,
+                const bf16* __restrict__ Upg, const float* __restrict__ knorm_g,
+                bf16* __restrict__ dq, bf16* __restrict__ dk,
                 bf16* __restrict__ dv, float* __restrict__ dbeta, float* __restrict__ dg) {
   extern __shared__ __align__(16) unsigned char smraw[];
   BchunkSmem& s = *reinterpret_cast<BchunkSmem*>(smraw);
@@ -242,45 +227,77 @@ __global__ void __launch_bounds__(NTB, 1)
     for (int idx = tid; idx < C * (D / 4); idx += NTB) {
       const int i = idx >> 5, j = idx & 31;
       const bool ok = i < nvalid && p.gate != kGateNone;
-      frag::cp16(s.G + i * D + j * 4, g + row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 4, ok);
+      frag::cp16(s.G + gsw(i, j * 4), g + row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 4, ok);
     }
   } else if (tid < C) {
     s.G[tid] = (tid < nvalid && p.gate != kGateNone) ? g[row_id(p, b, t0 + tid, h)] : 0.f;
   }
-  if (tid < C) s.beta[tid] = beta[cb * C + tid];
+  if (tid < C) {
+    s.beta[tid] = beta[cb * C + tid];
+    s.knorm[tid] = knorm_g[cb * C + tid];
+  }
   frag::cp_commit();
   frag::cp_wait<0>();
   __syncthreads();
-  if (tid < gk) cumsum_col(s.G, gk, tid);
+  // element (i, c) of the gate tile
+  auto gat = [&](int i, int c) -> float& { return gk == D ? s.G[gsw(i, c)] : s.G[i]; };
+  if (tid < gk) {
+    float acc = 0.f;
+    for (int i = 0; i < C; ++i) {
+      acc += gat(i, tid);
+      gat(i, tid) = acc;
+    }
+  }
   __syncthreads();
 
   const int r = centre_row(nvalid);
-  // per-element gate: gamma(i, c)
-  auto gam = [&](int i, int c) -> float { return gk == D ? s.G[i * D + c] : s.G[i]; };
+  if (tid < D) {
+    const int cg = (gk == D) ? tid : 0;
+    const float gr = gat(r, cg), gC = gat(C - 1, cg);
+    s.er[tid] = __expf(gr);
+    s.erc[tid] = __expf(gC - gr);
+  }
+  // gate tile -> e^{gamma - gamma_r} in place (every thread reads the centre row first)
+  {
+    float tmp[C * D / NTB];
+    const int cnt = (gk == D) ? C * D / NTB : (tid < C ? 1 : 0);
+#pragma unroll
+    for (int u = 0; u < C * D / NTB; ++u) {
+      if (u < cnt) {
+        const int idx = tid + u * NTB;
+        const int i = (gk == D) ? idx >> 7 : idx, c = (gk == D) ? idx & 127 : 0;
+        tmp[u] = __expf(gat(i, c) - gat(r, c));
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < C * D / NTB; ++u) {
+      if (u < cnt) {
+        const int idx = tid + u * NTB;
+        const int i = (gk == D) ? idx >> 7 : idx, c = (gk == D) ? idx & 127 : 0;
+        gat(i, c) = tmp[u];
+      }
+    }
+  }
+  __syncthreads();
+  // e^{gamma - gamma_r}(i, c)
+  auto epf = [&](int i, int c) -> float { return gat(i, c); };
+  // raw keys (i, c), (i, c + 1)
+  auto k2 = [&](int i, int c) -> float2 {
+    return frag::unpack(*reinterpret_cast<const uint32_t*>(s.k + i * LDD + c));
+  };
 
-  // ---- build: Q^c in place, key norms
+  // ---- build: Q^c in place
   for (int idx = tid; idx < C * (D / 8); idx += NTB) {
     const int i = idx >> 4, j = idx & 15;
     uint4 rq = *reinterpret_cast<const uint4*>(s.Qc + i * LDD + j * 8);
-    const uint4 rk = *reinterpret_cast<const uint4*>(s.k + i * LDD + j * 8);
     uint32_t* wq = reinterpret_cast<uint32_t*>(&rq);
-    const uint32_t* wk = reinterpret_cast<const uint32_t*>(&rk);
-    float g8[8], r8[8];
-    gate8(s.G, gk, i, j * 8, g8);
-    gate8(s.G, gk, r, j * 8, r8);
-    float nn = 0.f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float2 fq = frag::unpack(wq[e]), fk = frag::unpack(wk[e]);
-      wq[e] = frag::pack(fq.x * __expf(g8[2 * e] - r8[2 * e]), fq.y * __expf(g8[2 * e + 1] - r8[2 * e + 1]));
-      nn += fk.x * fk.x + fk.y * fk.y;
+      const float2 fq = frag::unpack(wq[e]);
+      wq[e] = frag::pack(fq.x * epf(i, j * 8 + 2 * e), fq.y * epf(i, j * 8 + 2 * e + 1));
     }
     *reinterpret_cast<uint4*>(s.Qc + i * LDD + j * 8) = rq;
-    nn += __shfl_xor_sync(0xffffffffu, nn, 8);
-    nn += __shfl_xor_sync(0xffffffffu, nn, 4);
-    nn += __shfl_xor_sync(0xffffffffu, nn, 2);
-    nn += __shfl_xor_sync(0xffffffffu, nn, 1);
-    if (j == 0) s.knorm[i] = nn;
   }
   __syncthreads();
 
@@ -338,15 +355,6 @@ __global__ void __launch_bounds__(NTB, 1)
 
   // Per-element bookkeeping: thread element (jt, e) -> row i, key column c.
   float dkacc[4][4], dgacc[4][4];
-  float gr4[4][2], gc4[4][2];  // gamma_r and gamma_C of this thread's columns
-#pragma unroll
-  for (int jt = 0; jt < 4; ++jt)
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int c = qt * 32 + jt * 8 + lc + u;
-      gr4[jt][u] = gam(r, c);
-      gc4[jt][u] = gam(C - 1, c);
-    }
   // consume dKt: dk += e^{gamma_C - gamma} dKt ; dgamma -= Kt dKt ; column sums of Kt dKt
   {
     float cs[4][2] = {};
@@ -355,13 +363,14 @@ __global__ void __launch_bounds__(NTB, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int i = rb * 16 + lr + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
-        const float et = __expf(gc4[jt][e & 1] - gam(i, c));
-        const float kt = __bfloat162float(s.k[i * LDD + c]) * et;
+        const float et = s.erc[c] * __fdividef(1.f, epf(i, c));
+        const float2 kk = k2(i, c - (e & 1));
+        const float kt = ((e & 1) ? kk.y : kk.x) * et;
         dkacc[jt][e] = et * akt[jt][e];
         dgacc[jt][e] = -kt * akt[jt][e];
         cs[jt][e & 1] += kt * akt[jt][e];
         // Q-side: Z = e^{gamma_r} dQs (dq and the q terms are finished in phase 4)
-        zq[jt][e] *= __expf(gr4[jt][e & 1]);
+        zq[jt][e] *= s.er[c];
       }
 #pragma unroll
     for (int jt = 0; jt < 4; ++jt)
@@ -405,8 +414,9 @@ __global__ void __launch_bounds__(NTB, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int i = rb * 16 + lr + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
-        const float ea = __expf(gam(i, c));
-        const float kh = __bfloat162float(s.k[i * LDD + c]) * ea;  // K e^gamma
+        const float ea = s.er[c] * epf(i, c);
+        const float2 kk = k2(i, c - (e & 1));
+        const float kh = ((e & 1) ? kk.y : kk.x) * ea;  // K e^gamma
         const float bi = s.beta[i];
         dkacc[jt][e] += ea * bi * lw[jt][e];
         dgacc[jt][e] += kh * bi * lw[jt][e];
@@ -439,15 +449,13 @@ __global__ void __launch_bounds__(NTB, 1)
     const uint4 rk = *reinterpret_cast<const uint4*>(s.k + i * LDD + j * 8);
     const uint32_t* wk = reinterpret_cast<const uint32_t*>(&rk);
     const float bi = s.beta[i];
-    float g8[8], r8[8];
-    gate8(s.G, gk, i, j * 8, g8);
-    gate8(s.G, gk, r, j * 8, r8);
     uint32_t okb[4], obc[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 fk = frag::unpack(wk[e]);
-      okb[e] = frag::pack(fk.x * __expf(r8[2 * e] - g8[2 * e]), fk.y * __expf(r8[2 * e + 1] - g8[2 * e + 1]));
-      obc[e] = frag::pack(bi * fk.x * __expf(g8[2 * e] - r8[2 * e]), bi * fk.y * __expf(g8[2 * e + 1] - r8[2 * e + 1]));
+      const float p0 = epf(i, j * 8 + 2 * e), p1 = epf(i, j * 8 + 2 * e + 1);
+      okb[e] = frag::pack(fk.x * __fdividef(1.f, p0), fk.y * __fdividef(1.f, p1));
+      obc[e] = frag::pack(bi * fk.x * p0, bi * fk.y * p1);
     }
     *reinterpret_cast<uint4*>(R0 + i * LDD + j * 8) = make_uint4(okb[0], okb[1], okb[2], okb[3]);
     *reinterpret_cast<uint4*>(R1 + i * LDD + j * 8) = make_uint4(obc[0], obc[1], obc[2], obc[3]);
@@ -468,7 +476,7 @@ __global__ void __launch_bounds__(NTB, 1)
         for (int u = 0; u < 2; ++u) {
           const int e = 2 * hh + u;
           const float zz = zq[jt][e] + dqc[jt][e];
-          out[u] = __expf(gam(i, c + u) - gr4[jt][u]) * zz;
+          out[u] = epf(i, c + u) * zz;
           dgacc[jt][e] += __bfloat162float(s.Qc[i * LDD + c + u]) * zz;
         }
         if (i < nvalid)
@@ -483,8 +491,9 @@ __global__ void __launch_bounds__(NTB, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int i = rb * 16 + lr + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
-        const float ep = __expf(gam(i, c) - gr4[jt][e & 1]);
-        const float kc = __bfloat162float(s.k[i * LDD + c]) * ep;
+        const float ep = epf(i, c);
+        const float2 kk = k2(i, c - (e & 1));
+        const float kc = ((e & 1) ? kk.y : kk.x) * ep;
         const float bi = s.beta[i];
         dkacc[jt][e] += ep * bi * x[jt][e];
         dgacc[jt][e] += kc * bi * x[jt][e];
@@ -500,8 +509,9 @@ __global__ void __launch_bounds__(NTB, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int i = rb * 16 + lr + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
-        const float em = __expf(gr4[jt][e & 1] - gam(i, c));
-        const float kb = __bfloat162float(s.k[i * LDD + c]) * em;
+        const float em = __fdividef(1.f, epf(i, c));
+        const float2 kk = k2(i, c - (e & 1));
+        const float kb = ((e & 1) ? kk.y : kk.x) * em;
         dkacc[jt][e] += em * y[jt][e];
         dgacc[jt][e] -= kb * y[jt][e];
       }
@@ -554,7 +564,7 @@ __global__ void __launch_bounds__(NTB, 1)
   // dgamma: last row gets the chunk-decay terms, then reverse cumulative sum per channel
   if (tid < D) {
     const int c = tid;
-    const float eC = __expf(gam(C - 1, c));
+    const float eC = s.er[c] * s.erc[c];
     float extra = s.ktk[c] + s.ktk[D + c] + s.ktk[2 * D + c] + s.ktk[3 * D + c];
     extra += eC * (s.dgc[c] + s.dgc[D + c] + s.dgc[2 * D + c] + s.dgc[3 * D + c]);
     sdg[(C - 1) * D + c] += extra;
@@ -596,6 +606,9 @@ cudaError_t launch_bwd_scan(const Problem& p, const Saved& sv, const bf16* dO, c
   return e;
 }
 
+static_assert(sizeof(BchunkSmem) + sizeof(float) * C * D <= 232448,
+              "chunk backward shared memory exceeds the 227 KB per-block limit");
+
 size_t bwd_chunk_smem(const Problem& p) {
   return sizeof(BchunkSmem) + sizeof(float) * (C * p.gk);
 }
@@ -619,7 +632,8 @@ cudaError_t launch_bwd_chunk(const Problem& p, const bf16* q, const bf16* k, con
                      + (double)C * D * C * 4;   // dM Kb, dA Kb, dM^T Q^c, dA^T K^c
   prof_begin(kKTcChunkBwd, bytes, nb * 2.0 * mac, st);
   k_bwd_chunk<<<dim3(p.NC, p.H, p.B), NTB, sm, st>>>(p, q, k, v, dO, g, sv.T, sv.beta, sv.h, dh,
-                                                     sv.U, dU, sv.W, sv.Up, dq, dk, dv, dbeta, dg);
+                                                     sv.U, dU, sv.W, sv.Up, sv.knorm, dq, dk, dv,
+                                                     dbeta, dg);
   e = cudaGetLastError();
   prof_end(st);
   return e;

@@ -121,3 +121,37 @@ def test_full_size_workloads_sampled_heads(name):
         heads = [(0, 0), (w.B // 2, w.H // 2), (w.B - 1, w.H - 1)]
     errs = _check(w, inp, heads=heads)
     print(name, {k: f"{v:.2e}" for k, v in errs.items()})
+
+
+# The bf16 head-dim-128 tensor-core path at ragged lengths, with both chunk
+# backward kernels: the warp-level mma.sync one (default) and the tcgen05/TMEM
+# one (selected by DR_TCGEN05_BWD=1).
+BWD_VARIANTS = ["mma_sync", "tcgen05"]
+
+
+@pytest.fixture(params=BWD_VARIANTS)
+def bwd_variant(request, monkeypatch):
+    monkeypatch.setenv("DR_TCGEN05_BWD", "1" if request.param == "tcgen05" else "0")
+    return request.param
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 129])
+@pytest.mark.parametrize("gate", ["none", "scalar", "channel"])
+def test_tensor_core_path_ragged(T, gate, bwd_variant):
+    w = WORKLOADS["kda_bf16_b4h16t8192"].with_(name=f"tc_T{T}_{gate}", B=1, H=2, T=T,
+                                               gate=gate, s0_std=0.1)
+    _check(w, make_inputs(w), dST=random_state(w, seed=11, std=0.5))
+
+
+@pytest.mark.parametrize("w", SMALL[1:5], ids=lambda w: w.name)
+def test_tcgen05_backward_small_workloads(w, monkeypatch):
+    monkeypatch.setenv("DR_TCGEN05_BWD", "1")
+    inp = make_inputs(w)
+    _check(w, inp, dST=random_state(w, seed=99, std=0.5))
+    _check(w, inp, save=False)
+
+
+def test_tcgen05_backward_full_size_sampled_heads(monkeypatch):
+    monkeypatch.setenv("DR_TCGEN05_BWD", "1")
+    w = WORKLOADS["kda_bf16_b4h16t8192"]
+    _check(w, make_inputs(w), heads=[(0, 0), (w.B - 1, w.H - 1)])
