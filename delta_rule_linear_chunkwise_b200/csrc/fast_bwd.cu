@@ -353,41 +353,58 @@ __global__ void __launch_bounds__(NTB, 1)
     frag::st_c(adm, s.dM, LDC, rb * 16, qt * 16);
   }
 
-  // Per-element bookkeeping: thread element (jt, e) -> row i, key column c.
-  float dkacc[4][4], dgacc[4][4];
-  // consume dKt: dk += e^{gamma_C - gamma} dKt ; dgamma -= Kt dKt ; column sums of Kt dKt
+  // The per-element epilogue works on three accumulators at this thread's
+  // fragment positions (rows i0, i0 + 8; key columns c), with ep = e^{gamma - gamma_r}:
+  //   Z = e^{gamma_r} dQs + dM Kb^c                               -> dq = ep Z
+  //   P = e^{gamma_C - gamma_r} dKt + dM^T Q^c + dA^T diag(beta) K^c
+  //   Q = e^{gamma_r} Lambda_W + dA Kb^c
+  // so that dk = P / ep + beta ep Q,  dgamma = k (beta ep Q - P / ep) + Q^c Z
+  // and d(beta_eff) = Lambda_U . v + k . (ep Q) summed over the row.
+  const int i0 = rb * 16 + lr;
+  const size_t rowg[2] = {row_id(p, b, t0 + min(i0, nvalid - 1), h) * D,
+                          row_id(p, b, t0 + min(i0 + 8, nvalid - 1), h) * D};
+  float(&Z)[4][4] = zq;
+  float(&P)[4][4] = akt;
+  // colsum(Kt .* dKt) for the chunk-end gate term, then the column scalings
   {
     float cs[4][2] = {};
 #pragma unroll
     for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int i = rb * 16 + lr + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
-        const float et = s.erc[c] * __fdividef(1.f, epf(i, c));
+        const int i = i0 + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
         const float2 kk = k2(i, c - (e & 1));
-        const float kt = ((e & 1) ? kk.y : kk.x) * et;
-        dkacc[jt][e] = et * akt[jt][e];
-        dgacc[jt][e] = -kt * akt[jt][e];
-        cs[jt][e & 1] += kt * akt[jt][e];
-        // Q-side: Z = e^{gamma_r} dQs (dq and the q terms are finished in phase 4)
-        zq[jt][e] *= s.er[c];
+        cs[jt][e & 1] += ((e & 1) ? kk.y : kk.x) * __fdividef(akt[jt][e], epf(i, c));
       }
 #pragma unroll
     for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        float x = cs[jt][u];
+        const int c = qt * 32 + jt * 8 + lc + u;
+        const float fr = s.er[c], frc = s.erc[c];
+        float x = cs[jt][u] * frc;
         x += __shfl_xor_sync(0xffffffffu, x, 4);
         x += __shfl_xor_sync(0xffffffffu, x, 8);
         x += __shfl_xor_sync(0xffffffffu, x, 16);
-        if (lr == 0) s.ktk[rb * D + qt * 32 + jt * 8 + lc + u] = x;
+        if (lr == 0) s.ktk[rb * D + c] = x;
+        Z[jt][u] *= fr;
+        Z[jt][2 + u] *= fr;
+        P[jt][u] *= frc;
+        P[jt][2 + u] *= frc;
       }
   }
   __syncthreads();
 
-  // ---- phase 2: Lambda = T^T [dU | dW]
-  float dbrow[2] = {0.f, 0.f};  // this thread's dbeta partials for rows lr, lr + 8
+  // ---- phase 2: Lambda = T^T [dU | dW]; dv = diag(beta) Lambda_U
+  float dbrow[2] = {0.f, 0.f};  // this thread's d(beta_eff) partials for rows i0, i0 + 8
+  float Q[4][4];
   {
+    uint32_t vv[4][2];
+#pragma unroll
+    for (int jt = 0; jt < 4; ++jt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+        vv[jt][hh] = *reinterpret_cast<const uint32_t*>(v + rowg[hh] + qt * 32 + jt * 8 + lc);
     float lu[4][4];
     frag::zero(lu);
     frag::mm_rows_at<4, 4, true>(lu, s.T, LDC, rb * 16, s.dU, LDD, qt * 32);
@@ -395,34 +412,26 @@ __global__ void __launch_bounds__(NTB, 1)
     for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
-        const int i = rb * 16 + lr + hh * 8, a = qt * 32 + jt * 8 + lc;
+        const int i = i0 + hh * 8, a = qt * 32 + jt * 8 + lc;
         const float bi = s.beta[i];
-        if (i < nvalid) {
-          const size_t rr = row_id(p, b, t0 + i, h) * D + a;
-          *reinterpret_cast<uint32_t*>(dv + rr) =
+        if (i < nvalid)
+          *reinterpret_cast<uint32_t*>(dv + rowg[hh] + a) =
               frag::pack(bi * lu[jt][2 * hh], bi * lu[jt][2 * hh + 1]);
-          const float2 vv = frag::unpack(*reinterpret_cast<const uint32_t*>(v + rr));
-          dbrow[hh] += lu[jt][2 * hh] * vv.x + lu[jt][2 * hh + 1] * vv.y;
-        }
+        const float2 vf = frag::unpack(vv[jt][hh]);
+        dbrow[hh] += lu[jt][2 * hh] * vf.x + lu[jt][2 * hh + 1] * vf.y;
       }
     frag::st_c(lu, R0, LDD, rb * 16, qt * 32);
-    float lw[4][4];
-    frag::zero(lw);
-    frag::mm_rows_at<4, 4, true>(lw, s.T, LDC, rb * 16, s.dW, LDD, qt * 32);
+    frag::zero(Q);
+    frag::mm_rows_at<4, 4, true>(Q, s.T, LDC, rb * 16, s.dW, LDD, qt * 32);
+    frag::st_c(Q, R1, LDD, rb * 16, qt * 32);
 #pragma unroll
     for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = rb * 16 + lr + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
-        const float ea = s.er[c] * epf(i, c);
-        const float2 kk = k2(i, c - (e & 1));
-        const float kh = ((e & 1) ? kk.y : kk.x) * ea;  // K e^gamma
-        const float bi = s.beta[i];
-        dkacc[jt][e] += ea * bi * lw[jt][e];
-        dgacc[jt][e] += kh * bi * lw[jt][e];
-        dbrow[e >> 1] += lw[jt][e] * kh;
+      for (int u = 0; u < 2; ++u) {
+        const float fr = s.er[qt * 32 + jt * 8 + lc + u];
+        Q[jt][u] *= fr;
+        Q[jt][2 + u] *= fr;
       }
-    frag::st_c(lw, R1, LDD, rb * 16, qt * 32);
   }
   __syncthreads();
 
@@ -454,134 +463,130 @@ __global__ void __launch_bounds__(NTB, 1)
     for (int e = 0; e < 4; ++e) {
       const float2 fk = frag::unpack(wk[e]);
       const float p0 = epf(i, j * 8 + 2 * e), p1 = epf(i, j * 8 + 2 * e + 1);
-      okb[e] = frag::pack(fk.x * __fdividef(1.f, p0), fk.y * __fdividef(1.f, p1));
+      okb[e] = frag::pack(__fdividef(fk.x, p0), __fdividef(fk.y, p1));
       obc[e] = frag::pack(bi * fk.x * p0, bi * fk.y * p1);
     }
     *reinterpret_cast<uint4*>(R0 + i * LDD + j * 8) = make_uint4(okb[0], okb[1], okb[2], okb[3]);
     *reinterpret_cast<uint4*>(R1 + i * LDD + j * 8) = make_uint4(obc[0], obc[1], obc[2], obc[3]);
   }
   __syncthreads();
-  {
-    // dQ^c = dM Kb^c -> dq = e^{gamma - gamma_r} (Z + dQ^c); dgamma += Q^c (Z + dQ^c)
-    float dqc[4][4];
-    frag::zero(dqc);
-    frag::mm_rows<4, 4, true>(dqc, s.dM, LDC, rb * 16, R0, LDD, qt * 32);
+  frag::mm_rows<4, 4, true>(Z, s.dM, LDC, rb * 16, R0, LDD, qt * 32);     // Z += dM Kb^c
+  frag::mm_rows<4, 4, true>(Q, sdA, LDC, rb * 16, R0, LDD, qt * 32);      // Q += dA Kb^c
+  frag::mm_rows_at<4, 4, true>(P, s.dM, LDC, rb * 16, s.Qc, LDD, qt * 32); // P += dM^T Q^c
+  frag::mm_rows_at<4, 4, true>(P, sdA, LDC, rb * 16, R1, LDD, qt * 32);   // P += dA^T beta K^c
+
+  // ---- per-element epilogue: dq out; P <- dk (before the Kaczmarz term), Q <- dgamma
 #pragma unroll
-    for (int jt = 0; jt < 4; ++jt)
+  for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int i = rb * 16 + lr + hh * 8, c = qt * 32 + jt * 8 + lc;
-        float out[2];
+    for (int hh = 0; hh < 2; ++hh) {
+      const int i = i0 + hh * 8, c = qt * 32 + jt * 8 + lc;
+      const float bi = s.beta[i];
+      const float2 kk = k2(i, c);
+      const float2 qc = frag::unpack(*reinterpret_cast<const uint32_t*>(s.Qc + i * LDD + c));
+      float outq[2];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int e = 2 * hh + u;
-          const float zz = zq[jt][e] + dqc[jt][e];
-          out[u] = epf(i, c + u) * zz;
-          dgacc[jt][e] += __bfloat162float(s.Qc[i * LDD + c + u]) * zz;
+      for (int u = 0; u < 2; ++u) {
+        const int e = 2 * hh + u;
+        const float ep = epf(i, c + u);
+        const float t1 = ep * Q[jt][e], t2 = __fdividef(P[jt][e], ep);
+        const float kv = u ? kk.y : kk.x, qv = u ? qc.y : qc.x;
+        float dgv = kv * (bi * t1 - t2) + qv * Z[jt][e];
+        if (i == C - 1) {  // chunk-end gate term: colsum(Kt .* dKt) + e^{gamma_C} colsum(dS' .* S)
+          const int cc = c + u;
+          const float eC = s.er[cc] * s.erc[cc];
+          dgv += s.ktk[cc] + s.ktk[D + cc] + s.ktk[2 * D + cc] + s.ktk[3 * D + cc] +
+                 eC * (s.dgc[cc] + s.dgc[D + cc] + s.dgc[2 * D + cc] + s.dgc[3 * D + cc]);
         }
-        if (i < nvalid)
-          *reinterpret_cast<uint32_t*>(dq + row_id(p, b, t0 + i, h) * D + c) = frag::pack(out[0], out[1]);
+        dbrow[hh] += kv * t1;
+        outq[u] = ep * Z[jt][e];
+        P[jt][e] = bi * t1 + t2;
+        Q[jt][e] = dgv;
       }
-    // x = dA Kb^c: dk += e^{gamma - gamma_r} beta x; dgamma += K^c beta x; dbeta += K^c . x
-    float x[4][4];
-    frag::zero(x);
-    frag::mm_rows<4, 4, true>(x, sdA, LDC, rb * 16, R0, LDD, qt * 32);
-#pragma unroll
-    for (int jt = 0; jt < 4; ++jt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = rb * 16 + lr + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
-        const float ep = epf(i, c);
-        const float2 kk = k2(i, c - (e & 1));
-        const float kc = ((e & 1) ? kk.y : kk.x) * ep;
-        const float bi = s.beta[i];
-        dkacc[jt][e] += ep * bi * x[jt][e];
-        dgacc[jt][e] += kc * bi * x[jt][e];
-        dbrow[e >> 1] += kc * x[jt][e];
-      }
-    // y = dM^T Q^c + dA^T (beta K^c): dk += e^{gamma_r - gamma} y; dgamma -= Kb^c y
-    float y[4][4];
-    frag::zero(y);
-    frag::mm_rows_at<4, 4, true>(y, s.dM, LDC, rb * 16, s.Qc, LDD, qt * 32);
-    frag::mm_rows_at<4, 4, true>(y, sdA, LDC, rb * 16, R1, LDD, qt * 32);
-#pragma unroll
-    for (int jt = 0; jt < 4; ++jt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = rb * 16 + lr + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
-        const float em = __fdividef(1.f, epf(i, c));
-        const float2 kk = k2(i, c - (e & 1));
-        const float kb = ((e & 1) ? kk.y : kk.x) * em;
-        dkacc[jt][e] += em * y[jt][e];
-        dgacc[jt][e] -= kb * y[jt][e];
-      }
-  }
-  // dbeta partials: reduce the 4 lanes that share a row, then one slot per quarter
+      if (i < nvalid)
+        *reinterpret_cast<uint32_t*>(dq + rowg[hh] + c) = frag::pack(outq[0], outq[1]);
+    }
+  // d(beta_eff) partials: reduce the 4 lanes that share a row, one slot per column quarter
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
     float xx = dbrow[hh];
     xx += __shfl_xor_sync(0xffffffffu, xx, 1);
     xx += __shfl_xor_sync(0xffffffffu, xx, 2);
-    if ((lane & 3) == 0) s.dbp[(rb * 16 + lr + hh * 8) * 4 + qt] = xx;
+    if ((lane & 3) == 0) s.dbp[(i0 + hh * 8) * 4 + qt] = xx;
   }
-  __syncthreads();  // R0/R1 free: reuse as the fp32 dgamma tile
+  __syncthreads();  // R0/R1 free: reuse for the dgamma reduction
   float* sdg = reinterpret_cast<float*>(s.R);
+  if (gk == D) {
 #pragma unroll
-  for (int jt = 0; jt < 4; ++jt)
+    for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int i = rb * 16 + lr + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
-      sdg[i * D + c] = dgacc[jt][e];
+      for (int e = 0; e < 4; ++e)
+        sdg[(i0 + (e >> 1) * 8) * D + qt * 32 + jt * 8 + lc + (e & 1)] = Q[jt][e];
+  } else {
+    // scalar gate: the row sums of dgamma, one slot per column quarter
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      float xx = 0.f;
+#pragma unroll
+      for (int jt = 0; jt < 4; ++jt) xx += Q[jt][2 * hh] + Q[jt][2 * hh + 1];
+      xx += __shfl_xor_sync(0xffffffffu, xx, 1);
+      xx += __shfl_xor_sync(0xffffffffu, xx, 2);
+      if ((lane & 3) == 0) sdg[(i0 + hh * 8) * 4 + qt] = xx;
     }
-  if (tid < C) {
-    const float db = s.dbp[tid * 4] + s.dbp[tid * 4 + 1] + s.dbp[tid * 4 + 2] + s.dbp[tid * 4 + 3];
-    s.dbp[tid * 4] = db;  // total d(beta_eff) of row tid
   }
+  __syncthreads();
+  float dbt = 0.f;
+  if (tid < C) dbt = s.dbp[tid * 4] + s.dbp[tid * 4 + 1] + s.dbp[tid * 4 + 2] + s.dbp[tid * 4 + 3];
+  const int gc = tid & 127, grq = tid >> 7;  // dgamma reverse scan: channel, row quarter
+  if (gk == D) {
+    float part = 0.f;
+#pragma unroll 4
+    for (int i = grq * 16; i < grq * 16 + 16; ++i) part += sdg[i * D + gc];
+    s.dgc[grq * D + gc] = part;  // the chunk-end term read dgc before the last two barriers
+  }
+  if (tid < C) s.dbp[tid * 4] = dbt;  // total d(beta_eff) of row tid
   __syncthreads();
   // dk (with the Kaczmarz chain rule) and dbeta
 #pragma unroll
   for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-      const int i = rb * 16 + lr + hh * 8, c = qt * 32 + jt * 8 + lc;
-      float out[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        float val = dkacc[jt][2 * hh + u];
-        if (p.beta_mode == kBetaKaczmarz)
-          val += -2.f * s.beta[i] * s.dbp[i * 4] * __bfloat162float(s.k[i * LDD + c + u]) /
-                 (s.knorm[i] + p.eps);
-        out[u] = val;
+      const int i = i0 + hh * 8, c = qt * 32 + jt * 8 + lc;
+      float o0 = P[jt][2 * hh], o1 = P[jt][2 * hh + 1];
+      if (p.beta_mode == kBetaKaczmarz) {
+        const float f = -2.f * s.beta[i] * s.dbp[i * 4] / (s.knorm[i] + p.eps);
+        const float2 kk = k2(i, c);
+        o0 += f * kk.x;
+        o1 += f * kk.y;
       }
-      if (i < nvalid)
-        *reinterpret_cast<uint32_t*>(dk + row_id(p, b, t0 + i, h) * D + c) = frag::pack(out[0], out[1]);
+      if (i < nvalid) *reinterpret_cast<uint32_t*>(dk + rowg[hh] + c) = frag::pack(o0, o1);
     }
   if (tid < nvalid) {
-    float db = s.dbp[tid * 4];
-    if (p.beta_mode == kBetaKaczmarz) db /= (s.knorm[tid] + p.eps);
-    dbeta[row_id(p, b, t0 + tid, h)] = db;
+    if (p.beta_mode == kBetaKaczmarz) dbt /= (s.knorm[tid] + p.eps);
+    dbeta[row_id(p, b, t0 + tid, h)] = dbt;
   }
-  // dgamma: last row gets the chunk-decay terms, then reverse cumulative sum per channel
-  if (tid < D) {
-    const int c = tid;
-    const float eC = s.er[c] * s.erc[c];
-    float extra = s.ktk[c] + s.ktk[D + c] + s.ktk[2 * D + c] + s.ktk[3 * D + c];
-    extra += eC * (s.dgc[c] + s.dgc[D + c] + s.dgc[2 * D + c] + s.dgc[3 * D + c]);
-    sdg[(C - 1) * D + c] += extra;
+  // dgamma: reverse cumulative sum over the chunk's rows
+  if (gk == D) {
     float run = 0.f;
-    for (int i = C - 1; i >= 0; --i) {
-      run += sdg[i * D + c];
-      sdg[i * D + c] = run;
-      if (gk == D && i < nvalid) dg[row_id(p, b, t0 + i, h) * D + c] = run;
+    for (int q2 = grq + 1; q2 < 4; ++q2) run += s.dgc[q2 * D + gc];
+#pragma unroll 4
+    for (int i = grq * 16 + 15; i >= grq * 16; --i) {
+      run += sdg[i * D + gc];
+      if (i < nvalid) dg[row_id(p, b, t0 + i, h) * D + gc] = run;
     }
-  }
-  if (gk == 1 && p.gate != kGateNone) {
-    __syncthreads();
-    if (tid < nvalid) {
-      float sum = 0.f;
-      for (int c = 0; c < D; ++c) sum += sdg[tid * D + c];
-      dg[row_id(p, b, t0 + tid, h)] = sum;
+  } else if (p.gate != kGateNone && warp == 0) {
+    // rows 2 lane, 2 lane + 1: suffix sums across the warp
+    const int ia = 2 * lane, ib = ia + 1;
+    const float a0 = sdg[ia * 4] + sdg[ia * 4 + 1] + sdg[ia * 4 + 2] + sdg[ia * 4 + 3];
+    const float a1 = sdg[ib * 4] + sdg[ib * 4 + 1] + sdg[ib * 4 + 2] + sdg[ib * 4 + 3];
+    float x = a0 + a1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_down_sync(0xffffffffu, x, o);
+      if (lane + o < 32) x += y;
     }
+    if (ia < nvalid) dg[row_id(p, b, t0 + ia, h)] = x;
+    if (ib < nvalid) dg[row_id(p, b, t0 + ib, h)] = x - a0;
   }
 }
 
