@@ -35,10 +35,11 @@ constexpr int NTS = 256;
 
 __device__ __forceinline__ int centre_row(int nvalid) { return (nvalid - 1) / 2; }
 
-// Position of gate element (i, c) in a [C][D] fp32 tile whose 4-column groups
-// are XOR-swizzled by row, so that the 8 rows of an mma fragment hit distinct
-// banks without padding the row.
-__device__ __forceinline__ int gsw(int i, int c) { return i * D + (c ^ ((i & 7) << 2)); }
+// Position of gate element (i, c) in a [C][D] fp32 tile whose 8-column groups
+// are XOR-swizzled by row (i mod 8), so that the column pairs an mma fragment
+// holds in its 8 rows hit distinct banks without padding the row; groups of 4
+// consecutive columns stay contiguous and 16-byte aligned.
+__device__ __forceinline__ int gsw(int i, int c) { return i * D + (c ^ ((i & 7) << 3)); }
 
 // ---------------------------------------------------------------------------
 // tc_bwd_scan (thin): streams W, Qh, Kt, M, dec and the dO slice of each chunk
@@ -280,24 +281,32 @@ __global__ void __launch_bounds__(NTB, 1)
     }
   }
   __syncthreads();
-  // e^{gamma - gamma_r}(i, c)
-  auto epf = [&](int i, int c) -> float { return gat(i, c); };
+  // e^{gamma - gamma_r} at (i, c), (i, c + 1), c even
+  auto ep2 = [&](int i, int c) -> float2 {
+    if (gk == D) return *reinterpret_cast<const float2*>(s.G + gsw(i, c));
+    const float x = s.G[i];
+    return make_float2(x, x);
+  };
+  // e^{gamma - gamma_r} at (i, c .. c + 3), c a multiple of 4
+  auto ep4 = [&](int i, int c) -> float4 {
+    if (gk == D) return *reinterpret_cast<const float4*>(s.G + gsw(i, c));
+    const float x = s.G[i];
+    return make_float4(x, x, x, x);
+  };
   // raw keys (i, c), (i, c + 1)
   auto k2 = [&](int i, int c) -> float2 {
     return frag::unpack(*reinterpret_cast<const uint32_t*>(s.k + i * LDD + c));
   };
 
-  // ---- build: Q^c in place
-  for (int idx = tid; idx < C * (D / 8); idx += NTB) {
-    const int i = idx >> 4, j = idx & 15;
-    uint4 rq = *reinterpret_cast<const uint4*>(s.Qc + i * LDD + j * 8);
-    uint32_t* wq = reinterpret_cast<uint32_t*>(&rq);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 fq = frag::unpack(wq[e]);
-      wq[e] = frag::pack(fq.x * epf(i, j * 8 + 2 * e), fq.y * epf(i, j * 8 + 2 * e + 1));
-    }
-    *reinterpret_cast<uint4*>(s.Qc + i * LDD + j * 8) = rq;
+  // ---- build: Q^c in place (4 columns per thread, one row per warp)
+  for (int idx = tid; idx < C * (D / 4); idx += NTB) {
+    const int i = idx >> 5, c = (idx & 31) * 4;
+    uint2 rq = *reinterpret_cast<const uint2*>(s.Qc + i * LDD + c);
+    const float4 f = ep4(i, c);
+    const float2 q0 = frag::unpack(rq.x), q1 = frag::unpack(rq.y);
+    rq.x = frag::pack(q0.x * f.x, q0.y * f.y);
+    rq.y = frag::pack(q1.x * f.z, q1.y * f.w);
+    *reinterpret_cast<uint2*>(s.Qc + i * LDD + c) = rq;
   }
   __syncthreads();
 
@@ -371,10 +380,11 @@ __global__ void __launch_bounds__(NTB, 1)
 #pragma unroll
     for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = i0 + (e >> 1) * 8, c = qt * 32 + jt * 8 + lc + (e & 1);
-        const float2 kk = k2(i, c - (e & 1));
-        cs[jt][e & 1] += ((e & 1) ? kk.y : kk.x) * __fdividef(akt[jt][e], epf(i, c));
+      for (int hh = 0; hh < 2; ++hh) {
+        const int i = i0 + hh * 8, c = qt * 32 + jt * 8 + lc;
+        const float2 kk = k2(i, c), f = ep2(i, c);
+        cs[jt][0] += kk.x * __fdividef(akt[jt][2 * hh], f.x);
+        cs[jt][1] += kk.y * __fdividef(akt[jt][2 * hh + 1], f.y);
       }
 #pragma unroll
     for (int jt = 0; jt < 4; ++jt)
@@ -452,22 +462,19 @@ __global__ void __launch_bounds__(NTB, 1)
   }
   __syncthreads();
 
-  // ---- phase 4: Kb^c into R0, beta K^c into R1
-  for (int idx = tid; idx < C * (D / 8); idx += NTB) {
-    const int i = idx >> 4, j = idx & 15;
-    const uint4 rk = *reinterpret_cast<const uint4*>(s.k + i * LDD + j * 8);
-    const uint32_t* wk = reinterpret_cast<const uint32_t*>(&rk);
+  // ---- phase 4: Kb^c into R0, beta K^c into R1 (4 columns per thread, one row per warp)
+  for (int idx = tid; idx < C * (D / 4); idx += NTB) {
+    const int i = idx >> 5, c = (idx & 31) * 4;
+    const uint2 rk = *reinterpret_cast<const uint2*>(s.k + i * LDD + c);
     const float bi = s.beta[i];
-    uint32_t okb[4], obc[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 fk = frag::unpack(wk[e]);
-      const float p0 = epf(i, j * 8 + 2 * e), p1 = epf(i, j * 8 + 2 * e + 1);
-      okb[e] = frag::pack(__fdividef(fk.x, p0), __fdividef(fk.y, p1));
-      obc[e] = frag::pack(bi * fk.x * p0, bi * fk.y * p1);
-    }
-    *reinterpret_cast<uint4*>(R0 + i * LDD + j * 8) = make_uint4(okb[0], okb[1], okb[2], okb[3]);
-    *reinterpret_cast<uint4*>(R1 + i * LDD + j * 8) = make_uint4(obc[0], obc[1], obc[2], obc[3]);
+    const float4 f = ep4(i, c);
+    const float2 k0 = frag::unpack(rk.x), k1 = frag::unpack(rk.y);
+    *reinterpret_cast<uint2*>(R0 + i * LDD + c) =
+        make_uint2(frag::pack(__fdividef(k0.x, f.x), __fdividef(k0.y, f.y)),
+                   frag::pack(__fdividef(k1.x, f.z), __fdividef(k1.y, f.w)));
+    *reinterpret_cast<uint2*>(R1 + i * LDD + c) =
+        make_uint2(frag::pack(bi * k0.x * f.x, bi * k0.y * f.y),
+                   frag::pack(bi * k1.x * f.z, bi * k1.y * f.w));
   }
   __syncthreads();
   frag::mm_rows<4, 4, true>(Z, s.dM, LDC, rb * 16, R0, LDD, qt * 32);     // Z += dM Kb^c
@@ -484,11 +491,12 @@ __global__ void __launch_bounds__(NTB, 1)
       const float bi = s.beta[i];
       const float2 kk = k2(i, c);
       const float2 qc = frag::unpack(*reinterpret_cast<const uint32_t*>(s.Qc + i * LDD + c));
+      const float2 f = ep2(i, c);
       float outq[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int e = 2 * hh + u;
-        const float ep = epf(i, c + u);
+        const float ep = u ? f.y : f.x;
         const float t1 = ep * Q[jt][e], t2 = __fdividef(P[jt][e], ep);
         const float kv = u ? kk.y : kk.x, qv = u ? qc.y : qc.x;
         float dgv = kv * (bi * t1 - t2) + qv * Z[jt][e];
