@@ -124,6 +124,15 @@ bool use_tcgen05_chunk_bwd() {
   return e && e[0] == '1';
 }
 
+// The forward state scan likewise: tcgen05 with the state in registers and the
+// products in TMEM (default), or warp-level mma.sync tiles (DR_MMA_SYNC_SCAN=1).
+cudaError_t fwd_scan(const dr::Problem& P, const dr::fast::Saved& sv, const float* S0,
+                     __nv_bfloat16* o, float* ST, bool save, cudaStream_t st) {
+  const char* e = getenv("DR_MMA_SYNC_SCAN");
+  if (e && e[0] == '1') return dr::fast::launch_fwd_scan(P, sv, S0, o, ST, save, st);
+  return dr::fast::launch_fwd_scan_tc(P, sv, S0, o, ST, save, st);
+}
+
 size_t saved_bytes(const Problem& p) {
   const size_t generic = (size_t)p.B * p.H * p.NC * p.dv * p.dk * sizeof(float);
   const size_t fast = dr::fast::saved_bytes(p);
@@ -176,7 +185,7 @@ dr_status dr_chunk_fwd(const dr_problem* p, const void* q, const void* k, const 
     using bf = __nv_bfloat16;
     e = dr::fast::launch_prep(P, (const bf*)q, (const bf*)k, (const bf*)v, beta, g, sv, st);
     if (e == cudaSuccess)
-      e = dr::fast::launch_fwd_scan(P, sv, S0, (bf*)o, ST, saved != nullptr, st);
+      e = fwd_scan(P, sv, S0, (bf*)o, ST, saved != nullptr, st);
     return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
   }
   if (p->dtype == DR_F32)
@@ -220,7 +229,7 @@ dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const 
     } else {
       sv = dr::fast::carve_saved(P, wsb);
       e = dr::fast::launch_prep(P, (const bf*)q, (const bf*)k, (const bf*)v, beta, g, sv, st);
-      if (e == cudaSuccess) e = dr::fast::launch_fwd_scan(P, sv, S0, nullptr, nullptr, true, st);
+      if (e == cudaSuccess) e = fwd_scan(P, sv, S0, nullptr, nullptr, true, st);
       if (e != cudaSuccess) return DR_ERR_CUDA;
       wsb += round_up(dr::fast::saved_bytes(P));
     }

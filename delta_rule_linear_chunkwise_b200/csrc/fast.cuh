@@ -2,6 +2,7 @@
 #pragma once
 
 #include "dr_common.cuh"
+#include "frag.cuh"
 
 namespace dr {
 namespace fast {
@@ -22,20 +23,76 @@ constexpr size_t kUBytes = kTileBytes;         // pseudo-values U / dU, bf16
 
 // The per-chunk tensors of the forward that the backward reuses ("saved"):
 // the state-independent chunk tiles written by tc_prep and the chunk start
-// states and pseudo-values written by the forward scan.  All row-major.
+// states and pseudo-values written by the forward scan.  T and h are
+// row-major; the tiles marked [ct] are core-tiled (see ct_off).
 struct Saved {
   __nv_bfloat16* T;    // [nb][64][64]    (I + A)^{-1}
   float* beta;         // [nb][64]        beta (Kaczmarz step applied)
   float* dec;          // [nb][128]       e^{gamma_C}
-  __nv_bfloat16* W;    // [nb][64][128]   T diag(beta) k e^gamma
-  __nv_bfloat16* Up;   // [nb][64][128]   T diag(beta) v
-  __nv_bfloat16* M;    // [nb][64][64]    tril(Q^c Kb^c^T)
-  __nv_bfloat16* Qh;   // [nb][64][128]   q e^gamma
-  __nv_bfloat16* Kt;   // [nb][64][128]   k e^{gamma_C - gamma}
+  __nv_bfloat16* W;    // [nb][64][128]   T diag(beta) k e^gamma               [ct]
+  __nv_bfloat16* Up;   // [nb][64][128]   T diag(beta) v                       [ct]
+  __nv_bfloat16* M;    // [nb][64][64]    tril(Q^c Kb^c^T)                     [ct]
+  __nv_bfloat16* Qh;   // [nb][64][128]   q e^gamma                            [ct]
+  __nv_bfloat16* Kt;   // [nb][64][128]   k e^{gamma_C - gamma}                [ct]
   __nv_bfloat16* h;    // [nb][128][128]  chunk start state S (value-major)
-  __nv_bfloat16* U;    // [nb][64][128]   U = U' - W S^T
+  __nv_bfloat16* U;    // [nb][64][128]   U = U' - W S^T                       [ct]
   float* knorm;        // [nb][64]        ||k||^2 of each row
 };
+
+// Core-tiled storage of an [R][ncol] bf16 tile: 8 x 8 blocks of 128
+// contiguous bytes in row-block-major order, element (r, c) at ct_off.  It is
+// the tcgen05 no-swizzle operand layout, so such a tile moves between HBM and
+// shared memory as one contiguous block; 16-byte chunk idx holds row
+// ct_row(idx), columns ct_col(idx) .. + 7.
+__host__ __device__ __forceinline__ size_t ct_off(int r, int c, int ncol) {
+  return ((size_t)(r >> 3) * (ncol >> 3) + (c >> 3)) * 64 + (r & 7) * 8 + (c & 7);
+}
+__host__ __device__ __forceinline__ int ct_row(int idx, int ncol) {
+  return ((idx >> 3) / (ncol >> 3)) * 8 + (idx & 7);
+}
+__host__ __device__ __forceinline__ int ct_col(int idx, int ncol) {
+  return ((idx >> 3) % (ncol >> 3)) * 8;
+}
+
+// cp.async of a core-tiled [R][ncol] global tile into a padded row-major
+// shared tile (row stride lds): chunk idx is read from g + 8 idx (a warp reads
+// 512 contiguous bytes) and lands at row ct_row, column ct_col (eight lanes
+// write eight rows: no bank conflicts when lds = 8 mod 64).
+template <int NTHREADS>
+__device__ __forceinline__ void cp_ct_to_rows(__nv_bfloat16* smem, int lds,
+                                              const __nv_bfloat16* g, int R, int ncol, int tid) {
+  for (int idx = tid; idx < R * ncol / 8; idx += NTHREADS)
+    frag::cp16(smem + ct_row(idx, ncol) * lds + ct_col(idx, ncol), g + 8 * idx, true);
+}
+// The same for columns c0 .. c0 + w - 1 of a core-tiled [R][128] tile (each
+// row block of the slice is w 16-byte chunks, contiguous in global memory).
+template <int NTHREADS>
+__device__ __forceinline__ void cp_ct_cols_to_rows(__nv_bfloat16* smem, int lds,
+                                                   const __nv_bfloat16* g, int R, int c0, int w,
+                                                   int tid) {
+  for (int idx = tid; idx < R * w / 8; idx += NTHREADS) {
+    const int grp = idx / w, k = idx % w;
+    frag::cp16(smem + (grp * 8 + (k & 7)) * lds + (k >> 3) * 8,
+               g + ((size_t)grp * 16 + (c0 >> 3)) * 64 + 8 * k, true);
+  }
+}
+// Columns c0 .. c0 + w - 1 of a core-tiled [R][128] tile into a core-tiled
+// [R][w] shared tile.
+template <int NTHREADS>
+__device__ __forceinline__ void cp_ct_cols(__nv_bfloat16* smem, const __nv_bfloat16* g, int R,
+                                           int c0, int w, int tid) {
+  for (int idx = tid; idx < R * w / 8; idx += NTHREADS) {
+    const int grp = idx / w, k = idx % w;
+    frag::cp16(smem + (size_t)grp * w * 8 + 8 * k, g + ((size_t)grp * 16 + (c0 >> 3)) * 64 + 8 * k,
+               true);
+  }
+}
+// A contiguous copy of `elems` bf16 (a multiple of 8).
+template <int NTHREADS>
+__device__ __forceinline__ void cp_linear(__nv_bfloat16* smem, const __nv_bfloat16* g, int elems,
+                                          int tid) {
+  for (int idx = tid; idx < elems / 8; idx += NTHREADS) frag::cp16(smem + 8 * idx, g + 8 * idx, true);
+}
 inline size_t saved_bytes(const Problem& p) {
   const size_t nb = (size_t)p.B * p.H * p.NC;
   return nb * (kTBytes + 2 * kBetaBytes + kDecBytes + 4 * kTileBytes + kMBytes + kStateBytes +
@@ -67,6 +124,9 @@ cudaError_t launch_prep(const Problem& p, const __nv_bfloat16* q, const __nv_bfl
 // chunk start states and pseudo-values.
 cudaError_t launch_fwd_scan(const Problem& p, const Saved& sv, const float* S0,
                             __nv_bfloat16* o, float* ST, bool save, cudaStream_t st);
+// The same on tcgen05: MMAs into tensor memory, fp32 state in registers.
+cudaError_t launch_fwd_scan_tc(const Problem& p, const Saved& sv, const float* S0,
+                               __nv_bfloat16* o, float* ST, bool save, cudaStream_t st);
 cudaError_t launch_bwd_scan(const Problem& p, const Saved& sv, const __nv_bfloat16* dO,
                             const float* dST, float* dS0, __nv_bfloat16* dU,
                             __nv_bfloat16* dh, cudaStream_t st);

@@ -30,6 +30,7 @@ namespace {
 constexpr int C = 64, D = 128;
 constexpr int LDD = D + 8;
 constexpr int LDC = C + 8;
+constexpr int CTD = -D, CTC = -C;  // leading dimensions of core-tiled [.][D] / [.][C] tiles
 constexpr int BV = 64;
 constexpr int NTS = 256;
 
@@ -44,11 +45,11 @@ __device__ __forceinline__ int gsw(int i, int c) { return i * D + (c ^ ((i & 7) 
 // ---------------------------------------------------------------------------
 // tc_bwd_scan (thin): streams W, Qh, Kt, M, dec and the dO slice of each chunk
 // through a two-stage cp.async pipeline; only the state-gradient chain runs here.
-struct BscanStage {
-  bf16 W[C * LDD];
-  bf16 Qh[C * LDD];
-  bf16 Kt[C * LDD];
-  bf16 M[C * LDC];
+struct BscanStage {  // W, Qh, Kt, M core-tiled, as saved
+  bf16 W[C * D];
+  bf16 Qh[C * D];
+  bf16 Kt[C * D];
+  bf16 M[C * C];
   bf16 dO[C * LDC];   // dO[:, a0 .. a0+63]
   float dec[D];
 };
@@ -62,17 +63,13 @@ __device__ void bscan_issue(const Problem& p, BscanStage& s, const Saved& sv, co
                             int b, int h, int n, int a0) {
   const int tid = threadIdx.x, t0 = n * C, nvalid = min(C, p.T - t0);
   const size_t cb = chunk_id(p, b, h, n);
-  for (int idx = tid; idx < C * (D / 8); idx += NTS) {
-    const int i = idx >> 4, j = idx & 15;
-    const size_t o = (cb * C + i) * D + j * 8;
-    frag::cp16(s.W + i * LDD + j * 8, sv.W + o, true);
-    frag::cp16(s.Qh + i * LDD + j * 8, sv.Qh + o, true);
-    frag::cp16(s.Kt + i * LDD + j * 8, sv.Kt + o, true);
-  }
+  cp_linear<NTS>(s.W, sv.W + cb * C * D, C * D, tid);
+  cp_linear<NTS>(s.Qh, sv.Qh + cb * C * D, C * D, tid);
+  cp_linear<NTS>(s.Kt, sv.Kt + cb * C * D, C * D, tid);
+  cp_linear<NTS>(s.M, sv.M + cb * C * C, C * C, tid);
   for (int idx = tid; idx < C * (C / 8); idx += NTS) {
     const int i = idx >> 3, j = idx & 7;
     const bool ok = i < nvalid;
-    frag::cp16(s.M + i * LDC + j * 8, sv.M + cb * C * C + i * C + j * 8, true);
     frag::cp16(s.dO + i * LDC + j * 8, dO + row_id(p, b, t0 + (ok ? i : 0), h) * D + a0 + j * 8, ok);
   }
   if (tid < D / 4) frag::cp16(s.dec + tid * 4, sv.dec + cb * D + tid * 4, true);
@@ -119,8 +116,8 @@ __global__ void __launch_bounds__(NTS, 1)
     {
       float du[4][4];
       frag::zero(du);
-      frag::mm_rows_at<4, 4, true>(du, st.M, LDC, rb * 16, st.dO, LDC, hf * 32);
-      frag::mm_rows<4, 8, false>(du, st.Kt, LDD, rb * 16, s.dS, LDD, hf * 32);
+      frag::mm_rows_at<4, 4, true>(du, st.M, CTC, rb * 16, st.dO, LDC, hf * 32);
+      frag::mm_rows<4, 8, false>(du, st.Kt, CTD, rb * 16, s.dS, LDD, hf * 32);
       frag::st_c(du, s.dU, LDC, rb * 16, hf * 32);
     }
     __syncthreads();
@@ -133,9 +130,9 @@ __global__ void __launch_bounds__(NTS, 1)
     {
       float pa[8][4], pb[8][4];
       frag::zero(pa);
-      frag::mm_rows_at<8, 4, true>(pa, st.dO, LDC, rb * 16, st.Qh, LDD, hf * 64);
+      frag::mm_rows_at<8, 4, true>(pa, st.dO, LDC, rb * 16, st.Qh, CTD, hf * 64);
       frag::zero(pb);
-      frag::mm_rows_at<8, 4, true>(pb, s.dU, LDC, rb * 16, st.W, LDD, hf * 64);
+      frag::mm_rows_at<8, 4, true>(pb, s.dU, LDC, rb * 16, st.W, CTD, hf * 64);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
 #pragma unroll
@@ -165,11 +162,11 @@ constexpr int NTB = 512;
 struct BchunkSmem {
   bf16 Qc[C * LDD];     // q e^{gamma - gamma_r}
   bf16 k[C * LDD];      // raw k
-  bf16 W[C * LDD];      // T diag(beta) k e^gamma      [j][c]
-  bf16 Up[C * LDD];     // T diag(beta) v              [j][a]
+  bf16 W[C * D];        // T diag(beta) k e^gamma      [j][c]  core-tiled
+  bf16 Up[C * D];       // T diag(beta) v              [j][a]  core-tiled
   bf16 dO[C * LDD];
   bf16 dU[C * LDD];
-  bf16 U[C * LDD];      // then dA [i][j] (stride LDC)
+  bf16 U[C * D];        // core-tiled; then dA [i][j] (stride LDC)
   bf16 dW[C * LDD];
   bf16 dM[C * LDC];     // tril(dO U^T)               [i][j]
   bf16 T[C * LDC];
@@ -215,11 +212,11 @@ __global__ void __launch_bounds__(NTB, 1)
     frag::cp16(s.Qc + i * LDD + j * 8, q + rr, ok);
     frag::cp16(s.k + i * LDD + j * 8, k + rr, ok);
     frag::cp16(s.dO + i * LDD + j * 8, dO + rr, ok);
-    frag::cp16(s.W + i * LDD + j * 8, Wg + (cb * C + i) * D + j * 8, true);
-    frag::cp16(s.Up + i * LDD + j * 8, Upg + (cb * C + i) * D + j * 8, true);
     frag::cp16(s.dU + i * LDD + j * 8, dUg + (cb * C + i) * D + j * 8, true);
-    frag::cp16(s.U + i * LDD + j * 8, Ug + (cb * C + i) * D + j * 8, true);
   }
+  cp_linear<NTB>(s.W, Wg + cb * C * D, C * D, tid);
+  cp_linear<NTB>(s.Up, Upg + cb * C * D, C * D, tid);
+  cp_linear<NTB>(s.U, Ug + cb * C * D, C * D, tid);
   for (int idx = tid; idx < C * (C / 8); idx += NTB) {
     const int i = idx >> 3, j = idx & 7;
     frag::cp16(s.T + i * LDC + j * 8, Tg + cb * C * C + i * C + j * 8, true);
@@ -331,9 +328,9 @@ __global__ void __launch_bounds__(NTB, 1)
     const bf16* dSh = R1 - ah * 64 * LDD;
     frag::mm_rows<4, 4, true>(zq, s.dO, LDD, rb * 16, Sh, LDD, qt * 32, ah * 64);
     frag::mm_rows<4, 4, true>(adw, s.dU, LDD, rb * 16, Sh, LDD, qt * 32, ah * 64);
-    frag::mm_rows<4, 4, true>(akt, s.U, LDD, rb * 16, dSh, LDD, qt * 32, ah * 64);
+    frag::mm_rows<4, 4, true>(akt, s.U, CTD, rb * 16, dSh, LDD, qt * 32, ah * 64);
     // dM += dO U^T  (U stored [j][a] = [n][k])
-    frag::mm_rows<2, 4, false>(adm, s.dO, LDD, rb * 16, s.U, LDD, qt * 16, ah * 64);
+    frag::mm_rows<2, 4, false>(adm, s.dO, LDD, rb * 16, s.U, CTD, qt * 16, ah * 64);
     // colsum(dS' .* S) over this half: thread -> column c, row quarter rq
     {
       const int c = tid & 127, rq = tid >> 7;
@@ -449,8 +446,8 @@ __global__ void __launch_bounds__(NTB, 1)
   {
     float da[2][4];
     frag::zero(da);
-    frag::mm_rows<2, 8, false>(da, R0, LDD, rb * 16, s.Up, LDD, qt * 16);
-    frag::mm_rows<2, 8, false>(da, R1, LDD, rb * 16, s.W, LDD, qt * 16);
+    frag::mm_rows<2, 8, false>(da, R0, LDD, rb * 16, s.Up, CTD, qt * 16);
+    frag::mm_rows<2, 8, false>(da, R1, LDD, rb * 16, s.W, CTD, qt * 16);
 #pragma unroll
     for (int jt = 0; jt < 2; ++jt)
 #pragma unroll

@@ -71,24 +71,14 @@ __device__ __forceinline__ bf16* slot(TcSmem& s, int kb) {
   return reinterpret_cast<bf16*>(s.arena + kb * 1024);
 }
 
-// cp.async of a row-major [R][Ncol] bf16 global tile into a K-major canonical
-// tile [R x Ncol] (rows = M/N, columns = K).
+// cp.async of a row-major bf16 global tile into a K-major canonical tile
+// [R x Ncol] (rows = M/N, columns = K), or into an MN-major tile [K x N].
 __device__ __forceinline__ void ld_kmaj(bf16* t, const bf16* g, size_t ld, int R, int Ncol,
                                         int valid_rows = 1 << 30) {
-  const int chunks = Ncol / 8;
-  for (int idx = threadIdx.x; idx < R * chunks; idx += NTT) {
-    const int r = idx / chunks, j = idx % chunks;
-    const bool ok = r < valid_rows;
-    frag::cp16(t + tc::kmaj_off(r, 8 * j, Ncol), g + (size_t)(ok ? r : 0) * ld + 8 * j, ok);
-  }
+  tc::cp_core_tile<NTT>(t, g, ld, R, Ncol, valid_rows, threadIdx.x);
 }
-// cp.async of a row-major [K][N] bf16 global tile into an MN-major canonical tile.
 __device__ __forceinline__ void ld_mnmaj(bf16* t, const bf16* g, size_t ld, int K, int N) {
-  const int chunks = N / 8;
-  for (int idx = threadIdx.x; idx < K * chunks; idx += NTT) {
-    const int k = idx / chunks, j = idx % chunks;
-    frag::cp16(t + tc::mnmaj_off(k, 8 * j, N), g + (size_t)k * ld + 8 * j, true);
-  }
+  tc::cp_core_tile<NTT>(t, g, ld, K, N, 1 << 30, threadIdx.x);
 }
 
 __device__ __forceinline__ uint32_t tmem_lane_addr(uint32_t base, int warp, int col) {
@@ -154,7 +144,7 @@ __global__ void __launch_bounds__(NTT, 1)
   const size_t tstride = (size_t)p.H * D;
   ld_kmaj(slot(s, A_DO), dO + tokrow, tstride, C, D, nvalid);
   ld_kmaj(slot(s, A_DU), dUg + cb * C * D, D, C, D);
-  ld_kmaj(slot(s, A_U), sv.U + cb * C * D, D, C, D);
+  cp_linear<NTT>(slot(s, A_U), sv.U + cb * C * D, C * D, tid);
   ld_mnmaj(slot(s, A_SE), sv.h + cb * D * D, D, D, D);
   ld_mnmaj(slot(s, A_DS), dhst + cb * D * D, D, D, D);
   for (int idx = tid; idx < C * (D / 8); idx += NTT) {
@@ -330,8 +320,8 @@ __global__ void __launch_bounds__(NTT, 1)
   // L1/L2 operands and raw q into the freed arena (overlaps the L0 epilogue)
   ld_mnmaj(slot(s, A_TT), sv.T + cb * C * C, C, C, C);
   ld_mnmaj(slot(s, A_DUM), dUg + cb * C * D, D, C, D);
-  ld_kmaj(slot(s, A_UP), sv.Up + cb * C * D, D, C, D);
-  ld_kmaj(slot(s, A_W), sv.W + cb * C * D, D, C, D);
+  cp_linear<NTT>(slot(s, A_UP), sv.Up + cb * C * D, C * D, tid);
+  cp_linear<NTT>(slot(s, A_W), sv.W + cb * C * D, C * D, tid);
   {
     bf16* qraw = slot(s, A_Q);  // row-major [64][LDK]
     for (int idx = tid; idx < C * (D / 8); idx += NTT) {

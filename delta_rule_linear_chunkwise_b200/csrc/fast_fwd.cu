@@ -74,16 +74,18 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
                     frag::pack(f[6], f[7]));
 }
 
-// Row-major bf16 global store of accumulators (rows r0.., cols n0..), 4-byte pairs.
+// bf16 store of accumulators (rows r0.., cols n0..) into a core-tiled global
+// tile with ncol columns, 4-byte pairs: each warp store fills one 8 x 8 block
+// (128 contiguous bytes).
 template <int NTL>
-__device__ __forceinline__ void st_c_global(const float (&c)[NTL][4], bf16* g, int ld, int r0,
+__device__ __forceinline__ void st_c_global(const float (&c)[NTL][4], bf16* g, int ncol, int r0,
                                             int n0) {
   const int l = threadIdx.x & 31;
   const int r = r0 + (l >> 2), cc = n0 + 2 * (l & 3);
 #pragma unroll
   for (int j = 0; j < NTL; ++j) {
-    *reinterpret_cast<uint32_t*>(g + (size_t)r * ld + cc + j * 8) = frag::pack(c[j][0], c[j][1]);
-    *reinterpret_cast<uint32_t*>(g + (size_t)(r + 8) * ld + cc + j * 8) =
+    *reinterpret_cast<uint32_t*>(g + ct_off(r, cc + j * 8, ncol)) = frag::pack(c[j][0], c[j][1]);
+    *reinterpret_cast<uint32_t*>(g + ct_off(r + 8, cc + j * 8, ncol)) =
         frag::pack(c[j][2], c[j][3]);
   }
 }
@@ -171,8 +173,8 @@ __global__ void __launch_bounds__(NT, 2)
     *reinterpret_cast<uint4*>(s.R1 + i * LDD + j * 8) = pack8(kc);
     *reinterpret_cast<uint4*>(s.R2 + i * LDD + j * 8) = pack8(kb);
     *reinterpret_cast<uint4*>(s.R3 + i * LDD + j * 8) = pack8(qc);
-    *reinterpret_cast<uint4*>(sv.Qh + (cb * C + i) * D + j * 8) = pack8(qh);
-    *reinterpret_cast<uint4*>(sv.Kt + (cb * C + i) * D + j * 8) = pack8(kt);
+    *reinterpret_cast<uint4*>(sv.Qh + cb * C * D + ct_off(i, j * 8, D)) = pack8(qh);
+    *reinterpret_cast<uint4*>(sv.Kt + cb * C * D + ct_off(i, j * 8, D)) = pack8(kt);
     nn += __shfl_xor_sync(0xffffffffu, nn, 8);
     nn += __shfl_xor_sync(0xffffffffu, nn, 4);
     nn += __shfl_xor_sync(0xffffffffu, nn, 2);
@@ -311,12 +313,12 @@ __global__ void __launch_bounds__(NT, 2)
 
 // ---------------------------------------------------------------------------
 // tc_fwd_scan
-struct FwdStage {
-  bf16 W[C * LDD];
-  bf16 Qh[C * LDD];
-  bf16 Kt[C * LDD];
-  bf16 M[C * LDC];
-  bf16 Up[C * LDC];   // U'[:, a0 .. a0+63]
+struct FwdStage {  // core-tiled, as saved
+  bf16 W[C * D];
+  bf16 Qh[C * D];
+  bf16 Kt[C * D];
+  bf16 M[C * C];
+  bf16 Up[C * BV];    // U'[:, a0 .. a0+63]
   float dec[D];
 };
 struct FwdSmem {
@@ -329,18 +331,11 @@ __device__ void fwd_issue(const Problem& p, FwdStage& s, const Saved& sv, int b,
                           int a0) {
   const int tid = threadIdx.x;
   const size_t cb = chunk_id(p, b, h, n);
-  for (int idx = tid; idx < C * (D / 8); idx += NT) {
-    const int i = idx >> 4, j = idx & 15;
-    const size_t o = (cb * C + i) * D + j * 8;
-    frag::cp16(s.W + i * LDD + j * 8, sv.W + o, true);
-    frag::cp16(s.Qh + i * LDD + j * 8, sv.Qh + o, true);
-    frag::cp16(s.Kt + i * LDD + j * 8, sv.Kt + o, true);
-  }
-  for (int idx = tid; idx < C * (C / 8); idx += NT) {
-    const int i = idx >> 3, j = idx & 7;
-    frag::cp16(s.M + i * LDC + j * 8, sv.M + cb * C * C + i * C + j * 8, true);
-    frag::cp16(s.Up + i * LDC + j * 8, sv.Up + (cb * C + i) * D + a0 + j * 8, true);
-  }
+  cp_linear<NT>(s.W, sv.W + cb * C * D, C * D, tid);
+  cp_linear<NT>(s.Qh, sv.Qh + cb * C * D, C * D, tid);
+  cp_linear<NT>(s.Kt, sv.Kt + cb * C * D, C * D, tid);
+  cp_linear<NT>(s.M, sv.M + cb * C * C, C * C, tid);
+  cp_ct_cols<NT>(s.Up, sv.Up + cb * C * D, C, a0, BV, tid);
   if (tid < D / 4) frag::cp16(s.dec + tid * 4, sv.dec + cb * D + tid * 4, true);
 }
 
@@ -388,13 +383,13 @@ __global__ void __launch_bounds__(NT, 1)
     {
       frag::zero(u);
       frag::zero(oc);
-      frag::mm_rows2<4, 8, false>(u, oc, st.W, st.Qh, LDD, rb * 16, s.S, LDD, hf * 32);
+      frag::mm_rows2<4, 8, false>(u, oc, st.W, st.Qh, -D, rb * 16, s.S, LDD, hf * 32);
 #pragma unroll
       for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const float2 up = frag::unpack(*reinterpret_cast<const uint32_t*>(
-              st.Up + (rb * 16 + lr + hh * 8) * LDC + hf * 32 + jt * 8 + lc));
+              st.Up + ct_off(rb * 16 + lr + hh * 8, hf * 32 + jt * 8 + lc, BV)));
           u[jt][2 * hh] = up.x - u[jt][2 * hh];
           u[jt][2 * hh + 1] = up.y - u[jt][2 * hh + 1];
         }
@@ -403,12 +398,12 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     if (save)
       for (int idx = tid; idx < C * (BV / 8); idx += NT) {
-        const int i = idx >> 3, j = idx & 7;
-        *reinterpret_cast<uint4*>(sv.U + (cb * C + i) * D + a0 + j * 8) =
+        const int grp = idx / BV, k = idx % BV, i = grp * 8 + (k & 7), j = k >> 3;
+        *reinterpret_cast<uint4*>(sv.U + cb * C * D + ct_off(i, a0 + j * 8, D)) =
             *reinterpret_cast<const uint4*>(s.U + i * LDC + j * 8);
       }
     // O += M U
-    frag::mm_rows<4, 4, true>(oc, st.M, LDC, rb * 16, s.U, LDC, hf * 32);
+    frag::mm_rows<4, 4, true>(oc, st.M, -C, rb * 16, s.U, LDC, hf * 32);
     if (o) {
 #pragma unroll
       for (int jt = 0; jt < 4; ++jt)
@@ -424,7 +419,7 @@ __global__ void __launch_bounds__(NT, 1)
     {
       float ds[8][4];
       frag::zero(ds);
-      frag::mm_rows_at<8, 4, true>(ds, s.U, LDC, rb * 16, st.Kt, LDD, hf * 64);
+      frag::mm_rows_at<8, 4, true>(ds, s.U, LDC, rb * 16, st.Kt, -D, hf * 64);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
 #pragma unroll

@@ -1,0 +1,326 @@
+// fast_scan_tc.cu -- the forward state scan on tcgen05 tensor cores (bf16
+// storage, d_k = d_v = 128, C = 64): one CTA per (b, h, value tile of BV
+// rows of the state), 256 threads, sequential over the chunks of the head.
+//
+// Per chunk n, with the chunk tiles the prep kernel produced (W, q e^gamma,
+// k e^{gamma_C - gamma}, M = tril(Q^c Kb^c^T), U', the chunk decay):
+//   MMA-A  D_A   = [W ; q e^gamma] S_n^T                 (M = 128, N = BV, K = 128)
+//   epilogue 1   U = U' - D_A[0:64]       (bf16 operand tile, saved for the backward)
+//   MMA-B  D_A[64:128] += M U    (A = [0 ; M], so the W rows are left untouched)
+//   MMA-C  D_S   = (k e^{gamma_C - gamma})^T U           (M = 128 keys, N = BV)
+//   epilogue 2   S_{n+1}^T = Diag(e^{gamma_C}) S_n^T + D_S   (fp32, registers)
+// and o_n = D_A[64:128].  The state lives in registers transposed, one key
+// column per TMEM lane, so the per-channel decay is one scalar per thread; the
+// bf16 copy of S^T in shared memory is the MN-major B operand of the next
+// MMA-A.  The chunk-start state h_n and o_{n-1} are written to global memory
+// while MMA-A of chunk n runs.  D_A is double-buffered in tensor memory for
+// that reason.  Chunk tiles stream through a two-stage cp.async pipeline into
+// the canonical no-swizzle core-matrix layouts.
+//
+// This is the affine state transfer of the chunkwise (WY/UT) form:
+//   S_{n+1} = S_n Diag(e^{gamma_C}) + (U' - W S_n^T)^T K~,
+//   O_n     = Q^ S_n^T + (M o L) (U' - W S_n^T).
+
+#include "dr_common.cuh"
+#include "fast.cuh"
+#include "frag.cuh"
+#include "tc.cuh"
+
+namespace dr {
+namespace fast {
+
+using frag::bf16;
+
+namespace {
+
+constexpr int C = 64, D = 128;
+constexpr int NTF = 256;
+constexpr uint32_t kSpinScan = 1u << 22;
+
+template <int BV>
+struct ScanStage {
+  bf16 AWQ[128 * D];   // [W ; q e^gamma], K-major (rows i | 64 + i, K = key c)
+  bf16 KT[C * D];      // k e^{gamma_C - gamma} as the MN-major A of MMA-C ([K = i][M = c])
+  bf16 MZ[128 * C];    // [0 ; M], K-major (K = j); the zero half is written once
+  bf16 UP[C * BV];     // U'[:, a0 .. a0 + BV), core-tiled
+  float dec[D];        // e^{gamma_C} per key column
+};
+
+template <int BV>
+struct ScanSmem {
+  ScanStage<BV> st[2];
+  bf16 SB[D * BV];     // bf16 S^T, MN-major B of MMA-A ([K = c][N = a])
+  bf16 UB[C * BV];     // bf16 U, MN-major B of MMA-B / MMA-C ([K = i][N = a])
+  uint64_t barA, barB;
+  uint32_t tmem;
+};
+
+// The chunk tiles are stored core-tiled in HBM (the layout of the operands
+// here), so each is one contiguous copy; U'[:, a0 .. a0 + BV) is one
+// contiguous run per block of 8 rows.
+template <int BV>
+__device__ __forceinline__ void scan_issue(const Problem& p, ScanStage<BV>& s, const Saved& sv,
+                                           size_t cb, int a0, bool with_o) {
+  const int tid = threadIdx.x;
+  cp_linear<NTF>(s.AWQ, sv.W + cb * C * D, C * D, tid);
+  if (with_o) {
+    cp_linear<NTF>(s.AWQ + C * D, sv.Qh + cb * C * D, C * D, tid);
+    cp_linear<NTF>(s.MZ + C * C, sv.M + cb * C * C, C * C, tid);
+  }
+  cp_linear<NTF>(s.KT, sv.Kt + cb * C * D, C * D, tid);
+  cp_ct_cols<NTF>(s.UP, sv.Up + cb * C * D, C, a0, BV, tid);
+  if (tid < D / 4) frag::cp16(s.dec + 4 * tid, sv.dec + cb * D + 4 * tid, true);
+}
+
+__device__ __forceinline__ uint32_t lane_addr(uint32_t base, int warp, int col) {
+  return base + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)col;
+}
+
+// Bounded wait on an mbarrier phase; the result is uniform over the CTA.
+__device__ __forceinline__ bool cta_wait(uint64_t* bar, int parity) {
+  const bool ok = tc::mbar_wait(bar, (uint32_t)(parity & 1), kSpinScan);
+  const int bad = __syncthreads_or(ok ? 0 : 1);
+  tc::fence_after_sync();
+  return bad == 0;
+}
+
+template <int BV>
+__global__ void __launch_bounds__(NTF, 1)
+    k_fwd_scan_tc(Problem p, Saved sv, const float* __restrict__ S0, bf16* __restrict__ o,
+                  float* __restrict__ ST, int save, int* __restrict__ err) {
+  constexpr int HB = BV / 2;             // value columns per thread in the state epilogue
+  constexpr int TCOLS = 3 * BV;          // tensor memory columns: D_A x 2, D_S
+  constexpr int TALLOC = TCOLS <= 256 ? 256 : 512;
+  extern __shared__ __align__(1024) unsigned char smraw[];
+  ScanSmem<BV>& s = *reinterpret_cast<ScanSmem<BV>*>(smraw);
+  const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int a0 = blockIdx.x * BV;
+  const bool with_o = o != nullptr;
+  const size_t sbase = ((size_t)b * p.H + h) * D * D;
+  // state epilogue ownership: key column c (= TMEM lane), value columns ah*HB ..
+  const int c = 32 * (warp & 3) + lane, ah = warp >> 2;
+  const uint32_t T_S = 2 * BV;  // D_A buffers at columns 0 and BV
+
+  if (warp == 0) tc::tmem_alloc(&s.tmem, TALLOC);
+  if (tid == 0) {
+    tc::mbar_init(&s.barA, 1);
+    tc::mbar_init(&s.barB, 1);
+  }
+  // zero halves of [0 ; M] in both stages
+  for (int idx = tid; idx < 2 * C * C / 8; idx += NTF) {
+    const int stg = idx / (C * C / 8), e = idx % (C * C / 8);
+    *reinterpret_cast<uint4*>(s.st[stg].MZ + 8 * e) = make_uint4(0, 0, 0, 0);
+  }
+  // fp32 state S^T[c][a0 + ah*HB + u]
+  float S[HB];
+#pragma unroll
+  for (int u = 0; u < HB; ++u)
+    S[u] = S0 ? S0[sbase + (size_t)(a0 + ah * HB + u) * D + c] : 0.f;
+
+  auto write_sb = [&]() {
+#pragma unroll
+    for (int u8 = 0; u8 < HB / 8; ++u8) {
+      float f[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = S[8 * u8 + e];
+      *reinterpret_cast<uint4*>(s.SB + tc::mnmaj_off(c, ah * HB + 8 * u8, BV)) =
+          make_uint4(frag::pack(f[0], f[1]), frag::pack(f[2], f[3]), frag::pack(f[4], f[5]),
+                     frag::pack(f[6], f[7]));
+    }
+  };
+  // h_n[a][c] (bf16) from the registers: lanes c, c + 1 swap so each stores a pair
+  auto store_h = [&](size_t cbn) {
+    bf16* hp = sv.h + cbn * D * D;
+#pragma unroll
+    for (int u = 0; u < HB; u += 2) {
+      const float x = (lane & 1) ? S[u] : S[u + 1];
+      const float y = __shfl_xor_sync(0xffffffffu, x, 1);
+      const int a = a0 + ah * HB + u + (lane & 1);
+      const int cc = c & ~1;
+      const uint32_t v = (lane & 1) ? frag::pack(y, S[u + 1]) : frag::pack(S[u], y);
+      *reinterpret_cast<uint32_t*>(hp + (size_t)a * D + cc) = v;
+    }
+  };
+  // o rows of chunk nn from D_A buffer `buf` (warps on lanes 64 .. 127)
+  auto store_o = [&](int nn, int buf) {
+    if ((warp & 3) < 2) return;
+    const int i = 32 * ((warp & 3) - 2) + lane;
+    const int t0 = nn * C, nvalid = min(C, p.T - t0);
+    uint32_t r[HB];
+#pragma unroll
+    for (int q16 = 0; q16 < HB / 16; ++q16)
+      tc::tmem_ld16_nowait(lane_addr(s.tmem, warp, buf * BV + ah * HB + 16 * q16), r + 16 * q16);
+    tc::tmem_wait_ld();
+    if (i < nvalid) {
+      bf16* op = o + row_id(p, b, t0 + i, h) * D + a0 + ah * HB;
+#pragma unroll
+      for (int e8 = 0; e8 < HB / 8; ++e8) {
+        const float* f = reinterpret_cast<const float*>(r + 8 * e8);
+        *reinterpret_cast<uint4*>(op + 8 * e8) =
+            make_uint4(frag::pack(f[0], f[1]), frag::pack(f[2], f[3]), frag::pack(f[4], f[5]),
+                       frag::pack(f[6], f[7]));
+      }
+    }
+  };
+
+  write_sb();
+  scan_issue<BV>(p, s.st[0], sv, chunk_id(p, b, h, 0), a0, with_o);
+  frag::cp_commit();
+  if (p.NC > 1) scan_issue<BV>(p, s.st[1], sv, chunk_id(p, b, h, 1), a0, with_o);
+  frag::cp_commit();
+  frag::cp_wait<1>();
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = s.tmem;
+
+  bool ok = true;
+  const uint32_t idA = tc::idesc_bf16(128, BV, false, true);
+  const uint32_t idC = tc::idesc_bf16(128, BV, true, true);
+  // descriptors: per-k-step advance of the start address (in 16-byte units)
+  const uint64_t dSB = tc::sdesc_mnmaj(s.SB, BV, 0), dUB = tc::sdesc_mnmaj(s.UB, BV, 0);
+  constexpr uint32_t kSB = 2 * (BV / 8) * 128 / 16, kUB = kSB, kKM = 256 / 16;
+  constexpr uint32_t kKT = 2 * (D / 8) * 128 / 16;
+  for (int n = 0; n < p.NC && ok; ++n) {
+    const size_t cb = chunk_id(p, b, h, n);
+    ScanStage<BV>& st = s.st[n & 1];
+    const int buf = n & 1;
+    const float dc = st.dec[c];  // read before the stage is refilled below
+    // MMA-A: [W ; q e^gamma] S^T
+    if (tid == 0) {
+      const uint64_t dA = tc::sdesc_kmaj(st.AWQ, D, 0);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        tc::mma(tbase + buf * BV, dA + ks * kKM, dSB + ks * kSB, idA, ks > 0 ? 1u : 0u);
+      tc::commit(&s.barA);
+    }
+    // while it runs: the previous chunk's output
+    if (with_o && n > 0) store_o(n - 1, buf ^ 1);
+    ok = cta_wait(&s.barA, n);
+    if (!ok) break;
+    // epilogue 1: U = U' - W S^T (rows i = lanes 0 .. 63)
+    uint4 usave[HB / 8];
+    if ((warp & 3) < 2) {
+      const int i = c;  // lanes 0 .. 63
+      uint32_t r[HB];
+#pragma unroll
+      for (int q16 = 0; q16 < HB / 16; ++q16)
+        tc::tmem_ld16_nowait(lane_addr(tbase, warp, buf * BV + ah * HB + 16 * q16), r + 16 * q16);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int e8 = 0; e8 < HB / 8; ++e8) {
+        const int a = ah * HB + 8 * e8;
+        const uint4 u8 = *reinterpret_cast<const uint4*>(st.UP + ct_off(i, a, BV));
+        const uint32_t* w8 = reinterpret_cast<const uint32_t*>(&u8);
+        const float* f = reinterpret_cast<const float*>(r + 8 * e8);
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 x = frag::unpack(w8[e]);
+          pk[e] = frag::pack(x.x - f[2 * e], x.y - f[2 * e + 1]);
+        }
+        usave[e8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(s.UB + tc::mnmaj_off(i, a, BV)) = usave[e8];
+      }
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    // MMA-B (output) and MMA-C (state increment)
+    if (tid == 0) {
+      if (with_o) {
+        const uint64_t dM = tc::sdesc_kmaj(st.MZ, C, 0);
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks)
+          tc::mma(tbase + buf * BV, dM + ks * kKM, dUB + ks * kUB, idA, 1u);
+      }
+      const uint64_t dK = tc::sdesc_mnmaj(st.KT, D, 0);
+#pragma unroll
+      for (int ks = 0; ks < C / 16; ++ks)
+        tc::mma(tbase + T_S, dK + ks * kKT, dUB + ks * kUB, idC, ks > 0 ? 1u : 0u);
+      tc::commit(&s.barB);
+    }
+    // while they run: U and the chunk-start state to global memory
+    if (save) {
+      if ((warp & 3) < 2) {
+        bf16* up = sv.U + cb * C * D;
+#pragma unroll
+        for (int e8 = 0; e8 < HB / 8; ++e8)
+          *reinterpret_cast<uint4*>(up + ct_off(c, a0 + ah * HB + 8 * e8, D)) = usave[e8];
+      }
+      store_h(cb);
+    }
+    ok = cta_wait(&s.barB, n);
+    if (!ok) break;
+    // this stage is consumed: refill it with chunk n + 2 (lands during the next step)
+    if (n + 2 < p.NC) scan_issue<BV>(p, st, sv, chunk_id(p, b, h, n + 2), a0, with_o);
+    frag::cp_commit();
+    // epilogue 2: S^T <- Diag(e^{gamma_C}) S^T + D_S
+    {
+      uint32_t r[HB];
+#pragma unroll
+      for (int q16 = 0; q16 < HB / 16; ++q16)
+        tc::tmem_ld16_nowait(lane_addr(tbase, warp, T_S + ah * HB + 16 * q16), r + 16 * q16);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < HB; ++e) S[e] = S[e] * dc + __uint_as_float(r[e]);
+      write_sb();
+    }
+    frag::cp_wait<1>();
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+  }
+  if (ok) {
+    if (with_o) store_o(p.NC - 1, (p.NC - 1) & 1);
+    if (ST) {
+#pragma unroll
+      for (int u = 0; u < HB; ++u) ST[sbase + (size_t)(a0 + ah * HB + u) * D + c] = S[u];
+    }
+  } else if (tid == 0 && err) {
+    atomicExch(err, 1);
+  }
+  frag::cp_wait<0>();
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tbase, TALLOC);
+}
+
+template <int BV>
+cudaError_t launch_fwd_scan_tc_bv(const Problem& p, const Saved& sv, const float* S0, bf16* o,
+                                  float* ST, bool save, cudaStream_t st) {
+  const size_t sm = sizeof(ScanSmem<BV>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(k_fwd_scan_tc<BV>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  const double nb = (double)p.B * p.H * p.NC, ntok = nb * C, heads = (double)p.B * p.H;
+  // reads W, Kt, U', dec (+ q e^gamma, M with the output); writes h, U (saving), o
+  double bytes = nb * (2.0 * kTileBytes + kTileBytes + kDecBytes);
+  if (o) bytes += nb * ((double)kTileBytes + kMBytes) + ntok * D * 2;
+  if (save) bytes += nb * ((double)kStateBytes + kUBytes);
+  bytes += heads * D * D * 4 * ((S0 ? 1 : 0) + (ST ? 1 : 0));
+  const double flops = nb * (2.0 * C * D * D * (o ? 3 : 2) + (o ? 2.0 * C * C * D : 0.0));
+  prof_begin(kKTcScanFwd, bytes, flops, st);
+  k_fwd_scan_tc<BV><<<dim3(D / BV, p.H, p.B), NTF, sm, st>>>(p, sv, S0, o, ST, save ? 1 : 0,
+                                                             device_error_word());
+  e = cudaGetLastError();
+  prof_end(st);
+  return e;
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_scan_tc(const Problem& p, const Saved& sv, const float* S0, bf16* o,
+                               float* ST, bool save, cudaStream_t st) {
+  // One CTA per (b, h, value tile): 64-row tiles while two per head still fit one wave
+  // of the 148 SMs, whole-state tiles otherwise.
+  if ((long)p.B * p.H * 2 <= 148) return launch_fwd_scan_tc_bv<64>(p, sv, S0, o, ST, save, st);
+  return launch_fwd_scan_tc_bv<128>(p, sv, S0, o, ST, save, st);
+}
+
+}  // namespace fast
+}  // namespace dr

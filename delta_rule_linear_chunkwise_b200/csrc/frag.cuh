@@ -42,26 +42,36 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t* r, const bf16* p) {
                : "memory");
 }
 
+// Element (r, c) of a shared tile with leading dimension ld: row-major with
+// row stride ld when ld > 0; when ld < 0, core-tiled with -ld columns (8 x 8
+// blocks of 128 contiguous bytes, row-block-major), the layout the tcgen05
+// operands and the saved chunk tiles use.  ldmatrix reads one such block per
+// 8 x 8 matrix, so the core-tiled form needs no padding against bank
+// conflicts.  c is a multiple of 8 wherever 16 contiguous bytes are addressed.
+__device__ __forceinline__ int toff(int r, int c, int ld) {
+  return ld > 0 ? r * ld + c : (((r >> 3) * ((-ld) >> 3) + (c >> 3)) * 64 + (r & 7) * 8 + (c & 7));
+}
+
 // A fragment of rows r0..r0+15, cols k0..k0+15 of a row-major tile.
 __device__ __forceinline__ void ld_a(uint32_t* a, const bf16* t, int ld, int r0, int k0) {
   const int l = threadIdx.x & 31;
-  ldsm_x4(a, t + (r0 + (l & 7) + ((l >> 3) & 1) * 8) * ld + k0 + (l >> 4) * 8);
+  ldsm_x4(a, t + toff(r0 + (l & 7) + ((l >> 3) & 1) * 8, k0 + (l >> 4) * 8, ld));
 }
 // A fragment of X^T (rows m0.., cols k0..) where X is stored row-major [k][m].
 __device__ __forceinline__ void ld_at(uint32_t* a, const bf16* x, int ld, int m0, int k0) {
   const int l = threadIdx.x & 31;
-  ldsm_x4_t(a, x + (k0 + (l & 7) + (l >> 4) * 8) * ld + m0 + ((l >> 3) & 1) * 8);
+  ldsm_x4_t(a, x + toff(k0 + (l & 7) + (l >> 4) * 8, m0 + ((l >> 3) & 1) * 8, ld));
 }
 // B fragments of two n-tiles (n0, n0+8), k0..k0+15, B stored as [n][k].
 // b[0..1] -> n-tile n0, b[2..3] -> n-tile n0+8.
 __device__ __forceinline__ void ld_b_nk(uint32_t* b, const bf16* t, int ld, int n0, int k0) {
   const int l = threadIdx.x & 31;
-  ldsm_x4(b, t + (n0 + (l & 7) + (l >> 4) * 8) * ld + k0 + ((l >> 3) & 1) * 8);
+  ldsm_x4(b, t + toff(n0 + (l & 7) + (l >> 4) * 8, k0 + ((l >> 3) & 1) * 8, ld));
 }
 // B fragments of two n-tiles, B stored as [k][n] (n contiguous).
 __device__ __forceinline__ void ld_b_kn(uint32_t* b, const bf16* t, int ld, int k0, int n0) {
   const int l = threadIdx.x & 31;
-  ldsm_x4_t(b, t + (k0 + (l & 7) + ((l >> 3) & 1) * 8) * ld + n0 + (l >> 4) * 8);
+  ldsm_x4_t(b, t + toff(k0 + (l & 7) + ((l >> 3) & 1) * 8, n0 + (l >> 4) * 8, ld));
 }
 
 // A fragment for k-step ks from accumulators of n-tiles 2ks, 2ks+1.
@@ -169,8 +179,8 @@ __device__ __forceinline__ void st_c(const float (&c)[NT][4], bf16* t, int ld, i
   const int r = r0 + (l >> 2), cc = n0 + 2 * (l & 3);
 #pragma unroll
   for (int j = 0; j < NT; ++j) {
-    *reinterpret_cast<uint32_t*>(t + r * ld + cc + j * 8) = pack(c[j][0], c[j][1]);
-    *reinterpret_cast<uint32_t*>(t + (r + 8) * ld + cc + j * 8) = pack(c[j][2], c[j][3]);
+    *reinterpret_cast<uint32_t*>(t + toff(r, cc + j * 8, ld)) = pack(c[j][0], c[j][1]);
+    *reinterpret_cast<uint32_t*>(t + toff(r + 8, cc + j * 8, ld)) = pack(c[j][2], c[j][3]);
   }
 }
 

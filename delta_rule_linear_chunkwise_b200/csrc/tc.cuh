@@ -28,6 +28,30 @@ __device__ __forceinline__ int mnmaj_off(int k, int n, int N) {
   return ((k >> 3) * (N >> 3) + (n >> 3)) * 64 + (k & 7) * 8 + (n & 7);  // in bf16 elements
 }
 
+// cp.async of a row-major [R][NCOL] bf16 global tile (row stride ld elements)
+// into the core-matrix layout above (K-major [R x K=NCOL], or MN-major
+// [K=R x N=NCOL]: both place element (r, c) at ((r/8)*(NCOL/8) + c/8)*64 +
+// (r%8)*8 + c%8).  16-byte chunk idx goes to shared offset 16*idx, so eight
+// consecutive lanes fill one core matrix (128 contiguous bytes, no bank
+// conflicts) while a warp reads 8 rows x 64 contiguous bytes of the source.
+// Rows at or beyond valid_rows are zero-filled.
+template <int NTHREADS>
+__device__ __forceinline__ void cp_core_tile(__nv_bfloat16* tile, const __nv_bfloat16* g,
+                                             size_t ld, int R, int NCOL, int valid_rows,
+                                             int tid) {
+  const int cpr = NCOL >> 3;  // core matrices per row group
+  for (int idx = tid; idx < R * cpr; idx += NTHREADS) {
+    const int core = idx >> 3, rr = idx & 7;
+    const int r = (core / cpr) * 8 + rr, c = (core % cpr) * 8;
+    const bool ok = r < valid_rows;
+    const __nv_bfloat16* src = g + (size_t)(ok ? r : 0) * ld + c;
+    const uint32_t dst = smem_u32(tile + 8 * idx);
+    const int n = ok ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n)
+                 : "memory");
+  }
+}
+
 // Shared-memory matrix descriptor (sm100 format, no swizzle).
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = 0;
@@ -123,6 +147,21 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// The same without the wait: issue several, then tmem_wait_ld() once before
+// the registers are read.
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
 // --- legacy warp-level MMA (m16n8k16, bf16 in, fp32 accumulate) ----------

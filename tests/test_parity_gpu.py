@@ -135,9 +135,17 @@ def bwd_variant(request, monkeypatch):
     return request.param
 
 
+# The forward scan likewise: tcgen05 (default) and warp-level mma.sync
+# (DR_MMA_SYNC_SCAN=1).
+@pytest.fixture(params=["tcgen05", "mma_sync"])
+def scan_variant(request, monkeypatch):
+    monkeypatch.setenv("DR_MMA_SYNC_SCAN", "1" if request.param == "mma_sync" else "0")
+    return request.param
+
+
 @pytest.mark.parametrize("T", [1, 63, 64, 65, 129])
 @pytest.mark.parametrize("gate", ["none", "scalar", "channel"])
-def test_tensor_core_path_ragged(T, gate, bwd_variant):
+def test_tensor_core_path_ragged(T, gate, bwd_variant, scan_variant):
     w = WORKLOADS["kda_bf16_b4h16t8192"].with_(name=f"tc_T{T}_{gate}", B=1, H=2, T=T,
                                                gate=gate, s0_std=0.1)
     _check(w, make_inputs(w), dST=random_state(w, seed=11, std=0.5))
@@ -155,3 +163,20 @@ def test_tcgen05_backward_full_size_sampled_heads(monkeypatch):
     monkeypatch.setenv("DR_TCGEN05_BWD", "1")
     w = WORKLOADS["kda_bf16_b4h16t8192"]
     _check(w, make_inputs(w), heads=[(0, 0), (w.B - 1, w.H - 1)])
+
+
+@pytest.mark.parametrize("w", SMALL[1:5], ids=lambda w: w.name)
+def test_mma_sync_scan_small_workloads(w, monkeypatch):
+    monkeypatch.setenv("DR_MMA_SYNC_SCAN", "1")
+    inp = make_inputs(w)
+    _check(w, inp, dST=random_state(w, seed=99, std=0.5))
+    _check(w, inp, save=False)
+
+
+def test_whole_state_scan_tiles():
+    """More than 74 heads: the forward scan takes the whole 128-row state per
+    CTA instead of two 64-row value tiles."""
+    w = WORKLOADS["kda_bf16_b4h16t8192"].with_(name="many_heads", B=8, H=10, T=100,
+                                               s0_std=0.1)
+    _check(w, make_inputs(w), dST=random_state(w, seed=12, std=0.5),
+           heads=[(0, 0), (3, 7), (7, 9)])
