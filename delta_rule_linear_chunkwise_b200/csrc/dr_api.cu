@@ -124,13 +124,22 @@ bool use_tcgen05_chunk_bwd() {
   return e && e[0] == '1';
 }
 
-// The forward state scan likewise: tcgen05 with the state in registers and the
+// The two state scans likewise: tcgen05 with the state in registers and the
 // products in TMEM (default), or warp-level mma.sync tiles (DR_MMA_SYNC_SCAN=1).
+bool use_mma_sync_scans() {
+  const char* e = getenv("DR_MMA_SYNC_SCAN");
+  return e && e[0] == '1';
+}
 cudaError_t fwd_scan(const dr::Problem& P, const dr::fast::Saved& sv, const float* S0,
                      __nv_bfloat16* o, float* ST, bool save, cudaStream_t st) {
-  const char* e = getenv("DR_MMA_SYNC_SCAN");
-  if (e && e[0] == '1') return dr::fast::launch_fwd_scan(P, sv, S0, o, ST, save, st);
+  if (use_mma_sync_scans()) return dr::fast::launch_fwd_scan(P, sv, S0, o, ST, save, st);
   return dr::fast::launch_fwd_scan_tc(P, sv, S0, o, ST, save, st);
+}
+cudaError_t bwd_scan(const dr::Problem& P, const dr::fast::Saved& sv, const __nv_bfloat16* dO,
+                     const float* dST, float* dS0, __nv_bfloat16* dU, __nv_bfloat16* dh,
+                     cudaStream_t st) {
+  if (use_mma_sync_scans()) return dr::fast::launch_bwd_scan(P, sv, dO, dST, dS0, dU, dh, st);
+  return dr::fast::launch_bwd_scan_tc(P, sv, dO, dST, dS0, dU, dh, st);
 }
 
 size_t saved_bytes(const Problem& p) {
@@ -236,7 +245,7 @@ dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const 
     const size_t nb = (size_t)P.B * P.H * P.NC;
     bf* dU = (bf*)wsb;
     bf* dh = (bf*)(wsb + round_up(nb * dr::fast::kUBytes));
-    e = dr::fast::launch_bwd_scan(P, sv, (const bf*)dO, dST, dS0, dU, dh, st);
+    e = bwd_scan(P, sv, (const bf*)dO, dST, dS0, dU, dh, st);
     if (e == cudaSuccess)
       e = use_tcgen05_chunk_bwd()
               ? dr::fast::launch_bwd_chunk_tc(P, (const bf*)q, (const bf*)k, (const bf*)v,

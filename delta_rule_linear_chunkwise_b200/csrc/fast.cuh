@@ -127,6 +127,9 @@ cudaError_t launch_fwd_scan(const Problem& p, const Saved& sv, const float* S0,
 // The same on tcgen05: MMAs into tensor memory, fp32 state in registers.
 cudaError_t launch_fwd_scan_tc(const Problem& p, const Saved& sv, const float* S0,
                                __nv_bfloat16* o, float* ST, bool save, cudaStream_t st);
+cudaError_t launch_bwd_scan_tc(const Problem& p, const Saved& sv, const __nv_bfloat16* dO,
+                               const float* dST, float* dS0, __nv_bfloat16* dU,
+                               __nv_bfloat16* dh, cudaStream_t st);
 cudaError_t launch_bwd_scan(const Problem& p, const Saved& sv, const __nv_bfloat16* dO,
                             const float* dST, float* dS0, __nv_bfloat16* dU,
                             __nv_bfloat16* dh, cudaStream_t st);

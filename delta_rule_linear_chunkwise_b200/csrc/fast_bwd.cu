@@ -122,8 +122,8 @@ __global__ void __launch_bounds__(NTS, 1)
     }
     __syncthreads();
     for (int idx = tid; idx < C * (BV / 8); idx += NTS) {
-      const int i = idx >> 3, j = idx & 7;
-      *reinterpret_cast<uint4*>(dUout + (cb * C + i) * D + a0 + j * 8) =
+      const int grp = idx / BV, k = idx % BV, i = grp * 8 + (k & 7), j = k >> 3;
+      *reinterpret_cast<uint4*>(dUout + cb * C * D + ct_off(i, a0 + j * 8, D)) =
           *reinterpret_cast<const uint4*>(s.dU + i * LDC + j * 8);
     }
     // dS <- dS Diag(dec) + dO^T Qh - dU^T W, rows a = 16rb.., keys 64hf..
@@ -165,7 +165,7 @@ struct BchunkSmem {
   bf16 W[C * D];        // T diag(beta) k e^gamma      [j][c]  core-tiled
   bf16 Up[C * D];       // T diag(beta) v              [j][a]  core-tiled
   bf16 dO[C * LDD];
-  bf16 dU[C * LDD];
+  bf16 dU[C * D];       // core-tiled
   bf16 U[C * D];        // core-tiled; then dA [i][j] (stride LDC)
   bf16 dW[C * LDD];
   bf16 dM[C * LDC];     // tril(dO U^T)               [i][j]
@@ -212,8 +212,8 @@ __global__ void __launch_bounds__(NTB, 1)
     frag::cp16(s.Qc + i * LDD + j * 8, q + rr, ok);
     frag::cp16(s.k + i * LDD + j * 8, k + rr, ok);
     frag::cp16(s.dO + i * LDD + j * 8, dO + rr, ok);
-    frag::cp16(s.dU + i * LDD + j * 8, dUg + (cb * C + i) * D + j * 8, true);
   }
+  cp_linear<NTB>(s.dU, dUg + cb * C * D, C * D, tid);
   cp_linear<NTB>(s.W, Wg + cb * C * D, C * D, tid);
   cp_linear<NTB>(s.Up, Upg + cb * C * D, C * D, tid);
   cp_linear<NTB>(s.U, Ug + cb * C * D, C * D, tid);
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(NTB, 1)
     const bf16* Sh = R0 - ah * 64 * LDD;
     const bf16* dSh = R1 - ah * 64 * LDD;
     frag::mm_rows<4, 4, true>(zq, s.dO, LDD, rb * 16, Sh, LDD, qt * 32, ah * 64);
-    frag::mm_rows<4, 4, true>(adw, s.dU, LDD, rb * 16, Sh, LDD, qt * 32, ah * 64);
+    frag::mm_rows<4, 4, true>(adw, s.dU, CTD, rb * 16, Sh, LDD, qt * 32, ah * 64);
     frag::mm_rows<4, 4, true>(akt, s.U, CTD, rb * 16, dSh, LDD, qt * 32, ah * 64);
     // dM += dO U^T  (U stored [j][a] = [n][k])
     frag::mm_rows<2, 4, false>(adm, s.dO, LDD, rb * 16, s.U, CTD, qt * 16, ah * 64);
@@ -414,7 +414,7 @@ __global__ void __launch_bounds__(NTB, 1)
         vv[jt][hh] = *reinterpret_cast<const uint32_t*>(v + rowg[hh] + qt * 32 + jt * 8 + lc);
     float lu[4][4];
     frag::zero(lu);
-    frag::mm_rows_at<4, 4, true>(lu, s.T, LDC, rb * 16, s.dU, LDD, qt * 32);
+    frag::mm_rows_at<4, 4, true>(lu, s.T, LDC, rb * 16, s.dU, CTD, qt * 32);
 #pragma unroll
     for (int jt = 0; jt < 4; ++jt)
 #pragma unroll

@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(NTT, 1)
   const size_t tokrow = row_id(p, b, t0, h) * D;  // row stride H * D
   const size_t tstride = (size_t)p.H * D;
   ld_kmaj(slot(s, A_DO), dO + tokrow, tstride, C, D, nvalid);
-  ld_kmaj(slot(s, A_DU), dUg + cb * C * D, D, C, D);
+  cp_linear<NTT>(slot(s, A_DU), dUg + cb * C * D, C * D, tid);
   cp_linear<NTT>(slot(s, A_U), sv.U + cb * C * D, C * D, tid);
   ld_mnmaj(slot(s, A_SE), sv.h + cb * D * D, D, D, D);
   ld_mnmaj(slot(s, A_DS), dhst + cb * D * D, D, D, D);
@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(NTT, 1)
   if (!ok) goto fail;
   // L1/L2 operands and raw q into the freed arena (overlaps the L0 epilogue)
   ld_mnmaj(slot(s, A_TT), sv.T + cb * C * C, C, C, C);
-  ld_mnmaj(slot(s, A_DUM), dUg + cb * C * D, D, C, D);
+  cp_linear<NTT>(slot(s, A_DUM), dUg + cb * C * D, C * D, tid);
   cp_linear<NTT>(slot(s, A_UP), sv.Up + cb * C * D, C * D, tid);
   cp_linear<NTT>(slot(s, A_W), sv.W + cb * C * D, C * D, tid);
   {

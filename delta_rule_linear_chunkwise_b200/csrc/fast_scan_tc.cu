@@ -312,6 +312,239 @@ cudaError_t launch_fwd_scan_tc_bv(const Problem& p, const Saved& sv, const float
   return e;
 }
 
+// ---------------------------------------------------------------------------
+// The reverse state-gradient scan on tcgen05.  Per chunk n, from the last to
+// the first, with dS = dS_{n+1} (the gradient of the chunk's end state):
+//   MMA-1  D_U  = M^T dO + (k e^{gamma_C - gamma}) dS^T     (M = 64, N = BV)
+//   MMA-2a D_S  = (q e^gamma)^T dO                           (M = 128 keys)
+//   epilogue 1   dU = D_U (bf16, saved for the chunk kernel; -dU is the operand)
+//   MMA-2b D_S += W^T (-dU)
+//   epilogue 2   dS_n^T = Diag(e^{gamma_C}) dS^T + D_S       (fp32, registers)
+// dh_n = dS_{n+1} is written out (bf16) while MMA-1 runs.  Each CTA owns the
+// value columns a0 .. a0 + BV of dS; the state gradient is held transposed,
+// one key per TMEM lane.
+template <int BV>
+struct BScanStage {
+  bf16 QH[C * D];     // q e^gamma, core-tiled [j][c]: MN-major A (M = key c, K = j)
+  bf16 KT[C * D];     // k e^{gamma_C - gamma}, core-tiled [i][c]: K-major A (M = i, K = c)
+  bf16 W[C * D];      // W, core-tiled [i][c]: MN-major A (M = key c, K = i)
+  bf16 M[C * C];      // M, core-tiled [j][i]: MN-major A of M^T (M = i, K = j)
+  bf16 DO[C * BV];    // dO[:, a0 .. a0 + BV), core-tiled [j][a]: MN-major B
+  float dec[D];
+};
+template <int BV>
+struct BScanSmem {
+  BScanStage<BV> st[2];
+  bf16 DSB[D * BV];   // bf16 dS^T, core-tiled [c][a]: MN-major B of MMA-1
+  bf16 DUB[C * BV];   // bf16 -dU, core-tiled [i][a]: MN-major B of MMA-2b
+  uint64_t barA, barB;
+  uint32_t tmem;
+};
+
+template <int BV>
+__device__ __forceinline__ void bscan_issue_tc(const Problem& p, BScanStage<BV>& s, const Saved& sv,
+                                               const bf16* __restrict__ dO, int b, int h, int n,
+                                               int a0) {
+  const int tid = threadIdx.x;
+  const size_t cb = chunk_id(p, b, h, n);
+  const int t0 = n * C, nvalid = min(C, p.T - t0);
+  cp_linear<NTF>(s.QH, sv.Qh + cb * C * D, C * D, tid);
+  cp_linear<NTF>(s.KT, sv.Kt + cb * C * D, C * D, tid);
+  cp_linear<NTF>(s.W, sv.W + cb * C * D, C * D, tid);
+  cp_linear<NTF>(s.M, sv.M + cb * C * C, C * C, tid);
+  for (int idx = tid; idx < C * BV / 8; idx += NTF) {
+    const int j = ct_row(idx, BV), col = ct_col(idx, BV);
+    const bool ok = j < nvalid;
+    frag::cp16(s.DO + 8 * idx, dO + row_id(p, b, t0 + (ok ? j : 0), h) * D + a0 + col, ok);
+  }
+  if (tid < D / 4) frag::cp16(s.dec + 4 * tid, sv.dec + cb * D + 4 * tid, true);
+}
+
+template <int BV>
+__global__ void __launch_bounds__(NTF, 1)
+    k_bwd_scan_tc(Problem p, Saved sv, const bf16* __restrict__ dO, const float* __restrict__ dST,
+                  float* __restrict__ dS0, bf16* __restrict__ dUout, bf16* __restrict__ dhout,
+                  int* __restrict__ err) {
+  constexpr int HB = BV / 2;
+  constexpr int TALLOC = 2 * BV <= 128 ? 128 : 256;
+  extern __shared__ __align__(1024) unsigned char smraw[];
+  BScanSmem<BV>& s = *reinterpret_cast<BScanSmem<BV>*>(smraw);
+  const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int a0 = blockIdx.x * BV;
+  const size_t sbase = ((size_t)b * p.H + h) * D * D;
+  const int c = 32 * (warp & 3) + lane, ah = warp >> 2;  // key (TMEM lane), value half
+  const uint32_t T_U = 0, T_S = BV;
+
+  if (warp == 0) tc::tmem_alloc(&s.tmem, TALLOC);
+  if (tid == 0) {
+    tc::mbar_init(&s.barA, 1);
+    tc::mbar_init(&s.barB, 1);
+  }
+  float dS[HB];  // dS^T[c][a0 + ah*HB + u]
+#pragma unroll
+  for (int u = 0; u < HB; ++u)
+    dS[u] = dST ? dST[sbase + (size_t)(a0 + ah * HB + u) * D + c] : 0.f;
+  auto write_dsb = [&]() {
+#pragma unroll
+    for (int u8 = 0; u8 < HB / 8; ++u8) {
+      const float* f = dS + 8 * u8;
+      *reinterpret_cast<uint4*>(s.DSB + tc::mnmaj_off(c, ah * HB + 8 * u8, BV)) =
+          make_uint4(frag::pack(f[0], f[1]), frag::pack(f[2], f[3]), frag::pack(f[4], f[5]),
+                     frag::pack(f[6], f[7]));
+    }
+  };
+  // dh (bf16, [a][c]) from the registers: lanes c, c + 1 swap so each stores a pair
+  auto store_dh = [&](size_t cbn) {
+    bf16* hp = dhout + cbn * D * D;
+#pragma unroll
+    for (int u = 0; u < HB; u += 2) {
+      const float x = (lane & 1) ? dS[u] : dS[u + 1];
+      const float y = __shfl_xor_sync(0xffffffffu, x, 1);
+      const int a = a0 + ah * HB + u + (lane & 1);
+      const uint32_t v = (lane & 1) ? frag::pack(y, dS[u + 1]) : frag::pack(dS[u], y);
+      *reinterpret_cast<uint32_t*>(hp + (size_t)a * D + (c & ~1)) = v;
+    }
+  };
+
+  write_dsb();
+  bscan_issue_tc<BV>(p, s.st[0], sv, dO, b, h, p.NC - 1, a0);
+  frag::cp_commit();
+  if (p.NC > 1) bscan_issue_tc<BV>(p, s.st[1], sv, dO, b, h, p.NC - 2, a0);
+  frag::cp_commit();
+  frag::cp_wait<1>();
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = s.tmem;
+
+  const uint32_t id1a = tc::idesc_bf16(64, BV, true, true);    // M^T dO
+  const uint32_t id1b = tc::idesc_bf16(64, BV, false, true);   // Kt dS^T
+  const uint32_t id2 = tc::idesc_bf16(128, BV, true, true);    // Qh^T dO, W^T (-dU)
+  const uint64_t dDSB = tc::sdesc_mnmaj(s.DSB, BV, 0), dDUB = tc::sdesc_mnmaj(s.DUB, BV, 0);
+  constexpr uint32_t kB = 2 * (BV / 8) * 128 / 16;   // MN-major B k-step (16-byte units)
+  constexpr uint32_t kA64 = 2 * (C / 8) * 128 / 16;  // MN-major A k-step, 64 wide
+  constexpr uint32_t kA128 = 2 * (D / 8) * 128 / 16; // MN-major A k-step, 128 wide
+  constexpr uint32_t kK = 256 / 16;                  // K-major k-step
+  // epilogue-1 ownership (M = 64 accumulator layout): row i = 16 (warp % 4) + lane, lane < 16
+  const int ri = 16 * (warp & 3) + (lane & 15);
+  bool ok = true;
+  for (int it = 0; it < p.NC && ok; ++it) {
+    const int n = p.NC - 1 - it;
+    const size_t cb = chunk_id(p, b, h, n);
+    BScanStage<BV>& st = s.st[it & 1];
+    const float dc = st.dec[c];  // read before the stage is refilled below
+    if (tid == 0) {
+      const uint64_t dM = tc::sdesc_mnmaj(st.M, C, 0), dDO = tc::sdesc_mnmaj(st.DO, BV, 0);
+      const uint64_t dKT = tc::sdesc_kmaj(st.KT, D, 0), dQH = tc::sdesc_mnmaj(st.QH, D, 0);
+#pragma unroll
+      for (int ks = 0; ks < C / 16; ++ks)
+        tc::mma(tbase + T_U, dM + ks * kA64, dDO + ks * kB, id1a, ks > 0 ? 1u : 0u);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        tc::mma(tbase + T_U, dKT + ks * kK, dDSB + ks * kB, id1b, 1u);
+#pragma unroll
+      for (int ks = 0; ks < C / 16; ++ks)
+        tc::mma(tbase + T_S, dQH + ks * kA128, dDO + ks * kB, id2, ks > 0 ? 1u : 0u);
+      tc::commit(&s.barA);
+    }
+    if (dhout) store_dh(cb);
+    ok = cta_wait(&s.barA, it);
+    if (!ok) break;
+    // epilogue 1: dU rows ri, value columns ah*HB ..
+    uint4 dusave[HB / 8];
+    {
+      uint32_t r[HB];
+#pragma unroll
+      for (int q16 = 0; q16 < HB / 16; ++q16)
+        tc::tmem_ld16_nowait(lane_addr(tbase, warp, T_U + ah * HB + 16 * q16), r + 16 * q16);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int e8 = 0; e8 < HB / 8; ++e8) {
+        const float* f = reinterpret_cast<const float*>(r + 8 * e8);
+        dusave[e8] = make_uint4(frag::pack(f[0], f[1]), frag::pack(f[2], f[3]),
+                                frag::pack(f[4], f[5]), frag::pack(f[6], f[7]));
+        if (lane < 16)
+          *reinterpret_cast<uint4*>(s.DUB + tc::mnmaj_off(ri, ah * HB + 8 * e8, BV)) =
+              make_uint4(frag::pack(-f[0], -f[1]), frag::pack(-f[2], -f[3]),
+                         frag::pack(-f[4], -f[5]), frag::pack(-f[6], -f[7]));
+      }
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (tid == 0) {
+      const uint64_t dW = tc::sdesc_mnmaj(st.W, D, 0);
+#pragma unroll
+      for (int ks = 0; ks < C / 16; ++ks)
+        tc::mma(tbase + T_S, dW + ks * kA128, dDUB + ks * kB, id2, 1u);
+      tc::commit(&s.barB);
+    }
+    if (lane < 16) {
+      bf16* up = dUout + cb * C * D;
+#pragma unroll
+      for (int e8 = 0; e8 < HB / 8; ++e8)
+        *reinterpret_cast<uint4*>(up + ct_off(ri, a0 + ah * HB + 8 * e8, D)) = dusave[e8];
+    }
+    ok = cta_wait(&s.barB, it);
+    if (!ok) break;
+    if (n >= 2) bscan_issue_tc<BV>(p, st, sv, dO, b, h, n - 2, a0);
+    frag::cp_commit();
+    // epilogue 2: dS^T <- Diag(e^{gamma_C}) dS^T + D_S
+    {
+      uint32_t r[HB];
+#pragma unroll
+      for (int q16 = 0; q16 < HB / 16; ++q16)
+        tc::tmem_ld16_nowait(lane_addr(tbase, warp, T_S + ah * HB + 16 * q16), r + 16 * q16);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < HB; ++e) dS[e] = dS[e] * dc + __uint_as_float(r[e]);
+      write_dsb();
+    }
+    frag::cp_wait<1>();
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+  }
+  if (ok) {
+    if (dS0) {
+#pragma unroll
+      for (int u = 0; u < HB; ++u) dS0[sbase + (size_t)(a0 + ah * HB + u) * D + c] = dS[u];
+    }
+  } else if (tid == 0 && err) {
+    atomicExch(err, 1);
+  }
+  frag::cp_wait<0>();
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tbase, TALLOC);
+}
+
+template <int BV>
+cudaError_t launch_bwd_scan_tc_bv(const Problem& p, const Saved& sv, const bf16* dO,
+                                  const float* dST, float* dS0, bf16* dU, bf16* dh,
+                                  cudaStream_t st) {
+  const size_t sm = sizeof(BScanSmem<BV>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(k_bwd_scan_tc<BV>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  const double nb = (double)p.B * p.H * p.NC, ntok = nb * C, heads = (double)p.B * p.H;
+  // reads W, Qh, Kt, M, dec, dO; writes dU, dh
+  const double bytes = nb * (3.0 * kTileBytes + kMBytes + kDecBytes) + ntok * D * 2 +
+                       nb * ((double)kUBytes + kStateBytes) +
+                       heads * D * D * 4 * ((dST ? 1 : 0) + (dS0 ? 1 : 0));
+  const double flops = nb * (2.0 * C * C * D + 2.0 * C * D * D * 3);
+  prof_begin(kKTcScanBwd, bytes, flops, st);
+  k_bwd_scan_tc<BV><<<dim3(D / BV, p.H, p.B), NTF, sm, st>>>(p, sv, dO, dST, dS0, dU, dh,
+                                                             device_error_word());
+  e = cudaGetLastError();
+  prof_end(st);
+  return e;
+}
+
 }  // namespace
 
 cudaError_t launch_fwd_scan_tc(const Problem& p, const Saved& sv, const float* S0, bf16* o,
@@ -320,6 +553,13 @@ cudaError_t launch_fwd_scan_tc(const Problem& p, const Saved& sv, const float* S
   // of the 148 SMs, whole-state tiles otherwise.
   if ((long)p.B * p.H * 2 <= 148) return launch_fwd_scan_tc_bv<64>(p, sv, S0, o, ST, save, st);
   return launch_fwd_scan_tc_bv<128>(p, sv, S0, o, ST, save, st);
+}
+
+cudaError_t launch_bwd_scan_tc(const Problem& p, const Saved& sv, const bf16* dO,
+                               const float* dST, float* dS0, bf16* dU, bf16* dh,
+                               cudaStream_t st) {
+  if ((long)p.B * p.H * 2 <= 148) return launch_bwd_scan_tc_bv<64>(p, sv, dO, dST, dS0, dU, dh, st);
+  return launch_bwd_scan_tc_bv<128>(p, sv, dO, dST, dS0, dU, dh, st);
 }
 
 }  // namespace fast
