@@ -47,6 +47,8 @@ def parse():
                     help="override the workload's batch size (smaller profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end run")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the single-token decode step instead of the training step")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target wall time of the timed oracle sample")
     return ap.parse_args()
@@ -265,10 +267,129 @@ def run_reference(args):
     }), flush=True)
 
 
+DECODE_METRIC = "decode tokens/s (one token per sequence per step, KDA bf16, d=128, fp32 state)"
+
+
+def run_decode(args):
+    """The single-token step (dr_decode_step) on a serving-sized batch: B
+    sequences x 16 heads, one token each per step, fp32 states resident in HBM
+    (B = 256: 256 MiB of state, larger than L2, read and written every step)."""
+    import torch
+    import torch.distributed as dist
+
+    from delta_rule_linear_chunkwise_b200 import WORKLOADS, binding, make_inputs
+    from delta_rule_linear_chunkwise_b200.workloads import random_state
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    w = WORKLOADS[args.workload or "kda_bf16_b4h16t8192"].with_(
+        name="kda_decode_bf16_b256h16d128", B=args.batch or 256, T=1)
+    inp = make_inputs(w, seed=w.seed + 1000 * rank)
+    S0 = random_state(w, seed=7 + rank, std=0.3)
+    d = {n: (None if x is None else x.to(dev)) for n, x in inp.items()}
+    S = S0.to(dev)
+    o = torch.empty(w.B, 1, w.H, w.dv, dtype=d["q"].dtype, device=dev)
+    kw = dict(beta_mode=w.beta_mode, eps=w.eps, o=o)
+
+    def step():
+        binding.decode_step(d["q"], d["k"], d["v"], d["beta"], d["g"], S, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    stream = torch.cuda.current_stream(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    binding.profile_enable(True)
+    with ClockSampler(local) as clk:
+        a.record(stream)
+        for _ in range(args.steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+    kernels = binding.profile_read()
+    binding.profile_enable(False)
+    assert binding.last_device_error() == binding.DR_OK
+    tot_ms = reduce_max(a.elapsed_time(b), dev)
+    value = aggregate_tokens_per_s(world, w.B, args.steps, tot_ms)
+
+    # end to end: the token's q, k, v, beta, g from pinned host memory, o back
+    hin = {n: x.pin_memory() for n, x in inp.items() if x is not None and n in
+           ("q", "k", "v", "beta", "g")}
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+
+    def e2e_step():
+        for n, x in hin.items():
+            d[n].copy_(x, non_blocking=True)
+        step()
+        ho.copy_(o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    a.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    t_e2e = reduce_max(a.elapsed_time(b), dev)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    top = max(kernels, key=lambda k: k["ms_total"])
+    per_launch_s = top["ms_total"] / top["launches"] / 1e3
+    gbs = top["bytes_per_launch"] / per_launch_s / 1e9
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        import time
+
+        import oracle
+        t0 = time.perf_counter()
+        _, _, used = oracle.recurrent_fwd(inp["q"], inp["k"], inp["v"], inp["beta"], inp["g"], S0,
+                                          eps=w.eps, return_threads=True)
+        dt = time.perf_counter() - t0
+        cpu = {"value": w.B / dt, "unit": "tokens/s", "cores": used, "kind": "oracle",
+               "sample": f"fp64 oracle recurrence, one token on all {w.B * w.H} heads "
+                         f"from the same state, wall clock {dt:.2f} s"}
+    out = {
+        "metric": DECODE_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "dk": w.dk, "dv": w.dv, "gate": w.gate,
+                   "state": "fp32 [B,H,128,128], resident, read and written each step",
+                   "l2": f"state {S.numel() * 4 >> 20} MiB per step, larger than L2",
+                   "parallelism": f"replicas x{world} (independent batches, no collective)"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_src} HBM copy",
+                     "kernel": top["name"], "us_per_launch": per_launch_s * 1e6,
+                     "algorithmic_bytes_per_launch": top["bytes_per_launch"], "traffic": None},
+        "cpu_baseline": cpu,
+        "e2e": {"value": aggregate_tokens_per_s(world, w.B, args.steps, t_e2e), "unit": "tokens/s",
+                "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in hin.values()),
+                "d2h_bytes_per_step": ho.numel() * ho.element_size()},
+        "gpu_launches": sum(k["launches"] for k in kernels),
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(out), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.decode:
+        run_decode(args)
         return
     import torch
     import torch.distributed as dist

@@ -63,6 +63,8 @@ def load() -> ctypes.CDLL:
     lib.dr_chunk_fwd.restype = i
     lib.dr_chunk_bwd.argtypes = [P] + [vp] * 15 + [vp, sz, vp]
     lib.dr_chunk_bwd.restype = i
+    lib.dr_decode_step.argtypes = [P] + [vp] * 7 + [vp]
+    lib.dr_decode_step.restype = i
     lib.dr_status_string.argtypes = [i]
     lib.dr_status_string.restype = ctypes.c_char_p
     lib.dr_last_device_error.argtypes = [vp]
@@ -253,6 +255,35 @@ def chunk_bwd(q, k, v, beta, g, S0, dO, dST=None, saved=None, *, beta_mode="dire
     plan = Plan(B, H, T, dk, dv, dtype=dtype, gate=gate, beta_mode=beta_mode, eps=eps,
                 chunk=chunk, device=q.device)
     return plan.bwd(q, k, v, beta, g, S0, dO, dST, saved, stream=stream)
+
+
+def decode_step(q, k, v, beta, g, S, *, beta_mode="direct", eps=1e-6, o=None, stream=None):
+    """One token per head through the recurrent update, S updated in place.
+
+    q, k ``[B,1,H,dk]``, v ``[B,1,H,dv]`` (bf16 or fp32), beta ``[B,1,H]``,
+    g ``None`` / ``[B,1,H]`` / ``[B,1,H,dk]`` fp32, S ``[B,H,dv,dk]`` fp32.
+    Returns o ``[B,1,H,dv]`` in the storage dtype."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    tdt = q.dtype
+    gate = "none" if g is None else ("channel" if g.dim() == 4 else "scalar")
+    prob = make_problem(B, H, T, dk, dv, dtype="bf16" if tdt == torch.bfloat16 else "f32",
+                        gate=gate, beta_mode=beta_mode, eps=eps)
+    _need(q, "q", tdt, (B, 1, H, dk), dev)
+    _need(k, "k", tdt, (B, 1, H, dk), dev)
+    _need(v, "v", tdt, (B, 1, H, dv), dev)
+    _need(beta, "beta", torch.float32, (B, 1, H), dev)
+    if g is not None:
+        _need(g, "g", torch.float32, (B, 1, H, dk) if gate == "channel" else (B, 1, H), dev)
+    _need(S, "S", torch.float32, (B, H, dv, dk), dev)
+    if o is None:
+        o = torch.empty(B, 1, H, dv, dtype=tdt, device=dev)
+    else:
+        _need(o, "o", tdt, (B, 1, H, dv), dev)
+    _check(load().dr_decode_step(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                 _ptr(g), _ptr(S), _ptr(o), _stream(stream)), "dr_decode_step")
+    return o
 
 
 def profile_enable(on: bool = True) -> None:

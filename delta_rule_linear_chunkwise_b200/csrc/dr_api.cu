@@ -207,6 +207,22 @@ dr_status dr_chunk_fwd(const dr_problem* p, const void* q, const void* k, const 
   return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
 }
 
+dr_status dr_decode_step(const dr_problem* p, const void* q, const void* k, const void* v,
+                         const float* beta, const float* g, float* S, void* o, void* stream) {
+  Problem P;
+  dr_status s = validate(p, &P);
+  if (s != DR_OK) return s;
+  if (p->T != 1) return DR_ERR_INVALID_ARG;
+  if (!q || !k || !v || !beta || !S || !o) return DR_ERR_INVALID_ARG;
+  if ((P.gate == DR_GATE_NONE) != (g == nullptr)) return DR_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, beta, g, S, o};
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return DR_ERR_INVALID_ARG;
+  const cudaError_t e = dr::launch_decode_step(P, p->dtype == DR_BF16, q, k, v, beta, g, S, o,
+                                               (cudaStream_t)stream);
+  return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+}
+
 dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const void* v,
                        const float* beta, const float* g, const float* S0, const void* dO,
                        const float* dST, const void* saved, void* dq, void* dk, void* dv,

@@ -66,7 +66,7 @@ __device__ __forceinline__ void store_f<__nv_bfloat16>(__nv_bfloat16* p, float x
 // Kernel ids for the opt-in per-kernel timing (profile.cu).
 enum {
   kKIntraFwd = 0, kKScanFwd, kKScanBwd, kKStateGrads, kKIntraBwd,
-  kKTcIntraFwd, kKTcScanFwd, kKTcScanBwd, kKTcChunkBwd
+  kKTcIntraFwd, kKTcScanFwd, kKTcScanBwd, kKTcChunkBwd, kKDecode
 };
 const char* kernel_name(int id);
 // Bracket one launch with events on its stream when profiling is enabled.
@@ -92,5 +92,10 @@ cudaError_t launch_generic_bwd(const Problem& p, const TIn* q, const TIn* k, con
                                const TIn* dO, const float* dST, const float* hsaved,
                                TIn* dq, TIn* dk, TIn* dv, float* dbeta, float* dg,
                                float* dS0, const Ws& ws, cudaStream_t st);
+
+// The single-token recurrent step (decode.cu); bf16 != 0 for bf16 q, k, v, o.
+cudaError_t launch_decode_step(const Problem& p, int bf16, const void* q, const void* k,
+                               const void* v, const float* beta, const float* g, float* S, void* o,
+                               cudaStream_t st);
 
 }  // namespace dr

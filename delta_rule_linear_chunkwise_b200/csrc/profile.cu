@@ -43,6 +43,7 @@ const char* kernel_name(int id) {
     case kKTcScanFwd: return "tc_scan_fwd";
     case kKTcScanBwd: return "tc_scan_bwd";
     case kKTcChunkBwd: return "tc_chunk_bwd";
+    case kKDecode: return "decode_step";
   }
   return "unknown";
 }

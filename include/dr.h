@@ -108,6 +108,27 @@ dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const 
                        float* dbeta, float* dg, float* dS0, void* ws, size_t ws_bytes,
                        void* stream);
 
+/* Single-token recurrent step (decode), the update itself applied to one
+   token per head: with alpha = exp(g) (1 for gate NONE),
+     P = S Diag(alpha),  e = v - P k,  S <- P + beta e k^T,  o = S q
+   ("Semidirect Fourier Delta Attention" explainer, gist.science, section
+   Kernarchitektur, with zero phase; the KLA abstract, "How AI settled the
+   complexity of the oldest SGD algorithm", reports the decode throughput of
+   this step).  In Kaczmarz mode beta carries eta and beta = eta / (||k||^2 +
+   eps).
+   p:   as for the chunkwise calls with T == 1 (chunk is not used but must be
+        64); any other T gives DR_ERR_INVALID_ARG.
+   In:  q, k [B,1,H,dk] and v [B,1,H,dv] in the storage dtype, beta [B,1,H]
+        fp32, g [B,1,H] (scalar gate) or [B,1,H,dk] (per-channel gate) fp32,
+        NULL iff gate NONE.
+   In/out: S [B,H,dv,dk] fp32, the state before the token on entry and after
+        it on return (the caller owns it; it is updated in place).
+   Out: o [B,1,H,dv] in the storage dtype.
+   All pointers 16-byte aligned device memory; no workspace; asynchronous on
+   `stream`.  Host-side argument errors return before any launch. */
+dr_status dr_decode_step(const dr_problem* p, const void* q, const void* k, const void* v,
+                         const float* beta, const float* g, float* S, void* o, void* stream);
+
 /* Size of the library's built-in forward scratch (64 MiB), held on every GPU
    that loads the library, until the process exits. */
 #define DR_STATIC_SCRATCH_BYTES (64u << 20)

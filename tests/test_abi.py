@@ -132,6 +132,26 @@ def test_bwd_argument_errors(lib):
     assert _bwd(lib, _prob(dk=48, dv=24)) == binding.DR_ERR_UNSUPPORTED
 
 
+def _dec(lib, p, **over):
+    names = ("q", "k", "v", "beta", "g", "S", "o")
+    args = {n: A + 0x1000 * i for i, n in enumerate(names)}
+    args.update(over)
+    vp = ctypes.c_void_p
+    return lib.dr_decode_step(ctypes.byref(p), *(vp(args[n]) if args[n] else None for n in names),
+                              None)
+
+
+def test_decode_argument_errors(lib):
+    p = _prob(T=1)
+    assert _dec(lib, _prob(T=2)) == binding.DR_ERR_INVALID_ARG         # one token per call
+    assert _dec(lib, p, S=None) == binding.DR_ERR_INVALID_ARG          # the state is in/out
+    assert _dec(lib, p, o=None) == binding.DR_ERR_INVALID_ARG
+    assert _dec(lib, p, g=None) == binding.DR_ERR_INVALID_ARG          # gate needs g
+    assert _dec(lib, _prob(T=1, gate="none")) == binding.DR_ERR_INVALID_ARG  # no gate, g given
+    assert _dec(lib, p, v=A + 0x2004) == binding.DR_ERR_INVALID_ARG    # misaligned
+    assert _dec(lib, _prob(T=1, dk=24)) == binding.DR_ERR_UNSUPPORTED
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "libdr.so"))
     monkeypatch.setattr(binding, "_lib", None)
