@@ -88,6 +88,8 @@ Layout layout(const Problem& p, int pass) {
   size_t fast = round_up(dr::fast::saved_bytes(p));
   if (pass == 1)
     fast += round_up(nb2 * dr::fast::kUBytes) + round_up(nb2 * dr::fast::kStateBytes);
+  // segmented (affine) scans: two [B][G][H] state buffers
+  fast += 2 * round_up(dr::fast::affine_map_bytes(p, dr::fast::affine_segments(p)));
   L.total = o > fast ? o : fast;
   return L;
 }
@@ -142,6 +144,54 @@ cudaError_t bwd_scan(const dr::Problem& P, const dr::fast::Saved& sv, const __nv
   return dr::fast::launch_bwd_scan_tc(P, sv, dO, dST, dS0, dU, dh, st);
 }
 
+// Segments of the chunk-parallel affine scan for this problem (1 = sequential).
+int scan_segments(const Problem& P) {
+  return use_mma_sync_scans() ? 1 : dr::fast::affine_segments(P);
+}
+
+// The forward state scan, plain or segmented.  Segmented: the transfer
+// matrices (into the saved tiles) and offsets of all segments in one
+// parallel pass, their composition into segment start states, then the
+// output pass of all segments in parallel.  aff: two affine buffers.
+cudaError_t fwd_scan_any(const Problem& P, const dr::fast::Saved& sv, const float* S0,
+                         __nv_bfloat16* o, float* ST, bool save, char* aff, cudaStream_t st) {
+  const int G = scan_segments(P);
+  if (G == 1) return fwd_scan(P, sv, S0, o, ST, save, st);
+  const int L = dr::fast::affine_seg_len(P, G);
+  float* Bm = (float*)aff;
+  float* Sst = (float*)(aff + round_up(dr::fast::affine_map_bytes(P, G)));
+  const int bv_maps = (long)4 * P.B * P.H * G <= 148 ? 64 : 128;
+  cudaError_t e = dr::fast::launch_fwd_scan_tc_seg(
+      P, sv, dr::fast::ScanSeg{G, L, 3, nullptr, sv.Pseg, Bm}, nullptr, false, bv_maps, st);
+  if (e == cudaSuccess) e = dr::fast::launch_affine_compose_fwd(P, G, S0, sv.Pseg, Bm, Sst, ST, st);
+  if (e == cudaSuccess)
+    e = dr::fast::launch_fwd_scan_tc_seg(P, sv, dr::fast::ScanSeg{G, L, 0, Sst, nullptr, nullptr},
+                                         o, save, 64, st);
+  return e;
+}
+
+// The backward state-gradient scan, plain or segmented (the segment offsets C
+// in parallel, their composition with the saved transfer matrices into
+// segment end gradients and dS0, then the output pass in parallel).
+cudaError_t bwd_scan_any(const Problem& P, const dr::fast::Saved& sv, const __nv_bfloat16* dO,
+                         const float* dST, float* dS0, __nv_bfloat16* dU, __nv_bfloat16* dh,
+                         char* aff, cudaStream_t st) {
+  const int G = scan_segments(P);
+  if (G == 1) return bwd_scan(P, sv, dO, dST, dS0, dU, dh, st);
+  const int L = dr::fast::affine_seg_len(P, G);
+  float* Cm = (float*)aff;
+  float* dSe = (float*)(aff + round_up(dr::fast::affine_map_bytes(P, G)));
+  cudaError_t e = dr::fast::launch_bwd_scan_tc_seg(
+      P, sv, dO, dr::fast::ScanSeg{G, L, 1, nullptr, Cm, nullptr}, nullptr, nullptr, 64, st);
+  if (e == cudaSuccess)
+    e = dr::fast::launch_affine_compose_bwd(P, G, dST, sv.Pseg, Cm, dSe, dS0, st);
+  if (e == cudaSuccess)
+    e = dr::fast::launch_bwd_scan_tc_seg(P, sv, dO,
+                                         dr::fast::ScanSeg{G, L, 0, dSe, nullptr, nullptr}, dU,
+                                         dh, 64, st);
+  return e;
+}
+
 size_t saved_bytes(const Problem& p) {
   const size_t generic = (size_t)p.B * p.H * p.NC * p.dv * p.dk * sizeof(float);
   const size_t fast = dr::fast::saved_bytes(p);
@@ -192,9 +242,10 @@ dr_status dr_chunk_fwd(const dr_problem* p, const void* q, const void* k, const 
     // (the backward reuses them), else to the workspace.
     dr::fast::Saved sv = dr::fast::carve_saved(P, saved ? saved : ws);
     using bf = __nv_bfloat16;
+    char* aff = (char*)ws + round_up(dr::fast::saved_bytes(P));
     e = dr::fast::launch_prep(P, (const bf*)q, (const bf*)k, (const bf*)v, beta, g, sv, st);
     if (e == cudaSuccess)
-      e = fwd_scan(P, sv, S0, (bf*)o, ST, saved != nullptr, st);
+      e = fwd_scan_any(P, sv, S0, (bf*)o, ST, saved != nullptr, aff, st);
     return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
   }
   if (p->dtype == DR_F32)
@@ -247,21 +298,21 @@ dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const 
     using bf = __nv_bfloat16;
     // The forward's per-chunk tensors come from its saved buffer or are
     // recomputed into the workspace.
-    char* wsb = (char*)ws;
+    char* wsb = (char*)ws + round_up(dr::fast::saved_bytes(P));
+    const size_t nb = (size_t)P.B * P.H * P.NC;
+    bf* dU = (bf*)wsb;
+    bf* dh = (bf*)(wsb + round_up(nb * dr::fast::kUBytes));
+    char* aff = wsb + round_up(nb * dr::fast::kUBytes) + round_up(nb * dr::fast::kStateBytes);
     dr::fast::Saved sv;
     if (saved) {
       sv = dr::fast::carve_saved(P, (void*)saved);
     } else {
-      sv = dr::fast::carve_saved(P, wsb);
+      sv = dr::fast::carve_saved(P, ws);
       e = dr::fast::launch_prep(P, (const bf*)q, (const bf*)k, (const bf*)v, beta, g, sv, st);
-      if (e == cudaSuccess) e = fwd_scan(P, sv, S0, nullptr, nullptr, true, st);
+      if (e == cudaSuccess) e = fwd_scan_any(P, sv, S0, nullptr, nullptr, true, aff, st);
       if (e != cudaSuccess) return DR_ERR_CUDA;
-      wsb += round_up(dr::fast::saved_bytes(P));
     }
-    const size_t nb = (size_t)P.B * P.H * P.NC;
-    bf* dU = (bf*)wsb;
-    bf* dh = (bf*)(wsb + round_up(nb * dr::fast::kUBytes));
-    e = bwd_scan(P, sv, (const bf*)dO, dST, dS0, dU, dh, st);
+    e = bwd_scan_any(P, sv, (const bf*)dO, dST, dS0, dU, dh, aff, st);
     if (e == cudaSuccess)
       e = use_tcgen05_chunk_bwd()
               ? dr::fast::launch_bwd_chunk_tc(P, (const bf*)q, (const bf*)k, (const bf*)v,

@@ -66,7 +66,7 @@ __device__ __forceinline__ void store_f<__nv_bfloat16>(__nv_bfloat16* p, float x
 // Kernel ids for the opt-in per-kernel timing (profile.cu).
 enum {
   kKIntraFwd = 0, kKScanFwd, kKScanBwd, kKStateGrads, kKIntraBwd,
-  kKTcIntraFwd, kKTcScanFwd, kKTcScanBwd, kKTcChunkBwd, kKDecode
+  kKTcIntraFwd, kKTcScanFwd, kKTcScanBwd, kKTcChunkBwd, kKDecode, kKAffine
 };
 const char* kernel_name(int id);
 // Bracket one launch with events on its stream when profiling is enabled.

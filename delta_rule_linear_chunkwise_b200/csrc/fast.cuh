@@ -12,6 +12,41 @@ inline bool eligible(const Problem& p, int dtype_bf16) {
   return dtype_bf16 && p.dk == 128 && p.dv == 128;
 }
 
+// Segmented scans (the chunk-parallel affine scan for long sequences with few
+// heads): the chunks of a head are split into G segments of L chunks and one
+// CTA runs one segment (blockIdx.z = b * G + segment).
+//   forward  mode 0: the output scan from the given segment start states;
+//            mode 1: the segment's transfer matrix P (start I, U' = 0);
+//            mode 2: its offset B (start 0), so that S_end = S_start P + B.
+//   backward mode 0: the gradient scan from the given segment end gradients;
+//            mode 1: the segment's offset C (end gradient 0), so that
+//            dS_start = dS_end P^T + C.
+//   forward  mode 3: modes 1 and 2 in one launch (blockIdx.x selects), the
+//            transfer matrices to ST and the offsets to ST2.
+struct ScanSeg {
+  int G, L, mode;
+  const float* S0;  // [B][G][H][128][128] start states (forward) / end gradients (backward)
+  float* ST;        // [B][G][H][128][128] end states (forward) / start gradients (backward)
+  float* ST2;       // mode 3: the offsets
+};
+
+// Number of sequence segments for the affine scan (1 = plain sequential scans):
+// used when the plain scans would occupy at most half of the 148 SMs and the
+// sequence is long, with as many segments as fill one wave.
+inline int affine_segments(const Problem& p) {
+  const long ctas = (long)p.B * p.H * 2;  // plain scans: two 64-row value tiles per head
+  if (ctas > 74 || p.NC < 64) return 1;
+  int G = (int)(148 / ctas);
+  if (G > 16) G = 16;
+  const int L = (p.NC + G - 1) / G;
+  return (p.NC + L - 1) / L;
+}
+inline int affine_seg_len(const Problem& p, int G) { return (p.NC + G - 1) / G; }
+// Bytes of one [B][G][H][128][128] fp32 buffer of segment maps or states.
+inline size_t affine_map_bytes(const Problem& p, int G) {
+  return G > 1 ? (size_t)p.B * G * p.H * 128 * 128 * 4 : 0;
+}
+
 // Per-chunk byte sizes of the tensors the fast path keeps between kernels.
 constexpr size_t kTBytes = 64 * 64 * 2;        // (I + A)^{-1}, bf16
 constexpr size_t kBetaBytes = 64 * 4;          // effective beta, fp32
@@ -37,6 +72,7 @@ struct Saved {
   __nv_bfloat16* h;    // [nb][128][128]  chunk start state S (value-major)
   __nv_bfloat16* U;    // [nb][64][128]   U = U' - W S^T                       [ct]
   float* knorm;        // [nb][64]        ||k||^2 of each row
+  float* Pseg;         // [B][G][H][128][128] segment transfer matrices (affine scan; else null)
 };
 
 // Core-tiled storage of an [R][ncol] bf16 tile: 8 x 8 blocks of 128
@@ -96,7 +132,8 @@ __device__ __forceinline__ void cp_linear(__nv_bfloat16* smem, const __nv_bfloat
 inline size_t saved_bytes(const Problem& p) {
   const size_t nb = (size_t)p.B * p.H * p.NC;
   return nb * (kTBytes + 2 * kBetaBytes + kDecBytes + 4 * kTileBytes + kMBytes + kStateBytes +
-               kUBytes);
+               kUBytes) +
+         affine_map_bytes(p, affine_segments(p));
 }
 inline Saved carve_saved(const Problem& p, void* base) {
   const size_t nb = (size_t)p.B * p.H * p.NC;
@@ -112,7 +149,8 @@ inline Saved carve_saved(const Problem& p, void* base) {
   s.Kt = (__nv_bfloat16*)c;           c += nb * kTileBytes;
   s.h = (__nv_bfloat16*)c;            c += nb * kStateBytes;
   s.U = (__nv_bfloat16*)c;             c += nb * kUBytes;
-  s.knorm = (float*)c;
+  s.knorm = (float*)c;                c += nb * kBetaBytes;
+  s.Pseg = affine_segments(p) > 1 ? (float*)c : nullptr;
   return s;
 }
 
@@ -127,6 +165,20 @@ cudaError_t launch_fwd_scan(const Problem& p, const Saved& sv, const float* S0,
 // The same on tcgen05: MMAs into tensor memory, fp32 state in registers.
 cudaError_t launch_fwd_scan_tc(const Problem& p, const Saved& sv, const float* S0,
                                __nv_bfloat16* o, float* ST, bool save, cudaStream_t st);
+// Segmented forms (see ScanSeg); bv = 64 or 128 value rows per CTA.
+cudaError_t launch_fwd_scan_tc_seg(const Problem& p, const Saved& sv, const ScanSeg& sg,
+                                   __nv_bfloat16* o, bool save, int bv, cudaStream_t st);
+cudaError_t launch_bwd_scan_tc_seg(const Problem& p, const Saved& sv, const __nv_bfloat16* dO,
+                                   const ScanSeg& sg, __nv_bfloat16* dU, __nv_bfloat16* dh,
+                                   int bv, cudaStream_t st);
+// Composition of the segment maps (fast_affine.cu).
+//   forward:  Sst[0] = S0 (or 0); Sst[g+1] = Sst[g] P[g] + Bm[g]; ST = Sst[G-1] P + Bm
+//   backward: dSe[G-1] = dST (or 0); dSe[g-1] = dSe[g] P[g]^T + Cm[g];
+//             dS0 = dSe[0] P[0]^T + Cm[0]
+cudaError_t launch_affine_compose_fwd(const Problem& p, int G, const float* S0, const float* P,
+                                      const float* Bm, float* Sst, float* ST, cudaStream_t st);
+cudaError_t launch_affine_compose_bwd(const Problem& p, int G, const float* dST, const float* P,
+                                      const float* Cm, float* dSe, float* dS0, cudaStream_t st);
 cudaError_t launch_bwd_scan_tc(const Problem& p, const Saved& sv, const __nv_bfloat16* dO,
                                const float* dST, float* dS0, __nv_bfloat16* dU,
                                __nv_bfloat16* dh, cudaStream_t st);

@@ -60,7 +60,7 @@ struct ScanSmem {
 // contiguous run per block of 8 rows.
 template <int BV>
 __device__ __forceinline__ void scan_issue(const Problem& p, ScanStage<BV>& s, const Saved& sv,
-                                           size_t cb, int a0, bool with_o) {
+                                           size_t cb, int a0, bool with_o, bool with_up) {
   const int tid = threadIdx.x;
   cp_linear<NTF>(s.AWQ, sv.W + cb * C * D, C * D, tid);
   if (with_o) {
@@ -68,7 +68,7 @@ __device__ __forceinline__ void scan_issue(const Problem& p, ScanStage<BV>& s, c
     cp_linear<NTF>(s.MZ + C * C, sv.M + cb * C * C, C * C, tid);
   }
   cp_linear<NTF>(s.KT, sv.Kt + cb * C * D, C * D, tid);
-  cp_ct_cols<NTF>(s.UP, sv.Up + cb * C * D, C, a0, BV, tid);
+  if (with_up) cp_ct_cols<NTF>(s.UP, sv.Up + cb * C * D, C, a0, BV, tid);
   if (tid < D / 4) frag::cp16(s.dec + 4 * tid, sv.dec + cb * D + 4 * tid, true);
 }
 
@@ -86,18 +86,31 @@ __device__ __forceinline__ bool cta_wait(uint64_t* bar, int parity) {
 
 template <int BV>
 __global__ void __launch_bounds__(NTF, 1)
-    k_fwd_scan_tc(Problem p, Saved sv, const float* __restrict__ S0, bf16* __restrict__ o,
-                  float* __restrict__ ST, int save, int* __restrict__ err) {
+    k_fwd_scan_tc(Problem p, Saved sv, ScanSeg sg, bf16* __restrict__ o, int save,
+                  int* __restrict__ err) {
   constexpr int HB = BV / 2;             // value columns per thread in the state epilogue
   constexpr int TCOLS = 3 * BV;          // tensor memory columns: D_A x 2, D_S
   constexpr int TALLOC = TCOLS <= 256 ? 256 : 512;
   extern __shared__ __align__(1024) unsigned char smraw[];
   ScanSmem<BV>& s = *reinterpret_cast<ScanSmem<BV>*>(smraw);
-  const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z / sg.G, seg = blockIdx.z % sg.G, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int a0 = blockIdx.x * BV;
+  int mode = sg.mode, xb = blockIdx.x;
+  float* __restrict__ ST = sg.ST;
+  if (mode == 3) {  // transfer matrices (first D/BV x-blocks) and offsets (the rest)
+    mode = xb < D / BV ? 1 : 2;
+    if (mode == 2) {
+      ST = sg.ST2;
+      xb -= D / BV;
+    }
+  }
+  const int a0 = xb * BV;
+  const int n0 = seg * sg.L, n1 = min(p.NC, n0 + sg.L);
+  if (n0 >= n1) return;
   const bool with_o = o != nullptr;
-  const size_t sbase = ((size_t)b * p.H + h) * D * D;
+  const bool with_up = mode != 1;
+  const float* __restrict__ S0 = mode == 0 ? sg.S0 : nullptr;
+  const size_t sbase = (((size_t)b * sg.G + seg) * p.H + h) * D * D;
   // state epilogue ownership: key column c (= TMEM lane), value columns ah*HB ..
   const int c = 32 * (warp & 3) + lane, ah = warp >> 2;
   const uint32_t T_S = 2 * BV;  // D_A buffers at columns 0 and BV
@@ -115,8 +128,10 @@ __global__ void __launch_bounds__(NTF, 1)
   // fp32 state S^T[c][a0 + ah*HB + u]
   float S[HB];
 #pragma unroll
-  for (int u = 0; u < HB; ++u)
-    S[u] = S0 ? S0[sbase + (size_t)(a0 + ah * HB + u) * D + c] : 0.f;
+  for (int u = 0; u < HB; ++u) {
+    const int a = a0 + ah * HB + u;
+    S[u] = mode == 1 ? (a == c ? 1.f : 0.f) : (S0 ? S0[sbase + (size_t)a * D + c] : 0.f);
+  }
 
   auto write_sb = [&]() {
 #pragma unroll
@@ -165,9 +180,9 @@ __global__ void __launch_bounds__(NTF, 1)
   };
 
   write_sb();
-  scan_issue<BV>(p, s.st[0], sv, chunk_id(p, b, h, 0), a0, with_o);
+  scan_issue<BV>(p, s.st[0], sv, chunk_id(p, b, h, n0), a0, with_o, with_up);
   frag::cp_commit();
-  if (p.NC > 1) scan_issue<BV>(p, s.st[1], sv, chunk_id(p, b, h, 1), a0, with_o);
+  if (n0 + 1 < n1) scan_issue<BV>(p, s.st[1], sv, chunk_id(p, b, h, n0 + 1), a0, with_o, with_up);
   frag::cp_commit();
   frag::cp_wait<1>();
   tc::fence_smem_to_async();
@@ -183,10 +198,11 @@ __global__ void __launch_bounds__(NTF, 1)
   const uint64_t dSB = tc::sdesc_mnmaj(s.SB, BV, 0), dUB = tc::sdesc_mnmaj(s.UB, BV, 0);
   constexpr uint32_t kSB = 2 * (BV / 8) * 128 / 16, kUB = kSB, kKM = 256 / 16;
   constexpr uint32_t kKT = 2 * (D / 8) * 128 / 16;
-  for (int n = 0; n < p.NC && ok; ++n) {
+  for (int n = n0; n < n1 && ok; ++n) {
+    const int it = n - n0;
     const size_t cb = chunk_id(p, b, h, n);
-    ScanStage<BV>& st = s.st[n & 1];
-    const int buf = n & 1;
+    ScanStage<BV>& st = s.st[it & 1];
+    const int buf = it & 1;
     const float dc = st.dec[c];  // read before the stage is refilled below
     // MMA-A: [W ; q e^gamma] S^T
     if (tid == 0) {
@@ -197,8 +213,8 @@ __global__ void __launch_bounds__(NTF, 1)
       tc::commit(&s.barA);
     }
     // while it runs: the previous chunk's output
-    if (with_o && n > 0) store_o(n - 1, buf ^ 1);
-    ok = cta_wait(&s.barA, n);
+    if (with_o && it > 0) store_o(n - 1, buf ^ 1);
+    ok = cta_wait(&s.barA, it);
     if (!ok) break;
     // epilogue 1: U = U' - W S^T (rows i = lanes 0 .. 63)
     uint4 usave[HB / 8];
@@ -212,7 +228,8 @@ __global__ void __launch_bounds__(NTF, 1)
 #pragma unroll
       for (int e8 = 0; e8 < HB / 8; ++e8) {
         const int a = ah * HB + 8 * e8;
-        const uint4 u8 = *reinterpret_cast<const uint4*>(st.UP + ct_off(i, a, BV));
+        const uint4 u8 = with_up ? *reinterpret_cast<const uint4*>(st.UP + ct_off(i, a, BV))
+                                 : make_uint4(0, 0, 0, 0);
         const uint32_t* w8 = reinterpret_cast<const uint32_t*>(&u8);
         const float* f = reinterpret_cast<const float*>(r + 8 * e8);
         uint32_t pk[4];
@@ -253,10 +270,10 @@ __global__ void __launch_bounds__(NTF, 1)
       }
       store_h(cb);
     }
-    ok = cta_wait(&s.barB, n);
+    ok = cta_wait(&s.barB, it);
     if (!ok) break;
     // this stage is consumed: refill it with chunk n + 2 (lands during the next step)
-    if (n + 2 < p.NC) scan_issue<BV>(p, st, sv, chunk_id(p, b, h, n + 2), a0, with_o);
+    if (n + 2 < n1) scan_issue<BV>(p, st, sv, chunk_id(p, b, h, n + 2), a0, with_o, with_up);
     frag::cp_commit();
     // epilogue 2: S^T <- Diag(e^{gamma_C}) S^T + D_S
     {
@@ -276,7 +293,7 @@ __global__ void __launch_bounds__(NTF, 1)
     tc::fence_after_sync();
   }
   if (ok) {
-    if (with_o) store_o(p.NC - 1, (p.NC - 1) & 1);
+    if (with_o) store_o(n1 - 1, (n1 - 1 - n0) & 1);
     if (ST) {
 #pragma unroll
       for (int u = 0; u < HB; ++u) ST[sbase + (size_t)(a0 + ah * HB + u) * D + c] = S[u];
@@ -291,22 +308,27 @@ __global__ void __launch_bounds__(NTF, 1)
 }
 
 template <int BV>
-cudaError_t launch_fwd_scan_tc_bv(const Problem& p, const Saved& sv, const float* S0, bf16* o,
-                                  float* ST, bool save, cudaStream_t st) {
+cudaError_t launch_fwd_scan_tc_bv(const Problem& p, const Saved& sv, const ScanSeg& sg, bf16* o,
+                                  bool save, cudaStream_t st) {
+  const float* S0 = sg.mode == 0 ? sg.S0 : nullptr;
+  float* ST = sg.ST;
+  const int maps = sg.mode == 3 ? 2 : 1;  // mode 3 runs both map kinds
   const size_t sm = sizeof(ScanSmem<BV>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_fwd_scan_tc<BV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const double nb = (double)p.B * p.H * p.NC, ntok = nb * C, heads = (double)p.B * p.H;
-  // reads W, Kt, U', dec (+ q e^gamma, M with the output); writes h, U (saving), o
-  double bytes = nb * (2.0 * kTileBytes + kTileBytes + kDecBytes);
+  // reads W, Kt, U' (not for a transfer-matrix pass), dec (+ q e^gamma, M with the
+  // output); writes h, U (saving), o, and the segment start / end states
+  double bytes = nb * (2.0 * kTileBytes + (sg.mode == 1 ? 0.0 : (double)kTileBytes) + kDecBytes);
   if (o) bytes += nb * ((double)kTileBytes + kMBytes) + ntok * D * 2;
   if (save) bytes += nb * ((double)kStateBytes + kUBytes);
-  bytes += heads * D * D * 4 * ((S0 ? 1 : 0) + (ST ? 1 : 0));
-  const double flops = nb * (2.0 * C * D * D * (o ? 3 : 2) + (o ? 2.0 * C * C * D : 0.0));
+  bytes += heads * sg.G * D * D * 4 * ((S0 ? 1 : 0) + (ST ? maps : 0));
+  const double flops =
+      maps * nb * (2.0 * C * D * D * (o ? 3 : 2) + (o ? 2.0 * C * C * D : 0.0));
   prof_begin(kKTcScanFwd, bytes, flops, st);
-  k_fwd_scan_tc<BV><<<dim3(D / BV, p.H, p.B), NTF, sm, st>>>(p, sv, S0, o, ST, save ? 1 : 0,
-                                                             device_error_word());
+  k_fwd_scan_tc<BV><<<dim3(maps * (D / BV), p.H, p.B * sg.G), NTF, sm, st>>>(
+      p, sv, sg, o, save ? 1 : 0, device_error_word());
   e = cudaGetLastError();
   prof_end(st);
   return e;
@@ -362,17 +384,21 @@ __device__ __forceinline__ void bscan_issue_tc(const Problem& p, BScanStage<BV>&
 
 template <int BV>
 __global__ void __launch_bounds__(NTF, 1)
-    k_bwd_scan_tc(Problem p, Saved sv, const bf16* __restrict__ dO, const float* __restrict__ dST,
-                  float* __restrict__ dS0, bf16* __restrict__ dUout, bf16* __restrict__ dhout,
-                  int* __restrict__ err) {
+    k_bwd_scan_tc(Problem p, Saved sv, const bf16* __restrict__ dO, ScanSeg sg,
+                  bf16* __restrict__ dUout, bf16* __restrict__ dhout, int* __restrict__ err) {
   constexpr int HB = BV / 2;
   constexpr int TALLOC = 2 * BV <= 128 ? 128 : 256;
   extern __shared__ __align__(1024) unsigned char smraw[];
   BScanSmem<BV>& s = *reinterpret_cast<BScanSmem<BV>*>(smraw);
-  const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z / sg.G, seg = blockIdx.z % sg.G, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int a0 = blockIdx.x * BV;
-  const size_t sbase = ((size_t)b * p.H + h) * D * D;
+  const int n0 = seg * sg.L, n1 = min(p.NC, n0 + sg.L);
+  if (n0 >= n1) return;
+  const bool outputs = sg.mode == 0;
+  const float* __restrict__ dST = outputs ? sg.S0 : nullptr;
+  float* __restrict__ dS0 = sg.ST;
+  const size_t sbase = (((size_t)b * sg.G + seg) * p.H + h) * D * D;
   const int c = 32 * (warp & 3) + lane, ah = warp >> 2;  // key (TMEM lane), value half
   const uint32_t T_U = 0, T_S = BV;
 
@@ -408,9 +434,9 @@ __global__ void __launch_bounds__(NTF, 1)
   };
 
   write_dsb();
-  bscan_issue_tc<BV>(p, s.st[0], sv, dO, b, h, p.NC - 1, a0);
+  bscan_issue_tc<BV>(p, s.st[0], sv, dO, b, h, n1 - 1, a0);
   frag::cp_commit();
-  if (p.NC > 1) bscan_issue_tc<BV>(p, s.st[1], sv, dO, b, h, p.NC - 2, a0);
+  if (n1 - 2 >= n0) bscan_issue_tc<BV>(p, s.st[1], sv, dO, b, h, n1 - 2, a0);
   frag::cp_commit();
   frag::cp_wait<1>();
   tc::fence_smem_to_async();
@@ -430,8 +456,8 @@ __global__ void __launch_bounds__(NTF, 1)
   // epilogue-1 ownership (M = 64 accumulator layout): row i = 16 (warp % 4) + lane, lane < 16
   const int ri = 16 * (warp & 3) + (lane & 15);
   bool ok = true;
-  for (int it = 0; it < p.NC && ok; ++it) {
-    const int n = p.NC - 1 - it;
+  for (int it = 0; it < n1 - n0 && ok; ++it) {
+    const int n = n1 - 1 - it;
     const size_t cb = chunk_id(p, b, h, n);
     BScanStage<BV>& st = s.st[it & 1];
     const float dc = st.dec[c];  // read before the stage is refilled below
@@ -449,7 +475,7 @@ __global__ void __launch_bounds__(NTF, 1)
         tc::mma(tbase + T_S, dQH + ks * kA128, dDO + ks * kB, id2, ks > 0 ? 1u : 0u);
       tc::commit(&s.barA);
     }
-    if (dhout) store_dh(cb);
+    if (outputs) store_dh(cb);
     ok = cta_wait(&s.barA, it);
     if (!ok) break;
     // epilogue 1: dU rows ri, value columns ah*HB ..
@@ -482,7 +508,7 @@ __global__ void __launch_bounds__(NTF, 1)
         tc::mma(tbase + T_S, dW + ks * kA128, dDUB + ks * kB, id2, 1u);
       tc::commit(&s.barB);
     }
-    if (lane < 16) {
+    if (outputs && lane < 16) {
       bf16* up = dUout + cb * C * D;
 #pragma unroll
       for (int e8 = 0; e8 < HB / 8; ++e8)
@@ -490,7 +516,7 @@ __global__ void __launch_bounds__(NTF, 1)
     }
     ok = cta_wait(&s.barB, it);
     if (!ok) break;
-    if (n >= 2) bscan_issue_tc<BV>(p, st, sv, dO, b, h, n - 2, a0);
+    if (n - 2 >= n0) bscan_issue_tc<BV>(p, st, sv, dO, b, h, n - 2, a0);
     frag::cp_commit();
     // epilogue 2: dS^T <- Diag(e^{gamma_C}) dS^T + D_S
     {
@@ -525,21 +551,23 @@ __global__ void __launch_bounds__(NTF, 1)
 
 template <int BV>
 cudaError_t launch_bwd_scan_tc_bv(const Problem& p, const Saved& sv, const bf16* dO,
-                                  const float* dST, float* dS0, bf16* dU, bf16* dh,
-                                  cudaStream_t st) {
+                                  const ScanSeg& sg, bf16* dU, bf16* dh, cudaStream_t st) {
+  const float* dST = sg.mode == 0 ? sg.S0 : nullptr;
+  float* dS0 = sg.ST;
   const size_t sm = sizeof(BScanSmem<BV>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_bwd_scan_tc<BV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const double nb = (double)p.B * p.H * p.NC, ntok = nb * C, heads = (double)p.B * p.H;
-  // reads W, Qh, Kt, M, dec, dO; writes dU, dh
+  // reads W, Qh, Kt, M, dec, dO; writes dU, dh (output pass) and the segment
+  // end / start gradients
   const double bytes = nb * (3.0 * kTileBytes + kMBytes + kDecBytes) + ntok * D * 2 +
-                       nb * ((double)kUBytes + kStateBytes) +
-                       heads * D * D * 4 * ((dST ? 1 : 0) + (dS0 ? 1 : 0));
+                       (sg.mode == 0 ? nb * ((double)kUBytes + kStateBytes) : 0.0) +
+                       heads * sg.G * D * D * 4 * ((dST ? 1 : 0) + (dS0 ? 1 : 0));
   const double flops = nb * (2.0 * C * C * D + 2.0 * C * D * D * 3);
   prof_begin(kKTcScanBwd, bytes, flops, st);
-  k_bwd_scan_tc<BV><<<dim3(D / BV, p.H, p.B), NTF, sm, st>>>(p, sv, dO, dST, dS0, dU, dh,
-                                                             device_error_word());
+  k_bwd_scan_tc<BV><<<dim3(D / BV, p.H, p.B * sg.G), NTF, sm, st>>>(p, sv, dO, sg, dU, dh,
+                                                                    device_error_word());
   e = cudaGetLastError();
   prof_end(st);
   return e;
@@ -551,15 +579,30 @@ cudaError_t launch_fwd_scan_tc(const Problem& p, const Saved& sv, const float* S
                                float* ST, bool save, cudaStream_t st) {
   // One CTA per (b, h, value tile): 64-row tiles while two per head still fit one wave
   // of the 148 SMs, whole-state tiles otherwise.
-  if ((long)p.B * p.H * 2 <= 148) return launch_fwd_scan_tc_bv<64>(p, sv, S0, o, ST, save, st);
-  return launch_fwd_scan_tc_bv<128>(p, sv, S0, o, ST, save, st);
+  const ScanSeg sg{1, p.NC, 0, S0, ST, nullptr};
+  if ((long)p.B * p.H * 2 <= 148) return launch_fwd_scan_tc_bv<64>(p, sv, sg, o, save, st);
+  return launch_fwd_scan_tc_bv<128>(p, sv, sg, o, save, st);
+}
+
+cudaError_t launch_fwd_scan_tc_seg(const Problem& p, const Saved& sv, const ScanSeg& sg, bf16* o,
+                                   bool save, int bv, cudaStream_t st) {
+  return bv == 64 ? launch_fwd_scan_tc_bv<64>(p, sv, sg, o, save, st)
+                  : launch_fwd_scan_tc_bv<128>(p, sv, sg, o, save, st);
 }
 
 cudaError_t launch_bwd_scan_tc(const Problem& p, const Saved& sv, const bf16* dO,
                                const float* dST, float* dS0, bf16* dU, bf16* dh,
                                cudaStream_t st) {
-  if ((long)p.B * p.H * 2 <= 148) return launch_bwd_scan_tc_bv<64>(p, sv, dO, dST, dS0, dU, dh, st);
-  return launch_bwd_scan_tc_bv<128>(p, sv, dO, dST, dS0, dU, dh, st);
+  const ScanSeg sg{1, p.NC, 0, dST, dS0, nullptr};
+  if ((long)p.B * p.H * 2 <= 148) return launch_bwd_scan_tc_bv<64>(p, sv, dO, sg, dU, dh, st);
+  return launch_bwd_scan_tc_bv<128>(p, sv, dO, sg, dU, dh, st);
+}
+
+cudaError_t launch_bwd_scan_tc_seg(const Problem& p, const Saved& sv, const bf16* dO,
+                                   const ScanSeg& sg, bf16* dU, bf16* dh, int bv,
+                                   cudaStream_t st) {
+  return bv == 64 ? launch_bwd_scan_tc_bv<64>(p, sv, dO, sg, dU, dh, st)
+                  : launch_bwd_scan_tc_bv<128>(p, sv, dO, sg, dU, dh, st);
 }
 
 }  // namespace fast

@@ -44,6 +44,7 @@ const char* kernel_name(int id) {
     case kKTcScanBwd: return "tc_scan_bwd";
     case kKTcChunkBwd: return "tc_chunk_bwd";
     case kKDecode: return "decode_step";
+    case kKAffine: return "affine_compose";
   }
   return "unknown";
 }

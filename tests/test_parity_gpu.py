@@ -180,3 +180,21 @@ def test_whole_state_scan_tiles():
                                                s0_std=0.1)
     _check(w, make_inputs(w), dST=random_state(w, seed=12, std=0.5),
            heads=[(0, 0), (3, 7), (7, 9)])
+
+
+# Long sequences with few heads take the chunk-parallel affine scan: segment
+# transfer matrices and offsets in parallel, composed across segments, then
+# the segments' output passes in parallel (forward and backward).
+@pytest.mark.parametrize("T", [4096, 4096 + 100])
+@pytest.mark.parametrize("name", ["kda_bf16_b4h16t8192", "kla_bf16_b1h16t65536",
+                                  "gdn_bf16_b4h8t2048"])
+def test_segmented_affine_scan(name, T):
+    w = WORKLOADS[name].with_(name=f"seg_{name}_T{T}", B=1, H=2, T=T, s0_std=0.1)
+    inp = make_inputs(w)
+    _check(w, inp, dST=random_state(w, seed=13, std=0.5))
+
+
+def test_segmented_affine_scan_recompute():
+    w = WORKLOADS["kda_bf16_b4h16t8192"].with_(name="seg_recompute", B=1, H=2, T=4096 + 33,
+                                               s0_std=0.1)
+    _check(w, make_inputs(w), dST=random_state(w, seed=14, std=0.5), save=False)
