@@ -235,16 +235,47 @@ __global__ void __launch_bounds__(NTB, 1)
     s.knorm[tid] = knorm_g[cb * C + tid];
   }
   frag::cp_commit();
-  frag::cp_wait<0>();
+  // the first value half of S and dS' (phase 1), in flight behind everything else
+  for (int idx = tid; idx < C * (D / 8); idx += NTB) {
+    const int a = idx >> 4, j = idx & 15;
+    frag::cp16(R0 + a * LDD + j * 8, hst + cb * D * D + (size_t)a * D + j * 8, true);
+    frag::cp16(R1 + a * LDD + j * 8, dhst + cb * D * D + (size_t)a * D + j * 8, true);
+  }
+  frag::cp_commit();
+  frag::cp_wait<1>();
   __syncthreads();
   // element (i, c) of the gate tile
   auto gat = [&](int i, int c) -> float& { return gk == D ? s.G[gsw(i, c)] : s.G[i]; };
-  if (tid < gk) {
-    float acc = 0.f;
-    for (int i = 0; i < C; ++i) {
-      acc += gat(i, tid);
-      gat(i, tid) = acc;
+  // cumulative gate down the chunk's rows
+  if (gk == D) {
+    // thread (column c, row quarter q): scan of 16 rows, then the quarter offsets
+    // (the key-column partials of the consume phase hold the quarter totals)
+    const int c = tid & 127, q = tid >> 7;
+    float run = 0.f;
+#pragma unroll
+    for (int i = 16 * q; i < 16 * q + 16; ++i) {
+      run += gat(i, c);
+      gat(i, c) = run;
     }
+    s.ktk[q * D + c] = run;
+    __syncthreads();
+    float off = 0.f;
+    for (int q2 = 0; q2 < q; ++q2) off += s.ktk[q2 * D + c];
+    if (q > 0) {
+#pragma unroll
+      for (int i = 16 * q; i < 16 * q + 16; ++i) gat(i, c) += off;
+    }
+  } else if (warp == 0) {
+    // rows 2 lane, 2 lane + 1: an inclusive scan across the warp
+    const float a0v = s.G[2 * lane], a1v = s.G[2 * lane + 1];
+    float x = a0v + a1v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    s.G[2 * lane + 1] = x;
+    s.G[2 * lane] = x - a1v;
   }
   __syncthreads();
 
@@ -314,12 +345,14 @@ __global__ void __launch_bounds__(NTB, 1)
   frag::zero(akt);
   frag::zero(adm);
   for (int ah = 0; ah < 2; ++ah) {
-    for (int idx = tid; idx < C * (D / 8); idx += NTB) {
-      const int a = idx >> 4, j = idx & 15;
-      frag::cp16(R0 + a * LDD + j * 8, hst + cb * D * D + (size_t)(ah * 64 + a) * D + j * 8, true);
-      frag::cp16(R1 + a * LDD + j * 8, dhst + cb * D * D + (size_t)(ah * 64 + a) * D + j * 8, true);
+    if (ah == 1) {
+      for (int idx = tid; idx < C * (D / 8); idx += NTB) {
+        const int a = idx >> 4, j = idx & 15;
+        frag::cp16(R0 + a * LDD + j * 8, hst + cb * D * D + (size_t)(64 + a) * D + j * 8, true);
+        frag::cp16(R1 + a * LDD + j * 8, dhst + cb * D * D + (size_t)(64 + a) * D + j * 8, true);
+      }
+      frag::cp_commit();
     }
-    frag::cp_commit();
     frag::cp_wait<0>();
     __syncthreads();
     // dQs += dO S ; dW' += dU S ; dKt += U dS'   (contraction over this half of a)

@@ -125,8 +125,23 @@ __global__ void __launch_bounds__(NT, 2)
       frag::cp16(G + i * D + j * 4, g + row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 4, ok);
     }
     frag::cp_commit();
-    frag::cp_wait<0>();
-  } else if (tid < C) {
+  }
+  // q into R3 (the factor pass rewrites it in place) and k into registers, in
+  // flight while the gate is summed; v follows after the factor pass.  Each
+  // thread owns the 16-byte column segment j = tid % 16 of ITEMS rows.
+  constexpr int ITEMS = C * (D / 8) / NT;
+  uint4 kr[ITEMS], vr[ITEMS];
+#pragma unroll
+  for (int it = 0; it < ITEMS; ++it) {
+    const int idx = tid + it * NT, i = idx >> 4, j = idx & 15;
+    const bool ok = i < nvalid;
+    const size_t rr = row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 8;
+    frag::cp16(s.R3 + i * LDD + j * 8, q + rr, ok);
+    kr[it] = ok ? *reinterpret_cast<const uint4*>(k + rr) : make_uint4(0, 0, 0, 0);
+  }
+  frag::cp_commit();
+  frag::cp_wait<0>();
+  if (gk != D && tid < C) {
     G[tid] = (tid < nvalid && p.gate != kGateNone) ? g[row_id(p, b, t0 + tid, h)] : 0.f;
   }
   __syncthreads();
@@ -135,39 +150,37 @@ __global__ void __launch_bounds__(NT, 2)
 
   // Factors: K^c, Kb^c, Q^c to shared memory; Qh, Kt, beta, dec to global.
   const int r = centre_row(nvalid);
-  constexpr int ITEMS = C * (D / 8) / NT;  // 16-byte row segments per thread
-  uint4 kr[ITEMS], qr[ITEMS], vr[ITEMS];
+  // per-column factors of this thread's segment: e^{-gamma_r}, e^{gamma_C - gamma_r}
+  float ier8[8], ecr8[8];
+  {
+    float r8[8], c8[8];
+    gate8(G, gk, r, (tid & 15) * 8, r8);
+    gate8(G, gk, C - 1, (tid & 15) * 8, c8);
 #pragma unroll
-  for (int it = 0; it < ITEMS; ++it) {
-    const int idx = tid + it * NT, i = idx >> 4, j = idx & 15;
-    kr[it] = qr[it] = vr[it] = make_uint4(0, 0, 0, 0);
-    if (i < nvalid) {
-      const size_t rr = row_id(p, b, t0 + i, h) * D + j * 8;
-      kr[it] = *reinterpret_cast<const uint4*>(k + rr);
-      qr[it] = *reinterpret_cast<const uint4*>(q + rr);
-      vr[it] = *reinterpret_cast<const uint4*>(v + rr);
+    for (int e = 0; e < 8; ++e) {
+      ier8[e] = __expf(-r8[e]);
+      ecr8[e] = __expf(c8[e] - r8[e]);
     }
   }
 #pragma unroll
   for (int it = 0; it < ITEMS; ++it) {
     const int idx = tid + it * NT, i = idx >> 4, j = idx & 15;
     const bool valid = i < nvalid;
-    const uint4 rk = kr[it], rq = qr[it];
-    float kv[8], qv[8], g8[8], r8[8], c8[8];
-    unpack8(rk, kv);
+    const uint4 rq = *reinterpret_cast<const uint4*>(s.R3 + i * LDD + j * 8);
+    float kv[8], qv[8], g8[8];
+    unpack8(kr[it], kv);
     unpack8(rq, qv);
     gate8(G, gk, i, j * 8, g8);
-    gate8(G, gk, r, j * 8, r8);
-    gate8(G, gk, C - 1, j * 8, c8);
     float kc[8], kb[8], qc[8], qh[8], kt[8], nn = 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const float ep = __expf(g8[e] - r8[e]), em = __expf(r8[e] - g8[e]);
+      const float eg = __expf(g8[e]);                              // e^gamma
+      const float ep = eg * ier8[e], em = __fdividef(1.f, ep);     // e^{+-(gamma - gamma_r)}
       kc[e] = kv[e] * ep;
       kb[e] = kv[e] * em;
       qc[e] = qv[e] * ep;
-      qh[e] = qv[e] * __expf(g8[e]);
-      kt[e] = kv[e] * __expf(c8[e] - g8[e]);
+      qh[e] = qv[e] * eg;
+      kt[e] = kb[e] * ecr8[e];  // k e^{gamma_C - gamma}
       nn += kv[e] * kv[e];
     }
     *reinterpret_cast<uint4*>(s.R1 + i * LDD + j * 8) = pack8(kc);
@@ -191,6 +204,13 @@ __global__ void __launch_bounds__(NT, 2)
     }
   }
   if (tid < D) sv.dec[cb * D + tid] = __expf(gk == D ? G[(C - 1) * D + tid] : G[C - 1]);
+#pragma unroll
+  for (int it = 0; it < ITEMS; ++it) {
+    const int idx = tid + it * NT, i = idx >> 4, j = idx & 15;
+    vr[it] = i < nvalid
+                 ? *reinterpret_cast<const uint4*>(v + row_id(p, b, t0 + i, h) * D + j * 8)
+                 : make_uint4(0, 0, 0, 0);
+  }
   __syncthreads();
 
   // [A ; M] = [K^c ; Q^c] Kb^c^T: warps 0-3 -> A rows 16w.., warps 4-7 -> M rows 16(w-4)..
