@@ -205,21 +205,15 @@ __global__ void __launch_bounds__(NTB, 1)
   bf16* sdA = s.U;
 
   // ---- loads: q (into Qc), k, dO, W, U', dU, U, T, gate, beta
+  // Loads in three cp.async groups, in the order of first use:
+  //   1: gate, q, k (gate scan, factor tile, Q^c)   2: dO, dU, U, first half of S and dS'
+  //   3 (issued after the first phase-1 half): second half of S and dS'; 4: W, U', T
   for (int idx = tid; idx < C * (D / 8); idx += NTB) {
     const int i = idx >> 4, j = idx & 15;
     const bool ok = i < nvalid;
     const size_t rr = row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 8;
     frag::cp16(s.Qc + i * LDD + j * 8, q + rr, ok);
     frag::cp16(s.k + i * LDD + j * 8, k + rr, ok);
-    frag::cp16(s.dO + i * LDD + j * 8, dO + rr, ok);
-  }
-  cp_linear<NTB>(s.dU, dUg + cb * C * D, C * D, tid);
-  cp_linear<NTB>(s.W, Wg + cb * C * D, C * D, tid);
-  cp_linear<NTB>(s.Up, Upg + cb * C * D, C * D, tid);
-  cp_linear<NTB>(s.U, Ug + cb * C * D, C * D, tid);
-  for (int idx = tid; idx < C * (C / 8); idx += NTB) {
-    const int i = idx >> 3, j = idx & 7;
-    frag::cp16(s.T + i * LDC + j * 8, Tg + cb * C * C + i * C + j * 8, true);
   }
   if (gk == D) {
     for (int idx = tid; idx < C * (D / 4); idx += NTB) {
@@ -235,7 +229,13 @@ __global__ void __launch_bounds__(NTB, 1)
     s.knorm[tid] = knorm_g[cb * C + tid];
   }
   frag::cp_commit();
-  // the first value half of S and dS' (phase 1), in flight behind everything else
+  for (int idx = tid; idx < C * (D / 8); idx += NTB) {
+    const int i = idx >> 4, j = idx & 15;
+    const bool ok = i < nvalid;
+    frag::cp16(s.dO + i * LDD + j * 8, dO + row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 8, ok);
+  }
+  cp_linear<NTB>(s.dU, dUg + cb * C * D, C * D, tid);
+  cp_linear<NTB>(s.U, Ug + cb * C * D, C * D, tid);
   for (int idx = tid; idx < C * (D / 8); idx += NTB) {
     const int a = idx >> 4, j = idx & 15;
     frag::cp16(R0 + a * LDD + j * 8, hst + cb * D * D + (size_t)a * D + j * 8, true);
@@ -352,8 +352,18 @@ __global__ void __launch_bounds__(NTB, 1)
         frag::cp16(R1 + a * LDD + j * 8, dhst + cb * D * D + (size_t)(64 + a) * D + j * 8, true);
       }
       frag::cp_commit();
+      // W, U' (phase 3) and T (phase 2) behind it
+      cp_linear<NTB>(s.W, Wg + cb * C * D, C * D, tid);
+      cp_linear<NTB>(s.Up, Upg + cb * C * D, C * D, tid);
+      for (int idx = tid; idx < C * (C / 8); idx += NTB) {
+        const int i = idx >> 3, j = idx & 7;
+        frag::cp16(s.T + i * LDC + j * 8, Tg + cb * C * C + i * C + j * 8, true);
+      }
+      frag::cp_commit();
+      frag::cp_wait<1>();
+    } else {
+      frag::cp_wait<0>();
     }
-    frag::cp_wait<0>();
     __syncthreads();
     // dQs += dO S ; dW' += dU S ; dKt += U dS'   (contraction over this half of a)
     // The half tiles hold local rows 0..63; mm_rows indexes B rows from k0 = 64ah.
@@ -433,6 +443,7 @@ __global__ void __launch_bounds__(NTB, 1)
         P[jt][2 + u] *= frc;
       }
   }
+  frag::cp_wait<0>();  // W, U', T
   __syncthreads();
 
   // ---- phase 2: Lambda = T^T [dU | dW]; dv = diag(beta) Lambda_U
