@@ -118,12 +118,15 @@ Ws carve(const Layout& L, void* base, int pass) {
   return w;
 }
 
-// The chunk-parallel backward has two implementations with identical results:
-// warp-level mma.sync tiles (default, 16 warps per CTA) and tcgen05 with TMEM
-// accumulators (DR_TCGEN05_BWD=1).
-bool use_tcgen05_chunk_bwd() {
+// The chunk-parallel backward has three implementations with identical
+// results: tcgen05 products with a 16-warp register epilogue (default),
+// warp-level mma.sync products with the same epilogue (DR_BWD_CHUNK=mma), and
+// tcgen05 with a 256-thread TMEM epilogue (DR_TCGEN05_BWD=1).
+int chunk_bwd_kind() {
   const char* e = getenv("DR_TCGEN05_BWD");
-  return e && e[0] == '1';
+  if (e && e[0] == '1') return 1;
+  const char* h = getenv("DR_BWD_CHUNK");
+  return (h && strcmp(h, "mma") == 0) ? 0 : 2;
 }
 
 // The two state scans likewise: tcgen05 with the state in registers and the
@@ -313,14 +316,14 @@ dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const 
       if (e != cudaSuccess) return DR_ERR_CUDA;
     }
     e = bwd_scan_any(P, sv, (const bf*)dO, dST, dS0, dU, dh, aff, st);
-    if (e == cudaSuccess)
-      e = use_tcgen05_chunk_bwd()
-              ? dr::fast::launch_bwd_chunk_tc(P, (const bf*)q, (const bf*)k, (const bf*)v,
-                                              (const bf*)dO, g, sv, dh, dU, (bf*)dq, (bf*)dk,
-                                              (bf*)dv, dbeta, dg, st)
-              : dr::fast::launch_bwd_chunk(P, (const bf*)q, (const bf*)k, (const bf*)v,
-                                           (const bf*)dO, g, sv, dh, dU, (bf*)dq, (bf*)dk,
-                                           (bf*)dv, dbeta, dg, st);
+    if (e == cudaSuccess) {
+      const int kind = chunk_bwd_kind();
+      auto launch = kind == 2 ? dr::fast::launch_bwd_chunk_hy
+                              : kind == 1 ? dr::fast::launch_bwd_chunk_tc
+                                          : dr::fast::launch_bwd_chunk;
+      e = launch(P, (const bf*)q, (const bf*)k, (const bf*)v, (const bf*)dO, g, sv, dh, dU,
+                 (bf*)dq, (bf*)dk, (bf*)dv, dbeta, dg, st);
+    }
     return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
   }
   if (p->dtype == DR_F32)

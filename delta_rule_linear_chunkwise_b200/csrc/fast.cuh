@@ -58,10 +58,10 @@ constexpr size_t kUBytes = kTileBytes;         // pseudo-values U / dU, bf16
 
 // The per-chunk tensors of the forward that the backward reuses ("saved"):
 // the state-independent chunk tiles written by tc_prep and the chunk start
-// states and pseudo-values written by the forward scan.  T and h are
-// row-major; the tiles marked [ct] are core-tiled (see ct_off).
+// states and pseudo-values written by the forward scan, all core-tiled (see
+// ct_off); the backward scan's dU and dh use the same layout.
 struct Saved {
-  __nv_bfloat16* T;    // [nb][64][64]    (I + A)^{-1}
+  __nv_bfloat16* T;    // [nb][64][64]    (I + A)^{-1}                         [ct]
   float* beta;         // [nb][64]        beta (Kaczmarz step applied)
   float* dec;          // [nb][128]       e^{gamma_C}
   __nv_bfloat16* W;    // [nb][64][128]   T diag(beta) k e^gamma               [ct]
@@ -69,7 +69,7 @@ struct Saved {
   __nv_bfloat16* M;    // [nb][64][64]    tril(Q^c Kb^c^T)                     [ct]
   __nv_bfloat16* Qh;   // [nb][64][128]   q e^gamma                            [ct]
   __nv_bfloat16* Kt;   // [nb][64][128]   k e^{gamma_C - gamma}                [ct]
-  __nv_bfloat16* h;    // [nb][128][128]  chunk start state S (value-major)
+  __nv_bfloat16* h;    // [nb][128][128]  chunk start state S [a][c]             [ct]
   __nv_bfloat16* U;    // [nb][64][128]   U = U' - W S^T                       [ct]
   float* knorm;        // [nb][64]        ||k||^2 of each row
   float* Pseg;         // [B][G][H][128][128] segment transfer matrices (affine scan; else null)
@@ -192,6 +192,14 @@ cudaError_t launch_bwd_chunk(const Problem& p, const __nv_bfloat16* q, const __n
                              __nv_bfloat16* dv, float* dbeta, float* dg, cudaStream_t st);
 
 cudaError_t launch_bwd_chunk_tc(const Problem& p, const __nv_bfloat16* q,
+                                const __nv_bfloat16* k, const __nv_bfloat16* v,
+                                const __nv_bfloat16* dO, const float* g, const Saved& sv,
+                                const __nv_bfloat16* dh, const __nv_bfloat16* dU,
+                                __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv,
+                                float* dbeta, float* dg, cudaStream_t st);
+
+// The same with the products on tcgen05 and the element-wise work on 16 warps.
+cudaError_t launch_bwd_chunk_hy(const Problem& p, const __nv_bfloat16* q,
                                 const __nv_bfloat16* k, const __nv_bfloat16* v,
                                 const __nv_bfloat16* dO, const float* g, const Saved& sv,
                                 const __nv_bfloat16* dh, const __nv_bfloat16* dU,

@@ -107,11 +107,9 @@ __global__ void __launch_bounds__(NTS, 1)
     frag::cp_wait<1>();
     __syncthreads();
     // dh_n: gradient of this chunk's end state
-    for (int idx = tid; idx < BV * (D / 8); idx += NTS) {
-      const int a = idx >> 4, j = idx & 15;
-      *reinterpret_cast<uint4*>(dhout + cb * D * D + (size_t)(a0 + a) * D + j * 8) =
-          *reinterpret_cast<const uint4*>(s.dS + a * LDD + j * 8);
-    }
+    for (int idx = tid; idx < BV * (D / 8); idx += NTS)  // core-tiled rows a0 ..
+      *reinterpret_cast<uint4*>(dhout + cb * D * D + ct_off(a0, 0, D) + 8 * idx) =
+          *reinterpret_cast<const uint4*>(s.dS + ct_row(idx, D) * LDD + ct_col(idx, D));
     // dU = M^T dO + Kt dS^T, rows i = 16rb.., values 32hf..
     {
       float du[4][4];
@@ -169,7 +167,7 @@ struct BchunkSmem {
   bf16 U[C * D];        // core-tiled; then dA [i][j] (stride LDC)
   bf16 dW[C * LDD];
   bf16 dM[C * LDC];     // tril(dO U^T)               [i][j]
-  bf16 T[C * LDC];
+  bf16 T[C * LDC];      // core-tiled [j][i]
   bf16 R[2 * C * LDD];  // S half | dS' half  ->  Lambda_U | Lambda_W
                         // -> Kb^c | beta K^c  ->  dgamma (fp32 [C][D])
   float beta[C];
@@ -236,11 +234,8 @@ __global__ void __launch_bounds__(NTB, 1)
   }
   cp_linear<NTB>(s.dU, dUg + cb * C * D, C * D, tid);
   cp_linear<NTB>(s.U, Ug + cb * C * D, C * D, tid);
-  for (int idx = tid; idx < C * (D / 8); idx += NTB) {
-    const int a = idx >> 4, j = idx & 15;
-    frag::cp16(R0 + a * LDD + j * 8, hst + cb * D * D + (size_t)a * D + j * 8, true);
-    frag::cp16(R1 + a * LDD + j * 8, dhst + cb * D * D + (size_t)a * D + j * 8, true);
-  }
+  cp_linear<NTB>(R0, hst + cb * D * D, C * D, tid);  // state rows 0 .. 63, core-tiled
+  cp_linear<NTB>(R1, dhst + cb * D * D, C * D, tid);
   frag::cp_commit();
   frag::cp_wait<1>();
   __syncthreads();
@@ -346,19 +341,13 @@ __global__ void __launch_bounds__(NTB, 1)
   frag::zero(adm);
   for (int ah = 0; ah < 2; ++ah) {
     if (ah == 1) {
-      for (int idx = tid; idx < C * (D / 8); idx += NTB) {
-        const int a = idx >> 4, j = idx & 15;
-        frag::cp16(R0 + a * LDD + j * 8, hst + cb * D * D + (size_t)(64 + a) * D + j * 8, true);
-        frag::cp16(R1 + a * LDD + j * 8, dhst + cb * D * D + (size_t)(64 + a) * D + j * 8, true);
-      }
+      cp_linear<NTB>(R0, hst + cb * D * D + C * D, C * D, tid);  // rows 64 .. 127
+      cp_linear<NTB>(R1, dhst + cb * D * D + C * D, C * D, tid);
       frag::cp_commit();
       // W, U' (phase 3) and T (phase 2) behind it
       cp_linear<NTB>(s.W, Wg + cb * C * D, C * D, tid);
       cp_linear<NTB>(s.Up, Upg + cb * C * D, C * D, tid);
-      for (int idx = tid; idx < C * (C / 8); idx += NTB) {
-        const int i = idx >> 3, j = idx & 7;
-        frag::cp16(s.T + i * LDC + j * 8, Tg + cb * C * C + i * C + j * 8, true);
-      }
+      cp_linear<NTB>(s.T, Tg + cb * C * C, C * C, tid);
       frag::cp_commit();
       frag::cp_wait<1>();
     } else {
@@ -366,12 +355,13 @@ __global__ void __launch_bounds__(NTB, 1)
     }
     __syncthreads();
     // dQs += dO S ; dW' += dU S ; dKt += U dS'   (contraction over this half of a)
-    // The half tiles hold local rows 0..63; mm_rows indexes B rows from k0 = 64ah.
-    const bf16* Sh = R0 - ah * 64 * LDD;
-    const bf16* dSh = R1 - ah * 64 * LDD;
-    frag::mm_rows<4, 4, true>(zq, s.dO, LDD, rb * 16, Sh, LDD, qt * 32, ah * 64);
-    frag::mm_rows<4, 4, true>(adw, s.dU, CTD, rb * 16, Sh, LDD, qt * 32, ah * 64);
-    frag::mm_rows<4, 4, true>(akt, s.U, CTD, rb * 16, dSh, LDD, qt * 32, ah * 64);
+    // The half tiles hold local rows 0..63 (core-tiled); mm_rows indexes B rows
+    // from k0 = 64ah.
+    const bf16* Sh = R0 - ah * 64 * D;
+    const bf16* dSh = R1 - ah * 64 * D;
+    frag::mm_rows<4, 4, true>(zq, s.dO, LDD, rb * 16, Sh, CTD, qt * 32, ah * 64);
+    frag::mm_rows<4, 4, true>(adw, s.dU, CTD, rb * 16, Sh, CTD, qt * 32, ah * 64);
+    frag::mm_rows<4, 4, true>(akt, s.U, CTD, rb * 16, dSh, CTD, qt * 32, ah * 64);
     // dM += dO U^T  (U stored [j][a] = [n][k])
     frag::mm_rows<2, 4, false>(adm, s.dO, LDD, rb * 16, s.U, CTD, qt * 16, ah * 64);
     // colsum(dS' .* S) over this half: thread -> column c, row quarter rq
@@ -380,7 +370,7 @@ __global__ void __launch_bounds__(NTB, 1)
       float acc = 0.f;
 #pragma unroll 4
       for (int a = rq * 16; a < rq * 16 + 16; ++a)
-        acc += __bfloat162float(R0[a * LDD + c]) * __bfloat162float(R1[a * LDD + c]);
+        acc += __bfloat162float(R0[ct_off(a, c, D)]) * __bfloat162float(R1[ct_off(a, c, D)]);
       s.dgc[rq * D + c] = (ah == 0 ? 0.f : s.dgc[rq * D + c]) + acc;
     }
     __syncthreads();
@@ -458,7 +448,7 @@ __global__ void __launch_bounds__(NTB, 1)
         vv[jt][hh] = *reinterpret_cast<const uint32_t*>(v + rowg[hh] + qt * 32 + jt * 8 + lc);
     float lu[4][4];
     frag::zero(lu);
-    frag::mm_rows_at<4, 4, true>(lu, s.T, LDC, rb * 16, s.dU, CTD, qt * 32);
+    frag::mm_rows_at<4, 4, true>(lu, s.T, CTC, rb * 16, s.dU, CTD, qt * 32);
 #pragma unroll
     for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
@@ -473,7 +463,7 @@ __global__ void __launch_bounds__(NTB, 1)
       }
     frag::st_c(lu, R0, LDD, rb * 16, qt * 32);
     frag::zero(Q);
-    frag::mm_rows_at<4, 4, true>(Q, s.T, LDC, rb * 16, s.dW, LDD, qt * 32);
+    frag::mm_rows_at<4, 4, true>(Q, s.T, CTC, rb * 16, s.dW, LDD, qt * 32);
     frag::st_c(Q, R1, LDD, rb * 16, qt * 32);
 #pragma unroll
     for (int jt = 0; jt < 4; ++jt)

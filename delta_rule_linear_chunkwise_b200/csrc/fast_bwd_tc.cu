@@ -72,13 +72,10 @@ __device__ __forceinline__ bf16* slot(TcSmem& s, int kb) {
 }
 
 // cp.async of a row-major bf16 global tile into a K-major canonical tile
-// [R x Ncol] (rows = M/N, columns = K), or into an MN-major tile [K x N].
+// [R x Ncol] (rows = M/N, columns = K).
 __device__ __forceinline__ void ld_kmaj(bf16* t, const bf16* g, size_t ld, int R, int Ncol,
                                         int valid_rows = 1 << 30) {
   tc::cp_core_tile<NTT>(t, g, ld, R, Ncol, valid_rows, threadIdx.x);
-}
-__device__ __forceinline__ void ld_mnmaj(bf16* t, const bf16* g, size_t ld, int K, int N) {
-  tc::cp_core_tile<NTT>(t, g, ld, K, N, 1 << 30, threadIdx.x);
 }
 
 __device__ __forceinline__ uint32_t tmem_lane_addr(uint32_t base, int warp, int col) {
@@ -145,8 +142,8 @@ __global__ void __launch_bounds__(NTT, 1)
   ld_kmaj(slot(s, A_DO), dO + tokrow, tstride, C, D, nvalid);
   cp_linear<NTT>(slot(s, A_DU), dUg + cb * C * D, C * D, tid);
   cp_linear<NTT>(slot(s, A_U), sv.U + cb * C * D, C * D, tid);
-  ld_mnmaj(slot(s, A_SE), sv.h + cb * D * D, D, D, D);
-  ld_mnmaj(slot(s, A_DS), dhst + cb * D * D, D, D, D);
+  cp_linear<NTT>(slot(s, A_SE), sv.h + cb * D * D, D * D, tid);
+  cp_linear<NTT>(slot(s, A_DS), dhst + cb * D * D, D * D, tid);
   for (int idx = tid; idx < C * (D / 8); idx += NTT) {
     const int i = idx >> 4, j = idx & 15;
     const bool ok = i < nvalid;
@@ -318,7 +315,7 @@ __global__ void __launch_bounds__(NTT, 1)
   bool ok = level_wait(s, 0);
   if (!ok) goto fail;
   // L1/L2 operands and raw q into the freed arena (overlaps the L0 epilogue)
-  ld_mnmaj(slot(s, A_TT), sv.T + cb * C * C, C, C, C);
+  cp_linear<NTT>(slot(s, A_TT), sv.T + cb * C * C, C * C, tid);
   cp_linear<NTT>(slot(s, A_DUM), dUg + cb * C * D, C * D, tid);
   cp_linear<NTT>(slot(s, A_UP), sv.Up + cb * C * D, C * D, tid);
   cp_linear<NTT>(slot(s, A_W), sv.W + cb * C * D, C * D, tid);

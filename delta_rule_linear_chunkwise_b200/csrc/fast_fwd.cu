@@ -316,10 +316,10 @@ __global__ void __launch_bounds__(NT, 2)
   }
   // T -> bf16: global and the tensor-core A operand (over the dead A tile)
   for (int idx = tid; idx < C * C / 8; idx += NT) {
-    const int i = idx >> 3, j = idx & 7;
-    const uint4 val = pack8(sT + i * LDA + j * 8);
-    *reinterpret_cast<uint4*>(sv.T + cb * C * C + i * C + j * 8) = val;
-    *reinterpret_cast<uint4*>(sTb + i * LDC + j * 8) = val;
+    const int i = ct_row(idx, C), j8 = ct_col(idx, C);
+    const uint4 val = pack8(sT + i * LDA + j8);
+    *reinterpret_cast<uint4*>(sv.T + cb * C * C + 8 * idx) = val;  // core-tiled
+    *reinterpret_cast<uint4*>(sTb + i * LDC + j8) = val;
   }
   __syncthreads();
   // W = T (beta k e^gamma) (warps 0-3), U' = T (beta v) (warps 4-7): rows 16rb.., 128 columns
@@ -392,12 +392,10 @@ __global__ void __launch_bounds__(NT, 1)
     FwdStage& st = s.st[n & 1];
     frag::cp_wait<1>();
     __syncthreads();
-    if (save)
-      for (int idx = tid; idx < BV * (D / 8); idx += NT) {
-        const int a = idx >> 4, j = idx & 15;
-        *reinterpret_cast<uint4*>(sv.h + cb * D * D + (size_t)(a0 + a) * D + j * 8) =
-            *reinterpret_cast<const uint4*>(s.S + a * LDD + j * 8);
-      }
+    if (save)  // rows a0 .. a0 + 63 of the core-tiled state: one contiguous block
+      for (int idx = tid; idx < BV * (D / 8); idx += NT)
+        *reinterpret_cast<uint4*>(sv.h + cb * D * D + ct_off(a0, 0, D) + 8 * idx) =
+            *reinterpret_cast<const uint4*>(s.S + ct_row(idx, D) * LDD + ct_col(idx, D));
     // U = U' - W S^T and the inter-chunk part of O; rows 16rb.., values 32hf..
     float oc[4][4], u[4][4];
     {

@@ -72,6 +72,38 @@ __device__ __forceinline__ void scan_issue(const Problem& p, ScanStage<BV>& s, c
   if (tid < D / 4) frag::cp16(s.dec + 4 * tid, sv.dec + cb * D + 4 * tid, true);
 }
 
+// Writes this thread's HB state values x[u] (rows a0h + u, key c; one key per
+// lane) as bf16 into a core-tiled [128][128] state tile.  Each 8 x 8 block is
+// transposed across the 8 lanes that hold its keys (xor shuffles), so every
+// lane stores 16 contiguous bytes (row a, keys c0 .. c0 + 7) and a warp writes
+// four whole 128-byte core matrices.
+template <int HB>
+__device__ __forceinline__ void store_state_ct(bf16* dst, const float* x, int a0h, int c,
+                                               int lane) {
+#pragma unroll
+  for (int u8 = 0; u8 < HB / 8; ++u8) {
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = x[8 * u8 + j];
+#pragma unroll
+    for (int sh = 1; sh < 8; sh <<= 1) {
+      const bool hi = lane & sh;
+#pragma unroll
+      for (int j0 = 0; j0 < 8; ++j0) {
+        if (j0 & sh) continue;
+        const int j1 = j0 | sh;
+        const float y = __shfl_xor_sync(0xffffffffu, hi ? v[j0] : v[j1], sh);
+        if (hi) v[j0] = y;
+        else v[j1] = y;
+      }
+    }
+    const int a = a0h + 8 * u8 + (lane & 7);
+    *reinterpret_cast<uint4*>(dst + ct_off(a, c & ~7, D)) =
+        make_uint4(frag::pack(v[0], v[1]), frag::pack(v[2], v[3]), frag::pack(v[4], v[5]),
+                   frag::pack(v[6], v[7]));
+  }
+}
+
 __device__ __forceinline__ uint32_t lane_addr(uint32_t base, int warp, int col) {
   return base + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)col;
 }
@@ -144,18 +176,9 @@ __global__ void __launch_bounds__(NTF, 1)
                      frag::pack(f[6], f[7]));
     }
   };
-  // h_n[a][c] (bf16) from the registers: lanes c, c + 1 swap so each stores a pair
+  // h_n (bf16, core-tiled [a][c]) from the registers
   auto store_h = [&](size_t cbn) {
-    bf16* hp = sv.h + cbn * D * D;
-#pragma unroll
-    for (int u = 0; u < HB; u += 2) {
-      const float x = (lane & 1) ? S[u] : S[u + 1];
-      const float y = __shfl_xor_sync(0xffffffffu, x, 1);
-      const int a = a0 + ah * HB + u + (lane & 1);
-      const int cc = c & ~1;
-      const uint32_t v = (lane & 1) ? frag::pack(y, S[u + 1]) : frag::pack(S[u], y);
-      *reinterpret_cast<uint32_t*>(hp + (size_t)a * D + cc) = v;
-    }
+    store_state_ct<HB>(sv.h + cbn * D * D, S, a0 + ah * HB, c, lane);
   };
   // o rows of chunk nn from D_A buffer `buf` (warps on lanes 64 .. 127)
   auto store_o = [&](int nn, int buf) {
@@ -420,17 +443,9 @@ __global__ void __launch_bounds__(NTF, 1)
                      frag::pack(f[6], f[7]));
     }
   };
-  // dh (bf16, [a][c]) from the registers: lanes c, c + 1 swap so each stores a pair
+  // dh (bf16, core-tiled [a][c]) from the registers
   auto store_dh = [&](size_t cbn) {
-    bf16* hp = dhout + cbn * D * D;
-#pragma unroll
-    for (int u = 0; u < HB; u += 2) {
-      const float x = (lane & 1) ? dS[u] : dS[u + 1];
-      const float y = __shfl_xor_sync(0xffffffffu, x, 1);
-      const int a = a0 + ah * HB + u + (lane & 1);
-      const uint32_t v = (lane & 1) ? frag::pack(y, dS[u + 1]) : frag::pack(dS[u], y);
-      *reinterpret_cast<uint32_t*>(hp + (size_t)a * D + (c & ~1)) = v;
-    }
+    store_state_ct<HB>(dhout + cbn * D * D, dS, a0 + ah * HB, c, lane);
   };
 
   write_dsb();

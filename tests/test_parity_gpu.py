@@ -126,12 +126,13 @@ def test_full_size_workloads_sampled_heads(name):
 # The bf16 head-dim-128 tensor-core path at ragged lengths, with both chunk
 # backward kernels: the warp-level mma.sync one (default) and the tcgen05/TMEM
 # one (selected by DR_TCGEN05_BWD=1).
-BWD_VARIANTS = ["mma_sync", "tcgen05"]
+BWD_VARIANTS = ["mma_sync", "tcgen05", "hybrid"]
 
 
 @pytest.fixture(params=BWD_VARIANTS)
 def bwd_variant(request, monkeypatch):
     monkeypatch.setenv("DR_TCGEN05_BWD", "1" if request.param == "tcgen05" else "0")
+    monkeypatch.setenv("DR_BWD_CHUNK", "mma" if request.param == "mma_sync" else "")
     return request.param
 
 
@@ -198,3 +199,17 @@ def test_segmented_affine_scan_recompute():
     w = WORKLOADS["kda_bf16_b4h16t8192"].with_(name="seg_recompute", B=1, H=2, T=4096 + 33,
                                                s0_std=0.1)
     _check(w, make_inputs(w), dST=random_state(w, seed=14, std=0.5), save=False)
+
+
+@pytest.mark.parametrize("w", SMALL[1:5], ids=lambda w: w.name)
+def test_mma_sync_backward_small_workloads(w, monkeypatch):
+    monkeypatch.setenv("DR_BWD_CHUNK", "mma")
+    inp = make_inputs(w)
+    _check(w, inp, dST=random_state(w, seed=99, std=0.5))
+    _check(w, inp, save=False)
+
+
+def test_mma_sync_backward_full_size_sampled_heads(monkeypatch):
+    monkeypatch.setenv("DR_BWD_CHUNK", "mma")
+    w = WORKLOADS["kda_bf16_b4h16t8192"]
+    _check(w, make_inputs(w), heads=[(0, 0), (w.B - 1, w.H - 1)])
