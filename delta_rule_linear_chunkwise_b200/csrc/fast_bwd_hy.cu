@@ -13,7 +13,8 @@
 //
 // Each level is a set of tcgen05.mma (M = 64, operands in shared memory in the
 // canonical core-matrix layout, fp32 accumulators in tensor memory) issued by
-// one thread.  An M = 64 accumulator occupies lanes 16 q .. 16 q + 15 of each
+// one thread, independent accumulation chains interleaved (long chains split
+// into partial sums).  An M = 64 accumulator occupies lanes 16 q .. 16 q + 15 of each
 // 32-lane quadrant q, and tcgen05.ld.16x256b returns it to the warps of that
 // quadrant in exactly the register fragment of a warp-level m16n8 product
 // (thread t: row t / 4 and t / 4 + 8, columns 2 (t % 4), + 1 of each 8-column
@@ -45,8 +46,8 @@ __device__ __forceinline__ int gsw(int i, int c) { return i * D + (c ^ ((i & 7) 
 // later levels reuse them once the earlier accumulators are in registers.
 constexpr uint32_t T_ZQ = 0, T_ADW = 128, T_AKT = 256, T_ADM = 384;
 constexpr uint32_t T_LU = 0, T_LW = 128;
-constexpr uint32_t T_DA = 256;
-constexpr uint32_t T_Z2 = 0, T_X = 128, T_Y = 256;
+constexpr uint32_t T_DA = 256;  // four 64-column partial sums of dA
+constexpr uint32_t T_Z2 = 0, T_X = 128, T_Y = 256, T_Y2 = 384;
 
 struct HySmem {
   bf16 SS[D * D];   // S = h_n [a][c], core-tiled (MN-major B);  then Lambda_U | Lambda_W;
@@ -71,16 +72,49 @@ struct HySmem {
   uint32_t tmem;
 };
 
-// KS k-steps of D[tm] (+)= A B (M = 64); A: K-major [64][K] or MN-major [K][64],
-// B: K-major [N][K] or MN-major [K][N] (extents: a_dim = K or 64, b_dim = K or N).
-__device__ __forceinline__ void issue_mma(uint32_t tm, const bf16* A, bool a_mn, int a_dim,
-                                          const bf16* B, bool b_mn, int b_dim, int N, int KS,
-                                          bool acc_first) {
-  const uint32_t id = tc::idesc_bf16(64, N, a_mn, b_mn);
-  for (int ks = 0; ks < KS; ++ks) {
-    const uint64_t a = a_mn ? tc::sdesc_mnmaj(A, 64, ks) : tc::sdesc_kmaj(A, a_dim, ks);
-    const uint64_t b = b_mn ? tc::sdesc_mnmaj(B, b_dim, ks) : tc::sdesc_kmaj(B, b_dim, ks);
-    tc::mma(tm, a, b, id, (ks > 0 || acc_first) ? 1u : 0u);
+// One product chain D[tm] (+)= A B (M = 64) over k-steps ks0, ks0 + kstride, ...
+// (count of them); A: K-major [64][K] (a_dim = K) or MN-major [K][64], B: K-major
+// [N][K] (b_dim = K) or MN-major [K][N] (b_dim = N).  The first step overwrites
+// the accumulator.
+struct Chain {
+  uint32_t tm;
+  uint64_t a0, b0;     // descriptors of k-step 0
+  uint32_t da, db;     // descriptor start-address advance per k-step (16-byte units)
+  uint32_t id;
+  int ks0, kstride, count;
+};
+__device__ __forceinline__ Chain chain(uint32_t tm, const bf16* A, bool a_mn, int a_dim,
+                                       const bf16* B, bool b_mn, int b_dim, int N, int ks0,
+                                       int kstride, int count) {
+  Chain c;
+  c.tm = tm;
+  c.a0 = a_mn ? tc::sdesc_mnmaj(A, 64, 0) : tc::sdesc_kmaj(A, a_dim, 0);
+  c.b0 = b_mn ? tc::sdesc_mnmaj(B, b_dim, 0) : tc::sdesc_kmaj(B, b_dim, 0);
+  c.da = a_mn ? 2 * (64 / 8) * 128 / 16 : 256 / 16;
+  c.db = b_mn ? 2 * (b_dim / 8) * 128 / 16 : 256 / 16;
+  c.id = tc::idesc_bf16(64, N, a_mn, b_mn);
+  c.ks0 = ks0;
+  c.kstride = kstride;
+  c.count = count;
+  return c;
+}
+// Issue the chains round-robin by step: a tcgen05.mma that accumulates into
+// the same tensor memory waits for the previous one (about 190 cycles for
+// M = 64, measured), so independent chains are interleaved to overlap.
+template <int NC>
+__device__ __forceinline__ void issue_chains(const Chain (&cs)[NC]) {
+  int steps = 0;
+#pragma unroll
+  for (int i = 0; i < NC; ++i) steps = max(steps, cs[i].count);
+  for (int j = 0; j < steps; ++j) {
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+      if (j < cs[i].count) {
+        const uint32_t ks = (uint32_t)(cs[i].ks0 + j * cs[i].kstride);
+        tc::mma(cs[i].tm, cs[i].a0 + ks * cs[i].da, cs[i].b0 + ks * cs[i].db, cs[i].id,
+                j > 0 ? 1u : 0u);
+      }
+    }
   }
 }
 
@@ -291,10 +325,11 @@ __global__ void __launch_bounds__(NTB, 1)
 
   // ---- level 1 (tensor memory): dQs = dO S, dW' = dU S, dKt = U dS', dM = dO U^T
   if (tid == 0) {
-    issue_mma(tb + T_ZQ, s.DO, false, D, s.SS, true, D, 128, D / 16, false);
-    issue_mma(tb + T_ADW, s.DU, false, D, s.SS, true, D, 128, D / 16, false);
-    issue_mma(tb + T_AKT, s.UU, false, D, s.SD, true, D, 128, D / 16, false);
-    issue_mma(tb + T_ADM, s.DO, false, D, s.UU, false, D, 64, D / 16, false);
+    const Chain cs[4] = {chain(tb + T_ZQ, s.DO, false, D, s.SS, true, D, 128, 0, 1, D / 16),
+                         chain(tb + T_ADW, s.DU, false, D, s.SS, true, D, 128, 0, 1, D / 16),
+                         chain(tb + T_AKT, s.UU, false, D, s.SD, true, D, 128, 0, 1, D / 16),
+                         chain(tb + T_ADM, s.DO, false, D, s.UU, false, D, 64, 0, 1, D / 16)};
+    issue_chains(cs);
     tc::commit(&s.bar);
   }
   // colsum(dS' .* S) while they run: thread -> column c, row quarter rq
@@ -384,8 +419,9 @@ __global__ void __launch_bounds__(NTB, 1)
 
   // ---- level 2: Lambda = T^T [dU | dW]; dv = diag(beta) Lambda_U
   if (tid == 0) {
-    issue_mma(tb + T_LU, s.TT, true, C, s.DU, true, D, 128, C / 16, false);
-    issue_mma(tb + T_LW, s.TT, true, C, sdW, true, D, 128, C / 16, false);
+    const Chain cs[2] = {chain(tb + T_LU, s.TT, true, C, s.DU, true, D, 128, 0, 1, C / 16),
+                         chain(tb + T_LW, s.TT, true, C, sdW, true, D, 128, 0, 1, C / 16)};
+    issue_chains(cs);
     tc::commit(&s.bar);
   }
   float dbrow[2] = {0.f, 0.f};  // this thread's d(beta_eff) partials for rows i0, i0 + 8
@@ -435,15 +471,26 @@ __global__ void __launch_bounds__(NTB, 1)
 
   // ---- level 3: dA = -strict_tril(Lambda_U U'^T + Lambda_W W^T), rows 16rb.., cols 16qt..
   if (tid == 0) {
-    issue_mma(tb + T_DA, sLU, false, D, sUp, false, D, 64, D / 16, false);
-    issue_mma(tb + T_DA, sLW, false, D, sW, false, D, 64, D / 16, true);
+    const Chain cs[4] = {chain(tb + T_DA, sLU, false, D, sUp, false, D, 64, 0, 2, D / 32),
+                         chain(tb + T_DA + 64, sLU, false, D, sUp, false, D, 64, 1, 2, D / 32),
+                         chain(tb + T_DA + 128, sLW, false, D, sW, false, D, 64, 0, 2, D / 32),
+                         chain(tb + T_DA + 192, sLW, false, D, sW, false, D, 64, 1, 2, D / 32)};
+    issue_chains(cs);
     tc::commit(&s.bar);
   }
   ok = hy_wait(&s.bar, 2);
   if (!ok) break;
   {
-    float da[2][4];
+    float da[2][4], dp[2][4];
     frag_ld2(tb + T_DA + 16 * qt, warp, da);
+#pragma unroll
+    for (int part = 1; part < 4; ++part) {
+      frag_ld2(tb + T_DA + 64 * part + 16 * qt, warp, dp);
+#pragma unroll
+      for (int jt = 0; jt < 2; ++jt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) da[jt][e] += dp[jt][e];
+    }
 #pragma unroll
     for (int jt = 0; jt < 2; ++jt)
 #pragma unroll
@@ -478,10 +525,11 @@ __global__ void __launch_bounds__(NTB, 1)
   tc::fence_after_sync();
   // ---- level 4: dM Kb^c, dA Kb^c, dM^T Q^c + dA^T beta K^c
   if (tid == 0) {
-    issue_mma(tb + T_Z2, sdM, false, C, sKb, true, D, 128, C / 16, false);
-    issue_mma(tb + T_X, sdA, false, C, sKb, true, D, 128, C / 16, false);
-    issue_mma(tb + T_Y, sdM, true, C, s.QC, true, D, 128, C / 16, false);
-    issue_mma(tb + T_Y, sdA, true, C, sBk, true, D, 128, C / 16, true);
+    const Chain cs[4] = {chain(tb + T_Z2, sdM, false, C, sKb, true, D, 128, 0, 1, C / 16),
+                         chain(tb + T_X, sdA, false, C, sKb, true, D, 128, 0, 1, C / 16),
+                         chain(tb + T_Y, sdM, true, C, s.QC, true, D, 128, 0, 1, C / 16),
+                         chain(tb + T_Y2, sdA, true, C, sBk, true, D, 128, 0, 1, C / 16)};
+    issue_chains(cs);
     tc::commit(&s.bar);
   }
   ok = hy_wait(&s.bar, 3);
@@ -499,6 +547,11 @@ __global__ void __launch_bounds__(NTB, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) Q[j][e] += t4[j][e];
     frag_ld4(tb + T_Y + 32 * qt, warp, t4);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) P[j][e] += t4[j][e];
+    frag_ld4(tb + T_Y2 + 32 * qt, warp, t4);
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll

@@ -123,10 +123,11 @@ def test_full_size_workloads_sampled_heads(name):
     print(name, {k: f"{v:.2e}" for k, v in errs.items()})
 
 
-# The bf16 head-dim-128 tensor-core path at ragged lengths, with both chunk
-# backward kernels: the warp-level mma.sync one (default) and the tcgen05/TMEM
-# one (selected by DR_TCGEN05_BWD=1).
-BWD_VARIANTS = ["mma_sync", "tcgen05", "hybrid"]
+# The bf16 head-dim-128 tensor-core path at ragged lengths, with each chunk
+# backward kernel: tcgen05 products with the 16-warp register epilogue
+# (default), the warp-level mma.sync one (DR_BWD_CHUNK=mma) and the tcgen05
+# one with a TMEM epilogue (DR_TCGEN05_BWD=1).
+BWD_VARIANTS = ["mma_sync", "tcgen05", "default"]
 
 
 @pytest.fixture(params=BWD_VARIANTS)
