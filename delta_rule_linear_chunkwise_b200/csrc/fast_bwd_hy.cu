@@ -36,6 +36,7 @@ namespace {
 constexpr int C = 64, D = 128;
 constexpr int LDD = D + 8;
 constexpr int NTB = 512;
+constexpr int LDG = D + 4;  // fp32 row stride of the dgamma tile (fragment stores conflict-free)
 constexpr uint32_t kSpinHy = 1u << 22;
 
 __device__ __forceinline__ int centre_row(int nvalid) { return (nvalid - 1) / 2; }
@@ -71,6 +72,10 @@ struct HySmem {
   uint64_t bar;
   uint32_t tmem;
 };
+
+static_assert(offsetof(HySmem, SD) == offsetof(HySmem, SS) + sizeof(bf16) * D * D &&
+                  sizeof(float) * C * LDG <= sizeof(bf16) * 2 * D * D,
+              "the padded dgamma tile spans the adjacent S and dS' tiles");
 
 // One product chain D[tm] (+)= A B (M = 64) over k-steps ks0, ks0 + kstride, ...
 // (count of them); A: K-major [64][K] (a_dim = K) or MN-major [K][64], B: K-major
@@ -332,16 +337,38 @@ __global__ void __launch_bounds__(NTB, 1)
     issue_chains(cs);
     tc::commit(&s.bar);
   }
-  // colsum(dS' .* S) while they run: thread -> column c, row quarter rq
+  // colsum(dS' .* S) while they run: thread -> 8 columns (16-byte core rows),
+  // 4 rows (one per row group of its quarter); eight lanes read the eight rows
+  // of one core matrix (128 contiguous bytes, no bank conflicts)
   {
-    const int c = tid & 127, rq = tid >> 7;
-    float acc = 0.f;
-#pragma unroll 4
-    for (int a = rq * 32; a < rq * 32 + 32; ++a) {
-      const int o = tc::mnmaj_off(a, c, D);
-      acc += __bfloat162float(s.SS[o]) * __bfloat162float(s.SD[o]);
+    const int alo = tid & 7, cg = (tid >> 3) & 15, ag = tid >> 7;
+    float acc[8] = {};
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int o = ct_off((ag * 4 + r) * 8 + alo, 8 * cg, D);
+      const uint4 x = *reinterpret_cast<const uint4*>(s.SS + o);
+      const uint4 y = *reinterpret_cast<const uint4*>(s.SD + o);
+      const uint32_t* wx = reinterpret_cast<const uint32_t*>(&x);
+      const uint32_t* wy = reinterpret_cast<const uint32_t*>(&y);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fx = frag::unpack(wx[e]), fy = frag::unpack(wy[e]);
+        acc[2 * e] += fx.x * fy.x;
+        acc[2 * e + 1] += fx.y * fy.y;
+      }
     }
-    s.dgc[rq * D + c] = acc;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float x = acc[e];
+      x += __shfl_xor_sync(0xffffffffu, x, 1);
+      x += __shfl_xor_sync(0xffffffffu, x, 2);
+      x += __shfl_xor_sync(0xffffffffu, x, 4);
+      acc[e] = x;
+    }
+    if (alo == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s.dgc[ag * D + 8 * cg + e] = acc[e];
+    }
   }
   ok = hy_wait(&s.bar, 0);
   if (!ok) break;
@@ -598,14 +625,14 @@ __global__ void __launch_bounds__(NTB, 1)
     xx += __shfl_xor_sync(0xffffffffu, xx, 2);
     if ((lane & 3) == 0) s.dbp[(i0 + hh * 8) * 4 + qt] = xx;
   }
-  __syncthreads();  // the S tile region is free: reuse for the dgamma reduction
+  __syncthreads();  // the S and dS' tile regions are free: the dgamma tile (row stride LDG)
   float* sdg = reinterpret_cast<float*>(s.SS);
   if (gk == D) {
 #pragma unroll
     for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        sdg[(i0 + (e >> 1) * 8) * D + qt * 32 + jt * 8 + lc + (e & 1)] = Q[jt][e];
+        sdg[(i0 + (e >> 1) * 8) * LDG + qt * 32 + jt * 8 + lc + (e & 1)] = Q[jt][e];
   } else {
     // scalar gate: the row sums of dgamma, one slot per column quarter
 #pragma unroll
@@ -625,7 +652,7 @@ __global__ void __launch_bounds__(NTB, 1)
   if (gk == D) {
     float part = 0.f;
 #pragma unroll 4
-    for (int i = grq * 16; i < grq * 16 + 16; ++i) part += sdg[i * D + gc];
+    for (int i = grq * 16; i < grq * 16 + 16; ++i) part += sdg[i * LDG + gc];
     s.dgc[grq * D + gc] = part;  // the chunk-end term read dgc before the last two barriers
   }
   if (tid < C) s.dbp[tid * 4] = dbt;  // total d(beta_eff) of row tid
@@ -655,7 +682,7 @@ __global__ void __launch_bounds__(NTB, 1)
     for (int q2 = grq + 1; q2 < 4; ++q2) run += s.dgc[q2 * D + gc];
 #pragma unroll 4
     for (int i = grq * 16 + 15; i >= grq * 16; --i) {
-      run += sdg[i * D + gc];
+      run += sdg[i * LDG + gc];
       if (i < nvalid) dg[row_id(p, b, t0 + i, h) * D + gc] = run;
     }
   } else if (p.gate != kGateNone && warp == 0) {
