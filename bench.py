@@ -47,6 +47,9 @@ def parse():
                     help="override the workload's batch size (smaller profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end run")
+    ap.add_argument("--policy", choices=["save", "recompute"], default="save",
+                    help="save: the forward keeps the chunk tiles and states for the backward; "
+                         "recompute: the backward recomputes them")
     ap.add_argument("--decode", action="store_true",
                     help="time the single-token decode step instead of the training step")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -411,13 +414,16 @@ def main():
     inp = make_inputs(w, seed=w.seed + 1000 * rank)
     d = {n: (None if x is None else x.to(dev)) for n, x in inp.items()}
     plan = binding.Plan.for_workload(w, device=dev)
-    saved = plan.new_saved()
-    o, ST, _ = plan.fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], saved=saved)
+    keep = args.policy == "save"
+    saved = plan.new_saved() if keep else None
+    o, ST, _ = plan.fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], saved=saved,
+                        save=keep)
     grads = plan.bwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], d["dO"], None, saved)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        plan.fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], o=o, ST=ST, saved=saved)
+        plan.fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], o=o, ST=ST, saved=saved,
+                 save=keep)
         plan.bwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], d["dO"], None, saved,
                  out=grads)
 
@@ -468,7 +474,7 @@ def main():
                 if x is not None:
                     dev_in[n].copy_(x, non_blocking=True)
             plan.fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"], dev_in["g"],
-                     dev_in["S0"], o=o, ST=ST, saved=saved)
+                     dev_in["S0"], o=o, ST=ST, saved=saved, save=keep)
             plan.bwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"], dev_in["g"],
                      dev_in["S0"], dev_in["dO"], None, saved, out=grads)
             hout["o"].copy_(o, non_blocking=True)
@@ -553,7 +559,8 @@ def main():
                    "parallelism": f"replicas x{world} (independent batches, no collective)",
                    "l2": f"L2 flushed between timed steps ({2 * L2_BYTES >> 20} MiB write); "
                          f"inputs {in_bytes >> 20} MiB per step",
-                   "policy": "forward saves chunk states; backward reads them"},
+                   "policy": ("forward saves chunk tiles and states; backward reads them"
+                              if keep else "backward recomputes the chunk tiles and states")},
         "roofline": roof,
         "step_roofline": step_roof,
         "cpu_baseline": cpu,
