@@ -186,9 +186,9 @@ __global__ void __launch_bounds__(NTB, 1)
   bf16* const sLW = s.SS + C * D;  // Lambda_W
   bf16* const sW = s.SD;           // W, U' for the third level
   bf16* const sUp = s.SD + C * D;
-  bf16* const sKb = s.SD;          // Kb^c, beta K^c for the fourth level
-  bf16* const sBk = s.SD + C * D;
-  bf16* const sdW = s.DO;          // dW, after the first level
+  bf16* const sKb = s.DU;          // Kb^c, beta K^c for the fourth level (built under level 3)
+  bf16* const sBk = s.DO;
+  bf16* const sdW = s.DO;          // dW, after the first level (then beta K^c)
   bf16* const sdM = s.UU;          // dM, dA [i][j], after the first level
   bf16* const sdA = s.UU + C * C;
 
@@ -397,6 +397,17 @@ __global__ void __launch_bounds__(NTB, 1)
       }
     frag::st_c(adm, sdM, -C, rb * 16, qt * 16);
   }
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  // ---- level 2: Lambda = T^T [dU | dW]; dv = diag(beta) Lambda_U (runs under the dKt pass)
+  if (tid == 0) {
+    const Chain cs[2] = {chain(tb + T_LU, s.TT, true, C, s.DU, true, D, 128, 0, 1, C / 16),
+                         chain(tb + T_LW, s.TT, true, C, sdW, true, D, 128, 0, 1, C / 16)};
+    issue_chains(cs);
+    tc::commit(&s.bar);
+  }
 
   // The per-element epilogue works on three accumulators at this thread's
   // fragment positions (rows i0, i0 + 8; key columns c), with ep = e^{gamma - gamma_r}:
@@ -438,18 +449,6 @@ __global__ void __launch_bounds__(NTB, 1)
         P[jt][u] *= frc;
         P[jt][2 + u] *= frc;
       }
-  }
-  tc::fence_smem_to_async();
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
-
-  // ---- level 2: Lambda = T^T [dU | dW]; dv = diag(beta) Lambda_U
-  if (tid == 0) {
-    const Chain cs[2] = {chain(tb + T_LU, s.TT, true, C, s.DU, true, D, 128, 0, 1, C / 16),
-                         chain(tb + T_LW, s.TT, true, C, sdW, true, D, 128, 0, 1, C / 16)};
-    issue_chains(cs);
-    tc::commit(&s.bar);
   }
   float dbrow[2] = {0.f, 0.f};  // this thread's d(beta_eff) partials for rows i0, i0 + 8
   float Q[4][4];
@@ -505,6 +504,24 @@ __global__ void __launch_bounds__(NTB, 1)
     issue_chains(cs);
     tc::commit(&s.bar);
   }
+  // ---- under level 3: Kb^c and beta K^c into the core-tiled operand tiles (dU, dW slots)
+  for (int idx = tid; idx < C * (D / 8); idx += NTB) {
+    const int i = ct_row(idx, D), c = ct_col(idx, D);
+    const uint4 rk = *reinterpret_cast<const uint4*>(s.k + i * LDD + c);
+    const float bi = s.beta[i];
+    const float4 f0 = ep4(i, c), f1 = ep4(i, c + 4);
+    const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+    const uint32_t* wk = reinterpret_cast<const uint32_t*>(&rk);
+    uint32_t okb[4], obc[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 kk = frag::unpack(wk[e]);
+      okb[e] = frag::pack(__fdividef(kk.x, f[2 * e]), __fdividef(kk.y, f[2 * e + 1]));
+      obc[e] = frag::pack(bi * kk.x * f[2 * e], bi * kk.y * f[2 * e + 1]);
+    }
+    *reinterpret_cast<uint4*>(sKb + 8 * idx) = make_uint4(okb[0], okb[1], okb[2], okb[3]);
+    *reinterpret_cast<uint4*>(sBk + 8 * idx) = make_uint4(obc[0], obc[1], obc[2], obc[3]);
+  }
   ok = hy_wait(&s.bar, 2);
   if (!ok) break;
   {
@@ -528,24 +545,6 @@ __global__ void __launch_bounds__(NTB, 1)
     frag::st_c(da, sdA, -C, rb * 16, qt * 16);
   }
 
-  // ---- Kb^c and beta K^c into the core-tiled operand tiles (W, U' are consumed)
-  for (int idx = tid; idx < C * (D / 8); idx += NTB) {
-    const int i = ct_row(idx, D), c = ct_col(idx, D);
-    const uint4 rk = *reinterpret_cast<const uint4*>(s.k + i * LDD + c);
-    const float bi = s.beta[i];
-    const float4 f0 = ep4(i, c), f1 = ep4(i, c + 4);
-    const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-    const uint32_t* wk = reinterpret_cast<const uint32_t*>(&rk);
-    uint32_t okb[4], obc[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 kk = frag::unpack(wk[e]);
-      okb[e] = frag::pack(__fdividef(kk.x, f[2 * e]), __fdividef(kk.y, f[2 * e + 1]));
-      obc[e] = frag::pack(bi * kk.x * f[2 * e], bi * kk.y * f[2 * e + 1]);
-    }
-    *reinterpret_cast<uint4*>(sKb + 8 * idx) = make_uint4(okb[0], okb[1], okb[2], okb[3]);
-    *reinterpret_cast<uint4*>(sBk + 8 * idx) = make_uint4(obc[0], obc[1], obc[2], obc[3]);
-  }
   tc::fence_smem_to_async();
   tc::fence_before_sync();
   __syncthreads();
