@@ -485,10 +485,10 @@ __global__ void __launch_bounds__(NTF, 1)
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks)
         tc::mma(tbase + T_U, dKT + ks * kK, dDSB + ks * kB, id1b, 1u);
+      tc::commit(&s.barA);  // dU is complete; the dU-free half of D_S runs under epilogue 1
 #pragma unroll
       for (int ks = 0; ks < C / 16; ++ks)
         tc::mma(tbase + T_S, dQH + ks * kA128, dDO + ks * kB, id2, ks > 0 ? 1u : 0u);
-      tc::commit(&s.barA);
     }
     if (outputs) store_dh(cb);
     ok = cta_wait(&s.barA, it);
