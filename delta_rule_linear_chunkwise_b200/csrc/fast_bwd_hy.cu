@@ -103,9 +103,11 @@ __device__ __forceinline__ Chain chain(uint32_t tm, const bf16* A, bool a_mn, in
   c.count = count;
   return c;
 }
-// Issue the chains round-robin by step: a tcgen05.mma that accumulates into
-// the same tensor memory waits for the previous one (about 190 cycles for
-// M = 64, measured), so independent chains are interleaved to overlap.
+// Issue the chains round-robin by step (consecutive instructions go to
+// independent accumulators).  Measured on B200: with the descriptors built
+// before the loop, one thread issues a tcgen05.mma of M = 64 or 128, N <= 128
+// every 55-70 cycles and the tensor core keeps pace, so a level costs about
+// its instruction count times that.
 template <int NC>
 __device__ __forceinline__ void issue_chains(const Chain (&cs)[NC]) {
   int steps = 0;

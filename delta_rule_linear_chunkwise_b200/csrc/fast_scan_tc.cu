@@ -367,7 +367,10 @@ cudaError_t launch_fwd_scan_tc_bv(const Problem& p, const Saved& sv, const ScanS
 //   epilogue 2   dS_n^T = Diag(e^{gamma_C}) dS^T + D_S       (fp32, registers)
 // dh_n = dS_{n+1} is written out (bf16) while MMA-1 runs.  Each CTA owns the
 // value columns a0 .. a0 + BV of dS; the state gradient is held transposed,
-// one key per TMEM lane.
+// one key per TMEM lane.  The dS-free half of MMA-1 (M^T dO) of the next chunk
+// is issued under epilogue 2 into the other D_U buffer, so a step's critical
+// path holds only the dS-dependent products.  The chunk tiles arrive by bulk
+// copies (one thread, the stage's mbarrier); the dO slice by cp.async.
 template <int BV>
 struct BScanStage {
   bf16 QH[C * D];     // q e^gamma, core-tiled [j][c]: MN-major A (M = key c, K = j)
@@ -382,27 +385,34 @@ struct BScanSmem {
   BScanStage<BV> st[2];
   bf16 DSB[D * BV];   // bf16 dS^T, core-tiled [c][a]: MN-major B of MMA-1
   bf16 DUB[C * BV];   // bf16 -dU, core-tiled [i][a]: MN-major B of MMA-2b
-  uint64_t barA, barB;
+  uint64_t barA, barB, full[2];
   uint32_t tmem;
 };
 
+// Fills a stage: the core-tiled chunk tiles by bulk copies from thread 0
+// (completing on `full`), the dO slice by cp.async from every thread (the
+// caller commits the group).
 template <int BV>
-__device__ __forceinline__ void bscan_issue_tc(const Problem& p, BScanStage<BV>& s, const Saved& sv,
-                                               const bf16* __restrict__ dO, int b, int h, int n,
-                                               int a0) {
+__device__ __forceinline__ void bscan_fill(const Problem& p, BScanStage<BV>& s, uint64_t* full,
+                                           const Saved& sv, const bf16* __restrict__ dO, int b,
+                                           int h, int n, int a0) {
   const int tid = threadIdx.x;
   const size_t cb = chunk_id(p, b, h, n);
   const int t0 = n * C, nvalid = min(C, p.T - t0);
-  cp_linear<NTF>(s.QH, sv.Qh + cb * C * D, C * D, tid);
-  cp_linear<NTF>(s.KT, sv.Kt + cb * C * D, C * D, tid);
-  cp_linear<NTF>(s.W, sv.W + cb * C * D, C * D, tid);
-  cp_linear<NTF>(s.M, sv.M + cb * C * C, C * C, tid);
+  if (tid == 0) {
+    constexpr uint32_t kT = C * D * 2, kM = C * C * 2, kDec = D * 4;
+    tc::mbar_arrive_expect_tx(full, 3 * kT + kM + kDec);
+    tc::bulk_g2s(s.QH, sv.Qh + cb * C * D, kT, full);
+    tc::bulk_g2s(s.KT, sv.Kt + cb * C * D, kT, full);
+    tc::bulk_g2s(s.W, sv.W + cb * C * D, kT, full);
+    tc::bulk_g2s(s.M, sv.M + cb * C * C, kM, full);
+    tc::bulk_g2s(s.dec, sv.dec + cb * D, kDec, full);
+  }
   for (int idx = tid; idx < C * BV / 8; idx += NTF) {
     const int j = ct_row(idx, BV), col = ct_col(idx, BV);
     const bool ok = j < nvalid;
     frag::cp16(s.DO + 8 * idx, dO + row_id(p, b, t0 + (ok ? j : 0), h) * D + a0 + col, ok);
   }
-  if (tid < D / 4) frag::cp16(s.dec + 4 * tid, sv.dec + cb * D + 4 * tid, true);
 }
 
 template <int BV>
@@ -410,7 +420,7 @@ __global__ void __launch_bounds__(NTF, 1)
     k_bwd_scan_tc(Problem p, Saved sv, const bf16* __restrict__ dO, ScanSeg sg,
                   bf16* __restrict__ dUout, bf16* __restrict__ dhout, int* __restrict__ err) {
   constexpr int HB = BV / 2;
-  constexpr int TALLOC = 2 * BV <= 128 ? 128 : 256;
+  constexpr int TALLOC = 3 * BV <= 256 ? 256 : 512;  // D_U x 2, D_S
   extern __shared__ __align__(1024) unsigned char smraw[];
   BScanSmem<BV>& s = *reinterpret_cast<BScanSmem<BV>*>(smraw);
   const int h = blockIdx.y, b = blockIdx.z / sg.G, seg = blockIdx.z % sg.G, tid = threadIdx.x;
@@ -423,12 +433,15 @@ __global__ void __launch_bounds__(NTF, 1)
   float* __restrict__ dS0 = sg.ST;
   const size_t sbase = (((size_t)b * sg.G + seg) * p.H + h) * D * D;
   const int c = 32 * (warp & 3) + lane, ah = warp >> 2;  // key (TMEM lane), value half
-  const uint32_t T_U = 0, T_S = BV;
+  const uint32_t T_S = 2 * BV;  // D_U buffers at columns 0 and BV
 
   if (warp == 0) tc::tmem_alloc(&s.tmem, TALLOC);
   if (tid == 0) {
     tc::mbar_init(&s.barA, 1);
     tc::mbar_init(&s.barB, 1);
+    tc::mbar_init(&s.full[0], 1);
+    tc::mbar_init(&s.full[1], 1);
+    tc::fence_mbar_init();
   }
   float dS[HB];  // dS^T[c][a0 + ah*HB + u]
 #pragma unroll
@@ -449,14 +462,19 @@ __global__ void __launch_bounds__(NTF, 1)
   };
 
   write_dsb();
-  bscan_issue_tc<BV>(p, s.st[0], sv, dO, b, h, n1 - 1, a0);
+  tc::fence_before_sync();
+  __syncthreads();  // barriers initialised
+  tc::fence_after_sync();
+  bscan_fill<BV>(p, s.st[0], &s.full[0], sv, dO, b, h, n1 - 1, a0);
   frag::cp_commit();
-  if (n1 - 2 >= n0) bscan_issue_tc<BV>(p, s.st[1], sv, dO, b, h, n1 - 2, a0);
+  if (n1 - 2 >= n0) bscan_fill<BV>(p, s.st[1], &s.full[1], sv, dO, b, h, n1 - 2, a0);
   frag::cp_commit();
+  int fills0 = 1, fills1 = n1 - 2 >= n0 ? 1 : 0;  // bulk fills issued per stage (uniform)
   frag::cp_wait<1>();
+  bool ok = tc::mbar_wait(&s.full[0], 0u, kSpinScan);
   tc::fence_smem_to_async();
   tc::fence_before_sync();
-  __syncthreads();
+  ok = __syncthreads_or(ok ? 0 : 1) == 0;
   tc::fence_after_sync();
   const uint32_t tbase = s.tmem;
 
@@ -470,18 +488,23 @@ __global__ void __launch_bounds__(NTF, 1)
   constexpr uint32_t kK = 256 / 16;                  // K-major k-step
   // epilogue-1 ownership (M = 64 accumulator layout): row i = 16 (warp % 4) + lane, lane < 16
   const int ri = 16 * (warp & 3) + (lane & 15);
-  bool ok = true;
+  // M^T dO of the chunk in stage `sg` into D_U buffer `ub` (overwrites it)
+  auto issue_mtdo = [&](int sg, int ub) {
+    const uint64_t dM = tc::sdesc_mnmaj(s.st[sg].M, C, 0), dDO = tc::sdesc_mnmaj(s.st[sg].DO, BV, 0);
+#pragma unroll
+    for (int ks = 0; ks < C / 16; ++ks)
+      tc::mma(tbase + ub * BV, dM + ks * kA64, dDO + ks * kB, id1a, ks > 0 ? 1u : 0u);
+  };
+  if (ok && tid == 0) issue_mtdo(0, 0);
   for (int it = 0; it < n1 - n0 && ok; ++it) {
     const int n = n1 - 1 - it;
     const size_t cb = chunk_id(p, b, h, n);
     BScanStage<BV>& st = s.st[it & 1];
+    const uint32_t T_U = (uint32_t)((it & 1) * BV);
     const float dc = st.dec[c];  // read before the stage is refilled below
     if (tid == 0) {
-      const uint64_t dM = tc::sdesc_mnmaj(st.M, C, 0), dDO = tc::sdesc_mnmaj(st.DO, BV, 0);
       const uint64_t dKT = tc::sdesc_kmaj(st.KT, D, 0), dQH = tc::sdesc_mnmaj(st.QH, D, 0);
-#pragma unroll
-      for (int ks = 0; ks < C / 16; ++ks)
-        tc::mma(tbase + T_U, dM + ks * kA64, dDO + ks * kB, id1a, ks > 0 ? 1u : 0u);
+      const uint64_t dDO = tc::sdesc_mnmaj(st.DO, BV, 0);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks)
         tc::mma(tbase + T_U, dKT + ks * kK, dDSB + ks * kB, id1b, 1u);
@@ -529,9 +552,26 @@ __global__ void __launch_bounds__(NTF, 1)
       for (int e8 = 0; e8 < HB / 8; ++e8)
         *reinterpret_cast<uint4*>(up + ct_off(ri, a0 + ah * HB + 8 * e8, D)) = dusave[e8];
     }
-    ok = cta_wait(&s.barB, it);
+    // the next chunk's stage (filled one step ago) must be complete before the
+    // barrier below, so that its M^T dO can be issued under epilogue 2
+    bool okF = true;
+    if (n - 1 >= n0) {
+      frag::cp_wait<0>();
+      okF = tc::mbar_wait(&s.full[(it + 1) & 1], (uint32_t)(((it + 1) >> 1) & 1), kSpinScan);
+      tc::fence_smem_to_async();
+    }
+    {
+      const bool okB = tc::mbar_wait(&s.barB, (uint32_t)(it & 1), kSpinScan);
+      ok = __syncthreads_or((okB && okF) ? 0 : 1) == 0;
+      tc::fence_after_sync();
+    }
     if (!ok) break;
-    if (n - 2 >= n0) bscan_issue_tc<BV>(p, st, sv, dO, b, h, n - 2, a0);
+    if (tid == 0 && n - 1 >= n0) issue_mtdo((it + 1) & 1, (it + 1) & 1);
+    // every read of this stage is done: refill it with chunk n - 2
+    if (n - 2 >= n0) {
+      bscan_fill<BV>(p, st, &s.full[it & 1], sv, dO, b, h, n - 2, a0);
+      ++((it & 1) ? fills1 : fills0);
+    }
     frag::cp_commit();
     // epilogue 2: dS^T <- Diag(e^{gamma_C}) dS^T + D_S
     {
@@ -544,7 +584,6 @@ __global__ void __launch_bounds__(NTF, 1)
       for (int e = 0; e < HB; ++e) dS[e] = dS[e] * dc + __uint_as_float(r[e]);
       write_dsb();
     }
-    frag::cp_wait<1>();
     tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
@@ -558,7 +597,12 @@ __global__ void __launch_bounds__(NTF, 1)
   } else if (tid == 0 && err) {
     atomicExch(err, 1);
   }
+  // copies still in flight (only after a failed wait) land before exit
   frag::cp_wait<0>();
+  if (tid == 0) {
+    if (fills0 > 0) tc::mbar_wait(&s.full[0], (uint32_t)((fills0 - 1) & 1), kSpinScan);
+    if (fills1 > 0) tc::mbar_wait(&s.full[1], (uint32_t)((fills1 - 1) & 1), kSpinScan);
+  }
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tbase, TALLOC);
