@@ -104,9 +104,13 @@ def aggregate_tokens_per_s(world: int, tokens_per_step: int, steps: int, max_ms:
     return world * tokens_per_step * steps / (max_ms / 1e3)
 
 
-def csrc_hash():
+def csrc_hash(files=None):
+    """Hash of kernel sources: the named files under csrc/ (every file if None)."""
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "delta_rule_linear_chunkwise_b200", "csrc", "*"))):
+    csrc = os.path.join(ROOT, "delta_rule_linear_chunkwise_b200", "csrc")
+    paths = sorted(glob.glob(os.path.join(csrc, "*"))) if files is None else \
+        [os.path.join(csrc, f) for f in sorted(files)]
+    for f in paths:
         with open(f, "rb") as fh:
             h.update(os.path.basename(f).encode() + fh.read())
     return h.hexdigest()[:16]
@@ -114,14 +118,21 @@ def csrc_hash():
 
 def ncu_traffic(kernel, workload):
     """DRAM bytes per launch from a committed ncu capture, if it was taken on
-    the current kernel sources (else None)."""
+    the current sources of that kernel (the record's `sources`: its translation
+    unit and the headers it includes), else None."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
     e = d.get(kernel)
-    if not e or e.get("csrc_hash") != csrc_hash() or e.get("workload") != workload:
+    if not e or e.get("workload") != workload:
+        return None
+    try:
+        cur = csrc_hash(e.get("sources"))
+    except OSError:
+        return None
+    if e.get("csrc_hash") != cur:
         return None
     return e.get("dram_bytes_per_launch")
 

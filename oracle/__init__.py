@@ -18,8 +18,10 @@ Two independent restatements live here:
   explainer, gist.science), never as a comparison target for the GPU.
 
 Layouts: q, k ``[B, T, H, dk]``; v, o, dO ``[B, T, H, dv]``; beta ``[B, T, H]``;
-g ``[B, T, H]`` (scalar gate) or ``[B, T, H, dk]`` (per-channel gate) or
-``None`` (no gate); states ``[B, H, dv, dk]``.
+g ``[B, T, H]`` (scalar gate) or ``[B, T, H, dk]`` (per-channel gate; also the
+phase gate of SFDA, selected with ``gate=GATE_PHASE``: log alpha_j at channel
+2j and the phase theta_j at 2j+1 of key pair j) or ``None`` (no gate); states
+``[B, H, dv, dk]``.
 """
 from __future__ import annotations
 
@@ -29,7 +31,7 @@ import subprocess
 
 import numpy as np
 
-GATE_NONE, GATE_SCALAR, GATE_CHANNEL = 0, 1, 2
+GATE_NONE, GATE_SCALAR, GATE_CHANNEL, GATE_PHASE = 0, 1, 2, 3
 BETA_DIRECT, BETA_KACZMARZ = 0, 1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -79,9 +81,15 @@ def _ptr(x):
     return x.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
 
 
-def gate_kind(g, dk: int) -> int:
+def gate_kind(g, dk: int, gate=None) -> int:
+    """The gate kind: ``gate`` when given (needed for the phase gate, which has
+    the per-channel gate's shape), else inferred from the shape of ``g``."""
     if g is None:
         return GATE_NONE
+    if gate is not None:
+        if gate == GATE_PHASE and (g.ndim != 4 or g.shape[-1] != dk or dk % 2):
+            raise ValueError("phase gate: g must be [B, T, H, dk] with dk even")
+        return gate
     return GATE_CHANNEL if (g.ndim == 4 and g.shape[-1] == dk) else GATE_SCALAR
 
 
@@ -92,28 +100,33 @@ def _dims(q, v):
 
 
 def recurrent_fwd(q, k, v, beta, g=None, S0=None, beta_mode=BETA_DIRECT, eps=1e-6,
-                  return_threads=False):
-    """Token-by-token forward.  Returns ``(o, S_T)`` as fp64 arrays."""
+                  return_threads=False, gate=None):
+    """Token-by-token forward.  Returns ``(o, S_T)`` as fp64 arrays.
+
+    ``gate=GATE_PHASE`` selects the SFDA rotation-decay gate: ``g[..., 2j]`` is
+    log alpha_j and ``g[..., 2j+1]`` the phase theta_j of key pair j."""
     q, k, v, beta, g, S0 = map(_f64, (q, k, v, beta, g, S0))
     B, T, H, dk, dv = _dims(q, v)
     o = np.zeros((B, T, H, dv))
     ST = np.zeros((B, H, dv, dk))
-    used = _load().oracle_fwd(B, H, T, dk, dv, gate_kind(g, dk), beta_mode, eps,
+    used = _load().oracle_fwd(B, H, T, dk, dv, gate_kind(g, dk, gate), beta_mode, eps,
                               _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(S0),
                               _ptr(o), _ptr(ST))
     return (o, ST, used) if return_threads else (o, ST)
 
 
 def recurrent_bwd(q, k, v, beta, g, S0, dO, dST=None, beta_mode=BETA_DIRECT, eps=1e-6,
-                  return_threads=False):
+                  return_threads=False, gate=None):
     """Hand-derived reverse mode of the recurrence.
 
     Returns a dict with ``dq, dk, dv, dbeta, dg, dS0`` (``dg`` is ``None`` when
-    there is no gate; in Kaczmarz mode ``dbeta`` is the gradient w.r.t. eta).
+    there is no gate; in Kaczmarz mode ``dbeta`` is the gradient w.r.t. eta;
+    for the phase gate ``dg[..., 2j]`` is d/d log alpha_j and ``dg[..., 2j+1]``
+    d/d theta_j).
     """
     q, k, v, beta, g, S0, dO, dST = map(_f64, (q, k, v, beta, g, S0, dO, dST))
     B, T, H, dk, dv = _dims(q, v)
-    gk = gate_kind(g, dk)
+    gk = gate_kind(g, dk, gate)
     dq = np.zeros_like(q)
     dkk = np.zeros_like(k)
     dvv = np.zeros_like(v)

@@ -185,3 +185,76 @@ def chunk_bwd(q, k, v, beta, g, S0, dO, dST=None, C=64, beta_mode=0, eps=1e-6):
                 dS = dS_prev
             dS0[b, h] = dS
     return dict(dq=dq, dk=dkk, dv=dvv, dbeta=db, dg=dg, dS0=dS0)
+
+
+# ---------------------------------------------------------------------------
+# Phase (SFDA rotation-decay) gate.  The token decay acts on a state row as
+# row -> Lambda_t row, Lambda_t the direct sum over key pairs (2j, 2j+1) of
+# alpha_j [[cos theta_j, -sin theta_j], [sin theta_j, cos theta_j]] ("Semidirect
+# Fourier Delta Attention", gist.science explainer, "Kernarchitektur"), i.e.
+# S_t = S_{t-1} Lambda_t^T (I - beta_t k_t k_t^T) + beta_t v_t k_t^T.  The
+# blocks of different tokens commute, so with Gamma_i = Lambda_1^T ... Lambda_i^T
+# (within the chunk) and the de-rotated state S~_i = S_i Gamma_i^{-1}, the chunk
+# is a plain delta rule with read keys Kh_i = Gamma_i k_i and write keys
+# Kb_i = Gamma_i^{-T} k_i (the page's "Konstruktives Chunk-WY-Theorem": the
+# phase-decay product plus the rank-one corrections stays a chunk-local
+# recursion):
+#     A  = diag(beta) strict_tril(Kh Kb^T),  (I + A) [U' | W] = diag(beta) [V | Kh]
+#     U  = U' - W S^T,     O = Qh S^T + tril(Qh Kb^T) U,   Qh_i = Gamma_i q_i
+#     S' = S Gamma_C + U^T Kt,   Kt_i = Gamma_C^T Kb_i
+# Written here with explicit d_k x d_k block matrices.
+
+def _phase_block(g_row):
+    """Lambda_t (d_k x d_k) from one token's phase gate row (log alpha_j at 2j,
+    theta_j at 2j+1)."""
+    dk = g_row.shape[0]
+    L = np.zeros((dk, dk))
+    for j in range(dk // 2):
+        a, th = np.exp(g_row[2 * j]), g_row[2 * j + 1]
+        L[2 * j:2 * j + 2, 2 * j:2 * j + 2] = a * np.array([[np.cos(th), -np.sin(th)],
+                                                             [np.sin(th), np.cos(th)]])
+    return L
+
+
+def chunk_fwd_phase(q, k, v, beta, g, S0=None, C=64, beta_mode=0, eps=1e-6,
+                    return_states=False):
+    """Chunkwise forward with the phase gate.  Returns ``(o, S_T)``."""
+    q, k, v, beta, g, S0 = map(_f64, (q, k, v, beta, g, S0))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dv, dk))
+    nc = (T + C - 1) // C
+    states = np.zeros((B, H, nc, dv, dk))
+    for b in range(B):
+        for h in range(H):
+            qh, kh, vh, _, bt, _, gh = _head_inputs(q, k, v, beta, g, b, h, beta_mode, eps)
+            S = np.zeros((dv, dk)) if S0 is None else S0[b, h].copy()
+            for n in range(nc):
+                t0, t1 = n * C, min(T, n * C + C)
+                qc, kc, vc = (_pad_chunk(x, t0, t1, C) for x in (qh, kh, vh))
+                bc = _pad_chunk(bt, t0, t1, C)
+                # padded rows: log alpha = 0, theta = 0 (identity decay)
+                gc = _pad_chunk(gh, t0, t1, C)
+                Gam = np.zeros((C, dk, dk))
+                acc = np.eye(dk)
+                for i in range(C):
+                    acc = acc @ _phase_block(gc[i]).T
+                    Gam[i] = acc
+                Kh = np.einsum("icd,id->ic", Gam, kc)
+                Kb = np.stack([np.linalg.solve(Gam[i].T, kc[i]) for i in range(C)])
+                Qh = np.einsum("icd,id->ic", Gam, qc)
+                Kt = Kb @ Gam[-1]                       # rows (Gamma_C^T Kb_i)^T
+                A = bc[:, None] * np.tril(Kh @ Kb.T, -1)
+                X = np.linalg.solve(np.eye(C) + A,
+                                    bc[:, None] * np.concatenate([vc, Kh], axis=1))
+                Up, W = X[:, :dv], X[:, dv:]
+                states[b, h, n] = S
+                U = Up - W @ S.T
+                O = Qh @ S.T + np.tril(Qh @ Kb.T) @ U
+                o[b, t0:t1, h] = O[: t1 - t0]
+                S = S @ Gam[-1] + U.T @ Kt
+            ST[b, h] = S
+    if return_states:
+        return o, ST, states
+    return o, ST

@@ -23,7 +23,18 @@
  * and KDA.
  *
  * Gate kinds: none (alpha = 1, DeltaNet), scalar (one log-gate per head and
- * token, GDN) and per-channel (one log-gate per key channel, KDA).
+ * token, GDN), per-channel (one log-gate per key channel, KDA) and phase
+ * (SFDA, same explainer, "Kernarchitektur": the complex diagonal
+ * Lambda_t = diag(alpha_t e^{i theta_t}) written in real coordinates as a
+ * direct sum of 2 x 2 rotation-decay blocks).  For the phase gate the key
+ * channels pair up as (2j, 2j+1), one complex coordinate each; g holds
+ * log alpha_j at channel 2j and theta_j at channel 2j+1, and the decay maps a
+ * state row's pair (x, y) -- the real and imaginary parts of that coordinate --
+ * to alpha_j (cos theta_j x - sin theta_j y, sin theta_j x + cos theta_j y).
+ * Keys, queries and values stay real, and the erase-and-write is the real
+ * rank-one correction above (the reading of the page's update in real
+ * coordinates); zero phase gives KDA with both channels of a pair sharing
+ * one decay.
  * Beta modes: direct (beta is the input) and Kaczmarz (KLA abstract,
  * thelatestinai.com): beta_t = eta_t / (||k_t||^2 + eps), the input being eta.
  *
@@ -39,13 +50,19 @@
  *   dg_t[c] = sum_a dP[a,c] P[a,c]    (gradient w.r.t. log alpha; summed over
  *                                      c for a scalar gate)
  *   dS_{t-1} = dP Diag(alpha_t)
+ * For the phase gate, with (Px, Py) and (dPx, dPy) a row's pair j of P, dP:
+ *   dg_t[2j]   = sum_a (dPx Px + dPy Py)          (d/d log alpha_j)
+ *   dg_t[2j+1] = sum_a (dPy Px - dPx Py)          (d/d theta_j)
+ *   dS_{t-1} pair = alpha_j (cos theta_j dPx + sin theta_j dPy,
+ *                            -sin theta_j dPx + cos theta_j dPy)   (Lambda^T dP)
  * Kaczmarz mode adds the chain through beta = eta/(n+eps), n = ||k||^2:
  *   deta = dbeta/(n+eps),  dk_t += -2 beta dbeta k_t/(n+eps).
  *
  * Layouts (row-major, all fp64):
  *   q, k      [B, T, H, dk]      v, o, dO  [B, T, H, dv]
  *   beta      [B, T, H]          (eta in Kaczmarz mode)
- *   g         [B, T, H] (scalar) or [B, T, H, dk] (per-channel); unused for none
+ *   g         [B, T, H] (scalar) or [B, T, H, dk] (per-channel, phase); unused
+ *             for none
  *   S0, ST, dST, dS0   [B, H, dv, dk]   (S0/dST may be NULL = zero)
  */
 #include <math.h>
@@ -58,6 +75,7 @@
 #define ORACLE_GATE_NONE 0
 #define ORACLE_GATE_SCALAR 1
 #define ORACLE_GATE_CHANNEL 2
+#define ORACLE_GATE_PHASE 3
 #define ORACLE_BETA_DIRECT 0
 #define ORACLE_BETA_KACZMARZ 1
 
@@ -75,6 +93,36 @@ static double oracle_alpha(const oproblem* p, const double* g, int b, int t, int
   return exp(g[row * p->dk + c]);
 }
 
+/* The decay of token t for head (b,h): alpha[c] for the diagonal gates; for
+   the phase gate ac[j] = alpha_j cos theta_j, as[j] = alpha_j sin theta_j. */
+static void oracle_decay(const oproblem* p, const double* g, int b, int t, int h,
+                         double* alpha, double* ac, double* as) {
+  if (p->gate != ORACLE_GATE_PHASE) {
+    for (int c = 0; c < p->dk; ++c) alpha[c] = oracle_alpha(p, g, b, t, h, c);
+    return;
+  }
+  size_t row = ((size_t)b * p->T + t) * p->H + h;
+  for (int j = 0; j < p->dk / 2; ++j) {
+    double al = exp(g[row * p->dk + 2 * j]), th = g[row * p->dk + 2 * j + 1];
+    ac[j] = al * cos(th);
+    as[j] = al * sin(th);
+  }
+}
+
+/* Applies the decay to one state row in place (row . Lambda^T). */
+static void oracle_decay_row(const oproblem* p, double* Sa, const double* alpha,
+                             const double* ac, const double* as) {
+  if (p->gate != ORACLE_GATE_PHASE) {
+    for (int c = 0; c < p->dk; ++c) Sa[c] *= alpha[c];
+    return;
+  }
+  for (int j = 0; j < p->dk / 2; ++j) {
+    double x = Sa[2 * j], y = Sa[2 * j + 1];
+    Sa[2 * j] = ac[j] * x - as[j] * y;
+    Sa[2 * j + 1] = as[j] * x + ac[j] * y;
+  }
+}
+
 /* Effective beta_t and the key norm n_t = ||k_t||^2. */
 static double oracle_beta(const oproblem* p, const double* beta, const double* kt,
                           size_t row, double* norm_out) {
@@ -85,19 +133,18 @@ static double oracle_beta(const oproblem* p, const double* beta, const double* k
   return beta[row];
 }
 
-/* One recurrence step in place: S <- P + beta (v - P k) k^T with P = S Diag(alpha).
+/* One recurrence step in place: S <- P + beta (v - P k) k^T with P = S Lambda^T
+   (P = S Diag(alpha) for the diagonal gates).
    If P_out is non-NULL it receives P; e_out receives e = v - P k. */
 static void oracle_step(const oproblem* p, double* S, const double* alpha,
-                        const double* kt, const double* vt, double bt, double* P_out,
-                        double* e_out) {
+                        const double* ac, const double* as, const double* kt,
+                        const double* vt, double bt, double* P_out, double* e_out) {
   const int dk = p->dk, dv = p->dv;
   for (int a = 0; a < dv; ++a) {
     double* Sa = S + (size_t)a * dk;
     double pk = 0.0;
-    for (int c = 0; c < dk; ++c) {
-      Sa[c] *= alpha[c];
-      pk += Sa[c] * kt[c];
-    }
+    oracle_decay_row(p, Sa, alpha, ac, as);
+    for (int c = 0; c < dk; ++c) pk += Sa[c] * kt[c];
     if (P_out) memcpy(P_out + (size_t)a * dk, Sa, sizeof(double) * dk);
     double e = vt[a] - pk;
     if (e_out) e_out[a] = e;
@@ -113,6 +160,8 @@ static void oracle_fwd_head(const oproblem* p, int b, int h, const double* q,
   const size_t SS = (size_t)dv * dk;
   double* S = (double*)malloc(sizeof(double) * SS);
   double* alpha = (double*)malloc(sizeof(double) * dk);
+  double* ac = (double*)malloc(sizeof(double) * (dk / 2 + 1));
+  double* as = (double*)malloc(sizeof(double) * (dk / 2 + 1));
   if (S0)
     memcpy(S, S0 + ((size_t)b * H + h) * SS, sizeof(double) * SS);
   else
@@ -122,9 +171,9 @@ static void oracle_fwd_head(const oproblem* p, int b, int h, const double* q,
     const double* qt = q + row * dk;
     const double* kt = k + row * dk;
     const double* vt = v + row * dv;
-    for (int c = 0; c < dk; ++c) alpha[c] = oracle_alpha(p, g, b, t, h, c);
+    oracle_decay(p, g, b, t, h, alpha, ac, as);
     double bt = oracle_beta(p, beta, kt, row, NULL);
-    oracle_step(p, S, alpha, kt, vt, bt, NULL, NULL);
+    oracle_step(p, S, alpha, ac, as, kt, vt, bt, NULL, NULL);
     double* ot = o + row * dv;
     for (int a = 0; a < dv; ++a) {
       double acc = 0.0;
@@ -136,6 +185,8 @@ static void oracle_fwd_head(const oproblem* p, int b, int h, const double* q,
   if (ST) memcpy(ST + ((size_t)b * H + h) * SS, S, sizeof(double) * SS);
   free(S);
   free(alpha);
+  free(ac);
+  free(as);
 }
 
 /* Checkpoint spacing: 64 tokens, doubled until there are no more checkpoints
@@ -160,6 +211,8 @@ static void oracle_bwd_head(const oproblem* p, int b, int h, const double* q,
   double* P = (double*)malloc(sizeof(double) * SS);
   double* dS = (double*)malloc(sizeof(double) * SS);
   double* alpha = (double*)malloc(sizeof(double) * dk);
+  double* ac = (double*)malloc(sizeof(double) * (dk / 2 + 1));
+  double* as = (double*)malloc(sizeof(double) * (dk / 2 + 1));
   double* e = (double*)malloc(sizeof(double) * dv);
   double* w = (double*)malloc(sizeof(double) * dv);
   double* dgc = (double*)malloc(sizeof(double) * dk);
@@ -173,9 +226,9 @@ static void oracle_bwd_head(const oproblem* p, int b, int h, const double* q,
   for (int t = 0; t < T; ++t) {
     if (t % L == 0) memcpy(ckpt + (size_t)(t / L) * SS, S, sizeof(double) * SS);
     size_t row = ((size_t)b * T + t) * H + h;
-    for (int c = 0; c < dk; ++c) alpha[c] = oracle_alpha(p, g, b, t, h, c);
+    oracle_decay(p, g, b, t, h, alpha, ac, as);
     double bt = oracle_beta(p, beta, k + row * dk, row, NULL);
-    oracle_step(p, S, alpha, k + row * dk, v + row * dv, bt, NULL, NULL);
+    oracle_step(p, S, alpha, ac, as, k + row * dk, v + row * dv, bt, NULL, NULL);
   }
 
   if (dST)
@@ -192,9 +245,9 @@ static void oracle_bwd_head(const oproblem* p, int b, int h, const double* q,
       size_t row = ((size_t)b * T + t) * H + h;
       double* Sn = Sbuf + (size_t)(t - t0 + 1) * SS;
       memcpy(Sn, Sbuf + (size_t)(t - t0) * SS, sizeof(double) * SS);
-      for (int c = 0; c < dk; ++c) alpha[c] = oracle_alpha(p, g, b, t, h, c);
+      oracle_decay(p, g, b, t, h, alpha, ac, as);
       double bt = oracle_beta(p, beta, k + row * dk, row, NULL);
-      oracle_step(p, Sn, alpha, k + row * dk, v + row * dv, bt, NULL, NULL);
+      oracle_step(p, Sn, alpha, ac, as, k + row * dk, v + row * dv, bt, NULL, NULL);
     }
     for (int t = t1 - 1; t >= t0; --t) {
       size_t row = ((size_t)b * T + t) * H + h;
@@ -206,7 +259,7 @@ static void oracle_bwd_head(const oproblem* p, int b, int h, const double* q,
       const double* Snew = Sbuf + (size_t)(t - t0 + 1) * SS;
       double n;
       double bt = oracle_beta(p, beta, kt, row, &n);
-      for (int c = 0; c < dk; ++c) alpha[c] = oracle_alpha(p, g, b, t, h, c);
+      oracle_decay(p, g, b, t, h, alpha, ac, as);
 
       /* o_t = S_t q_t */
       for (int a = 0; a < dv; ++a)
@@ -217,14 +270,14 @@ static void oracle_bwd_head(const oproblem* p, int b, int h, const double* q,
         for (int a = 0; a < dv; ++a) acc += Snew[(size_t)a * dk + c] * dot[a];
         dqt[c] = acc;
       }
-      /* P = S_{t-1} Diag(alpha), e = v - P k */
+      /* P = S_{t-1} Lambda^T (S_{t-1} Diag(alpha) for the diagonal gates),
+         e = v - P k */
       for (int a = 0; a < dv; ++a) {
+        double* Pa = P + (size_t)a * dk;
+        memcpy(Pa, Sprev + (size_t)a * dk, sizeof(double) * dk);
+        oracle_decay_row(p, Pa, alpha, ac, as);
         double pk = 0.0;
-        for (int c = 0; c < dk; ++c) {
-          double pac = Sprev[(size_t)a * dk + c] * alpha[c];
-          P[(size_t)a * dk + c] = pac;
-          pk += pac * kt[c];
-        }
+        for (int c = 0; c < dk; ++c) pk += Pa[c] * kt[c];
         e[a] = vt[a] - pk;
       }
       /* S_t = P + beta e k^T */
@@ -244,17 +297,32 @@ static void oracle_bwd_head(const oproblem* p, int b, int h, const double* q,
           acc += bt * dS[(size_t)a * dk + c] * e[a] - P[(size_t)a * dk + c] * dvt[a];
         dkt[c] = acc;
       }
-      /* dP = dS - de k^T ; dg ; dS_{t-1} = dP Diag(alpha) */
+      /* dP = dS - de k^T ; dg ; dS_{t-1} = dP Lambda (dP Diag(alpha)) */
       for (int c = 0; c < dk; ++c) dgc[c] = 0.0;
-      for (int a = 0; a < dv; ++a) {
-        for (int c = 0; c < dk; ++c) {
-          size_t ix = (size_t)a * dk + c;
-          double dp = dS[ix] - dvt[a] * kt[c];
-          dgc[c] += dp * P[ix];
-          dS[ix] = dp * alpha[c];
+      if (p->gate == ORACLE_GATE_PHASE) {
+        for (int a = 0; a < dv; ++a) {
+          for (int j = 0; j < dk / 2; ++j) {
+            size_t ix = (size_t)a * dk + 2 * j;
+            double dpx = dS[ix] - dvt[a] * kt[2 * j];
+            double dpy = dS[ix + 1] - dvt[a] * kt[2 * j + 1];
+            double px = P[ix], py = P[ix + 1];
+            dgc[2 * j] += dpx * px + dpy * py;
+            dgc[2 * j + 1] += dpy * px - dpx * py;
+            dS[ix] = ac[j] * dpx + as[j] * dpy;
+            dS[ix + 1] = -as[j] * dpx + ac[j] * dpy;
+          }
+        }
+      } else {
+        for (int a = 0; a < dv; ++a) {
+          for (int c = 0; c < dk; ++c) {
+            size_t ix = (size_t)a * dk + c;
+            double dp = dS[ix] - dvt[a] * kt[c];
+            dgc[c] += dp * P[ix];
+            dS[ix] = dp * alpha[c];
+          }
         }
       }
-      if (p->gate == ORACLE_GATE_CHANNEL) {
+      if (p->gate == ORACLE_GATE_CHANNEL || p->gate == ORACLE_GATE_PHASE) {
         for (int c = 0; c < dk; ++c) dg[row * dk + c] = dgc[c];
       } else if (p->gate == ORACLE_GATE_SCALAR) {
         double s = 0.0;
@@ -276,6 +344,8 @@ static void oracle_bwd_head(const oproblem* p, int b, int h, const double* q,
   free(P);
   free(dS);
   free(alpha);
+  free(ac);
+  free(as);
   free(e);
   free(w);
   free(dgc);
