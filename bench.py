@@ -28,6 +28,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "fwd+bwd tokens/s (GDN/KDA, bf16, d=128); % of B200 tensor-core/HBM roofline"
+# The SFDA phase-gate workload has a forward only (no backward is built for it).
+METRIC_FWD = "fwd tokens/s (SFDA phase gate, bf16, d=128); % of B200 tensor-core/HBM roofline"
 UNIT = "tokens/s"
 # Used only when the measured-peaks file is absent (an earlier measurement on this GPU pool).
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -66,8 +68,9 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def algorithmic_step(w):
-    """Per-step algorithmic FLOPs and HBM bytes of forward + backward.
+def algorithmic_step(w, fwd_only=False):
+    """Per-step algorithmic FLOPs and HBM bytes of forward + backward (or of
+    the forward alone).
 
     FLOPs per token-head: forward 10 C d + 6 d^2, backward with recompute
     28 C d + 14 d^2 (d = d_k = d_v).  Bytes: every input read and output
@@ -77,11 +80,14 @@ def algorithmic_step(w):
     head.  Chunk states and other scratch are policy, not algorithm."""
     C, d = w.chunk, w.dk
     es = 2 if w.dtype == "bf16" else 4
-    gb = {"none": 0, "scalar": 4, "channel": 4 * w.dk}[w.gate]
+    gb = {"none": 0, "scalar": 4, "channel": 4 * w.dk, "phase": 4 * w.dk}[w.gate]
     th = w.token_heads
-    flops = th * (10 * C * d + 6 * d * d + 28 * C * d + 14 * d * d)
     io = (2 * w.dk + w.dv) * es + gb + 4
     fwd = io + w.dv * es
+    if fwd_only:
+        state = w.B * w.H * w.dv * w.dk * 4 * (1 + (1 if w.s0_std > 0 else 0))  # S_T (+ S0)
+        return th * (10 * C * d + 6 * d * d), th * fwd + state
+    flops = th * (10 * C * d + 6 * d * d + 28 * C * d + 14 * d * d)
     bwd = io + w.dv * es + (2 * w.dk + w.dv) * es + gb + 4
     nstate = 2 + (2 if w.s0_std > 0 else 0)  # S_T, dS0 (+ S0 read twice)
     state = w.B * w.H * w.dv * w.dk * 4 * nstate
@@ -195,11 +201,14 @@ class ClockSampler:
 
 
 def cpu_baseline(w, inp, seconds):
-    """Time the fp64 oracle (forward + backward) on host cores on a bounded
-    sample: all heads, the first T_s tokens, T_s sized to about `seconds`."""
+    """Time the fp64 oracle (forward + backward; forward only for the phase
+    gate) on host cores on a bounded sample: all heads, the first T_s tokens,
+    T_s sized to about `seconds`."""
     import oracle
 
     mode = oracle.BETA_KACZMARZ if w.beta_mode == "kaczmarz" else oracle.BETA_DIRECT
+    phase = w.gate == "phase"
+    gate = oracle.GATE_PHASE if phase else None
 
     def run(Ts):
         sl = {n: (None if inp[n] is None else inp[n][:, :Ts].double().numpy())
@@ -207,9 +216,11 @@ def cpu_baseline(w, inp, seconds):
         S0 = None if inp["S0"] is None else inp["S0"].double().numpy()
         t0 = time.perf_counter()
         _, _, thr = oracle.recurrent_fwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0,
-                                         beta_mode=mode, eps=w.eps, return_threads=True)
-        oracle.recurrent_bwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0, sl["dO"],
-                             beta_mode=mode, eps=w.eps)
+                                         beta_mode=mode, eps=w.eps, return_threads=True,
+                                         gate=gate)
+        if not phase:
+            oracle.recurrent_bwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0, sl["dO"],
+                                 beta_mode=mode, eps=w.eps)
         return time.perf_counter() - t0, thr
 
     probe = min(w.T, 128)
@@ -218,7 +229,8 @@ def cpu_baseline(w, inp, seconds):
     dt, thr = run(Ts)
     tokens_equiv = w.B * Ts  # all heads of B x Ts tokens
     return {"value": tokens_equiv / dt, "unit": UNIT, "cores": thr, "kind": "oracle",
-            "sample": f"fp64 oracle forward+backward on all {w.B * w.H} heads x the first "
+            "sample": f"fp64 oracle {'forward' if phase else 'forward+backward'} on all "
+                      f"{w.B * w.H} heads x the first "
                       f"{Ts} of {w.T} tokens of the same inputs, wall clock {dt:.1f} s",
             "seconds": dt}
 
@@ -236,6 +248,7 @@ def run_reference(args):
     inp = make_inputs(w)
     oracle.build()
     mode = oracle.BETA_KACZMARZ if w.beta_mode == "kaczmarz" else oracle.BETA_DIRECT
+    phase = w.gate == "phase"   # forward only: the phase gate has no backward
     total_steps = args.steps + args.warmup
     budget = 150.0  # seconds for the whole run
     per_step = budget / max(total_steps, 1)
@@ -248,9 +261,11 @@ def run_reference(args):
     def step(sl, S0):
         t0 = time.perf_counter()
         _, _, thr = oracle.recurrent_fwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0,
-                                         beta_mode=mode, eps=w.eps, return_threads=True)
-        oracle.recurrent_bwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0, sl["dO"],
-                             beta_mode=mode, eps=w.eps)
+                                         beta_mode=mode, eps=w.eps, return_threads=True,
+                                         gate=oracle.GATE_PHASE if phase else None)
+        if not phase:
+            oracle.recurrent_bwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0, sl["dO"],
+                                 beta_mode=mode, eps=w.eps)
         return time.perf_counter() - t0, thr
 
     probe = min(w.T, 64)
@@ -265,10 +280,11 @@ def run_reference(args):
         times.append(dt)
     tot = sum(times)
     value = w.B * Ts * args.steps / tot
-    desc = (f"fp64 oracle forward+backward per step on all {w.B * w.H} heads x the first {Ts} "
-            f"of {w.T} tokens of the workload's inputs")
+    desc = (f"fp64 oracle {'forward' if phase else 'forward+backward'} per step on all "
+            f"{w.B * w.H} heads x the first {Ts} of {w.T} tokens of the workload's inputs")
     print(json.dumps({
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "impl": "reference", "metric": METRIC_FWD if phase else METRIC, "value": value,
+        "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": tot / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -425,20 +441,24 @@ def main():
     inp = make_inputs(w, seed=w.seed + 1000 * rank)
     d = {n: (None if x is None else x.to(dev)) for n, x in inp.items()}
     plan = binding.Plan.for_workload(w, device=dev)
-    keep = args.policy == "save"
+    fwd_only = w.gate == "phase"   # the phase gate has no backward
+    keep = args.policy == "save" and not fwd_only
     saved = plan.new_saved() if keep else None
     o, ST, _ = plan.fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], saved=saved,
                         save=keep)
-    grads = plan.bwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], d["dO"], None, saved)
+    grads = {} if fwd_only else \
+        plan.bwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], d["dO"], None, saved)
     stream = torch.cuda.current_stream(dev)
 
     def step():
         plan.fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], o=o, ST=ST, saved=saved,
                  save=keep)
-        plan.bwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], d["dO"], None, saved,
-                 out=grads)
+        if not fwd_only:
+            plan.bwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], d["dO"], None, saved,
+                     out=grads)
 
-    in_bytes = sum(x.numel() * x.element_size() for x in d.values() if x is not None)
+    in_bytes = sum(x.numel() * x.element_size() for n, x in d.items()
+                   if x is not None and not (fwd_only and n == "dO"))
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
     for _ in range(args.warmup):
@@ -472,7 +492,8 @@ def main():
     # copied in and every output copied back, inside the timed region.
     e2e = None
     if not args.no_e2e:
-        hin = {n: (None if x is None else x.pin_memory()) for n, x in inp.items()}
+        hin = {n: (None if x is None or (fwd_only and n == "dO") else x.pin_memory())
+               for n, x in inp.items()}
         hout = {"o": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
                 "ST": torch.empty(ST.shape, dtype=ST.dtype).pin_memory()}
         for n, x in grads.items():
@@ -486,8 +507,9 @@ def main():
                     dev_in[n].copy_(x, non_blocking=True)
             plan.fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"], dev_in["g"],
                      dev_in["S0"], o=o, ST=ST, saved=saved, save=keep)
-            plan.bwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"], dev_in["g"],
-                     dev_in["S0"], dev_in["dO"], None, saved, out=grads)
+            if not fwd_only:
+                plan.bwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"], dev_in["g"],
+                         dev_in["S0"], dev_in["dO"], None, saved, out=grads)
             hout["o"].copy_(o, non_blocking=True)
             hout["ST"].copy_(ST, non_blocking=True)
             for n, x in grads.items():
@@ -546,7 +568,7 @@ def main():
                  "algorithmic_flops_per_launch": top["flops_per_launch"],
                  "traffic": ncu_traffic(top["name"], w.name)})
 
-    flops, nbytes = algorithmic_step(w)
+    flops, nbytes = algorithmic_step(w, fwd_only)
     t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     t_roof = max(t_tc, t_hbm)
@@ -560,7 +582,8 @@ def main():
         cpu = cpu_baseline(w, inp, args.cpu_seconds)
 
     out = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC_FWD if fwd_only else METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
@@ -570,7 +593,8 @@ def main():
                    "parallelism": f"replicas x{world} (independent batches, no collective)",
                    "l2": f"L2 flushed between timed steps ({2 * L2_BYTES >> 20} MiB write); "
                          f"inputs {in_bytes >> 20} MiB per step",
-                   "policy": ("forward saves chunk tiles and states; backward reads them"
+                   "policy": ("forward only (no backward for the phase gate)" if fwd_only
+                              else "forward saves chunk tiles and states; backward reads them"
                               if keep else "backward recomputes the chunk tiles and states")},
         "roofline": roof,
         "step_roofline": step_roof,

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libdr.so")
 
 DR_OK, DR_ERR_INVALID_ARG, DR_ERR_UNSUPPORTED, DR_ERR_WORKSPACE, DR_ERR_CUDA, DR_ERR_TIMEOUT = range(6)
 DR_F32, DR_BF16 = 0, 1
-GATES = {"none": 0, "scalar": 1, "channel": 2}
+GATES = {"none": 0, "scalar": 1, "channel": 2, "phase": 3}
 BETA_MODES = {"direct": 0, "kaczmarz": 1}
 
 
@@ -166,7 +166,8 @@ class Plan:
 
     def _shapes(self):
         B, T, H, dk, dv = self.B, self.T, self.H, self.dk, self.dv
-        g = None if self.gate == "none" else ((B, T, H, dk) if self.gate == "channel" else (B, T, H))
+        g = None if self.gate == "none" else \
+            ((B, T, H, dk) if self.gate in ("channel", "phase") else (B, T, H))
         return (B, T, H, dk), (B, T, H, dv), (B, T, H), g, (B, H, dv, dk)
 
     def _check_inputs(self, q, k, v, beta, g, S0):
@@ -233,12 +234,20 @@ def last_device_error(stream=None) -> int:
     return load().dr_last_device_error(_stream(stream))
 
 
+def _gate_of(g, gate):
+    if gate is not None:
+        return gate
+    return "none" if g is None else ("channel" if g.dim() == 4 else "scalar")
+
+
 def chunk_fwd(q, k, v, beta, g=None, S0=None, *, beta_mode="direct", eps=1e-6, chunk=64,
-              save=True, stream=None):
-    """One-shot forward: ``(o, S_T, saved)`` for inputs laid out as in include/dr.h."""
+              save=True, stream=None, gate=None):
+    """One-shot forward: ``(o, S_T, saved)`` for inputs laid out as in include/dr.h.
+    ``gate="phase"`` reads g as the SFDA rotation-decay gate (same shape as the
+    per-channel gate); otherwise the gate kind follows from g's shape."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    gate = "none" if g is None else ("channel" if g.dim() == 4 else "scalar")
+    gate = _gate_of(g, gate)
     dtype = "bf16" if q.dtype == torch.bfloat16 else "f32"
     plan = Plan(B, H, T, dk, dv, dtype=dtype, gate=gate, beta_mode=beta_mode, eps=eps,
                 chunk=chunk, device=q.device)
@@ -246,28 +255,30 @@ def chunk_fwd(q, k, v, beta, g=None, S0=None, *, beta_mode="direct", eps=1e-6, c
 
 
 def chunk_bwd(q, k, v, beta, g, S0, dO, dST=None, saved=None, *, beta_mode="direct",
-              eps=1e-6, chunk=64, stream=None):
+              eps=1e-6, chunk=64, stream=None, gate=None):
     """One-shot backward: dict of ``dq, dk, dv, dbeta, dg, dS0``."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    gate = "none" if g is None else ("channel" if g.dim() == 4 else "scalar")
+    gate = _gate_of(g, gate)
     dtype = "bf16" if q.dtype == torch.bfloat16 else "f32"
     plan = Plan(B, H, T, dk, dv, dtype=dtype, gate=gate, beta_mode=beta_mode, eps=eps,
                 chunk=chunk, device=q.device)
     return plan.bwd(q, k, v, beta, g, S0, dO, dST, saved, stream=stream)
 
 
-def decode_step(q, k, v, beta, g, S, *, beta_mode="direct", eps=1e-6, o=None, stream=None):
+def decode_step(q, k, v, beta, g, S, *, beta_mode="direct", eps=1e-6, o=None, stream=None,
+                gate=None):
     """One token per head through the recurrent update, S updated in place.
 
     q, k ``[B,1,H,dk]``, v ``[B,1,H,dv]`` (bf16 or fp32), beta ``[B,1,H]``,
-    g ``None`` / ``[B,1,H]`` / ``[B,1,H,dk]`` fp32, S ``[B,H,dv,dk]`` fp32.
+    g ``None`` / ``[B,1,H]`` / ``[B,1,H,dk]`` fp32 (``gate="phase"`` for the
+    SFDA rotation-decay gate), S ``[B,H,dv,dk]`` fp32.
     Returns o ``[B,1,H,dv]`` in the storage dtype."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
     tdt = q.dtype
-    gate = "none" if g is None else ("channel" if g.dim() == 4 else "scalar")
+    gate = _gate_of(g, gate)
     prob = make_problem(B, H, T, dk, dv, dtype="bf16" if tdt == torch.bfloat16 else "f32",
                         gate=gate, beta_mode=beta_mode, eps=eps)
     _need(q, "q", tdt, (B, 1, H, dk), dev)
@@ -275,7 +286,8 @@ def decode_step(q, k, v, beta, g, S, *, beta_mode="direct", eps=1e-6, o=None, st
     _need(v, "v", tdt, (B, 1, H, dv), dev)
     _need(beta, "beta", torch.float32, (B, 1, H), dev)
     if g is not None:
-        _need(g, "g", torch.float32, (B, 1, H, dk) if gate == "channel" else (B, 1, H), dev)
+        _need(g, "g", torch.float32,
+              (B, 1, H, dk) if gate in ("channel", "phase") else (B, 1, H), dev)
     _need(S, "S", torch.float32, (B, H, dv, dk), dev)
     if o is None:
         o = torch.empty(B, 1, H, dv, dtype=tdt, device=dev)

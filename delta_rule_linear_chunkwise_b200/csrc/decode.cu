@@ -6,7 +6,11 @@
 // so a warp owns four rows (128 keys = 4 per lane: four 512-byte loads in
 // flight, then two warp reductions per row).  The step is HBM-bound: it reads and
 // writes the d_v x d_k fp32 state once per token.  In Kaczmarz mode
-// beta = eta / (||k||^2 + eps), each warp forming ||k||^2 itself.
+// beta = eta / (||k||^2 + eps), each warp forming ||k||^2 itself.  With the
+// SFDA phase gate (PHASE) the decay is the 2 x 2 rotation-decay block of each
+// key pair, (x, y) <- alpha (cos theta x - sin theta y, sin theta x + cos theta y)
+// (the explainer's Lambda_t = diag(alpha e^{i theta}) in real coordinates); a
+// lane's four keys are two whole pairs.
 
 #include "dr_common.cuh"
 
@@ -36,7 +40,7 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-template <typename T>
+template <typename T, bool PHASE>
 __global__ void __launch_bounds__(kDecodeThreads)
     k_decode_step(Problem p, const T* __restrict__ q, const T* __restrict__ k,
                   const T* __restrict__ v, const float* __restrict__ beta,
@@ -53,6 +57,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
   float4 s[kRows];
   float4 kk = make_float4(0.f, 0.f, 0.f, 0.f), qq = kk;
   float4 al = make_float4(1.f, 1.f, 1.f, 1.f);
+  float4 rot = make_float4(0.f, 0.f, 0.f, 0.f);  // PHASE: (a cos, a sin) of the two pairs
   float* srow = S + row0 * p.dk;
 #pragma unroll
   for (int r = 0; r < kRows; ++r)
@@ -61,7 +66,14 @@ __global__ void __launch_bounds__(kDecodeThreads)
   if (act) {
     kk = load4<T>(k + head * p.dk + c0);
     qq = load4<T>(q + head * p.dk + c0);
-    if (p.gate == kGateChannel) {
+    if (PHASE) {
+      const float4 gg = *reinterpret_cast<const float4*>(g + head * p.dk + c0);
+      float s0, c0r, s1, c1r;
+      sincosf(gg.y, &s0, &c0r);
+      sincosf(gg.w, &s1, &c1r);
+      const float a0 = __expf(gg.x), a1 = __expf(gg.z);
+      rot = make_float4(a0 * c0r, a0 * s0, a1 * c1r, a1 * s1);
+    } else if (p.gate == kGateChannel) {
       const float4 gg = *reinterpret_cast<const float4*>(g + head * p.dk + c0);
       al = make_float4(__expf(gg.x), __expf(gg.y), __expf(gg.z), __expf(gg.w));
     } else if (p.gate == kGateScalar) {
@@ -80,10 +92,18 @@ __global__ void __launch_bounds__(kDecodeThreads)
   float pk[kRows];
 #pragma unroll
   for (int r = 0; r < kRows; ++r) {
-    s[r].x *= al.x;
-    s[r].y *= al.y;
-    s[r].z *= al.z;
-    s[r].w *= al.w;
+    if (PHASE) {
+      const float x0 = s[r].x, y0 = s[r].y, x1 = s[r].z, y1 = s[r].w;
+      s[r].x = rot.x * x0 - rot.y * y0;
+      s[r].y = rot.y * x0 + rot.x * y0;
+      s[r].z = rot.z * x1 - rot.w * y1;
+      s[r].w = rot.w * x1 + rot.z * y1;
+    } else {
+      s[r].x *= al.x;
+      s[r].y *= al.y;
+      s[r].z *= al.z;
+      s[r].w *= al.w;
+    }
     pk[r] = s[r].x * kk.x + s[r].y * kk.y + s[r].z * kk.z + s[r].w * kk.w;
   }
 #pragma unroll
@@ -121,16 +141,26 @@ cudaError_t launch_decode_step(const Problem& p, int bf16, const void* q, const 
   const double heads = (double)p.B * p.H, es = bf16 ? 2.0 : 4.0;
   // reads and writes the fp32 state; reads q, k, v, beta, g; writes o
   const double bytes = heads * (2.0 * p.dv * p.dk * 4 + (2.0 * p.dk + 2.0 * p.dv) * es + 4 +
-                                (p.gate == kGateChannel ? p.dk * 4 : p.gate == kGateScalar ? 4 : 0));
+                                (p.gate == kGateChannel || p.gate == kGatePhase ? p.dk * 4
+                                 : p.gate == kGateScalar                        ? 4
+                                                                                : 0));
   const double flops = heads * p.dv * p.dk * 7.0;
   prof_begin(kKDecode, bytes, flops, st);
-  if (bf16)
-    k_decode_step<__nv_bfloat16><<<blocks, kDecodeThreads, 0, st>>>(
-        p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, beta, g, S,
-        (__nv_bfloat16*)o);
-  else
-    k_decode_step<float><<<blocks, kDecodeThreads, 0, st>>>(
+  using bf = __nv_bfloat16;
+  if (p.gate == kGatePhase) {
+    if (bf16)
+      k_decode_step<bf, true><<<blocks, kDecodeThreads, 0, st>>>(
+          p, (const bf*)q, (const bf*)k, (const bf*)v, beta, g, S, (bf*)o);
+    else
+      k_decode_step<float, true><<<blocks, kDecodeThreads, 0, st>>>(
+          p, (const float*)q, (const float*)k, (const float*)v, beta, g, S, (float*)o);
+  } else if (bf16) {
+    k_decode_step<bf, false><<<blocks, kDecodeThreads, 0, st>>>(
+        p, (const bf*)q, (const bf*)k, (const bf*)v, beta, g, S, (bf*)o);
+  } else {
+    k_decode_step<float, false><<<blocks, kDecodeThreads, 0, st>>>(
         p, (const float*)q, (const float*)k, (const float*)v, beta, g, S, (float*)o);
+  }
   const cudaError_t e = cudaGetLastError();
   prof_end(st);
   return e;

@@ -24,7 +24,7 @@ dr_status validate(const dr_problem* in, Problem* out) {
   if (in->B < 1 || in->H < 1 || in->T < 1 || in->dk < 1 || in->dv < 1)
     return DR_ERR_INVALID_ARG;
   if (in->dtype != DR_F32 && in->dtype != DR_BF16) return DR_ERR_INVALID_ARG;
-  if (in->gate < DR_GATE_NONE || in->gate > DR_GATE_CHANNEL) return DR_ERR_INVALID_ARG;
+  if (in->gate < DR_GATE_NONE || in->gate > DR_GATE_PHASE) return DR_ERR_INVALID_ARG;
   if (in->beta_mode != DR_BETA_DIRECT && in->beta_mode != DR_BETA_KACZMARZ)
     return DR_ERR_INVALID_ARG;
   if (!(in->eps >= 0.f)) return DR_ERR_INVALID_ARG;
@@ -40,7 +40,7 @@ dr_status validate(const dr_problem* in, Problem* out) {
   out->NC = (in->T + dr::kC - 1) / dr::kC;
   out->gate = in->gate;
   out->beta_mode = in->beta_mode;
-  out->gk = (in->gate == DR_GATE_CHANNEL) ? in->dk : 1;
+  out->gk = (in->gate == DR_GATE_CHANNEL || in->gate == DR_GATE_PHASE) ? in->dk : 1;
   out->eps = in->eps;
   return DR_OK;
 }
@@ -130,26 +130,27 @@ int chunk_bwd_kind() {
 }
 
 // The two state scans likewise: tcgen05 with the state in registers and the
-// products in TMEM (default), or warp-level mma.sync tiles (DR_MMA_SYNC_SCAN=1).
-bool use_mma_sync_scans() {
+// products in TMEM (default), or warp-level mma.sync tiles (DR_MMA_SYNC_SCAN=1;
+// not for the phase gate, whose pair-mixing decay only the tcgen05 scan has).
+bool use_mma_sync_scans(const Problem& P) {
   const char* e = getenv("DR_MMA_SYNC_SCAN");
-  return e && e[0] == '1';
+  return e && e[0] == '1' && P.gate != dr::kGatePhase;
 }
 cudaError_t fwd_scan(const dr::Problem& P, const dr::fast::Saved& sv, const float* S0,
                      __nv_bfloat16* o, float* ST, bool save, cudaStream_t st) {
-  if (use_mma_sync_scans()) return dr::fast::launch_fwd_scan(P, sv, S0, o, ST, save, st);
+  if (use_mma_sync_scans(P)) return dr::fast::launch_fwd_scan(P, sv, S0, o, ST, save, st);
   return dr::fast::launch_fwd_scan_tc(P, sv, S0, o, ST, save, st);
 }
 cudaError_t bwd_scan(const dr::Problem& P, const dr::fast::Saved& sv, const __nv_bfloat16* dO,
                      const float* dST, float* dS0, __nv_bfloat16* dU, __nv_bfloat16* dh,
                      cudaStream_t st) {
-  if (use_mma_sync_scans()) return dr::fast::launch_bwd_scan(P, sv, dO, dST, dS0, dU, dh, st);
+  if (use_mma_sync_scans(P)) return dr::fast::launch_bwd_scan(P, sv, dO, dST, dS0, dU, dh, st);
   return dr::fast::launch_bwd_scan_tc(P, sv, dO, dST, dS0, dU, dh, st);
 }
 
 // Segments of the chunk-parallel affine scan for this problem (1 = sequential).
 int scan_segments(const Problem& P) {
-  return use_mma_sync_scans() ? 1 : dr::fast::affine_segments(P);
+  return use_mma_sync_scans(P) ? 1 : dr::fast::affine_segments(P);
 }
 
 // The forward state scan, plain or segmented.  Segmented: the transfer
@@ -240,7 +241,10 @@ dr_status dr_chunk_fwd(const dr_problem* p, const void* q, const void* k, const 
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
   if (P.gate == DR_GATE_NONE) g = nullptr;
-  if (dr::fast::eligible(P, p->dtype == DR_BF16)) {
+  const bool fast = dr::fast::eligible(P, p->dtype == DR_BF16);
+  // the phase gate runs on the tensor-core path only
+  if (P.gate == DR_GATE_PHASE && !fast) return DR_ERR_UNSUPPORTED;
+  if (fast) {
     // Tensor-core path: the per-chunk tiles go to the saved buffer when given
     // (the backward reuses them), else to the workspace.
     dr::fast::Saved sv = dr::fast::carve_saved(P, saved ? saved : ws);
@@ -288,6 +292,7 @@ dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const 
   if (!q || !k || !v || !beta || !dO || !dq || !dk || !dv || !dbeta)
     return DR_ERR_INVALID_ARG;
   if ((P.gate == DR_GATE_NONE) != (g == nullptr)) return DR_ERR_INVALID_ARG;
+  if (P.gate == DR_GATE_PHASE) return DR_ERR_UNSUPPORTED;  // forward and decode only
   if (P.gate != DR_GATE_NONE && !dg) return DR_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, beta, g, S0, dO, dST, saved, dq, dk, dv, dbeta, dg, dS0};
   for (const void* x : ptrs)
@@ -343,7 +348,7 @@ const char* dr_status_string(dr_status s) {
   switch (s) {
     case DR_OK: return "ok";
     case DR_ERR_INVALID_ARG: return "invalid argument";
-    case DR_ERR_UNSUPPORTED: return "unsupported problem (chunk must be 64; dk, dv multiples of 16 up to 128)";
+    case DR_ERR_UNSUPPORTED: return "unsupported problem (chunk must be 64; dk, dv multiples of 16 up to 128; phase gate: bf16, dk = dv = 128, no backward)";
     case DR_ERR_WORKSPACE: return "workspace or saved buffer missing, misaligned or too small";
     case DR_ERR_CUDA: return "CUDA error";
     case DR_ERR_TIMEOUT: return "a bounded device-side wait timed out";

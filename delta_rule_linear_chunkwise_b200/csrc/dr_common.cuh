@@ -11,13 +11,13 @@ namespace dr {
 constexpr int kC = 64;         // chunk length (tokens); the only supported value
 constexpr int kThreads = 256;  // threads per CTA of the generic kernels
 
-enum { kGateNone = 0, kGateScalar = 1, kGateChannel = 2 };
+enum { kGateNone = 0, kGateScalar = 1, kGateChannel = 2, kGatePhase = 3 };
 enum { kBetaDirect = 0, kBetaKaczmarz = 1 };
 
 struct Problem {
   int B, H, T, dk, dv;
   int NC;         // number of chunks, ceil(T / 64)
-  int gate;       // kGate*
+  int gate;       // kGate* (kGatePhase: SFDA pairs, log alpha at 2j, theta at 2j + 1)
   int beta_mode;  // kBeta*
   int gk;         // columns of the cumulative gate per row: dk (per-channel) or 1
   float eps;

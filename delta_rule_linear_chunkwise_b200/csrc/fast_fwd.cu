@@ -101,6 +101,16 @@ struct PrepSmem {
   float beta[C];
 };
 
+// PHASE: the SFDA rotation-decay gate.  Its per-channel cumulative sums hold,
+// for key pair m, gamma (cumulative log alpha) at channel 2m and the cumulative
+// phase Theta at 2m + 1; the chunk's decay from its start to row i is then
+// Gamma_i ~ e^{gamma_i} e^{-i Theta_i} on each pair read as a complex number
+// (x + i y), and the factors below are those of the gate-free chunk form with
+// read keys Gamma_i k_i, write keys Gamma_i^{-T} k_i, queries Gamma_i q_i and
+// end-of-chunk keys Gamma_C^T Gamma_i^{-T} k_i ("Konstruktives Chunk-WY-
+// Theorem", SFDA explainer): per pair, a rotation and a scale.  The decay row
+// holds (e^{gamma_C} cos Theta_C, e^{gamma_C} sin Theta_C) per pair.
+template <bool PHASE>
 __global__ void __launch_bounds__(NT, 2)
     k_prep(Problem p, const bf16* __restrict__ q, const bf16* __restrict__ k,
            const bf16* __restrict__ v, const float* __restrict__ beta_in,
@@ -151,7 +161,9 @@ __global__ void __launch_bounds__(NT, 2)
   // Factors: K^c, Kb^c, Q^c to shared memory; Qh, Kt, beta, dec to global.
   const int r = centre_row(nvalid);
   // per-column factors of this thread's segment: e^{-gamma_r}, e^{gamma_C - gamma_r}
+  // (phase gate: at the even channels; e^{i Theta_r}, e^{i Theta_C} per pair)
   float ier8[8], ecr8[8];
+  float rc4[4], rs4[4], cc4[4], cs4[4], gr4[4];
   {
     float r8[8], c8[8];
     gate8(G, gk, r, (tid & 15) * 8, r8);
@@ -160,6 +172,14 @@ __global__ void __launch_bounds__(NT, 2)
     for (int e = 0; e < 8; ++e) {
       ier8[e] = __expf(-r8[e]);
       ecr8[e] = __expf(c8[e] - r8[e]);
+    }
+    if (PHASE) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        gr4[m] = r8[2 * m];
+        sincosf(r8[2 * m + 1], &rs4[m], &rc4[m]);
+        sincosf(c8[2 * m + 1], &cs4[m], &cc4[m]);
+      }
     }
   }
 #pragma unroll
@@ -172,16 +192,47 @@ __global__ void __launch_bounds__(NT, 2)
     unpack8(rq, qv);
     gate8(G, gk, i, j * 8, g8);
     float kc[8], kb[8], qc[8], qh[8], kt[8], nn = 0.f;
+    if (PHASE) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float eg = __expf(g8[e]);                              // e^gamma
-      const float ep = eg * ier8[e], em = __fdividef(1.f, ep);     // e^{+-(gamma - gamma_r)}
-      kc[e] = kv[e] * ep;
-      kb[e] = kv[e] * em;
-      qc[e] = qv[e] * ep;
-      qh[e] = qv[e] * eg;
-      kt[e] = kb[e] * ecr8[e];  // k e^{gamma_C - gamma}
-      nn += kv[e] * kv[e];
+      for (int m = 0; m < 4; ++m) {
+        const int e = 2 * m;
+        float sn, cs;
+        sincosf(g8[e + 1], &sn, &cs);                              // e^{-i Theta} = cs - i sn
+        const float eg = __expf(g8[e]);                            // e^gamma
+        // e^{+-(gamma - gamma_r)} from the centred exponent itself: within half
+        // a chunk's decay of 1, so it stays finite where e^gamma underflows
+        const float ep = __expf(g8[e] - gr4[m]), em = __expf(gr4[m] - g8[e]);
+        // e^{-i (Theta - Theta_r)} and e^{i (Theta_C - Theta)}
+        const float wr = cs * rc4[m] + sn * rs4[m], wi = cs * rs4[m] - sn * rc4[m];
+        const float tr = cc4[m] * cs + cs4[m] * sn, ti = cs4[m] * cs - cc4[m] * sn;
+        const float kx = kv[e], ky = kv[e + 1], qx = qv[e], qy = qv[e + 1];
+        const float kwx = wr * kx - wi * ky, kwy = wi * kx + wr * ky;
+        const float qwx = wr * qx - wi * qy, qwy = wi * qx + wr * qy;
+        kc[e] = ep * kwx;
+        kc[e + 1] = ep * kwy;
+        kb[e] = em * kwx;
+        kb[e + 1] = em * kwy;
+        qc[e] = ep * qwx;
+        qc[e + 1] = ep * qwy;
+        qh[e] = eg * (cs * qx + sn * qy);                          // Gamma q
+        qh[e + 1] = eg * (cs * qy - sn * qx);
+        const float sc = em * ecr8[e];                             // e^{gamma_C - gamma}
+        kt[e] = sc * (tr * kx - ti * ky);                          // Gamma_C^T Gamma^{-T} k
+        kt[e + 1] = sc * (ti * kx + tr * ky);
+        nn += kx * kx + ky * ky;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float eg = __expf(g8[e]);                              // e^gamma
+        const float ep = eg * ier8[e], em = __fdividef(1.f, ep);     // e^{+-(gamma - gamma_r)}
+        kc[e] = kv[e] * ep;
+        kb[e] = kv[e] * em;
+        qc[e] = qv[e] * ep;
+        qh[e] = qv[e] * eg;
+        kt[e] = kb[e] * ecr8[e];  // k e^{gamma_C - gamma}
+        nn += kv[e] * kv[e];
+      }
     }
     *reinterpret_cast<uint4*>(s.R1 + i * LDD + j * 8) = pack8(kc);
     *reinterpret_cast<uint4*>(s.R2 + i * LDD + j * 8) = pack8(kb);
@@ -203,7 +254,17 @@ __global__ void __launch_bounds__(NT, 2)
       sv.knorm[cb * C + i] = nn;
     }
   }
-  if (tid < D) sv.dec[cb * D + tid] = __expf(gk == D ? G[(C - 1) * D + tid] : G[C - 1]);
+  if (PHASE) {
+    if (tid < D / 2) {
+      float sn, cs;
+      sincosf(G[(C - 1) * D + 2 * tid + 1], &sn, &cs);
+      const float a = __expf(G[(C - 1) * D + 2 * tid]);
+      sv.dec[cb * D + 2 * tid] = a * cs;
+      sv.dec[cb * D + 2 * tid + 1] = a * sn;
+    }
+  } else if (tid < D) {
+    sv.dec[cb * D + tid] = __expf(gk == D ? G[(C - 1) * D + tid] : G[C - 1]);
+  }
 #pragma unroll
   for (int it = 0; it < ITEMS; ++it) {
     const int idx = tid + it * NT, i = idx >> 4, j = idx & 15;
@@ -247,8 +308,19 @@ __global__ void __launch_bounds__(NT, 2)
     unpack8(kr[it], kv);
     gate8(G, gk, i, j * 8, g8);
     const float bi = s.beta[i];
+    if (PHASE) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) kv[e] *= bi * __expf(g8[e]);
+      for (int m = 0; m < 4; ++m) {
+        float sn, cs;
+        sincosf(g8[2 * m + 1], &sn, &cs);
+        const float a = bi * __expf(g8[2 * m]), kx = kv[2 * m], ky = kv[2 * m + 1];
+        kv[2 * m] = a * (cs * kx + sn * ky);                 // beta Gamma k
+        kv[2 * m + 1] = a * (cs * ky - sn * kx);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) kv[e] *= bi * __expf(g8[e]);
+    }
     *reinterpret_cast<uint4*>(s.R1 + i * LDD + j * 8) = pack8(kv);
   }
   __syncthreads();  // A ready; the gate is no longer needed
@@ -465,7 +537,9 @@ __global__ void __launch_bounds__(NT, 1)
 cudaError_t launch_prep(const Problem& p, const bf16* q, const bf16* k, const bf16* v,
                         const float* beta, const float* g, const Saved& sv, cudaStream_t st) {
   const size_t sm = sizeof(PrepSmem);
-  cudaError_t e = cudaFuncSetAttribute(k_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  const bool phase = p.gate == kGatePhase;
+  cudaError_t e = cudaFuncSetAttribute(phase ? k_prep<true> : k_prep<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const double nb = (double)p.B * p.H * p.NC, ntok = nb * C;
   // reads q, k, v, g, beta; writes T, beta, dec, W, U', M, Qh, Kt
@@ -473,7 +547,10 @@ cudaError_t launch_prep(const Problem& p, const bf16* q, const bf16* k, const bf
                        nb * ((double)kTBytes + kBetaBytes + kDecBytes + 4.0 * kTileBytes + kMBytes);
   const double flops = nb * (2.0 * 2 * C * C * D + 2.0 * 2 * C * C * D);  // [A;M] Gram, W|U'
   prof_begin(kKTcIntraFwd, bytes, flops, st);
-  k_prep<<<dim3(p.NC, p.H, p.B), NT, sm, st>>>(p, q, k, v, beta, g, sv);
+  if (phase)
+    k_prep<true><<<dim3(p.NC, p.H, p.B), NT, sm, st>>>(p, q, k, v, beta, g, sv);
+  else
+    k_prep<false><<<dim3(p.NC, p.H, p.B), NT, sm, st>>>(p, q, k, v, beta, g, sv);
   e = cudaGetLastError();
   prof_end(st);
   return e;

@@ -116,7 +116,10 @@ __device__ __forceinline__ bool cta_wait(uint64_t* bar, int parity) {
   return bad == 0;
 }
 
-template <int BV>
+// PHASE: the SFDA rotation-decay gate.  The chunk decay then mixes the key
+// pair (2j, 2j + 1) of every state row as the complex product
+// (dec[2j] + i dec[2j+1]) (x + i y); the pair's two keys sit on adjacent lanes.
+template <int BV, bool PHASE>
 __global__ void __launch_bounds__(NTF, 1)
     k_fwd_scan_tc(Problem p, Saved sv, ScanSeg sg, bf16* __restrict__ o, int save,
                   int* __restrict__ err) {
@@ -226,7 +229,8 @@ __global__ void __launch_bounds__(NTF, 1)
     const size_t cb = chunk_id(p, b, h, n);
     ScanStage<BV>& st = s.st[it & 1];
     const int buf = it & 1;
-    const float dc = st.dec[c];  // read before the stage is refilled below
+    const float dc = st.dec[PHASE ? (c & ~1) : c];  // read before the stage is refilled below
+    const float di = PHASE ? ((c & 1) ? st.dec[c] : -st.dec[c | 1]) : 0.f;
     // MMA-A: [W ; q e^gamma] S^T
     if (tid == 0) {
       const uint64_t dA = tc::sdesc_kmaj(st.AWQ, D, 0);
@@ -305,8 +309,17 @@ __global__ void __launch_bounds__(NTF, 1)
       for (int q16 = 0; q16 < HB / 16; ++q16)
         tc::tmem_ld16_nowait(lane_addr(tbase, warp, T_S + ah * HB + 16 * q16), r + 16 * q16);
       tc::tmem_wait_ld();
+      if (PHASE) {
+        // own key c: Re (even c) or Im (odd c) of (dec_re + i dec_im)(x + i y)
 #pragma unroll
-      for (int e = 0; e < HB; ++e) S[e] = S[e] * dc + __uint_as_float(r[e]);
+        for (int e = 0; e < HB; ++e) {
+          const float partner = __shfl_xor_sync(0xffffffffu, S[e], 1);
+          S[e] = S[e] * dc + di * partner + __uint_as_float(r[e]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < HB; ++e) S[e] = S[e] * dc + __uint_as_float(r[e]);
+      }
       write_sb();
     }
     frag::cp_wait<1>();
@@ -337,7 +350,8 @@ cudaError_t launch_fwd_scan_tc_bv(const Problem& p, const Saved& sv, const ScanS
   float* ST = sg.ST;
   const int maps = sg.mode == 3 ? 2 : 1;  // mode 3 runs both map kinds
   const size_t sm = sizeof(ScanSmem<BV>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_fwd_scan_tc<BV>,
+  const bool phase = p.gate == kGatePhase;
+  cudaError_t e = cudaFuncSetAttribute(phase ? k_fwd_scan_tc<BV, true> : k_fwd_scan_tc<BV, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const double nb = (double)p.B * p.H * p.NC, ntok = nb * C, heads = (double)p.B * p.H;
@@ -350,8 +364,12 @@ cudaError_t launch_fwd_scan_tc_bv(const Problem& p, const Saved& sv, const ScanS
   const double flops =
       maps * nb * (2.0 * C * D * D * (o ? 3 : 2) + (o ? 2.0 * C * C * D : 0.0));
   prof_begin(kKTcScanFwd, bytes, flops, st);
-  k_fwd_scan_tc<BV><<<dim3(maps * (D / BV), p.H, p.B * sg.G), NTF, sm, st>>>(
-      p, sv, sg, o, save ? 1 : 0, device_error_word());
+  const dim3 grid(maps * (D / BV), p.H, p.B * sg.G);
+  if (phase)
+    k_fwd_scan_tc<BV, true><<<grid, NTF, sm, st>>>(p, sv, sg, o, save ? 1 : 0, device_error_word());
+  else
+    k_fwd_scan_tc<BV, false><<<grid, NTF, sm, st>>>(p, sv, sg, o, save ? 1 : 0,
+                                                    device_error_word());
   e = cudaGetLastError();
   prof_end(st);
   return e;

@@ -9,8 +9,12 @@ Kaczmarz workload); v ~ N(0, 1); beta (or eta) = sigmoid(N(0, 1)); log-gate
 g = logsigmoid(N(mu, 1)) with mu = 3 (mu = 4 for the long-context Kaczmarz
 workload), one per head and token (scalar gate) or per key channel (KDA);
 dO ~ N(0, 1); optional initial state S0 ~ N(0, 0.1) (0.1 is the standard
-deviation).  Values are drawn in fp32 from ``torch.Generator(seed)`` in the fixed
-order q, k, v, beta-logits, g-logits, dO, S0, then q/k/v/dO are rounded to
+deviation).  The SFDA phase gate (one rotation-decay per key pair) draws the
+pair decays log alpha = logsigmoid(N(mu, 1)) and then the phases theta ~
+U(-pi, pi) (a phase per pair and token; the explainer's cyclic counter uses
+2 pi / 5), interleaved as g[..., 2j] = log alpha_j, g[..., 2j+1] = theta_j.
+Values are drawn in fp32 from ``torch.Generator(seed)`` in the fixed
+order q, k, v, beta-logits, g-logits (then phases), dO, S0, then q/k/v/dO are rounded to
 bf16 (round-to-nearest-even) for bf16 workloads; beta, g and S0 stay fp32.  The
 oracle receives exactly these rounded values, upcast to fp64.
 
@@ -34,7 +38,7 @@ class Workload:
     dv: int = 128
     chunk: int = 64
     dtype: str = "bf16"          # "f32" or "bf16": storage type of q, k, v, o, dO
-    gate: str = "scalar"         # "none" | "scalar" | "channel"
+    gate: str = "scalar"         # "none" | "scalar" | "channel" | "phase"
     beta_mode: str = "direct"    # "direct" | "kaczmarz"
     g_mean: float = 3.0
     eps: float = 1e-6
@@ -69,6 +73,9 @@ WORKLOADS = {
     "kla_bf16_b1h16t65536": Workload("kla_bf16_b1h16t65536", B=1, H=16, T=65536,
                                      gate="scalar", beta_mode="kaczmarz", g_mean=4.0,
                                      normalize_k=False, seed=4),
+    # SFDA: the KDA sizes with the rotation-decay gate (forward and decode only)
+    "sfda_bf16_b4h16t8192": Workload("sfda_bf16_b4h16t8192", B=4, H=16, T=8192,
+                                     gate="phase", seed=5),
 }
 
 # The headline benchmark workload (KDA per-channel gate, B4 H16 T8192 d128).
@@ -99,9 +106,15 @@ def make_inputs(w: Workload, seed: int | None = None, device="cpu") -> dict:
         k = _l2norm(k)
     v = normal(B, T, H, dv)
     beta = torch.sigmoid(normal(B, T, H))
-    g_shape = (B, T, H, dk) if w.gate == "channel" else (B, T, H)
-    g_logit = normal(*g_shape, mean=w.g_mean)
-    g = None if w.gate == "none" else torch.nn.functional.logsigmoid(g_logit)
+    if w.gate == "phase":
+        logalpha = torch.nn.functional.logsigmoid(normal(B, T, H, dk // 2, mean=w.g_mean))
+        theta = (torch.rand(B, T, H, dk // 2, generator=gen, dtype=torch.float32) * 2 - 1) \
+            * torch.pi
+        g = torch.stack([logalpha, theta], dim=-1).reshape(B, T, H, dk).contiguous()
+    else:
+        g_shape = (B, T, H, dk) if w.gate == "channel" else (B, T, H)
+        g_logit = normal(*g_shape, mean=w.g_mean)
+        g = None if w.gate == "none" else torch.nn.functional.logsigmoid(g_logit)
     dO = normal(B, T, H, dv)
     S0 = normal(B, H, dv, dk, std=w.s0_std) if w.s0_std > 0 else None
     sdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32

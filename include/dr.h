@@ -31,8 +31,17 @@
  *    memory and keeps no pointer after a call returns.
  *  - Layouts: q, k [B, T, H, dk]; v, o, dO [B, T, H, dv] (storage dtype
  *    dr_problem.dtype); beta [B, T, H] fp32; g [B, T, H] fp32 (scalar gate)
- *    or [B, T, H, dk] fp32 (per-channel gate), NULL for gate NONE;
+ *    or [B, T, H, dk] fp32 (per-channel and phase gates), NULL for gate NONE;
  *    S0, ST, dST, dS0 [B, H, dv, dk] fp32.
+ *  - Phase gate (DR_GATE_PHASE, SFDA: the explainer's complex diagonal
+ *    Lambda_t = diag(alpha_t e^{i theta_t}), section "Kernarchitektur", in
+ *    real coordinates): key channels pair up as (2j, 2j+1); g[..., 2j] is
+ *    log alpha_j and g[..., 2j+1] the phase theta_j (radians), and the decay
+ *    maps each state row's pair (x, y) to
+ *    alpha_j (cos theta_j x - sin theta_j y, sin theta_j x + cos theta_j y)
+ *    before the erase-and-write (zero phase: KDA with each pair's channels
+ *    sharing one decay).  Supported by dr_chunk_fwd (bf16, dk = dv = 128) and
+ *    dr_decode_step; dr_chunk_bwd returns DR_ERR_UNSUPPORTED for it.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *    stream).  Arguments are validated on the host before any launch; a
  *    non-DR_OK status means nothing was launched, except DR_ERR_CUDA, which
@@ -60,7 +69,12 @@ typedef enum {
 } dr_status;
 
 typedef enum { DR_F32 = 0, DR_BF16 = 1 } dr_dtype;
-typedef enum { DR_GATE_NONE = 0, DR_GATE_SCALAR = 1, DR_GATE_CHANNEL = 2 } dr_gate;
+typedef enum {
+  DR_GATE_NONE = 0,     /* alpha = 1 (DeltaNet) */
+  DR_GATE_SCALAR = 1,   /* one log-gate per head and token (GDN) */
+  DR_GATE_CHANNEL = 2,  /* one log-gate per key channel (KDA) */
+  DR_GATE_PHASE = 3     /* SFDA rotation-decay per key pair (see above) */
+} dr_gate;
 typedef enum { DR_BETA_DIRECT = 0, DR_BETA_KACZMARZ = 1 } dr_beta_mode;
 
 /* Problem description.  Supported: B, H, T >= 1; chunk == 64;
@@ -85,6 +99,9 @@ dr_status dr_saved_size(const dr_problem* p, size_t* bytes);
 /* Chunkwise forward.
    In:  q, k, v, beta (eta in Kaczmarz mode), g (NULL iff gate NONE),
         S0 (NULL = zero initial state).
+   The phase gate needs dtype DR_BF16 and dk = dv = 128 (else
+   DR_ERR_UNSUPPORTED); its chunk decay is the per-pair rotation-decay
+   product, the rest of the chunk form is unchanged.
    Out: o (storage dtype), ST (final state, fp32; NULL = not wanted),
         saved (NULL = not wanted; else dr_saved_size bytes, which dr_chunk_bwd
         may then read instead of recomputing the states).
@@ -101,6 +118,7 @@ dr_status dr_chunk_fwd(const dr_problem* p, const void* q, const void* k, const 
    Out: dq, dk, dv (storage dtype), dbeta (fp32; d/deta in Kaczmarz mode),
         dg (fp32, shaped like g; ignored and may be NULL for gate NONE),
         dS0 (fp32; NULL = not wanted).
+   The phase gate has no backward yet: DR_ERR_UNSUPPORTED, nothing launched.
    ws:  at least dr_workspace_size(p, 1) bytes, 256-byte aligned. */
 dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const void* v,
                        const float* beta, const float* g, const float* S0, const void* dO,
@@ -119,8 +137,9 @@ dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const 
    p:   as for the chunkwise calls with T == 1 (chunk is not used but must be
         64); any other T gives DR_ERR_INVALID_ARG.
    In:  q, k [B,1,H,dk] and v [B,1,H,dv] in the storage dtype, beta [B,1,H]
-        fp32, g [B,1,H] (scalar gate) or [B,1,H,dk] (per-channel gate) fp32,
-        NULL iff gate NONE.
+        fp32, g [B,1,H] (scalar gate) or [B,1,H,dk] (per-channel or phase
+        gate) fp32, NULL iff gate NONE.  With the phase gate, P is the
+        rotation-decay of each key pair instead of S Diag(alpha).
    In/out: S [B,H,dv,dk] fp32, the state before the token on entry and after
         it on return (the caller owns it; it is updated in place).
    Out: o [B,1,H,dv] in the storage dtype.

@@ -157,3 +157,20 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         binding.load()
+
+
+def test_phase_gate_routing(lib):
+    # The SFDA phase gate: forward on the bf16 d = 128 tensor-core path only,
+    # no backward; an unknown gate value is an argument error.  Host-side
+    # checks only (fake pointers, nothing launched).
+    assert _fwd(lib, _prob(gate="phase")) == binding.DR_ERR_UNSUPPORTED          # dk = 64
+    assert _fwd(lib, _prob(gate="phase", dk=128, dv=128, dtype="f32")) == \
+        binding.DR_ERR_UNSUPPORTED
+    assert _bwd(lib, _prob(gate="phase", dk=128, dv=128)) == binding.DR_ERR_UNSUPPORTED
+    assert _fwd(lib, _prob(gate="phase", dk=128, dv=128), g=None) == binding.DR_ERR_INVALID_ARG
+    bad = _prob()
+    bad.gate = 4
+    assert _fwd(lib, bad) == binding.DR_ERR_INVALID_ARG
+    n = ctypes.c_size_t(0)
+    assert lib.dr_workspace_size(ctypes.byref(_prob(gate="phase", dk=128, dv=128)), 0,
+                                 ctypes.byref(n)) == binding.DR_OK and n.value > 0
