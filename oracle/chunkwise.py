@@ -258,3 +258,112 @@ def chunk_fwd_phase(q, k, v, beta, g, S0=None, C=64, beta_mode=0, eps=1e-6,
     if return_states:
         return o, ST, states
     return o, ST
+
+
+def _pairs(x):
+    """Real [..., d_k] -> complex [..., d_k / 2]: channel pair (2j, 2j+1) -> x + i y."""
+    return x[..., 0::2] + 1j * x[..., 1::2]
+
+
+def _unpairs(z):
+    out = np.empty(z.shape[:-1] + (2 * z.shape[-1],))
+    out[..., 0::2], out[..., 1::2] = z.real, z.imag
+    return out
+
+
+def chunk_bwd_phase(q, k, v, beta, g, S0, dO, dST=None, C=64, beta_mode=0, eps=1e-6):
+    """Chunkwise backward with the phase gate, through the triangular residual
+    system as in ``chunk_bwd``.  Returns ``dq, dk, dv, dbeta, dg, dS0`` with
+    ``dg[..., 2j]`` = d/d log alpha_j and ``dg[..., 2j+1]`` = d/d theta_j.
+
+    On a pair read as a complex number the chunk's cumulative decay is
+    zeta_i = e^{gamma_i - i Theta_i} (gamma, Theta: in-chunk cumulative sums of
+    log alpha and theta), and Kh = zeta k, Kb = k / conj(zeta), Qh = zeta q,
+    Kt = conj(zeta_C) / conj(zeta) k, S Gamma_C = conj(zeta_C) S per row.  For
+    w = c z the gradient (d/dRe + i d/dIm) maps back by conj(c), and for a real
+    parameter p of w, dL/dp = Re(conj(dL/dw) dw/dp); so each transformed tile
+    gives gamma gradients Re(conj(dX) X) (with the sign of its exponent) and
+    Theta gradients Im(conj(dX) X).
+    """
+    q, k, v, beta, g, S0, dO, dST = map(_f64, (q, k, v, beta, g, S0, dO, dST))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    nc = (T + C - 1) // C
+    _, _, states = chunk_fwd_phase(q, k, v, beta, g, S0, C, beta_mode, eps,
+                                   return_states=True)
+    dq, dkk, dvv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    db = np.zeros((B, T, H))
+    dg = np.zeros_like(g)
+    dS0 = np.zeros((B, H, dv, dk))
+    for b in range(B):
+        for h in range(H):
+            qh_, kh_, vh, _, bt, norm, gh = _head_inputs(q, k, v, beta, g, b, h, beta_mode, eps)
+            dS = np.zeros((dv, dk)) if dST is None else dST[b, h].copy()
+            for n in reversed(range(nc)):
+                t0, t1 = n * C, min(T, n * C + C)
+                m = t1 - t0
+                qc, kc, vc = (_pad_chunk(x, t0, t1, C) for x in (qh_, kh_, vh))
+                bc = _pad_chunk(bt, t0, t1, C)
+                gc = _pad_chunk(gh, t0, t1, C)
+                dOc = _pad_chunk(dO[b, :, h], t0, t1, C)
+                # per-pair cumulative decay zeta_i and the transformed tiles
+                gam = np.cumsum(gc[:, 0::2], axis=0)
+                Th = np.cumsum(gc[:, 1::2], axis=0)
+                zeta = np.exp(gam - 1j * Th)                     # [C, dk/2]
+                kz, qz = _pairs(kc), _pairs(qc)
+                Khz, Kbz, Qhz = zeta * kz, kz / np.conj(zeta), zeta * qz
+                Ktz = (np.conj(zeta[-1])[None, :] / np.conj(zeta)) * kz
+                Kh, Kb, Qh, Kt = (_unpairs(z) for z in (Khz, Kbz, Qhz, Ktz))
+                A = bc[:, None] * np.tril(Kh @ Kb.T, -1)
+                IA = np.eye(C) + A
+                X = np.linalg.solve(IA, bc[:, None] * np.concatenate([vc, Kh], axis=1))
+                Up, W = X[:, :dv], X[:, dv:]
+                Mm = np.tril(Qh @ Kb.T)
+                S = states[b, h, n]
+                U = Up - W @ S.T
+                SG = _unpairs(np.conj(zeta[-1])[None, :] * _pairs(S))   # S Gamma_C
+                # outputs and state transfer of this chunk
+                dU = Mm.T @ dOc + Kt @ dS.T
+                dMm = np.tril(dOc @ U.T)
+                dQh = dOc @ S + dMm @ Kb
+                dKb = dMm.T @ Qh
+                dKt = U @ dS
+                dW = -dU @ S
+                dS_prev = _unpairs(zeta[-1][None, :] * _pairs(dS)) + dOc.T @ Qh - dU.T @ W
+                # triangular residual system (I + A) X = R
+                Lam = np.linalg.solve(IA.T, np.concatenate([dU, dW], axis=1))
+                dA = -np.tril(Lam @ X.T, -1)
+                LamU, LamW = Lam[:, :dv], Lam[:, dv:]
+                dvc = bc[:, None] * LamU
+                dKh = bc[:, None] * LamW
+                dbc = np.sum(LamU * vc, axis=1) + np.sum(LamW * Kh, axis=1)
+                dbc += np.sum(dA * np.tril(Kh @ Kb.T, -1), axis=1)
+                dKh += bc[:, None] * (dA @ Kb)
+                dKb += dA.T @ (bc[:, None] * Kh)
+                # the per-pair complex factors
+                dKhz, dKbz, dQhz, dKtz = (_pairs(x) for x in (dKh, dKb, dQh, dKt))
+                dqc = _unpairs(np.conj(zeta) * dQhz)
+                dkc = _unpairs(np.conj(zeta) * dKhz + dKbz / zeta
+                               + (zeta[-1][None, :] / zeta) * dKtz)
+                pKh, pKb = np.conj(dKhz) * Khz, np.conj(dKbz) * Kbz
+                pQh, pKt = np.conj(dQhz) * Qhz, np.conj(dKtz) * Ktz
+                dgam = (pKh + pQh - pKb - pKt).real
+                dTh = (pKh + pQh + pKb + pKt).imag
+                pS = np.sum(np.conj(_pairs(dS)) * _pairs(SG), axis=0)    # decay of S
+                dgam[-1] += np.sum(pKt, axis=0).real + pS.real
+                dTh[-1] += -np.sum(pKt, axis=0).imag - pS.imag
+                dgc = np.zeros((C, dk))
+                dgc[:, 0::2] = np.cumsum(dgam[::-1], axis=0)[::-1]
+                dgc[:, 1::2] = np.cumsum(dTh[::-1], axis=0)[::-1]
+                if beta_mode == BETA_KACZMARZ:
+                    den = _pad_chunk(norm, t0, t1, C) + eps
+                    dkc += (-2.0 * bc * dbc / den)[:, None] * kc
+                    dbc = dbc / den
+                dq[b, t0:t1, h] = dqc[:m]
+                dkk[b, t0:t1, h] = dkc[:m]
+                dvv[b, t0:t1, h] = dvc[:m]
+                db[b, t0:t1, h] = dbc[:m]
+                dg[b, t0:t1, h] = dgc[:m]
+                dS = dS_prev
+            dS0[b, h] = dS
+    return dict(dq=dq, dk=dkk, dv=dvv, dbeta=db, dg=dg, dS0=dS0)

@@ -175,3 +175,20 @@ def test_phase_chunkwise_equals_recurrent(mode, C, T):
     o_c, S_c = cw.chunk_fwd_phase(x["q"], x["k"], x["v"], x["beta"], x["g"], x["S0"], C=C,
                                   beta_mode=mode)
     assert _rel(o_c, o_r) < 1e-10 and _rel(S_c, S_r) < 1e-10
+
+
+@pytest.mark.parametrize("mode", [oracle.BETA_DIRECT, oracle.BETA_KACZMARZ])
+@pytest.mark.parametrize("C,T", [(1, 5), (4, 13), (16, 37), (64, 70)])
+def test_phase_chunkwise_backward_equals_recurrent(mode, C, T):
+    # the residual-system backward of the chunk form with rotation-decay
+    # factors reaches the token-by-token gradients, d/d log alpha and d/d theta
+    # included (the same exactness claim, for the gradients)
+    from oracle import chunkwise as cw
+    x = _phase_inputs(40 + C + T, T=T, dk=6, dv=4)
+    if mode == oracle.BETA_KACZMARZ:
+        x["k"] = x["k"] * 1.3
+    args = (x["q"], x["k"], x["v"], x["beta"], x["g"], x["S0"], x["dO"], x["dST"])
+    g_r = oracle.recurrent_bwd(*args, beta_mode=mode, gate=oracle.GATE_PHASE)
+    g_c = cw.chunk_bwd_phase(*args, C=C, beta_mode=mode)
+    for name in ("dq", "dk", "dv", "dbeta", "dg", "dS0"):
+        assert _rel(g_c[name], g_r[name]) < 1e-9, name
