@@ -43,3 +43,16 @@ def test_one_token_hand_gradients():
     gr = oracle.recurrent_bwd(q, k, v, beta, g, S0, arr(d["dO"]))
     for name in ("dq", "dk", "dv", "dbeta", "dg", "dS0"):
         assert abs(gr[name].item() - d[name]) < 1e-12, name
+
+
+def test_sfda_two_token_rotation_example():
+    d = _load("sfda_two_token_rotation.json")
+    q = np.array(d["q"])[None, :, None, :]
+    k = np.array(d["k"])[None, :, None, :]
+    v = np.array(d["v"])[None, :, None, :]
+    beta = np.array(d["beta"])[None, :, None]
+    g = np.array(d["g"])[None, :, None, :]
+    S0 = np.array(d["S0"], dtype=float)[None, None]
+    o, ST = oracle.recurrent_fwd(q, k, v, beta, g, S0, gate=oracle.GATE_PHASE)
+    np.testing.assert_allclose(o[0, :, 0], np.array(d["o"]), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(ST[0, 0], np.array(d["ST"]), rtol=0, atol=1e-12)
