@@ -561,12 +561,20 @@ def main():
     else:
         roof = {"bound": "tensor" if tensor else "alu", "achieved": tflops, "peak": fpeak,
                 "unit": "TFLOP/s", "frac": flop_frac, "peak_source": fsrc}
+    traffic = ncu_traffic(top["name"], w.name)
+    design = top["design_bytes_per_launch"]
     roof.update({"kernel": top["name"], "launches": top["launches"],
                  "us_per_launch": per_launch_s * 1e6,
                  "share_of_step": top["ms_total"] / max(sum(step_ms), 1e-9),
                  "algorithmic_bytes_per_launch": top["bytes_per_launch"],
                  "algorithmic_flops_per_launch": top["flops_per_launch"],
-                 "traffic": ncu_traffic(top["name"], w.name)})
+                 "traffic": traffic,
+                 "traffic_over_algorithmic": (None if traffic is None
+                                              else traffic / top["bytes_per_launch"]),
+                 # everything the kernel moves by this design (saved chunk tiles and
+                 # states included), over the same time
+                 "design_bytes_per_launch": design,
+                 "design_frac": design / per_launch_s / 1e9 / peaks["hbm_gbs"]})
 
     flops, nbytes = algorithmic_step(w, fwd_only)
     t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
@@ -602,7 +610,11 @@ def main():
         "e2e": e2e,
         "gpu_launches": sum(k["launches"] for k in kernels),
         "kernels": {k["name"]: {"launches": k["launches"],
-                                "us_per_launch": k["ms_total"] / k["launches"] * 1e3}
+                                "us_per_launch": k["ms_total"] / k["launches"] * 1e3,
+                                "io_gbs": k["bytes_per_launch"] / (k["ms_total"] / k["launches"])
+                                / 1e6,
+                                "design_gbs": k["design_bytes_per_launch"]
+                                / (k["ms_total"] / k["launches"]) / 1e6}
                     for k in kernels},
         "clocks": clocks,
     }

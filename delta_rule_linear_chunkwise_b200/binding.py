@@ -32,7 +32,8 @@ class DrProblem(ctypes.Structure):
 class KernelTime(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int),
                 ("ms_total", ctypes.c_double), ("bytes_per_launch", ctypes.c_double),
-                ("flops_per_launch", ctypes.c_double)]
+                ("flops_per_launch", ctypes.c_double),
+                ("design_bytes_per_launch", ctypes.c_double)]
 
 
 class DrError(RuntimeError):
@@ -69,6 +70,8 @@ def load() -> ctypes.CDLL:
     lib.dr_status_string.restype = ctypes.c_char_p
     lib.dr_last_device_error.argtypes = [vp]
     lib.dr_last_device_error.restype = i
+    lib.dr_inject_timeout.argtypes = [i]
+    lib.dr_inject_timeout.restype = i
     lib.dr_version.argtypes = []
     lib.dr_version.restype = i
     lib.dr_profile_enable.argtypes = [i]
@@ -298,17 +301,26 @@ def decode_step(q, k, v, beta, g, S, *, beta_mode="direct", eps=1e-6, o=None, st
     return o
 
 
+def inject_timeout(launches: int = 1) -> None:
+    """Make the next ``launches`` chunk-backward launches take their bounded-wait
+    timeout path (fault injection for tests; see ``dr_inject_timeout``)."""
+    _check(load().dr_inject_timeout(launches), "dr_inject_timeout")
+
+
 def profile_enable(on: bool = True) -> None:
     """Bracket every library launch with CUDA events on its stream (or stop)."""
     _check(load().dr_profile_enable(1 if on else 0), "dr_profile_enable")
 
 
 def profile_read() -> list[dict]:
-    """Per-kernel launches, summed event time and work model since the last read."""
+    """Per-kernel launches, summed event time and work model since the last read:
+    ``bytes_per_launch`` is the operator's own inputs and outputs the launch
+    touches (algorithmic), ``design_bytes_per_launch`` all it moves by design."""
     buf = (KernelTime * 64)()
     n = load().dr_profile_read(buf, 64)
     if n < 0:
         raise DrError(DR_ERR_CUDA, "dr_profile_read")
     return [dict(name=buf[i].name.decode(), launches=buf[i].launches,
                  ms_total=buf[i].ms_total, bytes_per_launch=buf[i].bytes_per_launch,
-                 flops_per_launch=buf[i].flops_per_launch) for i in range(n)]
+                 flops_per_launch=buf[i].flops_per_launch,
+                 design_bytes_per_launch=buf[i].design_bytes_per_launch) for i in range(n)]

@@ -145,7 +145,7 @@ cudaError_t launch_decode_step(const Problem& p, int bf16, const void* q, const 
                                  : p.gate == kGateScalar                        ? 4
                                                                                 : 0));
   const double flops = heads * p.dv * p.dk * 7.0;
-  prof_begin(kKDecode, bytes, flops, st);
+  prof_begin(kKDecode, bytes, bytes, flops, st);  // all of it is operator I/O
   using bf = __nv_bfloat16;
   if (p.gate == kGatePhase) {
     if (bf16)

@@ -1,12 +1,26 @@
 // dr_api.cu -- the C ABI declared in include/dr.h: argument validation,
 // workspace carving and kernel dispatch.  No device memory is allocated here.
 
-#include <stdlib.h>
-#include <string.h>
+#include <atomic>
 
 #include "../../include/dr.h"
 #include "dr_common.cuh"
 #include "fast.cuh"
+
+namespace dr {
+
+namespace {
+std::atomic<int> g_injected_timeouts{0};
+}  // namespace
+
+bool take_injected_timeout() {
+  int n = g_injected_timeouts.load();
+  while (n > 0)
+    if (g_injected_timeouts.compare_exchange_weak(n, n - 1)) return true;
+  return false;
+}
+
+}  // namespace dr
 
 namespace {
 
@@ -118,40 +132,8 @@ Ws carve(const Layout& L, void* base, int pass) {
   return w;
 }
 
-// The chunk-parallel backward has three implementations with identical
-// results: tcgen05 products with a 16-warp register epilogue (default),
-// warp-level mma.sync products with the same epilogue (DR_BWD_CHUNK=mma), and
-// tcgen05 with a 256-thread TMEM epilogue (DR_TCGEN05_BWD=1).
-int chunk_bwd_kind() {
-  const char* e = getenv("DR_TCGEN05_BWD");
-  if (e && e[0] == '1') return 1;
-  const char* h = getenv("DR_BWD_CHUNK");
-  return (h && strcmp(h, "mma") == 0) ? 0 : 2;
-}
-
-// The two state scans likewise: tcgen05 with the state in registers and the
-// products in TMEM (default), or warp-level mma.sync tiles (DR_MMA_SYNC_SCAN=1;
-// not for the phase gate, whose pair-mixing decay only the tcgen05 scan has).
-bool use_mma_sync_scans(const Problem& P) {
-  const char* e = getenv("DR_MMA_SYNC_SCAN");
-  return e && e[0] == '1' && P.gate != dr::kGatePhase;
-}
-cudaError_t fwd_scan(const dr::Problem& P, const dr::fast::Saved& sv, const float* S0,
-                     __nv_bfloat16* o, float* ST, bool save, cudaStream_t st) {
-  if (use_mma_sync_scans(P)) return dr::fast::launch_fwd_scan(P, sv, S0, o, ST, save, st);
-  return dr::fast::launch_fwd_scan_tc(P, sv, S0, o, ST, save, st);
-}
-cudaError_t bwd_scan(const dr::Problem& P, const dr::fast::Saved& sv, const __nv_bfloat16* dO,
-                     const float* dST, float* dS0, __nv_bfloat16* dU, __nv_bfloat16* dh,
-                     cudaStream_t st) {
-  if (use_mma_sync_scans(P)) return dr::fast::launch_bwd_scan(P, sv, dO, dST, dS0, dU, dh, st);
-  return dr::fast::launch_bwd_scan_tc(P, sv, dO, dST, dS0, dU, dh, st);
-}
-
 // Segments of the chunk-parallel affine scan for this problem (1 = sequential).
-int scan_segments(const Problem& P) {
-  return use_mma_sync_scans(P) ? 1 : dr::fast::affine_segments(P);
-}
+int scan_segments(const Problem& P) { return dr::fast::affine_segments(P); }
 
 // The forward state scan, plain or segmented.  Segmented: the transfer
 // matrices (into the saved tiles) and offsets of all segments in one
@@ -160,7 +142,7 @@ int scan_segments(const Problem& P) {
 cudaError_t fwd_scan_any(const Problem& P, const dr::fast::Saved& sv, const float* S0,
                          __nv_bfloat16* o, float* ST, bool save, char* aff, cudaStream_t st) {
   const int G = scan_segments(P);
-  if (G == 1) return fwd_scan(P, sv, S0, o, ST, save, st);
+  if (G == 1) return dr::fast::launch_fwd_scan_tc(P, sv, S0, o, ST, save, st);
   const int L = dr::fast::affine_seg_len(P, G);
   float* Bm = (float*)aff;
   float* Sst = (float*)(aff + round_up(dr::fast::affine_map_bytes(P, G)));
@@ -181,7 +163,7 @@ cudaError_t bwd_scan_any(const Problem& P, const dr::fast::Saved& sv, const __nv
                          const float* dST, float* dS0, __nv_bfloat16* dU, __nv_bfloat16* dh,
                          char* aff, cudaStream_t st) {
   const int G = scan_segments(P);
-  if (G == 1) return bwd_scan(P, sv, dO, dST, dS0, dU, dh, st);
+  if (G == 1) return dr::fast::launch_bwd_scan_tc(P, sv, dO, dST, dS0, dU, dh, st);
   const int L = dr::fast::affine_seg_len(P, G);
   float* Cm = (float*)aff;
   float* dSe = (float*)(aff + round_up(dr::fast::affine_map_bytes(P, G)));
@@ -322,11 +304,7 @@ dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const 
     }
     e = bwd_scan_any(P, sv, (const bf*)dO, dST, dS0, dU, dh, aff, st);
     if (e == cudaSuccess) {
-      const int kind = chunk_bwd_kind();
-      auto launch = kind == 2 ? dr::fast::launch_bwd_chunk_hy
-                              : kind == 1 ? dr::fast::launch_bwd_chunk_tc
-                                          : dr::fast::launch_bwd_chunk;
-      e = launch(P, (const bf*)q, (const bf*)k, (const bf*)v, (const bf*)dO, g, sv, dh, dU,
+      e = dr::fast::launch_bwd_chunk_hy(P, (const bf*)q, (const bf*)k, (const bf*)v, (const bf*)dO, g, sv, dh, dU,
                  (bf*)dq, (bf*)dk, (bf*)dv, dbeta, dg, st);
     }
     return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
@@ -363,6 +341,12 @@ dr_status dr_last_device_error(void* stream) {
   return flag ? DR_ERR_TIMEOUT : DR_OK;
 }
 
-int dr_version(void) { return 100; }
+dr_status dr_inject_timeout(int launches) {
+  if (launches < 0) return DR_ERR_INVALID_ARG;
+  dr::g_injected_timeouts.store(launches);
+  return DR_OK;
+}
+
+int dr_version(void) { return 200; }
 
 }  // extern "C"

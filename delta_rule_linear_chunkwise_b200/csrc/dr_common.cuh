@@ -70,8 +70,12 @@ enum {
 };
 const char* kernel_name(int id);
 // Bracket one launch with events on its stream when profiling is enabled.
-// bytes / flops: the launch's algorithmic HBM traffic and arithmetic.
-void prof_begin(int kernel, double bytes, double flops, cudaStream_t st);
+// io_bytes: the operator's own inputs and outputs that the launch reads or
+// writes (q, k, v, g, beta, dO, o, the gradients, the states), each once: the
+// algorithmic bytes.  bytes: everything the launch moves by this library's
+// design, including the chunk tiles and states kept between kernels.
+// flops: its arithmetic.
+void prof_begin(int kernel, double io_bytes, double bytes, double flops, cudaStream_t st);
 void prof_end(cudaStream_t st);
 
 // Reads the device-side error word (bounded waits that gave up record a
@@ -79,6 +83,9 @@ void prof_end(cudaStream_t st);
 cudaError_t read_and_clear_device_error(int* flag);
 // Device address of that error word on the current device (nullptr on failure).
 int* device_error_word();
+// Fault injection (dr_inject_timeout): true, and one fewer pending, if the
+// next chunk-backward launch is to take its bounded-wait timeout path.
+bool take_injected_timeout();
 
 // Launchers of the generic (fp32 SIMT) kernels; TIn is float or __nv_bfloat16.
 template <typename TIn>

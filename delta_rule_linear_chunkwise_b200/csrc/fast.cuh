@@ -158,11 +158,6 @@ inline Saved carve_saved(const Problem& p, void* base) {
 cudaError_t launch_prep(const Problem& p, const __nv_bfloat16* q, const __nv_bfloat16* k,
                         const __nv_bfloat16* v, const float* beta, const float* g,
                         const Saved& sv, cudaStream_t st);
-// tc_fwd_scan: state chain, output and (when sv.h / sv.U are non-null) the
-// chunk start states and pseudo-values.
-cudaError_t launch_fwd_scan(const Problem& p, const Saved& sv, const float* S0,
-                            __nv_bfloat16* o, float* ST, bool save, cudaStream_t st);
-// The same on tcgen05: MMAs into tensor memory, fp32 state in registers.
 cudaError_t launch_fwd_scan_tc(const Problem& p, const Saved& sv, const float* S0,
                                __nv_bfloat16* o, float* ST, bool save, cudaStream_t st);
 // Segmented forms (see ScanSeg); bv = 64 or 128 value rows per CTA.
@@ -182,23 +177,7 @@ cudaError_t launch_affine_compose_bwd(const Problem& p, int G, const float* dST,
 cudaError_t launch_bwd_scan_tc(const Problem& p, const Saved& sv, const __nv_bfloat16* dO,
                                const float* dST, float* dS0, __nv_bfloat16* dU,
                                __nv_bfloat16* dh, cudaStream_t st);
-cudaError_t launch_bwd_scan(const Problem& p, const Saved& sv, const __nv_bfloat16* dO,
-                            const float* dST, float* dS0, __nv_bfloat16* dU,
-                            __nv_bfloat16* dh, cudaStream_t st);
-cudaError_t launch_bwd_chunk(const Problem& p, const __nv_bfloat16* q, const __nv_bfloat16* k,
-                             const __nv_bfloat16* v, const __nv_bfloat16* dO, const float* g,
-                             const Saved& sv, const __nv_bfloat16* dh,
-                             const __nv_bfloat16* dU, __nv_bfloat16* dq, __nv_bfloat16* dk,
-                             __nv_bfloat16* dv, float* dbeta, float* dg, cudaStream_t st);
-
-cudaError_t launch_bwd_chunk_tc(const Problem& p, const __nv_bfloat16* q,
-                                const __nv_bfloat16* k, const __nv_bfloat16* v,
-                                const __nv_bfloat16* dO, const float* g, const Saved& sv,
-                                const __nv_bfloat16* dh, const __nv_bfloat16* dU,
-                                __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv,
-                                float* dbeta, float* dg, cudaStream_t st);
-
-// The same with the products on tcgen05 and the element-wise work on 16 warps.
+// The chunk-parallel backward: products on tcgen05, element-wise work on 16 warps.
 cudaError_t launch_bwd_chunk_hy(const Problem& p, const __nv_bfloat16* q,
                                 const __nv_bfloat16* k, const __nv_bfloat16* v,
                                 const __nv_bfloat16* dO, const float* g, const Saved& sv,

@@ -120,7 +120,8 @@ cudaError_t launch_affine_compose_fwd(const Problem& p, int G, const float* S0, 
   const double heads = (double)p.B * p.H;
   // reads S0, every P_g (once per 16-row block, mostly from L2) and B_g; writes Sst, ST
   const double bytes = heads * D * D * 4.0 * (1 + 2.0 * G + G + 1);
-  prof_begin(kKAffine, bytes, heads * G * 2.0 * D * D * D, st);
+  const double io = heads * D * D * 4.0 * ((S0 ? 1 : 0) + (ST ? 1 : 0));
+  prof_begin(kKAffine, io, bytes, heads * G * 2.0 * D * D * D, st);
   k_affine_fwd<<<dim3(D / RB, p.H, p.B), NTA, 0, st>>>(p, G, S0, P, Bm, Sst, ST);
   const cudaError_t e = cudaGetLastError();
   prof_end(st);
@@ -135,7 +136,8 @@ cudaError_t launch_affine_compose_bwd(const Problem& p, int G, const float* dST,
   if (e != cudaSuccess) return e;
   const double heads = (double)p.B * p.H;
   const double bytes = heads * D * D * 4.0 * (1 + 2.0 * G + G + 1);
-  prof_begin(kKAffine, bytes, heads * G * 2.0 * D * D * D, st);
+  const double io = heads * D * D * 4.0 * ((dST ? 1 : 0) + (dS0 ? 1 : 0));
+  prof_begin(kKAffine, io, bytes, heads * G * 2.0 * D * D * D, st);
   k_affine_bwd<<<dim3(D / RB, p.H, p.B), NTA, sm, st>>>(p, G, dST, P, Cm, dSe, dS0);
   e = cudaGetLastError();
   prof_end(st);

@@ -1,7 +1,8 @@
 // fast_bwd_hy.cu -- chunk-parallel backward with the products on tcgen05 and
 // the element-wise work on all 16 warps (bf16 storage, d_k = d_v = 128, C = 64).
 //
-// Same algebra as tc_bwd_chunk (fast_bwd.cu): with ep = e^{gamma - gamma_r},
+// One CTA per (b, h, chunk).  With ep = e^{gamma - gamma_r} (gamma_r: the cumulative
+// gate at the chunk's centre row) and the chunk's saved tiles:
 //   level 1  dQs = dO S, dW' = dU S, dKt = U dS', dM = tril(dO U^T)
 //   level 2  Lambda = T^T [dU | dW]             (dv = diag(beta) Lambda_U)
 //   level 3  dA = -strict_tril(Lambda_U U'^T + Lambda_W W^T)
@@ -18,8 +19,7 @@
 // 32-lane quadrant q, and tcgen05.ld.16x256b returns it to the warps of that
 // quadrant in exactly the register fragment of a warp-level m16n8 product
 // (thread t: row t / 4 and t / 4 + 8, columns 2 (t % 4), + 1 of each 8-column
-// group), so warp w = 4 qt + rb owns rows 16 rb .., columns 32 qt .. as in the
-// warp-level kernel.
+// group), so warp w = 4 qt + rb owns rows 16 rb .., columns 32 qt ...
 
 #include "dr_common.cuh"
 #include "fast.cuh"
@@ -38,6 +38,9 @@ constexpr int LDD = D + 8;
 constexpr int NTB = 512;
 constexpr int LDG = D + 4;  // fp32 row stride of the dgamma tile (fragment stores conflict-free)
 constexpr uint32_t kSpinHy = 1u << 22;
+// Polls of the injected wait (dr_inject_timeout): short, so the test that
+// drives the timeout path ends within milliseconds.
+constexpr uint32_t kSpinInjected = 256;
 
 __device__ __forceinline__ int centre_row(int nvalid) { return (nvalid - 1) / 2; }
 // Gate tile element (i, c): 8-column groups XOR-swizzled by row.
@@ -70,6 +73,7 @@ struct HySmem {
   float er[D];
   float erc[D];
   uint64_t bar;
+  uint64_t never;   // fault injection: a barrier that nothing ever arrives on
   uint32_t tmem;
 };
 
@@ -158,8 +162,9 @@ __device__ __forceinline__ void frag_ld2(uint32_t col, int warp, float (&f)[2][4
 }
 
 // Bounded wait for the commit of level `phase`; CTA-uniform result.
-__device__ __forceinline__ bool hy_wait(uint64_t* bar, int phase) {
-  const bool ok = tc::mbar_wait(bar, (uint32_t)(phase & 1), kSpinHy);
+__device__ __forceinline__ bool hy_wait(uint64_t* bar, int phase,
+                                        uint32_t limit = kSpinHy) {
+  const bool ok = tc::mbar_wait(bar, (uint32_t)(phase & 1), limit);
   const int bad = __syncthreads_or(ok ? 0 : 1);
   tc::fence_after_sync();
   return bad == 0;
@@ -175,7 +180,7 @@ __global__ void __launch_bounds__(NTB, 1)
                 const bf16* __restrict__ Upg, const float* __restrict__ knorm_g,
                 bf16* __restrict__ dq, bf16* __restrict__ dk,
                 bf16* __restrict__ dv, float* __restrict__ dbeta, float* __restrict__ dg,
-                int* __restrict__ err) {
+                int* __restrict__ err, int inject_timeout) {
   extern __shared__ __align__(1024) unsigned char smraw[];
   HySmem& s = *reinterpret_cast<HySmem*>(smraw);
   const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
@@ -225,7 +230,10 @@ __global__ void __launch_bounds__(NTB, 1)
   cp_linear<NTB>(s.TT, Tg + cb * C * C, C * C, tid);
   frag::cp_commit();
   if (warp == 0) tc::tmem_alloc(&s.tmem, 512);
-  if (tid == 0) tc::mbar_init(&s.bar, 1);
+  if (tid == 0) {
+    tc::mbar_init(&s.bar, 1);
+    tc::mbar_init(&s.never, 1);
+  }
   frag::cp_wait<1>();
   __syncthreads();
   // element (i, c) of the gate tile
@@ -329,6 +337,14 @@ __global__ void __launch_bounds__(NTB, 1)
   const uint32_t tb = s.tmem;
   bool ok = true;
   do {  // leaves early (break) only when a bounded wait gives up
+
+  // Fault injection (dr_inject_timeout): wait, with a short limit, on a barrier
+  // that nothing arrives on.  Every copy has landed and no MMA has been issued,
+  // so the timeout path below leaves nothing in flight.
+  if (inject_timeout) {
+    ok = hy_wait(&s.never, 0, kSpinInjected);
+    if (!ok) break;
+  }
 
   // ---- level 1 (tensor memory): dQs = dO S, dW' = dU S, dKt = U dS', dM = dO U^T
   if (tid == 0) {
@@ -722,15 +738,16 @@ cudaError_t launch_bwd_chunk_hy(const Problem& p, const bf16* q, const bf16* k, 
       cudaFuncSetAttribute(k_bwd_chunk_hy, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const double nb = (double)p.B * p.H * p.NC, ntok = nb * C;
-  // reads q, k, v, dO, g, beta, T, h, dh, U, dU, W, U'; writes dq, dk, dv, dbeta, dg
-  const double bytes = ntok * (4 * D * 2 + p.gk * 4 + 4) + nb * C * C * 2 + nb * 2.0 * D * D * 2 +
-                       ntok * 4 * D * 2 + ntok * (3 * D * 2 + p.gk * 4 + 4);
+  // operator I/O: reads q, k, v, dO, g, beta; writes dq, dk, dv, dbeta, dg
+  const double io = ntok * (4 * D * 2 + p.gk * 4 + 4) + ntok * (3 * D * 2 + p.gk * 4 + 4);
+  // and by design the chunk tiles T, h, dh, U, dU, W, U' (and beta, ||k||^2 from the saved set)
+  const double bytes = io + nb * C * C * 2 + nb * 2.0 * D * D * 2 + ntok * 4 * D * 2 + ntok * 4;
   const double mac = (double)C * D * D * 3 + (double)C * C * D + (double)C * D * C * 2 +
                      (double)C * C * D * 2 + (double)C * D * C * 4;
-  prof_begin(kKTcChunkBwd, bytes, nb * 2.0 * mac, st);
+  prof_begin(kKTcChunkBwd, io, bytes, nb * 2.0 * mac, st);
   k_bwd_chunk_hy<<<dim3(p.NC, p.H, p.B), NTB, sm, st>>>(
       p, q, k, v, dO, g, sv.T, sv.beta, sv.h, dh, sv.U, dU, sv.W, sv.Up, sv.knorm, dq, dk, dv,
-      dbeta, dg, device_error_word());
+      dbeta, dg, device_error_word(), take_injected_timeout() ? 1 : 0);
   e = cudaGetLastError();
   prof_end(st);
   return e;

@@ -10,10 +10,6 @@
 //   (16 x 16 diagonal blocks per warp, off-diagonal block products in tf32);
 //   W = T diag(beta) (k e^gamma),  U' = T diag(beta) V  on tensor cores;
 //   Qh = q e^gamma,  Kt = k e^{gamma_C - gamma},  dec = e^{gamma_C}.
-// tc_fwd_scan (sequential over chunks, one CTA per (b, h, 64-wide value tile)):
-// with the fp32 state S in registers and its bf16 copy in shared memory,
-//   U = U' - W S^T,  O = Qh S^T + M U,  S <- S Diag(dec) + U^T Kt,
-// streaming the precomputed chunk tiles through a two-stage cp.async pipeline.
 
 #include "dr_common.cuh"
 #include "fast.cuh"
@@ -31,7 +27,6 @@ constexpr int LDD = D + 8;   // bf16 stride of 128-wide tiles
 constexpr int LDC = C + 8;   // bf16 stride of 64-wide tiles
 constexpr int LDA = C + 1;   // fp32 stride of the 64 x 64 solve tiles
 constexpr int NT = 256;      // threads per CTA (8 warps)
-constexpr int BV = 64;       // value columns per scan CTA
 
 __device__ __forceinline__ int centre_row(int nvalid) { return (nvalid - 1) / 2; }
 
@@ -160,26 +155,20 @@ __global__ void __launch_bounds__(NT, 2)
 
   // Factors: K^c, Kb^c, Q^c to shared memory; Qh, Kt, beta, dec to global.
   const int r = centre_row(nvalid);
-  // per-column factors of this thread's segment: e^{-gamma_r}, e^{gamma_C - gamma_r}
-  // (phase gate: at the even channels; e^{i Theta_r}, e^{i Theta_C} per pair)
-  float ier8[8], ecr8[8];
-  float rc4[4], rs4[4], cc4[4], cs4[4], gr4[4];
-  {
-    float r8[8], c8[8];
-    gate8(G, gk, r, (tid & 15) * 8, r8);
-    gate8(G, gk, C - 1, (tid & 15) * 8, c8);
+  // This thread's segment of the centre row's and the last row's cumulative gate
+  // (phase gate: log-decays at the even channels, e^{i Theta_r}, e^{i Theta_C} per pair).
+  // Every factor below is the exponential of a difference of cumulative gates:
+  // the centred ones stay within half the chunk's decay, and none is formed as a
+  // quotient of two exponentials that may underflow.
+  float r8[8], c8[8];
+  float rc4[4], rs4[4], cc4[4], cs4[4];
+  gate8(G, gk, r, (tid & 15) * 8, r8);
+  gate8(G, gk, C - 1, (tid & 15) * 8, c8);
+  if (PHASE) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      ier8[e] = __expf(-r8[e]);
-      ecr8[e] = __expf(c8[e] - r8[e]);
-    }
-    if (PHASE) {
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        gr4[m] = r8[2 * m];
-        sincosf(r8[2 * m + 1], &rs4[m], &rc4[m]);
-        sincosf(c8[2 * m + 1], &cs4[m], &cc4[m]);
-      }
+    for (int m = 0; m < 4; ++m) {
+      sincosf(r8[2 * m + 1], &rs4[m], &rc4[m]);
+      sincosf(c8[2 * m + 1], &cs4[m], &cc4[m]);
     }
   }
 #pragma unroll
@@ -201,7 +190,7 @@ __global__ void __launch_bounds__(NT, 2)
         const float eg = __expf(g8[e]);                            // e^gamma
         // e^{+-(gamma - gamma_r)} from the centred exponent itself: within half
         // a chunk's decay of 1, so it stays finite where e^gamma underflows
-        const float ep = __expf(g8[e] - gr4[m]), em = __expf(gr4[m] - g8[e]);
+        const float ep = __expf(g8[e] - r8[e]), em = __expf(r8[e] - g8[e]);
         // e^{-i (Theta - Theta_r)} and e^{i (Theta_C - Theta)}
         const float wr = cs * rc4[m] + sn * rs4[m], wi = cs * rs4[m] - sn * rc4[m];
         const float tr = cc4[m] * cs + cs4[m] * sn, ti = cs4[m] * cs - cc4[m] * sn;
@@ -216,7 +205,7 @@ __global__ void __launch_bounds__(NT, 2)
         qc[e + 1] = ep * qwy;
         qh[e] = eg * (cs * qx + sn * qy);                          // Gamma q
         qh[e + 1] = eg * (cs * qy - sn * qx);
-        const float sc = em * ecr8[e];                             // e^{gamma_C - gamma}
+        const float sc = __expf(c8[e] - g8[e]);                    // e^{gamma_C - gamma}
         kt[e] = sc * (tr * kx - ti * ky);                          // Gamma_C^T Gamma^{-T} k
         kt[e + 1] = sc * (ti * kx + tr * ky);
         nn += kx * kx + ky * ky;
@@ -224,13 +213,13 @@ __global__ void __launch_bounds__(NT, 2)
     } else {
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float eg = __expf(g8[e]);                              // e^gamma
-        const float ep = eg * ier8[e], em = __fdividef(1.f, ep);     // e^{+-(gamma - gamma_r)}
+        const float eg = __expf(g8[e]);                                  // e^gamma
+        const float ep = __expf(g8[e] - r8[e]), em = __expf(r8[e] - g8[e]);  // e^{+-(gamma - gamma_r)}
         kc[e] = kv[e] * ep;
         kb[e] = kv[e] * em;
         qc[e] = qv[e] * ep;
         qh[e] = qv[e] * eg;
-        kt[e] = kb[e] * ecr8[e];  // k e^{gamma_C - gamma}
+        kt[e] = kv[e] * __expf(c8[e] - g8[e]);  // k e^{gamma_C - gamma}
         nn += kv[e] * kv[e];
       }
     }
@@ -403,135 +392,6 @@ __global__ void __launch_bounds__(NT, 2)
   }
 }
 
-// ---------------------------------------------------------------------------
-// tc_fwd_scan
-struct FwdStage {  // core-tiled, as saved
-  bf16 W[C * D];
-  bf16 Qh[C * D];
-  bf16 Kt[C * D];
-  bf16 M[C * C];
-  bf16 Up[C * BV];    // U'[:, a0 .. a0+63]
-  float dec[D];
-};
-struct FwdSmem {
-  FwdStage st[2];
-  bf16 S[BV * LDD];   // bf16 copy of the state rows a0.. [a][c]
-  bf16 U[C * LDC];    // pseudo-values [i][a]
-};
-
-__device__ void fwd_issue(const Problem& p, FwdStage& s, const Saved& sv, int b, int h, int n,
-                          int a0) {
-  const int tid = threadIdx.x;
-  const size_t cb = chunk_id(p, b, h, n);
-  cp_linear<NT>(s.W, sv.W + cb * C * D, C * D, tid);
-  cp_linear<NT>(s.Qh, sv.Qh + cb * C * D, C * D, tid);
-  cp_linear<NT>(s.Kt, sv.Kt + cb * C * D, C * D, tid);
-  cp_linear<NT>(s.M, sv.M + cb * C * C, C * C, tid);
-  cp_ct_cols<NT>(s.Up, sv.Up + cb * C * D, C, a0, BV, tid);
-  if (tid < D / 4) frag::cp16(s.dec + tid * 4, sv.dec + cb * D + tid * 4, true);
-}
-
-__global__ void __launch_bounds__(NT, 1)
-    k_fwd_scan(Problem p, Saved sv, const float* __restrict__ S0, bf16* __restrict__ o,
-               float* __restrict__ ST, int save) {
-  extern __shared__ __align__(16) unsigned char smraw[];
-  FwdSmem& s = *reinterpret_cast<FwdSmem*>(smraw);
-  const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int rb = warp & 3, hf = warp >> 2;  // row block (16 rows), column half
-  const int a0 = blockIdx.x * BV;
-  const int lr = lane >> 2, lc = 2 * (lane & 3);
-  const size_t sbase = ((size_t)b * p.H + h) * D * D;
-
-  // fp32 state rows a0 + 16rb + .., key columns 64hf .. 64hf+63
-  float S[8][4];
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int a = rb * 16 + lr + (e >> 1) * 8, c = hf * 64 + j * 8 + lc + (e & 1);
-      S[j][e] = S0 ? S0[sbase + (size_t)(a0 + a) * D + c] : 0.f;
-    }
-  frag::st_c(S, s.S, LDD, rb * 16, hf * 64);
-
-  fwd_issue(p, s.st[0], sv, b, h, 0, a0);
-  frag::cp_commit();
-  if (p.NC > 1) fwd_issue(p, s.st[1], sv, b, h, 1, a0);
-  frag::cp_commit();
-  for (int n = 0; n < p.NC; ++n) {
-    const int t0 = n * C, nvalid = min(C, p.T - t0);
-    const size_t cb = chunk_id(p, b, h, n);
-    FwdStage& st = s.st[n & 1];
-    frag::cp_wait<1>();
-    __syncthreads();
-    if (save)  // rows a0 .. a0 + 63 of the core-tiled state: one contiguous block
-      for (int idx = tid; idx < BV * (D / 8); idx += NT)
-        *reinterpret_cast<uint4*>(sv.h + cb * D * D + ct_off(a0, 0, D) + 8 * idx) =
-            *reinterpret_cast<const uint4*>(s.S + ct_row(idx, D) * LDD + ct_col(idx, D));
-    // U = U' - W S^T and the inter-chunk part of O; rows 16rb.., values 32hf..
-    float oc[4][4], u[4][4];
-    {
-      frag::zero(u);
-      frag::zero(oc);
-      frag::mm_rows2<4, 8, false>(u, oc, st.W, st.Qh, -D, rb * 16, s.S, LDD, hf * 32);
-#pragma unroll
-      for (int jt = 0; jt < 4; ++jt)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const float2 up = frag::unpack(*reinterpret_cast<const uint32_t*>(
-              st.Up + ct_off(rb * 16 + lr + hh * 8, hf * 32 + jt * 8 + lc, BV)));
-          u[jt][2 * hh] = up.x - u[jt][2 * hh];
-          u[jt][2 * hh + 1] = up.y - u[jt][2 * hh + 1];
-        }
-      frag::st_c(u, s.U, LDC, rb * 16, hf * 32);
-    }
-    __syncthreads();
-    if (save)
-      for (int idx = tid; idx < C * (BV / 8); idx += NT) {
-        const int grp = idx / BV, k = idx % BV, i = grp * 8 + (k & 7), j = k >> 3;
-        *reinterpret_cast<uint4*>(sv.U + cb * C * D + ct_off(i, a0 + j * 8, D)) =
-            *reinterpret_cast<const uint4*>(s.U + i * LDC + j * 8);
-      }
-    // O += M U
-    frag::mm_rows<4, 4, true>(oc, st.M, -C, rb * 16, s.U, LDC, hf * 32);
-    if (o) {
-#pragma unroll
-      for (int jt = 0; jt < 4; ++jt)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int i = rb * 16 + lr + hh * 8;
-          if (i < nvalid)
-            *reinterpret_cast<uint32_t*>(o + row_id(p, b, t0 + i, h) * D + a0 + hf * 32 + jt * 8 + lc) =
-                frag::pack(oc[jt][2 * hh], oc[jt][2 * hh + 1]);
-        }
-    }
-    // S <- S Diag(dec) + U^T Kt for state rows 16rb.., key columns 64hf..
-    {
-      float ds[8][4];
-      frag::zero(ds);
-      frag::mm_rows_at<8, 4, true>(ds, s.U, LDC, rb * 16, st.Kt, -D, hf * 64);
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          S[j][e] = S[j][e] * st.dec[hf * 64 + j * 8 + lc + (e & 1)] + ds[j][e];
-    }
-    __syncthreads();  // this stage, the bf16 state and U are consumed
-    if (n + 2 < p.NC) fwd_issue(p, st, sv, b, h, n + 2, a0);
-    frag::cp_commit();
-    frag::st_c(S, s.S, LDD, rb * 16, hf * 64);
-  }
-  if (ST) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int a = rb * 16 + lr + (e >> 1) * 8, c = hf * 64 + j * 8 + lc + (e & 1);
-        ST[sbase + (size_t)(a0 + a) * D + c] = S[j][e];
-      }
-  }
-}
-
 }  // namespace
 
 cudaError_t launch_prep(const Problem& p, const bf16* q, const bf16* k, const bf16* v,
@@ -542,35 +402,16 @@ cudaError_t launch_prep(const Problem& p, const bf16* q, const bf16* k, const bf
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const double nb = (double)p.B * p.H * p.NC, ntok = nb * C;
-  // reads q, k, v, g, beta; writes T, beta, dec, W, U', M, Qh, Kt
-  const double bytes = ntok * (3 * D * 2 + p.gk * 4 + 4) +
-                       nb * ((double)kTBytes + kBetaBytes + kDecBytes + 4.0 * kTileBytes + kMBytes);
+  // reads q, k, v, g, beta (the operator's inputs); writes T, beta, dec, W, U', M, Qh, Kt
+  const double io = ntok * (3 * D * 2 + p.gk * 4 + 4);
+  const double bytes =
+      io + nb * ((double)kTBytes + 2 * kBetaBytes + kDecBytes + 4.0 * kTileBytes + kMBytes);
   const double flops = nb * (2.0 * 2 * C * C * D + 2.0 * 2 * C * C * D);  // [A;M] Gram, W|U'
-  prof_begin(kKTcIntraFwd, bytes, flops, st);
+  prof_begin(kKTcIntraFwd, io, bytes, flops, st);
   if (phase)
     k_prep<true><<<dim3(p.NC, p.H, p.B), NT, sm, st>>>(p, q, k, v, beta, g, sv);
   else
     k_prep<false><<<dim3(p.NC, p.H, p.B), NT, sm, st>>>(p, q, k, v, beta, g, sv);
-  e = cudaGetLastError();
-  prof_end(st);
-  return e;
-}
-
-cudaError_t launch_fwd_scan(const Problem& p, const Saved& sv, const float* S0, bf16* o,
-                            float* ST, bool save, cudaStream_t st) {
-  const size_t sm = sizeof(FwdSmem);
-  cudaError_t e =
-      cudaFuncSetAttribute(k_fwd_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  if (e != cudaSuccess) return e;
-  const double nb = (double)p.B * p.H * p.NC, ntok = nb * C, heads = (double)p.B * p.H;
-  // reads W, Qh, Kt, M, U', dec; writes o (+ chunk states and U when saving)
-  double bytes = nb * (3.0 * kTileBytes + kMBytes + kTileBytes + kDecBytes);
-  if (o) bytes += ntok * D * 2;
-  if (save) bytes += nb * ((double)kStateBytes + kUBytes);
-  bytes += heads * D * D * 4 * ((S0 ? 1 : 0) + (ST ? 1 : 0));
-  const double flops = nb * (D / BV) * (2.0 * C * BV * D * 3 + 2.0 * C * C * BV);
-  prof_begin(kKTcScanFwd, bytes, flops, st);
-  k_fwd_scan<<<dim3(D / BV, p.H, p.B), NT, sm, st>>>(p, sv, S0, o, ST, save ? 1 : 0);
   e = cudaGetLastError();
   prof_end(st);
   return e;

@@ -361,9 +361,12 @@ cudaError_t launch_fwd_scan_tc_bv(const Problem& p, const Saved& sv, const ScanS
   if (o) bytes += nb * ((double)kTileBytes + kMBytes) + ntok * D * 2;
   if (save) bytes += nb * ((double)kStateBytes + kUBytes);
   bytes += heads * sg.G * D * D * 4 * ((S0 ? 1 : 0) + (ST ? maps : 0));
+  // operator I/O: o, and S0 / S_T when they are the operator's own (unsegmented)
+  const double io = (o ? ntok * D * 2 : 0.0) +
+                    (sg.G == 1 ? heads * D * D * 4.0 * ((S0 ? 1 : 0) + (ST ? 1 : 0)) : 0.0);
   const double flops =
       maps * nb * (2.0 * C * D * D * (o ? 3 : 2) + (o ? 2.0 * C * C * D : 0.0));
-  prof_begin(kKTcScanFwd, bytes, flops, st);
+  prof_begin(kKTcScanFwd, io, bytes, flops, st);
   const dim3 grid(maps * (D / BV), p.H, p.B * sg.G);
   if (phase)
     k_fwd_scan_tc<BV, true><<<grid, NTF, sm, st>>>(p, sv, sg, o, save ? 1 : 0, device_error_word());
@@ -641,8 +644,11 @@ cudaError_t launch_bwd_scan_tc_bv(const Problem& p, const Saved& sv, const bf16*
   const double bytes = nb * (3.0 * kTileBytes + kMBytes + kDecBytes) + ntok * D * 2 +
                        (sg.mode == 0 ? nb * ((double)kUBytes + kStateBytes) : 0.0) +
                        heads * sg.G * D * D * 4 * ((dST ? 1 : 0) + (dS0 ? 1 : 0));
+  // operator I/O: dO, and dS_T / dS0 when they are the operator's own (unsegmented)
+  const double io = ntok * D * 2 +
+                    (sg.G == 1 ? heads * D * D * 4.0 * ((dST ? 1 : 0) + (dS0 ? 1 : 0)) : 0.0);
   const double flops = nb * (2.0 * C * C * D + 2.0 * C * D * D * 3);
-  prof_begin(kKTcScanBwd, bytes, flops, st);
+  prof_begin(kKTcScanBwd, io, bytes, flops, st);
   k_bwd_scan_tc<BV><<<dim3(D / BV, p.H, p.B * sg.G), NTF, sm, st>>>(p, sv, dO, sg, dU, dh,
                                                                     device_error_word());
   e = cudaGetLastError();

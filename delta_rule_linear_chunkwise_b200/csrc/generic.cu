@@ -666,41 +666,48 @@ size_t intra_bwd_smem(const Problem& p) {
 
 int pick_bv(const Problem& p) { return (p.dv % 32 == 0) ? 32 : 16; }
 
-// Work models per launch (whole grid): algorithmic HBM bytes = every tensor
-// the kernel must read or write once (inputs, outputs and the workspace
-// tensors it exchanges with the other kernels); FLOPs = 2 x multiply-adds of
-// its products, triangular products counted at their triangle.
+// Work models per launch (whole grid): io_bytes = the operator's inputs and
+// outputs the kernel reads or writes, each once (algorithmic); bytes = every
+// tensor it must read or write once, including the workspace tensors it
+// exchanges with the other kernels; FLOPs = 2 x multiply-adds of its products,
+// triangular products counted at their triangle.
 struct Work {
-  double bytes, flops;
+  double io_bytes, bytes, flops;
 };
 Work work_of(int kernel, const Problem& p, int es, bool states_io) {
   const double nb = (double)p.B * p.H * p.NC, C = kC, dk = p.dk, dv = p.dv, gk = p.gk;
   const double ntok = nb * C;  // padded token-heads
   const double grid_in = ntok * (gk * 4 + 4);          // g, beta
   const double st = nb * dv * dk * 4;                  // one fp32 state per chunk
-  Work w{0, 0};
+  Work w{0, 0, 0};
   switch (kernel) {
     case kKIntraFwd:
+      w.io_bytes = ntok * (2 * dk + dv) * es + grid_in;
       w.bytes = ntok * (2 * dk + dv) * es + grid_in +
                 ntok * (gk * 4 + 8) + nb * C * C * 8 + ntok * (dk + dv) * 4;
       w.flops = nb * (2 * C * C * dk + C * C * C / 3 + C * C * (dk + dv));
       break;
     case kKScanFwd:
+      w.io_bytes = ntok * (2 * dk + dv) * es;
       w.bytes = ntok * ((dk + dv) * 4 + gk * 4 + 2 * dk * es) + nb * C * C * 4 +
                 ntok * dv * es + (states_io ? st : 0);
       w.flops = nb * (6 * C * dk * dv + C * C * dv);
       break;
     case kKScanBwd:
+      w.io_bytes = ntok * (2 * dk + dv) * es;
       w.bytes = ntok * (dk * 4 + gk * 4 + 2 * dk * es + dv * es) + nb * C * C * 4 + st +
                 ntok * dv * 4;
       w.flops = nb * (6 * C * dk * dv + C * C * dv);
       break;
     case kKStateGrads:
+      w.io_bytes = ntok * dv * es;
       w.bytes = 2 * st + ntok * (dk * 4 + 2 * dv * 4 + dv * es) + ntok * (dv * 4 + 3 * dk * 4) +
                 nb * dk * 4;
       w.flops = nb * 8 * C * dk * dv;
       break;
     case kKIntraBwd:
+      w.io_bytes = ntok * ((2 * dk + 2 * dv) * es + gk * 4 + 4) +
+                   ntok * ((2 * dk + dv) * es + gk * 4 + 4);
       w.bytes = ntok * ((2 * dk + 2 * dv) * es + gk * 4 + 12) + nb * C * C * 4 +
                 ntok * (3 * dv + 4 * dk) * 4 + nb * dk * 4 + ntok * ((2 * dk + dv) * es + gk * 4 + 4);
       w.flops = nb * (C * C * dv + 2 * C * C * dk + 2 * C * C * (dk + dv) + 2 * C * C * dk);
@@ -713,7 +720,7 @@ template <typename F>
 cudaError_t timed_launch(int kernel, const Problem& p, int es, bool states_io, cudaStream_t st,
                          F&& launch) {
   const Work w = work_of(kernel, p, es, states_io);
-  prof_begin(kernel, w.bytes, w.flops, st);
+  prof_begin(kernel, w.io_bytes, w.bytes, w.flops, st);
   launch();
   cudaError_t e = cudaGetLastError();
   prof_end(st);

@@ -19,7 +19,7 @@ constexpr int kMaxRecords = 8192;
 
 struct Record {
   int kernel;
-  double bytes, flops;
+  double io_bytes, bytes, flops;
   cudaEvent_t start, stop;
 };
 
@@ -49,12 +49,13 @@ const char* kernel_name(int id) {
   return "unknown";
 }
 
-void prof_begin(int kernel, double bytes, double flops, cudaStream_t st) {
+void prof_begin(int kernel, double io_bytes, double bytes, double flops, cudaStream_t st) {
   if (!g_enabled) return;
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_nrec >= kMaxRecords) return;
   Record& r = g_rec[g_nrec];
   r.kernel = kernel;
+  r.io_bytes = io_bytes;
   r.bytes = bytes;
   r.flops = flops;
   cudaEventRecord(r.start, st);
@@ -107,10 +108,14 @@ int dr_profile_read(dr_kernel_time* out, int max_out) {
       strncpy(out[n].name, dr::kernel_name(r.kernel), sizeof(out[n].name) - 1);
       ++n;
     }
+    // running means over the kernel's launches (its launches may differ, e.g.
+    // the transfer-matrix and output passes of a segmented scan)
+    const double c = out[j].launches, w = 1.0 / (c + 1.0);
     out[j].launches += 1;
     out[j].ms_total += ms;
-    out[j].bytes_per_launch = r.bytes;
-    out[j].flops_per_launch = r.flops;
+    out[j].bytes_per_launch += (r.io_bytes - out[j].bytes_per_launch) * w;
+    out[j].flops_per_launch += (r.flops - out[j].flops_per_launch) * w;
+    out[j].design_bytes_per_launch += (r.bytes - out[j].design_bytes_per_launch) * w;
   }
   dr::g_nrec = 0;
   return n;

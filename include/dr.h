@@ -161,9 +161,12 @@ dr_status dr_decode_step(const dr_problem* p, const void* q, const void* k, cons
    the scratch is a static device array of DR_STATIC_SCRATCH_BYTES shared by
    every call in the process.
    - Returns DR_ERR_WORKSPACE, launching nothing, when the problem's forward
-     scratch (dr_workspace_size(p, 0)) exceeds DR_STATIC_SCRATCH_BYTES; for
-     example a per-channel gate with dk = dv = 128 fits at most about 400
-     (batch x head x 64-token chunk) blocks.
+     scratch exceeds DR_STATIC_SCRATCH_BYTES: the exact test is
+     dr_workspace_size(p, 0) <= DR_STATIC_SCRATCH_BYTES.  With dk = dv = 128
+     the forward keeps about 129 KiB per (batch x head x 64-token chunk)
+     block, so about 500 blocks fit; a long sequence with few heads (which
+     takes the chunk-parallel affine scan) also keeps 192 KiB per segment of
+     each head.
    - Uses the device current at the call, which must own `stream` and every
      pointer.  The first call on a device looks up the scratch's device
      address (cudaGetSymbolAddress) with that device current; make that first
@@ -185,6 +188,19 @@ const char* dr_status_string(dr_status s);
    DR_ERR_CUDA if the stream reported an error, else DR_OK. */
 dr_status dr_last_device_error(void* stream);
 
+/* Fault injection, for testing the timeout path without faulting a GPU.
+   Every wait of the library's tensor-core kernels on an mbarrier is bounded:
+   when one gives up, the kernel records DR_ERR_TIMEOUT in the device flag
+   that dr_last_device_error reports, lets its copies in flight land, frees
+   its tensor memory and returns, leaving the context usable; its outputs are
+   then undefined.  After dr_inject_timeout(n), each of the next n launches
+   of the chunk backward kernel (inside dr_chunk_bwd) first waits, with a
+   limit of a few hundred polls, on an mbarrier that nothing arrives on, once
+   all its inputs have landed and before its first tensor-core instruction,
+   and so takes that path.  n = 0 cancels pending injections; n < 0 gives
+   DR_ERR_INVALID_ARG.  Process-wide, host only. */
+dr_status dr_inject_timeout(int launches);
+
 /* Opt-in per-kernel timing, for benchmarking.  While enabled (on != 0),
    every kernel the library launches is bracketed by two CUDA events recorded
    on the launch stream.  The first enable creates the events (no device
@@ -192,21 +208,27 @@ dr_status dr_last_device_error(void* stream);
 dr_status dr_profile_enable(int on);
 
 /* Per-kernel summary of the launches recorded since the last read or enable:
-   name, launch count, summed event time, and the kernel's work model per
-   launch (algorithmic HBM bytes and FLOPs for the problem it ran on). */
+   name, launch count, summed event time, and the kernel's work model, the
+   mean over its launches: bytes_per_launch counts the operator's own inputs
+   and outputs that the launch reads or writes (q, k, v, g, beta, dO, o, the
+   gradients and the states, each once: the algorithmic bytes);
+   design_bytes_per_launch adds everything else the launch moves by this
+   library's design (the per-chunk tiles and states kept between kernels);
+   flops_per_launch is its arithmetic. */
 typedef struct {
   char name[32];
   int launches;
   double ms_total;
   double bytes_per_launch;
   double flops_per_launch;
+  double design_bytes_per_launch;
 } dr_kernel_time;
 
 /* Waits for the recorded events, writes up to max_out entries to out and
    returns their number (-1 on a CUDA error); clears the records. */
 int dr_profile_read(dr_kernel_time* out, int max_out);
 
-/* Library ABI version (major * 100 + minor). */
+/* Library ABI version (major * 100 + minor): 200. */
 int dr_version(void);
 
 #ifdef __cplusplus

@@ -174,3 +174,8 @@ def test_phase_gate_routing(lib):
     n = ctypes.c_size_t(0)
     assert lib.dr_workspace_size(ctypes.byref(_prob(gate="phase", dk=128, dv=128)), 0,
                                  ctypes.byref(n)) == binding.DR_OK and n.value > 0
+
+
+def test_inject_timeout_arguments(lib):
+    assert lib.dr_inject_timeout(-1) == binding.DR_ERR_INVALID_ARG
+    assert lib.dr_inject_timeout(0) == binding.DR_OK

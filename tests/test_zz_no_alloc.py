@@ -7,7 +7,6 @@ This file is collected last, so a run that stops at the first failure has
 already run every other test."""
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
@@ -26,20 +25,29 @@ def _lib():
     return lib
 
 
-def _rel(x, y):
-    x, y = x.double().cpu().numpy(), y.double().cpu().numpy()
-    return float(np.max(np.abs(x - y)) / np.max(np.abs(y)))
-
-
 @pytest.fixture(scope="module", autouse=True)
 def _cuda():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA GPU")
 
 
-def test_static_scratch_forward_matches_workspace_forward_twice():
+# Two problems: a short one (plain sequential scans) and a long one with few
+# heads, which takes the chunk-parallel affine scan and so also keeps segment
+# transfer matrices and states in the static scratch.
+CASES = [
+    WORKLOADS["kda_bf16_b4h16t8192"].with_(name="noalloc", B=2, H=4, T=1000, s0_std=0.1),
+    WORKLOADS["kda_bf16_b4h16t8192"].with_(name="noalloc_segmented", B=1, H=2, T=4096,
+                                           s0_std=0.1),
+]
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_static_scratch_forward_matches_workspace_forward_twice(w):
+    """Both entry points run the same kernels on the same inputs, so their
+    results must be bit-identical; two calls in a row with different inputs
+    check that nothing left in the shared scratch by one call leaks into the
+    next."""
     lib = _lib()
-    w = WORKLOADS["kda_bf16_b4h16t8192"].with_(name="noalloc", B=2, H=4, T=1000, s0_std=0.1)
     plan = binding.Plan.for_workload(w)
     assert binding.workspace_size(plan.prob, 0) <= STATIC_SCRATCH_BYTES
     stream = torch.cuda.current_stream()
@@ -56,8 +64,9 @@ def test_static_scratch_forward_matches_workspace_forward_twice():
         assert st == binding.DR_OK, binding.status_string(st)
         torch.cuda.synchronize()
         assert binding.last_device_error() == binding.DR_OK
-        assert _rel(o, o_ref) <= 2e-2
-        assert _rel(ST, ST_ref) <= 2e-2
+        assert torch.isfinite(o.float()).all() and torch.isfinite(ST).all()
+        assert torch.equal(o, o_ref)
+        assert torch.equal(ST, ST_ref)
 
 
 def test_static_scratch_rejects_problems_beyond_its_size():
