@@ -28,8 +28,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "fwd+bwd tokens/s (GDN/KDA, bf16, d=128); % of B200 tensor-core/HBM roofline"
-# The SFDA phase-gate workload has a forward only (no backward is built for it).
-METRIC_FWD = "fwd tokens/s (SFDA phase gate, bf16, d=128); % of B200 tensor-core/HBM roofline"
+# The SFDA phase-gate workload (a rotation-decay per key pair) measures the same step.
+METRIC_SFDA = "fwd+bwd tokens/s (SFDA phase gate, bf16, d=128); % of B200 tensor-core/HBM roofline"
 UNIT = "tokens/s"
 # Used only when the measured-peaks file is absent (an earlier measurement on this GPU pool).
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -68,9 +68,8 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def algorithmic_step(w, fwd_only=False):
-    """Per-step algorithmic FLOPs and HBM bytes of forward + backward (or of
-    the forward alone).
+def algorithmic_step(w):
+    """Per-step algorithmic FLOPs and HBM bytes of forward + backward.
 
     FLOPs per token-head: forward 10 C d + 6 d^2, backward with recompute
     28 C d + 14 d^2 (d = d_k = d_v).  Bytes: every input read and output
@@ -84,9 +83,6 @@ def algorithmic_step(w, fwd_only=False):
     th = w.token_heads
     io = (2 * w.dk + w.dv) * es + gb + 4
     fwd = io + w.dv * es
-    if fwd_only:
-        state = w.B * w.H * w.dv * w.dk * 4 * (1 + (1 if w.s0_std > 0 else 0))  # S_T (+ S0)
-        return th * (10 * C * d + 6 * d * d), th * fwd + state
     flops = th * (10 * C * d + 6 * d * d + 28 * C * d + 14 * d * d)
     bwd = io + w.dv * es + (2 * w.dk + w.dv) * es + gb + 4
     nstate = 2 + (2 if w.s0_std > 0 else 0)  # S_T, dS0 (+ S0 read twice)
@@ -201,9 +197,8 @@ class ClockSampler:
 
 
 def cpu_baseline(w, inp, seconds):
-    """Time the fp64 oracle (forward + backward; forward only for the phase
-    gate) on host cores on a bounded sample: all heads, the first T_s tokens,
-    T_s sized to about `seconds`."""
+    """Time the fp64 oracle (forward + backward) on host cores on a bounded
+    sample: all heads, the first T_s tokens, T_s sized to about `seconds`."""
     import oracle
 
     mode = oracle.BETA_KACZMARZ if w.beta_mode == "kaczmarz" else oracle.BETA_DIRECT
@@ -218,9 +213,8 @@ def cpu_baseline(w, inp, seconds):
         _, _, thr = oracle.recurrent_fwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0,
                                          beta_mode=mode, eps=w.eps, return_threads=True,
                                          gate=gate)
-        if not phase:
-            oracle.recurrent_bwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0, sl["dO"],
-                                 beta_mode=mode, eps=w.eps)
+        oracle.recurrent_bwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0, sl["dO"],
+                             beta_mode=mode, eps=w.eps, gate=gate)
         return time.perf_counter() - t0, thr
 
     probe = min(w.T, 128)
@@ -229,7 +223,7 @@ def cpu_baseline(w, inp, seconds):
     dt, thr = run(Ts)
     tokens_equiv = w.B * Ts  # all heads of B x Ts tokens
     return {"value": tokens_equiv / dt, "unit": UNIT, "cores": thr, "kind": "oracle",
-            "sample": f"fp64 oracle {'forward' if phase else 'forward+backward'} on all "
+            "sample": f"fp64 oracle forward+backward on all "
                       f"{w.B * w.H} heads x the first "
                       f"{Ts} of {w.T} tokens of the same inputs, wall clock {dt:.1f} s",
             "seconds": dt}
@@ -248,7 +242,7 @@ def run_reference(args):
     inp = make_inputs(w)
     oracle.build()
     mode = oracle.BETA_KACZMARZ if w.beta_mode == "kaczmarz" else oracle.BETA_DIRECT
-    phase = w.gate == "phase"   # forward only: the phase gate has no backward
+    phase = w.gate == "phase"
     total_steps = args.steps + args.warmup
     budget = 150.0  # seconds for the whole run
     per_step = budget / max(total_steps, 1)
@@ -263,9 +257,9 @@ def run_reference(args):
         _, _, thr = oracle.recurrent_fwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0,
                                          beta_mode=mode, eps=w.eps, return_threads=True,
                                          gate=oracle.GATE_PHASE if phase else None)
-        if not phase:
-            oracle.recurrent_bwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0, sl["dO"],
-                                 beta_mode=mode, eps=w.eps)
+        oracle.recurrent_bwd(sl["q"], sl["k"], sl["v"], sl["beta"], sl["g"], S0, sl["dO"],
+                             beta_mode=mode, eps=w.eps,
+                             gate=oracle.GATE_PHASE if phase else None)
         return time.perf_counter() - t0, thr
 
     probe = min(w.T, 64)
@@ -280,10 +274,10 @@ def run_reference(args):
         times.append(dt)
     tot = sum(times)
     value = w.B * Ts * args.steps / tot
-    desc = (f"fp64 oracle {'forward' if phase else 'forward+backward'} per step on all "
+    desc = (f"fp64 oracle forward+backward per step on all "
             f"{w.B * w.H} heads x the first {Ts} of {w.T} tokens of the workload's inputs")
     print(json.dumps({
-        "impl": "reference", "metric": METRIC_FWD if phase else METRIC, "value": value,
+        "impl": "reference", "metric": METRIC_SFDA if phase else METRIC, "value": value,
         "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": tot / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -441,24 +435,21 @@ def main():
     inp = make_inputs(w, seed=w.seed + 1000 * rank)
     d = {n: (None if x is None else x.to(dev)) for n, x in inp.items()}
     plan = binding.Plan.for_workload(w, device=dev)
-    fwd_only = w.gate == "phase"   # the phase gate has no backward
-    keep = args.policy == "save" and not fwd_only
+    keep = args.policy == "save"
     saved = plan.new_saved() if keep else None
     o, ST, _ = plan.fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], saved=saved,
                         save=keep)
-    grads = {} if fwd_only else \
-        plan.bwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], d["dO"], None, saved)
+    grads = plan.bwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], d["dO"], None, saved)
     stream = torch.cuda.current_stream(dev)
 
     def step():
         plan.fwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], o=o, ST=ST, saved=saved,
                  save=keep)
-        if not fwd_only:
-            plan.bwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], d["dO"], None, saved,
-                     out=grads)
+        plan.bwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"], d["dO"], None, saved,
+                 out=grads)
 
     in_bytes = sum(x.numel() * x.element_size() for n, x in d.items()
-                   if x is not None and not (fwd_only and n == "dO"))
+                   if x is not None)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
     for _ in range(args.warmup):
@@ -492,7 +483,7 @@ def main():
     # copied in and every output copied back, inside the timed region.
     e2e = None
     if not args.no_e2e:
-        hin = {n: (None if x is None or (fwd_only and n == "dO") else x.pin_memory())
+        hin = {n: (None if x is None else x.pin_memory())
                for n, x in inp.items()}
         hout = {"o": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
                 "ST": torch.empty(ST.shape, dtype=ST.dtype).pin_memory()}
@@ -507,9 +498,8 @@ def main():
                     dev_in[n].copy_(x, non_blocking=True)
             plan.fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"], dev_in["g"],
                      dev_in["S0"], o=o, ST=ST, saved=saved, save=keep)
-            if not fwd_only:
-                plan.bwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"], dev_in["g"],
-                         dev_in["S0"], dev_in["dO"], None, saved, out=grads)
+            plan.bwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"], dev_in["g"],
+                     dev_in["S0"], dev_in["dO"], None, saved, out=grads)
             hout["o"].copy_(o, non_blocking=True)
             hout["ST"].copy_(ST, non_blocking=True)
             for n, x in grads.items():
@@ -576,7 +566,7 @@ def main():
                  "design_bytes_per_launch": design,
                  "design_frac": design / per_launch_s / 1e9 / peaks["hbm_gbs"]})
 
-    flops, nbytes = algorithmic_step(w, fwd_only)
+    flops, nbytes = algorithmic_step(w)
     t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     t_roof = max(t_tc, t_hbm)
@@ -590,7 +580,7 @@ def main():
         cpu = cpu_baseline(w, inp, args.cpu_seconds)
 
     out = {
-        "metric": METRIC_FWD if fwd_only else METRIC, "value": value, "unit": UNIT,
+        "metric": METRIC_SFDA if w.gate == "phase" else METRIC, "value": value, "unit": UNIT,
         "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
@@ -601,9 +591,8 @@ def main():
                    "parallelism": f"replicas x{world} (independent batches, no collective)",
                    "l2": f"L2 flushed between timed steps ({2 * L2_BYTES >> 20} MiB write); "
                          f"inputs {in_bytes >> 20} MiB per step",
-                   "policy": ("forward only (no backward for the phase gate)" if fwd_only
-                              else "forward saves chunk tiles and states; backward reads them"
-                              if keep else "backward recomputes the chunk tiles and states")},
+                   "policy": ("forward saves chunk tiles and states; backward reads them" if keep
+                              else "backward recomputes the chunk tiles and states")},
         "roofline": roof,
         "step_roofline": step_roof,
         "cpu_baseline": cpu,

@@ -274,8 +274,10 @@ dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const 
   if (!q || !k || !v || !beta || !dO || !dq || !dk || !dv || !dbeta)
     return DR_ERR_INVALID_ARG;
   if ((P.gate == DR_GATE_NONE) != (g == nullptr)) return DR_ERR_INVALID_ARG;
-  if (P.gate == DR_GATE_PHASE) return DR_ERR_UNSUPPORTED;  // forward and decode only
   if (P.gate != DR_GATE_NONE && !dg) return DR_ERR_INVALID_ARG;
+  // the phase gate runs on the tensor-core path only
+  if (P.gate == DR_GATE_PHASE && !dr::fast::eligible(P, p->dtype == DR_BF16))
+    return DR_ERR_UNSUPPORTED;
   const void* ptrs[] = {q, k, v, beta, g, S0, dO, dST, saved, dq, dk, dv, dbeta, dg, dS0};
   for (const void* x : ptrs)
     if (!aligned16(x)) return DR_ERR_INVALID_ARG;
@@ -326,7 +328,7 @@ const char* dr_status_string(dr_status s) {
   switch (s) {
     case DR_OK: return "ok";
     case DR_ERR_INVALID_ARG: return "invalid argument";
-    case DR_ERR_UNSUPPORTED: return "unsupported problem (chunk must be 64; dk, dv multiples of 16 up to 128; phase gate: bf16, dk = dv = 128, no backward)";
+    case DR_ERR_UNSUPPORTED: return "unsupported problem (chunk must be 64; dk, dv multiples of 16 up to 128; phase gate: bf16, dk = dv = 128)";
     case DR_ERR_WORKSPACE: return "workspace or saved buffer missing, misaligned or too small";
     case DR_ERR_CUDA: return "CUDA error";
     case DR_ERR_TIMEOUT: return "a bounded device-side wait timed out";

@@ -90,28 +90,6 @@ __host__ __device__ __forceinline__ int ct_col(int idx, int ncol) {
   return ((idx >> 3) % (ncol >> 3)) * 8;
 }
 
-// cp.async of a core-tiled [R][ncol] global tile into a padded row-major
-// shared tile (row stride lds): chunk idx is read from g + 8 idx (a warp reads
-// 512 contiguous bytes) and lands at row ct_row, column ct_col (eight lanes
-// write eight rows: no bank conflicts when lds = 8 mod 64).
-template <int NTHREADS>
-__device__ __forceinline__ void cp_ct_to_rows(__nv_bfloat16* smem, int lds,
-                                              const __nv_bfloat16* g, int R, int ncol, int tid) {
-  for (int idx = tid; idx < R * ncol / 8; idx += NTHREADS)
-    frag::cp16(smem + ct_row(idx, ncol) * lds + ct_col(idx, ncol), g + 8 * idx, true);
-}
-// The same for columns c0 .. c0 + w - 1 of a core-tiled [R][128] tile (each
-// row block of the slice is w 16-byte chunks, contiguous in global memory).
-template <int NTHREADS>
-__device__ __forceinline__ void cp_ct_cols_to_rows(__nv_bfloat16* smem, int lds,
-                                                   const __nv_bfloat16* g, int R, int c0, int w,
-                                                   int tid) {
-  for (int idx = tid; idx < R * w / 8; idx += NTHREADS) {
-    const int grp = idx / w, k = idx % w;
-    frag::cp16(smem + (grp * 8 + (k & 7)) * lds + (k >> 3) * 8,
-               g + ((size_t)grp * 16 + (c0 >> 3)) * 64 + 8 * k, true);
-  }
-}
 // Columns c0 .. c0 + w - 1 of a core-tiled [R][128] tile into a core-tiled
 // [R][w] shared tile.
 template <int NTHREADS>
@@ -154,7 +132,8 @@ inline Saved carve_saved(const Problem& p, void* base) {
   return s;
 }
 
-// tc_prep: all state-independent per-chunk tensors (T, beta, dec, W, U', M, Qh, Kt).
+// tc_prep (fast_prep.cu): all state-independent per-chunk tensors (T, beta,
+// dec, W, U', M, Qh, Kt, ||k||^2), on tcgen05 with TMA loads.
 cudaError_t launch_prep(const Problem& p, const __nv_bfloat16* q, const __nv_bfloat16* k,
                         const __nv_bfloat16* v, const float* beta, const float* g,
                         const Saved& sv, cudaStream_t st);

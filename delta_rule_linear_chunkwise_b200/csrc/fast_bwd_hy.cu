@@ -1,25 +1,55 @@
 // fast_bwd_hy.cu -- chunk-parallel backward with the products on tcgen05 and
 // the element-wise work on all 16 warps (bf16 storage, d_k = d_v = 128, C = 64).
 //
-// One CTA per (b, h, chunk).  With ep = e^{gamma - gamma_r} (gamma_r: the cumulative
-// gate at the chunk's centre row) and the chunk's saved tiles:
-//   level 1  dQs = dO S, dW' = dU S, dKt = U dS', dM = tril(dO U^T)
+// One CTA per (b, h, chunk).  From the chunk's saved tiles (T, W, U', the
+// chunk-start state S = h_n, the pseudo-values U) and the state-gradient scan's
+// dU and dS' (the gradient of the chunk's end state):
+//   level 1  dQs = dO S, dW = -dU S, dKt = U dS', dM = tril(dO U^T)  (its diagonal
+//            kept apart in fp32: it enters dq and dk with the factor 1 and cancels in dg)
 //   level 2  Lambda = T^T [dU | dW]             (dv = diag(beta) Lambda_U)
 //   level 3  dA = -strict_tril(Lambda_U U'^T + Lambda_W W^T)
-//   level 4  dM Kb^c, dA Kb^c, dM^T Q^c + dA^T diag(beta) K^c
-// and the register epilogue over Z = e^{gamma_r} dQs + dM Kb^c,
-// P = e^{gamma_C - gamma_r} dKt + dM^T Q^c + dA^T beta K^c, Q = e^{gamma_r} Lambda_W + dA Kb^c:
-// dq = ep Z, dk = P / ep + beta ep Q, dgamma = k (beta ep Q - P / ep) + Q^c Z, then the
-// gate reverse cumulative sum and the Kaczmarz chain rule.
+//   level 4  the gate-scaled products of dM and dA with the keys and queries:
+//            F1_i = sum_{j<=i} dM_ij k_j e^{g_i - g_j},  F2_i = sum_{j<i} dA_ij k_j e^{g_i - g_j},
+//            G_j  = sum_{i>=j} (dM_ij q_i + dA_ij beta_i k_i) e^{g_i - g_j}
+//            (g: the within-chunk cumulative log-gate of each key channel)
+// which give dq, dk, dgamma and dbeta in a register epilogue, then the gate's
+// reverse cumulative sum and the Kaczmarz chain rule.  The chunk correction is
+// differentiated as the triangular residual system (I + A)[U' | W] = diag(beta)
+// [V | k e^g] (ReWY abstract): one transposed triangular product (level 2), no
+// adjoint of the inverse.
+//
+// Reference rows.  The gate factors of level 4 are exponentials of differences
+// of cumulative gates.  Every row i uses the reference row rho of its own
+// 32-row half (rows 15 and 47), e^{g_i - g_j} = e^{g_i - g_rho} e^{g_rho - g_j}:
+// the first factor spans at most 16 rows of decay, and the second does too for
+// j in the same half, while for j in the earlier half it is at most 1 (an
+// underflow there drops a term that is negligible against the kept ones).  So
+// no factor overflows unless the gates decay by more than about 5.5 nats per
+// token over 16 consecutive tokens ("centered matrix contractions", ReWY
+// abstract).  A factor that crosses halves is applied in two steps through the
+// half boundary, each at most 1 in size, so it underflows only where the
+// exact product would.  Products whose reference differs between output rows are split:
+// F1 and F2 read dM and dA through row-masked copies (rows of the other half
+// zero) against per-half key tiles, accumulating into one tensor-memory tile;
+// G (whose output rows are the keys) has one accumulator per half.
+//
+// PHASE: the SFDA rotation-decay gate ("Semidirect Fourier Delta Attention"
+// explainer, Kernarchitektur).  Key channels pair up as complex numbers, the
+// chunk's cumulative decay of a pair is zeta_i = e^{g_i - i Theta_i} (g, Theta:
+// the cumulative sums at the pair's even and odd channels), and every real
+// factor above becomes a per-pair complex one: u_i = zeta_i / zeta_rho scales
+// queries and read keys, 1 / conj(u_i) the write keys.  Gradients map back by
+// the conjugate factors, d/dg of a pair is Re(.) and d/dTheta is Im(.) of the
+// same products (with the write-key and chunk-end terms of opposite sign in g).
 //
 // Each level is a set of tcgen05.mma (M = 64, operands in shared memory in the
 // canonical core-matrix layout, fp32 accumulators in tensor memory) issued by
-// one thread, independent accumulation chains interleaved (long chains split
-// into partial sums).  An M = 64 accumulator occupies lanes 16 q .. 16 q + 15 of each
+// one thread.  An M = 64 accumulator occupies lanes 16 q .. 16 q + 15 of each
 // 32-lane quadrant q, and tcgen05.ld.16x256b returns it to the warps of that
-// quadrant in exactly the register fragment of a warp-level m16n8 product
-// (thread t: row t / 4 and t / 4 + 8, columns 2 (t % 4), + 1 of each 8-column
-// group), so warp w = 4 qt + rb owns rows 16 rb .., columns 32 qt ...
+// quadrant in the register fragment of a warp-level m16n8 product (thread t:
+// row t / 4 and t / 4 + 8, columns 2 (t % 4), + 1 of each 8-column group), so
+// warp w = 4 qt + rb owns rows 16 rb .., columns 32 qt ..; a thread's two
+// columns are one key pair.
 
 #include "dr_common.cuh"
 #include "fast.cuh"
@@ -41,37 +71,53 @@ constexpr uint32_t kSpinHy = 1u << 22;
 // Polls of the injected wait (dr_inject_timeout): short, so the test that
 // drives the timeout path ends within milliseconds.
 constexpr uint32_t kSpinInjected = 256;
+constexpr int kRho0 = 15, kRho1 = 47;  // reference rows of the two halves
 
-__device__ __forceinline__ int centre_row(int nvalid) { return (nvalid - 1) / 2; }
 // Gate tile element (i, c): 8-column groups XOR-swizzled by row.
 __device__ __forceinline__ int gsw(int i, int c) { return i * D + (c ^ ((i & 7) << 3)); }
 
-// Tensor memory columns (512 allocated): level 1 uses all four ranges, the
-// later levels reuse them once the earlier accumulators are in registers.
-constexpr uint32_t T_ZQ = 0, T_ADW = 128, T_AKT = 256, T_ADM = 384;
-constexpr uint32_t T_LU = 0, T_LW = 128;
-constexpr uint32_t T_DA = 256;  // four 64-column partial sums of dA
-constexpr uint32_t T_Z2 = 0, T_X = 128, T_Y = 256, T_Y2 = 384;
+// Tensor memory columns (512 allocated): each level reuses the columns whose
+// accumulators the previous levels have read back.
+constexpr uint32_t T_ZQ = 0, T_ADW = 128, T_AKT = 256, T_ADM = 384;  // level 1
+constexpr uint32_t T_LU = 0, T_LW = 128;                             // level 2
+constexpr uint32_t T_DA = 256;  // level 3: four 64-column partial sums of dA
+constexpr uint32_t T_F1 = 0, T_G0 = 128, T_F2 = 256, T_G1 = 384;     // level 4
+
+// Row-masked copy of a 64 x 64 matrix for level 4 ("X tile"): core-tiled
+// K-major (8 x 8 blocks of 128 bytes, rows of blocks 1 KB apart), rows 0..31
+// at bytes [0, 4K), zeros at [4K, 8K), rows 32..63 at [8K, 12K).  Read from
+// byte 0 it is the matrix with rows 32..63 zeroed, from byte 4K the matrix with
+// rows 0..31 zeroed; read by k-steps of 16 rows that skip the zero block, its
+// transpose.
+constexpr int kXElems = 3 * C * C / 2;  // 12 KB
 
 struct HySmem {
-  bf16 SS[D * D];   // S = h_n [a][c], core-tiled (MN-major B);  then Lambda_U | Lambda_W;
-                    // at the end the fp32 dgamma tile
-  bf16 SD[D * D];   // dS' [a][c];  then W | U' (level 3);  then Kb^c | beta K^c (level 4)
-  bf16 DO[C * D];   // dO [i][a] (K-major A);  then dW [j][c]
-  bf16 DU[C * D];   // dU [j][a]
-  bf16 UU[C * D];   // U [j][a];  then dM [i][j] | dA [i][j]
-  bf16 QC[C * D];   // Q^c [j][c], core-tiled
+  bf16 SS[D * D];   // S = h_n [a][c] (level 1);  Lambda_U | Lambda_W (levels 2-3);
+                    // beta k^{rho0} (level 4);  at the end the fp32 dgamma tile (with SD)
+  bf16 SD[D * D];   // dS' [a][c];  then W | U' (level 3)
+  bf16 DO[C * D];   // dO [i][a] (K-major A);  then dW [j][c] (level 2);  then Kb^{rho1} (level 4)
+  bf16 DU[C * D];   // dU [j][a];  then q^{rho0} (level 4)
+  bf16 UU[2 * kXElems];  // U [j][a] (level 1, first 16 KB);  then the X tiles of dM and dA
+  bf16 QC[C * D];   // Kb^{rho0} rows 0..31 | q^{rho1} rows 32..63 (level 4)
   bf16 QR[C * LDD]; // raw q, row-major padded
   bf16 k[C * LDD];  // raw k, row-major padded
-  bf16 TT[C * C];   // T [j][i], core-tiled (MN-major A of T^T)
-  float G[C * D];   // cumulative gate (gsw), then e^{gamma - gamma_r}
+  bf16 TT[C * C];   // T [i][j], core-tiled (MN-major A of T^T);  then beta k^{rho1} rows 32..63
+  float G[C * D];   // cumulative gate (gsw), then the factor u_i of each element
   float beta[C];
   float knorm[C];
   float dbp[C * 4];
   float dgc[4 * D];
   float ktk[4 * D];
-  float er[D];
-  float erc[D];
+  float er[2 * D];   // per half: conj(zeta_rho)                (real gates: e^{g_rho})
+  float erc[2 * D];  // per half: zeta_C / zeta_rho             (real gates: e^{g_C - g_rho})
+  // cross-half factors, each spanning at most 17 rows: write keys of the first
+  // half against the second reference, conj(zeta_31 / zeta_rho0) conj(zeta_rho1 / zeta_31),
+  // and queries / keys of the second half against the first reference,
+  // (zeta_rho1 / zeta_32) (zeta_32 / zeta_rho0); applied one after the other, so
+  // that no intermediate underflows where the product does not
+  float xk[2 * D];
+  float xq[2 * D];
+  float dmd[C];      // the diagonal of dM (fp32), added outside the level-4 products
   uint64_t bar;
   uint64_t never;   // fault injection: a barrier that nothing ever arrives on
   uint32_t tmem;
@@ -80,53 +126,27 @@ struct HySmem {
 static_assert(offsetof(HySmem, SD) == offsetof(HySmem, SS) + sizeof(bf16) * D * D &&
                   sizeof(float) * C * LDG <= sizeof(bf16) * 2 * D * D,
               "the padded dgamma tile spans the adjacent S and dS' tiles");
+static_assert(sizeof(bf16) * C * D <= sizeof(bf16) * 2 * kXElems, "U fits the X-tile region");
 
-// One product chain D[tm] (+)= A B (M = 64) over k-steps ks0, ks0 + kstride, ...
-// (count of them); A: K-major [64][K] (a_dim = K) or MN-major [K][64], B: K-major
-// [N][K] (b_dim = K) or MN-major [K][N] (b_dim = N).  The first step overwrites
-// the accumulator.
-struct Chain {
-  uint32_t tm;
-  uint64_t a0, b0;     // descriptors of k-step 0
-  uint32_t da, db;     // descriptor start-address advance per k-step (16-byte units)
-  uint32_t id;
-  int ks0, kstride, count;
+// --- complex helpers (a key pair as x + i y) -------------------------------
+struct cf {
+  float x, y;
 };
-__device__ __forceinline__ Chain chain(uint32_t tm, const bf16* A, bool a_mn, int a_dim,
-                                       const bf16* B, bool b_mn, int b_dim, int N, int ks0,
-                                       int kstride, int count) {
-  Chain c;
-  c.tm = tm;
-  c.a0 = a_mn ? tc::sdesc_mnmaj(A, 64, 0) : tc::sdesc_kmaj(A, a_dim, 0);
-  c.b0 = b_mn ? tc::sdesc_mnmaj(B, b_dim, 0) : tc::sdesc_kmaj(B, b_dim, 0);
-  c.da = a_mn ? 2 * (64 / 8) * 128 / 16 : 256 / 16;
-  c.db = b_mn ? 2 * (b_dim / 8) * 128 / 16 : 256 / 16;
-  c.id = tc::idesc_bf16(64, N, a_mn, b_mn);
-  c.ks0 = ks0;
-  c.kstride = kstride;
-  c.count = count;
-  return c;
+__device__ __forceinline__ cf cmul(cf a, cf b) { return {a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x}; }
+// conj(a) b
+__device__ __forceinline__ cf cmulc(cf a, cf b) { return {a.x * b.x + a.y * b.y, a.x * b.y - a.y * b.x}; }
+__device__ __forceinline__ cf cconj(cf a) { return {a.x, -a.y}; }
+// 1 / u, scaled so that |u|^2 is never formed (|u| up to e^{+-80} stays finite)
+__device__ __forceinline__ cf cinv(cf u) {
+  const float s = __fdividef(1.f, fmaxf(fabsf(u.x), fabsf(u.y)));
+  const float a = u.x * s, b = u.y * s;
+  const float t = __fdividef(s, a * a + b * b);
+  return {a * t, -b * t};
 }
-// Issue the chains round-robin by step (consecutive instructions go to
-// independent accumulators).  Measured on B200: with the descriptors built
-// before the loop, one thread issues a tcgen05.mma of M = 64 or 128, N <= 128
-// every 55-70 cycles and the tensor core keeps pace, so a level costs about
-// its instruction count times that.
-template <int NC>
-__device__ __forceinline__ void issue_chains(const Chain (&cs)[NC]) {
-  int steps = 0;
-#pragma unroll
-  for (int i = 0; i < NC; ++i) steps = max(steps, cs[i].count);
-  for (int j = 0; j < steps; ++j) {
-#pragma unroll
-    for (int i = 0; i < NC; ++i) {
-      if (j < cs[i].count) {
-        const uint32_t ks = (uint32_t)(cs[i].ks0 + j * cs[i].kstride);
-        tc::mma(cs[i].tm, cs[i].a0 + ks * cs[i].da, cs[i].b0 + ks * cs[i].db, cs[i].id,
-                j > 0 ? 1u : 0u);
-      }
-    }
-  }
+
+__device__ __forceinline__ void mma_step(uint32_t tm, uint64_t a, uint64_t b, uint32_t id,
+                                         uint32_t acc) {
+  tc::mma(tm, a, b, id, acc);
 }
 
 // Fragments of 32 (ld4) or 16 (ld2) accumulator columns from column `col`,
@@ -162,30 +182,48 @@ __device__ __forceinline__ void frag_ld2(uint32_t col, int warp, float (&f)[2][4
 }
 
 // Bounded wait for the commit of level `phase`; CTA-uniform result.
-__device__ __forceinline__ bool hy_wait(uint64_t* bar, int phase,
-                                        uint32_t limit = kSpinHy) {
+__device__ __forceinline__ bool hy_wait(uint64_t* bar, int phase, uint32_t limit = kSpinHy) {
   const bool ok = tc::mbar_wait(bar, (uint32_t)(phase & 1), limit);
   const int bad = __syncthreads_or(ok ? 0 : 1);
   tc::fence_after_sync();
   return bad == 0;
 }
 
+// Descriptors: K-major [rows][K = 64] tiles (X tiles, row groups 1 KB apart),
+// MN-major [K][N = 128] tiles (the level-4 key and query tiles), MN-major
+// [K][M = 64] (an X tile read as its transpose).
+__device__ __forceinline__ uint64_t dk64(const bf16* t, uint32_t byte_off) {
+  return tc::sdesc(tc::smem_u32(t) + byte_off, 128, 1024);
+}
+__device__ __forceinline__ uint64_t dmn128(const bf16* t, uint32_t byte_off) {
+  return tc::sdesc(tc::smem_u32(t) + byte_off, 2048, 128);
+}
+__device__ __forceinline__ uint64_t dmn64(const bf16* t, uint32_t byte_off) {
+  return tc::sdesc(tc::smem_u32(t) + byte_off, 1024, 128);
+}
+// Byte offset of k-step ks (rows 16 ks .. 16 ks + 15) of an X tile's transpose.
+__device__ __forceinline__ uint32_t xt_off(int ks) {
+  return ks < 2 ? ks * 2048u : 8192u + (ks - 2) * 2048u;
+}
+
+template <bool PHASE>
 __global__ void __launch_bounds__(NTB, 1)
     k_bwd_chunk_hy(Problem p, const bf16* __restrict__ q, const bf16* __restrict__ k,
-                const bf16* __restrict__ v, const bf16* __restrict__ dO,
-                const float* __restrict__ g, const bf16* __restrict__ Tg,
-                const float* __restrict__ beta, const bf16* __restrict__ hst,
-                const bf16* __restrict__ dhst, const bf16* __restrict__ Ug,
-                const bf16* __restrict__ dUg, const bf16* __restrict__ Wg,
-                const bf16* __restrict__ Upg, const float* __restrict__ knorm_g,
-                bf16* __restrict__ dq, bf16* __restrict__ dk,
-                bf16* __restrict__ dv, float* __restrict__ dbeta, float* __restrict__ dg,
-                int* __restrict__ err, int inject_timeout) {
+                   const bf16* __restrict__ v, const bf16* __restrict__ dO,
+                   const float* __restrict__ g, const bf16* __restrict__ Tg,
+                   const float* __restrict__ beta, const bf16* __restrict__ hst,
+                   const bf16* __restrict__ dhst, const bf16* __restrict__ Ug,
+                   const bf16* __restrict__ dUg, const bf16* __restrict__ Wg,
+                   const bf16* __restrict__ Upg, const float* __restrict__ knorm_g,
+                   bf16* __restrict__ dq, bf16* __restrict__ dk, bf16* __restrict__ dv,
+                   float* __restrict__ dbeta, float* __restrict__ dg, int* __restrict__ err,
+                   int inject_timeout) {
   extern __shared__ __align__(1024) unsigned char smraw[];
   HySmem& s = *reinterpret_cast<HySmem*>(smraw);
   const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, gk = p.gk;
   const int rb = warp & 3, qt = warp >> 2;
+  const int hf = rb >> 1;  // the half of this warp's fragment rows
   const int lr = lane >> 2, lc = 2 * (lane & 3);
   const int t0 = n * C, nvalid = min(C, p.T - t0);
   const size_t cb = chunk_id(p, b, h, n);
@@ -193,11 +231,16 @@ __global__ void __launch_bounds__(NTB, 1)
   bf16* const sLW = s.SS + C * D;  // Lambda_W
   bf16* const sW = s.SD;           // W, U' for the third level
   bf16* const sUp = s.SD + C * D;
-  bf16* const sKb = s.DU;          // Kb^c, beta K^c for the fourth level (built under level 3)
-  bf16* const sBk = s.DO;
-  bf16* const sdW = s.DO;          // dW, after the first level (then beta K^c)
-  bf16* const sdM = s.UU;          // dM, dA [i][j], after the first level
-  bf16* const sdA = s.UU + C * C;
+  bf16* const sdW = s.DO;          // dW, after the first level
+  bf16* const XM = s.UU;           // X tile of dM
+  bf16* const XA = s.UU + kXElems; // X tile of dA
+  // level-4 key and query tiles (MN-major [K][N = 128], core-tiled [rows][128])
+  bf16* const Kb1 = s.DO;              // k_j / conj(zeta_j / zeta_rho1), rows 0..63
+  bf16* const Q0 = s.DU;               // (zeta_i / zeta_rho0) q_i, rows 0..63
+  bf16* const Kb0 = s.QC;              // k_j / conj(zeta_j / zeta_rho0), rows 0..31
+  bf16* const Q1 = s.QC + 32 * D;      // (zeta_i / zeta_rho1) q_i, rows 32..63
+  bf16* const B0 = s.SS;               // beta_i (zeta_i / zeta_rho0) k_i, rows 0..63
+  bf16* const B1 = s.TT;               // beta_i (zeta_i / zeta_rho1) k_i, rows 32..63
 
   // Loads in three cp.async groups, in the order of first use:
   //   1: gate, q, k   2: dO, dU, U, S, dS', T (first level)   3: W, U' (third level)
@@ -229,6 +272,9 @@ __global__ void __launch_bounds__(NTB, 1)
   cp_linear<NTB>(s.SD, dhst + cb * D * D, D * D, tid);
   cp_linear<NTB>(s.TT, Tg + cb * C * C, C * C, tid);
   frag::cp_commit();
+  // the zero block of the dA tile (outside the U region)
+  for (int idx = tid; idx < C * C / 16; idx += NTB)
+    *reinterpret_cast<uint4*>(XA + C * C / 2 + 8 * idx) = make_uint4(0, 0, 0, 0);
   if (warp == 0) tc::tmem_alloc(&s.tmem, 512);
   if (tid == 0) {
     tc::mbar_init(&s.bar, 1);
@@ -238,24 +284,23 @@ __global__ void __launch_bounds__(NTB, 1)
   __syncthreads();
   // element (i, c) of the gate tile
   auto gat = [&](int i, int c) -> float& { return gk == D ? s.G[gsw(i, c)] : s.G[i]; };
-  // cumulative gate down the chunk's rows
+  // cumulative gate down the chunk's rows (padded rows carry a zero gate)
   if (gk == D) {
     // thread (column c, row quarter q): scan of 16 rows, then the quarter offsets
-    // (the key-column partials of the consume phase hold the quarter totals)
-    const int c = tid & 127, q = tid >> 7;
+    const int c = tid & 127, q4 = tid >> 7;
     float run = 0.f;
 #pragma unroll
-    for (int i = 16 * q; i < 16 * q + 16; ++i) {
+    for (int i = 16 * q4; i < 16 * q4 + 16; ++i) {
       run += gat(i, c);
       gat(i, c) = run;
     }
-    s.ktk[q * D + c] = run;
+    s.ktk[q4 * D + c] = run;
     __syncthreads();
     float off = 0.f;
-    for (int q2 = 0; q2 < q; ++q2) off += s.ktk[q2 * D + c];
-    if (q > 0) {
+    for (int q2 = 0; q2 < q4; ++q2) off += s.ktk[q2 * D + c];
+    if (q4 > 0) {
 #pragma unroll
-      for (int i = 16 * q; i < 16 * q + 16; ++i) gat(i, c) += off;
+      for (int i = 16 * q4; i < 16 * q4 + 16; ++i) gat(i, c) += off;
     }
   } else if (warp == 0) {
     // rows 2 lane, 2 lane + 1: an inclusive scan across the warp
@@ -271,15 +316,78 @@ __global__ void __launch_bounds__(NTB, 1)
   }
   __syncthreads();
 
-  const int r = centre_row(nvalid);
-  if (tid < D) {
+  // per-channel reference factors (phase gate: per pair, complex, at the pair's two channels)
+  if (PHASE) {
+    if (tid < D / 2) {
+      const int c = 2 * tid;
+      const float gC = gat(C - 1, c), tC = gat(C - 1, c + 1);
+      float gr[2], tr[2];
+      gr[0] = gat(kRho0, c), tr[0] = gat(kRho0, c + 1);
+      gr[1] = gat(kRho1, c), tr[1] = gat(kRho1, c + 1);
+      const float g31 = gat(31, c), t31 = gat(31, c + 1), g32 = gat(32, c), t32 = gat(32, c + 1);
+      float sn, cs;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        sincosf(tr[hh], &sn, &cs);
+        const float m = __expf(gr[hh]);
+        s.er[hh * D + c] = m * cs;  // conj(zeta_rho) = e^{g_rho} e^{+i Theta_rho}
+        s.er[hh * D + c + 1] = m * sn;
+        sincosf(tC - tr[hh], &sn, &cs);
+        const float mc = __expf(gC - gr[hh]);
+        s.erc[hh * D + c] = mc * cs;  // zeta_C / zeta_rho
+        s.erc[hh * D + c + 1] = -mc * sn;
+      }
+      // zeta_a / zeta_b = e^{g_a - g_b} e^{-i (Theta_a - Theta_b)}; the write-key
+      // factors are conjugated
+      sincosf(t31 - tr[0], &sn, &cs);
+      float m = __expf(g31 - gr[0]);
+      s.xk[c] = m * cs, s.xk[c + 1] = m * sn;
+      sincosf(tr[1] - t31, &sn, &cs);
+      m = __expf(gr[1] - g31);
+      s.xk[D + c] = m * cs, s.xk[D + c + 1] = m * sn;
+      sincosf(tr[1] - t32, &sn, &cs);
+      m = __expf(gr[1] - g32);
+      s.xq[c] = m * cs, s.xq[c + 1] = -m * sn;
+      sincosf(t32 - tr[0], &sn, &cs);
+      m = __expf(g32 - gr[0]);
+      s.xq[D + c] = m * cs, s.xq[D + c + 1] = -m * sn;
+    }
+  } else if (tid < D) {
     const int cg = (gk == D) ? tid : 0;
-    const float gr = gat(r, cg), gC = gat(C - 1, cg);
-    s.er[tid] = __expf(gr);
-    s.erc[tid] = __expf(gC - gr);
+    const float g0 = gat(kRho0, cg), g1 = gat(kRho1, cg), gC = gat(C - 1, cg);
+    const float g31 = gat(31, cg), g32 = gat(32, cg);
+    s.er[tid] = __expf(g0);
+    s.er[D + tid] = __expf(g1);
+    s.erc[tid] = __expf(gC - g0);
+    s.erc[D + tid] = __expf(gC - g1);
+    s.xk[tid] = __expf(g31 - g0);
+    s.xk[D + tid] = __expf(g1 - g31);
+    s.xq[tid] = __expf(g1 - g32);
+    s.xq[D + tid] = __expf(g32 - g0);
   }
-  // gate tile -> e^{gamma - gamma_r} in place (every thread reads the centre row first)
-  {
+  // gate tile -> factor u_i = zeta_i / zeta_rho (real gates: e^{g_i - g_rho}), rho the
+  // reference row of row i's half (every thread reads the reference rows first)
+  if (PHASE) {
+    float tmp[C * D / NTB];
+#pragma unroll
+    for (int u = 0; u < C * D / NTB / 2; ++u) {
+      const int idx = tid + u * NTB;  // a key pair of one row
+      const int i = idx >> 6, c = 2 * (idx & 63), rho = i < 32 ? kRho0 : kRho1;
+      float sn, cs;
+      sincosf(gat(i, c + 1) - gat(rho, c + 1), &sn, &cs);
+      const float m = __expf(gat(i, c) - gat(rho, c));
+      tmp[2 * u] = m * cs;
+      tmp[2 * u + 1] = -m * sn;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < C * D / NTB / 2; ++u) {
+      const int idx = tid + u * NTB;
+      const int i = idx >> 6, c = 2 * (idx & 63);
+      gat(i, c) = tmp[2 * u];
+      gat(i, c + 1) = tmp[2 * u + 1];
+    }
+  } else {
     float tmp[C * D / NTB];
     const int cnt = (gk == D) ? C * D / NTB : (tid < C ? 1 : 0);
 #pragma unroll
@@ -287,7 +395,7 @@ __global__ void __launch_bounds__(NTB, 1)
       if (u < cnt) {
         const int idx = tid + u * NTB;
         const int i = (gk == D) ? idx >> 7 : idx, c = (gk == D) ? idx & 127 : 0;
-        tmp[u] = __expf(gat(i, c) - gat(r, c));
+        tmp[u] = __expf(gat(i, c) - gat(i < 32 ? kRho0 : kRho1, c));
       }
     }
     __syncthreads();
@@ -300,35 +408,92 @@ __global__ void __launch_bounds__(NTB, 1)
       }
     }
   }
-  __syncthreads();
-  // e^{gamma - gamma_r} at (i, c), (i, c + 1), c even
+  // factor u at (i, c), (i, c + 1), c even (phase gate: the pair's complex u)
   auto ep2 = [&](int i, int c) -> float2 {
     if (gk == D) return *reinterpret_cast<const float2*>(s.G + gsw(i, c));
     const float x = s.G[i];
     return make_float2(x, x);
   };
-  // e^{gamma - gamma_r} at (i, c .. c + 3), c a multiple of 4
   auto ep4 = [&](int i, int c) -> float4 {
     if (gk == D) return *reinterpret_cast<const float4*>(s.G + gsw(i, c));
     const float x = s.G[i];
     return make_float4(x, x, x, x);
   };
-  // raw keys (i, c), (i, c + 1)
+  // raw keys / queries (i, c), (i, c + 1)
   auto k2 = [&](int i, int c) -> float2 {
     return frag::unpack(*reinterpret_cast<const uint32_t*>(s.k + i * LDD + c));
   };
-
-  // ---- build: Q^c = q e^{gamma - gamma_r} into the core-tiled operand tile
-  for (int idx = tid; idx < C * (D / 8); idx += NTB) {
+  auto q2 = [&](int i, int c) -> float2 {
+    return frag::unpack(*reinterpret_cast<const uint32_t*>(s.QR + i * LDD + c));
+  };
+  // Level-4 key/query tiles for the 8 channels c .. c + 7 of row i.  first: the
+  // tiles built under level 3 (write keys of both references, queries, and the
+  // beta keys of the second half); otherwise the beta keys of the first reference.
+  auto build_row = [&](int idx, bool first) {
     const int i = ct_row(idx, D), c = ct_col(idx, D);
+    const uint4 rk = *reinterpret_cast<const uint4*>(s.k + i * LDD + c);
     const uint4 rq = *reinterpret_cast<const uint4*>(s.QR + i * LDD + c);
+    const float bi = s.beta[i];
     const float4 f0 = ep4(i, c), f1 = ep4(i, c + 4);
-    const float2 q0 = frag::unpack(rq.x), q1 = frag::unpack(rq.y);
-    const float2 q2 = frag::unpack(rq.z), q3 = frag::unpack(rq.w);
-    *reinterpret_cast<uint4*>(s.QC + 8 * idx) =
-        make_uint4(frag::pack(q0.x * f0.x, q0.y * f0.y), frag::pack(q1.x * f0.z, q1.y * f0.w),
-                   frag::pack(q2.x * f1.x, q2.y * f1.y), frag::pack(q3.x * f1.z, q3.y * f1.w));
-  }
+    const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+    const uint32_t* wk = reinterpret_cast<const uint32_t*>(&rk);
+    const uint32_t* wq = reinterpret_cast<const uint32_t*>(&rq);
+    const bool h1 = i >= 32;
+    uint32_t okb[4], okbx[4], oq[4], oqx[4], obk[4], obkx[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 kk = frag::unpack(wk[e]), qq = frag::unpack(wq[e]);
+      const int cc = c + 2 * e;
+      float kb0, kb1, qf0, qf1, bk0, bk1, kbx0, kbx1, qx0, qx1, bkx0, bkx1;
+      if (PHASE) {
+        const cf uu{f[2 * e], f[2 * e + 1]}, kc{kk.x, kk.y}, qc{qq.x, qq.y};
+        const cf xk0{s.xk[cc], s.xk[cc + 1]}, xk1{s.xk[D + cc], s.xk[D + cc + 1]};
+        const cf xq0{s.xq[cc], s.xq[cc + 1]}, xq1{s.xq[D + cc], s.xq[D + cc + 1]};
+        const cf kb = cmul(kc, cconj(cinv(uu)));   // k / conj(u)
+        const cf qf = cmul(uu, qc), bk = cmul(uu, kc);
+        const cf kbx = cmul(cmul(kb, xk0), xk1), qx = cmul(cmul(qf, xq0), xq1);
+        const cf bkx = cmul(cmul(bk, xq0), xq1);
+        kb0 = kb.x, kb1 = kb.y, qf0 = qf.x, qf1 = qf.y, bk0 = bi * bk.x, bk1 = bi * bk.y;
+        kbx0 = kbx.x, kbx1 = kbx.y, qx0 = qx.x, qx1 = qx.y, bkx0 = bi * bkx.x, bkx1 = bi * bkx.y;
+      } else {
+        kb0 = __fdividef(kk.x, f[2 * e]), kb1 = __fdividef(kk.y, f[2 * e + 1]);
+        qf0 = qq.x * f[2 * e], qf1 = qq.y * f[2 * e + 1];
+        bk0 = bi * kk.x * f[2 * e], bk1 = bi * kk.y * f[2 * e + 1];
+        kbx0 = kb0 * s.xk[cc] * s.xk[D + cc], kbx1 = kb1 * s.xk[cc + 1] * s.xk[D + cc + 1];
+        qx0 = qf0 * s.xq[cc] * s.xq[D + cc], qx1 = qf1 * s.xq[cc + 1] * s.xq[D + cc + 1];
+        bkx0 = bk0 * s.xq[cc] * s.xq[D + cc], bkx1 = bk1 * s.xq[cc + 1] * s.xq[D + cc + 1];
+      }
+      okb[e] = frag::pack(kb0, kb1);
+      okbx[e] = frag::pack(kbx0, kbx1);
+      oq[e] = frag::pack(qf0, qf1);
+      oqx[e] = frag::pack(qx0, qx1);
+      obk[e] = frag::pack(bk0, bk1);
+      obkx[e] = frag::pack(bkx0, bkx1);
+    }
+    const uint4 vkb = make_uint4(okb[0], okb[1], okb[2], okb[3]);
+    const uint4 vkbx = make_uint4(okbx[0], okbx[1], okbx[2], okbx[3]);
+    const uint4 vq = make_uint4(oq[0], oq[1], oq[2], oq[3]);
+    const uint4 vqx = make_uint4(oqx[0], oqx[1], oqx[2], oqx[3]);
+    const uint4 vbk = make_uint4(obk[0], obk[1], obk[2], obk[3]);
+    const uint4 vbkx = make_uint4(obkx[0], obkx[1], obkx[2], obkx[3]);
+    // core-tiled offset of row i (idx) and of row i - 32 in a 32-row tile
+    const int o = 8 * idx, o32 = 8 * idx - 32 * D;
+    if (first) {
+      if (!h1) {
+        *reinterpret_cast<uint4*>(Kb0 + o) = vkb;
+        *reinterpret_cast<uint4*>(Kb1 + o) = vkbx;
+        *reinterpret_cast<uint4*>(Q0 + o) = vq;
+      } else {
+        *reinterpret_cast<uint4*>(Kb1 + o) = vkb;
+        *reinterpret_cast<uint4*>(Q0 + o) = vqx;
+        *reinterpret_cast<uint4*>(Q1 + o32) = vq;
+        *reinterpret_cast<uint4*>(B1 + o32) = vbk;
+      }
+    } else {
+      *reinterpret_cast<uint4*>(B0 + o) = h1 ? vbkx : vbk;
+    }
+  };
+
   frag::cp_wait<0>();
   tc::fence_smem_to_async();
   tc::fence_before_sync();
@@ -347,17 +512,28 @@ __global__ void __launch_bounds__(NTB, 1)
   }
 
   // ---- level 1 (tensor memory): dQs = dO S, dW' = dU S, dKt = U dS', dM = dO U^T
+  // (descriptors are built once; a k-step adds its byte offset / 16 to the start
+  // address field, which stays below 2^14 for any shared-memory address)
   if (tid == 0) {
-    const Chain cs[4] = {chain(tb + T_ZQ, s.DO, false, D, s.SS, true, D, 128, 0, 1, D / 16),
-                         chain(tb + T_ADW, s.DU, false, D, s.SS, true, D, 128, 0, 1, D / 16),
-                         chain(tb + T_AKT, s.UU, false, D, s.SD, true, D, 128, 0, 1, D / 16),
-                         chain(tb + T_ADM, s.DO, false, D, s.UU, false, D, 64, 0, 1, D / 16)};
-    issue_chains(cs);
+    const uint32_t id128 = tc::idesc_bf16(64, 128, false, true);
+    const uint32_t id64 = tc::idesc_bf16(64, 64, false, false);
+    const uint64_t aDO = tc::sdesc_kmaj(s.DO, D, 0), aDU = tc::sdesc_kmaj(s.DU, D, 0);
+    const uint64_t aUU = tc::sdesc_kmaj(s.UU, D, 0);
+    const uint64_t bSS = tc::sdesc_mnmaj(s.SS, D, 0), bSD = tc::sdesc_mnmaj(s.SD, D, 0);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const uint32_t acc = ks > 0 ? 1u : 0u;
+      const uint64_t ka = 16u * ks, kb = 256u * ks;  // K-major / MN-major k-step, 16-byte units
+      mma_step(tb + T_ZQ, aDO + ka, bSS + kb, id128, acc);
+      mma_step(tb + T_ADW, aDU + ka, bSS + kb, id128, acc);
+      mma_step(tb + T_AKT, aUU + ka, bSD + kb, id128, acc);
+      mma_step(tb + T_ADM, aDO + ka, aUU + ka, id64, acc);
+    }
     tc::commit(&s.bar);
   }
-  // colsum(dS' .* S) while they run: thread -> 8 columns (16-byte core rows),
-  // 4 rows (one per row group of its quarter); eight lanes read the eight rows
-  // of one core matrix (128 contiguous bytes, no bank conflicts)
+  // colsum(conj(dS') S) while they run (real gates: per channel sum of dS' .* S):
+  // thread -> 8 columns (16-byte core rows), 4 rows (one per row group of its
+  // quarter); eight lanes read the eight rows of one core matrix
   {
     const int alo = tid & 7, cg = (tid >> 3) & 15, ag = tid >> 7;
     float acc[8] = {};
@@ -371,8 +547,13 @@ __global__ void __launch_bounds__(NTB, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 fx = frag::unpack(wx[e]), fy = frag::unpack(wy[e]);
-        acc[2 * e] += fx.x * fy.x;
-        acc[2 * e + 1] += fx.y * fy.y;
+        if (PHASE) {  // conj(dS') S of the pair: (dx sx + dy sy) + i (dx sy - dy sx)
+          acc[2 * e] += fy.x * fx.x + fy.y * fx.y;
+          acc[2 * e + 1] += fy.x * fx.y - fy.y * fx.x;
+        } else {
+          acc[2 * e] += fx.x * fy.x;
+          acc[2 * e + 1] += fx.y * fy.y;
+        }
       }
     }
 #pragma unroll
@@ -399,7 +580,8 @@ __global__ void __launch_bounds__(NTB, 1)
   frag_ld4(tb + T_ADW + 32 * qt, warp, adw);
   frag_ld4(tb + T_AKT + 32 * qt, warp, akt);
   frag_ld2(tb + T_ADM + 16 * qt, warp, adm);
-  // dW = -dW', dM masked (inclusive lower), stored for the later phases
+  // dW = -dW', and dM masked (inclusive lower) into its X tile (rows of the
+  // second half 4 KB further on, after the zero block written here)
   {
 #pragma unroll
     for (int j = 0; j < 4; ++j)
@@ -411,9 +593,12 @@ __global__ void __launch_bounds__(NTB, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int i = rb * 16 + lr + (e >> 1) * 8, jj = qt * 16 + jt * 8 + lc + (e & 1);
-        if (jj > i) adm[jt][e] = 0.f;
+        if (jj == i) s.dmd[i] = adm[jt][e];
+        if (jj >= i) adm[jt][e] = 0.f;
       }
-    frag::st_c(adm, sdM, -C, rb * 16, qt * 16);
+    frag::st_c(adm, XM, -C, rb * 16 + (hf ? 32 : 0), qt * 16);
+    if (tid < C * C / 16)
+      *reinterpret_cast<uint4*>(XM + C * C / 2 + 8 * tid) = make_uint4(0, 0, 0, 0);
   }
   tc::fence_smem_to_async();
   tc::fence_before_sync();
@@ -421,25 +606,33 @@ __global__ void __launch_bounds__(NTB, 1)
   tc::fence_after_sync();
   // ---- level 2: Lambda = T^T [dU | dW]; dv = diag(beta) Lambda_U (runs under the dKt pass)
   if (tid == 0) {
-    const Chain cs[2] = {chain(tb + T_LU, s.TT, true, C, s.DU, true, D, 128, 0, 1, C / 16),
-                         chain(tb + T_LW, s.TT, true, C, sdW, true, D, 128, 0, 1, C / 16)};
-    issue_chains(cs);
+    const uint32_t id = tc::idesc_bf16(64, 128, true, true);
+    const uint64_t aT = tc::sdesc_mnmaj(s.TT, C, 0);
+    const uint64_t bU = tc::sdesc_mnmaj(s.DU, D, 0), bW = tc::sdesc_mnmaj(sdW, D, 0);
+#pragma unroll
+    for (int ks = 0; ks < C / 16; ++ks) {
+      const uint32_t acc = ks > 0 ? 1u : 0u;
+      mma_step(tb + T_LU, aT + 128u * ks, bU + 256u * ks, id, acc);
+      mma_step(tb + T_LW, aT + 128u * ks, bW + 256u * ks, id, acc);
+    }
     tc::commit(&s.bar);
   }
 
   // The per-element epilogue works on three accumulators at this thread's
-  // fragment positions (rows i0, i0 + 8; key columns c), with ep = e^{gamma - gamma_r}:
-  //   Z = e^{gamma_r} dQs + dM Kb^c                               -> dq = ep Z
-  //   P = e^{gamma_C - gamma_r} dKt + dM^T Q^c + dA^T diag(beta) K^c
-  //   Q = e^{gamma_r} Lambda_W + dA Kb^c
-  // so that dk = P / ep + beta ep Q,  dgamma = k (beta ep Q - P / ep) + Q^c Z
-  // and d(beta_eff) = Lambda_U . v + k . (ep Q) summed over the row.
+  // fragment positions (rows i0, i0 + 8 of half hf; key columns c, c + 1, one
+  // pair), with u the row's factor relative to its half's reference rho:
+  //   Z = conj(zeta_rho) dQs + F1                  -> dq = conj(u) Z
+  //   P = (zeta_C / zeta_rho) dKt + G              -> t2 = P / u
+  //   Q = conj(zeta_rho) Lambda_W + F2             -> t1 = conj(u) Q
+  // so that dk = beta t1 + t2, d(beta) = Lambda_U . v + k . t1, and, with
+  // E1 = conj(dq) q + beta conj(t1) k, E2 = conj(t2) k: dg = Re(E1 - E2) (real
+  // gates: q dq + k (beta t1 - t2)) and d Theta = Im(E1 + E2).
   const int i0 = rb * 16 + lr;
   const size_t rowg[2] = {row_id(p, b, t0 + min(i0, nvalid - 1), h) * D,
                           row_id(p, b, t0 + min(i0 + 8, nvalid - 1), h) * D};
   float(&Z)[4][4] = zq;
   float(&P)[4][4] = akt;
-  // colsum(Kt .* dKt) for the chunk-end gate term, then the column scalings
+  // colsum(conj(dKt) K~) for the chunk-end gate term, then the reference scalings
   {
     float cs[4][2] = {};
 #pragma unroll
@@ -448,25 +641,49 @@ __global__ void __launch_bounds__(NTB, 1)
       for (int hh = 0; hh < 2; ++hh) {
         const int i = i0 + hh * 8, c = qt * 32 + jt * 8 + lc;
         const float2 kk = k2(i, c), f = ep2(i, c);
-        cs[jt][0] += kk.x * __fdividef(akt[jt][2 * hh], f.x);
-        cs[jt][1] += kk.y * __fdividef(akt[jt][2 * hh + 1], f.y);
+        if (PHASE) {  // conj(dKt) (k / conj(u))
+          const cf kb = cmul(cf{kk.x, kk.y}, cconj(cinv(cf{f.x, f.y})));
+          const cf t = cmulc(cf{akt[jt][2 * hh], akt[jt][2 * hh + 1]}, kb);
+          cs[jt][0] += t.x;
+          cs[jt][1] += t.y;
+        } else {
+          cs[jt][0] += kk.x * __fdividef(akt[jt][2 * hh], f.x);
+          cs[jt][1] += kk.y * __fdividef(akt[jt][2 * hh + 1], f.y);
+        }
       }
 #pragma unroll
-    for (int jt = 0; jt < 4; ++jt)
+    for (int jt = 0; jt < 4; ++jt) {
+      const int c = qt * 32 + jt * 8 + lc;
+      const float2 fr = *reinterpret_cast<const float2*>(s.er + hf * D + c);
+      const float2 frc = *reinterpret_cast<const float2*>(s.erc + hf * D + c);
+      float x[2];
+      if (PHASE) {  // K~ = conj(zeta_C / zeta_rho) (k / conj(u))
+        const cf t = cmulc(cf{frc.x, frc.y}, cf{cs[jt][0], cs[jt][1]});
+        x[0] = t.x, x[1] = t.y;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const cf z = cmul(cf{fr.x, fr.y}, cf{Z[jt][2 * hh], Z[jt][2 * hh + 1]});
+          const cf pp = cmul(cf{frc.x, frc.y}, cf{P[jt][2 * hh], P[jt][2 * hh + 1]});
+          Z[jt][2 * hh] = z.x, Z[jt][2 * hh + 1] = z.y;
+          P[jt][2 * hh] = pp.x, P[jt][2 * hh + 1] = pp.y;
+        }
+      } else {
+        x[0] = cs[jt][0] * frc.x, x[1] = cs[jt][1] * frc.y;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          Z[jt][2 * hh] *= fr.x, Z[jt][2 * hh + 1] *= fr.y;
+          P[jt][2 * hh] *= frc.x, P[jt][2 * hh + 1] *= frc.y;
+        }
+      }
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int c = qt * 32 + jt * 8 + lc + u;
-        const float fr = s.er[c], frc = s.erc[c];
-        float x = cs[jt][u] * frc;
-        x += __shfl_xor_sync(0xffffffffu, x, 4);
-        x += __shfl_xor_sync(0xffffffffu, x, 8);
-        x += __shfl_xor_sync(0xffffffffu, x, 16);
-        if (lr == 0) s.ktk[rb * D + c] = x;
-        Z[jt][u] *= fr;
-        Z[jt][2 + u] *= fr;
-        P[jt][u] *= frc;
-        P[jt][2 + u] *= frc;
+        float y = x[u];
+        y += __shfl_xor_sync(0xffffffffu, y, 4);
+        y += __shfl_xor_sync(0xffffffffu, y, 8);
+        y += __shfl_xor_sync(0xffffffffu, y, 16);
+        if (lr == 0) s.ktk[rb * D + c + u] = y;
       }
+    }
   }
   float dbrow[2] = {0.f, 0.f};  // this thread's d(beta_eff) partials for rows i0, i0 + 8
   float Q[4][4];
@@ -497,13 +714,18 @@ __global__ void __launch_bounds__(NTB, 1)
     frag_ld4(tb + T_LW + 32 * qt, warp, Q);
     frag::st_c(Q, sLW, -D, rb * 16, qt * 32);
 #pragma unroll
-    for (int jt = 0; jt < 4; ++jt)
+    for (int jt = 0; jt < 4; ++jt) {
+      const float2 fr = *reinterpret_cast<const float2*>(s.er + hf * D + qt * 32 + jt * 8 + lc);
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const float fr = s.er[qt * 32 + jt * 8 + lc + u];
-        Q[jt][u] *= fr;
-        Q[jt][2 + u] *= fr;
+      for (int hh = 0; hh < 2; ++hh) {
+        if (PHASE) {
+          const cf z = cmul(cf{fr.x, fr.y}, cf{Q[jt][2 * hh], Q[jt][2 * hh + 1]});
+          Q[jt][2 * hh] = z.x, Q[jt][2 * hh + 1] = z.y;
+        } else {
+          Q[jt][2 * hh] *= fr.x, Q[jt][2 * hh + 1] *= fr.y;
+        }
       }
+    }
   }
   __syncthreads();
 
@@ -513,32 +735,46 @@ __global__ void __launch_bounds__(NTB, 1)
   __syncthreads();
   tc::fence_after_sync();
 
-  // ---- level 3: dA = -strict_tril(Lambda_U U'^T + Lambda_W W^T), rows 16rb.., cols 16qt..
+  // ---- level 3: dA = -strict_tril(Lambda_U U'^T + Lambda_W W^T): four partial sums
   if (tid == 0) {
-    const Chain cs[4] = {chain(tb + T_DA, sLU, false, D, sUp, false, D, 64, 0, 2, D / 32),
-                         chain(tb + T_DA + 64, sLU, false, D, sUp, false, D, 64, 1, 2, D / 32),
-                         chain(tb + T_DA + 128, sLW, false, D, sW, false, D, 64, 0, 2, D / 32),
-                         chain(tb + T_DA + 192, sLW, false, D, sW, false, D, 64, 1, 2, D / 32)};
-    issue_chains(cs);
+    const uint32_t id = tc::idesc_bf16(64, 64, false, false);
+    const uint64_t aLU = tc::sdesc_kmaj(sLU, D, 0), aLW = tc::sdesc_kmaj(sLW, D, 0);
+    const uint64_t bUp = tc::sdesc_kmaj(sUp, D, 0), bW = tc::sdesc_kmaj(sW, D, 0);
+#pragma unroll
+    for (int j = 0; j < D / 32; ++j)
+#pragma unroll
+      for (int part = 0; part < 4; ++part) {
+        const uint64_t ko = 16u * (2 * j + (part & 1));
+        mma_step(tb + T_DA + 64 * part, (part < 2 ? aLU : aLW) + ko, (part < 2 ? bUp : bW) + ko,
+                 id, j > 0 ? 1u : 0u);
+      }
     tc::commit(&s.bar);
   }
-  // ---- under level 3: Kb^c and beta K^c into the core-tiled operand tiles (dU, dW slots)
-  for (int idx = tid; idx < C * (D / 8); idx += NTB) {
-    const int i = ct_row(idx, D), c = ct_col(idx, D);
-    const uint4 rk = *reinterpret_cast<const uint4*>(s.k + i * LDD + c);
-    const float bi = s.beta[i];
-    const float4 f0 = ep4(i, c), f1 = ep4(i, c + 4);
-    const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-    const uint32_t* wk = reinterpret_cast<const uint32_t*>(&rk);
-    uint32_t okb[4], obc[4];
+  // ---- under level 3: the dA-free level-4 operands, then their products
+  //      F1 = dM Kb (per-half references) and the dM half of G for the first half
+  for (int idx = tid; idx < C * (D / 8); idx += NTB) build_row(idx, true);
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t idF = tc::idesc_bf16(64, 128, false, true);
+  const uint32_t idG = tc::idesc_bf16(64, 128, true, true);
+  // level-4 descriptors (k-step offsets in 16-byte units are added below)
+  const uint64_t xmK = dk64(XM, 0), xaK = dk64(XA, 0), xmT = dmn64(XM, 0), xaT = dmn64(XA, 0);
+  const uint64_t dKb0 = dmn128(Kb0, 0), dKb1 = dmn128(Kb1, 0), dQ0 = dmn128(Q0, 0);
+  const uint64_t dQ1 = dmn128(Q1, 0), dB0 = dmn128(B0, 0), dB1 = dmn128(B1, 0);
+  if (tid == 0) {
+    // F1: rows of the first half against Kb^{rho0} (k-steps 0, 1), rows of the
+    // second half against Kb^{rho1} (k-steps 0..3); one accumulator
+    mma_step(tb + T_F1, xmK, dKb0, idF, 0u);
+    mma_step(tb + T_G0, xmT + xt_off(0) / 16, dQ0, idG, 0u);
+    mma_step(tb + T_F1, xmK + 16, dKb0 + 256, idF, 1u);
+    mma_step(tb + T_G0, xmT + xt_off(1) / 16, dQ0 + 256, idG, 1u);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 kk = frag::unpack(wk[e]);
-      okb[e] = frag::pack(__fdividef(kk.x, f[2 * e]), __fdividef(kk.y, f[2 * e + 1]));
-      obc[e] = frag::pack(bi * kk.x * f[2 * e], bi * kk.y * f[2 * e + 1]);
+    for (int ks = 0; ks < 4; ++ks) {
+      mma_step(tb + T_F1, xmK + 256 + 16 * ks, dKb1 + 256 * ks, idF, 1u);
+      if (ks >= 2) mma_step(tb + T_G0, xmT + xt_off(ks) / 16, dQ0 + 256 * ks, idG, 1u);
     }
-    *reinterpret_cast<uint4*>(sKb + 8 * idx) = make_uint4(okb[0], okb[1], okb[2], okb[3]);
-    *reinterpret_cast<uint4*>(sBk + 8 * idx) = make_uint4(obc[0], obc[1], obc[2], obc[3]);
   }
   ok = hy_wait(&s.bar, 2);
   if (!ok) break;
@@ -560,42 +796,47 @@ __global__ void __launch_bounds__(NTB, 1)
         const int i = rb * 16 + lr + (e >> 1) * 8, jj = qt * 16 + jt * 8 + lc + (e & 1);
         da[jt][e] = (jj < i) ? -da[jt][e] : 0.f;
       }
-    frag::st_c(da, sdA, -C, rb * 16, qt * 16);
+    frag::st_c(da, XA, -C, rb * 16 + (hf ? 32 : 0), qt * 16);
   }
-
+  // beta k of the first reference into the Lambda tiles (level 3 has read them)
+  for (int idx = tid; idx < C * (D / 8); idx += NTB) build_row(idx, false);
   tc::fence_smem_to_async();
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  // ---- level 4: dM Kb^c, dA Kb^c, dM^T Q^c + dA^T beta K^c
+  // ---- level 4, dA part: F2 = dA Kb; G += dA^T beta k (first half); G of the second half
   if (tid == 0) {
-    const Chain cs[4] = {chain(tb + T_Z2, sdM, false, C, sKb, true, D, 128, 0, 1, C / 16),
-                         chain(tb + T_X, sdA, false, C, sKb, true, D, 128, 0, 1, C / 16),
-                         chain(tb + T_Y, sdM, true, C, s.QC, true, D, 128, 0, 1, C / 16),
-                         chain(tb + T_Y2, sdA, true, C, sBk, true, D, 128, 0, 1, C / 16)};
-    issue_chains(cs);
+    mma_step(tb + T_F2, xaK, dKb0, idF, 0u);
+    mma_step(tb + T_G1, xmT + xt_off(2) / 16, dQ1, idG, 0u);
+    mma_step(tb + T_G0, xaT + xt_off(0) / 16, dB0, idG, 1u);
+    mma_step(tb + T_F2, xaK + 16, dKb0 + 256, idF, 1u);
+    mma_step(tb + T_G1, xmT + xt_off(3) / 16, dQ1 + 256, idG, 1u);
+    mma_step(tb + T_G0, xaT + xt_off(1) / 16, dB0 + 256, idG, 1u);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      mma_step(tb + T_F2, xaK + 256 + 16 * ks, dKb1 + 256 * ks, idF, 1u);
+      if (ks >= 2) {
+        mma_step(tb + T_G0, xaT + xt_off(ks) / 16, dB0 + 256 * ks, idG, 1u);
+        mma_step(tb + T_G1, xaT + xt_off(ks) / 16, dB1 + 256 * (ks - 2), idG, 1u);
+      }
+    }
     tc::commit(&s.bar);
   }
   ok = hy_wait(&s.bar, 3);
   if (!ok) break;
   {
     float t4[4][4];
-    frag_ld4(tb + T_Z2 + 32 * qt, warp, t4);
+    frag_ld4(tb + T_F1 + 32 * qt, warp, t4);
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) Z[j][e] += t4[j][e];
-    frag_ld4(tb + T_X + 32 * qt, warp, t4);
+    frag_ld4(tb + T_F2 + 32 * qt, warp, t4);
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) Q[j][e] += t4[j][e];
-    frag_ld4(tb + T_Y + 32 * qt, warp, t4);
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) P[j][e] += t4[j][e];
-    frag_ld4(tb + T_Y2 + 32 * qt, warp, t4);
+    frag_ld4(tb + (hf ? T_G1 : T_G0) + 32 * qt, warp, t4);
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -609,30 +850,61 @@ __global__ void __launch_bounds__(NTB, 1)
     for (int hh = 0; hh < 2; ++hh) {
       const int i = i0 + hh * 8, c = qt * 32 + jt * 8 + lc;
       const float bi = s.beta[i];
-      const float2 kk = k2(i, c);
-      const float2 qc = frag::unpack(*reinterpret_cast<const uint32_t*>(s.QC + ct_off(i, c, D)));
-      const float2 f = ep2(i, c);
-      float outq[2];
+      const float2 kk = k2(i, c), qq = q2(i, c), f = ep2(i, c);
+      const int e0 = 2 * hh, e1 = 2 * hh + 1;
+      // the diagonal of dM enters dq and t2 with the factor 1 and cancels in dg
+      // exactly, so it is kept out of the bf16 products and of dg
+      const float dmi = s.dmd[i];
+      float dqo[2], dko[2], dgo[2];
+      if (PHASE) {
+        const cf uu{f.x, f.y}, kc{kk.x, kk.y}, qc{qq.x, qq.y};
+        const cf dqc = cmulc(uu, cf{Z[jt][e0], Z[jt][e1]});   // conj(u) Z
+        const cf t1 = cmulc(uu, cf{Q[jt][e0], Q[jt][e1]});    // conj(u) Q
+        const cf t2 = cmul(cf{P[jt][e0], P[jt][e1]}, cinv(uu));  // P / u
+        const cf a1 = cmulc(dqc, qc), a2 = cmulc(t1, kc), a3 = cmulc(t2, kc);
+        dgo[0] = a1.x + bi * a2.x - a3.x;  // Re(E1 - E2)
+        dgo[1] = a1.y + bi * a2.y + a3.y;  // Im(E1 + E2)
+        dqo[0] = dqc.x + dmi * kc.x, dqo[1] = dqc.y + dmi * kc.y;
+        dko[0] = bi * t1.x + t2.x + dmi * qc.x, dko[1] = bi * t1.y + t2.y + dmi * qc.y;
+        dbrow[hh] += kc.x * t1.x + kc.y * t1.y;
+      } else {
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int e = 2 * hh + u;
-        const float ep = u ? f.y : f.x;
-        const float t1 = ep * Q[jt][e], t2 = __fdividef(P[jt][e], ep);
-        const float kv = u ? kk.y : kk.x, qv = u ? qc.y : qc.x;
-        float dgv = kv * (bi * t1 - t2) + qv * Z[jt][e];
-        if (i == C - 1) {  // chunk-end gate term: colsum(Kt .* dKt) + e^{gamma_C} colsum(dS' .* S)
-          const int cc = c + u;
-          const float eC = s.er[cc] * s.erc[cc];
-          dgv += s.ktk[cc] + s.ktk[D + cc] + s.ktk[2 * D + cc] + s.ktk[3 * D + cc] +
-                 eC * (s.dgc[cc] + s.dgc[D + cc] + s.dgc[2 * D + cc] + s.dgc[3 * D + cc]);
+        for (int u = 0; u < 2; ++u) {
+          const int e = 2 * hh + u;
+          const float ep = u ? f.y : f.x, kv = u ? kk.y : kk.x, qv = u ? qq.y : qq.x;
+          const float t1 = ep * Q[jt][e], t2 = __fdividef(P[jt][e], ep);
+          const float dqs = ep * Z[jt][e];
+          dgo[u] = qv * dqs + kv * (bi * t1 - t2);
+          dqo[u] = dqs + dmi * kv;
+          dko[u] = bi * t1 + t2 + dmi * qv;
+          dbrow[hh] += kv * t1;
         }
-        dbrow[hh] += kv * t1;
-        outq[u] = ep * Z[jt][e];
-        P[jt][e] = bi * t1 + t2;
-        Q[jt][e] = dgv;
+      }
+      if (i == C - 1) {
+        // chunk-end gate term: colsum(conj(dKt) K~) + conj(zeta_C) colsum(conj(dS') S)
+        float kt[2], gs[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int cc = c + u;
+          kt[u] = s.ktk[cc] + s.ktk[D + cc] + s.ktk[2 * D + cc] + s.ktk[3 * D + cc];
+          gs[u] = s.dgc[cc] + s.dgc[D + cc] + s.dgc[2 * D + cc] + s.dgc[3 * D + cc];
+        }
+        const float2 fr = *reinterpret_cast<const float2*>(s.er + D + c);
+        const float2 frc = *reinterpret_cast<const float2*>(s.erc + D + c);
+        if (PHASE) {
+          const cf dec = cmul(cf{fr.x, fr.y}, cconj(cf{frc.x, frc.y}));  // conj(zeta_C)
+          const cf ps = cmul(dec, cf{gs[0], gs[1]});
+          dgo[0] += kt[0] + ps.x;
+          dgo[1] -= kt[1] + ps.y;
+        } else {
+          dgo[0] += kt[0] + fr.x * frc.x * gs[0];
+          dgo[1] += kt[1] + fr.y * frc.y * gs[1];
+        }
       }
       if (i < nvalid)
-        *reinterpret_cast<uint32_t*>(dq + rowg[hh] + c) = frag::pack(outq[0], outq[1]);
+        *reinterpret_cast<uint32_t*>(dq + rowg[hh] + c) = frag::pack(dqo[0], dqo[1]);
+      P[jt][e0] = dko[0], P[jt][e1] = dko[1];
+      Q[jt][e0] = dgo[0], Q[jt][e1] = dgo[1];
     }
   // d(beta_eff) partials: reduce the 4 lanes that share a row, one slot per column quarter
 #pragma unroll
@@ -696,7 +968,7 @@ __global__ void __launch_bounds__(NTB, 1)
   // dgamma: reverse cumulative sum over the chunk's rows
   if (gk == D) {
     float run = 0.f;
-    for (int q2 = grq + 1; q2 < 4; ++q2) run += s.dgc[q2 * D + gc];
+    for (int q2i = grq + 1; q2i < 4; ++q2i) run += s.dgc[q2i * D + gc];
 #pragma unroll 4
     for (int i = grq * 16 + 15; i >= grq * 16; --i) {
       run += sdg[i * LDG + gc];
@@ -718,7 +990,7 @@ __global__ void __launch_bounds__(NTB, 1)
   }
   } while (0);
   if (!ok) {
-    // a bounded wait gave up: record it and drain the copies in flight
+    // a bounded wait gave up: record it and let the copies in flight land
     if (tid == 0 && err) atomicExch(err, 1);
     frag::cp_wait<0>();
   }
@@ -734,18 +1006,21 @@ cudaError_t launch_bwd_chunk_hy(const Problem& p, const bf16* q, const bf16* k, 
                                 const bf16* dU, bf16* dq, bf16* dk, bf16* dv, float* dbeta,
                                 float* dg, cudaStream_t st) {
   const size_t sm = sizeof(HySmem) + 1024;
-  cudaError_t e =
-      cudaFuncSetAttribute(k_bwd_chunk_hy, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  const bool phase = p.gate == kGatePhase;
+  auto kern = phase ? k_bwd_chunk_hy<true> : k_bwd_chunk_hy<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const double nb = (double)p.B * p.H * p.NC, ntok = nb * C;
   // operator I/O: reads q, k, v, dO, g, beta; writes dq, dk, dv, dbeta, dg
   const double io = ntok * (4 * D * 2 + p.gk * 4 + 4) + ntok * (3 * D * 2 + p.gk * 4 + 4);
   // and by design the chunk tiles T, h, dh, U, dU, W, U' (and beta, ||k||^2 from the saved set)
   const double bytes = io + nb * C * C * 2 + nb * 2.0 * D * D * 2 + ntok * 4 * D * 2 + ntok * 4;
-  const double mac = (double)C * D * D * 3 + (double)C * C * D + (double)C * D * C * 2 +
-                     (double)C * C * D * 2 + (double)C * D * C * 4;
+  // level 1: 3 (C x D x D) + C^2 D; level 2: 2 C^2 D; level 3: 2 C^2 D;
+  // level 4 as issued: 24 products of 64 x 16 x 128
+  const double mac = 3.0 * C * D * D + (double)C * C * D + 2.0 * C * C * D + 2.0 * C * C * D +
+                     24.0 * 64 * 16 * 128;
   prof_begin(kKTcChunkBwd, io, bytes, nb * 2.0 * mac, st);
-  k_bwd_chunk_hy<<<dim3(p.NC, p.H, p.B), NTB, sm, st>>>(
+  kern<<<dim3(p.NC, p.H, p.B), NTB, sm, st>>>(
       p, q, k, v, dO, g, sv.T, sv.beta, sv.h, dh, sv.U, dU, sv.W, sv.Up, sv.knorm, dq, dk, dv,
       dbeta, dg, device_error_word(), take_injected_timeout() ? 1 : 0);
   e = cudaGetLastError();

@@ -1,0 +1,580 @@
+// fast_prep.cu -- the intra-chunk forward (WY / UT transform) on tcgen05 tensor
+// cores, fed by TMA (bf16 storage, d_k = d_v = 128, C = 64).
+//
+// One CTA per (b, h, chunk), 256 threads, two CTAs per SM.  Every quantity of
+// the chunk that does not depend on the state, computed once:
+//   g     inclusive within-chunk cumulative log-gate (per key channel; scalar
+//         gates broadcast; zero without a gate)
+//   beta  the write strength (Kaczmarz step beta = eta / (||k||^2 + eps) applied)
+//   A     = diag(beta) strict_tril(G),  M = tril(Gq)  with the gate-scaled Grams
+//         G_ij = sum_c k_ic k_jc e^{g_ic - g_jc},  Gq_ij = sum_c q_ic k_jc e^{g_ic - g_jc}
+//   T     = (I + A)^{-1}, in fp32 by column-parallel forward substitution
+//   W     = T diag(beta) (k e^g),  U' = T diag(beta) v   (T split into two bf16 terms)
+//   Qh    = q e^g,  Kt = k e^{g_C - g},  dec = e^{g_C}
+// and writes them to the saved buffer, core-tiled (8 x 8 blocks of 128
+// contiguous bytes), for the state scans and the backward.  This is the
+// chunk's triangular residual system (I + A)[U' | W] = diag(beta)[V | k e^g]
+// (ReWY abstract; the SFDA explainer's constructive chunk-WY theorem).
+//
+// Grams with per-half reference rows.  Row i of the Grams uses the reference
+// row rho of its own 32-row half (rows 15 and 47):
+//   G_ij = sum_c (k_ic e^{g_ic - g_rho,c}) (k_jc e^{g_rho,c - g_jc}),
+// where the first factor spans at most 16 rows of decay, and the second too for
+// j in the same half, while for j in the earlier half it is at most 1.  So no
+// operand overflows unless the gates decay by more than about 5.5 nats per
+// token over 16 tokens ("centered matrix contractions", ReWY abstract); the
+// first half's rows and the second half's are two tcgen05 products
+// ([K; Q] of the half, M = 64) against their own reference's write keys.
+//
+// PHASE: the SFDA rotation-decay gate ("Semidirect Fourier Delta Attention"
+// explainer, Kernarchitektur).  Key channels pair up as complex numbers; with
+// zeta_i = e^{g_i - i Theta_i} per pair (g, Theta: the cumulative sums at the
+// pair's even and odd channels) the chunk is a plain delta rule with read keys
+// zeta_i k_i, write keys k_i / conj(zeta_i), queries zeta_i q_i and end keys
+// conj(zeta_C / zeta_i) k_i (the explainer's constructive chunk-WY theorem),
+// so every real factor above becomes a per-pair complex one; dec holds
+// conj(zeta_C) per pair.
+//
+// Data movement: q, k, v and a per-channel gate arrive by TMA
+// (cp.async.bulk.tensor, 128-byte swizzled boxes of 64 tokens x 128 bytes, the
+// ragged tail zero-filled as out of bounds); the tcgen05 operands are written
+// core-tiled in place of the tiles they are computed from.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <string.h>
+
+#include <mutex>
+
+#include "dr_common.cuh"
+#include "fast.cuh"
+#include "frag.cuh"
+#include "tc.cuh"
+
+namespace dr {
+namespace fast {
+
+using frag::bf16;
+
+namespace {
+
+constexpr int C = 64, D = 128;
+constexpr int NTP = 256;
+constexpr int kRho0 = 15, kRho1 = 47;  // reference rows of the two halves
+constexpr uint32_t kSpinPrep = 1u << 22;
+constexpr uint32_t kBox = 8192;        // one TMA box: 64 rows x 128 bytes
+
+struct PrepSmem {
+  // TMA destinations (1 KB aligned), reused in place for the tcgen05 operands
+  alignas(1024) unsigned char Q[2 * kBox];  // q; then [K; Q] of the first half (Gram A, K-major)
+  alignas(1024) unsigned char K[2 * kBox];  // k; then [K; Q] of the second half
+  alignas(1024) unsigned char V[2 * kBox];  // v; then beta v (MN-major B of U')
+  alignas(1024) unsigned char G[4 * kBox];  // per-channel gate (fp32, four boxes) -> cumulative;
+                                            // then A^T (fp32 [j][i]) and T hi | lo (bf16)
+  alignas(1024) unsigned char KB[3 * kBox]; // write keys: rho0 rows 0..31 | rho1 rows 0..63;
+                                            // then beta k e^g (MN-major B of W)
+  float ref[3][D];   // cumulative gate at rows rho0, rho1 and C - 1
+  float rot[3][D];   // phase gate: (cos, sin) of the cumulative phase at those rows, per pair
+  float gs[C];       // scalar gate: cumulative per row
+  float eta[C];      // input beta (eta in Kaczmarz mode)
+  float beta[C];     // effective beta
+  uint64_t bar_tma, bar_mma;
+  uint32_t tmem;
+};
+
+// Byte offset of 16-byte chunk ch (0..7) of row r in a 128-byte-swizzled TMA
+// box (chunk index XOR row mod 8 within each 1 KB block).
+__device__ __forceinline__ uint32_t swz(int r, int ch) {
+  return (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4));
+}
+// Byte offset of 16-byte chunk j of row r in a core-tiled [rows][128] bf16 tile.
+__device__ __forceinline__ uint32_t ct16(int r, int j) {
+  return (uint32_t)((((r >> 3) * 16 + j) << 7) + ((r & 7) << 4));
+}
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, int c3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(tc::smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+      "r"(tc::smem_u32(bar))
+      : "memory");
+}
+
+// 32 consecutive fp32 TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+  tc::tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void unpack8(const uint4& r, float* f) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(&r);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 x = frag::unpack(w[e]);
+    f[2 * e] = x.x;
+    f[2 * e + 1] = x.y;
+  }
+}
+__device__ __forceinline__ uint4 pack8(const float* f) {
+  return make_uint4(frag::pack(f[0], f[1]), frag::pack(f[2], f[3]), frag::pack(f[4], f[5]),
+                    frag::pack(f[6], f[7]));
+}
+
+// Bounded wait on an mbarrier phase; CTA-uniform result.
+__device__ __forceinline__ bool prep_wait(uint64_t* bar, int parity) {
+  const bool ok = tc::mbar_wait(bar, (uint32_t)(parity & 1), kSpinPrep);
+  const int bad = __syncthreads_or(ok ? 0 : 1);
+  tc::fence_after_sync();
+  return bad == 0;
+}
+
+template <bool PHASE>
+__global__ void __launch_bounds__(NTP, 2)
+    k_prep_tc(Problem p, const __grid_constant__ CUtensorMap tq,
+              const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+              const __grid_constant__ CUtensorMap tg, const float* __restrict__ g_scalar,
+              const float* __restrict__ beta_in, Saved sv, int* __restrict__ err) {
+  extern __shared__ __align__(1024) unsigned char smraw[];
+  PrepSmem& s = *reinterpret_cast<PrepSmem*>(
+      (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int t0 = n * C, nvalid = min(C, p.T - t0);
+  const size_t cb = chunk_id(p, b, h, n);
+  const bool chan = p.gk == D;  // per-channel (or phase) gate in the G tile
+
+  if (warp == 0) tc::tmem_alloc(&s.tmem, 256);
+  if (tid == 0) {
+    tc::mbar_init(&s.bar_tma, 1);
+    tc::mbar_init(&s.bar_mma, 1);
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    tc::mbar_arrive_expect_tx(&s.bar_tma, 6 * kBox + (chan ? 4 * kBox : 0));
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      tma_load_4d(s.Q + x * kBox, &tq, 64 * x, h, t0, b, &s.bar_tma);
+      tma_load_4d(s.K + x * kBox, &tk, 64 * x, h, t0, b, &s.bar_tma);
+      tma_load_4d(s.V + x * kBox, &tv, 64 * x, h, t0, b, &s.bar_tma);
+    }
+    if (chan) {
+#pragma unroll
+      for (int x = 0; x < 4; ++x) tma_load_4d(s.G + x * kBox, &tg, 32 * x, h, t0, b, &s.bar_tma);
+    }
+  }
+  if (!chan && tid < C)
+    s.gs[tid] = (tid < nvalid && p.gate != kGateNone) ? g_scalar[row_id(p, b, t0 + tid, h)] : 0.f;
+  const float eta = (tid < C && tid < nvalid) ? beta_in[row_id(p, b, t0 + tid, h)] : 0.f;
+  bool ok = prep_wait(&s.bar_tma, 0);
+  const uint32_t tb = s.tmem;
+  do {  // leaves early (break) only when a bounded wait gives up
+  if (!ok) break;
+
+  // ---- cumulative gate down the rows
+  // per-channel element (r, c) of the gate tile: box c / 32, chunk (c % 32) / 4
+  auto gp = [&](int r, int c) -> float* {
+    return reinterpret_cast<float*>(s.G + (c >> 5) * kBox + swz(r, (c & 31) >> 2) + (c & 3) * 4);
+  };
+  if (chan) {
+    const int c = tid & 127, hf = tid >> 7;
+    float run = 0.f;
+#pragma unroll 8
+    for (int r = 32 * hf; r < 32 * hf + 32; ++r) {
+      run += *gp(r, c);
+      *gp(r, c) = run;
+    }
+    __syncthreads();
+    if (hf) {
+      const float off = *gp(31, c);
+#pragma unroll 8
+      for (int r = 32; r < 64; ++r) *gp(r, c) += off;
+    }
+  } else if (warp == 0) {
+    const float a0 = s.gs[2 * lane], a1 = s.gs[2 * lane + 1];
+    float x = a0 + a1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    s.gs[2 * lane + 1] = x;
+    s.gs[2 * lane] = x - a1;
+  }
+  __syncthreads();
+  if (tid < D) {
+    const int rows[3] = {kRho0, kRho1, C - 1};
+#pragma unroll
+    for (int k3 = 0; k3 < 3; ++k3) s.ref[k3][tid] = chan ? *gp(rows[k3], tid) : s.gs[rows[k3]];
+  }
+  __syncthreads();
+  if (PHASE && tid < D / 2) {
+#pragma unroll
+    for (int k3 = 0; k3 < 3; ++k3) {
+      float sn, cs;
+      sincosf(s.ref[k3][2 * tid + 1], &sn, &cs);
+      s.rot[k3][2 * tid] = cs;
+      s.rot[k3][2 * tid + 1] = sn;
+    }
+  }
+  // the chunk decay: e^{g_C} (phase gate: conj(zeta_C) per pair)
+  if (tid < D) {
+    float dv;
+    if (PHASE) {
+      const int c0 = tid & ~1;
+      float sn, cs;
+      sincosf(s.ref[2][c0 + 1], &sn, &cs);
+      dv = __expf(s.ref[2][c0]) * ((tid & 1) ? sn : cs);
+    } else {
+      dv = __expf(s.ref[2][tid]);
+    }
+    sv.dec[cb * D + tid] = dv;
+  }
+
+  // ---- factor pass.  Warp w: rows 8w .. 8w + 7; lane: row 8w + lane % 8 and the
+  // 16-byte chunks j = lane / 8 + 4 it (it = 0..3) of its 128 channels, so that
+  // the swizzled TMA tiles are read and the core-tiled operands written without
+  // bank conflicts.
+  const int r = 8 * warp + (lane & 7), jq = lane >> 3, hr = r >> 5;
+  uint4 qr[4], kr[4], vr[4];
+  float nn = 0.f;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int j = jq + 4 * it;
+    qr[it] = *reinterpret_cast<const uint4*>(s.Q + (j >> 3) * kBox + swz(r, j & 7));
+    kr[it] = *reinterpret_cast<const uint4*>(s.K + (j >> 3) * kBox + swz(r, j & 7));
+    vr[it] = *reinterpret_cast<const uint4*>(s.V + (j >> 3) * kBox + swz(r, j & 7));
+    float kv[8];
+    unpack8(kr[it], kv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) nn += kv[e] * kv[e];
+  }
+  nn += __shfl_xor_sync(0xffffffffu, nn, 8);
+  nn += __shfl_xor_sync(0xffffffffu, nn, 16);
+  if (tid < C) s.eta[tid] = eta;
+  __syncthreads();  // every thread holds its q, k, v: the tiles may be rewritten
+  const float br = (r < nvalid)
+                       ? ((p.beta_mode == kBetaKaczmarz) ? s.eta[r] / (nn + p.eps) : s.eta[r])
+                       : 0.f;
+  if (jq == 0) {
+    sv.beta[cb * C + r] = br;
+    sv.knorm[cb * C + r] = nn;
+  }
+  uint4 bkr[4];  // beta k e^g, held until the write-key tiles are free
+  {
+    unsigned char* GAh = hr ? s.K : s.Q;      // [K; Q] of this row's half
+    const int R = r & 31;                     // row within the half
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int j = jq + 4 * it, c0 = 8 * j;
+      float kv[8], qv[8], vv[8], gg[8];
+      unpack8(kr[it], kv);
+      unpack8(qr[it], qv);
+      unpack8(vr[it], vv);
+      if (chan) {
+        const float4 a = *reinterpret_cast<const float4*>(s.G + (j >> 2) * kBox + swz(r, 2 * (j & 3)));
+        const float4 c4 = *reinterpret_cast<const float4*>(s.G + (j >> 2) * kBox + swz(r, 2 * (j & 3) + 1));
+        gg[0] = a.x, gg[1] = a.y, gg[2] = a.z, gg[3] = a.w;
+        gg[4] = c4.x, gg[5] = c4.y, gg[6] = c4.z, gg[7] = c4.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gg[e] = s.gs[r];
+      }
+      float kc[8], qc[8], kb[8], kb1[8], qh[8], kt[8], bk[8], bv[8];
+      if (PHASE) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int e = 2 * m, cc = c0 + e;
+          float sn, cs;
+          sincosf(gg[e + 1], &sn, &cs);                  // e^{-i Theta} = cs - i sn
+          const float rhc = s.rot[hr][cc], rhs = s.rot[hr][cc + 1];   // e^{i Theta_rho}
+          // w = e^{-i (Theta - Theta_rho)} of this row's reference
+          const float wr = cs * rhc + sn * rhs, wi = cs * rhs - sn * rhc;
+          const float kx = kv[e], ky = kv[e + 1], qx = qv[e], qy = qv[e + 1];
+          const float kwx = wr * kx - wi * ky, kwy = wi * kx + wr * ky;
+          const float qwx = wr * qx - wi * qy, qwy = wi * qx + wr * qy;
+          const float ep = __expf(gg[e] - s.ref[hr][cc]), em = __expf(s.ref[hr][cc] - gg[e]);
+          kc[e] = ep * kwx, kc[e + 1] = ep * kwy;        // u k
+          qc[e] = ep * qwx, qc[e + 1] = ep * qwy;        // u q
+          kb[e] = em * kwx, kb[e + 1] = em * kwy;        // k / conj(u)
+          if (hr == 0) {  // write key of the second half's reference: e^{g_rho1 - g} e^{-i (Theta - Theta_rho1)} k
+            const float r1c = s.rot[1][cc], r1s = s.rot[1][cc + 1];
+            const float xr = cs * r1c + sn * r1s, xi = cs * r1s - sn * r1c;
+            const float e1 = __expf(s.ref[1][cc] - gg[e]);
+            kb1[e] = e1 * (xr * kx - xi * ky), kb1[e + 1] = e1 * (xi * kx + xr * ky);
+          }
+          const float eg = __expf(gg[e]);
+          qh[e] = eg * (cs * qx + sn * qy), qh[e + 1] = eg * (cs * qy - sn * qx);   // zeta q
+          bk[e] = br * eg * (cs * kx + sn * ky), bk[e + 1] = br * eg * (cs * ky - sn * kx);
+          // conj(zeta_C / zeta) k = e^{g_C - g} e^{i (Theta_C - Theta)} k
+          const float tcr = s.rot[2][cc] * cs + s.rot[2][cc + 1] * sn;
+          const float tci = s.rot[2][cc + 1] * cs - s.rot[2][cc] * sn;
+          const float ec = __expf(s.ref[2][cc] - gg[e]);
+          kt[e] = ec * (tcr * kx - tci * ky), kt[e + 1] = ec * (tci * kx + tcr * ky);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int cc = c0 + e;
+          const float d = gg[e] - s.ref[hr][cc];
+          const float ep = __expf(d), em = __expf(-d);
+          kc[e] = kv[e] * ep;
+          qc[e] = qv[e] * ep;
+          kb[e] = kv[e] * em;
+          if (hr == 0) kb1[e] = kv[e] * __expf(s.ref[1][cc] - gg[e]);
+          const float eg = __expf(gg[e]);
+          qh[e] = qv[e] * eg;
+          bk[e] = br * kv[e] * eg;
+          kt[e] = kv[e] * __expf(s.ref[2][cc] - gg[e]);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) bv[e] = br * vv[e];
+      *reinterpret_cast<uint4*>(GAh + ct16(R, j)) = pack8(kc);
+      *reinterpret_cast<uint4*>(GAh + ct16(32 + R, j)) = pack8(qc);
+      if (hr == 0) {
+        *reinterpret_cast<uint4*>(s.KB + ct16(r, j)) = pack8(kb);
+        *reinterpret_cast<uint4*>(s.KB + 4 * 2048 + ct16(r, j)) = pack8(kb1);
+      } else {
+        *reinterpret_cast<uint4*>(s.KB + 4 * 2048 + ct16(r, j)) = pack8(kb);
+      }
+      *reinterpret_cast<uint4*>(s.V + ct16(r, j)) = pack8(bv);
+      *reinterpret_cast<uint4*>(sv.Qh + cb * C * D + ct_off(r, c0, D)) = pack8(qh);
+      *reinterpret_cast<uint4*>(sv.Kt + cb * C * D + ct_off(r, c0, D)) = pack8(kt);
+      bkr[it] = pack8(bk);
+    }
+  }
+  if (jq == 0) s.beta[r] = br;
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+
+  // ---- Grams on tcgen05: D0 = [K; Q]_h0 (Kb^rho0 rows 0..31)^T (M = 64, N = 32)
+  //                        D1 = [K; Q]_h1 (Kb^rho1 rows 0..63)^T (M = 64, N = 64)
+  if (tid == 0) {
+    const uint32_t id0 = tc::idesc_bf16(64, 32, false, false);
+    const uint32_t id1 = tc::idesc_bf16(64, 64, false, false);
+    const uint64_t a0 = tc::sdesc_kmaj(reinterpret_cast<const bf16*>(s.Q), D, 0);
+    const uint64_t a1 = tc::sdesc_kmaj(reinterpret_cast<const bf16*>(s.K), D, 0);
+    const uint64_t b0 = tc::sdesc_kmaj(reinterpret_cast<const bf16*>(s.KB), D, 0);
+    const uint64_t b1 = tc::sdesc_kmaj(reinterpret_cast<const bf16*>(s.KB + 4 * 2048), D, 0);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const uint32_t acc = ks > 0 ? 1u : 0u;
+      tc::mma(tb + 0, a0 + 16u * ks, b0 + 16u * ks, id0, acc);
+      tc::mma(tb + 32, a1 + 16u * ks, b1 + 16u * ks, id1, acc);
+    }
+    tc::commit(&s.bar_mma);
+  }
+  ok = prep_wait(&s.bar_mma, 0);
+  if (!ok) break;
+  // ---- A^T (fp32, [j][i]) into the gate tile's first half; M (bf16) to global.
+  // An M = 64 accumulator: row 16 (warp % 4) + lane for lanes 0..15 of the warp.
+  float* At = reinterpret_cast<float*>(s.G);
+  {
+    const int qd = warp & 3, t = lane;
+    const int row = 16 * qd + (t & 15);
+    const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
+    float d[64];
+    if (warp < 4) {
+      tmem_ld32(tb + lane_base + 0, d);                  // D0: 32 columns
+#pragma unroll
+      for (int e = 32; e < 64; ++e) d[e] = 0.f;
+    } else {
+      tmem_ld32(tb + lane_base + 32, d);                 // D1: 64 columns
+      tmem_ld32(tb + lane_base + 64, d + 32);
+    }
+    if (t < 16) {
+      const bool isA = row < 32;
+      const int i = (warp < 4 ? 0 : 32) + (row & 31);    // chunk row of A or M
+      if (isA) {
+        const float bi = s.beta[i];
+#pragma unroll
+        for (int j = 0; j < 64; ++j) At[j * C + i] = (j < i) ? bi * d[j] : 0.f;
+      } else {
+        bf16* Mg = sv.M + cb * C * C;
+#pragma unroll
+        for (int j8 = 0; j8 < 8; ++j8) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = (8 * j8 + e <= i) ? d[8 * j8 + e] : 0.f;
+          *reinterpret_cast<uint4*>(Mg + ct_off(i, 8 * j8, C)) = pack8(f);
+        }
+      }
+    }
+  }
+  // beta k e^g into the write-key tile (the Grams have read it)
+  {
+#pragma unroll
+    for (int it = 0; it < 4; ++it)
+      *reinterpret_cast<uint4*>(s.KB + ct16(r, jq + 4 * it)) = bkr[it];
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  // ---- T = (I + A)^{-1}: thread j < 64 forward-substitutes column j in fp32,
+  //      T[i][j] = delta_ij - sum_{m < i} A[i][m] T[m][j], all rows in registers
+  //      (the updates of one step are independent), then T = T_hi + T_lo in bf16.
+  bf16* Thi = reinterpret_cast<bf16*>(s.G + 2 * kBox);
+  bf16* Tlo = reinterpret_cast<bf16*>(s.G + 3 * kBox);
+  if (tid < C) {
+    const int j = tid;
+    float acc[C];
+#pragma unroll
+    for (int i = 0; i < C; ++i) acc[i] = (i == j) ? 1.f : 0.f;
+#pragma unroll
+    for (int m = 0; m < C - 1; ++m) {
+      const float tm = acc[m];
+      const float* arow = At + m * C;  // A[.][m]
+#pragma unroll
+      for (int i4 = (m + 1) & ~3; i4 < C; i4 += 4) {
+        const float4 a = *reinterpret_cast<const float4*>(arow + i4);
+        if (i4 + 0 > m) acc[i4 + 0] -= a.x * tm;
+        if (i4 + 1 > m) acc[i4 + 1] -= a.y * tm;
+        if (i4 + 2 > m) acc[i4 + 2] -= a.z * tm;
+        if (i4 + 3 > m) acc[i4 + 3] -= a.w * tm;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < C; ++i) {
+      const bf16 hi = __float2bfloat16_rn(acc[i]);
+      const bf16 lo = __float2bfloat16_rn(acc[i] - __bfloat162float(hi));
+      const int o = ((i >> 3) * 8 + (j >> 3)) * 64 + (i & 7) * 8 + (j & 7);
+      Thi[o] = hi;
+      Tlo[o] = lo;
+    }
+  }
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  // ---- W = T (beta k e^g), U' = T (beta v): T_hi and T_lo terms, M = 64, N = 128
+  if (tid == 0) {
+    const uint32_t id = tc::idesc_bf16(64, 128, false, true);
+    const uint64_t ah = tc::sdesc_kmaj(Thi, C, 0), al = tc::sdesc_kmaj(Tlo, C, 0);
+    const uint64_t bk = tc::sdesc_mnmaj(reinterpret_cast<const bf16*>(s.KB), D, 0);
+    const uint64_t bw = tc::sdesc_mnmaj(reinterpret_cast<const bf16*>(s.V), D, 0);
+#pragma unroll
+    for (int ks = 0; ks < C / 16; ++ks) {
+      const uint32_t acc = ks > 0 ? 1u : 0u;
+      tc::mma(tb + 0, ah + 16u * ks, bk + 256u * ks, id, acc);
+      tc::mma(tb + 128, ah + 16u * ks, bw + 256u * ks, id, acc);
+      tc::mma(tb + 0, al + 16u * ks, bk + 256u * ks, id, 1u);
+      tc::mma(tb + 128, al + 16u * ks, bw + 256u * ks, id, 1u);
+    }
+    tc::commit(&s.bar_mma);
+  }
+  // T (bf16, the high part) to the saved buffer while they run
+  for (int idx = tid; idx < C * C / 8; idx += NTP)
+    *reinterpret_cast<uint4*>(sv.T + cb * C * C + 8 * idx) =
+        *reinterpret_cast<const uint4*>(Thi + 8 * idx);
+  ok = prep_wait(&s.bar_mma, 1);
+  if (!ok) break;
+  // ---- W (warps 0-3) and U' (warps 4-7), rows 16 (warp % 4) + lane, lanes 0..15
+  {
+    const int qd = warp & 3, row = 16 * qd + (lane & 15);
+    const uint32_t base = tb + ((uint32_t)(32 * qd) << 16) + (warp < 4 ? 0u : 128u);
+    bf16* out = (warp < 4 ? sv.W : sv.Up) + cb * C * D;
+#pragma unroll
+    for (int q32 = 0; q32 < 4; ++q32) {
+      float d[32];
+      tmem_ld32(base + 32 * q32, d);
+      if (lane < 16) {
+#pragma unroll
+        for (int e8 = 0; e8 < 4; ++e8)
+          *reinterpret_cast<uint4*>(out + ct_off(row, 32 * q32 + 8 * e8, D)) = pack8(d + 8 * e8);
+      }
+    }
+  }
+  } while (0);
+  if (!ok) {
+    // a bounded wait gave up: record it, and give the TMA loads in flight a
+    // bounded chance to land before the shared memory is released
+    if (tid == 0 && err) atomicExch(err, 1);
+    if (tid == 0) tc::mbar_wait(&s.bar_tma, 0u, kSpinPrep);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tb, 256);
+}
+
+// --- tensor maps (host) ------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// [B, T, H, 128] row-major, elements of `bytes` bytes; box: 128 bytes of
+// channels x 64 tokens of one head, 128-byte swizzle, out-of-range tokens zero.
+bool encode_btdh(CUtensorMap* m, const void* base, const Problem& p, int bytes) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)p.H, (cuuint64_t)p.T, (cuuint64_t)p.B};
+  const cuuint64_t row = (cuuint64_t)D * bytes;
+  const cuuint64_t strides[3] = {row, row * p.H, row * p.H * p.T};
+  const cuuint32_t box[4] = {(cuuint32_t)(128 / bytes), 1, (cuuint32_t)C, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_prep(const Problem& p, const bf16* q, const bf16* k, const bf16* v,
+                        const float* beta, const float* g, const Saved& sv, cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mg;
+  memset(&mg, 0, sizeof(mg));
+  const bool chan = p.gk == D;
+  if (!encode_btdh(&mq, q, p, 2) || !encode_btdh(&mk, k, p, 2) || !encode_btdh(&mv, v, p, 2) ||
+      (chan && !encode_btdh(&mg, g, p, 4)))
+    return cudaErrorInvalidValue;
+  const size_t sm = sizeof(PrepSmem) + 1024;
+  const bool phase = p.gate == kGatePhase;
+  auto kern = phase ? k_prep_tc<true> : k_prep_tc<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  const double nb = (double)p.B * p.H * p.NC, ntok = nb * C;
+  // reads q, k, v, g, beta (the operator's inputs); writes T, beta, dec, W, U', M, Qh, Kt, ||k||^2
+  const double io = ntok * (3 * D * 2 + p.gk * 4 + 4);
+  const double bytes =
+      io + nb * ((double)kTBytes + 2 * kBetaBytes + kDecBytes + 4.0 * kTileBytes + kMBytes);
+  // Grams (32 + 64 columns of M = 64, K = 128), the solve (C^3 / 3), W and U' (two T terms)
+  const double flops = nb * (2.0 * C * 96 * D + C * C * C / 3.0 + 2.0 * 2 * 2 * C * C * D);
+  prof_begin(kKTcIntraFwd, io, bytes, flops, st);
+  kern<<<dim3(p.NC, p.H, p.B), NTP, sm, st>>>(p, mq, mk, mv, mg, chan ? nullptr : g, beta, sv,
+                                             device_error_word());
+  e = cudaGetLastError();
+  prof_end(st);
+  return e;
+}
+
+}  // namespace fast
+}  // namespace dr

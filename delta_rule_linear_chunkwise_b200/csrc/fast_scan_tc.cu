@@ -436,7 +436,11 @@ __device__ __forceinline__ void bscan_fill(const Problem& p, BScanStage<BV>& s, 
   }
 }
 
-template <int BV>
+// PHASE: the SFDA rotation-decay gate.  The forward decay multiplies each
+// state row's key pair by dec = dec[2j] + i dec[2j+1] (the conjugate of the
+// chunk's cumulative complex decay), so the gradient goes back through the
+// adjoint, multiplication by conj(dec); the pair's keys sit on adjacent lanes.
+template <int BV, bool PHASE>
 __global__ void __launch_bounds__(NTF, 1)
     k_bwd_scan_tc(Problem p, Saved sv, const bf16* __restrict__ dO, ScanSeg sg,
                   bf16* __restrict__ dUout, bf16* __restrict__ dhout, int* __restrict__ err) {
@@ -522,7 +526,8 @@ __global__ void __launch_bounds__(NTF, 1)
     const size_t cb = chunk_id(p, b, h, n);
     BScanStage<BV>& st = s.st[it & 1];
     const uint32_t T_U = (uint32_t)((it & 1) * BV);
-    const float dc = st.dec[c];  // read before the stage is refilled below
+    const float dc = st.dec[PHASE ? (c & ~1) : c];  // read before the stage is refilled below
+    const float di = PHASE ? ((c & 1) ? -st.dec[c] : st.dec[c | 1]) : 0.f;
     if (tid == 0) {
       const uint64_t dKT = tc::sdesc_kmaj(st.KT, D, 0), dQH = tc::sdesc_mnmaj(st.QH, D, 0);
       const uint64_t dDO = tc::sdesc_mnmaj(st.DO, BV, 0);
@@ -601,8 +606,17 @@ __global__ void __launch_bounds__(NTF, 1)
       for (int q16 = 0; q16 < HB / 16; ++q16)
         tc::tmem_ld16_nowait(lane_addr(tbase, warp, T_S + ah * HB + 16 * q16), r + 16 * q16);
       tc::tmem_wait_ld();
+      if (PHASE) {
+        // own key c: Re (even c) or Im (odd c) of conj(dec_re + i dec_im) (x + i y)
 #pragma unroll
-      for (int e = 0; e < HB; ++e) dS[e] = dS[e] * dc + __uint_as_float(r[e]);
+        for (int e = 0; e < HB; ++e) {
+          const float partner = __shfl_xor_sync(0xffffffffu, dS[e], 1);
+          dS[e] = dS[e] * dc + di * partner + __uint_as_float(r[e]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < HB; ++e) dS[e] = dS[e] * dc + __uint_as_float(r[e]);
+      }
       write_dsb();
     }
     tc::fence_smem_to_async();
@@ -635,8 +649,8 @@ cudaError_t launch_bwd_scan_tc_bv(const Problem& p, const Saved& sv, const bf16*
   const float* dST = sg.mode == 0 ? sg.S0 : nullptr;
   float* dS0 = sg.ST;
   const size_t sm = sizeof(BScanSmem<BV>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_bwd_scan_tc<BV>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  auto kern = p.gate == kGatePhase ? k_bwd_scan_tc<BV, true> : k_bwd_scan_tc<BV, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const double nb = (double)p.B * p.H * p.NC, ntok = nb * C, heads = (double)p.B * p.H;
   // reads W, Qh, Kt, M, dec, dO; writes dU, dh (output pass) and the segment
@@ -649,8 +663,8 @@ cudaError_t launch_bwd_scan_tc_bv(const Problem& p, const Saved& sv, const bf16*
                     (sg.G == 1 ? heads * D * D * 4.0 * ((dST ? 1 : 0) + (dS0 ? 1 : 0)) : 0.0);
   const double flops = nb * (2.0 * C * C * D + 2.0 * C * D * D * 3);
   prof_begin(kKTcScanBwd, io, bytes, flops, st);
-  k_bwd_scan_tc<BV><<<dim3(D / BV, p.H, p.B * sg.G), NTF, sm, st>>>(p, sv, dO, sg, dU, dh,
-                                                                    device_error_word());
+  kern<<<dim3(D / BV, p.H, p.B * sg.G), NTF, sm, st>>>(p, sv, dO, sg, dU, dh,
+                                                       device_error_word());
   e = cudaGetLastError();
   prof_end(st);
   return e;

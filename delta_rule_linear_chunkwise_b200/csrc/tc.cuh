@@ -1,6 +1,6 @@
 // tc.cuh -- sm_100a tensor-core helpers: tcgen05 MMA with shared-memory
 // operands and tensor-memory (TMEM) accumulators, mbarriers with bounded
-// waits, and the legacy warp-level mma.sync used for latency-bound chains.
+// waits, bulk copies.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -186,17 +186,6 @@ __device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t* r) {
 }
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// --- legacy warp-level MMA (m16n8k16, bf16 in, fp32 accumulate) ----------
-// Not volatile: the instruction touches registers only, so the compiler may
-// interleave independent accumulation chains.
-__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, const uint32_t* b) {
-  asm(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
 }  // namespace tc

@@ -40,8 +40,10 @@
  *    maps each state row's pair (x, y) to
  *    alpha_j (cos theta_j x - sin theta_j y, sin theta_j x + cos theta_j y)
  *    before the erase-and-write (zero phase: KDA with each pair's channels
- *    sharing one decay).  Supported by dr_chunk_fwd (bf16, dk = dv = 128) and
- *    dr_decode_step; dr_chunk_bwd returns DR_ERR_UNSUPPORTED for it.
+ *    sharing one decay).  Supported by dr_chunk_fwd and dr_chunk_bwd (bf16,
+ *    dk = dv = 128; other shapes give DR_ERR_UNSUPPORTED) and by
+ *    dr_decode_step; dg[..., 2j] is then d/d log alpha_j and dg[..., 2j+1]
+ *    d/d theta_j.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *    stream).  Arguments are validated on the host before any launch; a
  *    non-DR_OK status means nothing was launched, except DR_ERR_CUDA, which
@@ -118,7 +120,8 @@ dr_status dr_chunk_fwd(const dr_problem* p, const void* q, const void* k, const 
    Out: dq, dk, dv (storage dtype), dbeta (fp32; d/deta in Kaczmarz mode),
         dg (fp32, shaped like g; ignored and may be NULL for gate NONE),
         dS0 (fp32; NULL = not wanted).
-   The phase gate has no backward yet: DR_ERR_UNSUPPORTED, nothing launched.
+   The phase gate needs dtype DR_BF16 and dk = dv = 128 (else
+   DR_ERR_UNSUPPORTED, nothing launched).
    ws:  at least dr_workspace_size(p, 1) bytes, 256-byte aligned. */
 dr_status dr_chunk_bwd(const dr_problem* p, const void* q, const void* k, const void* v,
                        const float* beta, const float* g, const float* S0, const void* dO,

@@ -58,10 +58,11 @@ def run_oracle(w, inp, heads, dST=None):
             for n in ("q", "k", "v", "beta", "g", "dO")}
     S0 = cat([pick(inp["S0"], b, h, True) for b, h in heads])
     dst = None if dST is None else cat([pick(dST, b, h, True) for b, h in heads])
+    gate = oracle.GATE_PHASE if w.gate == "phase" else None
     o, ST = oracle.recurrent_fwd(args["q"], args["k"], args["v"], args["beta"], args["g"],
-                                 S0, beta_mode=mode, eps=w.eps)
+                                 S0, beta_mode=mode, eps=w.eps, gate=gate)
     gr = oracle.recurrent_bwd(args["q"], args["k"], args["v"], args["beta"], args["g"], S0,
-                              args["dO"], dst, beta_mode=mode, eps=w.eps)
+                              args["dO"], dst, beta_mode=mode, eps=w.eps, gate=gate)
     out = dict(o=o[:, :, 0], ST=ST[:, 0], dq=gr["dq"][:, :, 0], dk=gr["dk"][:, :, 0],
                dv=gr["dv"][:, :, 0], dbeta=gr["dbeta"][:, :, 0],
                dg=None if gr["dg"] is None else gr["dg"][:, :, 0], dS0=gr["dS0"][:, 0])

@@ -160,13 +160,16 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
 
 
 def test_phase_gate_routing(lib):
-    # The SFDA phase gate: forward on the bf16 d = 128 tensor-core path only,
-    # no backward; an unknown gate value is an argument error.  Host-side
-    # checks only (fake pointers, nothing launched).
+    # The SFDA phase gate: forward and backward on the bf16 d = 128 tensor-core
+    # path only; an unknown gate value is an argument error.  Host-side checks
+    # only (fake pointers: every call here must be rejected before a launch).
     assert _fwd(lib, _prob(gate="phase")) == binding.DR_ERR_UNSUPPORTED          # dk = 64
     assert _fwd(lib, _prob(gate="phase", dk=128, dv=128, dtype="f32")) == \
         binding.DR_ERR_UNSUPPORTED
-    assert _bwd(lib, _prob(gate="phase", dk=128, dv=128)) == binding.DR_ERR_UNSUPPORTED
+    assert _bwd(lib, _prob(gate="phase")) == binding.DR_ERR_UNSUPPORTED          # dk = 64
+    assert _bwd(lib, _prob(gate="phase", dk=128, dv=128, dtype="f32")) == \
+        binding.DR_ERR_UNSUPPORTED
+    assert _bwd(lib, _prob(gate="phase", dk=128, dv=128), dg=None) == binding.DR_ERR_INVALID_ARG
     assert _fwd(lib, _prob(gate="phase", dk=128, dv=128), g=None) == binding.DR_ERR_INVALID_ARG
     bad = _prob()
     bad.gate = 4

@@ -23,18 +23,15 @@ def test_algorithmic_model_matches_per_token_head_figures():
     assert gbytes == g.token_heads * 2840 + g.B * g.H * 128 * 128 * 4 * 2
 
 
-def test_forward_only_model_for_the_phase_gate():
-    # SFDA workload: forward FLOPs 10 C d + 6 d^2 per token-head; bytes: q, k,
-    # v, g (d_k fp32 per token for the pair gates), beta read, o written, and
-    # the final state
+def test_phase_gate_step_model():
+    # SFDA workload: the same fwd+bwd model as KDA (the pair gate has d_k fp32
+    # values per token, like the per-channel gate, and so does its gradient)
     w = WORKLOADS["sfda_bf16_b4h16t8192"]
-    flops, nbytes = bench.algorithmic_step(w, fwd_only=True)
-    th, C, d = w.token_heads, w.chunk, w.dk
-    assert flops == th * (10 * C * d + 6 * d * d)
-    assert nbytes == th * (3 * d * 2 + 4 * d + 4 + d * 2) + w.B * w.H * d * d * 4
-    # the phase gate costs the per-channel gate's bytes in the full model too
     kda = WORKLOADS["kda_bf16_b4h16t8192"]
     assert bench.algorithmic_step(w) == bench.algorithmic_step(kda)
+    flops, nbytes = bench.algorithmic_step(w)
+    th, C, d = w.token_heads, w.chunk, w.dk
+    assert flops == th * (38 * C * d + 20 * d * d)
 
 
 def _free_port():

@@ -145,15 +145,16 @@ def test_tensor_core_path_ragged(T, gate):
 
 
 # Strong decay on the bf16 tensor-core path: log-gates logsigmoid(N(mu, 1)) with
-# mu = -1 (alpha ~ 0.25 per token), so that the cumulative log-decay across one
-# chunk reaches about -110: below where e^gamma itself underflows in fp32.  Every
-# factor the kernels form is the exponential of a centred difference of
-# cumulative gates.
+# mu = -1 (alpha ~ 0.25 per token; a chunk's cumulative log-decay reaches about
+# -110) and mu = -3 (alpha ~ 0.05; about -220), far below where e^gamma itself
+# underflows in fp32.  Every gate factor the kernels form is the exponential of
+# a difference of cumulative gates taken against a reference row of the same
+# 32-row half, so it spans at most 16 tokens of decay.
 STRONG = [("gdn", "gdn_bf16_b4h8t2048"), ("kda", "kda_bf16_b4h16t8192"),
           ("kla", "kla_bf16_b1h16t65536")]
 
 
-@pytest.mark.parametrize("mu", [-1.0])
+@pytest.mark.parametrize("mu", [-1.0, -3.0])
 @pytest.mark.parametrize("kind,name", STRONG, ids=[k for k, _ in STRONG])
 @pytest.mark.parametrize("save", [True, False], ids=["saved", "recompute"])
 def test_strong_decay_tensor_core(kind, name, mu, save):
@@ -162,7 +163,7 @@ def test_strong_decay_tensor_core(kind, name, mu, save):
     _check(w, make_inputs(w), dST=random_state(w, seed=15, std=0.5), save=save)
 
 
-@pytest.mark.parametrize("mu", [-1.0])
+@pytest.mark.parametrize("mu", [-1.0, -3.0])
 @pytest.mark.parametrize("kind,name", STRONG, ids=[k for k, _ in STRONG])
 def test_strong_decay_segmented_scan(kind, name, mu):
     """Long sequence, two heads: the chunk-parallel affine scan under strong decay."""

@@ -1,15 +1,16 @@
 """GPU parity of the SFDA phase gate (2 x 2 rotation-decay per key pair) against
-the fp64 oracle's token-by-token recurrence with the same gate: the chunkwise
-forward on the tensor-core path (o and the final state) and the decode step.
-Bar: 2e-2 max relative error for bf16 storage (o rounded to bf16; the chunk
-tiles are bf16 operands with fp32 accumulation); the decode step's fp32 state
-to 1e-4 and its fp32 output to 1e-4."""
+the fp64 oracle's token-by-token recurrence with the same gate and its
+hand-derived backward: the chunkwise forward on the tensor-core path (o and the
+final state), the chunkwise backward (dq, dk, dv, dbeta, d log alpha and d theta,
+dS0), and the decode step.  Bar: 2e-2 max relative error for bf16 storage (the
+chunk tiles are bf16 operands with fp32 accumulation); the decode step's fp32
+state to 1e-4 and its fp32 output to 1e-4."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
-from _parity import rel_err
+from _parity import compare, rel_err, run_gpu, run_oracle, select, tol
 from delta_rule_linear_chunkwise_b200 import WORKLOADS, binding, make_inputs
 from delta_rule_linear_chunkwise_b200.workloads import random_state
 
@@ -101,13 +102,61 @@ def test_sfda_zero_phase_matches_paired_kda():
     assert rel_err(S_p.cpu().numpy(), S_k.cpu().numpy()) < 1e-2
 
 
-def test_sfda_backward_is_unsupported():
-    w = SFDA.with_(B=1, H=1, T=64)
+def _bwd_check(w, heads=None, save=True, dST=True):
     inp = make_inputs(w)
-    d = {n: (None if x is None else x.cuda()) for n, x in inp.items()}
-    with pytest.raises(binding.DrError):
-        binding.Plan.for_workload(w).bwd(d["q"], d["k"], d["v"], d["beta"], d["g"], d["S0"],
-                                         d["dO"])
+    dst = random_state(w, seed=41, std=0.5) if dST else None
+    gpu = run_gpu(w, inp, dST=dst, save=save)
+    if heads is None:
+        heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    ref, heads = run_oracle(w, inp, heads, dST=dst)
+    errs = compare(w, select(gpu, heads), ref)
+    bad = {n: e for n, e in errs.items() if not (e <= tol(w))}
+    assert not bad, f"{w.name}: {errs}"
+    return errs
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200])
+def test_sfda_backward_ragged_all_heads(T):
+    _bwd_check(SFDA.with_(name=f"sfda_bwd_t{T}", B=2, H=3, T=T, s0_std=0.1))
+
+
+def test_sfda_backward_recompute_and_kaczmarz():
+    _bwd_check(SFDA.with_(name="sfda_bwd_rec", B=1, H=2, T=300, s0_std=0.1), save=False)
+    _bwd_check(SFDA.with_(name="sfda_bwd_kacz", B=1, H=2, T=300, beta_mode="kaczmarz",
+                          normalize_k=False, s0_std=0.1))
+
+
+@pytest.mark.parametrize("mu", [-1.0, -3.0])
+def test_sfda_backward_strong_decay(mu):
+    _bwd_check(SFDA.with_(name=f"sfda_bwd_strong{mu}", B=1, H=2, T=256, g_mean=mu,
+                          s0_std=0.3))
+
+
+def test_sfda_backward_segmented_affine_scan():
+    _bwd_check(SFDA.with_(name="sfda_bwd_seg", B=1, H=2, T=4096 + 100, s0_std=0.1))
+
+
+def test_sfda_backward_full_size_sampled_heads():
+    errs = _bwd_check(SFDA, heads=[(0, 0), (2, 7), (3, 15)], dST=False)
+    print("sfda backward full size", {k: f"{v:.2e}" for k, v in errs.items()})
+
+
+def test_sfda_zero_phase_backward_matches_paired_kda():
+    # zero phase: the SFDA backward is KDA's with each pair's decay shared, and
+    # d/d log alpha of a pair is the sum of its two channels' KDA gradients
+    w = SFDA.with_(name="sfda_zero_bwd", B=1, H=2, T=200, s0_std=0.1)
+    inp = make_inputs(w)
+    g = inp["g"].clone()
+    g[..., 1::2] = 0.0
+    gk = g.clone()
+    gk[..., 1::2] = g[..., 0::2]
+    ip = dict(inp, g=g)
+    ik = dict(inp, g=gk)
+    a = run_gpu(w, ip)
+    b = run_gpu(w.with_(gate="channel"), ik)
+    for n in ("dq", "dk", "dv", "dbeta", "dS0"):
+        assert rel_err(a[n], b[n]) < 1e-2, n
+    assert rel_err(a["dg"][..., 0::2], b["dg"][..., 0::2] + b["dg"][..., 1::2]) < 1e-2
 
 
 @pytest.mark.parametrize("kw", [{}, {"dtype": "f32"}, {"dk": 64, "dv": 32},
