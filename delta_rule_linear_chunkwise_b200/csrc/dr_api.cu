@@ -13,6 +13,19 @@ namespace {
 std::atomic<int> g_injected_timeouts{0};
 }  // namespace
 
+int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 bool take_injected_timeout() {
   int n = g_injected_timeouts.load();
   while (n > 0)

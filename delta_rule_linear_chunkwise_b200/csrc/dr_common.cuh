@@ -83,6 +83,8 @@ void prof_end(cudaStream_t st);
 cudaError_t read_and_clear_device_error(int* flag);
 // Device address of that error word on the current device (nullptr on failure).
 int* device_error_word();
+// Streaming multiprocessors of the current device (cached per device; 148 on B200).
+int sm_count();
 // Fault injection (dr_inject_timeout): true, and one fewer pending, if the
 // next chunk-backward launch is to take its bounded-wait timeout path.
 bool take_injected_timeout();

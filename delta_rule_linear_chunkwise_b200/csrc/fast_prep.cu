@@ -74,14 +74,26 @@ struct PrepSmem {
                                             // then A^T (fp32 [j][i]) and T hi | lo (bf16)
   alignas(1024) unsigned char KB[3 * kBox]; // write keys: rho0 rows 0..31 | rho1 rows 0..63;
                                             // then beta k e^g (MN-major B of W)
-  float ref[3][D];   // cumulative gate at rows rho0, rho1 and C - 1
-  float rot[3][D];   // phase gate: (cos, sin) of the cumulative phase at those rows, per pair
+  // per key channel (phase gate: per pair, complex, at the pair's two channels),
+  // for the two halves' reference rows rho0 = 15, rho1 = 47:
+  float ref[2][D];   // cumulative gate at rho
+  float rot[2][D];   // phase gate: (cos, sin) of the cumulative phase at rho
+  float zr[2][D];    // zeta_rho                     (real gates: e^{g_rho})
+  float ec[2][D];    // conj(zeta_C / zeta_rho)      (real gates: e^{g_C - g_rho})
+  // write keys of the first half against the second reference, in two steps
+  // through the half boundary: conj(zeta_31 / zeta_rho0), conj(zeta_rho1 / zeta_31)
+  float xk[2][D];
+  float tot[D];      // cumulative gate of the first half's last row
   float gs[C];       // scalar gate: cumulative per row
   float eta[C];      // input beta (eta in Kaczmarz mode)
   float beta[C];     // effective beta
   uint64_t bar_tma, bar_mma;
   uint32_t tmem;
 };
+
+static_assert(sizeof(float) * (64 * (64 + 4) + 32 * 33) <= 4 * kBox &&
+                  offsetof(PrepSmem, K) == offsetof(PrepSmem, Q) + 2 * kBox,
+              "the fp32 solve tiles fit the adjacent q and k regions");
 
 // Byte offset of 16-byte chunk ch (0..7) of row r in a 128-byte-swizzled TMA
 // box (chunk index XOR row mod 8 within each 1 KB block).
@@ -101,6 +113,15 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
       "r"(tc::smem_u32(bar))
       : "memory");
+}
+
+// L2 prefetch of one TMA box (no shared-memory destination).
+__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int c0, int c1, int c2,
+                                                int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
 }
 
 // 32 consecutive fp32 TMEM columns of this thread's lane.
@@ -149,7 +170,8 @@ __global__ void __launch_bounds__(NTP, 2)
     k_prep_tc(Problem p, const __grid_constant__ CUtensorMap tq,
               const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
               const __grid_constant__ CUtensorMap tg, const float* __restrict__ g_scalar,
-              const float* __restrict__ beta_in, Saved sv, int* __restrict__ err) {
+              const float* __restrict__ beta_in, Saved sv, int* __restrict__ err,
+              int pf_ahead) {
   extern __shared__ __align__(1024) unsigned char smraw[];
   PrepSmem& s = *reinterpret_cast<PrepSmem*>(
       (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -179,6 +201,26 @@ __global__ void __launch_bounds__(NTP, 2)
       for (int x = 0; x < 4; ++x) tma_load_4d(s.G + x * kBox, &tg, 32 * x, h, t0, b, &s.bar_tma);
     }
   }
+  // L2 prefetch of the tiles of the CTA pf_ahead places further in launch order
+  // (about one wave ahead), so that its TMA loads are served from L2 (measured:
+  // 478 against 493 us when issued after this CTA's own loads have landed)
+  if (tid == 32 && pf_ahead > 0) {
+    const long L = n + (long)p.NC * (h + (long)p.H * b) + pf_ahead;
+    if (L < (long)p.NC * p.H * p.B) {
+      const int n2 = (int)(L % p.NC), h2 = (int)((L / p.NC) % p.H), b2 = (int)(L / ((long)p.NC * p.H));
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        tma_prefetch_4d(&tq, 64 * x, h2, n2 * C, b2);
+        tma_prefetch_4d(&tk, 64 * x, h2, n2 * C, b2);
+        tma_prefetch_4d(&tv, 64 * x, h2, n2 * C, b2);
+      }
+      if (chan) {
+#pragma unroll
+        for (int x = 0; x < 4; ++x) tma_prefetch_4d(&tg, 32 * x, h2, n2 * C, b2);
+      }
+    }
+  }
+
   if (!chan && tid < C)
     s.gs[tid] = (tid < nvalid && p.gate != kGateNone) ? g_scalar[row_id(p, b, t0 + tid, h)] : 0.f;
   const float eta = (tid < C && tid < nvalid) ? beta_in[row_id(p, b, t0 + tid, h)] : 0.f;
@@ -186,26 +228,24 @@ __global__ void __launch_bounds__(NTP, 2)
   const uint32_t tb = s.tmem;
   do {  // leaves early (break) only when a bounded wait gives up
   if (!ok) break;
-
-  // ---- cumulative gate down the rows
+  // ---- cumulative gate down the rows (padded rows carry a zero gate): thread
+  // (channel c, half) scans its 32 rows in registers
   // per-channel element (r, c) of the gate tile: box c / 32, chunk (c % 32) / 4
   auto gp = [&](int r, int c) -> float* {
     return reinterpret_cast<float*>(s.G + (c >> 5) * kBox + swz(r, (c & 31) >> 2) + (c & 3) * 4);
   };
   if (chan) {
     const int c = tid & 127, hf = tid >> 7;
-    float run = 0.f;
-#pragma unroll 8
-    for (int r = 32 * hf; r < 32 * hf + 32; ++r) {
-      run += *gp(r, c);
-      *gp(r, c) = run;
-    }
+    float x[32];
+#pragma unroll
+    for (int r = 0; r < 32; ++r) x[r] = *gp(32 * hf + r, c);
+#pragma unroll
+    for (int r = 1; r < 32; ++r) x[r] += x[r - 1];
+    if (hf == 0) s.tot[c] = x[31];
     __syncthreads();
-    if (hf) {
-      const float off = *gp(31, c);
-#pragma unroll 8
-      for (int r = 32; r < 64; ++r) *gp(r, c) += off;
-    }
+    const float off = hf ? s.tot[c] : 0.f;
+#pragma unroll
+    for (int r = 0; r < 32; ++r) *gp(32 * hf + r, c) = x[r] + off;
   } else if (warp == 0) {
     const float a0 = s.gs[2 * lane], a1 = s.gs[2 * lane + 1];
     float x = a0 + a1;
@@ -218,39 +258,55 @@ __global__ void __launch_bounds__(NTP, 2)
     s.gs[2 * lane] = x - a1;
   }
   __syncthreads();
-  if (tid < D) {
-    const int rows[3] = {kRho0, kRho1, C - 1};
+  auto gam = [&](int r, int c) -> float { return chan ? *gp(r, c) : s.gs[r]; };
+  // per-channel reference factors and the chunk decay
+  if (PHASE) {
+    if (tid < D / 2) {
+      const int c = 2 * tid;
+      const float gC = gam(C - 1, c), tC = gam(C - 1, c + 1);
+      const float g31 = gam(31, c), t31 = gam(31, c + 1);
+      float gr[2], tr[2], sn, cs;
+      gr[0] = gam(kRho0, c), tr[0] = gam(kRho0, c + 1);
+      gr[1] = gam(kRho1, c), tr[1] = gam(kRho1, c + 1);
 #pragma unroll
-    for (int k3 = 0; k3 < 3; ++k3) s.ref[k3][tid] = chan ? *gp(rows[k3], tid) : s.gs[rows[k3]];
-  }
-  __syncthreads();
-  if (PHASE && tid < D / 2) {
-#pragma unroll
-    for (int k3 = 0; k3 < 3; ++k3) {
-      float sn, cs;
-      sincosf(s.ref[k3][2 * tid + 1], &sn, &cs);
-      s.rot[k3][2 * tid] = cs;
-      s.rot[k3][2 * tid + 1] = sn;
+      for (int hh = 0; hh < 2; ++hh) {
+        s.ref[hh][c] = gr[hh];
+        sincosf(tr[hh], &sn, &cs);
+        s.rot[hh][c] = cs, s.rot[hh][c + 1] = sn;
+        const float m = __expf(gr[hh]);
+        s.zr[hh][c] = m * cs, s.zr[hh][c + 1] = -m * sn;          // zeta_rho
+        sincosf(tC - tr[hh], &sn, &cs);
+        const float mc = __expf(gC - gr[hh]);
+        s.ec[hh][c] = mc * cs, s.ec[hh][c + 1] = mc * sn;         // conj(zeta_C / zeta_rho)
+      }
+      sincosf(t31 - tr[0], &sn, &cs);
+      float m = __expf(g31 - gr[0]);
+      s.xk[0][c] = m * cs, s.xk[0][c + 1] = m * sn;
+      sincosf(tr[1] - t31, &sn, &cs);
+      m = __expf(gr[1] - g31);
+      s.xk[1][c] = m * cs, s.xk[1][c + 1] = m * sn;
+      // the chunk decay conj(zeta_C) = e^{g_C} e^{+i Theta_C}
+      sincosf(tC, &sn, &cs);
+      const float a = __expf(gC);
+      sv.dec[cb * D + c] = a * cs;
+      sv.dec[cb * D + c + 1] = a * sn;
     }
-  }
-  // the chunk decay: e^{g_C} (phase gate: conj(zeta_C) per pair)
-  if (tid < D) {
-    float dv;
-    if (PHASE) {
-      const int c0 = tid & ~1;
-      float sn, cs;
-      sincosf(s.ref[2][c0 + 1], &sn, &cs);
-      dv = __expf(s.ref[2][c0]) * ((tid & 1) ? sn : cs);
-    } else {
-      dv = __expf(s.ref[2][tid]);
-    }
-    sv.dec[cb * D + tid] = dv;
+  } else if (tid < D) {
+    const int c = tid;
+    const float g0 = gam(kRho0, c), g1 = gam(kRho1, c), gC = gam(C - 1, c), g31 = gam(31, c);
+    s.ref[0][c] = g0, s.ref[1][c] = g1;
+    s.zr[0][c] = __expf(g0), s.zr[1][c] = __expf(g1);
+    s.ec[0][c] = __expf(gC - g0), s.ec[1][c] = __expf(gC - g1);
+    s.xk[0][c] = __expf(g31 - g0), s.xk[1][c] = __expf(g1 - g31);
+    sv.dec[cb * D + c] = __expf(gC);
   }
 
   // ---- factor pass.  Warp w: rows 8w .. 8w + 7; lane: row 8w + lane % 8 and the
   // 16-byte chunks j = lane / 8 + 4 it (it = 0..3) of its 128 channels, so that
   // the swizzled TMA tiles are read and the core-tiled operands written without
-  // bank conflicts.
+  // bank conflicts.  Per element two exponentials, e^{+-(g - g_rho)}; the other
+  // factors are those times per-channel reference factors (a product that
+  // underflows there is below e^{-37} of the row's leading terms).
   const int r = 8 * warp + (lane & 7), jq = lane >> 3, hr = r >> 5;
   uint4 qr[4], kr[4], vr[4];
   float nn = 0.f;
@@ -280,6 +336,7 @@ __global__ void __launch_bounds__(NTP, 2)
   {
     unsigned char* GAh = hr ? s.K : s.Q;      // [K; Q] of this row's half
     const int R = r & 31;                     // row within the half
+    const float sg = chan ? 0.f : s.gs[r];
 #pragma unroll
     for (int it = 0; it < 4; ++it) {
       const int j = jq + 4 * it, c0 = 8 * j;
@@ -292,9 +349,6 @@ __global__ void __launch_bounds__(NTP, 2)
         const float4 c4 = *reinterpret_cast<const float4*>(s.G + (j >> 2) * kBox + swz(r, 2 * (j & 3) + 1));
         gg[0] = a.x, gg[1] = a.y, gg[2] = a.z, gg[3] = a.w;
         gg[4] = c4.x, gg[5] = c4.y, gg[6] = c4.z, gg[7] = c4.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) gg[e] = s.gs[r];
       }
       float kc[8], qc[8], kb[8], kb1[8], qh[8], kt[8], bk[8], bv[8];
       if (PHASE) {
@@ -304,44 +358,49 @@ __global__ void __launch_bounds__(NTP, 2)
           float sn, cs;
           sincosf(gg[e + 1], &sn, &cs);                  // e^{-i Theta} = cs - i sn
           const float rhc = s.rot[hr][cc], rhs = s.rot[hr][cc + 1];   // e^{i Theta_rho}
-          // w = e^{-i (Theta - Theta_rho)} of this row's reference
+          // e^{-i (Theta - Theta_rho)}
           const float wr = cs * rhc + sn * rhs, wi = cs * rhs - sn * rhc;
+          const float d = gg[e] - s.ref[hr][cc];
+          const float ep = __expf(d), em = __expf(-d);
           const float kx = kv[e], ky = kv[e + 1], qx = qv[e], qy = qv[e + 1];
           const float kwx = wr * kx - wi * ky, kwy = wi * kx + wr * ky;
           const float qwx = wr * qx - wi * qy, qwy = wi * qx + wr * qy;
-          const float ep = __expf(gg[e] - s.ref[hr][cc]), em = __expf(s.ref[hr][cc] - gg[e]);
           kc[e] = ep * kwx, kc[e + 1] = ep * kwy;        // u k
           qc[e] = ep * qwx, qc[e + 1] = ep * qwy;        // u q
           kb[e] = em * kwx, kb[e + 1] = em * kwy;        // k / conj(u)
-          if (hr == 0) {  // write key of the second half's reference: e^{g_rho1 - g} e^{-i (Theta - Theta_rho1)} k
-            const float r1c = s.rot[1][cc], r1s = s.rot[1][cc + 1];
-            const float xr = cs * r1c + sn * r1s, xi = cs * r1s - sn * r1c;
-            const float e1 = __expf(s.ref[1][cc] - gg[e]);
-            kb1[e] = e1 * (xr * kx - xi * ky), kb1[e + 1] = e1 * (xi * kx + xr * ky);
+          const float zx = s.zr[hr][cc], zy = s.zr[hr][cc + 1];
+          qh[e] = zx * qc[e] - zy * qc[e + 1], qh[e + 1] = zx * qc[e + 1] + zy * qc[e];  // zeta q
+          bk[e] = br * (zx * kc[e] - zy * kc[e + 1]), bk[e + 1] = br * (zx * kc[e + 1] + zy * kc[e]);
+          const float ex = s.ec[hr][cc], ey = s.ec[hr][cc + 1];
+          kt[e] = ex * kb[e] - ey * kb[e + 1], kt[e + 1] = ex * kb[e + 1] + ey * kb[e];
+          if (hr == 0) {
+            const float ax = s.xk[0][cc], ay = s.xk[0][cc + 1];
+            const float bx = s.xk[1][cc], by = s.xk[1][cc + 1];
+            const float tx = ax * kb[e] - ay * kb[e + 1], ty = ax * kb[e + 1] + ay * kb[e];
+            kb1[e] = bx * tx - by * ty, kb1[e + 1] = bx * ty + by * tx;
           }
-          const float eg = __expf(gg[e]);
-          qh[e] = eg * (cs * qx + sn * qy), qh[e + 1] = eg * (cs * qy - sn * qx);   // zeta q
-          bk[e] = br * eg * (cs * kx + sn * ky), bk[e + 1] = br * eg * (cs * ky - sn * kx);
-          // conj(zeta_C / zeta) k = e^{g_C - g} e^{i (Theta_C - Theta)} k
-          const float tcr = s.rot[2][cc] * cs + s.rot[2][cc + 1] * sn;
-          const float tci = s.rot[2][cc + 1] * cs - s.rot[2][cc] * sn;
-          const float ec = __expf(s.ref[2][cc] - gg[e]);
-          kt[e] = ec * (tcr * kx - tci * ky), kt[e + 1] = ec * (tci * kx + tcr * ky);
         }
       } else {
+        float eps_ = 1.f, ems_ = 1.f;
+        if (!chan) {  // one factor per row
+          eps_ = __expf(sg - s.ref[hr][0]);
+          ems_ = __expf(s.ref[hr][0] - sg);
+        }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int cc = c0 + e;
-          const float d = gg[e] - s.ref[hr][cc];
-          const float ep = __expf(d), em = __expf(-d);
+          float ep = eps_, em = ems_;
+          if (chan) {
+            const float d = gg[e] - s.ref[hr][cc];
+            ep = __expf(d), em = __expf(-d);
+          }
           kc[e] = kv[e] * ep;
           qc[e] = qv[e] * ep;
           kb[e] = kv[e] * em;
-          if (hr == 0) kb1[e] = kv[e] * __expf(s.ref[1][cc] - gg[e]);
-          const float eg = __expf(gg[e]);
-          qh[e] = qv[e] * eg;
-          bk[e] = br * kv[e] * eg;
-          kt[e] = kv[e] * __expf(s.ref[2][cc] - gg[e]);
+          qh[e] = qc[e] * s.zr[hr][cc];
+          bk[e] = br * kc[e] * s.zr[hr][cc];
+          kt[e] = kb[e] * s.ec[hr][cc];
+          if (hr == 0) kb1[e] = kb[e] * s.xk[0][cc] * s.xk[1][cc];
         }
       }
 #pragma unroll
@@ -366,57 +425,65 @@ __global__ void __launch_bounds__(NTP, 2)
   __syncthreads();
   tc::fence_after_sync();
 
-  // ---- Grams on tcgen05: D0 = [K; Q]_h0 (Kb^rho0 rows 0..31)^T (M = 64, N = 32)
-  //                        D1 = [K; Q]_h1 (Kb^rho1 rows 0..63)^T (M = 64, N = 64)
+  // ---- Grams on tcgen05, one M = 128 product:
+  //   rows [K; Q] of the first half (0..63) and of the second half (64..127),
+  //   columns: the first reference's write keys of rows 0..31 (0..31) and the
+  //   second reference's of rows 0..63 (32..95).  Each half reads only the
+  //   columns of its own reference.
   if (tid == 0) {
-    const uint32_t id0 = tc::idesc_bf16(64, 32, false, false);
-    const uint32_t id1 = tc::idesc_bf16(64, 64, false, false);
-    const uint64_t a0 = tc::sdesc_kmaj(reinterpret_cast<const bf16*>(s.Q), D, 0);
-    const uint64_t a1 = tc::sdesc_kmaj(reinterpret_cast<const bf16*>(s.K), D, 0);
-    const uint64_t b0 = tc::sdesc_kmaj(reinterpret_cast<const bf16*>(s.KB), D, 0);
-    const uint64_t b1 = tc::sdesc_kmaj(reinterpret_cast<const bf16*>(s.KB + 4 * 2048), D, 0);
+    const uint32_t id = tc::idesc_bf16(128, 96, false, false);
+    const uint64_t a = tc::sdesc_kmaj(reinterpret_cast<const bf16*>(s.Q), D, 0);
+    const uint64_t bb = tc::sdesc_kmaj(reinterpret_cast<const bf16*>(s.KB), D, 0);
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      const uint32_t acc = ks > 0 ? 1u : 0u;
-      tc::mma(tb + 0, a0 + 16u * ks, b0 + 16u * ks, id0, acc);
-      tc::mma(tb + 32, a1 + 16u * ks, b1 + 16u * ks, id1, acc);
-    }
+    for (int ks = 0; ks < D / 16; ++ks) tc::mma(tb, a + 16u * ks, bb + 16u * ks, id, ks > 0 ? 1u : 0u);
     tc::commit(&s.bar_mma);
   }
   ok = prep_wait(&s.bar_mma, 0);
   if (!ok) break;
   // ---- A^T (fp32, [j][i]) into the gate tile's first half; M (bf16) to global.
-  // An M = 64 accumulator: row 16 (warp % 4) + lane for lanes 0..15 of the warp.
+  // Accumulator row = lane: quadrant 0 A rows of the first half, 1 its M rows,
+  // 2 and 3 those of the second half; warps w and w + 4 split the columns.
   float* At = reinterpret_cast<float*>(s.G);
   {
-    const int qd = warp & 3, t = lane;
-    const int row = 16 * qd + (t & 15);
-    const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
-    float d[64];
-    if (warp < 4) {
-      tmem_ld32(tb + lane_base + 0, d);                  // D0: 32 columns
-#pragma unroll
-      for (int e = 32; e < 64; ++e) d[e] = 0.f;
+    const int qd = warp & 3, side = warp >> 2, hq = qd >> 1;
+    const int i = 32 * hq + lane;                       // chunk row of A or M
+    const bool isA = (qd & 1) == 0;
+    const int w = hq ? 32 : 16;                         // columns this warp reads
+    float d[32];
+    const uint32_t ta = tb + ((uint32_t)(32 * qd) << 16) + (hq ? 32u : 0u) + (uint32_t)(side * w);
+    if (hq) {
+      tmem_ld32(ta, d);
     } else {
-      tmem_ld32(tb + lane_base + 32, d);                 // D1: 64 columns
-      tmem_ld32(tb + lane_base + 64, d + 32);
+      float t16[32];
+      tmem_ld32(ta, t16);  // 32 columns from the warp's start; the first 16 are its own
+#pragma unroll
+      for (int e = 0; e < 16; ++e) d[e] = t16[e];
     }
-    if (t < 16) {
-      const bool isA = row < 32;
-      const int i = (warp < 4 ? 0 : 32) + (row & 31);    // chunk row of A or M
-      if (isA) {
-        const float bi = s.beta[i];
+    const int j0 = side * w;                            // first column (row j of the chunk)
+    if (isA) {
+      const float bi = s.beta[i];
 #pragma unroll
-        for (int j = 0; j < 64; ++j) At[j * C + i] = (j < i) ? bi * d[j] : 0.f;
-      } else {
-        bf16* Mg = sv.M + cb * C * C;
+      for (int e = 0; e < 32; ++e)
+        if (e < w) At[(j0 + e) * C + i] = (j0 + e < i) ? bi * d[e] : 0.f;
+      if (hq == 0 && side == 1) {
+#pragma unroll 8
+        for (int j = 32; j < C; ++j) At[j * C + i] = 0.f;
+      }
+    } else {
+      bf16* Mg = sv.M + cb * C * C;
 #pragma unroll
-        for (int j8 = 0; j8 < 8; ++j8) {
+      for (int j8 = 0; j8 < 4; ++j8) {
+        if (8 * j8 < w) {
           float f[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = (8 * j8 + e <= i) ? d[8 * j8 + e] : 0.f;
-          *reinterpret_cast<uint4*>(Mg + ct_off(i, 8 * j8, C)) = pack8(f);
+          for (int e = 0; e < 8; ++e) f[e] = (j0 + 8 * j8 + e <= i) ? d[8 * j8 + e] : 0.f;
+          *reinterpret_cast<uint4*>(Mg + ct_off(i, j0 + 8 * j8, C)) = pack8(f);
         }
+      }
+      if (hq == 0 && side == 1) {
+        const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j8 = 4; j8 < 8; ++j8) *reinterpret_cast<uint4*>(Mg + ct_off(i, 8 * j8, C)) = pack8(z);
       }
     }
   }
@@ -428,22 +495,28 @@ __global__ void __launch_bounds__(NTP, 2)
   }
   tc::fence_before_sync();
   __syncthreads();
-  // ---- T = (I + A)^{-1}: thread j < 64 forward-substitutes column j in fp32,
-  //      T[i][j] = delta_ij - sum_{m < i} A[i][m] T[m][j], all rows in registers
-  //      (the updates of one step are independent), then T = T_hi + T_lo in bf16.
-  bf16* Thi = reinterpret_cast<bf16*>(s.G + 2 * kBox);
-  bf16* Tlo = reinterpret_cast<bf16*>(s.G + 3 * kBox);
+  // ---- T = (I + A)^{-1} in fp32, by blocks of 32:
+  //   T11 = (I + A11)^{-1}, T22 = (I + A22)^{-1} (thread j < 64 forward-substitutes
+  //   one column of one of them, all its rows in registers), then
+  //   T21 = -T22 (A21 T11) by two 32 x 32 products on all threads;
+  //   finally T = T_hi + T_lo in bf16, the tcgen05 operand.
+  // fp32 T, row stride TLD (16-byte rows of 8 consecutive rows in distinct banks),
+  // over the Gram operands (read); Y = A21 T11, row stride 33
+  constexpr int TLD = C + 4;
+  unsigned char* const qk = reinterpret_cast<unsigned char*>(&s) + offsetof(PrepSmem, Q);
+  float* Tf = reinterpret_cast<float*>(qk);
+  float* Yb = reinterpret_cast<float*>(qk + C * TLD * 4);
   if (tid < C) {
-    const int j = tid;
-    float acc[C];
+    const int blk = tid >> 5, j = tid & 31, o = 32 * blk;
+    float acc[32];
 #pragma unroll
-    for (int i = 0; i < C; ++i) acc[i] = (i == j) ? 1.f : 0.f;
+    for (int i = 0; i < 32; ++i) acc[i] = (i == j) ? 1.f : 0.f;
 #pragma unroll
-    for (int m = 0; m < C - 1; ++m) {
+    for (int m = 0; m < 31; ++m) {
       const float tm = acc[m];
-      const float* arow = At + m * C;  // A[.][m]
+      const float* arow = At + (o + m) * C + o;  // A[o + .][o + m]
 #pragma unroll
-      for (int i4 = (m + 1) & ~3; i4 < C; i4 += 4) {
+      for (int i4 = (m + 1) & ~3; i4 < 32; i4 += 4) {
         const float4 a = *reinterpret_cast<const float4*>(arow + i4);
         if (i4 + 0 > m) acc[i4 + 0] -= a.x * tm;
         if (i4 + 1 > m) acc[i4 + 1] -= a.y * tm;
@@ -452,13 +525,56 @@ __global__ void __launch_bounds__(NTP, 2)
       }
     }
 #pragma unroll
-    for (int i = 0; i < C; ++i) {
-      const bf16 hi = __float2bfloat16_rn(acc[i]);
-      const bf16 lo = __float2bfloat16_rn(acc[i] - __bfloat162float(hi));
-      const int o = ((i >> 3) * 8 + (j >> 3)) * 64 + (i & 7) * 8 + (j & 7);
-      Thi[o] = hi;
-      Tlo[o] = lo;
+    for (int i = 0; i < 32; ++i) Tf[(o + i) * TLD + o + j] = acc[i];
+    if (blk == 0) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) Tf[i * TLD + 32 + j] = 0.f;
     }
+  }
+  __syncthreads();
+  {
+    // Y = A21 T11: lane -> row ti of the second half, warp -> columns tj + 8 k
+    const int ti = tid & 31, tj = tid >> 5;
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int m = 0; m < 32; ++m) {
+      const float a = At[m * C + 32 + ti];
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) y[k4] += a * Tf[m * TLD + tj + 8 * k4];
+    }
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4) Yb[ti * 33 + tj + 8 * k4] = y[k4];
+  }
+  __syncthreads();
+  {
+    // T21 = -T22 Y: lane -> column tj, warp -> rows ti + 8 k of the second half
+    const int tj = tid & 31, ti = tid >> 5;
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int m = 0; m < 32; ++m) {
+      const float yv = Yb[m * 33 + tj];
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) y[k4] += Tf[(32 + ti + 8 * k4) * TLD + 32 + m] * yv;
+    }
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4) Tf[(32 + ti + 8 * k4) * TLD + tj] = -y[k4];
+  }
+  __syncthreads();
+  bf16* Thi = reinterpret_cast<bf16*>(s.G + 2 * kBox);
+  bf16* Tlo = reinterpret_cast<bf16*>(s.G + 3 * kBox);
+  for (int idx = tid; idx < C * C / 8; idx += NTP) {  // core-tiled [i][j], 16 bytes per thread
+    const int i = ct_row(idx, C), j8 = ct_col(idx, C);
+    float hi[8], lo[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float t = Tf[i * TLD + j8 + e];
+      hi[e] = __bfloat162float(__float2bfloat16_rn(t));
+      lo[e] = t - hi[e];
+    }
+    const uint4 vh = pack8(hi);
+    *reinterpret_cast<uint4*>(Thi + 8 * idx) = vh;
+    *reinterpret_cast<uint4*>(Tlo + 8 * idx) = pack8(lo);
+    *reinterpret_cast<uint4*>(sv.T + cb * C * C + 8 * idx) = vh;
   }
   tc::fence_smem_to_async();
   tc::fence_before_sync();
@@ -480,10 +596,6 @@ __global__ void __launch_bounds__(NTP, 2)
     }
     tc::commit(&s.bar_mma);
   }
-  // T (bf16, the high part) to the saved buffer while they run
-  for (int idx = tid; idx < C * C / 8; idx += NTP)
-    *reinterpret_cast<uint4*>(sv.T + cb * C * C + 8 * idx) =
-        *reinterpret_cast<const uint4*>(Thi + 8 * idx);
   ok = prep_wait(&s.bar_mma, 1);
   if (!ok) break;
   // ---- W (warps 0-3) and U' (warps 4-7), rows 16 (warp % 4) + lane, lanes 0..15
@@ -570,7 +682,7 @@ cudaError_t launch_prep(const Problem& p, const bf16* q, const bf16* k, const bf
   const double flops = nb * (2.0 * C * 96 * D + C * C * C / 3.0 + 2.0 * 2 * 2 * C * C * D);
   prof_begin(kKTcIntraFwd, io, bytes, flops, st);
   kern<<<dim3(p.NC, p.H, p.B), NTP, sm, st>>>(p, mq, mk, mv, mg, chan ? nullptr : g, beta, sv,
-                                             device_error_word());
+                                             device_error_word(), 2 * sm_count());
   e = cudaGetLastError();
   prof_end(st);
   return e;

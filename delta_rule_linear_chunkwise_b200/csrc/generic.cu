@@ -2,19 +2,18 @@
 // backward, for any supported head size and for fp32 or bf16 storage.
 //
 // Every product here is an fp32 FMA loop over shared memory; this path serves
-// fp32 inputs (whose tolerance rules out bf16 tensor-core operands) and is the
-// structural template of the tensor-core path.  Chunk math (per head, chunk of
-// C = 64 rows, gamma = inclusive within-chunk cumulative log-gate, r = centre
-// row of the chunk's valid rows):
-//   K^c = k e^{gamma - gamma_r},  Kb^c = k e^{gamma_r - gamma},  Q^c = q e^{gamma - gamma_r}
-//   A = diag(beta) strict_tril(K^c Kb^c^T),  M = tril(Q^c Kb^c^T)      (centred Grams)
+// fp32 inputs (whose tolerance rules out bf16 tensor-core operands) and every
+// head size the tensor-core path does not take.  Chunk math (per head, chunk of
+// C = 64 rows, gamma = inclusive within-chunk cumulative log-gate):
+//   A_ij = beta_i sum_c k_ic k_jc e^{gamma_ic - gamma_jc} (j < i),
+//   M_ij = sum_c q_ic k_jc e^{gamma_ic - gamma_jc} (j <= i)           (decayed Grams)
 //   T = (I + A)^{-1};  W = T diag(beta) (k e^{gamma});  U' = T diag(beta) V
 //   U = U' - W S^T;  O = (q e^{gamma}) S^T + M U
 //   S <- S Diag(e^{gamma_C}) + U^T (k e^{gamma_C - gamma})
-// The centring keeps every exponent of a Gram factor within half the chunk's
-// decay range (the "centered matrix contractions" of the ReWY abstract); the
-// products M and A depend only on gamma_i - gamma_j, so the centre row drops
-// out of the result.
+// Each pair's factor e^{gamma_i - gamma_j} (j <= i) is evaluated directly, so it
+// is at most 1 and never overflows whatever the decay; where it underflows the
+// exact term is below fp32 resolution.  The backward's gate-scaled products
+// are formed the same way.
 
 #include "dr_common.cuh"
 
@@ -41,7 +40,6 @@ constexpr int C = kC;
 constexpr int NT = kThreads;
 constexpr int LDC = C + 1;  // padded stride of C x C tiles
 
-__device__ __forceinline__ int centre_row(int nvalid) { return (nvalid - 1) / 2; }
 
 // gamma of row i, key channel c (gk == 1: scalar gate broadcast).
 __device__ __forceinline__ float gam_at(const float* sG, int gk, int i, int c) {
@@ -66,10 +64,9 @@ __global__ void __launch_bounds__(NT) k_intra_fwd(Problem p, const TIn* __restri
   const size_t cb = chunk_id(p, b, h, n);
 
   float* sK = sm;              // [C][LD] raw k
-  float* sQc = sK + C * LD;    // [C][LD] q e^{gamma-gamma_r}, later beta k e^{gamma}
-  float* sKc = sQc + C * LD;   // [C][LD] k e^{gamma-gamma_r}, later beta v
-  float* sKb = sKc + C * LD;   // [C][LD] k e^{gamma_r-gamma}
-  float* sA = sKb + C * LD;    // [C][LDC]
+  float* sQc = sK + C * LD;    // [C][LD] raw q, later beta k e^{gamma}
+  float* sKc = sQc + C * LD;   // [C][LD] beta v
+  float* sA = sKc + C * LD;    // [C][LDC]
   float* sT = sA + C * LDC;    // [C][LDC]
   float* sG = sT + C * LDC;    // [C][gk]
   float* sB = sG + C * gk;     // [C]
@@ -105,28 +102,33 @@ __global__ void __launch_bounds__(NT) k_intra_fwd(Problem p, const TIn* __restri
   __syncthreads();
   for (int idx = tid; idx < C * gk; idx += NT) ws.gam[cb * C * gk + idx] = sG[idx];
 
-  const int r = centre_row(nvalid);
   for (int idx = tid; idx < C * dk; idx += NT) {
     const int i = idx / dk, c = idx % dk;
-    const float gi = gam_at(sG, gk, i, c), gr = gam_at(sG, gk, r, c);
-    const float ep = expf(gi - gr), em = expf(gr - gi);
-    const float kv = sK[i * LD + c];
-    const float qv = (i < nvalid) ? load_f(q + row_id(p, b, t0 + i, h) * dk + c) : 0.f;
-    sQc[i * LD + c] = qv * ep;
-    sKc[i * LD + c] = kv * ep;
-    sKb[i * LD + c] = kv * em;
+    sQc[i * LD + c] = (i < nvalid) ? load_f(q + row_id(p, b, t0 + i, h) * dk + c) : 0.f;
   }
   __syncthreads();
 
-  // Gram products: A (strictly lower, beta-scaled) and M (inclusive lower).
+  // Gram products: A (strictly lower, beta-scaled) and M (inclusive lower),
+  // with each pair's factor e^{gamma_i - gamma_j} <= 1 evaluated directly.
   for (int idx = tid; idx < C * C; idx += NT) {
     const int i = idx / C, j = idx % C;
     float a = 0.f, m = 0.f;
     if (j <= i) {
-      for (int c = 0; c < dk; ++c) {
-        const float kb = sKb[j * LD + c];
-        a += sKc[i * LD + c] * kb;
-        m += sQc[i * LD + c] * kb;
+      if (gk == 1) {
+        for (int c = 0; c < dk; ++c) {
+          const float kj = sK[j * LD + c];
+          a += sK[i * LD + c] * kj;
+          m += sQc[i * LD + c] * kj;
+        }
+        const float f = expf(sG[i] - sG[j]);
+        a *= f;
+        m *= f;
+      } else {
+        for (int c = 0; c < dk; ++c) {
+          const float kj = sK[j * LD + c] * expf(sG[i * gk + c] - sG[j * gk + c]);
+          a += sK[i * LD + c] * kj;
+          m += sQc[i * LD + c] * kj;
+        }
       }
     }
     sA[i * LDC + j] = (j < i) ? sB[i] * a : 0.f;
@@ -440,13 +442,11 @@ __global__ void __launch_bounds__(NT) k_intra_bwd(Problem p, const TIn* __restri
   const int dk = p.dk, dv = p.dv, gk = p.gk;
   const int LD = (dk > dv ? dk : dv) + 1;
   const int t0 = n * C, nvalid = min(C, p.T - t0);
-  const int r = centre_row(nvalid);
   const size_t cb = chunk_id(p, b, h, n);
-  float* sKc = sm;               // [C][LD] k e^{gamma-gamma_r}
-  float* sKb = sKc + C * LD;     // [C][LD] k e^{gamma_r-gamma}
-  float* sM1 = sKb + C * LD;     // [C][LDC] T
+  float* sKc = sm;               // [C][LD] raw k
+  float* sM1 = sKc + C * LD;     // [C][LDC] T
   float* sM2 = sM1 + C * LDC;    // [C][LDC] dM, later dA
-  float* sR0 = sM2 + C * LDC;    // [C][LD] dO | Q^c | Lambda half
+  float* sR0 = sM2 + C * LDC;    // [C][LD] dO | raw q | Lambda half
   float* sR1 = sR0 + C * LD;     // [C][LD] U | dX half | X half
   float* sG = sR1 + C * LD;      // [C][gk]
   float* sB = sG + C * gk;       // [C]
@@ -477,42 +477,43 @@ __global__ void __launch_bounds__(NT) k_intra_bwd(Problem p, const TIn* __restri
     sM2[i * LDC + j] = acc;
   }
   __syncthreads();
-  // P1: centred factors; Q^c goes to sR0.
+  // P1: raw q into sR0 and raw k into sKc; each gate-scaled product below forms
+  // its pair factor e^{gamma_i - gamma_j} (<= 1) directly.
   for (int idx = tid; idx < C * dk; idx += NT) {
     const int i = idx / dk, c = idx % dk;
-    const float gi = gam_at(sG, gk, i, c), gr = gam_at(sG, gk, r, c);
     float kv = 0.f, qv = 0.f;
     if (i < nvalid) {
       const size_t rr = row_id(p, b, t0 + i, h) * dk + c;
       kv = load_f(k + rr);
       qv = load_f(q + rr);
     }
-    const float ep = expf(gi - gr), em = expf(gr - gi);
-    sR0[i * LD + c] = qv * ep;
-    sKc[i * LD + c] = kv * ep;
-    sKb[i * LD + c] = kv * em;
+    sR0[i * LD + c] = qv;
+    sKc[i * LD + c] = kv;
   }
   __syncthreads();
   if (tid < dk) {
     const int c = tid;
-    const float gr = gam_at(sG, gk, r, c);
     for (int i = 0; i < C; ++i) {
-      float dqm = 0.f;
-      for (int j = 0; j <= i; ++j) dqm += sM2[i * LDC + j] * sKb[j * LD + c];
+      // dq of the intra-chunk term: sum_{j <= i} dM_ij k_j e^{gamma_i - gamma_j}
       const float gi = gam_at(sG, gk, i, c);
+      float dqm = 0.f;
+      for (int j = 0; j <= i; ++j)
+        dqm += sM2[i * LDC + j] * sKc[j * LD + c] * expf(gi - gam_at(sG, gk, j, c));
       const float eg = expf(gi);
       const float dqs = ws.dQs[(cb * C + i) * dk + c];
       ws.dQs[(cb * C + i) * dk + c] = 0.f;  // reused below as this column's dbeta terms
-      const float qv = (i < nvalid) ? load_f(q + row_id(p, b, t0 + i, h) * dk + c) : 0.f;
-      if (i < nvalid) store_f(dq + row_id(p, b, t0 + i, h) * dk + c, expf(gi - gr) * dqm + eg * dqs);
-      dg_acc[i * dk + c] = sR0[i * LD + c] * dqm + qv * eg * dqs;
+      const float qv = sR0[i * LD + c];
+      if (i < nvalid) store_f(dq + row_id(p, b, t0 + i, h) * dk + c, dqm + eg * dqs);
+      dg_acc[i * dk + c] = qv * dqm + qv * eg * dqs;
     }
     for (int j = 0; j < C; ++j) {
-      float dkbm = 0.f;
-      for (int i = j; i < C; ++i) dkbm += sM2[i * LDC + j] * sR0[i * LD + c];
+      // the write-key side: sum_{i >= j} dM_ij q_i e^{gamma_i - gamma_j}
       const float gj = gam_at(sG, gk, j, c);
-      dk_acc[j * dk + c] = expf(gr - gj) * dkbm;
-      dg_acc[j * dk + c] -= sKb[j * LD + c] * dkbm;
+      float dkbm = 0.f;
+      for (int i = j; i < C; ++i)
+        dkbm += sM2[i * LDC + j] * sR0[i * LD + c] * expf(gam_at(sG, gk, i, c) - gj);
+      dk_acc[j * dk + c] = dkbm;
+      dg_acc[j * dk + c] -= sKc[j * LD + c] * dkbm;
     }
   }
   // P2: Lambda = T^T [dU | dW]; dA = -strict_tril(Lambda X^T), X = [U' | W].
@@ -578,19 +579,22 @@ __global__ void __launch_bounds__(NT) k_intra_bwd(Problem p, const TIn* __restri
     sM2[i * LDC + j] -= acc;
   }
   __syncthreads();
-  // P4: A = diag(beta) strict_tril(K^c Kb^c^T):
-  //   x = dA Kb^c;  dK^c += beta x;  dKb^c += dA^T (beta K^c);  dbeta += K^c . x
+  // P4: A_ij = beta_i sum_c k_ic k_jc e^{gamma_ic - gamma_jc} (j < i):
+  //   x_i = sum_{j<i} dA_ij k_j e^{gamma_i - gamma_j},  y_i = sum_{i2>i} dA_i2,i beta_i2 k_i2 e^{gamma_i2 - gamma_i}
+  //   dk += beta x + y;  dgamma += k (beta x - y);  dbeta += k . x
   if (tid < dk) {
     const int c = tid;
-    const float gr = gam_at(sG, gk, r, c);
     for (int i = 0; i < C; ++i) {
-      float x = 0.f, y = 0.f;
-      for (int j = 0; j < i; ++j) x += sM2[i * LDC + j] * sKb[j * LD + c];
-      for (int i2 = i + 1; i2 < C; ++i2) y += sM2[i2 * LDC + i] * sB[i2] * sKc[i2 * LD + c];
       const float gi = gam_at(sG, gk, i, c);
-      dk_acc[i * dk + c] += expf(gi - gr) * sB[i] * x + expf(gr - gi) * y;
-      dg_acc[i * dk + c] += sKc[i * LD + c] * sB[i] * x - sKb[i * LD + c] * y;
-      ws.dQs[(cb * C + i) * dk + c] += sKc[i * LD + c] * x;
+      float x = 0.f, y = 0.f;
+      for (int j = 0; j < i; ++j)
+        x += sM2[i * LDC + j] * sKc[j * LD + c] * expf(gi - gam_at(sG, gk, j, c));
+      for (int i2 = i + 1; i2 < C; ++i2)
+        y += sM2[i2 * LDC + i] * sB[i2] * sKc[i2 * LD + c] * expf(gam_at(sG, gk, i2, c) - gi);
+      const float kv = sKc[i * LD + c];
+      dk_acc[i * dk + c] += sB[i] * x + y;
+      dg_acc[i * dk + c] += kv * (sB[i] * x - y);
+      ws.dQs[(cb * C + i) * dk + c] += kv * x;
     }
     // P5: state-update key term Kt = k e^{gamma_C - gamma}, then reverse cumsum.
     const float gC = gam_at(sG, gk, C - 1, c);
@@ -649,7 +653,7 @@ __global__ void __launch_bounds__(NT) k_intra_bwd(Problem p, const TIn* __restri
 
 size_t intra_fwd_smem(const Problem& p) {
   const int LD = (p.dk > p.dv ? p.dk : p.dv) + 1;
-  return sizeof(float) * ((size_t)4 * C * LD + 2 * C * LDC + C * p.gk + C);
+  return sizeof(float) * ((size_t)3 * C * LD + 2 * C * LDC + C * p.gk + C);
 }
 size_t scan_smem(const Problem& p, int BV) {
   const int LDk = p.dk + 1;
@@ -661,7 +665,7 @@ size_t state_grads_smem(const Problem& p) {
 }
 size_t intra_bwd_smem(const Problem& p) {
   const int LD = (p.dk > p.dv ? p.dk : p.dv) + 1;
-  return sizeof(float) * ((size_t)4 * C * LD + 2 * C * LDC + C * p.gk + 3 * C);
+  return sizeof(float) * ((size_t)3 * C * LD + 2 * C * LDC + C * p.gk + 3 * C);
 }
 
 int pick_bv(const Problem& p) { return (p.dv % 32 == 0) ? 32 : 16; }

@@ -78,11 +78,14 @@ def test_beta_zero_keeps_state_up_to_decay():
     _check(w, inp, dST=random_state(w, seed=7))
 
 
-def test_strong_decay_gates():
-    """Per-channel gates with much stronger decay than the workloads
-    (g ~ logsigmoid(N(-1, 1)), i.e. alpha ~ 0.27 per token)."""
-    w = WORKLOADS["kda_bf16_b4h16t8192"].with_(name="strong_decay", B=1, H=2, T=150,
-                                               g_mean=-1.0, s0_std=0.3, dtype="f32")
+@pytest.mark.parametrize("mu", [-1.0, -3.0])
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_strong_decay_gates(gate, mu):
+    """fp32 storage (the CUDA-core path) with gates decaying much faster than the
+    workloads' (g ~ logsigmoid(N(mu, 1)): alpha ~ 0.25 and ~ 0.05 per token)."""
+    w = WORKLOADS["kda_bf16_b4h16t8192"].with_(name=f"strong_decay_{gate}_{mu}", B=1, H=2,
+                                               T=150, g_mean=mu, s0_std=0.3, dtype="f32",
+                                               gate=gate, dk=64, dv=64)
     _check(w, make_inputs(w), dST=random_state(w, seed=8))
 
 
