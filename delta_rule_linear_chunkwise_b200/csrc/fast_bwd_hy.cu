@@ -1,9 +1,10 @@
 // fast_bwd_hy.cu -- chunk-parallel backward with the products on tcgen05 and
 // the element-wise work on all 16 warps (bf16 storage, d_k = d_v = 128, C = 64).
 //
-// One CTA per (b, h, chunk).  From the chunk's saved tiles (T, W, U', the
-// chunk-start state S = h_n, the pseudo-values U) and the state-gradient scan's
-// dU and dS' (the gradient of the chunk's end state):
+// Persistent, one CTA per SM, looping over the (b, h, chunk) tiles.  From the
+// chunk's saved tiles (T, W, U', the chunk-start state S = h_n, the
+// pseudo-values U) and the state-gradient scan's dU and dS' (the gradient of
+// the chunk's end state):
 //   level 1  dQs = dO S, dW = -dU S, dKt = U dS', dM = tril(dO U^T)  (its diagonal
 //            kept apart in fp32: it enters dq and dk with the factor 1 and cancels in dg)
 //   level 2  Lambda = T^T [dU | dW]             (dv = diag(beta) Lambda_U)
@@ -13,7 +14,7 @@
 //            G_j  = sum_{i>=j} (dM_ij q_i + dA_ij beta_i k_i) e^{g_i - g_j}
 //            (g: the within-chunk cumulative log-gate of each key channel)
 // which give dq, dk, dgamma and dbeta in a register epilogue, then the gate's
-// reverse cumulative sum and the Kaczmarz chain rule.  The chunk correction is
+// reverse cumulative sum (in registers) and the Kaczmarz chain rule.  The chunk correction is
 // differentiated as the triangular residual system (I + A)[U' | W] = diag(beta)
 // [V | k e^g] (ReWY abstract): one transposed triangular product (level 2), no
 // adjoint of the inverse.
@@ -42,6 +43,11 @@
 // the conjugate factors, d/dg of a pair is Re(.) and d/dTheta is Im(.) of the
 // same products (with the write-key and chunk-end terms of opposite sign in g).
 //
+// Overlap: the level-1 tiles of the CTA's next chunk (dO, dU, U, S, dS', T;
+// 120 KB) are loaded while the epilogue of this one runs, into the tiles that
+// level 4 has released, so a chunk starts with its first products; q, k and the
+// gate (which the epilogue still reads) load under level 1.
+//
 // Each level is a set of tcgen05.mma (M = 64, operands in shared memory in the
 // canonical core-matrix layout, fp32 accumulators in tensor memory) issued by
 // one thread.  An M = 64 accumulator occupies lanes 16 q .. 16 q + 15 of each
@@ -66,7 +72,6 @@ namespace {
 constexpr int C = 64, D = 128;
 constexpr int LDD = D + 8;
 constexpr int NTB = 512;
-constexpr int LDG = D + 4;  // fp32 row stride of the dgamma tile (fragment stores conflict-free)
 constexpr uint32_t kSpinHy = 1u << 22;
 // Polls of the injected wait (dr_inject_timeout): short, so the test that
 // drives the timeout path ends within milliseconds.
@@ -118,14 +123,13 @@ struct HySmem {
   float xk[2 * D];
   float xq[2 * D];
   float dmd[C];      // the diagonal of dM (fp32), added outside the level-4 products
+  float blk[4 * D];  // dgamma totals of each 16-row block (scalar gate: row partial sums)
   uint64_t bar;
+  uint64_t full;    // the chunk tiles' bulk copies
   uint64_t never;   // fault injection: a barrier that nothing ever arrives on
   uint32_t tmem;
 };
 
-static_assert(offsetof(HySmem, SD) == offsetof(HySmem, SS) + sizeof(bf16) * D * D &&
-                  sizeof(float) * C * LDG <= sizeof(bf16) * 2 * D * D,
-              "the padded dgamma tile spans the adjacent S and dS' tiles");
 static_assert(sizeof(bf16) * C * D <= sizeof(bf16) * 2 * kXElems, "U fits the X-tile region");
 
 // --- complex helpers (a key pair as x + i y) -------------------------------
@@ -220,13 +224,11 @@ __global__ void __launch_bounds__(NTB, 1)
                    int inject_timeout) {
   extern __shared__ __align__(1024) unsigned char smraw[];
   HySmem& s = *reinterpret_cast<HySmem*>(smraw);
-  const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, gk = p.gk;
   const int rb = warp & 3, qt = warp >> 2;
   const int hf = rb >> 1;  // the half of this warp's fragment rows
   const int lr = lane >> 2, lc = 2 * (lane & 3);
-  const int t0 = n * C, nvalid = min(C, p.T - t0);
-  const size_t cb = chunk_id(p, b, h, n);
   bf16* const sLU = s.SS;          // Lambda_U, after the first level
   bf16* const sLW = s.SS + C * D;  // Lambda_W
   bf16* const sW = s.SD;           // W, U' for the third level
@@ -242,45 +244,132 @@ __global__ void __launch_bounds__(NTB, 1)
   bf16* const B0 = s.SS;               // beta_i (zeta_i / zeta_rho0) k_i, rows 0..63
   bf16* const B1 = s.TT;               // beta_i (zeta_i / zeta_rho1) k_i, rows 32..63
 
-  // Loads in three cp.async groups, in the order of first use:
-  //   1: gate, q, k   2: dO, dU, U, S, dS', T (first level)   3: W, U' (third level)
-  for (int idx = tid; idx < C * (D / 8); idx += NTB) {
-    const int i = idx >> 4, j = idx & 15;
-    const bool ok = i < nvalid;
-    const size_t rr = row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 8;
-    frag::cp16(s.QR + i * LDD + j * 8, q + rr, ok);
-    frag::cp16(s.k + i * LDD + j * 8, k + rr, ok);
-  }
-  if (gk == D) {
-    for (int idx = tid; idx < C * (D / 4); idx += NTB) {
-      const int i = idx >> 5, j = idx & 31;
-      const bool ok = i < nvalid && p.gate != kGateNone;
-      frag::cp16(s.G + gsw(i, j * 4), g + row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 4, ok);
+  // The level-1 tiles of chunk L (launch order: chunks, then heads, then
+  // batches): dU, U, S, dS' and T by bulk copies, one from lane 0 of each of
+  // warps 1..5, completing on `full` (whose transaction count thread 0 has set
+  // before the barrier that precedes them: expect_tiles), and dO by cp.async from
+  // every thread (one group).  Issued one chunk ahead, into the tiles level 4
+  // has released.
+  constexpr uint32_t kTileTx = sizeof(bf16) * (2 * C * D + 2 * D * D + C * C);
+  auto issue_tiles = [&](int n, int h, int b) {
+    const int t0 = n * C, nvalid = min(C, p.T - t0);
+    const size_t cb = chunk_id(p, b, h, n);
+    if (lane == 0 && warp >= 1 && warp <= 5) {
+      if (warp == 1) tc::bulk_g2s(s.DU, dUg + cb * C * D, sizeof(bf16) * C * D, &s.full);
+      if (warp == 2) tc::bulk_g2s(s.UU, Ug + cb * C * D, sizeof(bf16) * C * D, &s.full);
+      if (warp == 3) tc::bulk_g2s(s.SS, hst + cb * D * D, sizeof(bf16) * D * D, &s.full);
+      if (warp == 4) tc::bulk_g2s(s.SD, dhst + cb * D * D, sizeof(bf16) * D * D, &s.full);
+      if (warp == 5) tc::bulk_g2s(s.TT, Tg + cb * C * C, sizeof(bf16) * C * C, &s.full);
     }
-  } else if (tid < C) {
-    s.G[tid] = (tid < nvalid && p.gate != kGateNone) ? g[row_id(p, b, t0 + tid, h)] : 0.f;
-  }
-  if (tid < C) {
-    s.beta[tid] = beta[cb * C + tid];
-    s.knorm[tid] = knorm_g[cb * C + tid];
-  }
-  frag::cp_commit();
-  tc::cp_core_tile<NTB>(s.DO, dO + row_id(p, b, t0, h) * D, (size_t)p.H * D, C, D, nvalid, tid);
-  cp_linear<NTB>(s.DU, dUg + cb * C * D, C * D, tid);
-  cp_linear<NTB>(s.UU, Ug + cb * C * D, C * D, tid);
-  cp_linear<NTB>(s.SS, hst + cb * D * D, D * D, tid);
-  cp_linear<NTB>(s.SD, dhst + cb * D * D, D * D, tid);
-  cp_linear<NTB>(s.TT, Tg + cb * C * C, C * C, tid);
-  frag::cp_commit();
-  // the zero block of the dA tile (outside the U region)
-  for (int idx = tid; idx < C * C / 16; idx += NTB)
-    *reinterpret_cast<uint4*>(XA + C * C / 2 + 8 * idx) = make_uint4(0, 0, 0, 0);
+    tc::cp_core_tile<NTB>(s.DO, dO + row_id(p, b, t0, h) * D, (size_t)p.H * D, C, D, nvalid, tid);
+    frag::cp_commit();
+  };
+
   if (warp == 0) tc::tmem_alloc(&s.tmem, 512);
   if (tid == 0) {
     tc::mbar_init(&s.bar, 1);
     tc::mbar_init(&s.never, 1);
+    tc::mbar_init(&s.full, 1);
+    tc::fence_mbar_init();
   }
-  frag::cp_wait<1>();
+  // the zero block of the dA tile (outside the U region; nothing overwrites it)
+  for (int idx = tid; idx < C * C / 16; idx += NTB)
+    *reinterpret_cast<uint4*>(XA + C * C / 2 + 8 * idx) = make_uint4(0, 0, 0, 0);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tb = s.tmem;
+  bool ok = true, pending = false;
+  uint32_t fph = 0;  // phase of `full`
+  // this CTA's chunks: (n, h, b) from blockIdx.x, then every gridDim.x-th in
+  // launch order (advanced without divisions)
+  int n = blockIdx.x % p.NC, h = (blockIdx.x / p.NC) % p.H, b = blockIdx.x / (p.NC * p.H);
+  auto advance = [&](int& an, int& ah, int& ab) {
+    an += gridDim.x;
+    while (an >= p.NC) {
+      an -= p.NC;
+      if (++ah == p.H) {
+        ah = 0;
+        ++ab;
+      }
+    }
+  };
+  int nn = n, nh = h, nb = b;  // the chunk after this one
+  advance(nn, nh, nb);
+  if (b < p.B) {
+    if (tid == 0) tc::mbar_arrive_expect_tx(&s.full, kTileTx);
+    __syncthreads();
+    issue_tiles(n, h, b);
+    pending = true;
+  }
+  // Persistent: one CTA per SM.  A bounded wait that gives up leaves the loop (break).
+  for (bool first = true; b < p.B; n = nn, h = nh, b = nb, advance(nn, nh, nb), first = false) {
+  const int t0 = n * C, nvalid = min(C, p.T - t0);
+  const size_t cb = chunk_id(p, b, h, n);
+  frag::cp_wait<0>();  // dO
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  ok = hy_wait(&s.full, (int)fph);
+  if (!ok) break;
+  pending = false;
+  fph ^= 1u;
+
+  // Fault injection (dr_inject_timeout): wait, with a short limit, on a barrier
+  // that nothing arrives on.  Every copy has landed and no MMA has been issued,
+  // so the timeout path below leaves nothing in flight.
+  if (inject_timeout && first) {
+    ok = hy_wait(&s.never, 0, kSpinInjected);
+    if (!ok) break;
+  }
+
+  // ---- level 1 (tensor memory): dQs = dO S, dW' = dU S, dKt = U dS', dM = dO U^T
+  // (descriptors are built once; a k-step adds its byte offset / 16 to the start
+  // address field, which stays below 2^14 for any shared-memory address)
+  if (tid == 0) {
+    const uint32_t id128 = tc::idesc_bf16(64, 128, false, true);
+    const uint32_t id64 = tc::idesc_bf16(64, 64, false, false);
+    const uint64_t aDO = tc::sdesc_kmaj(s.DO, D, 0), aDU = tc::sdesc_kmaj(s.DU, D, 0);
+    const uint64_t aUU = tc::sdesc_kmaj(s.UU, D, 0);
+    const uint64_t bSS = tc::sdesc_mnmaj(s.SS, D, 0), bSD = tc::sdesc_mnmaj(s.SD, D, 0);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const uint32_t acc = ks > 0 ? 1u : 0u;
+      const uint64_t ka = 16u * ks, kb = 256u * ks;  // K-major / MN-major k-step, 16-byte units
+      mma_step(tb + T_ZQ, aDO + ka, bSS + kb, id128, acc);
+      mma_step(tb + T_ADW, aDU + ka, bSS + kb, id128, acc);
+      mma_step(tb + T_AKT, aUU + ka, bSD + kb, id128, acc);
+      mma_step(tb + T_ADM, aDO + ka, aUU + ka, id64, acc);
+    }
+    tc::commit(&s.bar);
+  }
+  // q, k, the gate, beta and ||k||^2 of this chunk by warps 1..15 (warp 0 issues
+  // level 1)
+  if (warp > 0) {
+    const int lt = tid - 32;
+    constexpr int NL = NTB - 32;
+    for (int idx = lt; idx < C * (D / 8); idx += NL) {
+      const int i = idx >> 4, j = idx & 15;
+      const bool ok = i < nvalid;
+      const size_t rr = row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 8;
+      frag::cp16(s.QR + i * LDD + j * 8, q + rr, ok);
+      frag::cp16(s.k + i * LDD + j * 8, k + rr, ok);
+    }
+    if (gk == D) {
+      for (int idx = lt; idx < C * (D / 4); idx += NL) {
+        const int i = idx >> 5, j = idx & 31;
+        const bool ok = i < nvalid && p.gate != kGateNone;
+        frag::cp16(s.G + gsw(i, j * 4), g + row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 4, ok);
+      }
+    } else if (lt < C) {
+      s.G[lt] = (lt < nvalid && p.gate != kGateNone) ? g[row_id(p, b, t0 + lt, h)] : 0.f;
+    }
+    if (lt >= C && lt < 2 * C) {
+      s.beta[lt - C] = beta[cb * C + lt - C];
+      s.knorm[lt - C] = knorm_g[cb * C + lt - C];
+    }
+  }
+  frag::cp_commit();
+  frag::cp_wait<0>();
   __syncthreads();
   // element (i, c) of the gate tile
   auto gat = [&](int i, int c) -> float& { return gk == D ? s.G[gsw(i, c)] : s.G[i]; };
@@ -494,44 +583,7 @@ __global__ void __launch_bounds__(NTB, 1)
     }
   };
 
-  frag::cp_wait<0>();
-  tc::fence_smem_to_async();
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tb = s.tmem;
-  bool ok = true;
-  do {  // leaves early (break) only when a bounded wait gives up
-
-  // Fault injection (dr_inject_timeout): wait, with a short limit, on a barrier
-  // that nothing arrives on.  Every copy has landed and no MMA has been issued,
-  // so the timeout path below leaves nothing in flight.
-  if (inject_timeout) {
-    ok = hy_wait(&s.never, 0, kSpinInjected);
-    if (!ok) break;
-  }
-
-  // ---- level 1 (tensor memory): dQs = dO S, dW' = dU S, dKt = U dS', dM = dO U^T
-  // (descriptors are built once; a k-step adds its byte offset / 16 to the start
-  // address field, which stays below 2^14 for any shared-memory address)
-  if (tid == 0) {
-    const uint32_t id128 = tc::idesc_bf16(64, 128, false, true);
-    const uint32_t id64 = tc::idesc_bf16(64, 64, false, false);
-    const uint64_t aDO = tc::sdesc_kmaj(s.DO, D, 0), aDU = tc::sdesc_kmaj(s.DU, D, 0);
-    const uint64_t aUU = tc::sdesc_kmaj(s.UU, D, 0);
-    const uint64_t bSS = tc::sdesc_mnmaj(s.SS, D, 0), bSD = tc::sdesc_mnmaj(s.SD, D, 0);
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      const uint32_t acc = ks > 0 ? 1u : 0u;
-      const uint64_t ka = 16u * ks, kb = 256u * ks;  // K-major / MN-major k-step, 16-byte units
-      mma_step(tb + T_ZQ, aDO + ka, bSS + kb, id128, acc);
-      mma_step(tb + T_ADW, aDU + ka, bSS + kb, id128, acc);
-      mma_step(tb + T_AKT, aUU + ka, bSD + kb, id128, acc);
-      mma_step(tb + T_ADM, aDO + ka, aUU + ka, id64, acc);
-    }
-    tc::commit(&s.bar);
-  }
-  // colsum(conj(dS') S) while they run (real gates: per channel sum of dS' .* S):
+  // colsum(conj(dS') S) while level 1 runs (real gates: per channel sum of dS' .* S):
   // thread -> 8 columns (16-byte core rows), 4 rows (one per row group of its
   // quarter); eight lanes read the eight rows of one core matrix
   {
@@ -821,9 +873,15 @@ __global__ void __launch_bounds__(NTB, 1)
       }
     }
     tc::commit(&s.bar);
+    if (nb < p.B) tc::mbar_arrive_expect_tx(&s.full, kTileTx);
   }
   ok = hy_wait(&s.bar, 3);
   if (!ok) break;
+  // the next chunk's level-1 tiles into the tiles level 4 has released
+  if (nb < p.B) {
+    issue_tiles(nn, nh, nb);
+    pending = true;
+  }
   {
     float t4[4][4];
     frag_ld4(tb + T_F1 + 32 * qt, warp, t4);
@@ -914,14 +972,31 @@ __global__ void __launch_bounds__(NTB, 1)
     xx += __shfl_xor_sync(0xffffffffu, xx, 2);
     if ((lane & 3) == 0) s.dbp[(i0 + hh * 8) * 4 + qt] = xx;
   }
-  __syncthreads();  // the S and dS' tile regions are free: the dgamma tile (row stride LDG)
-  float* sdg = reinterpret_cast<float*>(s.SS);
+  // dgamma: reverse cumulative sum over the chunk's rows.  Within this warp's
+  // 16 rows (rows i0 = 16 rb + lr and i0 + 8, lr = lane / 4 on the lanes that
+  // share its columns): suffix sums down the 8 lane rows by shuffles, the
+  // second 8 rows' total added to the first; the later row blocks' totals
+  // follow through shared memory.
   if (gk == D) {
 #pragma unroll
     for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        sdg[(i0 + (e >> 1) * 8) * LDG + qt * 32 + jt * 8 + lc + (e & 1)] = Q[jt][e];
+      for (int u = 0; u < 2; ++u) {
+        float lo = Q[jt][u], hi = Q[jt][2 + u];
+#pragma unroll
+        for (int d = 1; d < 8; d <<= 1) {
+          const float yl = __shfl_down_sync(0xffffffffu, lo, 4 * d);
+          const float yh = __shfl_down_sync(0xffffffffu, hi, 4 * d);
+          if (lr + d < 8) {
+            lo += yl;
+            hi += yh;
+          }
+        }
+        lo += __shfl_sync(0xffffffffu, hi, lane & 3);
+        Q[jt][u] = lo;
+        Q[jt][2 + u] = hi;
+        if (lr == 0) s.blk[rb * D + qt * 32 + jt * 8 + lc + u] = lo;
+      }
   } else {
     // scalar gate: the row sums of dgamma, one slot per column quarter
 #pragma unroll
@@ -931,20 +1006,46 @@ __global__ void __launch_bounds__(NTB, 1)
       for (int jt = 0; jt < 4; ++jt) xx += Q[jt][2 * hh] + Q[jt][2 * hh + 1];
       xx += __shfl_xor_sync(0xffffffffu, xx, 1);
       xx += __shfl_xor_sync(0xffffffffu, xx, 2);
-      if ((lane & 3) == 0) sdg[(i0 + hh * 8) * 4 + qt] = xx;
+      if ((lane & 3) == 0) s.blk[(i0 + hh * 8) * 4 + qt] = xx;
     }
   }
   __syncthreads();
   float dbt = 0.f;
-  if (tid < C) dbt = s.dbp[tid * 4] + s.dbp[tid * 4 + 1] + s.dbp[tid * 4 + 2] + s.dbp[tid * 4 + 3];
-  const int gc = tid & 127, grq = tid >> 7;  // dgamma reverse scan: channel, row quarter
-  if (gk == D) {
-    float part = 0.f;
-#pragma unroll 4
-    for (int i = grq * 16; i < grq * 16 + 16; ++i) part += sdg[i * LDG + gc];
-    s.dgc[grq * D + gc] = part;  // the chunk-end term read dgc before the last two barriers
+  if (tid < C) {
+    dbt = s.dbp[tid * 4] + s.dbp[tid * 4 + 1] + s.dbp[tid * 4 + 2] + s.dbp[tid * 4 + 3];
+    s.dbp[tid * 4] = dbt;  // total d(beta_eff) of row tid (read back by this thread only)
   }
-  if (tid < C) s.dbp[tid * 4] = dbt;  // total d(beta_eff) of row tid
+  if (gk == D) {
+#pragma unroll
+    for (int jt = 0; jt < 4; ++jt) {
+      const int c = qt * 32 + jt * 8 + lc;
+      float later[2] = {0.f, 0.f};
+      for (int r2 = rb + 1; r2 < 4; ++r2) {
+        const float2 t = *reinterpret_cast<const float2*>(s.blk + r2 * D + c);
+        later[0] += t.x;
+        later[1] += t.y;
+      }
+      if (i0 < nvalid)
+        *reinterpret_cast<float2*>(dg + rowg[0] + c) =
+            make_float2(Q[jt][0] + later[0], Q[jt][1] + later[1]);
+      if (i0 + 8 < nvalid)
+        *reinterpret_cast<float2*>(dg + rowg[1] + c) =
+            make_float2(Q[jt][2] + later[0], Q[jt][3] + later[1]);
+    }
+  } else if (p.gate != kGateNone && warp == 0) {
+    // rows 2 lane, 2 lane + 1: suffix sums across the warp
+    const int ia = 2 * lane, ib = ia + 1;
+    const float a0 = s.blk[ia * 4] + s.blk[ia * 4 + 1] + s.blk[ia * 4 + 2] + s.blk[ia * 4 + 3];
+    const float a1 = s.blk[ib * 4] + s.blk[ib * 4 + 1] + s.blk[ib * 4 + 2] + s.blk[ib * 4 + 3];
+    float x = a0 + a1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_down_sync(0xffffffffu, x, o);
+      if (lane + o < 32) x += y;
+    }
+    if (ia < nvalid) dg[row_id(p, b, t0 + ia, h)] = x;
+    if (ib < nvalid) dg[row_id(p, b, t0 + ib, h)] = x - a0;
+  }
   __syncthreads();
   // dk (with the Kaczmarz chain rule) and dbeta
 #pragma unroll
@@ -965,34 +1066,12 @@ __global__ void __launch_bounds__(NTB, 1)
     if (p.beta_mode == kBetaKaczmarz) dbt /= (s.knorm[tid] + p.eps);
     dbeta[row_id(p, b, t0 + tid, h)] = dbt;
   }
-  // dgamma: reverse cumulative sum over the chunk's rows
-  if (gk == D) {
-    float run = 0.f;
-    for (int q2i = grq + 1; q2i < 4; ++q2i) run += s.dgc[q2i * D + gc];
-#pragma unroll 4
-    for (int i = grq * 16 + 15; i >= grq * 16; --i) {
-      run += sdg[i * LDG + gc];
-      if (i < nvalid) dg[row_id(p, b, t0 + i, h) * D + gc] = run;
-    }
-  } else if (p.gate != kGateNone && warp == 0) {
-    // rows 2 lane, 2 lane + 1: suffix sums across the warp
-    const int ia = 2 * lane, ib = ia + 1;
-    const float a0 = sdg[ia * 4] + sdg[ia * 4 + 1] + sdg[ia * 4 + 2] + sdg[ia * 4 + 3];
-    const float a1 = sdg[ib * 4] + sdg[ib * 4 + 1] + sdg[ib * 4 + 2] + sdg[ib * 4 + 3];
-    float x = a0 + a1;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float y = __shfl_down_sync(0xffffffffu, x, o);
-      if (lane + o < 32) x += y;
-    }
-    if (ia < nvalid) dg[row_id(p, b, t0 + ia, h)] = x;
-    if (ib < nvalid) dg[row_id(p, b, t0 + ib, h)] = x - a0;
   }
-  } while (0);
   if (!ok) {
     // a bounded wait gave up: record it and let the copies in flight land
     if (tid == 0 && err) atomicExch(err, 1);
     frag::cp_wait<0>();
+    if (pending && tid == 0) tc::mbar_wait(&s.full, fph, kSpinHy);
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -1020,7 +1099,10 @@ cudaError_t launch_bwd_chunk_hy(const Problem& p, const bf16* q, const bf16* k, 
   const double mac = 3.0 * C * D * D + (double)C * C * D + 2.0 * C * C * D + 2.0 * C * C * D +
                      24.0 * 64 * 16 * 128;
   prof_begin(kKTcChunkBwd, io, bytes, nb * 2.0 * mac, st);
-  kern<<<dim3(p.NC, p.H, p.B), NTB, sm, st>>>(
+  // persistent: one CTA per SM (its shared memory allows no second one)
+  const long nchunks = (long)p.NC * p.H * p.B;
+  const int grid = (int)(nchunks < sm_count() ? nchunks : sm_count());
+  kern<<<grid, NTB, sm, st>>>(
       p, q, k, v, dO, g, sv.T, sv.beta, sv.h, dh, sv.U, dU, sv.W, sv.Up, sv.knorm, dq, dk, dv,
       dbeta, dg, device_error_word(), take_injected_timeout() ? 1 : 0);
   e = cudaGetLastError();
