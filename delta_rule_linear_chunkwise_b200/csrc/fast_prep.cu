@@ -91,7 +91,7 @@ struct PrepSmem {
   uint32_t tmem;
 };
 
-static_assert(sizeof(float) * (64 * (64 + 4) + 32 * 33) <= 4 * kBox &&
+static_assert(sizeof(float) * (64 * (64 + 4) + 32 * (32 + 4)) <= 4 * kBox &&
                   offsetof(PrepSmem, K) == offsetof(PrepSmem, Q) + 2 * kBox,
               "the fp32 solve tiles fit the adjacent q and k regions");
 
@@ -501,8 +501,8 @@ __global__ void __launch_bounds__(NTP, 2)
   //   T21 = -T22 (A21 T11) by two 32 x 32 products on all threads;
   //   finally T = T_hi + T_lo in bf16, the tcgen05 operand.
   // fp32 T, row stride TLD (16-byte rows of 8 consecutive rows in distinct banks),
-  // over the Gram operands (read); Y = A21 T11, row stride 33
-  constexpr int TLD = C + 4;
+  // over the Gram operands (read); Y = A21 T11, row stride YLD
+  constexpr int TLD = C + 4, YLD = 32 + 4;
   unsigned char* const qk = reinterpret_cast<unsigned char*>(&s) + offsetof(PrepSmem, Q);
   float* Tf = reinterpret_cast<float*>(qk);
   float* Yb = reinterpret_cast<float*>(qk + C * TLD * 4);
@@ -532,32 +532,38 @@ __global__ void __launch_bounds__(NTP, 2)
     }
   }
   __syncthreads();
+  // the two 32 x 32 products: thread -> row ti = tid / 8 (of the second half),
+  // columns tj .. tj + 3, tj = 4 (tid % 8) (per k-step one scalar and one
+  // 16-byte shared load for four FMAs)
+  const int ti = tid >> 3, tj = 4 * (tid & 7);
   {
-    // Y = A21 T11: lane -> row ti of the second half, warp -> columns tj + 8 k
-    const int ti = tid & 31, tj = tid >> 5;
+    // Y = A21 T11
     float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
     for (int m = 0; m < 32; ++m) {
       const float a = At[m * C + 32 + ti];
-#pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) y[k4] += a * Tf[m * TLD + tj + 8 * k4];
+      const float4 t = *reinterpret_cast<const float4*>(Tf + m * TLD + tj);
+      y[0] += a * t.x;
+      y[1] += a * t.y;
+      y[2] += a * t.z;
+      y[3] += a * t.w;
     }
-#pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4) Yb[ti * 33 + tj + 8 * k4] = y[k4];
+    *reinterpret_cast<float4*>(Yb + ti * YLD + tj) = make_float4(y[0], y[1], y[2], y[3]);
   }
   __syncthreads();
   {
-    // T21 = -T22 Y: lane -> column tj, warp -> rows ti + 8 k of the second half
-    const int tj = tid & 31, ti = tid >> 5;
+    // T21 = -T22 Y
     float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
     for (int m = 0; m < 32; ++m) {
-      const float yv = Yb[m * 33 + tj];
-#pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) y[k4] += Tf[(32 + ti + 8 * k4) * TLD + 32 + m] * yv;
+      const float a = Tf[(32 + ti) * TLD + 32 + m];
+      const float4 t = *reinterpret_cast<const float4*>(Yb + m * YLD + tj);
+      y[0] += a * t.x;
+      y[1] += a * t.y;
+      y[2] += a * t.z;
+      y[3] += a * t.w;
     }
-#pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4) Tf[(32 + ti + 8 * k4) * TLD + tj] = -y[k4];
+    *reinterpret_cast<float4*>(Tf + (32 + ti) * TLD + tj) = make_float4(-y[0], -y[1], -y[2], -y[3]);
   }
   __syncthreads();
   bf16* Thi = reinterpret_cast<bf16*>(s.G + 2 * kBox);
