@@ -12,10 +12,11 @@
 // and o_n = D_A[64:128].  The state lives in registers transposed, one key
 // column per TMEM lane, so the per-channel decay is one scalar per thread; the
 // bf16 copy of S^T in shared memory is the MN-major B operand of the next
-// MMA-A.  The chunk-start state h_n and o_{n-1} are written to global memory
-// while MMA-A of chunk n runs.  D_A is double-buffered in tensor memory for
-// that reason.  Chunk tiles stream through a two-stage cp.async pipeline into
-// the canonical no-swizzle core-matrix layouts.
+// MMA-A.  o_{n-1} is written to global memory while MMA-A of chunk n runs, the
+// chunk-start state h_n while MMA-B and MMA-C run.  D_A is double-buffered in tensor memory for
+// that reason.  Chunk tiles stream through a two-stage pipeline of bulk copies
+// (issued by the lanes of one warp, one mbarrier per stage) into the canonical
+// no-swizzle core-matrix layouts.
 //
 // This is the affine state transfer of the chunkwise (WY/UT) form:
 //   S_{n+1} = S_n Diag(e^{gamma_C}) + (U' - W S_n^T)^T K~,
@@ -51,25 +52,51 @@ struct ScanSmem {
   ScanStage<BV> st[2];
   bf16 SB[D * BV];     // bf16 S^T, MN-major B of MMA-A ([K = c][N = a])
   bf16 UB[C * BV];     // bf16 U, MN-major B of MMA-B / MMA-C ([K = i][N = a])
-  uint64_t barA, barB;
+  uint64_t barA, barB, full[2];
   uint32_t tmem;
 };
 
-// The chunk tiles are stored core-tiled in HBM (the layout of the operands
-// here), so each is one contiguous copy; U'[:, a0 .. a0 + BV) is one
-// contiguous run per block of 8 rows.
+// Bytes of one stage fill.
 template <int BV>
-__device__ __forceinline__ void scan_issue(const Problem& p, ScanStage<BV>& s, const Saved& sv,
-                                           size_t cb, int a0, bool with_o, bool with_up) {
-  const int tid = threadIdx.x;
-  cp_linear<NTF>(s.AWQ, sv.W + cb * C * D, C * D, tid);
-  if (with_o) {
-    cp_linear<NTF>(s.AWQ + C * D, sv.Qh + cb * C * D, C * D, tid);
-    cp_linear<NTF>(s.MZ + C * C, sv.M + cb * C * C, C * C, tid);
+__host__ __device__ constexpr uint32_t scan_fill_bytes(bool with_o, bool with_up) {
+  return (uint32_t)(sizeof(bf16) * (2 * C * D + (with_o ? C * D + C * C : 0) +
+                                    (with_up ? C * BV : 0)) +
+                    sizeof(float) * D);
+}
+
+// Fills a stage by bulk copies, completing on `full` (whose transaction count
+// thread 0 has set with scan_fill_bytes before a barrier that precedes this):
+// called by every thread, lane 0 of each warp issues one to three of the
+// copies (a bulk copy holds its issuing thread while the copy engine takes it,
+// so they are spread over the warps).  The chunk tiles are stored core-tiled in
+// HBM (the layout of the operands here), so each is one contiguous copy;
+// U'[:, a0 .. a0 + BV) is one contiguous run of BV / 8 core matrices per block
+// of 8 rows.
+template <int BV>
+__device__ __forceinline__ void scan_fill(ScanStage<BV>& s, uint64_t* full, const Saved& sv,
+                                          size_t cb, int a0, bool with_o, bool with_up,
+                                          int warp, int lane) {
+  if (lane != 0) return;
+  constexpr uint32_t kT = sizeof(bf16) * C * D, kM = sizeof(bf16) * C * C;
+  constexpr uint32_t kRun = sizeof(bf16) * 8 * BV;  // one 8-row block of the U' slice
+  auto up_run = [&](int grp) {
+    tc::bulk_g2s(s.UP + (size_t)grp * 8 * BV,
+                 sv.Up + cb * C * D + ((size_t)grp * 16 + (a0 >> 3)) * 64, kRun, full);
+  };
+  switch (warp) {
+    case 0: tc::bulk_g2s(s.AWQ, sv.W + cb * C * D, kT, full); break;
+    case 1: tc::bulk_g2s(s.KT, sv.Kt + cb * C * D, kT, full); break;
+    case 2: if (with_o) tc::bulk_g2s(s.AWQ + C * D, sv.Qh + cb * C * D, kT, full); break;
+    case 3: if (with_o) tc::bulk_g2s(s.MZ + C * C, sv.M + cb * C * C, kM, full); break;
+    case 4:
+      tc::bulk_g2s(s.dec, sv.dec + cb * D, sizeof(float) * D, full);
+      if (with_up) up_run(0);
+      break;
+    default:  // warps 5, 6, 7: U' runs 1..7
+      if (with_up)
+        for (int grp = 1 + 3 * (warp - 5); grp < 1 + 3 * (warp - 4) && grp < C / 8; ++grp) up_run(grp);
+      break;
   }
-  cp_linear<NTF>(s.KT, sv.Kt + cb * C * D, C * D, tid);
-  if (with_up) cp_ct_cols<NTF>(s.UP, sv.Up + cb * C * D, C, a0, BV, tid);
-  if (tid < D / 4) frag::cp16(s.dec + 4 * tid, sv.dec + cb * D + 4 * tid, true);
 }
 
 // Writes this thread's HB state values x[u] (rows a0h + u, key c; one key per
@@ -154,6 +181,9 @@ __global__ void __launch_bounds__(NTF, 1)
   if (tid == 0) {
     tc::mbar_init(&s.barA, 1);
     tc::mbar_init(&s.barB, 1);
+    tc::mbar_init(&s.full[0], 1);
+    tc::mbar_init(&s.full[1], 1);
+    tc::fence_mbar_init();
   }
   // zero halves of [0 ; M] in both stages
   for (int idx = tid; idx < 2 * C * C / 8; idx += NTF) {
@@ -206,18 +236,31 @@ __global__ void __launch_bounds__(NTF, 1)
   };
 
   write_sb();
-  scan_issue<BV>(p, s.st[0], sv, chunk_id(p, b, h, n0), a0, with_o, with_up);
-  frag::cp_commit();
-  if (n0 + 1 < n1) scan_issue<BV>(p, s.st[1], sv, chunk_id(p, b, h, n0 + 1), a0, with_o, with_up);
-  frag::cp_commit();
-  frag::cp_wait<1>();
+  tc::fence_before_sync();
+  __syncthreads();  // barriers initialised
+  tc::fence_after_sync();
+  int fills[2] = {0, 0};  // bulk fills issued per stage (uniform over the CTA)
+  constexpr int NTW = NTF / 32;
+  static_assert(NTW == 8, "the stage fill spreads its copies over eight warps");
+  const uint32_t fill_tx = scan_fill_bytes<BV>(with_o, with_up);
+  if (tid == 0) {
+    tc::mbar_arrive_expect_tx(&s.full[0], fill_tx);
+    if (n0 + 1 < n1) tc::mbar_arrive_expect_tx(&s.full[1], fill_tx);
+  }
+  __syncthreads();
+  scan_fill<BV>(s.st[0], &s.full[0], sv, chunk_id(p, b, h, n0), a0, with_o, with_up, warp, lane);
+  fills[0] = 1;
+  if (n0 + 1 < n1) {
+    scan_fill<BV>(s.st[1], &s.full[1], sv, chunk_id(p, b, h, n0 + 1), a0, with_o, with_up, warp,
+                  lane);
+    fills[1] = 1;
+  }
+  bool ok = tc::mbar_wait(&s.full[0], 0u, kSpinScan);
   tc::fence_smem_to_async();
   tc::fence_before_sync();
-  __syncthreads();
+  ok = __syncthreads_or(ok ? 0 : 1) == 0;
   tc::fence_after_sync();
   const uint32_t tbase = s.tmem;
-
-  bool ok = true;
   const uint32_t idA = tc::idesc_bf16(128, BV, false, true);
   const uint32_t idC = tc::idesc_bf16(128, BV, true, true);
   // descriptors: per-k-step advance of the start address (in 16-byte units)
@@ -231,8 +274,10 @@ __global__ void __launch_bounds__(NTF, 1)
     const int buf = it & 1;
     const float dc = st.dec[PHASE ? (c & ~1) : c];  // read before the stage is refilled below
     const float di = PHASE ? ((c & 1) ? st.dec[c] : -st.dec[c | 1]) : 0.f;
-    // MMA-A: [W ; q e^gamma] S^T
+    // MMA-A: [W ; q e^gamma] S^T (and the transaction count of this stage's refill,
+    // whose copies follow two barriers later)
     if (tid == 0) {
+      if (n + 2 < n1) tc::mbar_arrive_expect_tx(&s.full[it & 1], fill_tx);
       const uint64_t dA = tc::sdesc_kmaj(st.AWQ, D, 0);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks)
@@ -300,8 +345,11 @@ __global__ void __launch_bounds__(NTF, 1)
     ok = cta_wait(&s.barB, it);
     if (!ok) break;
     // this stage is consumed: refill it with chunk n + 2 (lands during the next step)
-    if (n + 2 < n1) scan_issue<BV>(p, st, sv, chunk_id(p, b, h, n + 2), a0, with_o, with_up);
-    frag::cp_commit();
+    if (n + 2 < n1) {
+      scan_fill<BV>(st, &s.full[it & 1], sv, chunk_id(p, b, h, n + 2), a0, with_o, with_up, warp,
+                    lane);
+      ++fills[it & 1];
+    }
     // epilogue 2: S^T <- Diag(e^{gamma_C}) S^T + D_S
     {
       uint32_t r[HB];
@@ -322,10 +370,12 @@ __global__ void __launch_bounds__(NTF, 1)
       }
       write_sb();
     }
-    frag::cp_wait<1>();
+    // the next chunk's stage (filled one step ago)
+    bool okF = true;
+    if (n + 1 < n1) okF = tc::mbar_wait(&s.full[(it + 1) & 1], (uint32_t)(((it + 1) >> 1) & 1), kSpinScan);
     tc::fence_smem_to_async();
     tc::fence_before_sync();
-    __syncthreads();
+    ok = __syncthreads_or(okF ? 0 : 1) == 0;
     tc::fence_after_sync();
   }
   if (ok) {
@@ -337,7 +387,11 @@ __global__ void __launch_bounds__(NTF, 1)
   } else if (tid == 0 && err) {
     atomicExch(err, 1);
   }
-  frag::cp_wait<0>();
+  // fills still in flight (only after a failed wait) land before exit
+  if (tid == 0) {
+    if (fills[0] > 0) tc::mbar_wait(&s.full[0], (uint32_t)((fills[0] - 1) & 1), kSpinScan);
+    if (fills[1] > 0) tc::mbar_wait(&s.full[1], (uint32_t)((fills[1] - 1) & 1), kSpinScan);
+  }
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tbase, TALLOC);
