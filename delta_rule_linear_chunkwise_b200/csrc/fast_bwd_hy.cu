@@ -515,71 +515,92 @@ __global__ void __launch_bounds__(NTB, 1)
   auto q2 = [&](int i, int c) -> float2 {
     return frag::unpack(*reinterpret_cast<const uint32_t*>(s.QR + i * LDD + c));
   };
-  // Level-4 key/query tiles for the 8 channels c .. c + 7 of row i.  first: the
-  // tiles built under level 3 (write keys of both references, queries, and the
-  // beta keys of the second half); otherwise the beta keys of the first reference.
+  // Level-4 key/query tiles for the 8 channels c .. c + 7 of row i (a warp's
+  // rows lie in one half).  first: the tiles built under level 3 -- rows of the
+  // first half: the write keys against both references and the queries; of the
+  // second half: the write keys, the queries against both references and the
+  // beta keys; otherwise the beta keys against the first reference.  Each case
+  // forms only the factors it stores.
   auto build_row = [&](int idx, bool first) {
     const int i = ct_row(idx, D), c = ct_col(idx, D);
+    const bool h1 = i >= 32;
     const uint4 rk = *reinterpret_cast<const uint4*>(s.k + i * LDD + c);
-    const uint4 rq = *reinterpret_cast<const uint4*>(s.QR + i * LDD + c);
     const float bi = s.beta[i];
     const float4 f0 = ep4(i, c), f1 = ep4(i, c + 4);
     const float f[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
     const uint32_t* wk = reinterpret_cast<const uint32_t*>(&rk);
-    const uint32_t* wq = reinterpret_cast<const uint32_t*>(&rq);
-    const bool h1 = i >= 32;
-    uint32_t okb[4], okbx[4], oq[4], oqx[4], obk[4], obkx[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 kk = frag::unpack(wk[e]), qq = frag::unpack(wq[e]);
-      const int cc = c + 2 * e;
-      float kb0, kb1, qf0, qf1, bk0, bk1, kbx0, kbx1, qx0, qx1, bkx0, bkx1;
-      if (PHASE) {
-        const cf uu{f[2 * e], f[2 * e + 1]}, kc{kk.x, kk.y}, qc{qq.x, qq.y};
-        const cf xk0{s.xk[cc], s.xk[cc + 1]}, xk1{s.xk[D + cc], s.xk[D + cc + 1]};
-        const cf xq0{s.xq[cc], s.xq[cc + 1]}, xq1{s.xq[D + cc], s.xq[D + cc + 1]};
-        const cf kb = cmul(kc, cconj(cinv(uu)));   // k / conj(u)
-        const cf qf = cmul(uu, qc), bk = cmul(uu, kc);
-        const cf kbx = cmul(cmul(kb, xk0), xk1), qx = cmul(cmul(qf, xq0), xq1);
-        const cf bkx = cmul(cmul(bk, xq0), xq1);
-        kb0 = kb.x, kb1 = kb.y, qf0 = qf.x, qf1 = qf.y, bk0 = bi * bk.x, bk1 = bi * bk.y;
-        kbx0 = kbx.x, kbx1 = kbx.y, qx0 = qx.x, qx1 = qx.y, bkx0 = bi * bkx.x, bkx1 = bi * bkx.y;
-      } else {
-        kb0 = __fdividef(kk.x, f[2 * e]), kb1 = __fdividef(kk.y, f[2 * e + 1]);
-        qf0 = qq.x * f[2 * e], qf1 = qq.y * f[2 * e + 1];
-        bk0 = bi * kk.x * f[2 * e], bk1 = bi * kk.y * f[2 * e + 1];
-        kbx0 = kb0 * s.xk[cc] * s.xk[D + cc], kbx1 = kb1 * s.xk[cc + 1] * s.xk[D + cc + 1];
-        qx0 = qf0 * s.xq[cc] * s.xq[D + cc], qx1 = qf1 * s.xq[cc + 1] * s.xq[D + cc + 1];
-        bkx0 = bk0 * s.xq[cc] * s.xq[D + cc], bkx1 = bk1 * s.xq[cc + 1] * s.xq[D + cc + 1];
-      }
-      okb[e] = frag::pack(kb0, kb1);
-      okbx[e] = frag::pack(kbx0, kbx1);
-      oq[e] = frag::pack(qf0, qf1);
-      oqx[e] = frag::pack(qx0, qx1);
-      obk[e] = frag::pack(bk0, bk1);
-      obkx[e] = frag::pack(bkx0, bkx1);
-    }
-    const uint4 vkb = make_uint4(okb[0], okb[1], okb[2], okb[3]);
-    const uint4 vkbx = make_uint4(okbx[0], okbx[1], okbx[2], okbx[3]);
-    const uint4 vq = make_uint4(oq[0], oq[1], oq[2], oq[3]);
-    const uint4 vqx = make_uint4(oqx[0], oqx[1], oqx[2], oqx[3]);
-    const uint4 vbk = make_uint4(obk[0], obk[1], obk[2], obk[3]);
-    const uint4 vbkx = make_uint4(obkx[0], obkx[1], obkx[2], obkx[3]);
     // core-tiled offset of row i (idx) and of row i - 32 in a 32-row tile
     const int o = 8 * idx, o32 = 8 * idx - 32 * D;
+    auto st4 = [](bf16* dst, const uint32_t (&w)[4]) {
+      *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    };
     if (first) {
+      const uint4 rq = *reinterpret_cast<const uint4*>(s.QR + i * LDD + c);
+      const uint32_t* wq = reinterpret_cast<const uint32_t*>(&rq);
+      uint32_t okb[4], oq[4], ox[4], obk[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 kk = frag::unpack(wk[e]), qq = frag::unpack(wq[e]);
+        const int cc = c + 2 * e;
+        if (PHASE) {
+          const cf uu{f[2 * e], f[2 * e + 1]}, kc{kk.x, kk.y}, qc{qq.x, qq.y};
+          const cf kb = cmul(kc, cconj(cinv(uu)));  // k / conj(u)
+          const cf qf = cmul(uu, qc);
+          okb[e] = frag::pack(kb.x, kb.y);
+          oq[e] = frag::pack(qf.x, qf.y);
+          if (!h1) {
+            const cf kbx = cmul(cmul(kb, cf{s.xk[cc], s.xk[cc + 1]}), cf{s.xk[D + cc], s.xk[D + cc + 1]});
+            ox[e] = frag::pack(kbx.x, kbx.y);
+          } else {
+            const cf xq0{s.xq[cc], s.xq[cc + 1]}, xq1{s.xq[D + cc], s.xq[D + cc + 1]};
+            const cf qx = cmul(cmul(qf, xq0), xq1);
+            const cf bk = cmul(uu, kc);
+            ox[e] = frag::pack(qx.x, qx.y);
+            obk[e] = frag::pack(bi * bk.x, bi * bk.y);
+          }
+        } else {
+          const float kb0 = __fdividef(kk.x, f[2 * e]), kb1 = __fdividef(kk.y, f[2 * e + 1]);
+          const float qf0 = qq.x * f[2 * e], qf1 = qq.y * f[2 * e + 1];
+          okb[e] = frag::pack(kb0, kb1);
+          oq[e] = frag::pack(qf0, qf1);
+          if (!h1) {
+            ox[e] = frag::pack(kb0 * s.xk[cc] * s.xk[D + cc], kb1 * s.xk[cc + 1] * s.xk[D + cc + 1]);
+          } else {
+            ox[e] = frag::pack(qf0 * s.xq[cc] * s.xq[D + cc], qf1 * s.xq[cc + 1] * s.xq[D + cc + 1]);
+            obk[e] = frag::pack(bi * kk.x * f[2 * e], bi * kk.y * f[2 * e + 1]);
+          }
+        }
+      }
       if (!h1) {
-        *reinterpret_cast<uint4*>(Kb0 + o) = vkb;
-        *reinterpret_cast<uint4*>(Kb1 + o) = vkbx;
-        *reinterpret_cast<uint4*>(Q0 + o) = vq;
+        st4(Kb0 + o, okb);
+        st4(Kb1 + o, ox);
+        st4(Q0 + o, oq);
       } else {
-        *reinterpret_cast<uint4*>(Kb1 + o) = vkb;
-        *reinterpret_cast<uint4*>(Q0 + o) = vqx;
-        *reinterpret_cast<uint4*>(Q1 + o32) = vq;
-        *reinterpret_cast<uint4*>(B1 + o32) = vbk;
+        st4(Kb1 + o, okb);
+        st4(Q0 + o, ox);
+        st4(Q1 + o32, oq);
+        st4(B1 + o32, obk);
       }
     } else {
-      *reinterpret_cast<uint4*>(B0 + o) = h1 ? vbkx : vbk;
+      uint32_t ob[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 kk = frag::unpack(wk[e]);
+        const int cc = c + 2 * e;
+        if (PHASE) {
+          cf bk = cmul(cf{f[2 * e], f[2 * e + 1]}, cf{kk.x, kk.y});
+          if (h1) bk = cmul(cmul(bk, cf{s.xq[cc], s.xq[cc + 1]}), cf{s.xq[D + cc], s.xq[D + cc + 1]});
+          ob[e] = frag::pack(bi * bk.x, bi * bk.y);
+        } else {
+          float b0 = bi * kk.x * f[2 * e], b1 = bi * kk.y * f[2 * e + 1];
+          if (h1) {
+            b0 = b0 * s.xq[cc] * s.xq[D + cc];
+            b1 = b1 * s.xq[cc + 1] * s.xq[D + cc + 1];
+          }
+          ob[e] = frag::pack(b0, b1);
+        }
+      }
+      st4(B0 + o, ob);
     }
   };
 
