@@ -76,13 +76,13 @@ struct PrepSmem {
                                             // then beta k e^g (MN-major B of W)
   // per key channel (phase gate: per pair, complex, at the pair's two channels),
   // for the two halves' reference rows rho0 = 15, rho1 = 47:
-  float ref[2][D];   // cumulative gate at rho
+  alignas(16) float ref[2][D];   // cumulative gate at rho
   float rot[2][D];   // phase gate: (cos, sin) of the cumulative phase at rho
-  float zr[2][D];    // zeta_rho                     (real gates: e^{g_rho})
-  float ec[2][D];    // conj(zeta_C / zeta_rho)      (real gates: e^{g_C - g_rho})
+  alignas(16) float zr[2][D];    // zeta_rho                     (real gates: e^{g_rho})
+  alignas(16) float ec[2][D];    // conj(zeta_C / zeta_rho)      (real gates: e^{g_C - g_rho})
   // write keys of the first half against the second reference, in two steps
   // through the half boundary: conj(zeta_31 / zeta_rho0), conj(zeta_rho1 / zeta_31)
-  float xk[2][D];
+  alignas(16) float xk[2][D];
   float tot[D];      // cumulative gate of the first half's last row
   float gs[C];       // scalar gate: cumulative per row
   float eta[C];      // input beta (eta in Kaczmarz mode)
@@ -141,6 +141,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   tc::tmem_wait_ld();
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 2^x (the ex2.approx.ftz instruction: relative error about 2^-22, flushes
+// results below the normal range to zero)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Eight consecutive floats of a 16-byte aligned shared-memory array.
+__device__ __forceinline__ void load8(const float* p, float* f) {
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  f[0] = a.x, f[1] = a.y, f[2] = a.z, f[3] = a.w, f[4] = b.x, f[5] = b.y, f[6] = b.z, f[7] = b.w;
 }
 
 __device__ __forceinline__ void unpack8(const uint4& r, float* f) {
@@ -386,21 +401,29 @@ __global__ void __launch_bounds__(NTP, 2)
           eps_ = __expf(sg - s.ref[hr][0]);
           ems_ = __expf(s.ref[hr][0] - sg);
         }
+        // the per-channel reference factors of these 8 channels (vector loads)
+        float r8[8], z8[8], e8[8], x0[8], x1[8];
+        load8(s.ref[hr] + c0, r8);
+        load8(s.zr[hr] + c0, z8);
+        load8(s.ec[hr] + c0, e8);
+        if (hr == 0) {
+          load8(s.xk[0] + c0, x0);
+          load8(s.xk[1] + c0, x1);
+        }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const int cc = c0 + e;
           float ep = eps_, em = ems_;
-          if (chan) {
-            const float d = gg[e] - s.ref[hr][cc];
-            ep = __expf(d), em = __expf(-d);
+          if (chan) {  // e^{+-(g - g_rho)} as 2^{+-(g - g_rho) log2 e}
+            const float d2 = (gg[e] - r8[e]) * kLog2e;
+            ep = ex2_approx(d2), em = ex2_approx(-d2);
           }
           kc[e] = kv[e] * ep;
           qc[e] = qv[e] * ep;
           kb[e] = kv[e] * em;
-          qh[e] = qc[e] * s.zr[hr][cc];
-          bk[e] = br * kc[e] * s.zr[hr][cc];
-          kt[e] = kb[e] * s.ec[hr][cc];
-          if (hr == 0) kb1[e] = kb[e] * s.xk[0][cc] * s.xk[1][cc];
+          qh[e] = qc[e] * z8[e];
+          bk[e] = br * kc[e] * z8[e];
+          kt[e] = kb[e] * e8[e];
+          if (hr == 0) kb1[e] = kb[e] * x0[e] * x1[e];
         }
       }
 #pragma unroll
