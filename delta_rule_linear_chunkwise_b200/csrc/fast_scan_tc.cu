@@ -56,47 +56,36 @@ struct ScanSmem {
   uint32_t tmem;
 };
 
-// Bytes of one stage fill.
-template <int BV>
-__host__ __device__ constexpr uint32_t scan_fill_bytes(bool with_o, bool with_up) {
-  return (uint32_t)(sizeof(bf16) * (2 * C * D + (with_o ? C * D + C * C : 0) +
-                                    (with_up ? C * BV : 0)) +
-                    sizeof(float) * D);
+// Bytes of one stage fill's bulk copies.
+__host__ __device__ constexpr uint32_t scan_fill_bytes(bool with_o) {
+  return (uint32_t)(sizeof(bf16) * (2 * C * D + (with_o ? C * D + C * C : 0)) + sizeof(float) * D);
 }
 
-// Fills a stage by bulk copies, completing on `full` (whose transaction count
-// thread 0 has set with scan_fill_bytes before a barrier that precedes this):
-// called by every thread, lane 0 of each warp issues one to three of the
-// copies (a bulk copy holds its issuing thread while the copy engine takes it,
-// so they are spread over the warps).  The chunk tiles are stored core-tiled in
-// HBM (the layout of the operands here), so each is one contiguous copy;
-// U'[:, a0 .. a0 + BV) is one contiguous run of BV / 8 core matrices per block
-// of 8 rows.
+// Fills a stage, called by every thread: the chunk tiles, stored core-tiled in
+// HBM (the layout of the operands here), by one bulk copy each from lane 0 of
+// warps 0..4, completing on `full` (whose transaction count thread 0 has set
+// with scan_fill_bytes before a barrier that precedes this; a bulk copy holds
+// its issuing thread while the copy engine takes it, so they are spread over
+// the warps), and U'[:, a0 .. a0 + BV) (one run of BV / 8 core matrices per
+// block of 8 rows) by cp.async from every thread, one group (committed also
+// when empty).
 template <int BV>
 __device__ __forceinline__ void scan_fill(ScanStage<BV>& s, uint64_t* full, const Saved& sv,
                                           size_t cb, int a0, bool with_o, bool with_up,
                                           int warp, int lane) {
-  if (lane != 0) return;
   constexpr uint32_t kT = sizeof(bf16) * C * D, kM = sizeof(bf16) * C * C;
-  constexpr uint32_t kRun = sizeof(bf16) * 8 * BV;  // one 8-row block of the U' slice
-  auto up_run = [&](int grp) {
-    tc::bulk_g2s(s.UP + (size_t)grp * 8 * BV,
-                 sv.Up + cb * C * D + ((size_t)grp * 16 + (a0 >> 3)) * 64, kRun, full);
-  };
-  switch (warp) {
-    case 0: tc::bulk_g2s(s.AWQ, sv.W + cb * C * D, kT, full); break;
-    case 1: tc::bulk_g2s(s.KT, sv.Kt + cb * C * D, kT, full); break;
-    case 2: if (with_o) tc::bulk_g2s(s.AWQ + C * D, sv.Qh + cb * C * D, kT, full); break;
-    case 3: if (with_o) tc::bulk_g2s(s.MZ + C * C, sv.M + cb * C * C, kM, full); break;
-    case 4:
-      tc::bulk_g2s(s.dec, sv.dec + cb * D, sizeof(float) * D, full);
-      if (with_up) up_run(0);
-      break;
-    default:  // warps 5, 6, 7: U' runs 1..7
-      if (with_up)
-        for (int grp = 1 + 3 * (warp - 5); grp < 1 + 3 * (warp - 4) && grp < C / 8; ++grp) up_run(grp);
-      break;
+  if (lane == 0) {
+    switch (warp) {
+      case 0: tc::bulk_g2s(s.AWQ, sv.W + cb * C * D, kT, full); break;
+      case 1: tc::bulk_g2s(s.KT, sv.Kt + cb * C * D, kT, full); break;
+      case 2: if (with_o) tc::bulk_g2s(s.AWQ + C * D, sv.Qh + cb * C * D, kT, full); break;
+      case 3: if (with_o) tc::bulk_g2s(s.MZ + C * C, sv.M + cb * C * C, kM, full); break;
+      case 4: tc::bulk_g2s(s.dec, sv.dec + cb * D, sizeof(float) * D, full); break;
+      default: break;
+    }
   }
+  if (with_up) cp_ct_cols<NTF>(s.UP, sv.Up + cb * C * D, C, a0, BV, threadIdx.x);
+  frag::cp_commit();
 }
 
 // Writes this thread's HB state values x[u] (rows a0h + u, key c; one key per
@@ -242,7 +231,7 @@ __global__ void __launch_bounds__(NTF, 1)
   int fills[2] = {0, 0};  // bulk fills issued per stage (uniform over the CTA)
   constexpr int NTW = NTF / 32;
   static_assert(NTW == 8, "the stage fill spreads its copies over eight warps");
-  const uint32_t fill_tx = scan_fill_bytes<BV>(with_o, with_up);
+  const uint32_t fill_tx = scan_fill_bytes(with_o);
   if (tid == 0) {
     tc::mbar_arrive_expect_tx(&s.full[0], fill_tx);
     if (n0 + 1 < n1) tc::mbar_arrive_expect_tx(&s.full[1], fill_tx);
@@ -254,7 +243,10 @@ __global__ void __launch_bounds__(NTF, 1)
     scan_fill<BV>(s.st[1], &s.full[1], sv, chunk_id(p, b, h, n0 + 1), a0, with_o, with_up, warp,
                   lane);
     fills[1] = 1;
+  } else {
+    frag::cp_commit();  // an empty group: one group per fill slot keeps the waits below exact
   }
+  frag::cp_wait<1>();
   bool ok = tc::mbar_wait(&s.full[0], 0u, kSpinScan);
   tc::fence_smem_to_async();
   tc::fence_before_sync();
@@ -349,6 +341,8 @@ __global__ void __launch_bounds__(NTF, 1)
       scan_fill<BV>(st, &s.full[it & 1], sv, chunk_id(p, b, h, n + 2), a0, with_o, with_up, warp,
                     lane);
       ++fills[it & 1];
+    } else {
+      frag::cp_commit();  // empty group
     }
     // epilogue 2: S^T <- Diag(e^{gamma_C}) S^T + D_S
     {
@@ -370,8 +364,10 @@ __global__ void __launch_bounds__(NTF, 1)
       }
       write_sb();
     }
-    // the next chunk's stage (filled one step ago)
+    // the next chunk's stage (filled one step ago; its U' group is the older of
+    // the two outstanding ones)
     bool okF = true;
+    frag::cp_wait<1>();
     if (n + 1 < n1) okF = tc::mbar_wait(&s.full[(it + 1) & 1], (uint32_t)(((it + 1) >> 1) & 1), kSpinScan);
     tc::fence_smem_to_async();
     tc::fence_before_sync();
@@ -388,6 +384,7 @@ __global__ void __launch_bounds__(NTF, 1)
     atomicExch(err, 1);
   }
   // fills still in flight (only after a failed wait) land before exit
+  frag::cp_wait<0>();
   if (tid == 0) {
     if (fills[0] > 0) tc::mbar_wait(&s.full[0], (uint32_t)((fills[0] - 1) & 1), kSpinScan);
     if (fills[1] > 0) tc::mbar_wait(&s.full[1], (uint32_t)((fills[1] - 1) & 1), kSpinScan);
