@@ -120,8 +120,8 @@ struct HySmem {
   // and queries / keys of the second half against the first reference,
   // (zeta_rho1 / zeta_32) (zeta_32 / zeta_rho0); applied one after the other, so
   // that no intermediate underflows where the product does not
-  float xk[2 * D];
-  float xq[2 * D];
+  alignas(16) float xk[2 * D];
+  alignas(16) float xq[2 * D];
   float dmd[C];      // the diagonal of dM (fp32), added outside the level-4 products
   float blk[4 * D];  // dgamma totals of each 16-row block (scalar gate: row partial sums)
   uint64_t bar;
@@ -476,26 +476,32 @@ __global__ void __launch_bounds__(NTB, 1)
       gat(i, c) = tmp[2 * u];
       gat(i, c + 1) = tmp[2 * u + 1];
     }
-  } else {
-    float tmp[C * D / NTB];
-    const int cnt = (gk == D) ? C * D / NTB : (tid < C ? 1 : 0);
+  } else if (gk == D) {
+    // thread: channels c4 .. c4 + 3 of rows i4 + 16 u (16-byte accesses; the
+    // swizzle keeps groups of 4 channels contiguous)
+    const int c4 = 4 * (tid & 31), i4 = tid >> 5;
+    const float4 r0 = *reinterpret_cast<const float4*>(s.G + gsw(kRho0, c4));
+    const float4 r1 = *reinterpret_cast<const float4*>(s.G + gsw(kRho1, c4));
+    float4 v[C * D / NTB / 4];
 #pragma unroll
-    for (int u = 0; u < C * D / NTB; ++u) {
-      if (u < cnt) {
-        const int idx = tid + u * NTB;
-        const int i = (gk == D) ? idx >> 7 : idx, c = (gk == D) ? idx & 127 : 0;
-        tmp[u] = __expf(gat(i, c) - gat(i < 32 ? kRho0 : kRho1, c));
-      }
-    }
+    for (int u = 0; u < C * D / NTB / 4; ++u)
+      v[u] = *reinterpret_cast<const float4*>(s.G + gsw(i4 + 16 * u, c4));
     __syncthreads();
 #pragma unroll
-    for (int u = 0; u < C * D / NTB; ++u) {
-      if (u < cnt) {
-        const int idx = tid + u * NTB;
-        const int i = (gk == D) ? idx >> 7 : idx, c = (gk == D) ? idx & 127 : 0;
-        gat(i, c) = tmp[u];
-      }
+    for (int u = 0; u < C * D / NTB / 4; ++u) {
+      const int i = i4 + 16 * u;
+      const float4 r = i < 32 ? r0 : r1;
+      *reinterpret_cast<float4*>(s.G + gsw(i, c4)) =
+          make_float4(frag::ex2_approx((v[u].x - r.x) * frag::kLog2e),
+                      frag::ex2_approx((v[u].y - r.y) * frag::kLog2e),
+                      frag::ex2_approx((v[u].z - r.z) * frag::kLog2e),
+                      frag::ex2_approx((v[u].w - r.w) * frag::kLog2e));
     }
+  } else {
+    float t = 0.f;
+    if (tid < C) t = __expf(s.G[tid] - s.G[tid < 32 ? kRho0 : kRho1]);
+    __syncthreads();
+    if (tid < C) s.G[tid] = t;
   }
   // factor u at (i, c), (i, c + 1), c even (phase gate: the pair's complex u)
   auto ep2 = [&](int i, int c) -> float2 {
@@ -538,6 +544,13 @@ __global__ void __launch_bounds__(NTB, 1)
       const uint4 rq = *reinterpret_cast<const uint4*>(s.QR + i * LDD + c);
       const uint32_t* wq = reinterpret_cast<const uint32_t*>(&rq);
       uint32_t okb[4], oq[4], ox[4], obk[4];
+      // the cross-half factors of these 8 channels (real gates): write keys of
+      // the first half, queries of the second
+      float xa[8], xb[8];
+      if (!PHASE) {
+        frag::load8((h1 ? s.xq : s.xk) + c, xa);
+        frag::load8((h1 ? s.xq : s.xk) + D + c, xb);
+      }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 kk = frag::unpack(wk[e]), qq = frag::unpack(wq[e]);
@@ -564,9 +577,9 @@ __global__ void __launch_bounds__(NTB, 1)
           okb[e] = frag::pack(kb0, kb1);
           oq[e] = frag::pack(qf0, qf1);
           if (!h1) {
-            ox[e] = frag::pack(kb0 * s.xk[cc] * s.xk[D + cc], kb1 * s.xk[cc + 1] * s.xk[D + cc + 1]);
+            ox[e] = frag::pack(kb0 * xa[2 * e] * xb[2 * e], kb1 * xa[2 * e + 1] * xb[2 * e + 1]);
           } else {
-            ox[e] = frag::pack(qf0 * s.xq[cc] * s.xq[D + cc], qf1 * s.xq[cc + 1] * s.xq[D + cc + 1]);
+            ox[e] = frag::pack(qf0 * xa[2 * e] * xb[2 * e], qf1 * xa[2 * e + 1] * xb[2 * e + 1]);
             obk[e] = frag::pack(bi * kk.x * f[2 * e], bi * kk.y * f[2 * e + 1]);
           }
         }
@@ -583,6 +596,11 @@ __global__ void __launch_bounds__(NTB, 1)
       }
     } else {
       uint32_t ob[4];
+      float xa[8], xb[8];  // the queries' cross-half factors (second half, real gates)
+      if (!PHASE && h1) {
+        frag::load8(s.xq + c, xa);
+        frag::load8(s.xq + D + c, xb);
+      }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 kk = frag::unpack(wk[e]);
@@ -594,8 +612,8 @@ __global__ void __launch_bounds__(NTB, 1)
         } else {
           float b0 = bi * kk.x * f[2 * e], b1 = bi * kk.y * f[2 * e + 1];
           if (h1) {
-            b0 = b0 * s.xq[cc] * s.xq[D + cc];
-            b1 = b1 * s.xq[cc + 1] * s.xq[D + cc + 1];
+            b0 = b0 * xa[2 * e] * xb[2 * e];
+            b1 = b1 * xa[2 * e + 1] * xb[2 * e + 1];
           }
           ob[e] = frag::pack(b0, b1);
         }

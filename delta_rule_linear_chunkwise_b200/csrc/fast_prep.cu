@@ -143,21 +143,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// 2^x (the ex2.approx.ftz instruction: relative error about 2^-22, flushes
-// results below the normal range to zero)
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-constexpr float kLog2e = 1.4426950408889634f;
-
-// Eight consecutive floats of a 16-byte aligned shared-memory array.
-__device__ __forceinline__ void load8(const float* p, float* f) {
-  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
-  f[0] = a.x, f[1] = a.y, f[2] = a.z, f[3] = a.w, f[4] = b.x, f[5] = b.y, f[6] = b.z, f[7] = b.w;
-}
-
 __device__ __forceinline__ void unpack8(const uint4& r, float* f) {
   const uint32_t* w = reinterpret_cast<const uint32_t*>(&r);
 #pragma unroll
@@ -403,19 +388,19 @@ __global__ void __launch_bounds__(NTP, 2)
         }
         // the per-channel reference factors of these 8 channels (vector loads)
         float r8[8], z8[8], e8[8], x0[8], x1[8];
-        load8(s.ref[hr] + c0, r8);
-        load8(s.zr[hr] + c0, z8);
-        load8(s.ec[hr] + c0, e8);
+        frag::load8(s.ref[hr] + c0, r8);
+        frag::load8(s.zr[hr] + c0, z8);
+        frag::load8(s.ec[hr] + c0, e8);
         if (hr == 0) {
-          load8(s.xk[0] + c0, x0);
-          load8(s.xk[1] + c0, x1);
+          frag::load8(s.xk[0] + c0, x0);
+          frag::load8(s.xk[1] + c0, x1);
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           float ep = eps_, em = ems_;
           if (chan) {  // e^{+-(g - g_rho)} as 2^{+-(g - g_rho) log2 e}
-            const float d2 = (gg[e] - r8[e]) * kLog2e;
-            ep = ex2_approx(d2), em = ex2_approx(-d2);
+            const float d2 = (gg[e] - r8[e]) * frag::kLog2e;
+            ep = frag::ex2_approx(d2), em = frag::ex2_approx(-d2);
           }
           kc[e] = kv[e] * ep;
           qc[e] = qv[e] * ep;

@@ -1,5 +1,6 @@
-// frag.cuh -- bf16 packing, the warp-level accumulator fragment store, and
-// cp.async staging shared by the tensor-core kernels.
+// frag.cuh -- bf16 packing, the warp-level accumulator fragment store,
+// cp.async staging and small element-wise helpers shared by the tensor-core
+// kernels.
 //
 // Accumulator fragments (the register layout tcgen05.ld.16x256b returns for an
 // M = 64 accumulator, the same as a warp-level m16n8 product's C):
@@ -43,6 +44,21 @@ __device__ __forceinline__ void st_c(const float (&c)[NT][4], bf16* t, int ld, i
     *reinterpret_cast<uint32_t*>(t + toff(r, cc + j * 8, ld)) = pack(c[j][0], c[j][1]);
     *reinterpret_cast<uint32_t*>(t + toff(r + 8, cc + j * 8, ld)) = pack(c[j][2], c[j][3]);
   }
+}
+
+// 2^x (the ex2.approx.ftz instruction: relative error about 2^-22, flushes
+// results below the normal range to zero)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Eight consecutive floats of a 16-byte aligned shared-memory array.
+__device__ __forceinline__ void load8(const float* p, float* f) {
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  f[0] = a.x, f[1] = a.y, f[2] = a.z, f[3] = a.w, f[4] = b.x, f[5] = b.y, f[6] = b.z, f[7] = b.w;
 }
 
 // cp.async 16-byte copy (zero-filled when !valid).
