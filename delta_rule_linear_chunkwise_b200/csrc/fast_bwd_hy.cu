@@ -80,6 +80,9 @@ constexpr int kRho0 = 15, kRho1 = 47;  // reference rows of the two halves
 
 // Gate tile element (i, c): 8-column groups XOR-swizzled by row.
 __device__ __forceinline__ int gsw(int i, int c) { return i * D + (c ^ ((i & 7) << 3)); }
+// v tile element (i, a) (bf16): 16-byte chunks XOR-swizzled by row, so that the
+// fragment reads (8 rows, 4 consecutive pairs) hit distinct banks.
+__device__ __forceinline__ int vsw(int i, int a) { return i * D + (a ^ ((i & 7) << 3)); }
 
 // Tensor memory columns (512 allocated): each level reuses the columns whose
 // accumulators the previous levels have read back.
@@ -103,7 +106,8 @@ struct HySmem {
   bf16 DO[C * D];   // dO [i][a] (K-major A);  then dW [j][c] (level 2);  then Kb^{rho1} (level 4)
   bf16 DU[C * D];   // dU [j][a];  then q^{rho0} (level 4)
   bf16 UU[2 * kXElems];  // U [j][a] (level 1, first 16 KB);  then the X tiles of dM and dA
-  bf16 QC[C * D];   // Kb^{rho0} rows 0..31 | q^{rho1} rows 32..63 (level 4)
+  bf16 QC[C * D];   // v (rows of 16-byte chunks XOR-swizzled by row, for dv and dbeta);
+                    // then Kb^{rho0} rows 0..31 | q^{rho1} rows 32..63 (level 4)
   bf16 QR[C * LDD]; // raw q, row-major padded
   bf16 k[C * LDD];  // raw k, row-major padded
   bf16 TT[C * C];   // T [i][j], core-tiled (MN-major A of T^T);  then beta k^{rho1} rows 32..63
@@ -353,6 +357,7 @@ __global__ void __launch_bounds__(NTB, 1)
       const size_t rr = row_id(p, b, t0 + (ok ? i : 0), h) * D + j * 8;
       frag::cp16(s.QR + i * LDD + j * 8, q + rr, ok);
       frag::cp16(s.k + i * LDD + j * 8, k + rr, ok);
+      frag::cp16(s.QC + vsw(i, 8 * j), v + rr, ok);
     }
     if (gk == D) {
       for (int idx = lt; idx < C * (D / 4); idx += NL) {
@@ -784,7 +789,7 @@ __global__ void __launch_bounds__(NTB, 1)
     for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh)
-        vv[jt][hh] = *reinterpret_cast<const uint32_t*>(v + rowg[hh] + qt * 32 + jt * 8 + lc);
+        vv[jt][hh] = *reinterpret_cast<const uint32_t*>(s.QC + vsw(i0 + 8 * hh, qt * 32 + jt * 8 + lc));
     ok = hy_wait(&s.bar, 1);
     if (!ok) break;
     float lu[4][4];
