@@ -83,7 +83,6 @@ struct PrepSmem {
   // write keys of the first half against the second reference, in two steps
   // through the half boundary: conj(zeta_31 / zeta_rho0), conj(zeta_rho1 / zeta_31)
   alignas(16) float xk[2][D];
-  float tot[D];      // cumulative gate of the first half's last row
   float gs[C];       // scalar gate: cumulative per row
   float eta[C];      // input beta (eta in Kaczmarz mode)
   float beta[C];     // effective beta
@@ -228,24 +227,38 @@ __global__ void __launch_bounds__(NTP, 2)
   const uint32_t tb = s.tmem;
   do {  // leaves early (break) only when a bounded wait gives up
   if (!ok) break;
-  // ---- cumulative gate down the rows (padded rows carry a zero gate): thread
-  // (channel c, half) scans its 32 rows in registers
+  // ---- cumulative gate down the rows (padded rows carry a zero gate)
   // per-channel element (r, c) of the gate tile: box c / 32, chunk (c % 32) / 4
   auto gp = [&](int r, int c) -> float* {
     return reinterpret_cast<float*>(s.G + (c >> 5) * kBox + swz(r, (c & 31) >> 2) + (c & 3) * 4);
   };
   if (chan) {
-    const int c = tid & 127, hf = tid >> 7;
-    float x[32];
+    // thread: channels 4 qd .. 4 qd + 3 (one 16-byte chunk of a swizzled box), rows
+    // 8 sg .. 8 sg + 7, scanned in registers; then the totals of the earlier row
+    // segments, through the write-key tile (not yet written)
+    const int qd = tid & 31, sg = tid >> 5, c4 = 4 * qd;
+    float4* segtot = reinterpret_cast<float4*>(s.KB);  // [8 segments][32 channel quads]
+    float4 x[8];
 #pragma unroll
-    for (int r = 0; r < 32; ++r) x[r] = *gp(32 * hf + r, c);
+    for (int r = 0; r < 8; ++r) x[r] = *reinterpret_cast<const float4*>(gp(8 * sg + r, c4));
 #pragma unroll
-    for (int r = 1; r < 32; ++r) x[r] += x[r - 1];
-    if (hf == 0) s.tot[c] = x[31];
+    for (int r = 1; r < 8; ++r) {
+      x[r].x += x[r - 1].x;
+      x[r].y += x[r - 1].y;
+      x[r].z += x[r - 1].z;
+      x[r].w += x[r - 1].w;
+    }
+    segtot[sg * 32 + qd] = x[7];
     __syncthreads();
-    const float off = hf ? s.tot[c] : 0.f;
+    float4 off = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s2 = 0; s2 < sg; ++s2) {
+      const float4 t = segtot[s2 * 32 + qd];
+      off.x += t.x, off.y += t.y, off.z += t.z, off.w += t.w;
+    }
 #pragma unroll
-    for (int r = 0; r < 32; ++r) *gp(32 * hf + r, c) = x[r] + off;
+    for (int r = 0; r < 8; ++r)
+      *reinterpret_cast<float4*>(gp(8 * sg + r, c4)) =
+          make_float4(x[r].x + off.x, x[r].y + off.y, x[r].z + off.z, x[r].w + off.w);
   } else if (warp == 0) {
     const float a0 = s.gs[2 * lane], a1 = s.gs[2 * lane + 1];
     float x = a0 + a1;
