@@ -115,7 +115,7 @@ struct HySmem {
   float beta[C];
   float knorm[C];
   float dbp[C * 4];
-  float dgc[4 * D];
+  alignas(16) float dgc[4 * D];
   float ktk[4 * D];
   float er[2 * D];   // per half: conj(zeta_rho)                (real gates: e^{g_rho})
   float erc[2 * D];  // per half: zeta_C / zeta_rho             (real gates: e^{g_C - g_rho})
@@ -135,6 +135,8 @@ struct HySmem {
 };
 
 static_assert(sizeof(bf16) * C * D <= sizeof(bf16) * 2 * kXElems, "U fits the X-tile region");
+static_assert(offsetof(HySmem, ktk) == offsetof(HySmem, dgc) + sizeof(float) * 4 * D,
+              "the gate scan's segment totals span the adjacent dgc and ktk tiles");
 
 // --- complex helpers (a key pair as x + i y) -------------------------------
 struct cf {
@@ -380,21 +382,35 @@ __global__ void __launch_bounds__(NTB, 1)
   auto gat = [&](int i, int c) -> float& { return gk == D ? s.G[gsw(i, c)] : s.G[i]; };
   // cumulative gate down the chunk's rows (padded rows carry a zero gate)
   if (gk == D) {
-    // thread (column c, row quarter q): scan of 16 rows, then the quarter offsets
-    const int c = tid & 127, q4 = tid >> 7;
-    float run = 0.f;
+    // warps 0..7, thread: channels 4 qd .. 4 qd + 3 (16 bytes; the swizzle keeps
+    // them together), rows 8 sg .. 8 sg + 7, scanned in registers; then the
+    // totals of the earlier row segments through the dgc | ktk tiles (free here)
+    const int qd = tid & 31, sg = tid >> 5, c4 = 4 * qd;
+    float4* segtot = reinterpret_cast<float4*>(s.dgc);  // [8 segments][32 channel quads]
+    float4 x[8];
+    if (sg < 8) {
 #pragma unroll
-    for (int i = 16 * q4; i < 16 * q4 + 16; ++i) {
-      run += gat(i, c);
-      gat(i, c) = run;
+      for (int r = 0; r < 8; ++r) x[r] = *reinterpret_cast<const float4*>(s.G + gsw(8 * sg + r, c4));
+#pragma unroll
+      for (int r = 1; r < 8; ++r) {
+        x[r].x += x[r - 1].x;
+        x[r].y += x[r - 1].y;
+        x[r].z += x[r - 1].z;
+        x[r].w += x[r - 1].w;
+      }
+      segtot[sg * 32 + qd] = x[7];
     }
-    s.ktk[q4 * D + c] = run;
     __syncthreads();
-    float off = 0.f;
-    for (int q2 = 0; q2 < q4; ++q2) off += s.ktk[q2 * D + c];
-    if (q4 > 0) {
+    if (sg < 8) {
+      float4 off = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s2 = 0; s2 < sg; ++s2) {
+        const float4 t = segtot[s2 * 32 + qd];
+        off.x += t.x, off.y += t.y, off.z += t.z, off.w += t.w;
+      }
 #pragma unroll
-      for (int i = 16 * q4; i < 16 * q4 + 16; ++i) gat(i, c) += off;
+      for (int r = 0; r < 8; ++r)
+        *reinterpret_cast<float4*>(s.G + gsw(8 * sg + r, c4)) =
+            make_float4(x[r].x + off.x, x[r].y + off.y, x[r].z + off.z, x[r].w + off.w);
     }
   } else if (warp == 0) {
     // rows 2 lane, 2 lane + 1: an inclusive scan across the warp
