@@ -34,10 +34,38 @@ __device__ __forceinline__ int toff(int r, int c, int ld) {
   return ld > 0 ? r * ld + c : (((r >> 3) * ((-ld) >> 3) + (c >> 3)) * 64 + (r & 7) * 8 + (c & 7));
 }
 
-// Store accumulators (rows r0.., cols n0..) as bf16 into a row-major tile.
+// stmatrix / ldmatrix of four 8 x 8 bf16 matrices: lanes 8 m .. 8 m + 7 give the
+// row addresses (16 bytes each) of matrix m; register m of thread t holds the
+// pair (row t / 4, columns 2 (t % 4), + 1) of matrix m -- the accumulator
+// fragment layout above.
+__device__ __forceinline__ void stm_x4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2,
+                                       uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+               "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+               : "memory");
+}
+__device__ __forceinline__ void ldm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+
+// Store accumulators (rows r0 .. r0 + 15, cols n0 .. n0 + 8 NT - 1) as bf16 into
+// a tile (toff layout); a core-tiled tile takes whole 8 x 8 matrices by
+// stmatrix (each is one 128-byte core matrix).
 template <int NT>
 __device__ __forceinline__ void st_c(const float (&c)[NT][4], bf16* t, int ld, int r0, int n0 = 0) {
   const int l = threadIdx.x & 31;
+  if (ld < 0 && NT % 2 == 0) {
+    // matrices of one stmatrix: (r0, j), (r0 + 8, j), (r0, j + 1), (r0 + 8, j + 1)
+    const int m = l >> 3, rr = r0 + (l & 7) + ((m & 1) ? 8 : 0);
+#pragma unroll
+    for (int j = 0; j < NT; j += 2)
+      stm_x4(tc::smem_u32(t + toff(rr, n0 + 8 * (j + (m >> 1)), ld)), pack(c[j][0], c[j][1]),
+             pack(c[j][2], c[j][3]), pack(c[j + 1][0], c[j + 1][1]), pack(c[j + 1][2], c[j + 1][3]));
+    return;
+  }
   const int r = r0 + (l >> 2), cc = n0 + 2 * (l & 3);
 #pragma unroll
   for (int j = 0; j < NT; ++j) {
