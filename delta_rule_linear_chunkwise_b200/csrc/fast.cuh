@@ -69,7 +69,7 @@ struct Saved {
   __nv_bfloat16* M;    // [nb][64][64]    tril(Q^c Kb^c^T)                     [ct]
   __nv_bfloat16* Qh;   // [nb][64][128]   q e^gamma                            [ct]
   __nv_bfloat16* Kt;   // [nb][64][128]   k e^{gamma_C - gamma}                [ct]
-  __nv_bfloat16* h;    // [nb][128][128]  chunk start state S [a][c]             [ct]
+  __nv_bfloat16* h;    // [nb][128][128]  chunk start state S [c][a]             [ct]
   __nv_bfloat16* U;    // [nb][64][128]   U = U' - W S^T                       [ct]
   float* knorm;        // [nb][64]        ||k||^2 of each row
   float* Pseg;         // [B][G][H][128][128] segment transfer matrices (affine scan; else null)

@@ -100,9 +100,9 @@ constexpr uint32_t T_F1 = 0, T_G0 = 128, T_F2 = 256, T_G1 = 384;     // level 4
 constexpr int kXElems = 3 * C * C / 2;  // 12 KB
 
 struct HySmem {
-  bf16 SS[D * D];   // S = h_n [a][c] (level 1);  Lambda_U | Lambda_W (levels 2-3);
+  bf16 SS[D * D];   // S = h_n stored [c][a] (level 1);  Lambda_U | Lambda_W (levels 2-3);
                     // beta k^{rho0} (level 4);  at the end the fp32 dgamma tile (with SD)
-  bf16 SD[D * D];   // dS' [a][c];  then W | U' (level 3)
+  bf16 SD[D * D];   // dS' stored [c][a];  then W | U' (level 3)
   bf16 DO[C * D];   // dO [i][a] (K-major A);  then dW [j][c] (level 2);  then Kb^{rho1} (level 4)
   bf16 DU[C * D];   // dU [j][a];  then q^{rho0} (level 4)
   bf16 UU[2 * kXElems];  // U [j][a] (level 1, first 16 KB);  then the X tiles of dM and dA
@@ -332,18 +332,18 @@ __global__ void __launch_bounds__(NTB, 1)
   // (descriptors are built once; a k-step adds its byte offset / 16 to the start
   // address field, which stays below 2^14 for any shared-memory address)
   if (tid == 0) {
-    const uint32_t id128 = tc::idesc_bf16(64, 128, false, true);
+    const uint32_t id128 = tc::idesc_bf16(64, 128, false, false);  // B = the state, K-major [c][a]
     const uint32_t id64 = tc::idesc_bf16(64, 64, false, false);
     const uint64_t aDO = tc::sdesc_kmaj(s.DO, D, 0), aDU = tc::sdesc_kmaj(s.DU, D, 0);
     const uint64_t aUU = tc::sdesc_kmaj(s.UU, D, 0);
-    const uint64_t bSS = tc::sdesc_mnmaj(s.SS, D, 0), bSD = tc::sdesc_mnmaj(s.SD, D, 0);
+    const uint64_t bSS = tc::sdesc_kmaj(s.SS, D, 0), bSD = tc::sdesc_kmaj(s.SD, D, 0);
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
       const uint32_t acc = ks > 0 ? 1u : 0u;
-      const uint64_t ka = 16u * ks, kb = 256u * ks;  // K-major / MN-major k-step, 16-byte units
-      mma_step(tb + T_ZQ, aDO + ka, bSS + kb, id128, acc);
-      mma_step(tb + T_ADW, aDU + ka, bSS + kb, id128, acc);
-      mma_step(tb + T_AKT, aUU + ka, bSD + kb, id128, acc);
+      const uint64_t ka = 16u * ks;  // K-major k-step, 16-byte units
+      mma_step(tb + T_ZQ, aDO + ka, bSS + ka, id128, acc);
+      mma_step(tb + T_ADW, aDU + ka, bSS + ka, id128, acc);
+      mma_step(tb + T_AKT, aUU + ka, bSD + ka, id128, acc);
       mma_step(tb + T_ADM, aDO + ka, aUU + ka, id64, acc);
     }
     tc::commit(&s.bar);
@@ -643,42 +643,48 @@ __global__ void __launch_bounds__(NTB, 1)
     }
   };
 
-  // colsum(conj(dS') S) while level 1 runs (real gates: per channel sum of dS' .* S):
-  // thread -> 8 columns (16-byte core rows), 4 rows (one per row group of its
-  // quarter); eight lanes read the eight rows of one core matrix
+  // colsum(conj(dS') S) while level 1 runs (real gates: per key channel c the sum
+  // over a of dS'[c][a] S[c][a]; the state tiles are stored [c][a]).  Thread:
+  // row r of the core matrices of row blocks 4 q .. 4 q + 3 (keys c), 16-byte
+  // chunk j (8 values a); eight lanes read one whole core matrix.  Partial sums
+  // reduce over the warp's four chunks, then land in one of four slots per key
+  // (warp % 4), summed by the reader.
   {
-    const int alo = tid & 7, cg = (tid >> 3) & 15, ag = tid >> 7;
-    float acc[8] = {};
+    const int r = tid & 7, j = (tid >> 3) & 15, q = tid >> 7;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int o = ct_off((ag * 4 + r) * 8 + alo, 8 * cg, D);
+    for (int rr = 0; rr < 4; ++rr) {
+      const int c = (4 * q + rr) * 8 + r;
+      const int o = ct_off(c, 8 * j, D);
       const uint4 x = *reinterpret_cast<const uint4*>(s.SS + o);
       const uint4 y = *reinterpret_cast<const uint4*>(s.SD + o);
       const uint32_t* wx = reinterpret_cast<const uint32_t*>(&x);
       const uint32_t* wy = reinterpret_cast<const uint32_t*>(&y);
+      float pr = 0.f, cross = 0.f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 fx = frag::unpack(wx[e]), fy = frag::unpack(wy[e]);
-        if (PHASE) {  // conj(dS') S of the pair: (dx sx + dy sy) + i (dx sy - dy sx)
-          acc[2 * e] += fy.x * fx.x + fy.y * fx.y;
-          acc[2 * e + 1] += fy.x * fx.y - fy.y * fx.x;
-        } else {
-          acc[2 * e] += fx.x * fy.x;
-          acc[2 * e + 1] += fx.y * fy.y;
+        pr += fx.x * fy.x + fx.y * fy.y;
+        if (PHASE) {
+          // the pair's odd key (lane ^ 1) for the cross term of conj(dS') S:
+          // Im = sum_a (dx sy - dy sx), x the even key, y the odd one
+          const float2 gx = frag::unpack(__shfl_xor_sync(0xffffffffu, wx[e], 1));
+          const float2 gy = frag::unpack(__shfl_xor_sync(0xffffffffu, wy[e], 1));
+          cross += fy.x * gx.x + fy.y * gx.y - gy.x * fx.x - gy.y * fx.y;
         }
       }
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      float x = acc[e];
-      x += __shfl_xor_sync(0xffffffffu, x, 1);
-      x += __shfl_xor_sync(0xffffffffu, x, 2);
-      x += __shfl_xor_sync(0xffffffffu, x, 4);
-      acc[e] = x;
-    }
-    if (alo == 0) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s.dgc[ag * D + 8 * cg + e] = acc[e];
+      pr += __shfl_xor_sync(0xffffffffu, pr, 8);
+      pr += __shfl_xor_sync(0xffffffffu, pr, 16);
+      if (PHASE) {
+        cross += __shfl_xor_sync(0xffffffffu, cross, 8);
+        cross += __shfl_xor_sync(0xffffffffu, cross, 16);
+        const float po = __shfl_xor_sync(0xffffffffu, pr, 1);
+        if ((lane >> 3) == 0 && (r & 1) == 0) {
+          s.dgc[(warp & 3) * D + c] = pr + po;     // Re: dx sx + dy sy
+          s.dgc[(warp & 3) * D + c + 1] = cross;  // Im
+        }
+      } else if ((lane >> 3) == 0) {
+        s.dgc[(warp & 3) * D + c] = pr;
+      }
     }
   }
   ok = hy_wait(&s.bar, 0);

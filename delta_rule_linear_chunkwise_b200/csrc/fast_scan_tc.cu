@@ -88,33 +88,17 @@ __device__ __forceinline__ void scan_fill(ScanStage<BV>& s, uint64_t* full, cons
   frag::cp_commit();
 }
 
-// Writes this thread's HB state values x[u] (rows a0h + u, key c; one key per
-// lane) as bf16 into a core-tiled [128][128] state tile.  Each 8 x 8 block is
-// transposed across the 8 lanes that hold its keys (xor shuffles), so every
-// lane stores 16 contiguous bytes (row a, keys c0 .. c0 + 7) and a warp writes
-// four whole 128-byte core matrices.
+// Writes this thread's HB state values x[u] (value rows a0h + u of key c; one
+// key per lane) as bf16 into a core-tiled state tile stored transposed, [key
+// c][value a] (the K-major B operand of the chunk backward's products with the
+// state): a thread's values are 16-byte runs of its own row, and a warp writes
+// four whole 128-byte core matrices per store.
 template <int HB>
-__device__ __forceinline__ void store_state_ct(bf16* dst, const float* x, int a0h, int c,
-                                               int lane) {
+__device__ __forceinline__ void store_state_ct(bf16* dst, const float* x, int a0h, int c) {
 #pragma unroll
   for (int u8 = 0; u8 < HB / 8; ++u8) {
-    float v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = x[8 * u8 + j];
-#pragma unroll
-    for (int sh = 1; sh < 8; sh <<= 1) {
-      const bool hi = lane & sh;
-#pragma unroll
-      for (int j0 = 0; j0 < 8; ++j0) {
-        if (j0 & sh) continue;
-        const int j1 = j0 | sh;
-        const float y = __shfl_xor_sync(0xffffffffu, hi ? v[j0] : v[j1], sh);
-        if (hi) v[j0] = y;
-        else v[j1] = y;
-      }
-    }
-    const int a = a0h + 8 * u8 + (lane & 7);
-    *reinterpret_cast<uint4*>(dst + ct_off(a, c & ~7, D)) =
+    const float* v = x + 8 * u8;
+    *reinterpret_cast<uint4*>(dst + ct_off(c, a0h + 8 * u8, D)) =
         make_uint4(frag::pack(v[0], v[1]), frag::pack(v[2], v[3]), frag::pack(v[4], v[5]),
                    frag::pack(v[6], v[7]));
   }
@@ -198,9 +182,9 @@ __global__ void __launch_bounds__(NTF, 1)
                      frag::pack(f[6], f[7]));
     }
   };
-  // h_n (bf16, core-tiled [a][c]) from the registers
+  // h_n (bf16, core-tiled [c][a]) from the registers
   auto store_h = [&](size_t cbn) {
-    store_state_ct<HB>(sv.h + cbn * D * D, S, a0 + ah * HB, c, lane);
+    store_state_ct<HB>(sv.h + cbn * D * D, S, a0 + ah * HB, c);
   };
   // o rows of chunk nn from D_A buffer `buf` (warps on lanes 64 .. 127)
   auto store_o = [&](int nn, int buf) {
@@ -532,9 +516,9 @@ __global__ void __launch_bounds__(NTF, 1)
                      frag::pack(f[6], f[7]));
     }
   };
-  // dh (bf16, core-tiled [a][c]) from the registers
+  // dh (bf16, core-tiled [c][a]) from the registers
   auto store_dh = [&](size_t cbn) {
-    store_state_ct<HB>(dhout + cbn * D * D, dS, a0 + ah * HB, c, lane);
+    store_state_ct<HB>(dhout + cbn * D * D, dS, a0 + ah * HB, c);
   };
 
   write_dsb();
