@@ -52,7 +52,7 @@ struct ScanSmem {
   ScanStage<BV> st[2];
   bf16 SB[D * BV];     // bf16 S^T, MN-major B of MMA-A ([K = c][N = a])
   bf16 UB[C * BV];     // bf16 U, MN-major B of MMA-B / MMA-C ([K = i][N = a])
-  uint64_t barA, barB, full[2];
+  uint64_t barA, barB, barO, full[2];
   uint32_t tmem;
 };
 
@@ -62,25 +62,35 @@ __host__ __device__ constexpr uint32_t scan_fill_bytes(bool with_o) {
 }
 
 // Fills a stage, called by every thread: the chunk tiles, stored core-tiled in
-// HBM (the layout of the operands here), by one bulk copy each from lane 0 of
-// warps 0..4, completing on `full` (whose transaction count thread 0 has set
-// with scan_fill_bytes before a barrier that precedes this; a bulk copy holds
-// its issuing thread while the copy engine takes it, so they are spread over
-// the warps), and U'[:, a0 .. a0 + BV) (one run of BV / 8 core matrices per
-// block of 8 rows) by cp.async from every thread, one group (committed also
-// when empty).
+// HBM (the layout of the operands here), by bulk copies from lane 0 of warps 1,
+// 4 and 5 (the warps that neither issue MMA-A nor store o at the top of a step;
+// a bulk copy holds its issuing thread while the copy engine takes it),
+// completing on `full` (whose transaction count thread 0 has set with
+// scan_fill_bytes before a barrier that precedes this), and U'[:, a0 .. a0 + BV)
+// (one run of BV / 8 core matrices per block of 8 rows) by cp.async from every
+// thread, one group (committed also when empty).
+// The stage's M tile was last read by the output product (MMA-B) of the step
+// two chunks back, which completes on its own barrier: when `mb_parity` >= 0 the
+// copy of M waits (bounded) for that phase of `barO` first.
 template <int BV>
 __device__ __forceinline__ void scan_fill(ScanStage<BV>& s, uint64_t* full, const Saved& sv,
                                           size_t cb, int a0, bool with_o, bool with_up,
-                                          int warp, int lane) {
+                                          int warp, int lane, uint64_t* barO, int mb_parity) {
   constexpr uint32_t kT = sizeof(bf16) * C * D, kM = sizeof(bf16) * C * C;
   if (lane == 0) {
     switch (warp) {
-      case 0: tc::bulk_g2s(s.AWQ, sv.W + cb * C * D, kT, full); break;
-      case 1: tc::bulk_g2s(s.KT, sv.Kt + cb * C * D, kT, full); break;
-      case 2: if (with_o) tc::bulk_g2s(s.AWQ + C * D, sv.Qh + cb * C * D, kT, full); break;
-      case 3: if (with_o) tc::bulk_g2s(s.MZ + C * C, sv.M + cb * C * C, kM, full); break;
-      case 4: tc::bulk_g2s(s.dec, sv.dec + cb * D, sizeof(float) * D, full); break;
+      case 1:
+        tc::bulk_g2s(s.AWQ, sv.W + cb * C * D, kT, full);
+        tc::bulk_g2s(s.KT, sv.Kt + cb * C * D, kT, full);
+        break;
+      case 4:
+        if (with_o) {
+          tc::bulk_g2s(s.AWQ + C * D, sv.Qh + cb * C * D, kT, full);
+          if (mb_parity < 0 || tc::mbar_wait(barO, (uint32_t)(mb_parity & 1), kSpinScan))
+            tc::bulk_g2s(s.MZ + C * C, sv.M + cb * C * C, kM, full);
+        }
+        break;
+      case 5: tc::bulk_g2s(s.dec, sv.dec + cb * D, sizeof(float) * D, full); break;
       default: break;
     }
   }
@@ -109,9 +119,9 @@ __device__ __forceinline__ uint32_t lane_addr(uint32_t base, int warp, int col) 
 }
 
 // Bounded wait on an mbarrier phase; the result is uniform over the CTA.
-__device__ __forceinline__ bool cta_wait(uint64_t* bar, int parity) {
+__device__ __forceinline__ bool cta_wait(uint64_t* bar, int parity, bool local_bad = false) {
   const bool ok = tc::mbar_wait(bar, (uint32_t)(parity & 1), kSpinScan);
-  const int bad = __syncthreads_or(ok ? 0 : 1);
+  const int bad = __syncthreads_or((ok && !local_bad) ? 0 : 1);
   tc::fence_after_sync();
   return bad == 0;
 }
@@ -154,6 +164,7 @@ __global__ void __launch_bounds__(NTF, 1)
   if (tid == 0) {
     tc::mbar_init(&s.barA, 1);
     tc::mbar_init(&s.barB, 1);
+    tc::mbar_init(&s.barO, 1);
     tc::mbar_init(&s.full[0], 1);
     tc::mbar_init(&s.full[1], 1);
     tc::fence_mbar_init();
@@ -187,8 +198,10 @@ __global__ void __launch_bounds__(NTF, 1)
     store_state_ct<HB>(sv.h + cbn * D * D, S, a0 + ah * HB, c);
   };
   // o rows of chunk nn from D_A buffer `buf` (warps on lanes 64 .. 127)
-  auto store_o = [&](int nn, int buf) {
-    if ((warp & 3) < 2) return;
+  auto store_o = [&](int nn, int buf, int ph) -> bool {
+    if ((warp & 3) < 2) return true;
+    if (!tc::mbar_wait(&s.barO, (uint32_t)(ph & 1), kSpinScan)) return false;
+    tc::fence_after_sync();
     const int i = 32 * ((warp & 3) - 2) + lane;
     const int t0 = nn * C, nvalid = min(C, p.T - t0);
     uint32_t r[HB];
@@ -206,6 +219,7 @@ __global__ void __launch_bounds__(NTF, 1)
                        frag::pack(f[6], f[7]));
       }
     }
+    return true;
   };
 
   write_sb();
@@ -221,16 +235,10 @@ __global__ void __launch_bounds__(NTF, 1)
     if (n0 + 1 < n1) tc::mbar_arrive_expect_tx(&s.full[1], fill_tx);
   }
   __syncthreads();
-  scan_fill<BV>(s.st[0], &s.full[0], sv, chunk_id(p, b, h, n0), a0, with_o, with_up, warp, lane);
+  scan_fill<BV>(s.st[0], &s.full[0], sv, chunk_id(p, b, h, n0), a0, with_o, with_up, warp, lane,
+                &s.barO, -1);
   fills[0] = 1;
-  if (n0 + 1 < n1) {
-    scan_fill<BV>(s.st[1], &s.full[1], sv, chunk_id(p, b, h, n0 + 1), a0, with_o, with_up, warp,
-                  lane);
-    fills[1] = 1;
-  } else {
-    frag::cp_commit();  // an empty group: one group per fill slot keeps the waits below exact
-  }
-  frag::cp_wait<1>();
+  frag::cp_wait<0>();
   bool ok = tc::mbar_wait(&s.full[0], 0u, kSpinScan);
   tc::fence_smem_to_async();
   tc::fence_before_sync();
@@ -250,19 +258,26 @@ __global__ void __launch_bounds__(NTF, 1)
     const int buf = it & 1;
     const float dc = st.dec[PHASE ? (c & ~1) : c];  // read before the stage is refilled below
     const float di = PHASE ? ((c & 1) ? st.dec[c] : -st.dec[c | 1]) : 0.f;
-    // MMA-A: [W ; q e^gamma] S^T (and the transaction count of this stage's refill,
-    // whose copies follow two barriers later)
+    // MMA-A: [W ; q e^gamma] S^T
     if (tid == 0) {
-      if (n + 2 < n1) tc::mbar_arrive_expect_tx(&s.full[it & 1], fill_tx);
       const uint64_t dA = tc::sdesc_kmaj(st.AWQ, D, 0);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks)
         tc::mma(tbase + buf * BV, dA + ks * kKM, dSB + ks * kSB, idA, ks > 0 ? 1u : 0u);
       tc::commit(&s.barA);
     }
-    // while it runs: the previous chunk's output
-    if (with_o && it > 0) store_o(n - 1, buf ^ 1);
-    ok = cta_wait(&s.barA, it);
+    // while it runs: the next chunk's tiles into the other stage (consumed by the
+    // previous step; it lands by the end of this one) and the previous chunk's output
+    if (n + 1 < n1) {
+      scan_fill<BV>(s.st[(it + 1) & 1], &s.full[(it + 1) & 1], sv, chunk_id(p, b, h, n + 1), a0,
+                    with_o, with_up, warp, lane, &s.barO, it - 1);
+      ++fills[(it + 1) & 1];
+    } else {
+      frag::cp_commit();  // empty group
+    }
+    bool badO = false;
+    if (with_o && it > 0) badO = !store_o(n - 1, buf ^ 1, it - 1);
+    ok = cta_wait(&s.barA, it, badO);
     if (!ok) break;
     // epilogue 1: U = U' - W S^T (rows i = lanes 0 .. 63)
     uint4 usave[HB / 8];
@@ -294,19 +309,20 @@ __global__ void __launch_bounds__(NTF, 1)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    // MMA-B (output) and MMA-C (state increment)
+    // MMA-C (state increment, thread 0) and MMA-B (output, thread 32, its own
+    // barrier: only the next step's output store waits for it)
     if (tid == 0) {
-      if (with_o) {
-        const uint64_t dM = tc::sdesc_kmaj(st.MZ, C, 0);
-#pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks)
-          tc::mma(tbase + buf * BV, dM + ks * kKM, dUB + ks * kUB, idA, 1u);
-      }
       const uint64_t dK = tc::sdesc_mnmaj(st.KT, D, 0);
 #pragma unroll
       for (int ks = 0; ks < C / 16; ++ks)
         tc::mma(tbase + T_S, dK + ks * kKT, dUB + ks * kUB, idC, ks > 0 ? 1u : 0u);
       tc::commit(&s.barB);
+    } else if (with_o && tid == 32) {
+      const uint64_t dM = tc::sdesc_kmaj(st.MZ, C, 0);
+#pragma unroll
+      for (int ks = 0; ks < C / 16; ++ks)
+        tc::mma(tbase + buf * BV, dM + ks * kKM, dUB + ks * kUB, idA, 1u);
+      tc::commit(&s.barO);
     }
     // while they run: U and the chunk-start state to global memory
     if (save) {
@@ -320,14 +336,9 @@ __global__ void __launch_bounds__(NTF, 1)
     }
     ok = cta_wait(&s.barB, it);
     if (!ok) break;
-    // this stage is consumed: refill it with chunk n + 2 (lands during the next step)
-    if (n + 2 < n1) {
-      scan_fill<BV>(st, &s.full[it & 1], sv, chunk_id(p, b, h, n + 2), a0, with_o, with_up, warp,
-                    lane);
-      ++fills[it & 1];
-    } else {
-      frag::cp_commit();  // empty group
-    }
+    // this stage is consumed: the transaction count of its refill (chunk n + 2,
+    // whose copies the next step issues after the barrier below)
+    if (tid == 0 && n + 2 < n1) tc::mbar_arrive_expect_tx(&s.full[it & 1], fill_tx);
     // epilogue 2: S^T <- Diag(e^{gamma_C}) S^T + D_S
     {
       uint32_t r[HB];
@@ -348,10 +359,9 @@ __global__ void __launch_bounds__(NTF, 1)
       }
       write_sb();
     }
-    // the next chunk's stage (filled one step ago; its U' group is the older of
-    // the two outstanding ones)
+    // the next chunk's stage (filled at the top of this step)
     bool okF = true;
-    frag::cp_wait<1>();
+    frag::cp_wait<0>();
     if (n + 1 < n1) okF = tc::mbar_wait(&s.full[(it + 1) & 1], (uint32_t)(((it + 1) >> 1) & 1), kSpinScan);
     tc::fence_smem_to_async();
     tc::fence_before_sync();
@@ -359,7 +369,7 @@ __global__ void __launch_bounds__(NTF, 1)
     tc::fence_after_sync();
   }
   if (ok) {
-    if (with_o) store_o(n1 - 1, (n1 - 1 - n0) & 1);
+    if (with_o && !store_o(n1 - 1, (n1 - 1 - n0) & 1, n1 - 1 - n0) && err) atomicExch(err, 1);
     if (ST) {
 #pragma unroll
       for (int u = 0; u < HB; ++u) ST[sbase + (size_t)(a0 + ah * HB + u) * D + c] = S[u];
