@@ -154,6 +154,12 @@ __device__ __forceinline__ cf cinv(cf u) {
   return {a * t, -b * t};
 }
 
+// Barrier among `count` threads (whole warps) on hardware barrier `id` (1..15;
+// barrier 0 is __syncthreads).
+__device__ __forceinline__ void named_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ void mma_step(uint32_t tm, uint64_t a, uint64_t b, uint32_t id,
                                          uint32_t acc) {
   tc::mma(tm, a, b, id, acc);
@@ -348,8 +354,9 @@ __global__ void __launch_bounds__(NTB, 1)
     }
     tc::commit(&s.bar);
   }
-  // q, k, the gate, beta and ||k||^2 of this chunk by warps 1..15 (warp 0 issues
-  // level 1)
+  // q, k, v, the gate, beta and ||k||^2 of this chunk by warps 1..15, then the
+  // gate's cumulative sum by warps 8..15, while warp 0 issues level 1 (named
+  // barriers 1 and 2 hold only the warps that take part)
   if (warp > 0) {
     const int lt = tid - 32;
     constexpr int NL = NTB - 32;
@@ -374,57 +381,54 @@ __global__ void __launch_bounds__(NTB, 1)
       s.beta[lt - C] = beta[cb * C + lt - C];
       s.knorm[lt - C] = knorm_g[cb * C + lt - C];
     }
+    frag::cp_commit();
+    frag::cp_wait<0>();
+    named_sync(1, NTB - 32);  // warps 1..15: their copies have landed
+    if (gk == D) {
+      if (warp >= 8) {
+        // thread: channels 4 lane .. + 3 (16 bytes; the swizzle keeps them
+        // together), rows 8 sg .. 8 sg + 7 (sg = warp - 8), scanned in registers;
+        // then the totals of the earlier row segments through the dgc | ktk tiles
+        const int sg = warp - 8, c4 = 4 * lane;
+        float4* segtot = reinterpret_cast<float4*>(s.dgc);  // [8 segments][32 channel quads]
+        float4 x[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) x[r] = *reinterpret_cast<const float4*>(s.G + gsw(8 * sg + r, c4));
+#pragma unroll
+        for (int r = 1; r < 8; ++r) {
+          x[r].x += x[r - 1].x;
+          x[r].y += x[r - 1].y;
+          x[r].z += x[r - 1].z;
+          x[r].w += x[r - 1].w;
+        }
+        segtot[sg * 32 + lane] = x[7];
+        named_sync(2, NTB / 2);  // warps 8..15
+        float4 off = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s2 = 0; s2 < sg; ++s2) {
+          const float4 t = segtot[s2 * 32 + lane];
+          off.x += t.x, off.y += t.y, off.z += t.z, off.w += t.w;
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+          *reinterpret_cast<float4*>(s.G + gsw(8 * sg + r, c4)) =
+              make_float4(x[r].x + off.x, x[r].y + off.y, x[r].z + off.z, x[r].w + off.w);
+      }
+    } else if (warp == 1) {
+      // rows 2 lane, 2 lane + 1: an inclusive scan across the warp
+      const float a0v = s.G[2 * lane], a1v = s.G[2 * lane + 1];
+      float x = a0v + a1v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      s.G[2 * lane + 1] = x;
+      s.G[2 * lane] = x - a1v;
+    }
   }
-  frag::cp_commit();
-  frag::cp_wait<0>();
   __syncthreads();
   // element (i, c) of the gate tile
   auto gat = [&](int i, int c) -> float& { return gk == D ? s.G[gsw(i, c)] : s.G[i]; };
-  // cumulative gate down the chunk's rows (padded rows carry a zero gate)
-  if (gk == D) {
-    // warps 0..7, thread: channels 4 qd .. 4 qd + 3 (16 bytes; the swizzle keeps
-    // them together), rows 8 sg .. 8 sg + 7, scanned in registers; then the
-    // totals of the earlier row segments through the dgc | ktk tiles (free here)
-    const int qd = tid & 31, sg = tid >> 5, c4 = 4 * qd;
-    float4* segtot = reinterpret_cast<float4*>(s.dgc);  // [8 segments][32 channel quads]
-    float4 x[8];
-    if (sg < 8) {
-#pragma unroll
-      for (int r = 0; r < 8; ++r) x[r] = *reinterpret_cast<const float4*>(s.G + gsw(8 * sg + r, c4));
-#pragma unroll
-      for (int r = 1; r < 8; ++r) {
-        x[r].x += x[r - 1].x;
-        x[r].y += x[r - 1].y;
-        x[r].z += x[r - 1].z;
-        x[r].w += x[r - 1].w;
-      }
-      segtot[sg * 32 + qd] = x[7];
-    }
-    __syncthreads();
-    if (sg < 8) {
-      float4 off = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s2 = 0; s2 < sg; ++s2) {
-        const float4 t = segtot[s2 * 32 + qd];
-        off.x += t.x, off.y += t.y, off.z += t.z, off.w += t.w;
-      }
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-        *reinterpret_cast<float4*>(s.G + gsw(8 * sg + r, c4)) =
-            make_float4(x[r].x + off.x, x[r].y + off.y, x[r].z + off.z, x[r].w + off.w);
-    }
-  } else if (warp == 0) {
-    // rows 2 lane, 2 lane + 1: an inclusive scan across the warp
-    const float a0v = s.G[2 * lane], a1v = s.G[2 * lane + 1];
-    float x = a0v + a1v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    s.G[2 * lane + 1] = x;
-    s.G[2 * lane] = x - a1v;
-  }
-  __syncthreads();
 
   // per-channel reference factors (phase gate: per pair, complex, at the pair's two channels)
   if (PHASE) {
