@@ -872,9 +872,11 @@ __global__ void __launch_bounds__(NTB, 1)
       }
     tc::commit(&s.bar);
   }
-  // ---- under level 3: the dA-free level-4 operands, then their products
-  //      F1 = dM Kb (per-half references) and the dM half of G for the first half
-  for (int idx = tid; idx < C * (D / 8); idx += NTB) build_row(idx, true);
+  // ---- under level 3: the dA-free level-4 operands (warps 1..15: warp 0 issues
+  //      level 3), then their products F1 = dM Kb (per-half references) and the
+  //      dM half of G for the first half
+  if (warp > 0)
+    for (int idx = tid - 32; idx < C * (D / 8); idx += NTB - 32) build_row(idx, true);
   tc::fence_smem_to_async();
   tc::fence_before_sync();
   __syncthreads();
