@@ -887,6 +887,10 @@ __global__ void __launch_bounds__(NTB, 1)
   const uint64_t xmK = dk64(XM, 0), xaK = dk64(XA, 0), xmT = dmn64(XM, 0), xaT = dmn64(XA, 0);
   const uint64_t dKb0 = dmn128(Kb0, 0), dKb1 = dmn128(Kb1, 0), dQ0 = dmn128(Q0, 0);
   const uint64_t dQ1 = dmn128(Q1, 0), dB0 = dmn128(B0, 0), dB1 = dmn128(B1, 0);
+  ok = hy_wait(&s.bar, 2);
+  if (!ok) break;
+  // level 4, dM part (thread 0, after the barrier above: the other warps go on
+  // to the dA readout without waiting for the issue)
   if (tid == 0) {
     // F1: rows of the first half against Kb^{rho0} (k-steps 0, 1), rows of the
     // second half against Kb^{rho1} (k-steps 0..3); one accumulator
@@ -900,8 +904,6 @@ __global__ void __launch_bounds__(NTB, 1)
       if (ks >= 2) mma_step(tb + T_G0, xmT + xt_off(ks) / 16, dQ0 + 256 * ks, idG, 1u);
     }
   }
-  ok = hy_wait(&s.bar, 2);
-  if (!ok) break;
   {
     float da[2][4], dp[2][4];
     frag_ld2(tb + T_DA + 16 * qt, warp, da);
@@ -922,8 +924,10 @@ __global__ void __launch_bounds__(NTB, 1)
       }
     frag::st_c(da, XA, -C, rb * 16 + (hf ? 32 : 0), qt * 16);
   }
-  // beta k of the first reference into the Lambda tiles (level 3 has read them)
-  for (int idx = tid; idx < C * (D / 8); idx += NTB) build_row(idx, false);
+  // beta k of the first reference into the Lambda tiles (level 3 has read them;
+  // warps 1..15: warp 0 issued the dM part of level 4)
+  if (warp > 0)
+    for (int idx = tid - 32; idx < C * (D / 8); idx += NTB - 32) build_row(idx, false);
   tc::fence_smem_to_async();
   tc::fence_before_sync();
   __syncthreads();
