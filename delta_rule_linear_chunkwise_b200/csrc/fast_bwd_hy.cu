@@ -165,6 +165,33 @@ __device__ __forceinline__ void mma_step(uint32_t tm, uint64_t a, uint64_t b, ui
   tc::mma(tm, a, b, id, acc);
 }
 
+// The raw registers of frag_ld4 / frag_ld2 (below) without the wait: several
+// loads are issued back to back, then one tc::tmem_wait_ld(), then frag_of.
+__device__ __forceinline__ void frag_ld4_raw(uint32_t col, int warp, uint32_t (&r)[16]) {
+  const uint32_t ta = col + ((uint32_t)(32 * (warp & 3)) << 16);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(ta));
+}
+__device__ __forceinline__ void frag_ld2_raw(uint32_t col, int warp, uint32_t (&r)[8]) {
+  const uint32_t ta = col + ((uint32_t)(32 * (warp & 3)) << 16);
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(ta));
+}
+template <int NT>
+__device__ __forceinline__ void frag_of(const uint32_t (&r)[4 * NT], float (&f)[NT][4]) {
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) f[j][e] = __uint_as_float(r[4 * j + e]);
+}
+
 // Fragments of 32 (ld4) or 16 (ld2) accumulator columns from column `col`,
 // rows of this warp's quadrant.
 __device__ __forceinline__ void frag_ld4(uint32_t col, int warp, float (&f)[4][4]) {
@@ -698,10 +725,18 @@ __global__ void __launch_bounds__(NTB, 1)
   cp_linear<NTB>(sUp, Upg + cb * C * D, C * D, tid);
   frag::cp_commit();
   float zq[4][4], adw[4][4], akt[4][4], adm[2][4];
-  frag_ld4(tb + T_ZQ + 32 * qt, warp, zq);
-  frag_ld4(tb + T_ADW + 32 * qt, warp, adw);
-  frag_ld4(tb + T_AKT + 32 * qt, warp, akt);
-  frag_ld2(tb + T_ADM + 16 * qt, warp, adm);
+  {
+    uint32_t rz[16], rw[16], rk[16], rm[8];
+    frag_ld4_raw(tb + T_ZQ + 32 * qt, warp, rz);
+    frag_ld4_raw(tb + T_ADW + 32 * qt, warp, rw);
+    frag_ld4_raw(tb + T_AKT + 32 * qt, warp, rk);
+    frag_ld2_raw(tb + T_ADM + 16 * qt, warp, rm);
+    tc::tmem_wait_ld();
+    frag_of<4>(rz, zq);
+    frag_of<4>(rw, adw);
+    frag_of<4>(rk, akt);
+    frag_of<2>(rm, adm);
+  }
   // dW = -dW', and dM masked (inclusive lower) into its X tile (rows of the
   // second half 4 KB further on, after the zero block written here)
   {
@@ -959,22 +994,19 @@ __global__ void __launch_bounds__(NTB, 1)
     pending = true;
   }
   {
-    float t4[4][4];
-    frag_ld4(tb + T_F1 + 32 * qt, warp, t4);
+    uint32_t r1[16], r2[16], r3[16];
+    frag_ld4_raw(tb + T_F1 + 32 * qt, warp, r1);
+    frag_ld4_raw(tb + T_F2 + 32 * qt, warp, r2);
+    frag_ld4_raw(tb + (hf ? T_G1 : T_G0) + 32 * qt, warp, r3);
+    tc::tmem_wait_ld();
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) Z[j][e] += t4[j][e];
-    frag_ld4(tb + T_F2 + 32 * qt, warp, t4);
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) Q[j][e] += t4[j][e];
-    frag_ld4(tb + (hf ? T_G1 : T_G0) + 32 * qt, warp, t4);
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) P[j][e] += t4[j][e];
+      for (int e = 0; e < 4; ++e) {
+        Z[j][e] += __uint_as_float(r1[4 * j + e]);
+        Q[j][e] += __uint_as_float(r2[4 * j + e]);
+        P[j][e] += __uint_as_float(r3[4 * j + e]);
+      }
   }
 
   // ---- per-element epilogue: dq out; P <- dk (before the Kaczmarz term), Q <- dgamma
