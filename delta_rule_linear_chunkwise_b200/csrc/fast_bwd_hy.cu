@@ -45,12 +45,14 @@
 //
 // Overlap: the level-1 tiles of the CTA's next chunk (dO, dU, U, S, dS', T;
 // 120 KB) are loaded while the epilogue of this one runs, into the tiles that
-// level 4 has released, so a chunk starts with its first products; q, k and the
-// gate (which the epilogue still reads) load under level 1.
+// level 4 has released, so a chunk starts with its first products; q, k, v and
+// the gate (which the epilogue still reads) load, and the gate's cumulative sum
+// runs, on warps 1..15 while warp 0 issues level 1.  Likewise the tile builds
+// under levels 3 and 4 leave warp 0 to its MMA issue.
 //
 // Each level is a set of tcgen05.mma (M = 64, operands in shared memory in the
 // canonical core-matrix layout, fp32 accumulators in tensor memory) issued by
-// one thread.  An M = 64 accumulator occupies lanes 16 q .. 16 q + 15 of each
+// one thread (thread 0).  An M = 64 accumulator occupies lanes 16 q .. 16 q + 15 of each
 // 32-lane quadrant q, and tcgen05.ld.16x256b returns it to the warps of that
 // quadrant in the register fragment of a warp-level m16n8 product (thread t:
 // row t / 4 and t / 4 + 8, columns 2 (t % 4), + 1 of each 8-column group), so
