@@ -275,10 +275,12 @@ __global__ void __launch_bounds__(NTF, 1)
     } else {
       frag::cp_commit();  // empty group
     }
-    bool badO = false;
-    if (with_o && it > 0) badO = !store_o(n - 1, buf ^ 1, it - 1);
-    ok = cta_wait(&s.barA, it, badO);
-    if (!ok) break;
+    bool bad = false;
+    if (with_o && it > 0) bad = !store_o(n - 1, buf ^ 1, it - 1);
+    // each thread waits for MMA-A itself; the barrier after epilogue 1 settles a
+    // failed wait for the whole CTA
+    bad = !tc::mbar_wait(&s.barA, (uint32_t)(it & 1), kSpinScan) || bad;
+    tc::fence_after_sync();
     // epilogue 1: U = U' - W S^T (rows i = lanes 0 .. 63)
     uint4 usave[HB / 8];
     if ((warp & 3) < 2) {
@@ -307,8 +309,9 @@ __global__ void __launch_bounds__(NTF, 1)
     }
     tc::fence_smem_to_async();
     tc::fence_before_sync();
-    __syncthreads();
+    ok = __syncthreads_or(bad ? 1 : 0) == 0;
     tc::fence_after_sync();
+    if (!ok) break;
     // MMA-C (state increment, thread 0) and MMA-B (output, thread 32, its own
     // barrier: only the next step's output store waits for it)
     if (tid == 0) {
@@ -334,8 +337,10 @@ __global__ void __launch_bounds__(NTF, 1)
       }
       store_h(cb);
     }
-    ok = cta_wait(&s.barB, it);
-    if (!ok) break;
+    // each thread waits for MMA-C itself (the barrier at the end of the step
+    // settles a failed wait)
+    const bool badB = !tc::mbar_wait(&s.barB, (uint32_t)(it & 1), kSpinScan);
+    tc::fence_after_sync();
     // this stage is consumed: the transaction count of its refill (chunk n + 2,
     // whose copies the next step issues after the barrier below)
     if (tid == 0 && n + 2 < n1) tc::mbar_arrive_expect_tx(&s.full[it & 1], fill_tx);
@@ -365,7 +370,7 @@ __global__ void __launch_bounds__(NTF, 1)
     if (n + 1 < n1) okF = tc::mbar_wait(&s.full[(it + 1) & 1], (uint32_t)(((it + 1) >> 1) & 1), kSpinScan);
     tc::fence_smem_to_async();
     tc::fence_before_sync();
-    ok = __syncthreads_or(okF ? 0 : 1) == 0;
+    ok = __syncthreads_or((okF && !badB) ? 0 : 1) == 0;
     tc::fence_after_sync();
   }
   if (ok) {
