@@ -118,13 +118,6 @@ __device__ __forceinline__ uint32_t lane_addr(uint32_t base, int warp, int col) 
   return base + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)col;
 }
 
-// Bounded wait on an mbarrier phase; the result is uniform over the CTA.
-__device__ __forceinline__ bool cta_wait(uint64_t* bar, int parity, bool local_bad = false) {
-  const bool ok = tc::mbar_wait(bar, (uint32_t)(parity & 1), kSpinScan);
-  const int bad = __syncthreads_or((ok && !local_bad) ? 0 : 1);
-  tc::fence_after_sync();
-  return bad == 0;
-}
 
 // PHASE: the SFDA rotation-decay gate.  The chunk decay then mixes the key
 // pair (2j, 2j + 1) of every state row as the complex product
@@ -590,8 +583,10 @@ __global__ void __launch_bounds__(NTF, 1)
         tc::mma(tbase + T_S, dQH + ks * kA128, dDO + ks * kB, id2, ks > 0 ? 1u : 0u);
     }
     if (outputs) store_dh(cb);
-    ok = cta_wait(&s.barA, it);
-    if (!ok) break;
+    // each thread waits for MMA-1 itself; the barrier after epilogue 1 settles a
+    // failed wait for the whole CTA
+    const bool badA = !tc::mbar_wait(&s.barA, (uint32_t)(it & 1), kSpinScan);
+    tc::fence_after_sync();
     // epilogue 1: dU rows ri, value columns ah*HB ..
     uint4 dusave[HB / 8];
     {
@@ -613,8 +608,9 @@ __global__ void __launch_bounds__(NTF, 1)
     }
     tc::fence_smem_to_async();
     tc::fence_before_sync();
-    __syncthreads();
+    ok = __syncthreads_or(badA ? 1 : 0) == 0;
     tc::fence_after_sync();
+    if (!ok) break;
     if (tid == 0) {
       const uint64_t dW = tc::sdesc_mnmaj(st.W, D, 0);
 #pragma unroll
