@@ -234,6 +234,14 @@ __device__ __forceinline__ bool hy_wait(uint64_t* bar, int phase, uint32_t limit
   return bad == 0;
 }
 
+// Bounded wait for the commit of level `phase` by this thread alone (no
+// barrier): a failure is carried to the next barrier the chunk needs anyway.
+__device__ __forceinline__ bool hy_wait_local(uint64_t* bar, int phase) {
+  const bool ok = tc::mbar_wait(bar, (uint32_t)(phase & 1), kSpinHy);
+  tc::fence_after_sync();
+  return ok;
+}
+
 // Descriptors: K-major [rows][K = 64] tiles (X tiles, row groups 1 KB apart),
 // MN-major [K][N = 128] tiles (the level-4 key and query tiles), MN-major
 // [K][M = 64] (an X tile read as its transpose).
@@ -362,6 +370,7 @@ __global__ void __launch_bounds__(NTB, 1)
     ok = hy_wait(&s.never, 0, kSpinInjected);
     if (!ok) break;
   }
+  bool bad = false;  // a level wait of this thread gave up (settled at the next barrier)
 
   // ---- level 1 (tensor memory): dQs = dO S, dW' = dU S, dKt = U dS', dM = dO U^T
   // (descriptors are built once; a k-step adds its byte offset / 16 to the start
@@ -720,8 +729,7 @@ __global__ void __launch_bounds__(NTB, 1)
       }
     }
   }
-  ok = hy_wait(&s.bar, 0);
-  if (!ok) break;
+  bad = !hy_wait_local(&s.bar, 0) || bad;
   // W and U' into the dS' tile (its level-1 reads are complete)
   cp_linear<NTB>(sW, Wg + cb * C * D, C * D, tid);
   cp_linear<NTB>(sUp, Upg + cb * C * D, C * D, tid);
@@ -761,8 +769,9 @@ __global__ void __launch_bounds__(NTB, 1)
   }
   tc::fence_smem_to_async();
   tc::fence_before_sync();
-  __syncthreads();
+  ok = __syncthreads_or(bad ? 1 : 0) == 0;
   tc::fence_after_sync();
+  if (!ok) break;
   // ---- level 2: Lambda = T^T [dU | dW]; dv = diag(beta) Lambda_U (runs under the dKt pass)
   if (tid == 0) {
     const uint32_t id = tc::idesc_bf16(64, 128, true, true);
@@ -853,8 +862,7 @@ __global__ void __launch_bounds__(NTB, 1)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh)
         vv[jt][hh] = *reinterpret_cast<const uint32_t*>(s.QC + vsw(i0 + 8 * hh, qt * 32 + jt * 8 + lc));
-    ok = hy_wait(&s.bar, 1);
-    if (!ok) break;
+    bad = !hy_wait_local(&s.bar, 1) || bad;
     float lu[4][4];
     frag_ld4(tb + T_LU + 32 * qt, warp, lu);
 #pragma unroll
@@ -886,13 +894,13 @@ __global__ void __launch_bounds__(NTB, 1)
       }
     }
   }
-  __syncthreads();
 
   frag::cp_wait<0>();  // W, U'
   tc::fence_smem_to_async();
   tc::fence_before_sync();
-  __syncthreads();
+  ok = __syncthreads_or(bad ? 1 : 0) == 0;
   tc::fence_after_sync();
+  if (!ok) break;
 
   // ---- level 3: dA = -strict_tril(Lambda_U U'^T + Lambda_W W^T): four partial sums
   if (tid == 0) {
@@ -924,8 +932,7 @@ __global__ void __launch_bounds__(NTB, 1)
   const uint64_t xmK = dk64(XM, 0), xaK = dk64(XA, 0), xmT = dmn64(XM, 0), xaT = dmn64(XA, 0);
   const uint64_t dKb0 = dmn128(Kb0, 0), dKb1 = dmn128(Kb1, 0), dQ0 = dmn128(Q0, 0);
   const uint64_t dQ1 = dmn128(Q1, 0), dB0 = dmn128(B0, 0), dB1 = dmn128(B1, 0);
-  ok = hy_wait(&s.bar, 2);
-  if (!ok) break;
+  bad = !hy_wait_local(&s.bar, 2) || bad;
   // level 4, dM part (thread 0, after the barrier above: the other warps go on
   // to the dA readout without waiting for the issue)
   if (tid == 0) {
@@ -967,8 +974,9 @@ __global__ void __launch_bounds__(NTB, 1)
     for (int idx = tid - 32; idx < C * (D / 8); idx += NTB - 32) build_row(idx, false);
   tc::fence_smem_to_async();
   tc::fence_before_sync();
-  __syncthreads();
+  ok = __syncthreads_or(bad ? 1 : 0) == 0;
   tc::fence_after_sync();
+  if (!ok) break;
   // ---- level 4, dA part: F2 = dA Kb; G += dA^T beta k (first half); G of the second half
   if (tid == 0) {
     mma_step(tb + T_F2, xaK, dKb0, idF, 0u);
@@ -988,8 +996,7 @@ __global__ void __launch_bounds__(NTB, 1)
     tc::commit(&s.bar);
     if (nb < p.B) tc::mbar_arrive_expect_tx(&s.full, kTileTx);
   }
-  ok = hy_wait(&s.bar, 3);
-  if (!ok) break;
+  bad = !hy_wait_local(&s.bar, 3) || bad;
   // the next chunk's level-1 tiles into the tiles level 4 has released
   if (nb < p.B) {
     issue_tiles(nn, nh, nb);
@@ -1119,7 +1126,8 @@ __global__ void __launch_bounds__(NTB, 1)
       if ((lane & 3) == 0) s.blk[(i0 + hh * 8) * 4 + qt] = xx;
     }
   }
-  __syncthreads();
+  ok = __syncthreads_or(bad ? 1 : 0) == 0;
+  if (!ok) break;
   float dbt = 0.f;
   if (tid < C) {
     dbt = s.dbp[tid * 4] + s.dbp[tid * 4 + 1] + s.dbp[tid * 4 + 2] + s.dbp[tid * 4 + 3];
