@@ -730,10 +730,6 @@ __global__ void __launch_bounds__(NTB, 1)
     }
   }
   bad = !hy_wait_local(&s.bar, 0) || bad;
-  // W and U' into the dS' tile (its level-1 reads are complete)
-  cp_linear<NTB>(sW, Wg + cb * C * D, C * D, tid);
-  cp_linear<NTB>(sUp, Upg + cb * C * D, C * D, tid);
-  frag::cp_commit();
   float zq[4][4], adw[4][4], akt[4][4], adm[2][4];
   {
     uint32_t rz[16], rw[16], rk[16], rm[8];
@@ -772,6 +768,12 @@ __global__ void __launch_bounds__(NTB, 1)
   ok = __syncthreads_or(bad ? 1 : 0) == 0;
   tc::fence_after_sync();
   if (!ok) break;
+  // W and U' into the dS' tile: level 1 and every thread's colsum have read it
+  // (the barrier above; a thread's own level-1 wait alone does not cover the
+  // other threads' colsum reads)
+  cp_linear<NTB>(sW, Wg + cb * C * D, C * D, tid);
+  cp_linear<NTB>(sUp, Upg + cb * C * D, C * D, tid);
+  frag::cp_commit();
   // ---- level 2: Lambda = T^T [dU | dW]; dv = diag(beta) Lambda_U (runs under the dKt pass)
   if (tid == 0) {
     const uint32_t id = tc::idesc_bf16(64, 128, true, true);
