@@ -79,6 +79,11 @@ constexpr uint32_t kSpinHy = 1u << 22;
 // drives the timeout path ends within milliseconds.
 constexpr uint32_t kSpinInjected = 256;
 constexpr int kRho0 = 15, kRho1 = 47;  // reference rows of the two halves
+// rows of HySmem::grow
+constexpr int kGR0 = 0, kGR1 = 1, kG31 = 2, kG32 = 3, kGC = 4;
+__device__ __forceinline__ int grow_slot(int i) {
+  return i == kRho0 ? kGR0 : i == kRho1 ? kGR1 : i == 31 ? kG31 : i == 32 ? kG32 : i == 63 ? kGC : -1;
+}
 
 // Gate tile element (i, c): 8-column groups XOR-swizzled by row.
 __device__ __forceinline__ int gsw(int i, int c) { return i * D + (c ^ ((i & 7) << 3)); }
@@ -130,6 +135,10 @@ struct HySmem {
   alignas(16) float xq[2 * D];
   float dmd[C];      // the diagonal of dM (fp32), added outside the level-4 products
   float blk[4 * D];  // dgamma totals of each 16-row block (scalar gate: row partial sums)
+  // the cumulative gate at rows 15, 47 (the references), 31, 32 and 63, kept apart
+  // from the gate tile (which the factor pass overwrites in place); a scalar gate
+  // uses column 0
+  alignas(16) float grow[5][D];
   uint64_t bar;
   uint64_t full;    // the chunk tiles' bulk copies
   uint64_t never;   // fault injection: a barrier that nothing ever arrives on
@@ -447,9 +456,12 @@ __global__ void __launch_bounds__(NTB, 1)
           off.x += t.x, off.y += t.y, off.z += t.z, off.w += t.w;
         }
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
-          *reinterpret_cast<float4*>(s.G + gsw(8 * sg + r, c4)) =
-              make_float4(x[r].x + off.x, x[r].y + off.y, x[r].z + off.z, x[r].w + off.w);
+        for (int r = 0; r < 8; ++r) {
+          const float4 y = make_float4(x[r].x + off.x, x[r].y + off.y, x[r].z + off.z, x[r].w + off.w);
+          *reinterpret_cast<float4*>(s.G + gsw(8 * sg + r, c4)) = y;
+          const int slot = grow_slot(8 * sg + r);
+          if (slot >= 0) *reinterpret_cast<float4*>(&s.grow[slot][c4]) = y;
+        }
       }
     } else if (warp == 1) {
       // rows 2 lane, 2 lane + 1: an inclusive scan across the warp
@@ -462,6 +474,9 @@ __global__ void __launch_bounds__(NTB, 1)
       }
       s.G[2 * lane + 1] = x;
       s.G[2 * lane] = x - a1v;
+      const int so = grow_slot(2 * lane + 1), se = grow_slot(2 * lane);
+      if (so >= 0) s.grow[so][0] = x;
+      if (se >= 0) s.grow[se][0] = x - a1v;
     }
   }
   __syncthreads();
@@ -472,11 +487,12 @@ __global__ void __launch_bounds__(NTB, 1)
   if (PHASE) {
     if (tid < D / 2) {
       const int c = 2 * tid;
-      const float gC = gat(C - 1, c), tC = gat(C - 1, c + 1);
+      const float gC = s.grow[kGC][c], tC = s.grow[kGC][c + 1];
       float gr[2], tr[2];
-      gr[0] = gat(kRho0, c), tr[0] = gat(kRho0, c + 1);
-      gr[1] = gat(kRho1, c), tr[1] = gat(kRho1, c + 1);
-      const float g31 = gat(31, c), t31 = gat(31, c + 1), g32 = gat(32, c), t32 = gat(32, c + 1);
+      gr[0] = s.grow[kGR0][c], tr[0] = s.grow[kGR0][c + 1];
+      gr[1] = s.grow[kGR1][c], tr[1] = s.grow[kGR1][c + 1];
+      const float g31 = s.grow[kG31][c], t31 = s.grow[kG31][c + 1];
+      const float g32 = s.grow[kG32][c], t32 = s.grow[kG32][c + 1];
       float sn, cs;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
@@ -506,8 +522,8 @@ __global__ void __launch_bounds__(NTB, 1)
     }
   } else if (tid < D) {
     const int cg = (gk == D) ? tid : 0;
-    const float g0 = gat(kRho0, cg), g1 = gat(kRho1, cg), gC = gat(C - 1, cg);
-    const float g31 = gat(31, cg), g32 = gat(32, cg);
+    const float g0 = s.grow[kGR0][cg], g1 = s.grow[kGR1][cg], gC = s.grow[kGC][cg];
+    const float g31 = s.grow[kG31][cg], g32 = s.grow[kG32][cg];
     s.er[tid] = __expf(g0);
     s.er[D + tid] = __expf(g1);
     s.erc[tid] = __expf(gC - g0);
@@ -518,38 +534,29 @@ __global__ void __launch_bounds__(NTB, 1)
     s.xq[D + tid] = __expf(g32 - g0);
   }
   // gate tile -> factor u_i = zeta_i / zeta_rho (real gates: e^{g_i - g_rho}), rho the
-  // reference row of row i's half (every thread reads the reference rows first)
+  // reference row of row i's half (the references from the snapshot: each thread
+  // rewrites only the elements it reads)
   if (PHASE) {
-    float tmp[C * D / NTB];
 #pragma unroll
     for (int u = 0; u < C * D / NTB / 2; ++u) {
       const int idx = tid + u * NTB;  // a key pair of one row
-      const int i = idx >> 6, c = 2 * (idx & 63), rho = i < 32 ? kRho0 : kRho1;
+      const int i = idx >> 6, c = 2 * (idx & 63), rs = i < 32 ? kGR0 : kGR1;
       float sn, cs;
-      sincosf(gat(i, c + 1) - gat(rho, c + 1), &sn, &cs);
-      const float m = __expf(gat(i, c) - gat(rho, c));
-      tmp[2 * u] = m * cs;
-      tmp[2 * u + 1] = -m * sn;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int u = 0; u < C * D / NTB / 2; ++u) {
-      const int idx = tid + u * NTB;
-      const int i = idx >> 6, c = 2 * (idx & 63);
-      gat(i, c) = tmp[2 * u];
-      gat(i, c + 1) = tmp[2 * u + 1];
+      sincosf(gat(i, c + 1) - s.grow[rs][c + 1], &sn, &cs);
+      const float m = __expf(gat(i, c) - s.grow[rs][c]);
+      gat(i, c) = m * cs;
+      gat(i, c + 1) = -m * sn;
     }
   } else if (gk == D) {
     // thread: channels c4 .. c4 + 3 of rows i4 + 16 u (16-byte accesses; the
     // swizzle keeps groups of 4 channels contiguous)
     const int c4 = 4 * (tid & 31), i4 = tid >> 5;
-    const float4 r0 = *reinterpret_cast<const float4*>(s.G + gsw(kRho0, c4));
-    const float4 r1 = *reinterpret_cast<const float4*>(s.G + gsw(kRho1, c4));
+    const float4 r0 = *reinterpret_cast<const float4*>(&s.grow[kGR0][c4]);
+    const float4 r1 = *reinterpret_cast<const float4*>(&s.grow[kGR1][c4]);
     float4 v[C * D / NTB / 4];
 #pragma unroll
     for (int u = 0; u < C * D / NTB / 4; ++u)
       v[u] = *reinterpret_cast<const float4*>(s.G + gsw(i4 + 16 * u, c4));
-    __syncthreads();
 #pragma unroll
     for (int u = 0; u < C * D / NTB / 4; ++u) {
       const int i = i4 + 16 * u;
@@ -560,11 +567,8 @@ __global__ void __launch_bounds__(NTB, 1)
                       frag::ex2_approx((v[u].z - r.z) * frag::kLog2e),
                       frag::ex2_approx((v[u].w - r.w) * frag::kLog2e));
     }
-  } else {
-    float t = 0.f;
-    if (tid < C) t = __expf(s.G[tid] - s.G[tid < 32 ? kRho0 : kRho1]);
-    __syncthreads();
-    if (tid < C) s.G[tid] = t;
+  } else if (tid < C) {
+    s.G[tid] = __expf(s.G[tid] - s.grow[tid < 32 ? kGR0 : kGR1][0]);
   }
   // factor u at (i, c), (i, c + 1), c even (phase gate: the pair's complex u)
   auto ep2 = [&](int i, int c) -> float2 {
