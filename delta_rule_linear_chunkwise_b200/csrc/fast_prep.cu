@@ -156,13 +156,6 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
                     frag::pack(f[6], f[7]));
 }
 
-// Bounded wait on an mbarrier phase; CTA-uniform result.
-__device__ __forceinline__ bool prep_wait(uint64_t* bar, int parity) {
-  const bool ok = tc::mbar_wait(bar, (uint32_t)(parity & 1), kSpinPrep);
-  const int bad = __syncthreads_or(ok ? 0 : 1);
-  tc::fence_after_sync();
-  return bad == 0;
-}
 
 template <bool PHASE>
 __global__ void __launch_bounds__(NTP, 2)
@@ -223,15 +216,21 @@ __global__ void __launch_bounds__(NTP, 2)
   if (!chan && tid < C)
     s.gs[tid] = (tid < nvalid && p.gate != kGateNone) ? g_scalar[row_id(p, b, t0 + tid, h)] : 0.f;
   const float eta = (tid < C && tid < nvalid) ? beta_in[row_id(p, b, t0 + tid, h)] : 0.f;
-  bool ok = prep_wait(&s.bar_tma, 0);
+  // each thread waits for the TMA tiles itself; a failed wait is settled at the
+  // barrier after the gate scan (and the MMA waits below at the next barrier)
+  bool bad = !tc::mbar_wait(&s.bar_tma, 0u, kSpinPrep);
+  tc::fence_after_sync();
+  bool ok = true;
   const uint32_t tb = s.tmem;
   do {  // leaves early (break) only when a bounded wait gives up
-  if (!ok) break;
   // ---- cumulative gate down the rows (padded rows carry a zero gate)
   // per-channel element (r, c) of the gate tile: box c / 32, chunk (c % 32) / 4
   auto gp = [&](int r, int c) -> float* {
     return reinterpret_cast<float*>(s.G + (c >> 5) * kBox + swz(r, (c & 31) >> 2) + (c & 3) * 4);
   };
+  // a scalar gate arrives by plain loads of threads 0..63: visible to warp 0's scan
+  // only after a barrier (the per-channel gate came by TMA, which each thread waited for)
+  if (!chan) __syncthreads();
   if (chan) {
     // thread: channels 4 qd .. 4 qd + 3 (one 16-byte chunk of a swizzled box), rows
     // 8 sg .. 8 sg + 7, scanned in registers; then the totals of the earlier row
@@ -270,7 +269,8 @@ __global__ void __launch_bounds__(NTP, 2)
     s.gs[2 * lane + 1] = x;
     s.gs[2 * lane] = x - a1;
   }
-  __syncthreads();
+  ok = __syncthreads_or(bad ? 1 : 0) == 0;
+  if (!ok) break;
   auto gam = [&](int r, int c) -> float { return chan ? *gp(r, c) : s.gs[r]; };
   // per-channel reference factors and the chunk decay
   if (PHASE) {
@@ -459,8 +459,8 @@ __global__ void __launch_bounds__(NTP, 2)
     for (int ks = 0; ks < D / 16; ++ks) tc::mma(tb, a + 16u * ks, bb + 16u * ks, id, ks > 0 ? 1u : 0u);
     tc::commit(&s.bar_mma);
   }
-  ok = prep_wait(&s.bar_mma, 0);
-  if (!ok) break;
+  bad = !tc::mbar_wait(&s.bar_mma, 0u, kSpinPrep);
+  tc::fence_after_sync();
   // ---- A^T (fp32, [j][i]) into the gate tile's first half; M (bf16) to global.
   // Accumulator row = lane: quadrant 0 A rows of the first half, 1 its M rows,
   // 2 and 3 those of the second half; warps w and w + 4 split the columns.
@@ -515,7 +515,8 @@ __global__ void __launch_bounds__(NTP, 2)
       *reinterpret_cast<uint4*>(s.KB + ct16(r, jq + 4 * it)) = bkr[it];
   }
   tc::fence_before_sync();
-  __syncthreads();
+  ok = __syncthreads_or(bad ? 1 : 0) == 0;
+  if (!ok) break;
   // ---- T = (I + A)^{-1} in fp32, by blocks of 32:
   //   T11 = (I + A11)^{-1}, T22 = (I + A22)^{-1} (thread j < 64 forward-substitutes
   //   one column of one of them, all its rows in registers), then
@@ -623,8 +624,13 @@ __global__ void __launch_bounds__(NTP, 2)
     }
     tc::commit(&s.bar_mma);
   }
-  ok = prep_wait(&s.bar_mma, 1);
-  if (!ok) break;
+  // each warp waits for W, U' itself (the TMEM reads below are warp-wide); a
+  // warp whose wait gives up records it and skips its stores
+  if (!__all_sync(0xffffffffu, tc::mbar_wait(&s.bar_mma, 1u, kSpinPrep))) {
+    if (lane == 0 && err) atomicExch(err, 1);
+    break;
+  }
+  tc::fence_after_sync();
   // ---- W (warps 0-3) and U' (warps 4-7), rows 16 (warp % 4) + lane, lanes 0..15
   {
     const int qd = warp & 3, row = 16 * qd + (lane & 15);
