@@ -47,7 +47,8 @@
 // 120 KB) are loaded while the epilogue of this one runs, into the tiles that
 // level 4 has released, so a chunk starts with its first products; q, k, v and
 // the gate (which the epilogue still reads) load, and the gate's cumulative sum
-// runs, on warps 1..15 while warp 0 issues level 1.  Likewise the tile builds
+// runs, on warps 1..15 while warp 0 issues level 1; warps 1..4 form the state
+// tiles' column sums while those copies land.  Likewise the tile builds
 // under levels 3 and 4 leave warp 0 to its MMA issue.
 //
 // Each level is a set of tcgen05.mma (M = 64, operands in shared memory in the
@@ -119,10 +120,10 @@ struct HySmem {
   bf16 k[C * LDD];  // raw k, row-major padded
   bf16 TT[C * C];   // T [i][j], core-tiled (MN-major A of T^T);  then beta k^{rho1} rows 32..63
   float G[C * D];   // cumulative gate (gsw), then the factor u_i of each element
-  float beta[C];
-  float knorm[C];
+  alignas(16) float beta[C];
+  alignas(16) float knorm[C];
   float dbp[C * 4];
-  alignas(16) float dgc[4 * D];
+  alignas(16) float dgc[4 * D];  // colsum(conj(dS') S) (first D; the gate scan's scratch)
   float ktk[4 * D];
   float er[2 * D];   // per half: conj(zeta_rho)                (real gates: e^{g_rho})
   float erc[2 * D];  // per half: zeta_C / zeta_rho             (real gates: e^{g_C - g_rho})
@@ -404,6 +405,7 @@ __global__ void __launch_bounds__(NTB, 1)
   // q, k, v, the gate, beta and ||k||^2 of this chunk by warps 1..15, then the
   // gate's cumulative sum by warps 8..15, while warp 0 issues level 1 (named
   // barriers 1 and 2 hold only the warps that take part)
+  float dsc[4][2];  // warps 1..4: colsum(conj(dS') S) of this lane's keys (lanes 0..7)
   if (warp > 0) {
     const int lt = tid - 32;
     constexpr int NL = NTB - 32;
@@ -424,11 +426,55 @@ __global__ void __launch_bounds__(NTB, 1)
     } else if (lt < C) {
       s.G[lt] = (lt < nvalid && p.gate != kGateNone) ? g[row_id(p, b, t0 + lt, h)] : 0.f;
     }
-    if (lt >= C && lt < 2 * C) {
-      s.beta[lt - C] = beta[cb * C + lt - C];
-      s.knorm[lt - C] = knorm_g[cb * C + lt - C];
-    }
+    if (lt >= C && lt < C + C / 4)
+      frag::cp16(s.beta + 4 * (lt - C), beta + cb * C + 4 * (lt - C), true);
+    else if (lt >= C + C / 4 && lt < C + C / 2)
+      frag::cp16(s.knorm + 4 * (lt - C - C / 4), knorm_g + cb * C + 4 * (lt - C - C / 4), true);
     frag::cp_commit();
+    // colsum(conj(dS') S) on warps 1..4 while the copies land (real gates: per key
+    // channel c the sum over a of dS'[c][a] S[c][a]; the state tiles are stored
+    // [c][a]).  Lane: row r of the core matrices (key c = 8 kb + r) and 16-byte
+    // chunk j = 4 jh + (lane / 8) of 8 values a; a warp takes key blocks
+    // kb = warp - 1 + 4 m, sums its four chunks per lane, then over the lanes.
+    if (warp <= 4) {
+      const int r = lane & 7, jl = lane >> 3;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int c = (warp - 1 + 4 * m) * 8 + r;
+        float pr = 0.f, cross = 0.f;
+#pragma unroll
+        for (int jh = 0; jh < 4; ++jh) {
+          const int o = ct_off(c, 8 * (4 * jh + jl), D);
+          const uint4 x = *reinterpret_cast<const uint4*>(s.SS + o);
+          const uint4 y = *reinterpret_cast<const uint4*>(s.SD + o);
+          const uint32_t* wx = reinterpret_cast<const uint32_t*>(&x);
+          const uint32_t* wy = reinterpret_cast<const uint32_t*>(&y);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 fx = frag::unpack(wx[e]), fy = frag::unpack(wy[e]);
+            pr += fx.x * fy.x + fx.y * fy.y;
+            if (PHASE) {
+              // the pair's odd key (lane ^ 1) for the cross term of conj(dS') S:
+              // Im = sum_a (dx sy - dy sx), x the even key, y the odd one
+              const float2 gx = frag::unpack(__shfl_xor_sync(0xffffffffu, wx[e], 1));
+              const float2 gy = frag::unpack(__shfl_xor_sync(0xffffffffu, wy[e], 1));
+              cross += fy.x * gx.x + fy.y * gx.y - gy.x * fx.x - gy.y * fx.y;
+            }
+          }
+        }
+        pr += __shfl_xor_sync(0xffffffffu, pr, 8);
+        pr += __shfl_xor_sync(0xffffffffu, pr, 16);
+        if (PHASE) {
+          cross += __shfl_xor_sync(0xffffffffu, cross, 8);
+          cross += __shfl_xor_sync(0xffffffffu, cross, 16);
+          const float po = __shfl_xor_sync(0xffffffffu, pr, 1);
+          dsc[m][0] = pr + po;  // Re: dx sx + dy sy (even keys)
+          dsc[m][1] = cross;    // Im
+        } else {
+          dsc[m][0] = pr;
+        }
+      }
+    }
     frag::cp_wait<0>();
     named_sync(1, NTB - 32);  // warps 1..15: their copies have landed
     if (gk == D) {
@@ -480,6 +526,21 @@ __global__ void __launch_bounds__(NTB, 1)
     }
   }
   __syncthreads();
+  // the colsum into dgc (after the barrier: the gate scan used it as scratch)
+  if (warp >= 1 && warp <= 4 && lane < 8) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int c = (warp - 1 + 4 * m) * 8 + lane;
+      if (PHASE) {
+        if ((lane & 1) == 0) {
+          s.dgc[c] = dsc[m][0];
+          s.dgc[c + 1] = dsc[m][1];
+        }
+      } else {
+        s.dgc[c] = dsc[m][0];
+      }
+    }
+  }
   // element (i, c) of the gate tile
   auto gat = [&](int i, int c) -> float& { return gk == D ? s.G[gsw(i, c)] : s.G[i]; };
 
@@ -689,50 +750,6 @@ __global__ void __launch_bounds__(NTB, 1)
     }
   };
 
-  // colsum(conj(dS') S) while level 1 runs (real gates: per key channel c the sum
-  // over a of dS'[c][a] S[c][a]; the state tiles are stored [c][a]).  Thread:
-  // row r of the core matrices of row blocks 4 q .. 4 q + 3 (keys c), 16-byte
-  // chunk j (8 values a); eight lanes read one whole core matrix.  Partial sums
-  // reduce over the warp's four chunks, then land in one of four slots per key
-  // (warp % 4), summed by the reader.
-  {
-    const int r = tid & 7, j = (tid >> 3) & 15, q = tid >> 7;
-#pragma unroll
-    for (int rr = 0; rr < 4; ++rr) {
-      const int c = (4 * q + rr) * 8 + r;
-      const int o = ct_off(c, 8 * j, D);
-      const uint4 x = *reinterpret_cast<const uint4*>(s.SS + o);
-      const uint4 y = *reinterpret_cast<const uint4*>(s.SD + o);
-      const uint32_t* wx = reinterpret_cast<const uint32_t*>(&x);
-      const uint32_t* wy = reinterpret_cast<const uint32_t*>(&y);
-      float pr = 0.f, cross = 0.f;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 fx = frag::unpack(wx[e]), fy = frag::unpack(wy[e]);
-        pr += fx.x * fy.x + fx.y * fy.y;
-        if (PHASE) {
-          // the pair's odd key (lane ^ 1) for the cross term of conj(dS') S:
-          // Im = sum_a (dx sy - dy sx), x the even key, y the odd one
-          const float2 gx = frag::unpack(__shfl_xor_sync(0xffffffffu, wx[e], 1));
-          const float2 gy = frag::unpack(__shfl_xor_sync(0xffffffffu, wy[e], 1));
-          cross += fy.x * gx.x + fy.y * gx.y - gy.x * fx.x - gy.y * fx.y;
-        }
-      }
-      pr += __shfl_xor_sync(0xffffffffu, pr, 8);
-      pr += __shfl_xor_sync(0xffffffffu, pr, 16);
-      if (PHASE) {
-        cross += __shfl_xor_sync(0xffffffffu, cross, 8);
-        cross += __shfl_xor_sync(0xffffffffu, cross, 16);
-        const float po = __shfl_xor_sync(0xffffffffu, pr, 1);
-        if ((lane >> 3) == 0 && (r & 1) == 0) {
-          s.dgc[(warp & 3) * D + c] = pr + po;     // Re: dx sx + dy sy
-          s.dgc[(warp & 3) * D + c + 1] = cross;  // Im
-        }
-      } else if ((lane >> 3) == 0) {
-        s.dgc[(warp & 3) * D + c] = pr;
-      }
-    }
-  }
   bad = !hy_wait_local(&s.bar, 0) || bad;
   float zq[4][4], adw[4][4], akt[4][4], adm[2][4];
   {
@@ -1068,7 +1085,7 @@ __global__ void __launch_bounds__(NTB, 1)
         for (int u = 0; u < 2; ++u) {
           const int cc = c + u;
           kt[u] = s.ktk[cc] + s.ktk[D + cc] + s.ktk[2 * D + cc] + s.ktk[3 * D + cc];
-          gs[u] = s.dgc[cc] + s.dgc[D + cc] + s.dgc[2 * D + cc] + s.dgc[3 * D + cc];
+          gs[u] = s.dgc[cc];
         }
         const float2 fr = *reinterpret_cast<const float2*>(s.er + D + c);
         const float2 frc = *reinterpret_cast<const float2*>(s.erc + D + c);
