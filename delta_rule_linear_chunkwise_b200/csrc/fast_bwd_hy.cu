@@ -441,18 +441,23 @@ __global__ void __launch_bounds__(NTB, 1)
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const int c = (warp - 1 + 4 * m) * 8 + r;
-        float pr = 0.f, cross = 0.f;
+        float pr = 0.f, pr2 = 0.f, cross = 0.f;  // two sums: shorter dependency chains
+        uint4 xs[4], ys[4];
 #pragma unroll
         for (int jh = 0; jh < 4; ++jh) {
           const int o = ct_off(c, 8 * (4 * jh + jl), D);
-          const uint4 x = *reinterpret_cast<const uint4*>(s.SS + o);
-          const uint4 y = *reinterpret_cast<const uint4*>(s.SD + o);
-          const uint32_t* wx = reinterpret_cast<const uint32_t*>(&x);
-          const uint32_t* wy = reinterpret_cast<const uint32_t*>(&y);
+          xs[jh] = *reinterpret_cast<const uint4*>(s.SS + o);
+          ys[jh] = *reinterpret_cast<const uint4*>(s.SD + o);
+        }
+#pragma unroll
+        for (int jh = 0; jh < 4; ++jh) {
+          const uint32_t* wx = reinterpret_cast<const uint32_t*>(&xs[jh]);
+          const uint32_t* wy = reinterpret_cast<const uint32_t*>(&ys[jh]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 fx = frag::unpack(wx[e]), fy = frag::unpack(wy[e]);
-            pr += fx.x * fy.x + fx.y * fy.y;
+            pr += fx.x * fy.x;
+            pr2 += fx.y * fy.y;
             if (PHASE) {
               // the pair's odd key (lane ^ 1) for the cross term of conj(dS') S:
               // Im = sum_a (dx sy - dy sx), x the even key, y the odd one
@@ -462,6 +467,7 @@ __global__ void __launch_bounds__(NTB, 1)
             }
           }
         }
+        pr += pr2;
         pr += __shfl_xor_sync(0xffffffffu, pr, 8);
         pr += __shfl_xor_sync(0xffffffffu, pr, 16);
         if (PHASE) {
