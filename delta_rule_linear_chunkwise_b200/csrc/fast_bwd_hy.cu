@@ -47,8 +47,8 @@
 // 120 KB) are loaded while the epilogue of this one runs, into the tiles that
 // level 4 has released, so a chunk starts with its first products; q, k, v and
 // the gate (which the epilogue still reads) load, and the gate's cumulative sum
-// runs, on warps 1..15 while warp 0 issues level 1; warps 1..4 form the state
-// tiles' column sums while those copies land.  Likewise the tile builds
+// runs, on warps 1..15 while warp 0 issues level 1; for real gates warps 1..4
+// form the state tiles' column sums while those copies land.  Likewise the tile builds
 // under levels 3 and 4 leave warp 0 to its MMA issue.
 //
 // Each level is a set of tcgen05.mma (M = 64, operands in shared memory in the
@@ -123,7 +123,8 @@ struct HySmem {
   alignas(16) float beta[C];
   alignas(16) float knorm[C];
   float dbp[C * 4];
-  alignas(16) float dgc[4 * D];  // colsum(conj(dS') S) (first D; the gate scan's scratch)
+  alignas(16) float dgc[4 * D];  // colsum(conj(dS') S) (real gates: the first D; phase gate:
+                                 // four slots per key) and the gate scan's scratch
   float ktk[4 * D];
   float er[2 * D];   // per half: conj(zeta_rho)                (real gates: e^{g_rho})
   float erc[2 * D];  // per half: zeta_C / zeta_rho             (real gates: e^{g_C - g_rho})
@@ -252,6 +253,15 @@ __device__ __forceinline__ bool hy_wait_local(uint64_t* bar, int phase) {
   return ok;
 }
 
+// The wait for a level's MMAs.  Real gates: each thread alone (hy_wait_local),
+// a failure settled at the next barrier the chunk needs.  The phase gate, whose
+// per-element work is heavier, runs faster with the CTA held at a barrier after
+// each level (hy_wait; measured on the SFDA workload: 1195 against 1090 us).
+template <bool PHASE>
+__device__ __forceinline__ bool level_wait_t(uint64_t* bar, int phase) {
+  return PHASE ? hy_wait(bar, phase) : hy_wait_local(bar, phase);
+}
+
 // Descriptors: K-major [rows][K = 64] tiles (X tiles, row groups 1 KB apart),
 // MN-major [K][N = 128] tiles (the level-4 key and query tiles), MN-major
 // [K][M = 64] (an X tile read as its transpose).
@@ -285,6 +295,7 @@ __global__ void __launch_bounds__(NTB, 1)
   HySmem& s = *reinterpret_cast<HySmem*>(smraw);
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, gk = p.gk;
+  auto level_wait = [](uint64_t* bar, int phase) { return level_wait_t<PHASE>(bar, phase); };
   const int rb = warp & 3, qt = warp >> 2;
   const int hf = rb >> 1;  // the half of this warp's fragment rows
   const int lr = lane >> 2, lc = 2 * (lane & 3);
@@ -405,7 +416,7 @@ __global__ void __launch_bounds__(NTB, 1)
   // q, k, v, the gate, beta and ||k||^2 of this chunk by warps 1..15, then the
   // gate's cumulative sum by warps 8..15, while warp 0 issues level 1 (named
   // barriers 1 and 2 hold only the warps that take part)
-  float dsc[4][2];  // warps 1..4: colsum(conj(dS') S) of this lane's keys (lanes 0..7)
+  float dsc[4];  // real gates, warps 1..4: colsum(dS' S) of this lane's keys (lanes 0..7)
   if (warp > 0) {
     const int lt = tid - 32;
     constexpr int NL = NTB - 32;
@@ -431,17 +442,19 @@ __global__ void __launch_bounds__(NTB, 1)
     else if (lt >= C + C / 4 && lt < C + C / 2)
       frag::cp16(s.knorm + 4 * (lt - C - C / 4), knorm_g + cb * C + 4 * (lt - C - C / 4), true);
     frag::cp_commit();
-    // colsum(conj(dS') S) on warps 1..4 while the copies land (real gates: per key
+    // real gates: colsum(dS' S) on warps 1..4 while the copies land (per key
     // channel c the sum over a of dS'[c][a] S[c][a]; the state tiles are stored
     // [c][a]).  Lane: row r of the core matrices (key c = 8 kb + r) and 16-byte
     // chunk j = 4 jh + (lane / 8) of 8 values a; a warp takes key blocks
     // kb = warp - 1 + 4 m, sums its four chunks per lane, then over the lanes.
-    if (warp <= 4) {
+    // (The phase gate's cross term needs a shuffle per element pair: its sums run
+    // on all 16 warps after the gate scan.)
+    if (!PHASE && warp <= 4) {
       const int r = lane & 7, jl = lane >> 3;
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const int c = (warp - 1 + 4 * m) * 8 + r;
-        float pr = 0.f, pr2 = 0.f, cross = 0.f;  // two sums: shorter dependency chains
+        float pr = 0.f, pr2 = 0.f;  // two sums: shorter dependency chains
         uint4 xs[4], ys[4];
 #pragma unroll
         for (int jh = 0; jh < 4; ++jh) {
@@ -458,27 +471,12 @@ __global__ void __launch_bounds__(NTB, 1)
             const float2 fx = frag::unpack(wx[e]), fy = frag::unpack(wy[e]);
             pr += fx.x * fy.x;
             pr2 += fx.y * fy.y;
-            if (PHASE) {
-              // the pair's odd key (lane ^ 1) for the cross term of conj(dS') S:
-              // Im = sum_a (dx sy - dy sx), x the even key, y the odd one
-              const float2 gx = frag::unpack(__shfl_xor_sync(0xffffffffu, wx[e], 1));
-              const float2 gy = frag::unpack(__shfl_xor_sync(0xffffffffu, wy[e], 1));
-              cross += fy.x * gx.x + fy.y * gx.y - gy.x * fx.x - gy.y * fx.y;
-            }
           }
         }
         pr += pr2;
         pr += __shfl_xor_sync(0xffffffffu, pr, 8);
         pr += __shfl_xor_sync(0xffffffffu, pr, 16);
-        if (PHASE) {
-          cross += __shfl_xor_sync(0xffffffffu, cross, 8);
-          cross += __shfl_xor_sync(0xffffffffu, cross, 16);
-          const float po = __shfl_xor_sync(0xffffffffu, pr, 1);
-          dsc[m][0] = pr + po;  // Re: dx sx + dy sy (even keys)
-          dsc[m][1] = cross;    // Im
-        } else {
-          dsc[m][0] = pr;
-        }
+        dsc[m] = pr;
       }
     }
     frag::cp_wait<0>();
@@ -532,20 +530,10 @@ __global__ void __launch_bounds__(NTB, 1)
     }
   }
   __syncthreads();
-  // the colsum into dgc (after the barrier: the gate scan used it as scratch)
-  if (warp >= 1 && warp <= 4 && lane < 8) {
+  // real gates: the colsum into dgc (after the barrier: the gate scan used it as scratch)
+  if (!PHASE && warp >= 1 && warp <= 4 && lane < 8) {
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int c = (warp - 1 + 4 * m) * 8 + lane;
-      if (PHASE) {
-        if ((lane & 1) == 0) {
-          s.dgc[c] = dsc[m][0];
-          s.dgc[c + 1] = dsc[m][1];
-        }
-      } else {
-        s.dgc[c] = dsc[m][0];
-      }
-    }
+    for (int m = 0; m < 4; ++m) s.dgc[(warp - 1 + 4 * m) * 8 + lane] = dsc[m];
   }
   // element (i, c) of the gate tile
   auto gat = [&](int i, int c) -> float& { return gk == D ? s.G[gsw(i, c)] : s.G[i]; };
@@ -756,7 +744,44 @@ __global__ void __launch_bounds__(NTB, 1)
     }
   };
 
-  bad = !hy_wait_local(&s.bar, 0) || bad;
+  // phase gate: colsum(conj(dS') S) while level 1 runs.  Thread: row r of the
+  // core matrices of row blocks 4 q .. 4 q + 3 (keys c), 16-byte chunk j (8
+  // values a); eight lanes read one whole core matrix.  Partial sums reduce over
+  // the warp's four chunks, then land in one of four slots per key (warp % 4),
+  // summed by the reader.
+  if (PHASE) {
+    const int r = tid & 7, j = (tid >> 3) & 15, q = tid >> 7;
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+      const int c = (4 * q + rr) * 8 + r;
+      const int o = ct_off(c, 8 * j, D);
+      const uint4 x = *reinterpret_cast<const uint4*>(s.SS + o);
+      const uint4 y = *reinterpret_cast<const uint4*>(s.SD + o);
+      const uint32_t* wx = reinterpret_cast<const uint32_t*>(&x);
+      const uint32_t* wy = reinterpret_cast<const uint32_t*>(&y);
+      float pr = 0.f, cross = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fx = frag::unpack(wx[e]), fy = frag::unpack(wy[e]);
+        pr += fx.x * fy.x + fx.y * fy.y;
+        // the pair's odd key (lane ^ 1) for the cross term of conj(dS') S:
+        // Im = sum_a (dx sy - dy sx), x the even key, y the odd one
+        const float2 gx = frag::unpack(__shfl_xor_sync(0xffffffffu, wx[e], 1));
+        const float2 gy = frag::unpack(__shfl_xor_sync(0xffffffffu, wy[e], 1));
+        cross += fy.x * gx.x + fy.y * gx.y - gy.x * fx.x - gy.y * fx.y;
+      }
+      pr += __shfl_xor_sync(0xffffffffu, pr, 8);
+      pr += __shfl_xor_sync(0xffffffffu, pr, 16);
+      cross += __shfl_xor_sync(0xffffffffu, cross, 8);
+      cross += __shfl_xor_sync(0xffffffffu, cross, 16);
+      const float po = __shfl_xor_sync(0xffffffffu, pr, 1);
+      if ((lane >> 3) == 0 && (r & 1) == 0) {
+        s.dgc[(warp & 3) * D + c] = pr + po;     // Re: dx sx + dy sy
+        s.dgc[(warp & 3) * D + c + 1] = cross;  // Im
+      }
+    }
+  }
+  bad = !level_wait(&s.bar, 0) || bad;
   float zq[4][4], adw[4][4], akt[4][4], adm[2][4];
   {
     uint32_t rz[16], rw[16], rk[16], rm[8];
@@ -891,7 +916,7 @@ __global__ void __launch_bounds__(NTB, 1)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh)
         vv[jt][hh] = *reinterpret_cast<const uint32_t*>(s.QC + vsw(i0 + 8 * hh, qt * 32 + jt * 8 + lc));
-    bad = !hy_wait_local(&s.bar, 1) || bad;
+    bad = !level_wait(&s.bar, 1) || bad;
     float lu[4][4];
     frag_ld4(tb + T_LU + 32 * qt, warp, lu);
 #pragma unroll
@@ -961,7 +986,7 @@ __global__ void __launch_bounds__(NTB, 1)
   const uint64_t xmK = dk64(XM, 0), xaK = dk64(XA, 0), xmT = dmn64(XM, 0), xaT = dmn64(XA, 0);
   const uint64_t dKb0 = dmn128(Kb0, 0), dKb1 = dmn128(Kb1, 0), dQ0 = dmn128(Q0, 0);
   const uint64_t dQ1 = dmn128(Q1, 0), dB0 = dmn128(B0, 0), dB1 = dmn128(B1, 0);
-  bad = !hy_wait_local(&s.bar, 2) || bad;
+  bad = !level_wait(&s.bar, 2) || bad;
   // level 4, dM part (thread 0, after the barrier above: the other warps go on
   // to the dA readout without waiting for the issue)
   if (tid == 0) {
@@ -1025,7 +1050,7 @@ __global__ void __launch_bounds__(NTB, 1)
     tc::commit(&s.bar);
     if (nb < p.B) tc::mbar_arrive_expect_tx(&s.full, kTileTx);
   }
-  bad = !hy_wait_local(&s.bar, 3) || bad;
+  bad = !level_wait(&s.bar, 3) || bad;
   // the next chunk's level-1 tiles into the tiles level 4 has released
   if (nb < p.B) {
     issue_tiles(nn, nh, nb);
@@ -1091,7 +1116,8 @@ __global__ void __launch_bounds__(NTB, 1)
         for (int u = 0; u < 2; ++u) {
           const int cc = c + u;
           kt[u] = s.ktk[cc] + s.ktk[D + cc] + s.ktk[2 * D + cc] + s.ktk[3 * D + cc];
-          gs[u] = s.dgc[cc];
+          gs[u] = PHASE ? s.dgc[cc] + s.dgc[D + cc] + s.dgc[2 * D + cc] + s.dgc[3 * D + cc]
+                        : s.dgc[cc];
         }
         const float2 fr = *reinterpret_cast<const float2*>(s.er + D + c);
         const float2 frc = *reinterpret_cast<const float2*>(s.erc + D + c);
