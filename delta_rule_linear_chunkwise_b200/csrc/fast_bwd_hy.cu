@@ -173,6 +173,24 @@ __device__ __forceinline__ void named_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// 4 x 4 transpose of 32-bit words across the four lanes of a quad (lq = lane % 4):
+// on entry lane lq holds a[j] = element (lq, j), on exit a[j] = element (j, lq).
+// Two exchange rounds (lane masks 1 and 2), two shuffles each.
+__device__ __forceinline__ void quad_transpose(uint32_t (&a)[4], int lq) {
+#pragma unroll
+  for (int m = 1; m <= 2; m <<= 1)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (j & m) continue;
+      const uint32_t send = (lq & m) ? a[j] : a[j | m];
+      const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, m);
+      if (lq & m)
+        a[j] = recv;
+      else
+        a[j | m] = recv;
+    }
+}
+
 __device__ __forceinline__ void mma_step(uint32_t tm, uint64_t a, uint64_t b, uint32_t id,
                                          uint32_t acc) {
   tc::mma(tm, a, b, id, acc);
@@ -1074,9 +1092,10 @@ __global__ void __launch_bounds__(NTB, 1)
 
   // ---- per-element epilogue: dq out; P <- dk (before the Kaczmarz term), Q <- dgamma
 #pragma unroll
-  for (int jt = 0; jt < 4; ++jt)
+  for (int hh = 0; hh < 2; ++hh) {
+    uint32_t dqp[4];  // dq pairs of this row (column group jt), stored after a quad transpose
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
+    for (int jt = 0; jt < 4; ++jt) {
       const int i = i0 + hh * 8, c = qt * 32 + jt * 8 + lc;
       const float bi = s.beta[i];
       const float2 kk = k2(i, c), qq = q2(i, c), f = ep2(i, c);
@@ -1131,11 +1150,17 @@ __global__ void __launch_bounds__(NTB, 1)
           dgo[1] += kt[1] + fr.y * frc.y * gs[1];
         }
       }
-      if (i < nvalid)
-        *reinterpret_cast<uint32_t*>(dq + rowg[hh] + c) = frag::pack(dqo[0], dqo[1]);
+      dqp[jt] = frag::pack(dqo[0], dqo[1]);
       P[jt][e0] = dko[0], P[jt][e1] = dko[1];
       Q[jt][e0] = dgo[0], Q[jt][e1] = dgo[1];
     }
+    // after the quad transpose lane lq holds channels qt * 32 + 8 lq .. + 7 of
+    // the row (one 16-byte store instead of four 4-byte ones)
+    quad_transpose(dqp, lane & 3);
+    if (i0 + 8 * hh < nvalid)
+      *reinterpret_cast<uint4*>(dq + rowg[hh] + qt * 32 + 8 * (lane & 3)) =
+          make_uint4(dqp[0], dqp[1], dqp[2], dqp[3]);
+  }
   // d(beta_eff) partials: reduce the 4 lanes that share a row, one slot per column quarter
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
@@ -1220,11 +1245,12 @@ __global__ void __launch_bounds__(NTB, 1)
     if (ib < nvalid) dg[row_id(p, b, t0 + ib, h)] = x - a0;
   }
   __syncthreads();
-  // dk (with the Kaczmarz chain rule) and dbeta
+  // dk (with the Kaczmarz chain rule; quad-transposed into 16-byte stores) and dbeta
 #pragma unroll
-  for (int jt = 0; jt < 4; ++jt)
+  for (int hh = 0; hh < 2; ++hh) {
+    uint32_t dkp[4];
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
+    for (int jt = 0; jt < 4; ++jt) {
       const int i = i0 + hh * 8, c = qt * 32 + jt * 8 + lc;
       float o0 = P[jt][2 * hh], o1 = P[jt][2 * hh + 1];
       if (p.beta_mode == kBetaKaczmarz) {
@@ -1233,8 +1259,13 @@ __global__ void __launch_bounds__(NTB, 1)
         o0 += f * kk.x;
         o1 += f * kk.y;
       }
-      if (i < nvalid) *reinterpret_cast<uint32_t*>(dk + rowg[hh] + c) = frag::pack(o0, o1);
+      dkp[jt] = frag::pack(o0, o1);
     }
+    quad_transpose(dkp, lane & 3);
+    if (i0 + 8 * hh < nvalid)
+      *reinterpret_cast<uint4*>(dk + rowg[hh] + qt * 32 + 8 * (lane & 3)) =
+          make_uint4(dkp[0], dkp[1], dkp[2], dkp[3]);
+  }
   if (tid < nvalid) {
     if (p.beta_mode == kBetaKaczmarz) dbt /= (s.knorm[tid] + p.eps);
     dbeta[row_id(p, b, t0 + tid, h)] = dbt;
