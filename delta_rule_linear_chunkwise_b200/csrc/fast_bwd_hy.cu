@@ -941,14 +941,30 @@ __global__ void __launch_bounds__(NTB, 1)
     for (int jt = 0; jt < 4; ++jt)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
-        const int i = i0 + hh * 8, a = qt * 32 + jt * 8 + lc;
-        const float bi = s.beta[i];
-        if (i < nvalid)
-          *reinterpret_cast<uint32_t*>(dv + rowg[hh] + a) =
-              frag::pack(bi * lu[jt][2 * hh], bi * lu[jt][2 * hh + 1]);
         const float2 vf = frag::unpack(vv[jt][hh]);
         dbrow[hh] += lu[jt][2 * hh] * vf.x + lu[jt][2 * hh + 1] * vf.y;
       }
+    // dv = diag(beta) Lambda_U.  Real gates: transposed across the quad of lanes
+    // that share a row into one 16-byte store per row and lane; the phase gate
+    // (short of registers here) stores its pairs directly.
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int i = i0 + hh * 8;
+      const float bi = s.beta[i];
+      uint32_t dvp[4];
+#pragma unroll
+      for (int jt = 0; jt < 4; ++jt) dvp[jt] = frag::pack(bi * lu[jt][2 * hh], bi * lu[jt][2 * hh + 1]);
+      if (PHASE) {
+#pragma unroll
+        for (int jt = 0; jt < 4; ++jt)
+          if (i < nvalid) *reinterpret_cast<uint32_t*>(dv + rowg[hh] + qt * 32 + jt * 8 + lc) = dvp[jt];
+      } else {
+        quad_transpose(dvp, lane & 3);
+        if (i < nvalid)
+          *reinterpret_cast<uint4*>(dv + rowg[hh] + qt * 32 + 8 * (lane & 3)) =
+              make_uint4(dvp[0], dvp[1], dvp[2], dvp[3]);
+      }
+    }
     frag::st_c(lu, sLU, -D, rb * 16, qt * 32);
     frag_ld4(tb + T_LW + 32 * qt, warp, Q);
     frag::st_c(Q, sLW, -D, rb * 16, qt * 32);
