@@ -173,24 +173,6 @@ __device__ __forceinline__ void named_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// 4 x 4 transpose of 32-bit words across the four lanes of a quad (lq = lane % 4):
-// on entry lane lq holds a[j] = element (lq, j), on exit a[j] = element (j, lq).
-// Two exchange rounds (lane masks 1 and 2), two shuffles each.
-__device__ __forceinline__ void quad_transpose(uint32_t (&a)[4], int lq) {
-#pragma unroll
-  for (int m = 1; m <= 2; m <<= 1)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (j & m) continue;
-      const uint32_t send = (lq & m) ? a[j] : a[j | m];
-      const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, m);
-      if (lq & m)
-        a[j] = recv;
-      else
-        a[j | m] = recv;
-    }
-}
-
 __device__ __forceinline__ void mma_step(uint32_t tm, uint64_t a, uint64_t b, uint32_t id,
                                          uint32_t acc) {
   tc::mma(tm, a, b, id, acc);
@@ -959,7 +941,7 @@ __global__ void __launch_bounds__(NTB, 1)
         for (int jt = 0; jt < 4; ++jt)
           if (i < nvalid) *reinterpret_cast<uint32_t*>(dv + rowg[hh] + qt * 32 + jt * 8 + lc) = dvp[jt];
       } else {
-        quad_transpose(dvp, lane & 3);
+        frag::quad_transpose(dvp, lane & 3);
         if (i < nvalid)
           *reinterpret_cast<uint4*>(dv + rowg[hh] + qt * 32 + 8 * (lane & 3)) =
               make_uint4(dvp[0], dvp[1], dvp[2], dvp[3]);
@@ -1172,7 +1154,7 @@ __global__ void __launch_bounds__(NTB, 1)
     }
     // after the quad transpose lane lq holds channels qt * 32 + 8 lq .. + 7 of
     // the row (one 16-byte store instead of four 4-byte ones)
-    quad_transpose(dqp, lane & 3);
+    frag::quad_transpose(dqp, lane & 3);
     if (i0 + 8 * hh < nvalid)
       *reinterpret_cast<uint4*>(dq + rowg[hh] + qt * 32 + 8 * (lane & 3)) =
           make_uint4(dqp[0], dqp[1], dqp[2], dqp[3]);
@@ -1277,7 +1259,7 @@ __global__ void __launch_bounds__(NTB, 1)
       }
       dkp[jt] = frag::pack(o0, o1);
     }
-    quad_transpose(dkp, lane & 3);
+    frag::quad_transpose(dkp, lane & 3);
     if (i0 + 8 * hh < nvalid)
       *reinterpret_cast<uint4*>(dk + rowg[hh] + qt * 32 + 8 * (lane & 3)) =
           make_uint4(dkp[0], dkp[1], dkp[2], dkp[3]);

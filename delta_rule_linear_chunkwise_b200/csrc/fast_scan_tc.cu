@@ -202,16 +202,38 @@ __global__ void __launch_bounds__(NTF, 1)
     for (int q16 = 0; q16 < HB / 16; ++q16)
       tc::tmem_ld16_nowait(lane_addr(s.tmem, warp, buf * BV + ah * HB + 16 * q16), r + 16 * q16);
     tc::tmem_wait_ld();
-    if (i < nvalid) {
-      bf16* op = o + row_id(p, b, t0 + i, h) * D + a0 + ah * HB;
+    // the row's HB values as bf16 pairs, 16-byte block e8 = w[4 e8 .. 4 e8 + 3];
+    // blocks transposed across each quad of lanes (four consecutive rows), so that
+    // one store instruction writes 64 contiguous bytes of each of 8 rows instead
+    // of 16 bytes of each of 32
+    uint32_t w[HB / 2];
 #pragma unroll
-      for (int e8 = 0; e8 < HB / 8; ++e8) {
-        const float* f = reinterpret_cast<const float*>(r + 8 * e8);
-        *reinterpret_cast<uint4*>(op + 8 * e8) =
-            make_uint4(frag::pack(f[0], f[1]), frag::pack(f[2], f[3]), frag::pack(f[4], f[5]),
-                       frag::pack(f[6], f[7]));
-      }
+    for (int q = 0; q < HB / 2; ++q) {
+      const float* f = reinterpret_cast<const float*>(r);
+      w[q] = frag::pack(f[2 * q], f[2 * q + 1]);
     }
+    const int lq = lane & 3, iq = i - lq;  // the quad's first row
+#pragma unroll
+    for (int bg = 0; bg < HB / 32; ++bg)
+#pragma unroll
+      for (int pw = 0; pw < 4; ++pw) {
+        uint32_t a[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) a[j] = w[4 * (4 * bg + j) + pw];
+        frag::quad_transpose(a, lq);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[4 * (4 * bg + j) + pw] = a[j];
+      }
+    // now w[4 (4 bg + k) .. + 3] is block 4 bg + lq of row iq + k
+#pragma unroll
+    for (int bg = 0; bg < HB / 32; ++bg)
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (iq + k < nvalid) {
+          bf16* op = o + row_id(p, b, t0 + iq + k, h) * D + a0 + ah * HB + 8 * (4 * bg + lq);
+          const int q0 = 4 * (4 * bg + k);
+          *reinterpret_cast<uint4*>(op) = make_uint4(w[q0], w[q0 + 1], w[q0 + 2], w[q0 + 3]);
+        }
     return true;
   };
 

@@ -101,5 +101,24 @@ __device__ __forceinline__ void cp_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// 4 x 4 transpose of 32-bit words across the four lanes of a quad (lq = lane % 4):
+// on entry lane lq holds a[j] = element (lq, j), on exit a[j] = element (j, lq).
+// Two exchange rounds (lane masks 1 and 2), two shuffles each; every lane of the
+// warp takes part.
+__device__ __forceinline__ void quad_transpose(uint32_t (&a)[4], int lq) {
+#pragma unroll
+  for (int m = 1; m <= 2; m <<= 1)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (j & m) continue;
+      const uint32_t send = (lq & m) ? a[j] : a[j | m];
+      const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, m);
+      if (lq & m)
+        a[j] = recv;
+      else
+        a[j | m] = recv;
+    }
+}
+
 }  // namespace frag
 }  // namespace dr
